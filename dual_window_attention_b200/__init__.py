@@ -1,0 +1,263 @@
+"""IP-TTCD block forward on B200 (sm_100a): thin Python binding over libttcd.so.
+
+The binding only marshals arguments: device memory comes from PyTorch, every
+step of the computation runs in the library's CUDA kernels.  There is no CPU
+fallback; if the library is missing or a tensor is not on a CUDA device the
+call raises.
+
+    import dual_window_attention_b200 as ttcd
+    o_T, o_S, lse_T, lse_S = ttcd.dual_window_attn(q, k, v, w_S=512, w_T=8192)
+    out, state = ttcd.block_forward(x, beta, weights, params)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Dict, Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttcd.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+F32, BF16 = 0, 1
+
+
+class TTCDError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("d_ff", ctypes.c_int), ("w_S", ctypes.c_int),
+                ("w_T", ctypes.c_int), ("chunk", ctypes.c_int), ("conv_k", ctypes.c_int),
+                ("rms_eps", ctypes.c_float), ("l2_eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("dtype", ctypes.c_int)]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_qkv", "w_o", "g_attn", "g_mlp", "w_gate",
+                                               "w_up", "w_down", "w_proj", "conv_T", "conv_S")]
+
+
+WEIGHT_NAMES = tuple(n for n, _ in _Weights._fields_)
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libttcd.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library {path} is missing: build it with "
+                          "`python -m dual_window_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    P, W = ctypes.POINTER(_Params), ctypes.POINTER(_Weights)
+    lib.ttcd_dual_window_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
+    lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
+    lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
+    lib.ttcd_fastweight_mlp_workspace_size.argtypes = [P]
+    lib.ttcd_fastweight_mlp_workspace_size.restype = sz
+    lib.ttcd_block_forward_workspace_size.argtypes = [P]
+    lib.ttcd_block_forward_workspace_size.restype = sz
+    lib.ttcd_block_workspace_offset.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(sz)]
+    lib.ttcd_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
+    lib.ttcd_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.ttcd_set_wait_timeout_ns.restype = None
+    lib.ttcd_test_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+    lib.ttcd_status_string.argtypes = [i]
+    lib.ttcd_status_string.restype = ctypes.c_char_p
+    lib.ttcd_version.restype = ctypes.c_char_p
+    for fn in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward",
+               "ttcd_block_workspace_offset", "ttcd_get_device_error", "ttcd_test_bounded_wait"):
+        getattr(lib, fn).restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().ttcd_status_string(status).decode()
+
+
+def version() -> str:
+    return load_library().ttcd_version().decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise TTCDError(status, what)
+
+
+@dataclasses.dataclass
+class BlockParams:
+    """Mirror of ttcd_block_params (names follow the pages: w_T, w_S, chunk C)."""
+
+    B: int
+    T: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    d_ff: int
+    w_S: int
+    w_T: int
+    chunk: int
+    conv_k: int = 4
+    rms_eps: float = 1e-6
+    l2_eps: float = 1e-6
+    rope_theta: float = 10000.0
+    softmax_scale: float = 0.0
+    dtype: int = BF16
+
+    def c(self) -> _Params:
+        return _Params(*[getattr(self, f) for f, _ in _Params._fields_])
+
+    @classmethod
+    def from_shape(cls, shape) -> "BlockParams":
+        return cls(B=shape.B, T=shape.T, d_model=shape.d_model, n_q_heads=shape.n_q_heads,
+                   n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim, d_ff=shape.d_ff,
+                   w_S=shape.w_S, w_T=shape.w_T, chunk=shape.chunk, conv_k=shape.conv_k,
+                   rms_eps=shape.rms_eps, l2_eps=shape.l2_eps, rope_theta=shape.rope_theta,
+                   dtype=F32 if shape.dtype == "f32" else BF16)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == F32 else torch.bfloat16
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libttcd takes CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("libttcd takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _weights(w: Dict[str, torch.Tensor]) -> _Weights:
+    return _Weights(*[_ptr(w.get(n)) for n in WEIGHT_NAMES])
+
+
+def dual_window_attn(q, k, v, w_S: int, w_T: int, scale: float = 0.0, o_T=None, o_S=None,
+                     lse: bool = False, stream=None):
+    """Fused dual-window attention; returns (o_T, o_S, lse_T, lse_S) (lse None unless asked)."""
+    lib = load_library()
+    B, T, Hq, hd = q.shape
+    Hkv = k.shape[2]
+    o_T = torch.empty_like(q) if o_T is None else o_T
+    o_S = torch.empty_like(q) if o_S is None else o_S
+    lse_T = lse_S = None
+    if lse:
+        lse_T = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+        lse_S = torch.empty_like(lse_T)
+    dt = BF16 if q.dtype == torch.bfloat16 else F32
+    st = lib.ttcd_dual_window_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o_T), _ptr(o_S), _ptr(lse_T),
+                                   _ptr(lse_S), B, T, Hq, Hkv, hd, w_S, w_T, scale, dt,
+                                   _stream(stream))
+    _check(st, "ttcd_dual_window_attn")
+    return o_T, o_S, lse_T, lse_S
+
+
+def block_forward_workspace_size(p: BlockParams) -> int:
+    pc = p.c()
+    return load_library().ttcd_block_forward_workspace_size(ctypes.byref(pc))
+
+
+def fastweight_mlp_workspace_size(p: BlockParams) -> int:
+    pc = p.c()
+    return load_library().ttcd_fastweight_mlp_workspace_size(ctypes.byref(pc))
+
+
+def workspace_offset(p: BlockParams, name: str) -> int:
+    pc = p.c()
+    off = ctypes.c_size_t(0)
+    _check(load_library().ttcd_block_workspace_offset(ctypes.byref(pc), name.encode(),
+                                                      ctypes.byref(off)), "workspace_offset")
+    return off.value
+
+
+def workspace_view(ws: torch.Tensor, p: BlockParams, name: str, dtype: torch.dtype, shape):
+    """View of a named intermediate inside a block_forward workspace (uint8 tensor)."""
+    off = workspace_offset(p, name)
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    return ws[off:off + nbytes].view(dtype).view(*shape)
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def block_forward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, out=None,
+                  state_out: bool = False, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
+    """One IP-TTCD block forward.  Returns (out, state_out or None, workspace)."""
+    lib = load_library()
+    need = block_forward_workspace_size(p)
+    if need == 0:
+        raise TTCDError(ERR_INVALID_ARG, "ttcd_block_forward_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    out = torch.empty_like(x) if out is None else out
+    st_t = (torch.empty(p.B, p.d_model, p.d_ff, device=x.device, dtype=torch.float32)
+            if state_out else None)
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_block_forward(_ptr(x), _ptr(beta), ctypes.byref(wc), ctypes.byref(pc),
+                                _ptr(st_t), _ptr(out), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    _check(st, "ttcd_block_forward")
+    return out, st_t, workspace
+
+
+def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams, h_S=None,
+                   state_in=None, state_out: bool = False, y=None,
+                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """In-place fast-weight MLP.  Returns (y, state_out or None, workspace)."""
+    lib = load_library()
+    need = fastweight_mlp_workspace_size(p)
+    if need == 0:
+        raise TTCDError(ERR_INVALID_ARG, "ttcd_fastweight_mlp_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, u_T.device)
+    y = torch.empty_like(u_S) if y is None else y
+    st_t = (torch.empty(p.B, p.d_model, p.d_ff, device=u_T.device, dtype=torch.float32)
+            if state_out else None)
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_fastweight_mlp(_ptr(u_T), _ptr(u_S), _ptr(h_S), _ptr(beta), ctypes.byref(wc),
+                                 ctypes.byref(pc), _ptr(state_in), _ptr(st_t), _ptr(y),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ttcd_fastweight_mlp")
+    return y, st_t, workspace
+
+
+def get_device_error(stream=None) -> Tuple[int, int]:
+    """(status, raw flags) of the device error word; clears it.  Synchronises."""
+    flags = ctypes.c_uint32(0)
+    st = load_library().ttcd_get_device_error(ctypes.byref(flags), _stream(stream))
+    return st, flags.value
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    load_library().ttcd_set_wait_timeout_ns(ns)
+
+
+def test_bounded_wait(timeout_ns: int, stream=None) -> int:
+    return load_library().ttcd_test_bounded_wait(timeout_ns, _stream(stream))

@@ -1,0 +1,387 @@
+// Persistent warp-specialised tcgen05 GEMM for sm_100a:  C = A * B^T.
+//
+//   A [rows, K] bf16 K-major, B [N, K] bf16 K-major, fp32 accumulators in TMEM.
+//   warp 0      : TMA producer (one elected lane), STAGES-deep smem ring
+//   warp 1      : TMEM allocation + tcgen05.mma issue (one elected lane)
+//   warps 2..5  : epilogue, each owns one 32-lane quarter of the accumulator
+//   Two TMEM accumulators (2*BN columns) let the epilogue of tile j overlap the
+//   main loop of tile j+1.
+//
+// The A rows may be cut into groups (fast-weight chunks): sequence b, chunk i
+// covers rows [b*T + i*C, b*T + min((i+1)*C, T)) and reads B rows starting at
+// (b*Nc + i) * b_group_rows.  A plain GEMM is one sequence with one chunk.
+#pragma once
+#include "ptx.cuh"
+
+namespace ttcd {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 64;  // bf16 elements per 128-byte swizzled row
+constexpr int GEMM_THREADS = 192;
+
+struct TileCtx {
+  int row0;        // first A row (== output row) of the tile
+  int valid_rows;  // rows of this tile inside its group (<= 128)
+  int tn;          // column-tile index
+  int group;       // b * Nc + i
+  int b_row0;      // first B row of this group
+};
+
+struct GemmGeom {
+  int n_seq, T, C, Nc;  // row groups
+  int K;                // reduction length (multiple of 64 not required: TMA zero-fills)
+  int tiles_m;          // ceil(C / 128)
+  int tiles_n;          // column tiles
+  int b_group_rows;     // B row offset per group (0 = shared B)
+  __host__ __device__ int total() const { return n_seq * Nc * tiles_m * tiles_n; }
+  __device__ bool tile(int t, TileCtx& c) const {
+    const int tn = t % tiles_n;
+    const int r = t / tiles_n;
+    const int tm = r % tiles_m;
+    const int g = r / tiles_m;
+    const int b = g / Nc, i = g % Nc;
+    const int len = min(C, T - i * C);
+    const int m0 = tm * GEMM_BM;
+    c.valid_rows = min(GEMM_BM, len - m0);
+    c.row0 = b * T + i * C + m0;
+    c.tn = tn;
+    c.group = g;
+    c.b_row0 = g * b_group_rows;
+    return c.valid_rows > 0;
+  }
+};
+
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
+  }
+}
+__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+__device__ __forceinline__ void store_x32(__nv_bfloat16* dst, const float (&v)[32]) { store_bf16x32(dst, v); }
+__device__ __forceinline__ void store_x32(float* dst, const float (&v)[32]) { store_f32x32(dst, v); }
+
+__device__ __forceinline__ void load_x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w = s[q];
+    v[8 * q + 0] = bf16lo_to_f32(w.x); v[8 * q + 1] = bf16hi_to_f32(w.x);
+    v[8 * q + 2] = bf16lo_to_f32(w.y); v[8 * q + 3] = bf16hi_to_f32(w.y);
+    v[8 * q + 4] = bf16lo_to_f32(w.z); v[8 * q + 5] = bf16hi_to_f32(w.z);
+    v[8 * q + 6] = bf16lo_to_f32(w.w); v[8 * q + 7] = bf16hi_to_f32(w.w);
+  }
+}
+__device__ __forceinline__ void load_x32(const float* src, float (&v)[32]) {
+  const float4* s = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float4 w = s[q];
+    v[4 * q] = w.x; v[4 * q + 1] = w.y; v[4 * q + 2] = w.z; v[4 * q + 3] = w.w;
+  }
+}
+
+template <int BN, int STAGES, bool DUAL_B, class Epi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
+                   const __grid_constant__ CUtensorMap mapB0,
+                   const __grid_constant__ CUtensorMap mapB1, const GemmGeom geo, const Epi epi,
+                   const DevStatus st) {
+  constexpr int A_BYTES = GEMM_BM * 128;
+  constexpr int B_BYTES = BN * 128;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
+  constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN, false, false);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mapA);
+    tma_prefetch_map(&mapB0);
+    if (DUAL_B) tma_prefetch_map(&mapB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = geo.total();
+  const int nk = (geo.K + GEMM_BK - 1) / GEMM_BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        TileCtx c;
+        if (!geo.tile(t, c)) continue;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, st, abort)) { ok = false; break; }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(sa, &mapA, &full[s], kb * GEMM_BK, c.row0);
+          if (DUAL_B) {
+            tma_load_2d(sb, &mapB0, &full[s], kb * GEMM_BK, c.b_row0 + c.tn * (BN / 2));
+            tma_load_2d(sb + (BN / 2) * 128, &mapB1, &full[s], kb * GEMM_BK,
+                        c.b_row0 + c.tn * (BN / 2));
+          } else {
+            tma_load_2d(sb, &mapB0, &full[s], kb * GEMM_BK, c.b_row0 + c.tn * BN);
+          }
+        }
+      }
+      // Let every load this thread issued land before the CTA can exit.
+      volatile int no_abort = 0;
+      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+        mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        TileCtx c;
+        if (!geo.tile(t, c)) continue;
+        const int ab = j & 1;
+        if (!mbar_wait(&acce[ab], ((j >> 1) & 1) ^ 1, st, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, st, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            const uint64_t da = sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t db = sdesc_sw128(sb + k * 32, 16, 1024);
+            mma_bf16_ss(d_tmem, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&accf[ab]);
+        ++j;
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, st, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    int j = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      TileCtx c;
+      if (!geo.tile(t, c)) continue;
+      const int ab = j & 1;
+      if (!mbar_wait(&accf[ab], (j >> 1) & 1, st, abort)) break;
+      tc_fence_after();
+      epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r);
+      tc_fence_before();
+      mbar_arrive(&acce[ab]);
+      ++j;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int BN, int STAGES>
+constexpr int gemm_smem_bytes() {
+  return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + 256;
+}
+
+// ------------------------------------------------------------------ epilogues
+
+// C[row, col] = bf16(acc * col_scale[col]) (col_scale nullable), columns < N.
+struct EpiStoreBF16 {
+  __nv_bfloat16* out;
+  long long ldo;
+  int N;
+  const float* col_scale;
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      const int col = c.tn * BN + cc;
+      if (col >= N) break;
+      float v[32];
+      tmem_ld32f(taddr + cc, v);
+      if (col_scale) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= __ldg(col_scale + col + i);
+      }
+      if (ok) store_bf16x32(out + row * ldo + col, v);
+    }
+  }
+};
+
+// out[row, col] = resid[row % resid_rows, col] + acc;  columns < N.
+template <class OutT, class ResT>
+struct EpiResidual {
+  OutT* out;
+  long long ldo;
+  const ResT* resid;  // nullable
+  long long ld_res;
+  long long resid_rows;
+  int N;
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      const int col = c.tn * BN + cc;
+      if (col >= N) break;
+      float v[32];
+      tmem_ld32f(taddr + cc, v);
+      if (ok) {
+        if (resid) {
+          float x[32];
+          load_x32(resid + (row % resid_rows) * ld_res + col, x);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += x[i];
+        }
+        store_x32(out + row * ldo + col, v);
+      }
+    }
+  }
+};
+
+// Gate/up tile: accumulator columns [0, BN/2) are gate, [BN/2, BN) are up for
+// output columns tn*BN/2 + [0, BN/2).  Z = silu(gate) * up, fp32.
+struct EpiSwiGLU {
+  float* out;
+  long long ldo;
+  int N;  // d_ff
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN / 2; cc += 32) {
+      const int col = c.tn * (BN / 2) + cc;
+      if (col >= N) break;
+      float g[32], u[32];
+      tmem_ld32f(taddr + cc, g);
+      tmem_ld32f(taddr + BN / 2 + cc, u);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
+      if (ok) store_f32x32(out + row * ldo + col, g);
+    }
+  }
+};
+
+// QKV projection with rotary embedding on the query and key heads.
+// Column n of the accumulator is feature n of [q heads | k heads | v heads].
+template <int HD>
+struct EpiQKVRope {
+  __nv_bfloat16* q;
+  __nv_bfloat16* k;
+  __nv_bfloat16* v;
+  int Hq, Hkv, T;
+  const float2* rope_cs;  // [T][HD/2] (cos, sin)
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+    static_assert(BN % HD == 0, "column tile must hold whole heads");
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+    const int t = static_cast<int>(row % T);
+    const int n_heads = Hq + 2 * Hkv;
+#pragma unroll 1
+    for (int h0 = 0; h0 < BN; h0 += HD) {
+      const int head = (c.tn * BN + h0) / HD;
+      if (head >= n_heads) break;
+      float x[HD];
+#pragma unroll
+      for (int cc = 0; cc < HD; cc += 32) {
+        float tmp[32];
+        tmem_ld32f(taddr + h0 + cc, tmp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[cc + i] = tmp[i];
+      }
+      if (!ok) continue;
+      __nv_bfloat16* dst;
+      if (head < Hq + Hkv) {
+        const float2* cs = rope_cs + static_cast<long long>(t) * (HD / 2);
+#pragma unroll
+        for (int i = 0; i < HD / 2; ++i) {
+          const float2 e = __ldg(cs + i);
+          const float a = x[i], b = x[i + HD / 2];
+          x[i] = a * e.x - b * e.y;
+          x[i + HD / 2] = b * e.x + a * e.y;
+        }
+        dst = head < Hq ? q + (row * Hq + head) * HD : k + (row * Hkv + (head - Hq)) * HD;
+      } else {
+        dst = v + (row * Hkv + (head - Hq - Hkv)) * HD;
+      }
+#pragma unroll
+      for (int cc = 0; cc < HD; cc += 32) {
+        float tmp[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) tmp[i] = x[cc + i];
+        store_bf16x32(dst + cc, tmp);
+      }
+    }
+  }
+};
+
+}  // namespace ttcd

@@ -1,0 +1,208 @@
+/*
+ * ttcd.h — C ABI of libttcd: the forward pass of one IP-TTCD block
+ * (In-Place Test-Time Context Distillation) on NVIDIA B200 (sm_100a).
+ *
+ * Sources of the definitions (cited by page title and section):
+ *   [README]  GitHub README "TTCD: Test-Time Training via Context Distillation",
+ *             sections "Model configuration" and "Fused inference kernels".
+ *   [REVIEW]  papernotes.org review "Learning What to Remember: Test-Time
+ *             Training via Context Distillation", section 方法详解 (overall
+ *             framework, flowchart A-F) and 关键设计 2-3 (in-place fast weight,
+ *             off-policy approximation, short convs, W_proj, R_i, K_i, Delta W).
+ *   [PODCAST] podcast transcript "Test-Time Training via Context Distillation:
+ *             Learning What to Remember", cues 19 (sliding window) and 29
+ *             (practical update).
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument named as a tensor is a DEVICE pointer, owned by the
+ *     caller; the library never allocates or frees device memory.  Scratch
+ *     space comes only from the caller's `workspace` (size from the matching
+ *     *_workspace_size query).  Parameter structs are HOST pointers, read during
+ *     the call only.
+ *   - Layouts are dense row-major with the last index fastest: activations
+ *     [B, T, ...], weights in the `[out, in]` Linear convention (y = x W^T).
+ *   - Every device pointer must be 16-byte aligned; each tensor's innermost
+ *     extent times its element size must be a multiple of 16 bytes.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and keep no state between calls except the device error word
+ *     read by ttcd_get_device_error().
+ *   - Arguments are validated on the host before any launch; a bad argument
+ *     returns TTCD_ERR_INVALID_ARG or TTCD_ERR_UNSUPPORTED and launches nothing.
+ *     A launch failure returns TTCD_ERR_CUDA.  Every device-side wait is
+ *     bounded: one that gives up sets the device error word (reported as
+ *     TTCD_ERR_TIMEOUT by ttcd_get_device_error) and the kernel returns.  No
+ *     entry point aborts, traps or throws.
+ */
+#ifndef TTCD_H_
+#define TTCD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTCD_OK = 0,
+  TTCD_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent sizes   */
+  TTCD_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head_dim, dtype)    */
+  TTCD_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed    */
+  TTCD_ERR_TIMEOUT = 4,      /* a bounded device wait gave up                  */
+  TTCD_ERR_WORKSPACE = 5     /* workspace smaller than the size query returned */
+} ttcd_status;
+
+typedef enum { TTCD_F32 = 0, TTCD_BF16 = 1 } ttcd_dtype;
+
+/* Shape and hyper-parameters of one block.  Names follow the pages:
+ * window_size = teacher window w_T, student window w_S, fast-weight chunk C,
+ * conv width ([README] "Model configuration"). */
+typedef struct {
+  int B;              /* sequences in the batch                                */
+  int T;              /* tokens per sequence                                   */
+  int d_model;        /* d                                                     */
+  int n_q_heads;      /* Hq                                                    */
+  int n_kv_heads;     /* Hkv, Hq % Hkv == 0; query head h reads KV head h/(Hq/Hkv) */
+  int head_dim;       /* hd in {32, 64, 128}                                   */
+  int d_ff;           /* f                                                     */
+  int w_S;            /* student window, 1 <= w_S <= w_T                       */
+  int w_T;            /* teacher window                                        */
+  int chunk;          /* C >= 1; a partial last chunk is allowed               */
+  int conv_k;         /* depthwise conv width, 1..8                            */
+  float rms_eps;      /* RMSNorm epsilon (1e-6)                                */
+  float l2_eps;       /* key normalisation epsilon (1e-6)                      */
+  float rope_theta;   /* RoPE base (1e4)                                       */
+  float softmax_scale;/* 0 => 1/sqrt(head_dim)                                 */
+  ttcd_dtype dtype;   /* type of x, weights and out (beta/state are fp32)      */
+} ttcd_block_params;
+
+/* Slow weights W^(0) of one block, device pointers in params.dtype.
+ * w_qkv rows: Hq*hd query rows, then Hkv*hd key rows, then Hkv*hd value rows. */
+typedef struct {
+  const void* w_qkv;  /* [(Hq + 2 Hkv) hd, d]                                  */
+  const void* w_o;    /* [d, Hq hd]   shared by teacher and student            */
+  const void* g_attn; /* [d]          input RMSNorm gain                       */
+  const void* g_mlp;  /* [d]          MLP RMSNorm gain (shared by both paths)  */
+  const void* w_gate; /* [f, d]                                                */
+  const void* w_up;   /* [f, d]                                                */
+  const void* w_down; /* [d, f]       W_down^(0), the in-place fast weight's base */
+  const void* w_proj; /* [f, f]       learned projection of the value residual */
+  const void* conv_T; /* [f, k]       teacher conv taps, tap m multiplies t-m  */
+  const void* conv_S; /* [f, k]       student conv taps                        */
+} ttcd_block_weights;
+
+/*
+ * ttcd_dual_window_attn — fused dual-window causal sliding-window attention.
+ *
+ * Defines ([README] "Fused inference kernels", fused_dual_attn; [REVIEW]
+ * 方法详解 overall framework; [PODCAST] cue 19): for every query t and head h,
+ *   o_W[t,h] = sum_{j in win_W(t)} softmax_j(scale * q[t,h].k[j,g]) v[j,g],
+ *   win_W(t) = { j : max(0, t-W+1) <= j <= t },  g = h / (Hq/Hkv),
+ * for W = w_T (teacher, o_T) and W = w_S (student, o_S), computed in one pass
+ * over K/V that reuses each Q.K^T tile for both windows.
+ *   q          [B, T, Hq, hd]  bf16, device
+ *   k, v       [B, T, Hkv, hd] bf16, device
+ *   o_T, o_S   [B, T, Hq, hd]  bf16, device, written
+ *   lse_T/lse_S [B, Hq, T] fp32 natural-log log-sum-exp, device, nullable
+ *   scale      softmax scale; 0 => 1/sqrt(hd)
+ *   dtype      must be TTCD_BF16 (TTCD_F32 -> TTCD_ERR_UNSUPPORTED)
+ * Errors: hd not in {32,64,128}, Hq % Hkv != 0, w_S < 1, w_S > w_T, B or T < 1,
+ * null/misaligned pointers -> TTCD_ERR_INVALID_ARG / TTCD_ERR_UNSUPPORTED.
+ */
+ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, void* o_T,
+                                  void* o_S, float* lse_T, float* lse_S, int B, int T, int Hq,
+                                  int Hkv, int hd, int w_S, int w_T, float scale,
+                                  ttcd_dtype dtype, void* stream);
+
+/*
+ * ttcd_fastweight_mlp — the in-place fast-weight MLP of one block (off-policy).
+ *
+ * Defines ([REVIEW] 关键设计 2 and 3, flowchart C-F; [PODCAST] cue 29):
+ *   Z_P   = silu(u_P W_gate^T) * (u_P W_up^T)            P in {T, S}, slow weights
+ *   Zb_P  = conv_P(Z_P)   causal depthwise, tap m multiplies t-m, zero history
+ *   r_t   = W_down W_proj (Zb_T - Zb_S)[t]               value residual
+ *   k_t   = Zb_S[t] / sqrt(||Zb_S[t]||^2 + l2_eps)       key
+ *   dW_i  = sum_{t in chunk i} beta_t r_t k_t^T          [d, f]
+ *   S_0   = state_in (or 0),  S_{i+1} = S_i + dW_i       fp32 exclusive prefix
+ *   y_t   = h_S[t] + (W_down + S_{i(t)}) Z_S[t]          (h_S term if non-null)
+ *   state_out = S_{n_chunks} (includes a partial last chunk)
+ *   u_T, u_S   [B, T, d] post-RMSNorm activations, params.dtype, device
+ *   h_S        [B, T, d] params.dtype, device, nullable (residual added to y)
+ *   beta       [B, T] fp32, device
+ *   state_in   [B, d, f] fp32, device, nullable;  state_out likewise
+ *   y          [B, T, d] params.dtype, device, written
+ *   workspace  >= ttcd_fastweight_mlp_workspace_size(p) bytes, device, 256-aligned
+ */
+ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,
+                                const float* beta, const ttcd_block_weights* w,
+                                const ttcd_block_params* p, const float* state_in,
+                                float* state_out, void* y, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/*
+ * ttcd_block_forward — forward pass of one IP-TTCD block (student path output).
+ *
+ * Defines ([REVIEW] 方法详解 overall framework + flowchart A-F; readings of the
+ * unstated skeleton: pre-norm, no biases, rotate-half RoPE at positions 0..T-1):
+ *   xn = RMSNorm(x; g_attn);  q,k,v = xn W_qkv^T;  q,k = RoPE(q,k)
+ *   o_T, o_S = ttcd_dual_window_attn(q, k, v)
+ *   h_P = x + o_P W_o^T;  u_P = RMSNorm(h_P; g_mlp)
+ *   out = ttcd_fastweight_mlp(u_T, u_S, h_S, beta, ...)
+ *   x, out     [B, T, d] params.dtype, device
+ *   beta       [B, T] fp32, device
+ *   state_out  [B, d, f] fp32, device, nullable (final fast-weight state)
+ *   workspace  >= ttcd_block_forward_workspace_size(p) bytes, device, 256-aligned
+ * The workspace holds every intermediate after the call; their byte offsets
+ * are returned by ttcd_block_workspace_offset().
+ */
+ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_block_weights* w,
+                               const ttcd_block_params* p, float* state_out, void* out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by each entry point; 0 if the parameters are invalid. */
+size_t ttcd_fastweight_mlp_workspace_size(const ttcd_block_params* p);
+size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
+
+/*
+ * Byte offset inside the block_forward workspace of a named intermediate, for
+ * inspection after a call (same layout for ttcd_fastweight_mlp where named).
+ * Names and layouts (row-major):
+ *   "xn"   bf16 [B*T, d]          "q" bf16 [B*T, Hq*hd]   "k","v" bf16 [B*T, Hkv*hd]
+ *   "o"    bf16 [2, B*T, Hq*hd]   (o_T rows, then o_S rows)
+ *   "h"    fp32 [2, B*T, d]       "u" bf16 [2, B*T, d]
+ *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f]
+ *   "D"    bf16 [P, f]            "Kt" bf16 [f, P]        "ssq" fp32 [P]
+ *   "Rt"   bf16 [d, P]            "Wall" bf16 [B*n_chunks, d, f]
+ * where P = B * n_chunks * Cp, Cp = chunk rounded up to 64, and token t of
+ * sequence b sits at padded index (b*n_chunks + t/C)*Cp + t%C.
+ * Returns TTCD_ERR_INVALID_ARG for an unknown name or invalid params.
+ */
+ttcd_status ttcd_block_workspace_offset(const ttcd_block_params* p, const char* name,
+                                        size_t* offset);
+
+/* Reads and clears the device error word on the current device (synchronises
+ * `stream`).  *flags receives the raw bits; returns TTCD_ERR_TIMEOUT if a wait
+ * gave up since the last call, TTCD_OK otherwise. */
+ttcd_status ttcd_get_device_error(uint32_t* flags, void* stream);
+
+/* Bound in nanoseconds on every device-side wait (default 2e9 = 2 s). */
+void ttcd_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * ttcd_test_bounded_wait — failure-detection self-test.  Launches one CTA that
+ * waits on an mbarrier nothing ever arrives at, bounded by `timeout_ns`; the
+ * wait gives up, records TTCD_ERR_TIMEOUT in the device error word and the
+ * kernel returns normally.  The paper has no counterpart; this exists so a
+ * test can check the timeout path without hanging a GPU.
+ */
+ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream);
+
+const char* ttcd_status_string(ttcd_status s);
+
+/* Library version string, e.g. "ttcd 0.1 sm_100a". */
+const char* ttcd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTCD_H_ */

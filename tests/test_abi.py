@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments on the host, and answers size queries."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dual_window_attention_b200 as ttcd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttcd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dual_window_attention_b200 import build
+    build.build()
+    return ttcd.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttcd_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _params(**kw):
+    base = dict(B=1, T=256, d_model=64, n_q_heads=2, n_kv_heads=1, head_dim=32, d_ff=128,
+                w_S=16, w_T=64, chunk=32, conv_k=4, dtype=ttcd.F32)
+    base.update(kw)
+    return ttcd.BlockParams(**base)
+
+
+def test_status_strings(lib):
+    assert ttcd.status_string(ttcd.OK) == "ok"
+    assert "timed out" in ttcd.status_string(ttcd.ERR_TIMEOUT)
+    assert ttcd.version().startswith("ttcd")
+
+
+def test_workspace_sizes(lib):
+    p = _params()
+    assert ttcd.block_forward_workspace_size(p) > ttcd.fastweight_mlp_workspace_size(p) > 0
+    for bad in (dict(head_dim=48), dict(w_S=65), dict(n_kv_heads=3), dict(conv_k=9),
+                dict(chunk=0), dict(T=0), dict(d_model=96), dict(dtype=7)):
+        assert ttcd.block_forward_workspace_size(_params(**bad)) == 0, bad
+
+
+def test_workspace_offsets_are_ordered_and_aligned(lib):
+    p = _params()
+    names = ["xn", "q", "k", "v", "o", "h", "u", "Z", "Zs16", "D", "Kt", "ssq", "Rt", "Wall"]
+    offs = [ttcd.workspace_offset(p, n) for n in names]
+    assert all(o % 1024 == 0 for o in offs)
+    assert offs == sorted(offs)
+    with pytest.raises(ttcd.TTCDError):
+        ttcd.workspace_offset(p, "nope")
+
+
+def test_attention_rejects_bad_arguments_on_host(lib):
+    fake = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+    f = lib.ttcd_dual_window_attn
+    # null pointer
+    assert f(None, fake, fake, fake, fake, None, None, 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    # misaligned pointer
+    assert f(ctypes.c_void_p((1 << 20) + 2), fake, fake, fake, fake, None, None, 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    # w_S > w_T, Hq % Hkv, bad sizes
+    assert f(fake, fake, fake, fake, fake, None, None, 1, 256, 2, 1, 32, 65, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    assert f(fake, fake, fake, fake, fake, None, None, 1, 256, 3, 2, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    assert f(fake, fake, fake, fake, fake, None, None, 0, 256, 2, 1, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    # unsupported head_dim / dtype
+    assert f(fake, fake, fake, fake, fake, None, None, 1, 256, 2, 1, 48, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_UNSUPPORTED
+    assert f(fake, fake, fake, fake, fake, None, None, 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.F32, None) == ttcd.ERR_UNSUPPORTED
+
+
+def test_block_and_mlp_reject_bad_arguments_on_host(lib):
+    fake = 1 << 20
+    p = _params().c()
+    w = ttcd._Weights(*([fake] * 10))
+    wnull = ttcd._Weights(*([fake] * 9 + [0]))
+    ws_need = lib.ttcd_block_forward_workspace_size(ctypes.byref(p))
+    bf = lib.ttcd_block_forward
+    assert bf(None, fake, ctypes.byref(w), ctypes.byref(p), None, fake, fake, ws_need, None) == ttcd.ERR_INVALID_ARG
+    assert bf(fake, fake, ctypes.byref(wnull), ctypes.byref(p), None, fake, fake, ws_need, None) == ttcd.ERR_INVALID_ARG
+    assert bf(fake, fake, ctypes.byref(w), ctypes.byref(p), None, fake, fake, ws_need - 1, None) == ttcd.ERR_WORKSPACE
+    bad = _params(head_dim=48).c()
+    assert bf(fake, fake, ctypes.byref(w), ctypes.byref(bad), None, fake, fake, ws_need, None) == ttcd.ERR_UNSUPPORTED
+    mf = lib.ttcd_fastweight_mlp
+    need = lib.ttcd_fastweight_mlp_workspace_size(ctypes.byref(p))
+    assert mf(fake, fake, None, fake, ctypes.byref(w), ctypes.byref(p), None, None, fake, fake, need - 1, None) == ttcd.ERR_WORKSPACE
+    assert mf(fake, None, None, fake, ctypes.byref(w), ctypes.byref(p), None, None, fake, fake, need, None) == ttcd.ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 128, 2, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ttcd.dual_window_attn(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous(), 16, 64)

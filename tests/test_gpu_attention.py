@@ -1,0 +1,103 @@
+"""GPU parity of the fused dual-window attention against the float64 oracle.
+
+Definition: GitHub README "TTCD", section "Fused inference kernels"; podcast
+cue 19 (a window of w keys ends at the query).  Tolerance for bf16 outputs:
+max|d| / max|ref| <= 1e-2; index masks bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ttcd_oracle as orc
+from tests.helpers import TOL_OUT, np64, rel_max
+from ttcd_workloads import make_attention_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ttcd():
+    import dual_window_attention_b200 as m
+    m.load_library()
+    return m
+
+
+CASES = [
+    # B, T, Hq, Hkv, hd, w_S, w_T
+    (1, 256, 2, 1, 32, 16, 64),        # tiny workload head layout
+    (1, 1000, 4, 2, 64, 100, 300),     # ragged T, windows not multiples of the tile
+    (2, 700, 4, 1, 128, 128, 512),     # batch 2, tile-aligned windows, GQA 4:1
+    (1, 640, 3, 3, 128, 1, 1000),      # student window 1, teacher window > T
+    (1, 513, 2, 2, 64, 200, 200),      # equal windows
+    (1, 300, 6, 2, 32, 33, 129),       # hd 32, GQA 3:1
+]
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,hd,wS,wT", CASES)
+def test_dual_window_attention_parity(ttcd, B, T, Hq, Hkv, hd, wS, wT):
+    q, k, v = make_attention_inputs(B, T, Hq, Hkv, hd, seed=T + hd)
+    o_T, o_S, lse_T, lse_S = ttcd.dual_window_attn(q.cuda(), k.cuda(), v.cuda(), wS, wT, lse=True)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    rT, rS, rlT, rlS = orc.dual_window_attention(np64(q), np64(k), np64(v), wS, wT, hd ** -0.5)
+    assert rel_max(o_T, rT) <= TOL_OUT
+    assert rel_max(o_S, rS) <= TOL_OUT
+    np.testing.assert_allclose(np64(lse_T), rlT, atol=2e-3, rtol=0)
+    np.testing.assert_allclose(np64(lse_S), rlS, atol=2e-3, rtol=0)
+
+
+@pytest.mark.parametrize("w", [1, 16, 100, 128, 300])
+def test_mask_probe_key_counts_bit_exact(ttcd, w):
+    """Q = 0: every visible key gets weight 1, so exp(lse[t]) counts the window exactly."""
+    B, T, H, hd = 1, 600, 1, 64
+    q = torch.zeros(B, T, H, hd, dtype=torch.bfloat16, device="cuda")
+    _, k, v = make_attention_inputs(B, T, H, H, hd, seed=1)
+    _, _, lse_T, lse_S = ttcd.dual_window_attn(q, k.cuda(), v.cuda(), w, max(w, 200), lse=True)
+    counts_S = np.minimum(np.arange(T) + 1, w)
+    counts_T = np.minimum(np.arange(T) + 1, max(w, 200))
+    np.testing.assert_array_equal(np.rint(np.exp(np64(lse_S)[0, 0])), counts_S)
+    np.testing.assert_array_equal(np.rint(np.exp(np64(lse_T)[0, 0])), counts_T)
+
+
+@pytest.mark.parametrize("j", [0, 5, 127, 128, 255, 400])
+def test_mask_probe_one_hot_value_bit_exact(ttcd, j):
+    """V one-hot at key j: o[t] is nonzero exactly for the queries whose window holds j."""
+    B, T, H, hd, wS, wT = 1, 512, 1, 64, 37, 160
+    q = torch.zeros(B, T, H, hd, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros_like(q)
+    v = torch.zeros_like(q)
+    v[0, j, 0, 0] = 1.0
+    o_T, o_S, _, _ = ttcd.dual_window_attn(q, k, v, wS, wT)
+    t = np.arange(T)
+    for o, w in ((o_S, wS), (o_T, wT)):
+        seen = np64(o)[0, :, 0, 0] != 0
+        np.testing.assert_array_equal(seen, (j <= t) & (j >= t - w + 1))
+
+
+def test_full_size_sampled_rows(ttcd):
+    """T = 65536, 16/8 heads, hd 128, w_S 512, w_T 8192: sampled rows vs the oracle."""
+    B, T, Hq, Hkv, hd, wS, wT = 1, 65536, 16, 8, 128, 512, 8192
+    q, k, v = make_attention_inputs(B, T, Hq, Hkv, hd, seed=0)
+    o_T, o_S, _, _ = ttcd.dual_window_attn(q.cuda(), k.cuda(), v.cuda(), wS, wT)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    rng = np.random.default_rng(0)
+    rows = np.concatenate([[0, 1, 127, 128, 511, 512, 8191, 8192, 65535],
+                           rng.integers(0, T, 40)])
+    qn, kn, vn = np64(q), np64(k), np64(v)
+    oT, oS = np64(o_T), np64(o_S)
+    scale = hd ** -0.5
+    err = {wT: 0.0, wS: 0.0}
+    refmax = {wT: 0.0, wS: 0.0}
+    for t in rows:
+        for h in rng.choice(Hq, 2, replace=False):
+            g = h // (Hq // Hkv)
+            for w, got in ((wT, oT), (wS, oS)):
+                j0 = max(0, t - w + 1)
+                s = kn[0, j0:t + 1, g] @ qn[0, t, h] * scale
+                p = np.exp(s - s.max())
+                ref = (p[:, None] * vn[0, j0:t + 1, g]).sum(0) / p.sum()
+                err[w] = max(err[w], np.max(np.abs(got[0, t, h] - ref)))
+                refmax[w] = max(refmax[w], np.max(np.abs(ref)))
+    assert err[wT] / refmax[wT] <= TOL_OUT and err[wS] / refmax[wS] <= TOL_OUT
+    assert torch.isfinite(o_T).all() and torch.isfinite(o_S).all()
