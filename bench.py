@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""Benchmark of the IP-TTCD block forward (prefill) on B200.
+
+One step = one ttcd_block_forward over one batch of the Qwen3-0.6B-shaped
+block at T = 65536 (d 1024, 16/8 heads, hd 128, d_ff 3072, w_S 512, w_T 8192,
+C 1024, conv width 4), with synthetic seeded inputs already resident in HBM.
+Prints one JSON line (rank 0).  Multi-GPU runs are independent replicas
+(weak scaling, no collective on the data path); launch with torchrun.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from ttcd_workloads import QWEN3_0P6B_64K, make_block_inputs  # noqa: E402
+
+METRIC = "IP-TTCD block prefill tokens/s @64K (Qwen3-0.6B shape); dual-attn % BF16 peak"
+UNIT = "tokens/s"
+STAGES = ["rope+rmsnorm_in", "qkv_gemm_rope", "dual_window_attn", "o_proj_residual",
+          "rmsnorm_mlp", "gate_up_swiglu", "conv_residual_keys", "M_wdown_wproj",
+          "R_gemm", "chunk_scan_dW", "out_gemm"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def attention_flops(shape) -> float:
+    """4 * hd * Hq FLOPs per (query, key) pair inside the teacher window."""
+    T, w = shape.T, shape.w_T
+    pairs = w * (w + 1) // 2 + (T - w) * w if T >= w else T * (T + 1) // 2
+    return 4.0 * shape.head_dim * shape.n_q_heads * shape.B * pairs
+
+
+def stage_costs(s):
+    """(bound, algorithmic amount) per stage: FLOPs for tensor stages, bytes for HBM ones."""
+    BT, d, f, hd = s.B * s.T, s.d_model, s.d_ff, s.head_dim
+    Hq, Hkv = s.n_q_heads, s.n_kv_heads
+    dqkv = (Hq + 2 * Hkv) * hd
+    Cp = (s.chunk + 63) // 64 * 64
+    P = s.B * s.n_chunks * Cp
+    return [
+        ("hbm", BT * d * 2 * 2 + s.T * hd // 2 * 8),
+        ("tensor", 2.0 * BT * d * dqkv),
+        ("tensor", attention_flops(s)),
+        ("tensor", 2.0 * 2 * BT * Hq * hd * d),
+        ("hbm", 2 * BT * d * 4 + 2 * BT * d * 2),
+        ("tensor", 2.0 * 2 * BT * d * 2 * f),
+        ("hbm", 2 * BT * f * 4 + 3 * BT * f * 2),
+        ("tensor", 2.0 * d * f * f),
+        ("tensor", 2.0 * d * f * P),
+        ("tensor", 2.0 * d * f * P),
+        ("tensor", 2.0 * BT * f * d),
+    ]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML during the timed region."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_throughput(shape, sample_tokens: int, repeats: int = 1):
+    """Time the float64 oracle on the first `sample_tokens` tokens (tokens/s, seconds)."""
+    from oracle import ttcd_oracle as orc
+    inp = make_block_inputs(shape.with_(T=sample_tokens, n_layers=1), seed=0)
+    w = {k: v.double().numpy() for k, v in inp["layers"][0].items()}
+    x = inp["x"].double().numpy()
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        orc.block_forward(x, w["beta"], w, n_q_heads=shape.n_q_heads, n_kv_heads=shape.n_kv_heads,
+                          head_dim=shape.head_dim, w_S=shape.w_S, w_T=shape.w_T,
+                          chunk=shape.chunk, rms_eps=shape.rms_eps, l2_eps=shape.l2_eps,
+                          rope_theta=shape.rope_theta)
+        times.append(time.perf_counter() - t0)
+    return shape.B * sample_tokens / statistics.median(times), times
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def workload_config(shape, extra=None):
+    cfg = {"workload": shape.name, "B": shape.B, "T": shape.T, "d_model": shape.d_model,
+           "n_q_heads": shape.n_q_heads, "n_kv_heads": shape.n_kv_heads,
+           "head_dim": shape.head_dim, "d_ff": shape.d_ff, "w_S": shape.w_S, "w_T": shape.w_T,
+           "chunk": shape.chunk, "conv_k": shape.conv_k,
+           "l2": "no flush: one step reads and writes ~10 GB, far above the 126 MB L2"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the float64 CPU oracle, timed on the host's cores (rank 0 only)."""
+    if rank != 0:
+        return
+    shape = QWEN3_0P6B_64K
+    sample = args.ref_sample_tokens
+    for _ in range(args.warmup):
+        oracle_throughput(shape, sample)
+    _, times = oracle_throughput(shape, sample, repeats=args.steps)
+    total = sum(times)
+    value = shape.B * sample * args.steps / total
+    desc = (f"first {sample} tokens of the workload per step (attention windows truncated by "
+            f"position), float64 NumPy oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(shape, {"sample_tokens": sample}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import dual_window_attention_b200 as ttcd
+    ttcd.load_library()
+    shape = QWEN3_0P6B_64K
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", local)
+    inp = make_block_inputs(shape, seed=0)
+    x = inp["x"].to(dev)
+    w = {k: v.to(dev) for k, v in inp["layers"][0].items()}
+    beta = w["beta"]
+    p = ttcd.BlockParams.from_shape(shape)
+    ws = ttcd.alloc_workspace(ttcd.block_forward_workspace_size(p), dev)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ttcd.block_forward(x, beta, w, p, out=out, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, flags = ttcd.get_device_error()
+    if st != ttcd.OK:
+        raise RuntimeError(f"device error after warm-up: flags={flags}")
+
+    # ---- device-timed region: K steps, stage events on the launch stream
+    n_ev = len(STAGES) + 1
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+              for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    launches0 = ttcd.kernel_launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            ttcd.set_stage_events(events[i])
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    ttcd.set_stage_events(None)
+    launches = ttcd.kernel_launch_count() - launches0
+    barrier(world, local)
+    ms = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    st, flags = ttcd.get_device_error()
+    if st != ttcd.OK:
+        raise RuntimeError(f"device error in timed region: flags={flags}")
+    tokens = shape.B * shape.T * world
+    value = tokens / (ms / 1000.0)
+
+    # per-stage times (mean over steps) and roofline fractions
+    costs = stage_costs(shape)
+    stage_ms = [statistics.mean(events[i][k].elapsed_time(events[i][k + 1])
+                                for i in range(args.steps)) for k in range(len(STAGES))]
+    stages = {}
+    for name, (bound, amt), t in zip(STAGES, costs, stage_ms):
+        if bound == "tensor":
+            ach, peak, unit = amt / (t / 1e3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        else:
+            ach, peak, unit = amt / (t / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        stages[name] = {"ms": round(t, 4), "bound": bound, "achieved": round(ach, 2),
+                        "unit": unit, "frac": round(ach / peak, 4)}
+    att = stages["dual_window_attn"]
+    total_flops = sum(a for b, a in costs if b == "tensor")
+
+    # ---- end to end through the public API with host buffers
+    x_h = inp["x"].pin_memory()
+    b_h = inp["layers"][0]["beta"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_d, b_d = torch.empty_like(x), torch.empty_like(beta)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        b_d.copy_(b_h, non_blocking=True)
+        ttcd.block_forward(x_d, b_d, w, p, out=out, workspace=ws, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier(world, local)
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    ms_e2e = max_over_ranks(world, s2.elapsed_time(e2)) / args.steps
+    assert torch.equal(out_h, out.cpu())
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(shape, {"parallelism": f"replicas{world}"}),
+            "tflops_per_s": total_flops / (ms / 1e3) / 1e12,
+            "roofline": {"kernel": "dual_window_attn_kernel<128>", "bound": "tensor",
+                         "achieved": att["achieved"], "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": att["frac"],
+                         "traffic": args.attn_traffic_bytes,
+                         "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                         "flops_per_launch": attention_flops(shape)},
+            "stages": stages,
+            "e2e": {"value": tokens / (ms_e2e / 1000.0), "unit": UNIT,
+                    "h2d_bytes_per_step": x_h.numel() * x_h.element_size() +
+                    b_h.numel() * b_h.element_size(),
+                    "d2h_bytes_per_step": out_h.numel() * out_h.element_size()},
+            "gpu_launches": launches,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, times = oracle_throughput(shape, args.cpu_sample_tokens)
+        line["cpu_baseline"] = {
+            "value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"first {args.cpu_sample_tokens} tokens of the workload (attention windows "
+                      f"truncated by position), float64 NumPy oracle, {times[0]:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=2048)
+    ap.add_argument("--ref-sample-tokens", type=int, default=512)
+    ap.add_argument("--attn-traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

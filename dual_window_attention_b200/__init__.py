@@ -77,6 +77,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_status_string.argtypes = [i]
     lib.ttcd_status_string.restype = ctypes.c_char_p
     lib.ttcd_version.restype = ctypes.c_char_p
+    lib.ttcd_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
+    lib.ttcd_set_stage_events.restype = i
+    lib.ttcd_kernel_launch_count.argtypes = []
+    lib.ttcd_kernel_launch_count.restype = ctypes.c_ulonglong
     for fn in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward",
                "ttcd_block_workspace_offset", "ttcd_get_device_error", "ttcd_test_bounded_wait"):
         getattr(lib, fn).restype = i
@@ -257,6 +261,19 @@ def get_device_error(stream=None) -> Tuple[int, int]:
 
 def set_wait_timeout_ns(ns: int) -> None:
     load_library().ttcd_set_wait_timeout_ns(ns)
+
+
+def set_stage_events(events) -> None:
+    """Record torch.cuda.Event objects at the block's stage boundaries (None = off)."""
+    if not events:
+        _check(load_library().ttcd_set_stage_events(None, 0), "set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(load_library().ttcd_set_stage_events(arr, len(events)), "set_stage_events")
+
+
+def kernel_launch_count() -> int:
+    return int(load_library().ttcd_kernel_launch_count())
 
 
 def test_bounded_wait(timeout_ns: int, stream=None) -> int:

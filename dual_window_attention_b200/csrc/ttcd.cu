@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/ttcd.h"
@@ -97,9 +98,20 @@ bool map_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
   return make_map(m, ptr, cols, rows, cols * 2, 64, box_rows);
 }
 
-#define TTCD_CHECK_LAUNCH()                                   \
-  do {                                                        \
+std::atomic<unsigned long long> g_launches{0};
+constexpr int kMaxStageEvents = 16;
+cudaEvent_t g_stage_events[kMaxStageEvents];
+int g_n_stage_events = 0;
+
+// Records the stage-boundary event `k` on stream s when profiling hooks are set.
+void stage_mark(cudaStream_t s, int k) {
+  if (k < g_n_stage_events) cudaEventRecord(g_stage_events[k], s);
+}
+
+#define TTCD_CHECK_LAUNCH()                                      \
+  do {                                                           \
     if (cudaGetLastError() != cudaSuccess) return TTCD_ERR_CUDA; \
+    g_launches.fetch_add(1, std::memory_order_relaxed);          \
   } while (0)
 
 template <int BN, int STAGES, bool DUAL, class Epi>
@@ -298,8 +310,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
                          const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
                          const __nv_bfloat16* w_down, const void* w_proj, bool proj_f32,
                          const TapT* conv_T, const TapT* conv_S, const float* beta,
-                         const float* state_in, float* state_out, const ResT* h_S, OutT* y) {
+                         const float* state_in, float* state_out, const ResT* h_S, OutT* y,
+                         int mark) {
   const Dims m = dims_of(p);
+  stage_mark(c.s, mark);
   __nv_bfloat16* u = at<__nv_bfloat16>(ws, L, B_U);
   float* Z = at<float>(ws, L, B_Z);
   __nv_bfloat16* Zs16 = at<__nv_bfloat16>(ws, L, B_ZS16);
@@ -321,6 +335,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiSwiGLU e{Z, m.f, m.f};
     TTCD_TRY((launch_gemm<128, 6, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, m.f / 64, m.d), e)));
   }
+  stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
   if (cudaMemsetAsync(ssq, 0, m.P * sizeof(float), c.s) != cudaSuccess) return TTCD_ERR_CUDA;
   {
@@ -333,6 +348,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
                                                       m.Nc, m.P, p->l2_eps);
     TTCD_CHECK_LAUNCH();
   }
+  stage_mark(c.s, mark + 2);
   // M = W_down W_proj (associativity of W_down (W_proj d_t)).
   {
     dim3 tb(32, 8), tg(cdiv(m.f, 32), cdiv(m.f, 32));
@@ -347,6 +363,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiStoreBF16 e{M, m.f, m.f, nullptr};
     TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, plain_geom(m.d, m.f / 128 + (m.f % 128 ? 1 : 0), m.f), e)));
   }
+  stage_mark(c.s, mark + 3);
   // R^T = M D^T, scaled per token by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
@@ -354,6 +371,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiStoreBF16 e{Rt, m.P, static_cast<int>(m.P), kscale};
     TTCD_TRY((launch_gemm<256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.P, 256), m.f), e)));
   }
+  stage_mark(c.s, mark + 4);
   // Delta W per chunk, fp32 exclusive prefix scan, W_i = bf16(W_down + S_i).
   {
     CUtensorMap mR, mK;
@@ -379,6 +397,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     kern<<<p->B * a.tiles_m * a.tiles_n, GEMM_THREADS, smem, c.s>>>(mR, mK, a, c.st);
     TTCD_CHECK_LAUNCH();
   }
+  stage_mark(c.s, mark + 5);
   // y = h_S + (W_down + S_i) Z_S, one GEMM per chunk with its own weight.
   {
     CUtensorMap mA, mB;
@@ -397,6 +416,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
     TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, e)));
   }
+  stage_mark(c.s, mark + 6);
   return TTCD_OK;
 }
 
@@ -427,6 +447,16 @@ const char* ttcd_status_string(ttcd_status s) {
 }
 
 const char* ttcd_version(void) { return "ttcd 0.1 sm_100a"; }
+
+ttcd_status ttcd_set_stage_events(void* const* events, int n_events) {
+  if (n_events < 0 || n_events > kMaxStageEvents || (n_events > 0 && !events))
+    return TTCD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_n_stage_events = n_events;
+  return TTCD_OK;
+}
+
+unsigned long long ttcd_kernel_launch_count(void) { return g_launches.load(); }
 
 void ttcd_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
 
@@ -511,7 +541,7 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
         static_cast<const __nv_bfloat16*>(w->w_up), static_cast<const __nv_bfloat16*>(w->w_down),
         w->w_proj, false, static_cast<const __nv_bfloat16*>(w->conv_T),
         static_cast<const __nv_bfloat16*>(w->conv_S), beta, state_in, state_out,
-        static_cast<const __nv_bfloat16*>(h_S), static_cast<__nv_bfloat16*>(y));
+        static_cast<const __nv_bfloat16*>(h_S), static_cast<__nv_bfloat16*>(y), 0);
   }
   TTCD_TRY(cast_bf16<float>(c, u_T, u, m.BT * m.d));
   TTCD_TRY(cast_bf16<float>(c, u_S, u + m.BT * m.d, m.BT * m.d));
@@ -524,7 +554,7 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
   return run_mlp_core<float, float, float>(
       c, p, L, workspace, wg, wu, wd, w->w_proj, true, static_cast<const float*>(w->conv_T),
       static_cast<const float*>(w->conv_S), beta, state_in, state_out,
-      static_cast<const float*>(h_S), static_cast<float*>(y));
+      static_cast<const float*>(h_S), static_cast<float*>(y), 0);
 }
 
 ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_block_weights* w,
@@ -571,6 +601,7 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
   }
 
   // Rotary table, input RMSNorm.
+  stage_mark(c.s, 0);
   rope_table_kernel<<<cdiv(static_cast<long long>(p->T) * (m.hd / 2), 256), 256, 0, c.s>>>(
       rope, p->T, m.hd, static_cast<double>(p->rope_theta));
   TTCD_CHECK_LAUNCH();
@@ -582,6 +613,7 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w->g_attn), xn,
         m.BT, m.d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
+  stage_mark(c.s, 1);
 
   // Shared Q/K/V with RoPE.
   {
@@ -595,10 +627,12 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
       default: TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
     }
   }
+  stage_mark(c.s, 2);
   // Dual-window attention: o_T rows then o_S rows.
   const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
   TTCD_TRY(run_attn(c, q, k, v, o, o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq,
                     m.Hkv, m.hd, p->w_S, p->w_T, sc));
+  stage_mark(c.s, 3);
   // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
   {
     CUtensorMap mA, mB;
@@ -614,6 +648,7 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
       TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, e)));
     }
   }
+  stage_mark(c.s, 4);
   // u_P = RMSNorm(h_P; g_mlp) in bf16 for the gate/up GEMM.
   if (f32)
     rmsnorm_kernel<float, float><<<cdiv(2 * m.BT, 8), 256, 0, c.s>>>(
@@ -628,11 +663,11 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
     return run_mlp_core<float, float, float>(c, p, L, ws, wg, wu, wd, w->w_proj, true,
                                              static_cast<const float*>(w->conv_T),
                                              static_cast<const float*>(w->conv_S), beta, nullptr,
-                                             state_out, h_S, static_cast<float*>(out));
+                                             state_out, h_S, static_cast<float*>(out), 5);
   return run_mlp_core<__nv_bfloat16, float, __nv_bfloat16>(
       c, p, L, ws, wg, wu, wd, w->w_proj, false, static_cast<const __nv_bfloat16*>(w->conv_T),
       static_cast<const __nv_bfloat16*>(w->conv_S), beta, nullptr, state_out, h_S,
-      static_cast<__nv_bfloat16*>(out));
+      static_cast<__nv_bfloat16*>(out), 5);
 }
 
 __global__ void bounded_wait_test_kernel(DevStatus st) {

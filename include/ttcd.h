@@ -25,7 +25,7 @@
  *     extent times its element size must be a multiple of 16 bytes.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and keep no state between calls except the device error word
- *     read by ttcd_get_device_error().
+ *     read by ttcd_get_device_error() and the profiling hooks below.
  *   - Arguments are validated on the host before any launch; a bad argument
  *     returns TTCD_ERR_INVALID_ARG or TTCD_ERR_UNSUPPORTED and launches nothing.
  *     A launch failure returns TTCD_ERR_CUDA.  Every device-side wait is
@@ -196,6 +196,23 @@ void ttcd_set_wait_timeout_ns(uint64_t ns);
  * test can check the timeout path without hanging a GPU.
  */
 ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream);
+
+/*
+ * Profiling hooks (not part of the method; used by the benchmark).
+ * ttcd_set_stage_events: when n_events > 0, ttcd_block_forward records
+ * events[k] (cudaEvent_t handles owned by the caller) on its stream at stage
+ * boundary k: 0 start, 1 after the input RMSNorm, 2 after QKV+RoPE, 3 after
+ * attention, 4 after o_proj, 5 after the MLP RMSNorm, 6 after gate/up+SwiGLU,
+ * 7 after conv/residual/keys, 8 after M = W_down W_proj, 9 after R, 10 after
+ * the chunk scan, 11 after the output GEMM.  ttcd_fastweight_mlp records
+ * boundaries 0..6 of its own part (start, gate/up, conv, M, R, scan, output).
+ * Boundaries at or beyond n_events are skipped; n_events = 0 disables.
+ * Process-wide setting, not thread-safe.  At most 16 events.
+ */
+ttcd_status ttcd_set_stage_events(void* const* events, int n_events);
+
+/* Number of kernels this library has launched since it was loaded. */
+unsigned long long ttcd_kernel_launch_count(void);
 
 const char* ttcd_status_string(ttcd_status s);
 
