@@ -268,6 +268,9 @@ def set_stage_events(events) -> None:
     if not events:
         _check(load_library().ttcd_set_stage_events(None, 0), "set_stage_events")
         return
+    for e in events:  # torch creates the underlying CUDA event on first record
+        if not e.cuda_event:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(load_library().ttcd_set_stage_events(arr, len(events)), "set_stage_events")
 

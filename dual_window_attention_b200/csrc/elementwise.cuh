@@ -66,12 +66,12 @@ __global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double
 // papernotes.org review, 关键设计 3: Zbar_P = conv_P(Z_P) (depthwise, causal),
 // D = Zbar_T - Zbar_S, K = l2-norm(Zbar_S).  The per-row norm needs the whole
 // d_ff row, so this kernel writes Zbar_S unnormalised (transposed, Kt) and adds
-// its squares into ssq[p]; the scale beta_t / ||.|| is applied to the value
+// its squares into ssq_part[channel block][p]; the scale beta_t / ||.|| is applied to the value
 // residual instead (Delta W = sum beta r k^T is linear in that scale).
 //
 // Z     fp32 [2, BT, f]: teacher rows then student rows
 // taps  [f, k] (tap m multiplies t - m), TapT = bf16 or fp32
-// D     bf16 [P, f]      Kt bf16 [f, P]     Zs16 bf16 [BT, f]    ssq fp32 [P] (+=)
+// D     bf16 [P, f]      Kt bf16 [f, P]     Zs16 bf16 [BT, f]    ssq_part fp32 [f/64, P]
 // Padded index p = (b*Nc + i)*Cp + j holds token t = i*C + j when j < C and t < T;
 // other p get D = 0 and Kt = 0.
 // Block: 64 padded positions x 64 channels, 256 threads (thread = one position,
@@ -82,9 +82,10 @@ __global__ void __launch_bounds__(256)
     conv_residual_key_kernel(const float* __restrict__ Z, const TapT* __restrict__ tapT,
                              const TapT* __restrict__ tapS, __nv_bfloat16* __restrict__ D,
                              __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ Zs16,
-                             float* __restrict__ ssq, int T, int f, int k, int C, int Cp, int Nc,
-                             long long BT, long long P) {
+                             float* __restrict__ ssq_part, int T, int f, int k, int C, int Cp,
+                             int Nc, long long BT, long long P) {
   __shared__ __nv_bfloat16 tileK[CONV_TC][CONV_TP + 8];
+  __shared__ float sq_part[4][CONV_TP];
   const long long p0 = static_cast<long long>(blockIdx.x) * CONV_TP;
   const int c0 = blockIdx.y * CONV_TC;
   const int tp = threadIdx.x & 63;   // position within tile
@@ -157,8 +158,12 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int c = 0; c < 16; ++c) tileK[cg * 16 + c][tp] = __float2bfloat16_rn(zbS[c]);
-  if (valid) atomicAdd(ssq + p, sq);
+  sq_part[cg][tp] = sq;
   __syncthreads();
+  // Deterministic per-(channel block, position) partial sums; summed in order later.
+  if (cg == 0 && p < P)
+    ssq_part[static_cast<long long>(blockIdx.y) * P + p] =
+        ((sq_part[0][tp] + sq_part[1][tp]) + sq_part[2][tp]) + sq_part[3][tp];
   // Transposed store: each warp writes rows of Kt (64 positions = 128 bytes).
   for (int r = threadIdx.x >> 3; r < CONV_TC; r += 32) {
     const int seg = threadIdx.x & 7;  // 8 x 16 bytes per row
@@ -170,19 +175,22 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// kscale[p] = beta[b, t] / sqrt(ssq[p] + eps) for real tokens, 0 for padding.
-__global__ void key_scale_kernel(const float* __restrict__ ssq, const float* __restrict__ beta,
-                                 float* __restrict__ kscale, int T, int C, int Cp, int Nc,
-                                 long long P, float eps) {
+// kscale[p] = beta[b, t] / sqrt(ssq[p] + eps) for real tokens, 0 for padding, where
+// ssq[p] = sum over channel blocks (in order) of ssq_part[blk][p].
+__global__ void key_scale_kernel(const float* __restrict__ ssq_part, int n_part,
+                                 const float* __restrict__ beta, float* __restrict__ kscale,
+                                 int T, int C, int Cp, int Nc, long long P, float eps) {
   const long long p = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (p >= P) return;
+  float ssq = 0.f;
+  for (int i = 0; i < n_part; ++i) ssq += ssq_part[static_cast<long long>(i) * P + p];
   const long long seq_len_p = static_cast<long long>(Nc) * Cp;
   const int b = static_cast<int>(p / seq_len_p);
   const long long rem = p % seq_len_p;
   const int i = static_cast<int>(rem / Cp), j = static_cast<int>(rem % Cp);
   const int t = i * C + j;
   const bool valid = j < C && t < T;
-  kscale[p] = valid ? beta[static_cast<long long>(b) * T + t] * rsqrtf(ssq[p] + eps) : 0.f;
+  kscale[p] = valid ? beta[static_cast<long long>(b) * T + t] * rsqrtf(ssq + eps) : 0.f;
 }
 
 template <class InT>

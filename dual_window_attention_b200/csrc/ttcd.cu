@@ -105,7 +105,8 @@ int g_n_stage_events = 0;
 
 // Records the stage-boundary event `k` on stream s when profiling hooks are set.
 void stage_mark(cudaStream_t s, int k) {
-  if (k < g_n_stage_events) cudaEventRecord(g_stage_events[k], s);
+  if (k < g_n_stage_events && cudaEventRecord(g_stage_events[k], s) != cudaSuccess)
+    cudaGetLastError();  // a failed profiling record must not be reported as a launch error
 }
 
 #define TTCD_CHECK_LAUNCH()                                      \
@@ -218,7 +219,7 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
   sz[B_ZS16] = m.BT * m.f * 2;
   sz[B_D] = m.P * m.f * 2;
   sz[B_KT] = m.P * m.f * 2;
-  sz[B_SSQ] = m.P * 4;
+  sz[B_SSQ] = m.P * 4 * (m.f / 64);
   sz[B_KSCALE] = m.P * 4;
   sz[B_RT] = m.P * m.d * 2;
   sz[B_WALL] = static_cast<size_t>(p->B) * m.Nc * m.d * m.f * 2;
@@ -337,15 +338,14 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   }
   stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
-  if (cudaMemsetAsync(ssq, 0, m.P * sizeof(float), c.s) != cudaSuccess) return TTCD_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(m.P / CONV_TP), m.f / CONV_TC);
     conv_residual_key_kernel<TapT><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kt, Zs16, ssq,
                                                           p->T, m.f, p->conv_k, p->chunk, m.Cp,
                                                           m.Nc, m.BT, m.P);
     TTCD_CHECK_LAUNCH();
-    key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, beta, kscale, p->T, p->chunk, m.Cp,
-                                                      m.Nc, m.P, p->l2_eps);
+    key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, m.f / CONV_TC, beta, kscale, p->T,
+                                                      p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
     TTCD_CHECK_LAUNCH();
   }
   stage_mark(c.s, mark + 2);
@@ -451,6 +451,8 @@ const char* ttcd_version(void) { return "ttcd 0.1 sm_100a"; }
 ttcd_status ttcd_set_stage_events(void* const* events, int n_events) {
   if (n_events < 0 || n_events > kMaxStageEvents || (n_events > 0 && !events))
     return TTCD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return TTCD_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
   g_n_stage_events = n_events;
   return TTCD_OK;

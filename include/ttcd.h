@@ -171,7 +171,7 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  *   "o"    bf16 [2, B*T, Hq*hd]   (o_T rows, then o_S rows)
  *   "h"    fp32 [2, B*T, d]       "u" bf16 [2, B*T, d]
  *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f]
- *   "D"    bf16 [P, f]            "Kt" bf16 [f, P]        "ssq" fp32 [P]
+ *   "D"    bf16 [P, f]            "Kt" bf16 [f, P]        "ssq" fp32 [f/64, P]
  *   "Rt"   bf16 [d, P]            "Wall" bf16 [B*n_chunks, d, f]
  * where P = B * n_chunks * Cp, Cp = chunk rounded up to 64, and token t of
  * sequence b sits at padded index (b*n_chunks + t/C)*Cp + t%C.
