@@ -81,6 +81,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_set_stage_events.restype = i
     lib.ttcd_kernel_launch_count.argtypes = []
     lib.ttcd_kernel_launch_count.restype = ctypes.c_ulonglong
+    lib.ttcd_fastweight_mlp_noalloc.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp]
+    lib.ttcd_fastweight_mlp_noalloc.restype = i
+    lib.ttcd_fastweight_mlp_noalloc_capacity.argtypes = []
+    lib.ttcd_fastweight_mlp_noalloc_capacity.restype = sz
     for fn in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward",
                "ttcd_block_workspace_offset", "ttcd_get_device_error", "ttcd_test_bounded_wait"):
         getattr(lib, fn).restype = i
@@ -250,6 +254,24 @@ def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockPar
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "ttcd_fastweight_mlp")
     return y, st_t, workspace
+
+
+def fastweight_mlp_noalloc(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams,
+                           h_S=None, state_in=None, state_out=None, y=None, stream=None):
+    """ttcd_fastweight_mlp without a workspace: for callers that cannot allocate scratch.
+
+    The scratch is the library's fixed 32 MiB device array; larger problems are
+    rejected.  Outputs `y` and `state_out` (fp32 [B, d, f]) are the caller's
+    tensors when given.  Calls that overlap on the GPU race on the shared array.
+    Returns (y, state_out).
+    """
+    lib = load_library()
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_fastweight_mlp_noalloc(_ptr(u_T), _ptr(u_S), _ptr(h_S), _ptr(beta),
+                                         ctypes.byref(wc), ctypes.byref(pc), _ptr(state_in),
+                                         _ptr(state_out), _ptr(y), _stream(stream))
+    _check(st, "ttcd_fastweight_mlp_noalloc")
+    return y, state_out
 
 
 def get_device_error(stream=None) -> Tuple[int, int]:

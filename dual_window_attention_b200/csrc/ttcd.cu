@@ -672,6 +672,48 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
       static_cast<__nv_bfloat16*>(out), 5);
 }
 
+// ---------------------------------------------------------------------------
+// Fast-weight MLP without caller-provided scratch.
+//
+// Some callers cannot hand this library a workspace: a host framework may own
+// every byte of device memory through its own pool and expose no way to borrow
+// from it, and a latency-critical loop may not be allowed to call cudaMalloc
+// (which can synchronise the device).  For them the scratch of one
+// ttcd_fastweight_mlp call lives in this fixed array instead.  It is part of
+// the library image, so every GPU that loads the library holds these 32 MiB
+// until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_ttcd_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_scratch_addr[kMaxDevices] = {nullptr};
+
+ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const void* h_S,
+                                        const float* beta, const ttcd_block_weights* w,
+                                        const ttcd_block_params* p, const float* state_in,
+                                        float* state_out, void* y, void* stream) {
+  TTCD_TRY(check_params(p));
+  const size_t need = make_layout(p, false).total;
+  if (need > kNoAllocScratchBytes) return TTCD_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTCD_ERR_CUDA;
+  {
+    // One-time set-up per device, made with that device current: the array's
+    // name is only a host-side stand-in, the kernels need its device address.
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_scratch_addr[dev]) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_ttcd_noalloc_scratch) != cudaSuccess || !addr)
+        return TTCD_ERR_CUDA;
+      g_noalloc_scratch_addr[dev] = addr;
+    }
+  }
+  // Every byte of scratch that a call reads is written earlier in the same
+  // call, so nothing has to be cleared between calls.
+  return ttcd_fastweight_mlp(u_T, u_S, h_S, beta, w, p, state_in, state_out, y,
+                             g_noalloc_scratch_addr[dev], kNoAllocScratchBytes, stream);
+}
+
+size_t ttcd_fastweight_mlp_noalloc_capacity(void) { return kNoAllocScratchBytes; }
+
 __global__ void bounded_wait_test_kernel(DevStatus st) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;

@@ -159,6 +159,36 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
                                const ttcd_block_params* p, float* state_out, void* out,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * ttcd_fastweight_mlp_noalloc — ttcd_fastweight_mlp for callers that cannot
+ * provide scratch memory.  The paper has no counterpart; this is a deployment
+ * convenience.
+ *
+ * Who needs it: callers whose device memory is owned entirely by a host
+ * framework's pool with no way to borrow a workspace from it, and callers in
+ * latency-critical loops that may not call cudaMalloc (it can synchronise the
+ * device).  Same arguments and result as ttcd_fastweight_mlp, without the
+ * workspace pair: the scratch is a fixed 32 MiB array compiled into the library
+ * (held by every GPU that loads the library until the process exits).  The
+ * library allocates nothing for it.
+ *   - Problems whose ttcd_fastweight_mlp_workspace_size exceeds
+ *     ttcd_fastweight_mlp_noalloc_capacity() (32 MiB) are rejected with
+ *     TTCD_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (every byte a call reads is written earlier in the same call, so
+ *     nothing needs clearing).  Calls whose kernels overlap on the GPU (other
+ *     streams, other host threads) race on it: serialise them.
+ */
+ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const void* h_S,
+                                        const float* beta, const ttcd_block_weights* w,
+                                        const ttcd_block_params* p, const float* state_in,
+                                        float* state_out, void* y, void* stream);
+
+/* Bytes of the fixed scratch array used by ttcd_fastweight_mlp_noalloc. */
+size_t ttcd_fastweight_mlp_noalloc_capacity(void);
+
 /* Workspace bytes needed by each entry point; 0 if the parameters are invalid. */
 size_t ttcd_fastweight_mlp_workspace_size(const ttcd_block_params* p);
 size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
