@@ -328,6 +328,51 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_attention(args, world, rank, local):
+    """Fused dual-window attention alone (Qwen3-0.6B head layout) for each window pair."""
+    import dual_window_attention_b200 as ttcd
+    from ttcd_workloads import QWEN3_0P6B_64K, make_attention_inputs
+    ttcd.load_library()
+    peaks, peak_kind = load_peaks()
+    s0 = QWEN3_0P6B_64K.with_(T=args.T, B=args.B)
+    q, k, v = make_attention_inputs(s0.B, s0.T, s0.n_q_heads, s0.n_kv_heads, s0.head_dim, seed=0)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    o_T, o_S = torch.empty_like(q), torch.empty_like(q)
+    pairs = [(int(a), int(b)) for a, b in (w.split("/") for w in args.windows.split(","))]
+    stream = torch.cuda.current_stream()
+    for wS, wT in pairs:
+        shape = s0.with_(w_S=wS, w_T=wT)
+        for _ in range(args.warmup):
+            ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, local)
+        e0.record(stream)
+        for _ in range(args.steps):
+            ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+        assert ttcd.get_device_error()[0] == ttcd.OK
+        fl = attention_flops(shape)
+        ach = fl / (ms / 1e3) / 1e12
+        if rank == 0:
+            print(json.dumps({
+                "metric": "fused dual-window attention tokens/s (Qwen3-0.6B heads)",
+                "value": shape.B * shape.T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "dual_window_attention", "B": shape.B, "T": shape.T,
+                           "n_q_heads": 16, "n_kv_heads": 8, "head_dim": 128, "w_S": wS,
+                           "w_T": wT},
+                "roofline": {"kernel": "dual_window_attn_kernel<128>", "bound": "tensor",
+                             "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": ach / peaks["bf16_tflops"],
+                             "peak_source": f"{peak_kind} bf16_tflops (burst: kernel timed alone)",
+                             "flops_per_launch": fl}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -337,6 +382,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=2048)
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
+    ap.add_argument("--mode", choices=["block", "attn"], default="block",
+                    help="block: the whole IP-TTCD block (default); attn: attention alone")
+    ap.add_argument("--T", type=int, default=65536, help="--mode attn: tokens per sequence")
+    ap.add_argument("--B", type=int, default=1, help="--mode attn: sequences")
+    ap.add_argument("--windows", default="512/8192",
+                    help="--mode attn: comma-separated w_S/w_T pairs")
     ap.add_argument("--attn-traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture")
     args = ap.parse_args()
@@ -344,6 +395,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.mode == "attn":
+            run_attention(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

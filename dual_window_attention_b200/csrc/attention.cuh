@@ -7,22 +7,30 @@
 // (long-window teacher and short-window student over a shared backbone);
 // podcast cue 19 (each token sees the last w tokens).
 //
-// One CTA owns a 128-row query tile of one (sequence, query head).  K/V tiles
-// of 128 keys are visited from the diagonal outwards ("near to far").  Every
-// Q.K^T tile is computed once; its exponentials are shared by both windows:
-//   - while the tile touches some row's student window, the student part of P
-//     accumulates into O_S (TMEM) and the teacher-only part into O_X;
-//   - afterwards only O_X accumulates.
-// Each accumulator keeps the running-max reference it was last rescaled to;
-// at the end  O_T = (O_S a + O_X) / (l_S a + l_X),  a = 2^(m_S - m_X).
-// Rescaling is lazy: the reference only moves when a row maximum grows by more
-// than 2^8, which keeps every exponential <= 256 and is exact in real
-// arithmetic (the same reference divides out in l).
+// Work unit: one CTA owns the same 128-row query block of up to two query
+// heads that share one KV head (GQA), so every K/V tile it loads serves both.
+// Each head's rows have one TMEM accumulator O and run in two phases over key
+// tiles of 128, visited from the diagonal outwards:
+//   phase 1 (student): tiles 0..jS, scores masked to the student window
+//            [t-w_S+1, t]; when it ends, O/l is the student output o_S;
+//   phase 2 (teacher): tiles jX..n-1, scores masked to the teacher-only band
+//            [t-w_T+1, t-w_S], accumulated on top of the same O, m, l; at the
+//            end O/l is the teacher output o_T.
+// So each Q.K^T product and each exponential serves both windows; the one
+// tile that straddles the student edge (jX <= jS) is computed in both phases.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 softmax (thread = query row) and epilogue.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O_S [256,256+HD), O_X [384,384+HD).
-// P of tile j overwrites S_{j%2}: P_S in columns [0,64), P_X in [64,128) as bf16 pairs.
+// Pipeline (one CTA, 384 threads):
+//   warp 0      TMA producer: Q of both heads once, then K and V per visit
+//   warp 1      TMEM owner and tcgen05.mma issuer (one thread), ping-pong:
+//               PV_A(v), QK_A(v+1), PV_B(v), QK_B(v+1), ...
+//   warps 4..7  softmax of head A (thread = query row), warps 8..11 head B
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+HD), O_B [384,384+HD);
+// P (bf16 pairs) overwrites the first 64 columns of its S and is the A operand
+// of the PV product straight from TMEM.  Because QK_A(v) is issued after
+// PV_A(v-1), "S_A(v) ready" implies O_A holds every earlier tile, so the
+// softmax warps may rescale or read O without a further wait.
+// Rescaling is lazy: the running-max reference moves only when a row maximum
+// grows by more than 2^8 (exponentials stay <= 256; exact in real arithmetic).
 #pragma once
 #include "gemm.cuh"
 
@@ -37,44 +45,106 @@ struct AttnArgs {
   int w_S, w_T;
   float scale_log2;  // softmax scale * log2(e)
   int n_qt;          // query tiles per sequence
+  int pairs;         // head pairs per KV group = ceil(G / 2)
 };
 
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;
-constexpr int ATT_KS = 3;  // K stages
+constexpr int ATT_KS = 2;  // K stages
 constexpr int ATT_VS = 2;  // V stages
-constexpr int ATT_THREADS = 192;
+constexpr int ATT_THREADS = 384;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 template <int HD>
 struct AttnCfg {
   static constexpr int PANELS = HD > 64 ? 2 : 1;  // 64-column (128-byte) panels per tile
   static constexpr int TILE_BYTES = PANELS * ATT_BM * 128;
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE_BYTES;
+  static constexpr int QA_OFF = 0;
+  static constexpr int QB_OFF = TILE_BYTES;
+  static constexpr int K_OFF = 2 * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + ATT_KS * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + ATT_VS * TILE_BYTES;
   // at least 120 KB so that a single CTA (which takes all 512 TMEM columns)
   // is resident per SM
-  static constexpr int SMEM = (1024 + BAR_OFF + 512) > 122880 ? (1024 + BAR_OFF + 512) : 122880;
-  // bytes each TMA tile load delivers (box is 64 columns even when HD = 32)
-  static constexpr uint32_t LOAD_BYTES = PANELS * ATT_BM * 128;
+  static constexpr int SMEM_RAW = 1024 + BAR_OFF + 512;
+  static constexpr int SMEM = SMEM_RAW > 122880 ? SMEM_RAW : 122880;
+  static constexpr uint32_t LOAD_BYTES = PANELS * ATT_BM * 128;  // box is 64 columns even at HD 32
 };
 
-// Key-window geometry of a (query tile, key tile) pair.
-struct TileGeom {
-  int q0, k0;
-  __device__ bool has_S(int w_S) const { return k0 + ATT_BN - 1 >= q0 - w_S + 1; }
-  __device__ bool has_X(int w_S, int w_T) const {
-    return k0 <= q0 + ATT_BM - 1 - w_S && k0 + ATT_BN - 1 >= q0 - w_T + 1;
+// Visit schedule of one 128-row query tile; identical for every role.
+struct Visits {
+  int n_tiles;  // key tiles that touch the teacher window
+  int jS;       // last student tile
+  int jX;       // first teacher-only tile
+  int nv;       // visits
+  int vX;       // first phase-2 visit (== nv when there is no phase 2)
+  __device__ Visits(int qt, int w_S, int w_T) {
+    n_tiles = min(qt, (w_T + ATT_BN - 2) / ATT_BN) + 1;
+    jS = min(n_tiles - 1, (w_S + ATT_BN - 2) / ATT_BN);
+    jX = w_S / ATT_BN;
+    const bool phase2 = w_T > w_S && jX <= n_tiles - 1;
+    vX = jS + 1;
+    nv = vX + (phase2 ? n_tiles - jX : 0);
   }
-  // every (row, key) of the tile lies in the window w
-  __device__ bool full(int w) const { return k0 + ATT_BN - 1 <= q0 && k0 >= q0 + ATT_BM - w; }
+  __device__ int tile(int v) const { return v < vX ? v : jX + (v - vX); }
 };
 
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x on the FMA pipe for a pair: round-to-nearest range reduction with the
+// 1.5 * 2^23 shifter, then 2^f for f in [-0.5, 0.5] by a cubic whose
+// coefficients were fitted to 2^f (relative error weighted least squares on
+// Chebyshev nodes, Lawson reweighting; max relative error 1.0e-4), and the
+// integer part added to the exponent field.  Inputs are clamped at -126.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
+  constexpr float C1 = 0.6932829022407532f, C2 = 0.24221095442771912f,
+                  C3 = 0.05500892922282219f;
+  float x0, x1;
+  f2unpack(x, x0, x1);
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t xc = f2pack(x0, x1);
+  const uint64_t t = add2(xc, f2pack(SHIFT, SHIFT));
+  const uint64_t n = add2(t, f2pack(-SHIFT, -SHIFT));
+  const uint64_t fr = fma2(n, f2pack(-1.0f, -1.0f), xc);
+  uint64_t p = fma2(fr, f2pack(C3, C3), f2pack(C2, C2));
+  p = fma2(p, fr, f2pack(C1, C1));
+  p = fma2(p, fr, f2pack(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2pack(r0, r1);
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < N / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + 32 * c, r);
 #pragma unroll
@@ -84,7 +154,7 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
 }
 
 template <int HD>
-__device__ __forceinline__ void tmem_scale_rows(uint32_t taddr, float alpha) {
+__device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
 #pragma unroll
   for (int c = 0; c < HD; c += 32) {
     uint32_t r[32];
@@ -97,6 +167,20 @@ __device__ __forceinline__ void tmem_scale_rows(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
+// Normalise this thread's O row by 1/l and store it (bf16) to dst.
+template <int HD>
+__device__ __forceinline__ void tmem_store_row(uint32_t taddr, float inv_l, __nv_bfloat16* dst,
+                                               bool ok) {
+#pragma unroll
+  for (int c = 0; c < HD; c += 32) {
+    float v[32];
+    tmem_ld32f(taddr + c, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= inv_l;
+    if (ok) store_bf16x32(dst + c, v);
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     dual_window_attn_kernel(const __grid_constant__ CUtensorMap mapQ,
@@ -106,45 +190,50 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   using Cfg = AttnCfg<HD>;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(ATT_BM, ATT_BN, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(ATT_BM, HD, false, true);
-  constexpr uint32_t COL_O_S = 256, COL_O_X = 384;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + ATT_KS;
-  uint64_t* v_full = k_empty + ATT_KS;
-  uint64_t* v_empty = v_full + ATT_VS;
-  uint64_t* s_full = v_empty + ATT_VS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* o_done = pv_done + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* q_full = bars;                  // 1
+  uint64_t* k_full = bars + 1;              // KS
+  uint64_t* k_empty = k_full + ATT_KS;      // KS
+  uint64_t* v_full = k_empty + ATT_KS;      // VS
+  uint64_t* v_empty = v_full + ATT_VS;      // VS
+  uint64_t* s_full = v_empty + ATT_VS;      // 2 (per head)
+  uint64_t* p_full = s_full + 2;            // 2 (per head, 128 arrivals)
+  uint64_t* o_done = p_full + 2;            // 2 (per head)
+  uint64_t* drain = o_done + 2;             // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: longest (latest) query tiles first; heads of a GQA group adjacent.
-  const int per_tile = a.B * a.Hq;
-  const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / per_tile;
-  const int bh = static_cast<int>(blockIdx.x) % per_tile;
-  const int b = bh / a.Hq;
-  const int h = bh % a.Hq;
-  const int g = h / (a.Hq / a.Hkv);
+  // Work item: longest (latest) query tiles first.
+  const int G = a.Hq / a.Hkv;
+  const int per_qt = a.B * a.Hkv * a.pairs;
+  const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / per_qt;
+  int rem = static_cast<int>(blockIdx.x) % per_qt;
+  const int pair = rem % a.pairs;
+  rem /= a.pairs;
+  const int g = rem % a.Hkv;
+  const int b = rem / a.Hkv;
+  const int hA = g * G + 2 * pair;
+  const bool hasB = 2 * pair + 1 < G;
+  const int hB = hasB ? hA + 1 : hA;
   const int q0 = qt * ATT_BM;
-  const int n_tiles = min(qt, (a.w_T + ATT_BN - 2) / ATT_BN) + 1;
+  const Visits vis(qt, a.w_S, a.w_T);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < ATT_KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < ATT_VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&p_full[s], 128); }
-    mbar_init(pv_done, 1);
-    mbar_init(o_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_done[s], 1);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -160,28 +249,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
+  // Register split: the launch gives 384 x 168 = 64512 registers; the control
+  // warpgroup (warps 0-3) keeps 128 x 56, the two softmax warpgroups take
+  // 256 x 224, which adds up to the same 64512.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------- TMA producer
       const int row_base = b * a.T;
       int issued_k = 0, issued_v = 0;
-      mbar_arrive_expect_tx(q_full, Cfg::LOAD_BYTES);
+      mbar_arrive_expect_tx(q_full, (hasB ? 2 : 1) * Cfg::LOAD_BYTES);
 #pragma unroll
-      for (int p = 0; p < Cfg::PANELS; ++p)
-        tma_load_2d(smem + Cfg::Q_OFF + p * ATT_BM * 128, &mapQ, q_full, h * HD + 64 * p,
+      for (int p = 0; p < Cfg::PANELS; ++p) {
+        tma_load_2d(smem + Cfg::QA_OFF + p * ATT_BM * 128, &mapQ, q_full, hA * HD + 64 * p,
                     row_base + q0);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int row = row_base + q0 - ATT_BN * j;
-        const int ks = j % ATT_KS, vs = j % ATT_VS;
-        if (!mbar_wait(&k_empty[ks], ((j / ATT_KS) & 1) ^ 1, st, abort)) break;
+        if (hasB)
+          tma_load_2d(smem + Cfg::QB_OFF + p * ATT_BM * 128, &mapQ, q_full, hB * HD + 64 * p,
+                      row_base + q0);
+      }
+      for (int v = 0; v < vis.nv; ++v) {
+        const int row = row_base + q0 - ATT_BN * vis.tile(v);
+        const int ks = v % ATT_KS, vs = v % ATT_VS;
+        if (!mbar_wait(&k_empty[ks], ((v / ATT_KS) & 1) ^ 1, st, abort)) break;
         mbar_arrive_expect_tx(&k_full[ks], Cfg::LOAD_BYTES);
 #pragma unroll
         for (int p = 0; p < Cfg::PANELS; ++p)
           tma_load_2d(smem + Cfg::K_OFF + ks * Cfg::TILE_BYTES + p * ATT_BN * 128, &mapK,
                       &k_full[ks], g * HD + 64 * p, row);
         ++issued_k;
-        if (!mbar_wait(&v_empty[vs], ((j / ATT_VS) & 1) ^ 1, st, abort)) break;
+        if (!mbar_wait(&v_empty[vs], ((v / ATT_VS) & 1) ^ 1, st, abort)) break;
         mbar_arrive_expect_tx(&v_full[vs], Cfg::LOAD_BYTES);
 #pragma unroll
         for (int p = 0; p < Cfg::PANELS; ++p)
@@ -195,182 +291,167 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_wait(&k_full[j % ATT_KS], (j / ATT_KS) & 1, st, &no_abort);
       for (int j = max(0, issued_v - ATT_VS); j < issued_v; ++j)
         mbar_wait(&v_full[j % ATT_VS], (j / ATT_VS) & 1, st, &no_abort);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------- MMA issuer
-      bool ok = mbar_wait(q_full, 0, st, abort);
-      const uint32_t sq = smem_u32(smem + Cfg::Q_OFF);
-      bool x_started = false;
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(&p_full[jj & 1], (jj >> 1) & 1, st, abort)) return false;
-        if (!mbar_wait(&v_full[jj % ATT_VS], (jj / ATT_VS) & 1, st, abort)) return false;
-        tc_fence_after();
-        const TileGeom tg{q0, q0 - ATT_BN * jj};
-        const uint32_t sv = smem_u32(smem + Cfg::V_OFF + (jj % ATT_VS) * Cfg::TILE_BYTES);
-        const uint32_t p_col = tmem + (jj & 1) * 128;
-        if (tg.has_S(a.w_S)) {
-#pragma unroll
-          for (int kk = 0; kk < ATT_BN / 16; ++kk)
-            mma_bf16_ts(tmem + COL_O_S, p_col + kk * 8, sdesc_sw128(sv + kk * 2048, ATT_BM * 128, 1024),
-                        IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        if (tg.has_X(a.w_S, a.w_T)) {
-#pragma unroll
-          for (int kk = 0; kk < ATT_BN / 16; ++kk)
-            mma_bf16_ts(tmem + COL_O_X, p_col + 64 + kk * 8,
-                        sdesc_sw128(sv + kk * 2048, ATT_BM * 128, 1024), IDESC_PV,
-                        (x_started || kk > 0) ? 1u : 0u);
-          x_started = true;
-        }
-        mma_commit(&v_empty[jj % ATT_VS]);
-        mma_commit(pv_done);
-        return true;
-      };
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const int ks = j % ATT_KS;
-        if (!mbar_wait(&k_full[ks], (j / ATT_KS) & 1, st, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + Cfg::K_OFF + ks * Cfg::TILE_BYTES);
-        const uint32_t s_col = tmem + (j & 1) * 128;
+      const uint32_t sq[2] = {smem_u32(smem + Cfg::QA_OFF), smem_u32(smem + Cfg::QB_OFF)};
+      const int nh = hasB ? 2 : 1;
+      auto issue_qk = [&](int h, int v) {
+        const uint32_t sk = smem_u32(smem + Cfg::K_OFF + (v % ATT_KS) * Cfg::TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (ATT_BM * 128) + (kk & 3) * 32;
-          mma_bf16_ss(s_col, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024),
-                      IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + h * 128, sdesc_sw128(sq[h] + off, 16, 1024),
+                      sdesc_sw128(sk + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[j & 1]);
-        mma_commit(&k_empty[ks]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        mma_commit(&s_full[h]);
+      };
+      auto issue_pv = [&](int h, int v) {
+        const uint32_t sv = smem_u32(smem + Cfg::V_OFF + (v % ATT_VS) * Cfg::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < ATT_BN / 16; ++kk)
+          mma_bf16_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8,
+                      sdesc_sw128(sv + kk * 2048, ATT_BM * 128, 1024), IDESC_PV,
+                      (v > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&o_done[h]);
+      };
+      bool ok = mbar_wait(q_full, 0, st, abort) && mbar_wait(&k_full[0], 0, st, abort);
+      if (ok) {
+        tc_fence_after();
+        for (int h = 0; h < nh; ++h) issue_qk(h, 0);
+        mma_commit(&k_empty[0]);
       }
-      if (ok && issue_pv(n_tiles - 1)) mma_commit(o_done);
+      for (int v = 0; v < vis.nv && ok; ++v) {
+        const bool more = v + 1 < vis.nv;
+        if (!mbar_wait(&v_full[v % ATT_VS], (v / ATT_VS) & 1, st, abort)) { ok = false; break; }
+        if (more && !mbar_wait(&k_full[(v + 1) % ATT_KS], ((v + 1) / ATT_KS) & 1, st, abort)) {
+          ok = false;
+          break;
+        }
+        for (int h = 0; h < nh; ++h) {
+          if (!mbar_wait(&p_full[h], v & 1, st, abort)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(h, v);
+          if (more) issue_qk(h, v + 1);
+        }
+        if (!ok) break;
+        if (more) mma_commit(&k_empty[(v + 1) % ATT_KS]);
+        mma_commit(&v_empty[v % ATT_VS]);
+      }
       mma_commit(drain);
       volatile int no_abort = 0;
       mbar_wait(drain, 0, st, &no_abort);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
     // --------------------------------------------------------------- softmax rows
+    const int h_local = (warp - 4) >> 2;  // 0: head A, 1: head B
+    const bool active = h_local == 0 || hasB;
+    const int head = h_local == 0 ? hA : hB;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int t = q0 + r;  // query position inside the sequence
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    float m_ref = 0.f, mS = 0.f, mX = 0.f, lS = 0.f, lX = 0.f;
-    bool x_started = false;
-    bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const TileGeom tg{q0, q0 - ATT_BN * j};
-      const bool hs = tg.has_S(a.w_S);
-      const bool hx = tg.has_X(a.w_S, a.w_T);
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, st, abort)) { ok = false; break; }
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + h_local * 128;
+    const uint32_t o_addr = tmem + lane_off + 256 + h_local * 128;
+    const bool row_ok = t < a.T;
+    const long long orow = (static_cast<long long>(b) * a.T + t) * a.Hq + head;
+    const long long li = (static_cast<long long>(b) * a.Hq + head) * a.T + t;
+    const float sl2 = a.scale_log2;
+    float m_ref = 0.f, l = 0.f;
+    bool ok = active;
+    for (int v = 0; v < vis.nv && ok; ++v) {
+      const int j = vis.tile(v);
+      const int k0 = q0 - ATT_BN * j;
+      const bool ph2 = v >= vis.vX;
+      if (!mbar_wait(&s_full[h_local], v & 1, st, abort)) { ok = false; break; }
       tc_fence_after();
-      float s[128];
-      tmem_ld128(lane_addr + (j & 1) * 128, s);
-      // Masks: teacher-valid keys, and which of those are student keys.
-      const bool maskT = !tg.full(a.w_T);
-      const bool all_student = hs && !hx && tg.full(a.w_S);
-      float tile_max = -INFINITY;
-      uint32_t in_S_bits[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const int key = tg.k0 + c;
-        const bool vT = !maskT || (key <= t && key >= t - a.w_T + 1);
-        const bool vS = key <= t && key >= t - a.w_S + 1;
-        if (vS) in_S_bits[c >> 5] |= 1u << (c & 31);
-        s[c] = vT ? s[c] * a.scale_log2 : -INFINITY;
-        tile_max = fmaxf(tile_max, s[c]);
+      if (v == vis.vX) {
+        // end of the student phase: O / l is o_S (PV of every earlier tile has landed)
+        tmem_store_row<HD>(o_addr, 1.f / l, a.o_S + orow * HD, row_ok);
+        if (row_ok && a.lse_S) a.lse_S[li] = (m_ref + __log2f(l)) * 0.6931471805599453f;
       }
-      if (j == 0) {
-        m_ref = tile_max;
-        mS = m_ref;
+      float s[128];
+      tmem_ld_cols<128>(s_addr, s);
+      // visible key columns [lo, hi] of this row in this tile
+      const int lo = ph2 ? t - a.w_T + 1 - k0 : t - a.w_S + 1 - k0;
+      const int hi = ph2 ? t - a.w_S - k0 : t - k0;
+      const bool unmasked = ph2 ? (k0 >= q0 + ATT_BM - a.w_T && k0 + ATT_BN - 1 <= q0 - a.w_S)
+                                : (j >= 1 && k0 >= q0 + ATT_BM - a.w_S);
+      if (!unmasked) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
+      }
+      float mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+      for (int c = 3; c < 127; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+      mx = fmaxf(mx, s[127]);
+      const float m_tile = mx * sl2;
+      if (v == 0) {
+        m_ref = m_tile;
       } else {
-        const bool grow = tile_max > m_ref + ATT_RESCALE_THRESHOLD;
+        const bool grow = m_tile > m_ref + ATT_RESCALE_THRESHOLD;
         if (__any_sync(0xffffffffu, grow)) {
-          const float m_new = grow ? tile_max : m_ref;
-          // O may only be touched once the previous PV product has landed.
-          if (!mbar_wait(pv_done, (j - 1) & 1, st, abort)) { ok = false; break; }
-          tc_fence_after();
-          if (hs) {
-            const float al = ex2_approx(mS - m_new);
-            tmem_scale_rows<HD>(lane_addr + COL_O_S, al);
-            lS *= al;
-            mS = m_new;
-          }
-          if (hx && x_started) {
-            const float al = ex2_approx(mX - m_new);
-            tmem_scale_rows<HD>(lane_addr + COL_O_X, al);
-            lX *= al;
-            mX = m_new;
-          }
+          const float m_new = grow ? m_tile : m_ref;
+          const float al = ex2_approx(m_ref - m_new);
+          tmem_scale_row<HD>(o_addr, al);
+          l *= al;
           m_ref = m_new;
         }
       }
-      if (hx && !x_started) { mX = m_ref; x_started = true; }
-      // Exponentials once; split into the student and teacher-only parts.
-      uint32_t pS[64], pX[64];
-      float sumS = 0.f, sumX = 0.f;
+      // exponentials, row sum, bf16 pack
+      const uint64_t sc2 = f2pack(sl2, sl2);
+      const uint64_t nm2 = f2pack(-m_ref, -m_ref);
+      uint64_t acc = f2pack(0.f, 0.f);
+      uint32_t P[64];
+      if (unmasked) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float e0 = ex2_approx(s[c] - m_ref);
-        const float e1 = ex2_approx(s[c + 1] - m_ref);
-        const bool s0 = all_student || ((in_S_bits[c >> 5] >> (c & 31)) & 1u);
-        const bool s1 = all_student || ((in_S_bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
-        const float a0 = s0 ? e0 : 0.f, a1 = s1 ? e1 : 0.f;
-        const float b0 = s0 ? 0.f : e0, b1 = s1 ? 0.f : e1;
-        sumS += a0 + a1;
-        sumX += b0 + b1;
-        pS[c >> 1] = pack_bf16x2(a0, a1);
-        pX[c >> 1] = pack_bf16x2(b0, b1);
+        for (int c = 0; c < 128; c += 2) {
+          uint64_t x = fma2(f2pack(s[c], s[c + 1]), sc2, nm2);
+          uint64_t e;
+          if ((c & 14) == 14) {  // one pair in eight on the FMA pipe
+            e = exp2_poly2(x);
+          } else {
+            float x0, x1;
+            f2unpack(x, x0, x1);
+            e = f2pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc = add2(acc, e);
+          float e0, e1;
+          f2unpack(e, e0, e1);
+          P[c >> 1] = pack_bf16x2(e0, e1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          uint64_t x = fma2(f2pack(s[c], s[c + 1]), sc2, nm2);
+          float x0, x1;
+          f2unpack(x, x0, x1);
+          const uint64_t e = f2pack(ex2_approx(x0), ex2_approx(x1));
+          acc = add2(acc, e);
+          float e0, e1;
+          f2unpack(e, e0, e1);
+          P[c >> 1] = pack_bf16x2(e0, e1);
+        }
       }
-      const uint32_t p_addr = lane_addr + (j & 1) * 128;
-      if (hs) {
-        lS += sumS;
-        tmem_st32(p_addr, *reinterpret_cast<uint32_t(*)[32]>(&pS[0]));
-        tmem_st32(p_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pS[32]));
-      }
-      if (hx) {
-        lX += sumX;
-        tmem_st32(p_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&pX[0]));
-        tmem_st32(p_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&pX[32]));
-      }
+      float a0, a1;
+      f2unpack(acc, a0, a1);
+      l += a0 + a1;
+      tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&P[0]));
+      tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&P[32]));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[h_local]);
     }
     // ------------------------------------------------------------------ epilogue
-    if (ok && mbar_wait(o_done, 0, st, abort)) {
+    if (ok && mbar_wait(&o_done[h_local], (vis.nv - 1) & 1, st, abort)) {
       tc_fence_after();
-      const bool row_ok = t < a.T;
-      const float inv_S = 1.f / lS;
-      const float sc = x_started ? ex2_approx(mS - mX) : 0.f;
-      const float lT = x_started ? lS * sc + lX : lS;
-      const float inv_T = 1.f / lT;
-      const long long orow = (static_cast<long long>(b) * a.T + t) * a.Hq + h;
-#pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        float os[32], ox[32];
-        tmem_ld32f(lane_addr + COL_O_S + c, os);
-        if (x_started) {
-          tmem_ld32f(lane_addr + COL_O_X + c, ox);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ox[i] = 0.f;
-        }
-        float vs[32], vt[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          vs[i] = os[i] * inv_S;
-          vt[i] = x_started ? (os[i] * sc + ox[i]) * inv_T : vs[i];
-        }
-        if (row_ok) {
-          store_bf16x32(a.o_S + orow * HD + c, vs);
-          store_bf16x32(a.o_T + orow * HD + c, vt);
-        }
-      }
-      if (row_ok) {
-        const float ln2 = 0.6931471805599453f;
-        const long long li = (static_cast<long long>(b) * a.Hq + h) * a.T + t;
-        if (a.lse_S) a.lse_S[li] = (mS + __log2f(lS)) * ln2;
-        if (a.lse_T) a.lse_T[li] = ((x_started ? mX : mS) + __log2f(lT)) * ln2;
+      const float inv_l = 1.f / l;
+      const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
+      tmem_store_row<HD>(o_addr, inv_l, a.o_T + orow * HD, row_ok);
+      if (row_ok && a.lse_T) a.lse_T[li] = lse;
+      if (vis.vX == vis.nv) {  // no teacher-only keys: o_T == o_S
+        tmem_store_row<HD>(o_addr, inv_l, a.o_S + orow * HD, row_ok);
+        if (row_ok && a.lse_S) a.lse_S[li] = lse;
       }
     }
   }

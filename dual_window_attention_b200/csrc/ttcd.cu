@@ -282,11 +282,12 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   a.w_T = w_T;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_qt = (T + ATT_BM - 1) / ATT_BM;
+  a.pairs = (Hq / Hkv + 1) / 2;
   auto kern = dual_window_attn_kernel<HD>;
   constexpr int smem = AttnCfg<HD>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
-  const long long grid = static_cast<long long>(a.n_qt) * B * Hq;
+  const long long grid = static_cast<long long>(a.n_qt) * B * Hkv * a.pairs;
   if (grid >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
   kern<<<static_cast<unsigned>(grid), ATT_THREADS, smem, c.s>>>(mq, mk, mv, a, c.st);
   TTCD_CHECK_LAUNCH();
