@@ -36,9 +36,10 @@
 
 namespace ttcd {
 
+template <class OutT>
 struct AttnArgs {
-  __nv_bfloat16* o_T;  // [B, T, Hq, HD]
-  __nv_bfloat16* o_S;
+  OutT* o_T;  // [B, T, Hq, HD]
+  OutT* o_S;
   float* lse_T;  // [B, Hq, T], nullable
   float* lse_S;
   int B, T, Hq, Hkv;
@@ -167,25 +168,24 @@ __device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
-// Normalise this thread's O row by 1/l and store it (bf16) to dst.
-template <int HD>
-__device__ __forceinline__ void tmem_store_row(uint32_t taddr, float inv_l, __nv_bfloat16* dst,
-                                               bool ok) {
+// Normalise this thread's O row by 1/l and store it to dst.
+template <int HD, class OutT>
+__device__ __forceinline__ void tmem_store_row(uint32_t taddr, float inv_l, OutT* dst, bool ok) {
 #pragma unroll
   for (int c = 0; c < HD; c += 32) {
     float v[32];
     tmem_ld32f(taddr + c, v);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= inv_l;
-    if (ok) store_bf16x32(dst + c, v);
+    if (ok) store_x32(dst + c, v);
   }
 }
 
-template <int HD>
+template <int HD, class OutT>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     dual_window_attn_kernel(const __grid_constant__ CUtensorMap mapQ,
                             const __grid_constant__ CUtensorMap mapK,
-                            const __grid_constant__ CUtensorMap mapV, const AttnArgs a,
+                            const __grid_constant__ CUtensorMap mapV, const AttnArgs<OutT> a,
                             const DevStatus st) {
   using Cfg = AttnCfg<HD>;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(ATT_BM, ATT_BN, false, false);
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tc_fence_after();
       if (v == vis.vX) {
         // end of the student phase: O / l is o_S (PV of every earlier tile has landed)
-        tmem_store_row<HD>(o_addr, 1.f / l, a.o_S + orow * HD, row_ok);
+        tmem_store_row<HD, OutT>(o_addr, 1.f / l, a.o_S + orow * HD, row_ok);
         if (row_ok && a.lse_S) a.lse_S[li] = (m_ref + __log2f(l)) * 0.6931471805599453f;
       }
       float s[128];
@@ -447,10 +447,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
-      tmem_store_row<HD>(o_addr, inv_l, a.o_T + orow * HD, row_ok);
+      tmem_store_row<HD, OutT>(o_addr, inv_l, a.o_T + orow * HD, row_ok);
       if (row_ok && a.lse_T) a.lse_T[li] = lse;
       if (vis.vX == vis.nv) {  // no teacher-only keys: o_T == o_S
-        tmem_store_row<HD>(o_addr, inv_l, a.o_S + orow * HD, row_ok);
+        tmem_store_row<HD, OutT>(o_addr, inv_l, a.o_S + orow * HD, row_ok);
         if (row_ok && a.lse_S) a.lse_S[li] = lse;
       }
     }

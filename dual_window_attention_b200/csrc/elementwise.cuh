@@ -8,6 +8,38 @@ namespace ttcd {
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
+__device__ __forceinline__ void store8(__nv_bfloat16* dst, const float (&v)[8]) {
+  uint4 w;
+  w.x = pack_bf16x2(v[0], v[1]);
+  w.y = pack_bf16x2(v[2], v[3]);
+  w.z = pack_bf16x2(v[4], v[5]);
+  w.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(dst) = w;
+}
+__device__ __forceinline__ void store8(float* dst, const float (&v)[8]) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, float a, float b, float c, float d) {
+  uint2 w;
+  w.x = pack_bf16x2(a, b);
+  w.y = pack_bf16x2(c, d);
+  *reinterpret_cast<uint2*>(dst) = w;
+}
+__device__ __forceinline__ void store4(float* dst, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+}
+template <class E>
+__device__ __forceinline__ E from_f32(float v);
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) {
+  return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -18,9 +50,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 // RMSNorm as the block's pre-norm (papernotes.org review, 方法详解: the shared
 // backbone; the pages leave the skeleton unstated, a pre-norm decoder layer is
 // the plain reading).
-template <class InT, class GT>
+template <class InT, class GT, class OutT>
 __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict__ g,
-                               __nv_bfloat16* __restrict__ out, long long rows, int d, float eps) {
+                               OutT* __restrict__ out, long long rows, int d, float eps) {
   const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -35,17 +67,12 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   }
   ss = warp_sum(ss);
   const float rs = rsqrtf(ss / d + eps);
-  __nv_bfloat16* y = out + row * d;
+  OutT* y = out + row * d;
   for (int c = lane * 8; c < d; c += 256) {
-    uint4 w;
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = to_f32(x[c + i]) * rs * to_f32(g[c + i]);
-    w.x = pack_bf16x2(v[0], v[1]);
-    w.y = pack_bf16x2(v[2], v[3]);
-    w.z = pack_bf16x2(v[4], v[5]);
-    w.w = pack_bf16x2(v[6], v[7]);
-    *reinterpret_cast<uint4*>(y + c) = w;
+    store8(y + c, v);
   }
 }
 
@@ -65,113 +92,113 @@ __global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double
 // Fused short causal convolutions, residual difference and student keys.
 // papernotes.org review, 关键设计 3: Zbar_P = conv_P(Z_P) (depthwise, causal),
 // D = Zbar_T - Zbar_S, K = l2-norm(Zbar_S).  The per-row norm needs the whole
-// d_ff row, so this kernel writes Zbar_S unnormalised (transposed, Kt) and adds
-// its squares into ssq_part[channel block][p]; the scale beta_t / ||.|| is applied to the value
-// residual instead (Delta W = sum beta r k^T is linear in that scale).
+// d_ff row, so this kernel writes Zbar_S unnormalised (transposed, Kt) and the
+// squares of its 64-channel slice into ssq_part[channel block][p]; the scale
+// beta_t / ||.|| is applied to the value residual instead (Delta W = sum beta r
+// k^T is linear in that scale).
 //
 // Z     fp32 [2, BT, f]: teacher rows then student rows
 // taps  [f, k] (tap m multiplies t - m), TapT = bf16 or fp32
 // D     bf16 [P, f]      Kt bf16 [f, P]     Zs16 bf16 [BT, f]    ssq_part fp32 [f/64, P]
 // Padded index p = (b*Nc + i)*Cp + j holds token t = i*C + j when j < C and t < T;
 // other p get D = 0 and Kt = 0.
-// Block: 64 padded positions x 64 channels, 256 threads (thread = one position,
-// 16 channels).
-constexpr int CONV_TP = 64, CONV_TC = 64;
-template <class TapT>
+// Block: 64 padded positions (inside one chunk, since Cp is a multiple of 64) x
+// 64 channels, 256 threads.  The Z rows t0-(k-1) .. t0+63 of both paths are
+// staged in shared memory with coalesced 16-byte loads (16 threads per 256-byte
+// row); thread (cq, tr) then owns channels 4cq..4cq+3 of positions tr + 16 i.
+constexpr int CONV_TP = 64, CONV_TC = 64, CONV_MAXK = 8;
+template <class TapT, class E>
 __global__ void __launch_bounds__(256)
     conv_residual_key_kernel(const float* __restrict__ Z, const TapT* __restrict__ tapT,
-                             const TapT* __restrict__ tapS, __nv_bfloat16* __restrict__ D,
-                             __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ Zs16,
+                             const TapT* __restrict__ tapS, E* __restrict__ D,
+                             E* __restrict__ Kt, E* __restrict__ Zs16,
                              float* __restrict__ ssq_part, int T, int f, int k, int C, int Cp,
                              int Nc, long long BT, long long P) {
-  __shared__ __nv_bfloat16 tileK[CONV_TC][CONV_TP + 8];
-  __shared__ float sq_part[4][CONV_TP];
+  constexpr int ROWS = CONV_TP + CONV_MAXK - 1;
+  __shared__ __align__(16) float zT[ROWS][CONV_TC];
+  __shared__ __align__(16) float zS[ROWS][CONV_TC];
+  __shared__ float taps[2][CONV_MAXK][CONV_TC];
+  // the key tile reuses zT's storage once the convolutions are done
+  typedef E KRow[CONV_TP + 16 / sizeof(E)];
+  KRow* tileK = reinterpret_cast<KRow*>(&zT[0][0]);
+  static_assert(sizeof(zT) >= sizeof(KRow) * CONV_TC, "key tile must fit in zT");
   const long long p0 = static_cast<long long>(blockIdx.x) * CONV_TP;
   const int c0 = blockIdx.y * CONV_TC;
-  const int tp = threadIdx.x & 63;   // position within tile
-  const int cg = threadIdx.x >> 6;   // 16-channel group
-  const long long p = p0 + tp;
   const long long seq_len_p = static_cast<long long>(Nc) * Cp;
-  const int b = static_cast<int>(p / seq_len_p);
-  const long long rem = p % seq_len_p;
-  const int i = static_cast<int>(rem / Cp), j = static_cast<int>(rem % Cp);
-  const int t = i * C + j;
-  const bool valid = p < P && j < C && t < T;
-  const int cbase = c0 + cg * 16;
-  float zbS[16];
-  float sq = 0.f;
-  if (valid) {
-    float zbT[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) { zbT[c] = 0.f; zbS[c] = 0.f; }
-    const long long rowT = static_cast<long long>(b) * T + t;
-    for (int m = 0; m < k; ++m) {
-      if (t - m < 0) break;
-      const float* zt = Z + (rowT - m) * f + cbase;
-      const float* zs = Z + (BT + rowT - m) * f + cbase;
-#pragma unroll
-      for (int c4 = 0; c4 < 16; c4 += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(zt + c4);
-        const float4 s = *reinterpret_cast<const float4*>(zs + c4);
-        const float wa[4] = {a.x, a.y, a.z, a.w};
-        const float ws[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = cbase + c4 + e;
-          zbT[c4 + e] += to_f32(tapT[c * k + m]) * wa[e];
-          zbS[c4 + e] += to_f32(tapS[c * k + m]) * ws[e];
-        }
-      }
-      if (m == 0) {
-        uint4 w0, w1;
-        w0.x = pack_bf16x2(zs[0], zs[1]);   w0.y = pack_bf16x2(zs[2], zs[3]);
-        w0.z = pack_bf16x2(zs[4], zs[5]);   w0.w = pack_bf16x2(zs[6], zs[7]);
-        w1.x = pack_bf16x2(zs[8], zs[9]);   w1.y = pack_bf16x2(zs[10], zs[11]);
-        w1.z = pack_bf16x2(zs[12], zs[13]); w1.w = pack_bf16x2(zs[14], zs[15]);
-        uint4* dz = reinterpret_cast<uint4*>(Zs16 + rowT * f + cbase);
-        dz[0] = w0;
-        dz[1] = w1;
-      }
-    }
-    uint4 w0, w1;
-    float dd[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      dd[c] = zbT[c] - zbS[c];
-      sq += zbS[c] * zbS[c];
-    }
-    w0.x = pack_bf16x2(dd[0], dd[1]);   w0.y = pack_bf16x2(dd[2], dd[3]);
-    w0.z = pack_bf16x2(dd[4], dd[5]);   w0.w = pack_bf16x2(dd[6], dd[7]);
-    w1.x = pack_bf16x2(dd[8], dd[9]);   w1.y = pack_bf16x2(dd[10], dd[11]);
-    w1.z = pack_bf16x2(dd[12], dd[13]); w1.w = pack_bf16x2(dd[14], dd[15]);
-    uint4* dD = reinterpret_cast<uint4*>(D + p * f + cbase);
-    dD[0] = w0;
-    dD[1] = w1;
-  } else {
-#pragma unroll
-    for (int c = 0; c < 16; ++c) zbS[c] = 0.f;
-    if (p < P) {
-      uint4* dD = reinterpret_cast<uint4*>(D + p * f + cbase);
-      dD[0] = make_uint4(0, 0, 0, 0);
-      dD[1] = make_uint4(0, 0, 0, 0);
-    }
+  const int b = static_cast<int>(p0 / seq_len_p);
+  const long long rem0 = p0 % seq_len_p;
+  const int ci = static_cast<int>(rem0 / Cp), j0 = static_cast<int>(rem0 % Cp);
+  const int t0 = ci * C + j0;               // token of position p0 (if valid)
+  const int n_valid = max(0, min(CONV_TP, min(C - j0, T - t0)));
+  const long long rowT0 = static_cast<long long>(b) * T;
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < 2 * CONV_MAXK * CONV_TC; i += 256) {
+    const int path = i / (CONV_MAXK * CONV_TC), m = (i / CONV_TC) % CONV_MAXK, c = i % CONV_TC;
+    const TapT* tp = path ? tapS : tapT;
+    taps[path][m][c] = m < k ? to_f32(tp[static_cast<long long>(c0 + c) * k + m]) : 0.f;
   }
-#pragma unroll
-  for (int c = 0; c < 16; ++c) tileK[cg * 16 + c][tp] = __float2bfloat16_rn(zbS[c]);
-  sq_part[cg][tp] = sq;
-  __syncthreads();
-  // Deterministic per-(channel block, position) partial sums; summed in order later.
-  if (cg == 0 && p < P)
-    ssq_part[static_cast<long long>(blockIdx.y) * P + p] =
-        ((sq_part[0][tp] + sq_part[1][tp]) + sq_part[2][tp]) + sq_part[3][tp];
-  // Transposed store: each warp writes rows of Kt (64 positions = 128 bytes).
-  for (int r = threadIdx.x >> 3; r < CONV_TC; r += 32) {
-    const int seg = threadIdx.x & 7;  // 8 x 16 bytes per row
-    const long long pp = p0 + seg * 8;
-    if (pp < P) {
-      const uint4 w = *reinterpret_cast<const uint4*>(&tileK[r][seg * 8]);
-      *reinterpret_cast<uint4*>(Kt + static_cast<long long>(c0 + r) * P + pp) = w;
+  // Stage rows t0-(k-1) .. t0+n_valid-1 (missing rows are zero).
+  const int halo = k - 1;
+  for (int i = tid; i < (n_valid + halo) * 16; i += 256) {
+    const int rr = i >> 4, cq = i & 15;
+    const int t = t0 - halo + rr;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), s = a;
+    if (t >= 0) {
+      a = *reinterpret_cast<const float4*>(Z + (rowT0 + t) * f + c0 + 4 * cq);
+      s = *reinterpret_cast<const float4*>(Z + (BT + rowT0 + t) * f + c0 + 4 * cq);
     }
+    *reinterpret_cast<float4*>(&zT[CONV_MAXK - 1 - halo + rr][4 * cq]) = a;
+    *reinterpret_cast<float4*>(&zS[CONV_MAXK - 1 - halo + rr][4 * cq]) = s;
+  }
+  __syncthreads();
+
+  const int cq = tid & 15, tr = tid >> 4;
+  float keys[CONV_TP / 16][4];
+#pragma unroll
+  for (int it = 0; it < CONV_TP / 16; ++it) {
+    const int jj = tr + 16 * it;  // position within the tile
+    const long long p = p0 + jj;
+    const bool valid = jj < n_valid;
+    float zbT[4] = {0.f, 0.f, 0.f, 0.f}, zbS[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) {
+      for (int m = 0; m < k; ++m) {
+        const int row = CONV_MAXK - 1 + jj - m;
+        const float4 a = *reinterpret_cast<const float4*>(&zT[row][4 * cq]);
+        const float4 s = *reinterpret_cast<const float4*>(&zS[row][4 * cq]);
+        zbT[0] += taps[0][m][4 * cq + 0] * a.x; zbS[0] += taps[1][m][4 * cq + 0] * s.x;
+        zbT[1] += taps[0][m][4 * cq + 1] * a.y; zbS[1] += taps[1][m][4 * cq + 1] * s.y;
+        zbT[2] += taps[0][m][4 * cq + 2] * a.z; zbS[2] += taps[1][m][4 * cq + 2] * s.z;
+        zbT[3] += taps[0][m][4 * cq + 3] * a.w; zbS[3] += taps[1][m][4 * cq + 3] * s.w;
+      }
+    }
+    // D (zeros at padding) and the bf16 copy of Z_S, 8 bytes per thread, 128 bytes per row.
+    store4(D + p * f + c0 + 4 * cq, zbT[0] - zbS[0], zbT[1] - zbS[1], zbT[2] - zbS[2],
+           zbT[3] - zbS[3]);
+    if (valid && Zs16) {
+      const float4 s = *reinterpret_cast<const float4*>(&zS[CONV_MAXK - 1 + jj][4 * cq]);
+      store4(Zs16 + (rowT0 + t0 + jj) * f + c0 + 4 * cq, s.x, s.y, s.z, s.w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) keys[it][e] = zbS[e];
+    // squares of this 64-channel slice, reduced over the 16 threads of the row
+    float sq = zbS[0] * zbS[0] + zbS[1] * zbS[1] + zbS[2] * zbS[2] + zbS[3] * zbS[3];
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (cq == 0) ssq_part[static_cast<long long>(blockIdx.y) * P + p] = sq;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < CONV_TP / 16; ++it)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tileK[4 * cq + e][tr + 16 * it] = from_f32<E>(keys[it][e]);
+  __syncthreads();
+  // Transposed store of the keys: each row of Kt gets 64 positions in 16-byte segments.
+  constexpr int SEG_E = 16 / sizeof(E), SEGS = CONV_TP / SEG_E;
+  for (int i = tid; i < CONV_TC * SEGS; i += 256) {
+    const int r = i / SEGS, seg = i % SEGS;
+    const uint4 w = *reinterpret_cast<const uint4*>(&tileK[r][seg * SEG_E]);
+    *reinterpret_cast<uint4*>(Kt + static_cast<long long>(c0 + r) * P + p0 + seg * SEG_E) = w;
   }
 }
 
@@ -201,9 +228,9 @@ __global__ void cast_to_bf16_kernel(const InT* __restrict__ in, __nv_bfloat16* _
 }
 
 // out[c, r] = in[r, c] for an [R, Cn] matrix.
-template <class InT>
-__global__ void transpose_to_bf16_kernel(const InT* __restrict__ in, __nv_bfloat16* __restrict__ out,
-                                         int R, int Cn) {
+template <class InT, class OutT>
+__global__ void transpose_kernel(const InT* __restrict__ in, OutT* __restrict__ out, int R,
+                                 int Cn) {
   __shared__ float tile[32][33];
   const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
   for (int y = threadIdx.y; y < 32; y += blockDim.y) {
@@ -213,7 +240,7 @@ __global__ void transpose_to_bf16_kernel(const InT* __restrict__ in, __nv_bfloat
   __syncthreads();
   for (int y = threadIdx.y; y < 32; y += blockDim.y) {
     const int c = bx + y, r = by + threadIdx.x;
-    if (r < R && c < Cn) out[static_cast<long long>(c) * R + r] = __float2bfloat16_rn(tile[threadIdx.x][y]);
+    if (r < R && c < Cn) out[static_cast<long long>(c) * R + r] = from_f32<OutT>(tile[threadIdx.x][y]);
   }
 }
 

@@ -99,7 +99,7 @@ __device__ __forceinline__ void load_x32(const float* src, float (&v)[32]) {
   }
 }
 
-template <int BN, int STAGES, bool DUAL_B, class Epi>
+template <class E, int BN, int STAGES, bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
@@ -110,7 +110,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
-  constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN, false, false);
+  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, false);
+  constexpr int BK = ElemTraits<E>::BK;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = geo.total();
-  const int nk = (geo.K + GEMM_BK - 1) / GEMM_BK;
+  const int nk = (geo.K + BK - 1) / BK;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -168,13 +169,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(sa, &mapA, &full[s], kb * GEMM_BK, c.row0);
+          tma_load_2d(sa, &mapA, &full[s], kb * BK, c.row0);
           if (DUAL_B) {
-            tma_load_2d(sb, &mapB0, &full[s], kb * GEMM_BK, c.b_row0 + c.tn * (BN / 2));
-            tma_load_2d(sb + (BN / 2) * 128, &mapB1, &full[s], kb * GEMM_BK,
+            tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * (BN / 2));
+            tma_load_2d(sb + (BN / 2) * 128, &mapB1, &full[s], kb * BK,
                         c.b_row0 + c.tn * (BN / 2));
           } else {
-            tma_load_2d(sb, &mapB0, &full[s], kb * GEMM_BK, c.b_row0 + c.tn * BN);
+            tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * BN);
           }
         }
       }
@@ -202,10 +203,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k) {
+          for (int k = 0; k < 4; ++k) {  // 4 MMAs of 32 bytes of K per 128-byte row
             const uint64_t da = sdesc_sw128(sa + k * 32, 16, 1024);
             const uint64_t db = sdesc_sw128(sb + k * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
+            mma_ss<E>(d_tmem, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -249,9 +250,10 @@ constexpr int gemm_smem_bytes() {
 
 // ------------------------------------------------------------------ epilogues
 
-// C[row, col] = bf16(acc * col_scale[col]) (col_scale nullable), columns < N.
-struct EpiStoreBF16 {
-  __nv_bfloat16* out;
+// C[row, col] = OutT(acc * col_scale[col]) (col_scale nullable), columns < N.
+template <class OutT>
+struct EpiStore {
+  OutT* out;
   long long ldo;
   int N;
   const float* col_scale;
@@ -269,10 +271,11 @@ struct EpiStoreBF16 {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] *= __ldg(col_scale + col + i);
       }
-      if (ok) store_bf16x32(out + row * ldo + col, v);
+      if (ok) store_x32(out + row * ldo + col, v);
     }
   }
 };
+using EpiStoreBF16 = EpiStore<__nv_bfloat16>;
 
 // out[row, col] = resid[row % resid_rows, col] + acc;  columns < N.
 template <class OutT, class ResT>

@@ -18,24 +18,26 @@
 
 namespace ttcd {
 
+template <class E>
 struct ScanArgs {
   int d, f, Nc, Cp;
-  const __nv_bfloat16* w_down;  // [d, f]
-  const float* state_in;        // [B, d, f] nullable
-  float* state_out;             // [B, d, f] nullable
-  __nv_bfloat16* w_all;         // [B*Nc, d, f]
+  const E* w_down;        // [d, f]
+  const float* state_in;  // [B, d, f] nullable
+  float* state_out;       // [B, d, f] nullable
+  E* w_all;               // [B*Nc, d, f]
   int tiles_m, tiles_n;
 };
 
-template <int STAGES>
+template <class E, int STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fastweight_scan_kernel(const __grid_constant__ CUtensorMap mapR,
-                           const __grid_constant__ CUtensorMap mapK, const ScanArgs a,
+                           const __grid_constant__ CUtensorMap mapK, const ScanArgs<E> a,
                            const DevStatus st) {
   constexpr int BN = 128;
   constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN, false, false);
+  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, false);
+  constexpr int BK = ElemTraits<E>::BK;
   constexpr uint32_t COL_STATE = 256;
 
   extern __shared__ uint8_t smem_raw[];
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int tm = (blockIdx.x / a.tiles_n) % a.tiles_m;
   const int b = blockIdx.x / (a.tiles_n * a.tiles_m);
   const int m0 = tm * GEMM_BM, n0 = tn * BN;
-  const int kpc = a.Cp / GEMM_BK;  // k-blocks per chunk
+  const int kpc = a.Cp / BK;  // k-blocks per chunk
   const long long P = static_cast<long long>(gridDim.x / (a.tiles_n * a.tiles_m)) * a.Nc * a.Cp;
   (void)P;
 
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, st, abort)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
-          const int x = (b * a.Nc + i) * a.Cp + kb * GEMM_BK;
+          const int x = (b * a.Nc + i) * a.Cp + kb * BK;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           tma_load_2d(sa, &mapR, &full[s], x, m0);
           tma_load_2d(sa + A_BYTES, &mapK, &full[s], x, n0);
@@ -109,9 +111,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k)
-            mma_bf16_ss(tmem + ab * BN, sdesc_sw128(sa + k * 32, 16, 1024),
-                        sdesc_sw128(sb + k * 32, 16, 1024), IDESC, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)
+            mma_ss<E>(tmem + ab * BN, sdesc_sw128(sa + k * 32, 16, 1024),
+                      sdesc_sw128(sb + k * 32, 16, 1024), IDESC, (kb | k) != 0 ? 1u : 0u);
           mma_commit(&empty[s]);
         }
         if (!ok) break;
@@ -148,8 +150,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         load_x32(a.w_down + static_cast<long long>(row) * a.f + col, w);
 #pragma unroll
         for (int e = 0; e < 32; ++e) w[e] += s[e];
-        store_bf16x32(a.w_all + (static_cast<long long>(b) * a.Nc) * dfs +
-                          static_cast<long long>(row) * a.f + col, w);
+        store_x32(a.w_all + (static_cast<long long>(b) * a.Nc) * dfs +
+                      static_cast<long long>(row) * a.f + col, w);
       }
     }
     tmem_st_wait();
@@ -178,8 +180,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             load_x32(a.w_down + static_cast<long long>(row) * a.f + col, w);
 #pragma unroll
             for (int e = 0; e < 32; ++e) w[e] += s[e];
-            store_bf16x32(a.w_all + (static_cast<long long>(b) * a.Nc + i + 1) * dfs +
-                              static_cast<long long>(row) * a.f + col, w);
+            store_x32(a.w_all + (static_cast<long long>(b) * a.Nc + i + 1) * dfs +
+                          static_cast<long long>(row) * a.f + col, w);
           } else if (a.state_out) {
             store_f32x32(a.state_out + b * dfs + static_cast<long long>(row) * a.f + col, s);
           }

@@ -80,22 +80,27 @@ ttcd_status make_ctx(void* stream, Ctx& c) {
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 2-D bf16 tensor map: `outer` rows of `inner` elements, row pitch in bytes,
-// box of box_inner x box_outer elements, 128-byte swizzle.
+// 2-D tensor map of element type E (bf16 or fp32): `outer` rows of `inner`
+// elements, row pitch in bytes, box of box_inner x box_outer elements,
+// 128-byte swizzle.
+template <class E>
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt =
+      sizeof(E) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+// Row-major [rows, cols] operand; the box spans one 128-byte swizzle row of K.
+template <class E>
 bool map_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_map(m, ptr, cols, rows, cols * 2, 64, box_rows);
+  return make_map<E>(m, ptr, cols, rows, cols * sizeof(E), ElemTraits<E>::BK, box_rows);
 }
 
 std::atomic<unsigned long long> g_launches{0};
@@ -115,12 +120,12 @@ void stage_mark(cudaStream_t s, int k) {
     g_launches.fetch_add(1, std::memory_order_relaxed);          \
   } while (0)
 
-template <int BN, int STAGES, bool DUAL, class Epi>
+template <class E, int BN, int STAGES, bool DUAL, class Epi>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
                         const CUtensorMap& B1, const GemmGeom& geo, const Epi& epi) {
   const int total = geo.total();
   if (total <= 0) return TTCD_OK;
-  auto kern = gemm_tc_kernel<BN, STAGES, DUAL, Epi>;
+  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi>;
   constexpr int smem = gemm_smem_bytes<BN, STAGES>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -172,11 +177,10 @@ struct Layout {
 };
 enum Buf {
   B_XN, B_Q, B_K, B_V, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KT, B_SSQ, B_KSCALE, B_RT,
-  B_WALL, B_M, B_WPROJT, B_WQKV16, B_WO16, B_WGATE16, B_WUP16, B_WDOWN16, B_COUNT
+  B_WALL, B_M, B_WPROJT, B_COUNT
 };
 const char* kBufNames[B_COUNT] = {"xn", "q", "k", "v", "o", "h", "rope", "u", "Z", "Zs16", "D",
-                                  "Kt", "ssq", "kscale", "Rt", "Wall", "M", "WprojT", "wqkv16",
-                                  "wo16", "wgate16", "wup16", "wdown16"};
+                                  "Kt", "ssq", "kscale", "Rt", "Wall", "M", "WprojT"};
 
 struct Dims {
   long long BT, P;
@@ -197,39 +201,32 @@ Dims dims_of(const ttcd_block_params* p) {
   return m;
 }
 
+// Operand buffers hold bf16 for TTCD_BF16 and fp32 (tf32 tensor-core operands)
+// for TTCD_F32; q, k, v stay bf16 (the attention kernel takes bf16).
 Layout make_layout(const ttcd_block_params* p, bool block) {
   const Dims m = dims_of(p);
   size_t sz[B_COUNT] = {0};
-  const bool f32 = p->dtype == TTCD_F32;
+  const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
   if (block) {
-    sz[B_XN] = m.BT * m.d * 2;
+    sz[B_XN] = m.BT * m.d * e;
     sz[B_Q] = m.BT * m.Hq * m.hd * 2;
     sz[B_K] = m.BT * m.Hkv * m.hd * 2;
     sz[B_V] = m.BT * m.Hkv * m.hd * 2;
-    sz[B_O] = 2 * m.BT * m.Hq * m.hd * 2;
+    sz[B_O] = 2 * m.BT * m.Hq * m.hd * e;
     sz[B_H] = 2 * m.BT * m.d * 4;
     sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 8;
-    if (f32) {
-      sz[B_WQKV16] = static_cast<size_t>(m.dqkv) * m.d * 2;
-      sz[B_WO16] = static_cast<size_t>(m.d) * m.Hq * m.hd * 2;
-    }
   }
-  sz[B_U] = 2 * m.BT * m.d * 2;
+  sz[B_U] = 2 * m.BT * m.d * e;
   sz[B_Z] = 2 * m.BT * m.f * 4;
-  sz[B_ZS16] = m.BT * m.f * 2;
-  sz[B_D] = m.P * m.f * 2;
-  sz[B_KT] = m.P * m.f * 2;
+  sz[B_ZS16] = e == 2 ? m.BT * m.f * 2 : 0;  // fp32 mode reads Z_S directly
+  sz[B_D] = m.P * m.f * e;
+  sz[B_KT] = m.P * m.f * e;
   sz[B_SSQ] = m.P * 4 * (m.f / 64);
   sz[B_KSCALE] = m.P * 4;
-  sz[B_RT] = m.P * m.d * 2;
-  sz[B_WALL] = static_cast<size_t>(p->B) * m.Nc * m.d * m.f * 2;
-  sz[B_M] = static_cast<size_t>(m.d) * m.f * 2;
-  sz[B_WPROJT] = static_cast<size_t>(m.f) * m.f * 2;
-  if (f32) {
-    sz[B_WGATE16] = static_cast<size_t>(m.f) * m.d * 2;
-    sz[B_WUP16] = static_cast<size_t>(m.f) * m.d * 2;
-    sz[B_WDOWN16] = static_cast<size_t>(m.d) * m.f * 2;
-  }
+  sz[B_RT] = m.P * m.d * e;
+  sz[B_WALL] = static_cast<size_t>(p->B) * m.Nc * m.d * m.f * e;
+  sz[B_M] = static_cast<size_t>(m.d) * m.f * e;
+  sz[B_WPROJT] = static_cast<size_t>(m.f) * m.f * e;
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_COUNT; ++i) {
@@ -245,13 +242,6 @@ T* at(void* ws, const Layout& L, Buf b) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + L.off[b]);
 }
 
-template <class InT>
-ttcd_status cast_bf16(const Ctx& c, const void* in, __nv_bfloat16* out, long long n) {
-  cast_to_bf16_kernel<InT><<<cdiv(n, 256), 256, 0, c.s>>>(static_cast<const InT*>(in), out, n);
-  TTCD_CHECK_LAUNCH();
-  return TTCD_OK;
-}
-
 #define TTCD_TRY(x)                    \
   do {                                 \
     ttcd_status _s = (x);              \
@@ -259,19 +249,20 @@ ttcd_status cast_bf16(const Ctx& c, const void* in, __nv_bfloat16* out, long lon
   } while (0)
 
 // ------------------------------------------------------------------ attention
-template <int HD>
-ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* v, void* o_T,
-                        void* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv,
+template <int HD, class OutT>
+ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
+                        OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv,
                         int w_S, int w_T, float scale) {
   CUtensorMap mq, mk, mv;
   const long long BT = static_cast<long long>(B) * T;
-  if (!make_map(&mq, q, static_cast<uint64_t>(Hq) * HD, BT, static_cast<uint64_t>(Hq) * HD * 2, 64, 128) ||
-      !make_map(&mk, k, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128) ||
-      !make_map(&mv, v, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128))
+  using bf = __nv_bfloat16;
+  if (!make_map<bf>(&mq, q, static_cast<uint64_t>(Hq) * HD, BT, static_cast<uint64_t>(Hq) * HD * 2, 64, 128) ||
+      !make_map<bf>(&mk, k, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128) ||
+      !make_map<bf>(&mv, v, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128))
     return TTCD_ERR_CUDA;
-  AttnArgs a;
-  a.o_T = static_cast<__nv_bfloat16*>(o_T);
-  a.o_S = static_cast<__nv_bfloat16*>(o_S);
+  AttnArgs<OutT> a;
+  a.o_T = o_T;
+  a.o_S = o_S;
   a.lse_T = lse_T;
   a.lse_S = lse_S;
   a.B = B;
@@ -283,7 +274,7 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_qt = (T + ATT_BM - 1) / ATT_BM;
   a.pairs = (Hq / Hkv + 1) / 2;
-  auto kern = dual_window_attn_kernel<HD>;
+  auto kern = dual_window_attn_kernel<HD, OutT>;
   constexpr int smem = AttnCfg<HD>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -294,8 +285,9 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   return TTCD_OK;
 }
 
-ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, void* o_T,
-                     void* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv, int hd,
+template <class OutT>
+ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
+                     OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv, int hd,
                      int w_S, int w_T, float scale) {
   switch (hd) {
     case 32: return launch_attn<32>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale);
@@ -306,42 +298,41 @@ ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, 
 }
 
 // ------------------------------------------------------------------ fast-weight MLP body
-// u (bf16 [2BT, d], teacher rows first) is already in the workspace.
-template <class OutT, class ResT, class TapT>
+// u (operand type E, [2BT, d], teacher rows first) is already in the workspace.
+template <class E, class OutT, class ResT>
 ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
-                         const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
-                         const __nv_bfloat16* w_down, const void* w_proj, bool proj_f32,
-                         const TapT* conv_T, const TapT* conv_S, const float* beta,
+                         const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
+                         const E* conv_T, const E* conv_S, const float* beta,
                          const float* state_in, float* state_out, const ResT* h_S, OutT* y,
                          int mark) {
   const Dims m = dims_of(p);
-  stage_mark(c.s, mark);
-  __nv_bfloat16* u = at<__nv_bfloat16>(ws, L, B_U);
+  E* u = at<E>(ws, L, B_U);
   float* Z = at<float>(ws, L, B_Z);
-  __nv_bfloat16* Zs16 = at<__nv_bfloat16>(ws, L, B_ZS16);
-  __nv_bfloat16* D = at<__nv_bfloat16>(ws, L, B_D);
-  __nv_bfloat16* Kt = at<__nv_bfloat16>(ws, L, B_KT);
+  E* Zs = sizeof(E) == 2 ? at<E>(ws, L, B_ZS16) : nullptr;
+  E* D = at<E>(ws, L, B_D);
+  E* Kt = at<E>(ws, L, B_KT);
   float* ssq = at<float>(ws, L, B_SSQ);
   float* kscale = at<float>(ws, L, B_KSCALE);
-  __nv_bfloat16* Rt = at<__nv_bfloat16>(ws, L, B_RT);
-  __nv_bfloat16* Wall = at<__nv_bfloat16>(ws, L, B_WALL);
-  __nv_bfloat16* M = at<__nv_bfloat16>(ws, L, B_M);
-  __nv_bfloat16* WprojT = at<__nv_bfloat16>(ws, L, B_WPROJT);
+  E* Rt = at<E>(ws, L, B_RT);
+  E* Wall = at<E>(ws, L, B_WALL);
+  E* M = at<E>(ws, L, B_M);
+  E* WprojT = at<E>(ws, L, B_WPROJT);
+  stage_mark(c.s, mark);
 
   // Z_P = silu(u_P W_gate^T) * (u_P W_up^T), both paths stacked (slow weights).
   {
     CUtensorMap mA, mB0, mB1;
-    if (!map_rows(&mA, u, 2 * m.BT, m.d, 128) || !map_rows(&mB0, w_gate, m.f, m.d, 64) ||
-        !map_rows(&mB1, w_up, m.f, m.d, 64))
+    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 64) ||
+        !map_rows<E>(&mB1, w_up, m.f, m.d, 64))
       return TTCD_ERR_CUDA;
     EpiSwiGLU e{Z, m.f, m.f};
-    TTCD_TRY((launch_gemm<128, 6, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, m.f / 64, m.d), e)));
+    TTCD_TRY((launch_gemm<E, 128, 6, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, m.f / 64, m.d), e)));
   }
   stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
   {
     dim3 grid(static_cast<unsigned>(m.P / CONV_TP), m.f / CONV_TC);
-    conv_residual_key_kernel<TapT><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kt, Zs16, ssq,
+    conv_residual_key_kernel<E, E><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kt, Zs, ssq,
                                                           p->T, m.f, p->conv_k, p->chunk, m.Cp,
                                                           m.Nc, m.BT, m.P);
     TTCD_CHECK_LAUNCH();
@@ -353,33 +344,31 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   // M = W_down W_proj (associativity of W_down (W_proj d_t)).
   {
     dim3 tb(32, 8), tg(cdiv(m.f, 32), cdiv(m.f, 32));
-    if (proj_f32)
-      transpose_to_bf16_kernel<float><<<tg, tb, 0, c.s>>>(static_cast<const float*>(w_proj), WprojT, m.f, m.f);
-    else
-      transpose_to_bf16_kernel<__nv_bfloat16><<<tg, tb, 0, c.s>>>(static_cast<const __nv_bfloat16*>(w_proj), WprojT, m.f, m.f);
+    transpose_kernel<E, E><<<tg, tb, 0, c.s>>>(w_proj, WprojT, m.f, m.f);
     TTCD_CHECK_LAUNCH();
     CUtensorMap mA, mB;
-    if (!map_rows(&mA, w_down, m.d, m.f, 128) || !map_rows(&mB, WprojT, m.f, m.f, 128))
+    if (!map_rows<E>(&mA, w_down, m.d, m.f, 128) || !map_rows<E>(&mB, WprojT, m.f, m.f, 128))
       return TTCD_ERR_CUDA;
-    EpiStoreBF16 e{M, m.f, m.f, nullptr};
-    TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, plain_geom(m.d, m.f / 128 + (m.f % 128 ? 1 : 0), m.f), e)));
+    EpiStore<E> e{M, m.f, m.f, nullptr};
+    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.f, 128), m.f), e)));
   }
   stage_mark(c.s, mark + 3);
   // R^T = M D^T, scaled per token by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
-    if (!map_rows(&mA, M, m.d, m.f, 128) || !map_rows(&mB, D, m.P, m.f, 256)) return TTCD_ERR_CUDA;
-    EpiStoreBF16 e{Rt, m.P, static_cast<int>(m.P), kscale};
-    TTCD_TRY((launch_gemm<256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.P, 256), m.f), e)));
+    if (!map_rows<E>(&mA, M, m.d, m.f, 128) || !map_rows<E>(&mB, D, m.P, m.f, 256))
+      return TTCD_ERR_CUDA;
+    EpiStore<E> e{Rt, m.P, static_cast<int>(m.P), kscale};
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.P, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 4);
-  // Delta W per chunk, fp32 exclusive prefix scan, W_i = bf16(W_down + S_i).
+  // Delta W per chunk, fp32 exclusive prefix scan, W_i = W_down + S_i.
   {
     CUtensorMap mR, mK;
-    if (!make_map(&mR, Rt, m.P, m.d, m.P * 2, 64, 128) ||
-        !make_map(&mK, Kt, m.P, m.f, m.P * 2, 64, 128))
+    if (!make_map<E>(&mR, Rt, m.P, m.d, m.P * sizeof(E), ElemTraits<E>::BK, 128) ||
+        !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), ElemTraits<E>::BK, 128))
       return TTCD_ERR_CUDA;
-    ScanArgs a;
+    ScanArgs<E> a;
     a.d = m.d;
     a.f = m.f;
     a.Nc = m.Nc;
@@ -392,7 +381,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     a.tiles_n = cdiv(m.f, 128);
     constexpr int STAGES = 6;
     constexpr int smem = gemm_smem_bytes<128, STAGES>();
-    auto kern = fastweight_scan_kernel<STAGES>;
+    auto kern = fastweight_scan_kernel<E, STAGES>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
     kern<<<p->B * a.tiles_m * a.tiles_n, GEMM_THREADS, smem, c.s>>>(mR, mK, a, c.st);
@@ -402,8 +391,9 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   // y = h_S + (W_down + S_i) Z_S, one GEMM per chunk with its own weight.
   {
     CUtensorMap mA, mB;
-    if (!map_rows(&mA, Zs16, m.BT, m.f, 128) ||
-        !map_rows(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 128))
+    const void* zs = Zs ? static_cast<const void*>(Zs) : static_cast<const void*>(Z + m.BT * m.f);
+    if (!map_rows<E>(&mA, zs, m.BT, m.f, 128) ||
+        !map_rows<E>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 128))
       return TTCD_ERR_CUDA;
     GemmGeom g;
     g.n_seq = p->B;
@@ -415,7 +405,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     g.tiles_n = cdiv(m.d, 128);
     g.b_group_rows = m.d;
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, e)));
+    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, e)));
   }
   stage_mark(c.s, mark + 6);
   return TTCD_OK;
@@ -514,7 +504,9 @@ ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, v
   Ctx c;
   TTCD_TRY(make_ctx(stream, c));
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(hd));
-  return run_attn(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, hd, w_S, w_T, sc);
+  return run_attn<__nv_bfloat16>(c, q, k, v, static_cast<__nv_bfloat16*>(o_T),
+                                 static_cast<__nv_bfloat16*>(o_S), lse_T, lse_S, B, T, Hq, Hkv,
+                                 hd, w_S, w_T, sc);
 }
 
 ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,
@@ -534,31 +526,103 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
   Ctx c;
   TTCD_TRY(make_ctx(stream, c));
   const Dims m = dims_of(p);
-  __nv_bfloat16* u = at<__nv_bfloat16>(workspace, L, B_U);
+  const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
+  uint8_t* u = at<uint8_t>(workspace, L, B_U);
+  if (cudaMemcpyAsync(u, u_T, m.BT * m.d * e, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
+      cudaMemcpyAsync(u + m.BT * m.d * e, u_S, m.BT * m.d * e, cudaMemcpyDeviceToDevice, c.s) !=
+          cudaSuccess)
+    return TTCD_ERR_CUDA;
   if (p->dtype == TTCD_BF16) {
-    if (cudaMemcpyAsync(u, u_T, m.BT * m.d * 2, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
-        cudaMemcpyAsync(u + m.BT * m.d, u_S, m.BT * m.d * 2, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
-      return TTCD_ERR_CUDA;
-    return run_mlp_core<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(
-        c, p, L, workspace, static_cast<const __nv_bfloat16*>(w->w_gate),
-        static_cast<const __nv_bfloat16*>(w->w_up), static_cast<const __nv_bfloat16*>(w->w_down),
-        w->w_proj, false, static_cast<const __nv_bfloat16*>(w->conv_T),
-        static_cast<const __nv_bfloat16*>(w->conv_S), beta, state_in, state_out,
-        static_cast<const __nv_bfloat16*>(h_S), static_cast<__nv_bfloat16*>(y), 0);
+    using bf = __nv_bfloat16;
+    return run_mlp_core<bf, bf, bf>(
+        c, p, L, workspace, static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up),
+        static_cast<const bf*>(w->w_down), static_cast<const bf*>(w->w_proj),
+        static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), beta, state_in,
+        state_out, static_cast<const bf*>(h_S), static_cast<bf*>(y), 0);
   }
-  TTCD_TRY(cast_bf16<float>(c, u_T, u, m.BT * m.d));
-  TTCD_TRY(cast_bf16<float>(c, u_S, u + m.BT * m.d, m.BT * m.d));
-  __nv_bfloat16* wg = at<__nv_bfloat16>(workspace, L, B_WGATE16);
-  __nv_bfloat16* wu = at<__nv_bfloat16>(workspace, L, B_WUP16);
-  __nv_bfloat16* wd = at<__nv_bfloat16>(workspace, L, B_WDOWN16);
-  TTCD_TRY(cast_bf16<float>(c, w->w_gate, wg, static_cast<long long>(m.f) * m.d));
-  TTCD_TRY(cast_bf16<float>(c, w->w_up, wu, static_cast<long long>(m.f) * m.d));
-  TTCD_TRY(cast_bf16<float>(c, w->w_down, wd, static_cast<long long>(m.f) * m.d));
   return run_mlp_core<float, float, float>(
-      c, p, L, workspace, wg, wu, wd, w->w_proj, true, static_cast<const float*>(w->conv_T),
+      c, p, L, workspace, static_cast<const float*>(w->w_gate),
+      static_cast<const float*>(w->w_up), static_cast<const float*>(w->w_down),
+      static_cast<const float*>(w->w_proj), static_cast<const float*>(w->conv_T),
       static_cast<const float*>(w->conv_S), beta, state_in, state_out,
       static_cast<const float*>(h_S), static_cast<float*>(y), 0);
 }
+
+}  // extern "C"
+
+namespace {
+// The block for operand type E (bf16: kind::f16 tensor cores; fp32: kind::tf32).
+template <class E>
+ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
+                      const ttcd_block_weights* w, const ttcd_block_params* p, float* state_out,
+                      void* out, void* ws, const Layout& L) {
+  const Dims m = dims_of(p);
+  E* xn = at<E>(ws, L, B_XN);
+  __nv_bfloat16* q = at<__nv_bfloat16>(ws, L, B_Q);
+  __nv_bfloat16* k = at<__nv_bfloat16>(ws, L, B_K);
+  __nv_bfloat16* v = at<__nv_bfloat16>(ws, L, B_V);
+  E* o = at<E>(ws, L, B_O);
+  float* h = at<float>(ws, L, B_H);
+  float2* rope = at<float2>(ws, L, B_ROPE);
+  E* u = at<E>(ws, L, B_U);
+  const E* xin = static_cast<const E*>(x);
+
+  // Rotary table, input RMSNorm.
+  stage_mark(c.s, 0);
+  rope_table_kernel<<<cdiv(static_cast<long long>(p->T) * (m.hd / 2), 256), 256, 0, c.s>>>(
+      rope, p->T, m.hd, static_cast<double>(p->rope_theta));
+  TTCD_CHECK_LAUNCH();
+  rmsnorm_kernel<E, E, E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(
+      xin, static_cast<const E*>(w->g_attn), xn, m.BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  stage_mark(c.s, 1);
+
+  // Shared Q/K/V with RoPE.
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<E>(&mA, xn, m.BT, m.d, 128) || !map_rows<E>(&mB, w->w_qkv, m.dqkv, m.d, 128))
+      return TTCD_ERR_CUDA;
+    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 128), m.d);
+    switch (m.hd) {
+      case 32: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 64: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      default: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+    }
+  }
+  stage_mark(c.s, 2);
+  // Dual-window attention: o_T rows then o_S rows.
+  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
+  TTCD_TRY(run_attn<E>(c, q, k, v, o, o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq,
+                       m.Hkv, m.hd, p->w_S, p->w_T, sc));
+  stage_mark(c.s, 3);
+  // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
+        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 128))
+      return TTCD_ERR_CUDA;
+    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 128), m.Hq * m.hd);
+    EpiResidual<float, E> e{h, m.d, xin, m.d, m.BT, m.d};
+    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, e)));
+  }
+  stage_mark(c.s, 4);
+  // u_P = RMSNorm(h_P; g_mlp), the gate/up operand.
+  rmsnorm_kernel<float, E, E><<<cdiv(2 * m.BT, 8), 256, 0, c.s>>>(
+      h, static_cast<const E*>(w->g_mlp), u, 2 * m.BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+
+  const float* h_S = h + m.BT * m.d;
+  return run_mlp_core<E, E, float>(c, p, L, ws, static_cast<const E*>(w->w_gate),
+                                   static_cast<const E*>(w->w_up),
+                                   static_cast<const E*>(w->w_down),
+                                   static_cast<const E*>(w->w_proj),
+                                   static_cast<const E*>(w->conv_T),
+                                   static_cast<const E*>(w->conv_S), beta, nullptr, state_out,
+                                   h_S, static_cast<E*>(out), 5);
+}
+}  // namespace
+
+extern "C" {
 
 ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_block_weights* w,
                                const ttcd_block_params* p, float* state_out, void* out,
@@ -571,106 +635,9 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
   if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
   Ctx c;
   TTCD_TRY(make_ctx(stream, c));
-  const Dims m = dims_of(p);
-  const bool f32 = p->dtype == TTCD_F32;
-  void* ws = workspace;
-  __nv_bfloat16* xn = at<__nv_bfloat16>(ws, L, B_XN);
-  __nv_bfloat16* q = at<__nv_bfloat16>(ws, L, B_Q);
-  __nv_bfloat16* k = at<__nv_bfloat16>(ws, L, B_K);
-  __nv_bfloat16* v = at<__nv_bfloat16>(ws, L, B_V);
-  __nv_bfloat16* o = at<__nv_bfloat16>(ws, L, B_O);
-  float* h = at<float>(ws, L, B_H);
-  float2* rope = at<float2>(ws, L, B_ROPE);
-  __nv_bfloat16* u = at<__nv_bfloat16>(ws, L, B_U);
-
-  const __nv_bfloat16 *wqkv, *wo, *wg, *wu, *wd;
-  if (f32) {
-    wqkv = at<__nv_bfloat16>(ws, L, B_WQKV16);
-    wo = at<__nv_bfloat16>(ws, L, B_WO16);
-    wg = at<__nv_bfloat16>(ws, L, B_WGATE16);
-    wu = at<__nv_bfloat16>(ws, L, B_WUP16);
-    wd = at<__nv_bfloat16>(ws, L, B_WDOWN16);
-    TTCD_TRY(cast_bf16<float>(c, w->w_qkv, const_cast<__nv_bfloat16*>(wqkv), static_cast<long long>(m.dqkv) * m.d));
-    TTCD_TRY(cast_bf16<float>(c, w->w_o, const_cast<__nv_bfloat16*>(wo), static_cast<long long>(m.d) * m.Hq * m.hd));
-    TTCD_TRY(cast_bf16<float>(c, w->w_gate, const_cast<__nv_bfloat16*>(wg), static_cast<long long>(m.f) * m.d));
-    TTCD_TRY(cast_bf16<float>(c, w->w_up, const_cast<__nv_bfloat16*>(wu), static_cast<long long>(m.f) * m.d));
-    TTCD_TRY(cast_bf16<float>(c, w->w_down, const_cast<__nv_bfloat16*>(wd), static_cast<long long>(m.f) * m.d));
-  } else {
-    wqkv = static_cast<const __nv_bfloat16*>(w->w_qkv);
-    wo = static_cast<const __nv_bfloat16*>(w->w_o);
-    wg = static_cast<const __nv_bfloat16*>(w->w_gate);
-    wu = static_cast<const __nv_bfloat16*>(w->w_up);
-    wd = static_cast<const __nv_bfloat16*>(w->w_down);
-  }
-
-  // Rotary table, input RMSNorm.
-  stage_mark(c.s, 0);
-  rope_table_kernel<<<cdiv(static_cast<long long>(p->T) * (m.hd / 2), 256), 256, 0, c.s>>>(
-      rope, p->T, m.hd, static_cast<double>(p->rope_theta));
-  TTCD_CHECK_LAUNCH();
-  if (f32)
-    rmsnorm_kernel<float, float><<<cdiv(m.BT, 8), 256, 0, c.s>>>(
-        static_cast<const float*>(x), static_cast<const float*>(w->g_attn), xn, m.BT, m.d, p->rms_eps);
-  else
-    rmsnorm_kernel<__nv_bfloat16, __nv_bfloat16><<<cdiv(m.BT, 8), 256, 0, c.s>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w->g_attn), xn,
-        m.BT, m.d, p->rms_eps);
-  TTCD_CHECK_LAUNCH();
-  stage_mark(c.s, 1);
-
-  // Shared Q/K/V with RoPE.
-  {
-    CUtensorMap mA, mB;
-    if (!map_rows(&mA, xn, m.BT, m.d, 128) || !map_rows(&mB, wqkv, m.dqkv, m.d, 128))
-      return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 128), m.d);
-    switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      case 64: TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      default: TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-    }
-  }
-  stage_mark(c.s, 2);
-  // Dual-window attention: o_T rows then o_S rows.
-  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
-  TTCD_TRY(run_attn(c, q, k, v, o, o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq,
-                    m.Hkv, m.hd, p->w_S, p->w_T, sc));
-  stage_mark(c.s, 3);
-  // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
-  {
-    CUtensorMap mA, mB;
-    if (!map_rows(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
-        !map_rows(&mB, wo, m.d, static_cast<long long>(m.Hq) * m.hd, 128))
-      return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 128), m.Hq * m.hd);
-    if (f32) {
-      EpiResidual<float, float> e{h, m.d, static_cast<const float*>(x), m.d, m.BT, m.d};
-      TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, e)));
-    } else {
-      EpiResidual<float, __nv_bfloat16> e{h, m.d, static_cast<const __nv_bfloat16*>(x), m.d, m.BT, m.d};
-      TTCD_TRY((launch_gemm<128, 6, false>(c, mA, mB, mB, g, e)));
-    }
-  }
-  stage_mark(c.s, 4);
-  // u_P = RMSNorm(h_P; g_mlp) in bf16 for the gate/up GEMM.
-  if (f32)
-    rmsnorm_kernel<float, float><<<cdiv(2 * m.BT, 8), 256, 0, c.s>>>(
-        h, static_cast<const float*>(w->g_mlp), u, 2 * m.BT, m.d, p->rms_eps);
-  else
-    rmsnorm_kernel<float, __nv_bfloat16><<<cdiv(2 * m.BT, 8), 256, 0, c.s>>>(
-        h, static_cast<const __nv_bfloat16*>(w->g_mlp), u, 2 * m.BT, m.d, p->rms_eps);
-  TTCD_CHECK_LAUNCH();
-
-  const float* h_S = h + m.BT * m.d;
-  if (f32)
-    return run_mlp_core<float, float, float>(c, p, L, ws, wg, wu, wd, w->w_proj, true,
-                                             static_cast<const float*>(w->conv_T),
-                                             static_cast<const float*>(w->conv_S), beta, nullptr,
-                                             state_out, h_S, static_cast<float*>(out), 5);
-  return run_mlp_core<__nv_bfloat16, float, __nv_bfloat16>(
-      c, p, L, ws, wg, wu, wd, w->w_proj, false, static_cast<const __nv_bfloat16*>(w->conv_T),
-      static_cast<const __nv_bfloat16*>(w->conv_S), beta, nullptr, state_out, h_S,
-      static_cast<__nv_bfloat16*>(out), 5);
+  if (p->dtype == TTCD_F32)
+    return run_block<float>(c, x, beta, w, p, state_out, out, workspace, L);
+  return run_block<__nv_bfloat16>(c, x, beta, w, p, state_out, out, workspace, L);
 }
 
 // ---------------------------------------------------------------------------

@@ -197,12 +197,13 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  * Byte offset inside the block_forward workspace of a named intermediate, for
  * inspection after a call (same layout for ttcd_fastweight_mlp where named).
  * Names and layouts (row-major):
- *   "xn"   bf16 [B*T, d]          "q" bf16 [B*T, Hq*hd]   "k","v" bf16 [B*T, Hkv*hd]
- *   "o"    bf16 [2, B*T, Hq*hd]   (o_T rows, then o_S rows)
- *   "h"    fp32 [2, B*T, d]       "u" bf16 [2, B*T, d]
- *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f]
- *   "D"    bf16 [P, f]            "Kt" bf16 [f, P]        "ssq" fp32 [f/64, P]
- *   "Rt"   bf16 [d, P]            "Wall" bf16 [B*n_chunks, d, f]
+ *   (E = bf16 for TTCD_BF16, fp32 for TTCD_F32; q, k, v are always bf16)
+ *   "xn"   E [B*T, d]             "q" bf16 [B*T, Hq*hd]   "k","v" bf16 [B*T, Hkv*hd]
+ *   "o"    E [2, B*T, Hq*hd]      (o_T rows, then o_S rows)
+ *   "h"    fp32 [2, B*T, d]       "u" E [2, B*T, d]
+ *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f] (TTCD_BF16 only)
+ *   "D"    E [P, f]               "Kt" E [f, P]           "ssq" fp32 [f/64, P]
+ *   "Rt"   E [d, P]               "Wall" E [B*n_chunks, d, f]
  * where P = B * n_chunks * Cp, Cp = chunk rounded up to 64, and token t of
  * sequence b sits at padded index (b*n_chunks + t/C)*Cp + t%C.
  * Returns TTCD_ERR_INVALID_ARG for an unknown name or invalid params.
