@@ -212,7 +212,8 @@ def run_reference(args, world, rank):
 def run_ours(args, world, rank, local):
     import dual_window_attention_b200 as ttcd
     ttcd.load_library()
-    shape = QWEN3_0P6B_64K
+    shape = QWEN3_0P6B_64K if args.T == QWEN3_0P6B_64K.T else QWEN3_0P6B_64K.with_(
+        name=f"qwen3_0.6b_block_T{args.T}", T=args.T)
     peaks, peak_kind = load_peaks()
     dev = torch.device("cuda", local)
     inp = make_block_inputs(shape, seed=0)
@@ -384,7 +385,9 @@ def main():
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
     ap.add_argument("--mode", choices=["block", "attn"], default="block",
                     help="block: the whole IP-TTCD block (default); attn: attention alone")
-    ap.add_argument("--T", type=int, default=65536, help="--mode attn: tokens per sequence")
+    ap.add_argument("--T", type=int, default=65536,
+                    help="tokens per sequence (65536 is the benchmark workload; smaller values "
+                         "are for profiling)")
     ap.add_argument("--B", type=int, default=1, help="--mode attn: sequences")
     ap.add_argument("--windows", default="512/8192",
                     help="--mode attn: comma-separated w_S/w_T pairs")

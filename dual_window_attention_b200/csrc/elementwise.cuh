@@ -118,10 +118,12 @@ __global__ void __launch_bounds__(256)
   __shared__ __align__(16) float zT[ROWS][CONV_TC];
   __shared__ __align__(16) float zS[ROWS][CONV_TC];
   __shared__ float taps[2][CONV_MAXK][CONV_TC];
-  // the key tile reuses zT's storage once the convolutions are done
-  typedef E KRow[CONV_TP + 16 / sizeof(E)];
-  KRow* tileK = reinterpret_cast<KRow*>(&zT[0][0]);
-  static_assert(sizeof(zT) >= sizeof(KRow) * CONV_TC, "key tile must fit in zT");
+  // The key tile (token-major fp32, odd row stride of 65 words so that both its
+  // row writes and its column reads spread over the banks) reuses zT's storage
+  // once the convolutions are done.
+  constexpr int KSTRIDE = CONV_TC + 1;
+  float* tileK = &zT[0][0];
+  static_assert(sizeof(zT) >= sizeof(float) * KSTRIDE * CONV_TP, "key tile must fit in zT");
   const long long p0 = static_cast<long long>(blockIdx.x) * CONV_TP;
   const int c0 = blockIdx.y * CONV_TC;
   const long long seq_len_p = static_cast<long long>(Nc) * Cp;
@@ -191,14 +193,18 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int it = 0; it < CONV_TP / 16; ++it)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) tileK[4 * cq + e][tr + 16 * it] = from_f32<E>(keys[it][e]);
+    for (int e = 0; e < 4; ++e) tileK[(tr + 16 * it) * KSTRIDE + 4 * cq + e] = keys[it][e];
   __syncthreads();
-  // Transposed store of the keys: each row of Kt gets 64 positions in 16-byte segments.
+  // Transposed store of the keys: each row of Kt (one channel) gets 64 positions
+  // in 16-byte segments; consecutive threads write consecutive segments.
   constexpr int SEG_E = 16 / sizeof(E), SEGS = CONV_TP / SEG_E;
   for (int i = tid; i < CONV_TC * SEGS; i += 256) {
     const int r = i / SEGS, seg = i % SEGS;
-    const uint4 w = *reinterpret_cast<const uint4*>(&tileK[r][seg * SEG_E]);
-    *reinterpret_cast<uint4*>(Kt + static_cast<long long>(c0 + r) * P + p0 + seg * SEG_E) = w;
+    __align__(16) E vals[SEG_E];
+#pragma unroll
+    for (int j = 0; j < SEG_E; ++j) vals[j] = from_f32<E>(tileK[(seg * SEG_E + j) * KSTRIDE + r]);
+    *reinterpret_cast<uint4*>(Kt + static_cast<long long>(c0 + r) * P + p0 + seg * SEG_E) =
+        *reinterpret_cast<const uint4*>(vals);
   }
 }
 

@@ -322,11 +322,11 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   // Z_P = silu(u_P W_gate^T) * (u_P W_up^T), both paths stacked (slow weights).
   {
     CUtensorMap mA, mB0, mB1;
-    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 64) ||
-        !map_rows<E>(&mB1, w_up, m.f, m.d, 64))
+    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 128) ||
+        !map_rows<E>(&mB1, w_up, m.f, m.d, 128))
       return TTCD_ERR_CUDA;
     EpiSwiGLU e{Z, m.f, m.f};
-    TTCD_TRY((launch_gemm<E, 128, 6, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, m.f / 64, m.d), e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
   }
   stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
@@ -347,10 +347,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     transpose_kernel<E, E><<<tg, tb, 0, c.s>>>(w_proj, WprojT, m.f, m.f);
     TTCD_CHECK_LAUNCH();
     CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, w_down, m.d, m.f, 128) || !map_rows<E>(&mB, WprojT, m.f, m.f, 128))
+    if (!map_rows<E>(&mA, w_down, m.d, m.f, 128) || !map_rows<E>(&mB, WprojT, m.f, m.f, 256))
       return TTCD_ERR_CUDA;
     EpiStore<E> e{M, m.f, m.f, nullptr};
-    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.f, 128), m.f), e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 3);
   // R^T = M D^T, scaled per token by beta_t / ||Zbar_S[t]||.
@@ -393,7 +393,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     CUtensorMap mA, mB;
     const void* zs = Zs ? static_cast<const void*>(Zs) : static_cast<const void*>(Z + m.BT * m.f);
     if (!map_rows<E>(&mA, zs, m.BT, m.f, 128) ||
-        !map_rows<E>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 128))
+        !map_rows<E>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 256))
       return TTCD_ERR_CUDA;
     GemmGeom g;
     g.n_seq = p->B;
@@ -402,10 +402,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     g.Nc = m.Nc;
     g.K = m.f;
     g.tiles_m = cdiv(p->chunk, 128);
-    g.tiles_n = cdiv(m.d, 128);
+    g.tiles_n = cdiv(m.d, 256);
     g.b_group_rows = m.d;
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, e)));
   }
   stage_mark(c.s, mark + 6);
   return TTCD_OK;
@@ -580,13 +580,13 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
   // Shared Q/K/V with RoPE.
   {
     CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, xn, m.BT, m.d, 128) || !map_rows<E>(&mB, w->w_qkv, m.dqkv, m.d, 128))
+    if (!map_rows<E>(&mA, xn, m.BT, m.d, 128) || !map_rows<E>(&mB, w->w_qkv, m.dqkv, m.d, 256))
       return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 128), m.d);
+    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
     switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      case 64: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      default: TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
     }
   }
   stage_mark(c.s, 2);
@@ -599,11 +599,11 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
   {
     CUtensorMap mA, mB;
     if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
-        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 128))
+        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
       return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 128), m.Hq * m.hd);
+    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
     EpiResidual<float, E> e{h, m.d, xin, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 128, 6, false>(c, mA, mB, mB, g, e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, e)));
   }
   stage_mark(c.s, 4);
   // u_P = RMSNorm(h_P; g_mlp), the gate/up operand.
