@@ -92,119 +92,103 @@ __global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double
 // Fused short causal convolutions, residual difference and student keys.
 // papernotes.org review, 关键设计 3: Zbar_P = conv_P(Z_P) (depthwise, causal),
 // D = Zbar_T - Zbar_S, K = l2-norm(Zbar_S).  The per-row norm needs the whole
-// d_ff row, so this kernel writes Zbar_S unnormalised (transposed, Kt) and the
-// squares of its 64-channel slice into ssq_part[channel block][p]; the scale
-// beta_t / ||.|| is applied to the value residual instead (Delta W = sum beta r
-// k^T is linear in that scale).
+// d_ff row, so this kernel writes Zbar_S unnormalised (Kp) and the squares of
+// its 64-channel slice into ssq_part[channel block][p]; the scale
+// beta_t / ||.|| is applied to the value residual instead (Delta W = sum
+// beta r k^T is linear in that scale).
 //
 // Z     fp32 [2, BT, f]: teacher rows then student rows
 // taps  [f, k] (tap m multiplies t - m), TapT = bf16 or fp32
-// D     bf16 [P, f]      Kt bf16 [f, P]     Zs16 bf16 [BT, f]    ssq_part fp32 [f/64, P]
+// D, Kp E [P, f]         Zs16 E [BT, f] (nullable)        ssq_part fp32 [f/64, P]
 // Padded index p = (b*Nc + i)*Cp + j holds token t = i*C + j when j < C and t < T;
-// other p get D = 0 and Kt = 0.
-// Block: 64 padded positions (inside one chunk, since Cp is a multiple of 64) x
-// 64 channels, 256 threads.  The Z rows t0-(k-1) .. t0+63 of both paths are
-// staged in shared memory with coalesced 16-byte loads (16 threads per 256-byte
-// row); thread (cq, tr) then owns channels 4cq..4cq+3 of positions tr + 16 i.
-constexpr int CONV_TP = 64, CONV_TC = 64, CONV_MAXK = 8;
-template <class TapT, class E>
-__global__ void __launch_bounds__(256)
+// other p get D = 0 and Kp = 0.
+// Block: 64 channels x 64 padded positions (inside one chunk: Cp is a multiple
+// of 64), 256 threads; thread (cq, tg) owns channels 4cq..4cq+3 of positions
+// 4tg..4tg+3 and slides a k-row window over them in registers.  A warp's loads
+// and stores cover two 256-byte (fp32) or 128-byte (bf16) row segments.
+// Blocks of one position tile run back to back over the channel blocks, so
+// concurrently running blocks read whole rows of Z.
+constexpr int CONV_TP = 64, CONV_TC = 64;
+template <class TapT, class E, int CONV_MAXK>  // conv width k <= CONV_MAXK
+__global__ void __launch_bounds__(256, CONV_MAXK <= 4 ? 3 : 1)
     conv_residual_key_kernel(const float* __restrict__ Z, const TapT* __restrict__ tapT,
                              const TapT* __restrict__ tapS, E* __restrict__ D,
-                             E* __restrict__ Kt, E* __restrict__ Zs16,
+                             E* __restrict__ Kp, E* __restrict__ Zs16,
                              float* __restrict__ ssq_part, int T, int f, int k, int C, int Cp,
                              int Nc, long long BT, long long P) {
-  constexpr int ROWS = CONV_TP + CONV_MAXK - 1;
-  __shared__ __align__(16) float zT[ROWS][CONV_TC];
-  __shared__ __align__(16) float zS[ROWS][CONV_TC];
-  __shared__ float taps[2][CONV_MAXK][CONV_TC];
-  // The key tile (token-major fp32, odd row stride of 65 words so that both its
-  // row writes and its column reads spread over the banks) reuses zT's storage
-  // once the convolutions are done.
-  constexpr int KSTRIDE = CONV_TC + 1;
-  float* tileK = &zT[0][0];
-  static_assert(sizeof(zT) >= sizeof(float) * KSTRIDE * CONV_TP, "key tile must fit in zT");
-  const long long p0 = static_cast<long long>(blockIdx.x) * CONV_TP;
-  const int c0 = blockIdx.y * CONV_TC;
+  const int cblk = blockIdx.x;
+  const long long p0 = static_cast<long long>(blockIdx.y) * CONV_TP;
+  const int c0 = cblk * CONV_TC;
+  const int tid = threadIdx.x;
+  const int cq = tid & 15, tg = tid >> 4;
+  const int c = c0 + 4 * cq;
   const long long seq_len_p = static_cast<long long>(Nc) * Cp;
   const int b = static_cast<int>(p0 / seq_len_p);
   const long long rem0 = p0 % seq_len_p;
   const int ci = static_cast<int>(rem0 / Cp), j0 = static_cast<int>(rem0 % Cp);
-  const int t0 = ci * C + j0;               // token of position p0 (if valid)
-  const int n_valid = max(0, min(CONV_TP, min(C - j0, T - t0)));
+  const int tc0 = ci * C;                       // first token of this chunk
+  const int len = min(C, T - tc0);              // tokens of this chunk
   const long long rowT0 = static_cast<long long>(b) * T;
-  const int tid = threadIdx.x;
 
-  for (int i = tid; i < 2 * CONV_MAXK * CONV_TC; i += 256) {
-    const int path = i / (CONV_MAXK * CONV_TC), m = (i / CONV_TC) % CONV_MAXK, c = i % CONV_TC;
-    const TapT* tp = path ? tapS : tapT;
-    taps[path][m][c] = m < k ? to_f32(tp[static_cast<long long>(c0 + c) * k + m]) : 0.f;
-  }
-  // Stage rows t0-(k-1) .. t0+n_valid-1 (missing rows are zero).
-  const int halo = k - 1;
-  for (int i = tid; i < (n_valid + halo) * 16; i += 256) {
-    const int rr = i >> 4, cq = i & 15;
-    const int t = t0 - halo + rr;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), s = a;
-    if (t >= 0) {
-      a = *reinterpret_cast<const float4*>(Z + (rowT0 + t) * f + c0 + 4 * cq);
-      s = *reinterpret_cast<const float4*>(Z + (BT + rowT0 + t) * f + c0 + 4 * cq);
-    }
-    *reinterpret_cast<float4*>(&zT[CONV_MAXK - 1 - halo + rr][4 * cq]) = a;
-    *reinterpret_cast<float4*>(&zS[CONV_MAXK - 1 - halo + rr][4 * cq]) = s;
-  }
-  __syncthreads();
-
-  const int cq = tid & 15, tr = tid >> 4;
-  float keys[CONV_TP / 16][4];
+  float wT[CONV_MAXK][4], wS[CONV_MAXK][4];
 #pragma unroll
-  for (int it = 0; it < CONV_TP / 16; ++it) {
-    const int jj = tr + 16 * it;  // position within the tile
-    const long long p = p0 + jj;
-    const bool valid = jj < n_valid;
-    float zbT[4] = {0.f, 0.f, 0.f, 0.f}, zbS[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int m = 0; m < CONV_MAXK; ++m)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      wT[m][e] = m < k ? to_f32(tapT[static_cast<long long>(c + e) * k + m]) : 0.f;
+      wS[m][e] = m < k ? to_f32(tapS[static_cast<long long>(c + e) * k + m]) : 0.f;
+    }
+  // history: rows t-1 .. t-(k-1) of both paths for the first of this thread's positions
+  const int jfirst = j0 + 4 * tg;
+  float4 hT[CONV_MAXK - 1], hS[CONV_MAXK - 1];  // hT[m-1] = Z_T row (t - m)
+#pragma unroll
+  for (int m = 1; m < CONV_MAXK; ++m) {
+    hT[m - 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    hS[m - 1] = hT[m - 1];
+    const int t = tc0 + jfirst - m;
+    if (m < k && t >= 0 && jfirst < len) {
+      hT[m - 1] = *reinterpret_cast<const float4*>(Z + (rowT0 + t) * f + c);
+      hS[m - 1] = *reinterpret_cast<const float4*>(Z + (BT + rowT0 + t) * f + c);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = jfirst + q;
+    const long long p = p0 + 4 * tg + q;
+    const bool valid = j < len;
+    float4 zt = make_float4(0.f, 0.f, 0.f, 0.f), zs = zt;
     if (valid) {
-      for (int m = 0; m < k; ++m) {
-        const int row = CONV_MAXK - 1 + jj - m;
-        const float4 a = *reinterpret_cast<const float4*>(&zT[row][4 * cq]);
-        const float4 s = *reinterpret_cast<const float4*>(&zS[row][4 * cq]);
-        zbT[0] += taps[0][m][4 * cq + 0] * a.x; zbS[0] += taps[1][m][4 * cq + 0] * s.x;
-        zbT[1] += taps[0][m][4 * cq + 1] * a.y; zbS[1] += taps[1][m][4 * cq + 1] * s.y;
-        zbT[2] += taps[0][m][4 * cq + 2] * a.z; zbS[2] += taps[1][m][4 * cq + 2] * s.z;
-        zbT[3] += taps[0][m][4 * cq + 3] * a.w; zbS[3] += taps[1][m][4 * cq + 3] * s.w;
-      }
+      zt = *reinterpret_cast<const float4*>(Z + (rowT0 + tc0 + j) * f + c);
+      zs = *reinterpret_cast<const float4*>(Z + (BT + rowT0 + tc0 + j) * f + c);
     }
-    // D (zeros at padding) and the bf16 copy of Z_S, 8 bytes per thread, 128 bytes per row.
-    store4(D + p * f + c0 + 4 * cq, zbT[0] - zbS[0], zbT[1] - zbS[1], zbT[2] - zbS[2],
-           zbT[3] - zbS[3]);
-    if (valid && Zs16) {
-      const float4 s = *reinterpret_cast<const float4*>(&zS[CONV_MAXK - 1 + jj][4 * cq]);
-      store4(Zs16 + (rowT0 + t0 + jj) * f + c0 + 4 * cq, s.x, s.y, s.z, s.w);
-    }
+    float bT[4] = {wT[0][0] * zt.x, wT[0][1] * zt.y, wT[0][2] * zt.z, wT[0][3] * zt.w};
+    float bS[4] = {wS[0][0] * zs.x, wS[0][1] * zs.y, wS[0][2] * zs.z, wS[0][3] * zs.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) keys[it][e] = zbS[e];
-    // squares of this 64-channel slice, reduced over the 16 threads of the row
-    float sq = zbS[0] * zbS[0] + zbS[1] * zbS[1] + zbS[2] * zbS[2] + zbS[3] * zbS[3];
+    for (int m = 1; m < CONV_MAXK; ++m) {
+      bT[0] += wT[m][0] * hT[m - 1].x; bS[0] += wS[m][0] * hS[m - 1].x;
+      bT[1] += wT[m][1] * hT[m - 1].y; bS[1] += wS[m][1] * hS[m - 1].y;
+      bT[2] += wT[m][2] * hT[m - 1].z; bS[2] += wS[m][2] * hS[m - 1].z;
+      bT[3] += wT[m][3] * hT[m - 1].w; bS[3] += wS[m][3] * hS[m - 1].w;
+    }
+    if (!valid) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bT[e] = bS[e] = 0.f;
+    }
+    store4(D + p * f + c, bT[0] - bS[0], bT[1] - bS[1], bT[2] - bS[2], bT[3] - bS[3]);
+    store4(Kp + p * f + c, bS[0], bS[1], bS[2], bS[3]);
+    if (valid && Zs16) store4(Zs16 + (rowT0 + tc0 + j) * f + c, zs.x, zs.y, zs.z, zs.w);
+    float sq = bS[0] * bS[0] + bS[1] * bS[1] + bS[2] * bS[2] + bS[3] * bS[3];
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (cq == 0) ssq_part[static_cast<long long>(blockIdx.y) * P + p] = sq;
-  }
-  __syncthreads();
+    if (cq == 0) ssq_part[static_cast<long long>(cblk) * P + p] = sq;
+    // slide the window
 #pragma unroll
-  for (int it = 0; it < CONV_TP / 16; ++it)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) tileK[(tr + 16 * it) * KSTRIDE + 4 * cq + e] = keys[it][e];
-  __syncthreads();
-  // Transposed store of the keys: each row of Kt (one channel) gets 64 positions
-  // in 16-byte segments; consecutive threads write consecutive segments.
-  constexpr int SEG_E = 16 / sizeof(E), SEGS = CONV_TP / SEG_E;
-  for (int i = tid; i < CONV_TC * SEGS; i += 256) {
-    const int r = i / SEGS, seg = i % SEGS;
-    __align__(16) E vals[SEG_E];
-#pragma unroll
-    for (int j = 0; j < SEG_E; ++j) vals[j] = from_f32<E>(tileK[(seg * SEG_E + j) * KSTRIDE + r]);
-    *reinterpret_cast<uint4*>(Kt + static_cast<long long>(c0 + r) * P + p0 + seg * SEG_E) =
-        *reinterpret_cast<const uint4*>(vals);
+    for (int m = CONV_MAXK - 2; m > 0; --m) {
+      hT[m] = hT[m - 1];
+      hS[m] = hS[m - 1];
+    }
+    hT[0] = zt;
+    hS[0] = zs;
   }
 }
 

@@ -250,27 +250,26 @@ constexpr int gemm_smem_bytes() {
 
 // ------------------------------------------------------------------ epilogues
 
-// C[row, col] = OutT(acc * col_scale[col]) (col_scale nullable), columns < N.
+// C[row, col] = OutT(acc * row_scale[row]) (row_scale nullable), columns < N.
 template <class OutT>
 struct EpiStore {
   OutT* out;
   long long ldo;
   int N;
-  const float* col_scale;
+  const float* row_scale;
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const float sc = (row_scale && ok) ? __ldg(row_scale + row) : 1.f;
 #pragma unroll 1
     for (int cc = 0; cc < BN; cc += 32) {
       const int col = c.tn * BN + cc;
       if (col >= N) break;
       float v[32];
       tmem_ld32f(taddr + cc, v);
-      if (col_scale) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= __ldg(col_scale + col + i);
-      }
+      for (int i = 0; i < 32; ++i) v[i] *= sc;
       if (ok) store_x32(out + row * ldo + col, v);
     }
   }

@@ -7,8 +7,10 @@
 //
 // One CTA owns a 128 x 128 tile (rows of d, columns of f) of one sequence's
 // d x f state.  It walks the chunks in order.  For chunk i the tensor cores
-// form Delta W_i = Rt[:, chunk i] . Kt[:, chunk i]^T (contraction over the
-// chunk's padded tokens) in one of two TMEM accumulators, while the epilogue
+// form Delta W_i = R[chunk i]^T . Kp[chunk i] (contraction over the chunk's
+// padded tokens; R [P, d] and Kp [P, f] are token-major, so both operands are
+// MN-major tiles: boxes of BK MN-elements x BK tokens, 128-byte swizzled) in
+// one of two TMEM accumulators, while the epilogue
 // warps fold the previous chunk into the fp32 running state S (a third TMEM
 // region) and emit W_{i+1} = bf16(W_down + S_{i+1}) for the output GEMM.
 // Chunk 0 reads W_0 = bf16(W_down + state_in).  The last state is written to
@@ -28,16 +30,21 @@ struct ScanArgs {
   int tiles_m, tiles_n;
 };
 
-template <class E, int STAGES>
+// MN = true: R [P, d] and Kp [P, f] token-major, read as MN-major operands
+// (bf16).  MN = false: their transposes Rt [d, P] and Kt [f, P], read as
+// K-major operands (used for tf32, whose operands stay K-major).
+template <class E, int STAGES, bool MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fastweight_scan_kernel(const __grid_constant__ CUtensorMap mapR,
                            const __grid_constant__ CUtensorMap mapK, const ScanArgs<E> a,
                            const DevStatus st) {
   constexpr int BN = 128;
-  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;
+  constexpr int BK = ElemTraits<E>::BK;          // tokens per k-block == MN elements per box
+  constexpr int BOX_BYTES = BK * BK * static_cast<int>(sizeof(E));
+  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;  // 16 KB each either way
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, false);
-  constexpr int BK = ElemTraits<E>::BK;
+  constexpr int KSTEP_BYTES = (32 / static_cast<int>(sizeof(E))) * 128;  // tokens per MMA x 128 B
+  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, MN, MN);
   constexpr uint32_t COL_STATE = 256;
 
   extern __shared__ uint8_t smem_raw[];
@@ -87,10 +94,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, st, abort)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
-          const int x = (b * a.Nc + i) * a.Cp + kb * BK;
+          const int y = (b * a.Nc + i) * a.Cp + kb * BK;  // first token of the k-block
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(sa, &mapR, &full[s], x, m0);
-          tma_load_2d(sa + A_BYTES, &mapK, &full[s], x, n0);
+          if constexpr (MN) {
+#pragma unroll
+            for (int q = 0; q < GEMM_BM / BK; ++q)
+              tma_load_2d(sa + q * BOX_BYTES, &mapR, &full[s], m0 + q * BK, y);
+#pragma unroll
+            for (int q = 0; q < BN / BK; ++q)
+              tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
+          } else {
+            tma_load_2d(sa, &mapR, &full[s], y, m0);
+            tma_load_2d(sa + A_BYTES, &mapK, &full[s], y, n0);
+          }
         }
       }
       volatile int no_abort = 0;
@@ -111,9 +127,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_ss<E>(tmem + ab * BN, sdesc_sw128(sa + k * 32, 16, 1024),
-                      sdesc_sw128(sb + k * 32, 16, 1024), IDESC, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t da = MN ? sdesc_sw128(sa + k * KSTEP_BYTES, BOX_BYTES, 1024)
+                                   : sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t db = MN ? sdesc_sw128(sb + k * KSTEP_BYTES, BOX_BYTES, 1024)
+                                   : sdesc_sw128(sb + k * 32, 16, 1024);
+            mma_ss<E>(tmem + ab * BN, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
           mma_commit(&empty[s]);
         }
         if (!ok) break;

@@ -176,11 +176,11 @@ struct Layout {
   size_t total;
 };
 enum Buf {
-  B_XN, B_Q, B_K, B_V, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KT, B_SSQ, B_KSCALE, B_RT,
-  B_WALL, B_M, B_WPROJT, B_COUNT
+  B_XN, B_Q, B_K, B_V, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ, B_KSCALE, B_R,
+  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_COUNT
 };
 const char* kBufNames[B_COUNT] = {"xn", "q", "k", "v", "o", "h", "rope", "u", "Z", "Zs16", "D",
-                                  "Kt", "ssq", "kscale", "Rt", "Wall", "M", "WprojT"};
+                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt"};
 
 struct Dims {
   long long BT, P;
@@ -220,13 +220,17 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
   sz[B_Z] = 2 * m.BT * m.f * 4;
   sz[B_ZS16] = e == 2 ? m.BT * m.f * 2 : 0;  // fp32 mode reads Z_S directly
   sz[B_D] = m.P * m.f * e;
-  sz[B_KT] = m.P * m.f * e;
+  sz[B_KP] = m.P * m.f * e;
   sz[B_SSQ] = m.P * 4 * (m.f / 64);
   sz[B_KSCALE] = m.P * 4;
-  sz[B_RT] = m.P * m.d * e;
+  sz[B_R] = m.P * m.d * e;
   sz[B_WALL] = static_cast<size_t>(p->B) * m.Nc * m.d * m.f * e;
   sz[B_M] = static_cast<size_t>(m.d) * m.f * e;
   sz[B_WPROJT] = static_cast<size_t>(m.f) * m.f * e;
+  if (e == 4) {  // tf32 operands stay K-major: transposed copies for the chunk scan
+    sz[B_RT] = m.P * m.d * e;
+    sz[B_KT] = m.P * m.f * e;
+  }
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_COUNT; ++i) {
@@ -310,10 +314,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   float* Z = at<float>(ws, L, B_Z);
   E* Zs = sizeof(E) == 2 ? at<E>(ws, L, B_ZS16) : nullptr;
   E* D = at<E>(ws, L, B_D);
-  E* Kt = at<E>(ws, L, B_KT);
+  E* Kp = at<E>(ws, L, B_KP);
   float* ssq = at<float>(ws, L, B_SSQ);
   float* kscale = at<float>(ws, L, B_KSCALE);
-  E* Rt = at<E>(ws, L, B_RT);
+  E* R = at<E>(ws, L, B_R);
   E* Wall = at<E>(ws, L, B_WALL);
   E* M = at<E>(ws, L, B_M);
   E* WprojT = at<E>(ws, L, B_WPROJT);
@@ -331,10 +335,15 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
   {
-    dim3 grid(static_cast<unsigned>(m.P / CONV_TP), m.f / CONV_TC);
-    conv_residual_key_kernel<E, E><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kt, Zs, ssq,
-                                                          p->T, m.f, p->conv_k, p->chunk, m.Cp,
-                                                          m.Nc, m.BT, m.P);
+    dim3 grid(m.f / CONV_TC, static_cast<unsigned>(m.P / CONV_TP));
+    if (p->conv_k <= 4)
+      conv_residual_key_kernel<E, E, 4><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
+                                                               p->T, m.f, p->conv_k, p->chunk,
+                                                               m.Cp, m.Nc, m.BT, m.P);
+    else
+      conv_residual_key_kernel<E, E, 8><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
+                                                               p->T, m.f, p->conv_k, p->chunk,
+                                                               m.Cp, m.Nc, m.BT, m.P);
     TTCD_CHECK_LAUNCH();
     key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, m.f / CONV_TC, beta, kscale, p->T,
                                                       p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
@@ -353,21 +362,36 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 3);
-  // R^T = M D^T, scaled per token by beta_t / ||Zbar_S[t]||.
+  // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, M, m.d, m.f, 128) || !map_rows<E>(&mB, D, m.P, m.f, 256))
+    if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, 256))
       return TTCD_ERR_CUDA;
-    EpiStore<E> e{Rt, m.P, static_cast<int>(m.P), kscale};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.P, 256), m.f), e)));
+    EpiStore<E> e{R, m.d, m.d, kscale};
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 4);
   // Delta W per chunk, fp32 exclusive prefix scan, W_i = W_down + S_i.
   {
     CUtensorMap mR, mK;
-    if (!make_map<E>(&mR, Rt, m.P, m.d, m.P * sizeof(E), ElemTraits<E>::BK, 128) ||
-        !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), ElemTraits<E>::BK, 128))
-      return TTCD_ERR_CUDA;
+    constexpr uint32_t BK = ElemTraits<E>::BK;
+    constexpr bool MN = sizeof(E) == 2;
+    if (MN) {
+      if (!make_map<E>(&mR, R, m.d, m.P, m.d * sizeof(E), BK, BK) ||
+          !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), BK, BK))
+        return TTCD_ERR_CUDA;
+    } else {
+      E* Rt = at<E>(ws, L, B_RT);
+      E* Kt = at<E>(ws, L, B_KT);
+      dim3 tb(32, 8);
+      transpose_kernel<E, E><<<dim3(cdiv(m.d, 32), cdiv(m.P, 32)), tb, 0, c.s>>>(R, Rt, static_cast<int>(m.P), m.d);
+      TTCD_CHECK_LAUNCH();
+      transpose_kernel<E, E><<<dim3(cdiv(m.f, 32), cdiv(m.P, 32)), tb, 0, c.s>>>(Kp, Kt, static_cast<int>(m.P), m.f);
+      TTCD_CHECK_LAUNCH();
+      if (!make_map<E>(&mR, Rt, m.P, m.d, m.P * sizeof(E), BK, 128) ||
+          !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), BK, 128))
+        return TTCD_ERR_CUDA;
+    }
     ScanArgs<E> a;
     a.d = m.d;
     a.f = m.f;
@@ -381,7 +405,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     a.tiles_n = cdiv(m.f, 128);
     constexpr int STAGES = 6;
     constexpr int smem = gemm_smem_bytes<128, STAGES>();
-    auto kern = fastweight_scan_kernel<E, STAGES>;
+    auto kern = fastweight_scan_kernel<E, STAGES, MN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
     kern<<<p->B * a.tiles_m * a.tiles_n, GEMM_THREADS, smem, c.s>>>(mR, mK, a, c.st);

@@ -202,8 +202,9 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  *   "o"    E [2, B*T, Hq*hd]      (o_T rows, then o_S rows)
  *   "h"    fp32 [2, B*T, d]       "u" E [2, B*T, d]
  *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f] (TTCD_BF16 only)
- *   "D"    E [P, f]               "Kt" E [f, P]           "ssq" fp32 [f/64, P]
- *   "Rt"   E [d, P]               "Wall" E [B*n_chunks, d, f]
+ *   "D"    E [P, f]               "Kp" E [P, f] (unnormalised keys)  "ssq" fp32 [f/64, P]
+ *   "R"    E [P, d] (value residual times beta_t / ||Zbar_S[t]||)
+ *   "Wall" E [B*n_chunks, d, f]   (W_down + S_i per chunk)
  * where P = B * n_chunks * Cp, Cp = chunk rounded up to 64, and token t of
  * sequence b sits at padded index (b*n_chunks + t/C)*Cp + t%C.
  * Returns TTCD_ERR_INVALID_ARG for an unknown name or invalid params.
