@@ -99,12 +99,62 @@ __device__ __forceinline__ void load_x32(const float* src, float (&v)[32]) {
   }
 }
 
+// Per-warp staging of epilogue output for TMA stores: two 4 KB buffers, each
+// 32 rows x 128 bytes in the 128-byte swizzle (16-byte chunk j of row r sits
+// at slot j ^ (r & 7)), so a warp writing one chunk per row touches every bank
+// once per 8 rows.  One lane issues the store of the whole 32-row box.
+struct EpiStage {
+  uint8_t* buf;            // 2 x 4096 bytes, 1024-aligned; nullptr: direct stores
+  const CUtensorMap* map;  // output tensor map (box: 128 bytes x 32 rows)
+  int toggle;
+  __device__ bool on() const { return buf != nullptr; }
+  // Before writing into the current buffer: its previous store has read it.
+  __device__ void acquire() {
+    if ((threadIdx.x & 31) == 0) bulk_wait_read<1>();
+    __syncwarp();
+  }
+  __device__ void write_f32(int r, const float (&v)[32]) {
+    uint8_t* b = buf + toggle * 4096 + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(b + ((j ^ (r & 7)) << 4)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  }
+  __device__ void write_bf16(int r, const float (&lo)[32], const float (&hi)[32]) {
+    uint8_t* b = buf + toggle * 4096 + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float* v = j < 4 ? &lo[8 * j] : &hi[8 * (j - 4)];
+      uint4 w;
+      w.x = pack_bf16x2(v[0], v[1]);
+      w.y = pack_bf16x2(v[2], v[3]);
+      w.z = pack_bf16x2(v[4], v[5]);
+      w.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4*>(b + ((j ^ (r & 7)) << 4)) = w;
+    }
+  }
+  __device__ void flush(int x, int y) {
+    fence_async_smem();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+      tma_store_2d(map, buf + toggle * 4096, x, y);
+      bulk_commit();
+    }
+    toggle ^= 1;
+  }
+  __device__ void drain() {
+    if (buf && (threadIdx.x & 31) == 0) bulk_wait<0>();
+  }
+};
+
 template <class E, int BN, int STAGES, bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
-                   const __grid_constant__ CUtensorMap mapB1, const GemmGeom geo, const Epi epi,
+                   const __grid_constant__ CUtensorMap mapB1,
+                   const __grid_constant__ CUtensorMap mapOut, const GemmGeom geo, const Epi epi,
                    const DevStatus st) {
+  constexpr bool STAGED = Epi::kStaged;
   constexpr int A_BYTES = GEMM_BM * 128;
   constexpr int B_BYTES = BN * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -116,7 +166,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* staging = smem + STAGES * STAGE_BYTES;  // 4 warps x 8 KB when STAGED
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + (STAGED ? 4 * 8192 : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
@@ -128,6 +179,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    if (STAGED) tma_prefetch_map(&mapOut);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -223,6 +275,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
+    EpiStage stg{STAGED ? staging + (warp - 2) * 8192 : nullptr, &mapOut, 0};
     int j = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       TileCtx c;
@@ -230,11 +283,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int ab = j & 1;
       if (!mbar_wait(&accf[ab], (j >> 1) & 1, st, abort)) break;
       tc_fence_after();
-      epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r);
+      epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r,
+                           stg);
       tc_fence_before();
       mbar_arrive(&acce[ab]);
       ++j;
     }
+    stg.drain();
   }
   __syncthreads();
   if (warp == 1) {
@@ -243,34 +298,74 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool STAGED = false>
 constexpr int gemm_smem_bytes() {
-  return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + 256;
+  return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + (STAGED ? 4 * 8192 : 0) + 256;
 }
 
 // ------------------------------------------------------------------ epilogues
 
+// Writes one row's 32 (fp32) or 64 (bf16) output columns starting at `col`:
+// through the warp's staging buffer and a TMA store when all 32 rows of the
+// warp lie inside the tile, else with direct stores for the valid rows.
+template <class OutT>
+struct OutChunk {
+  static constexpr int COLS = sizeof(OutT) == 4 ? 32 : 64;
+};
+__device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok, float* out_row, int col,
+                                     int y, const float (&v)[32], const float (&)[32]) {
+  if (staged) {
+    stg.acquire();
+    stg.write_f32(threadIdx.x & 31, v);
+    stg.flush(col, y);
+  } else if (ok) {
+    store_f32x32(out_row + col, v);
+  }
+}
+__device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok,
+                                     __nv_bfloat16* out_row, int col, int y,
+                                     const float (&lo)[32], const float (&hi)[32]) {
+  if (staged) {
+    stg.acquire();
+    stg.write_bf16(threadIdx.x & 31, lo, hi);
+    stg.flush(col, y);
+  } else if (ok) {
+    store_bf16x32(out_row + col, lo);
+    store_bf16x32(out_row + col + 32, hi);
+  }
+}
+
 // C[row, col] = OutT(acc * row_scale[row]) (row_scale nullable), columns < N.
+// N must be a multiple of 64 for bf16 output.
 template <class OutT>
 struct EpiStore {
+  static constexpr bool kStaged = true;
   OutT* out;
   long long ldo;
   int N;
   const float* row_scale;
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const int wrow = r & ~31;
+    const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
     const float sc = (row_scale && ok) ? __ldg(row_scale + row) : 1.f;
+    constexpr int CW = OutChunk<OutT>::COLS;
 #pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
+    for (int cc = 0; cc < BN; cc += CW) {
       const int col = c.tn * BN + cc;
       if (col >= N) break;
-      float v[32];
-      tmem_ld32f(taddr + cc, v);
+      float lo[32], hi[32];
+      tmem_ld32f(taddr + cc, lo);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= sc;
-      if (ok) store_x32(out + row * ldo + col, v);
+      for (int i = 0; i < 32; ++i) lo[i] *= sc;
+      if (CW == 64) {
+        tmem_ld32f(taddr + cc + 32, hi);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hi[i] *= sc;
+      }
+      emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, lo, hi);
     }
   }
 };
@@ -279,6 +374,7 @@ using EpiStoreBF16 = EpiStore<__nv_bfloat16>;
 // out[row, col] = resid[row % resid_rows, col] + acc;  columns < N.
 template <class OutT, class ResT>
 struct EpiResidual {
+  static constexpr bool kStaged = true;
   OutT* out;
   long long ldo;
   const ResT* resid;  // nullable
@@ -286,24 +382,32 @@ struct EpiResidual {
   long long resid_rows;
   int N;
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const int wrow = r & ~31;
+    const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
+    const ResT* res_row = resid ? resid + (row % resid_rows) * ld_res : nullptr;
+    constexpr int CW = OutChunk<OutT>::COLS;
 #pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
+    for (int cc = 0; cc < BN; cc += CW) {
       const int col = c.tn * BN + cc;
       if (col >= N) break;
-      float v[32];
-      tmem_ld32f(taddr + cc, v);
-      if (ok) {
-        if (resid) {
-          float x[32];
-          load_x32(resid + (row % resid_rows) * ld_res + col, x);
+      float lo[32], hi[32];
+      tmem_ld32f(taddr + cc, lo);
+      if (CW == 64) tmem_ld32f(taddr + cc + 32, hi);
+      if (ok && res_row) {
+        float x[32];
+        load_x32(res_row + col, x);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] += x[i];
+        for (int i = 0; i < 32; ++i) lo[i] += x[i];
+        if (CW == 64) {
+          load_x32(res_row + col + 32, x);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hi[i] += x[i];
         }
-        store_x32(out + row * ldo + col, v);
       }
+      emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, lo, hi);
     }
   }
 };
@@ -311,13 +415,16 @@ struct EpiResidual {
 // Gate/up tile: accumulator columns [0, BN/2) are gate, [BN/2, BN) are up for
 // output columns tn*BN/2 + [0, BN/2).  Z = silu(gate) * up, fp32.
 struct EpiSwiGLU {
+  static constexpr bool kStaged = true;
   float* out;
   long long ldo;
   int N;  // d_ff
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const int wrow = r & ~31;
+    const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
 #pragma unroll 1
     for (int cc = 0; cc < BN / 2; cc += 32) {
       const int col = c.tn * (BN / 2) + cc;
@@ -327,7 +434,7 @@ struct EpiSwiGLU {
       tmem_ld32f(taddr + BN / 2 + cc, u);
 #pragma unroll
       for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
-      if (ok) store_f32x32(out + row * ldo + col, g);
+      emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, g, u);
     }
   }
 };
@@ -336,13 +443,14 @@ struct EpiSwiGLU {
 // Column n of the accumulator is feature n of [q heads | k heads | v heads].
 template <int HD>
 struct EpiQKVRope {
+  static constexpr bool kStaged = false;
   __nv_bfloat16* q;
   __nv_bfloat16* k;
   __nv_bfloat16* v;
   int Hq, Hkv, T;
   const float2* rope_cs;  // [T][HD/2] (cos, sin)
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&) const {
     static_assert(BN % HD == 0, "column tile must hold whole heads");
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;

@@ -120,17 +120,26 @@ void stage_mark(cudaStream_t s, int k) {
     g_launches.fetch_add(1, std::memory_order_relaxed);          \
   } while (0)
 
+// Output tensor map for the staged epilogue: boxes of 128 bytes x 32 rows.
+template <class OutT>
+bool make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                  uint64_t ld_elems) {
+  return make_map<OutT>(m, ptr, cols, rows, ld_elems * sizeof(OutT), 128 / sizeof(OutT), 32);
+}
+
 template <class E, int BN, int STAGES, bool DUAL, class Epi>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
-                        const CUtensorMap& B1, const GemmGeom& geo, const Epi& epi) {
+                        const CUtensorMap& B1, const CUtensorMap* out_map, const GemmGeom& geo,
+                        const Epi& epi) {
   const int total = geo.total();
   if (total <= 0) return TTCD_OK;
+  if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
   auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi>;
-  constexpr int smem = gemm_smem_bytes<BN, STAGES>();
+  constexpr int smem = gemm_smem_bytes<BN, STAGES, Epi::kStaged>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
   const int grid = total < c.sms ? total : c.sms;
-  kern<<<grid, GEMM_THREADS, smem, c.s>>>(A, B0, B1, geo, epi, c.st);
+  kern<<<grid, GEMM_THREADS, smem, c.s>>>(A, B0, B1, out_map ? *out_map : A, geo, epi, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
 }
@@ -329,8 +338,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 128) ||
         !map_rows<E>(&mB1, w_up, m.f, m.d, 128))
       return TTCD_ERR_CUDA;
+    CUtensorMap mo;
+    if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
     EpiSwiGLU e{Z, m.f, m.f};
-    TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
   }
   stage_mark(c.s, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
@@ -358,8 +369,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     CUtensorMap mA, mB;
     if (!map_rows<E>(&mA, w_down, m.d, m.f, 128) || !map_rows<E>(&mB, WprojT, m.f, m.f, 256))
       return TTCD_ERR_CUDA;
+    CUtensorMap mo;
+    if (!make_out_map<E>(&mo, M, m.d, m.f, m.f)) return TTCD_ERR_CUDA;
     EpiStore<E> e{M, m.f, m.f, nullptr};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 3);
   // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
@@ -367,8 +380,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     CUtensorMap mA, mB;
     if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, 256))
       return TTCD_ERR_CUDA;
+    CUtensorMap mo;
+    if (!make_out_map<E>(&mo, R, m.P, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiStore<E> e{R, m.d, m.d, kscale};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
   }
   stage_mark(c.s, mark + 4);
   // Delta W per chunk, fp32 exclusive prefix scan, W_i = W_down + S_i.
@@ -428,8 +443,10 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     g.tiles_m = cdiv(p->chunk, 128);
     g.tiles_n = cdiv(m.d, 256);
     g.b_group_rows = m.d;
+    CUtensorMap mo;
+    if (!make_out_map<OutT>(&mo, y, m.BT, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
   }
   stage_mark(c.s, mark + 6);
   return TTCD_OK;
@@ -608,9 +625,9 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
       return TTCD_ERR_CUDA;
     const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
     switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
     }
   }
   stage_mark(c.s, 2);
@@ -626,8 +643,10 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
         !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
       return TTCD_ERR_CUDA;
     const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
+    CUtensorMap mo;
+    if (!make_out_map<float>(&mo, h, 2 * m.BT, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiResidual<float, E> e{h, m.d, xin, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, g, e)));
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
   }
   stage_mark(c.s, 4);
   // u_P = RMSNorm(h_P; g_mlp), the gate/up operand.
