@@ -76,13 +76,15 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   }
 }
 
-// cs[t][i] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
+// cs[i][t] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
+// Frequency-major, so a warp reading one frequency for 32 consecutive tokens
+// reads 256 contiguous bytes.
 __global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double theta) {
   const int half = hd / 2;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(T) * half) return;
-  const int t = static_cast<int>(idx / half);
-  const int i = static_cast<int>(idx % half);
+  const int i = static_cast<int>(idx / T);
+  const int t = static_cast<int>(idx % T);
   const double inv = pow(theta, -2.0 * i / hd);
   double s, c;
   sincos(static_cast<double>(t) * inv, &s, &c);

@@ -104,8 +104,9 @@ __device__ __forceinline__ void load_x32(const float* src, float (&v)[32]) {
 // at slot j ^ (r & 7)), so a warp writing one chunk per row touches every bank
 // once per 8 rows.  One lane issues the store of the whole 32-row box.
 struct EpiStage {
-  uint8_t* buf;            // 2 x 4096 bytes, 1024-aligned; nullptr: direct stores
-  const CUtensorMap* map;  // output tensor map (box: 128 bytes x 32 rows)
+  uint8_t* buf;             // 2 x 4096 bytes, 1024-aligned; nullptr: direct stores
+  const CUtensorMap* map;   // first output tensor map (box: 128 bytes x 32 rows)
+  const CUtensorMap* map2;  // second output tensor map (same box), when an epilogue has two
   int toggle;
   __device__ bool on() const { return buf != nullptr; }
   // Before writing into the current buffer: its previous store has read it.
@@ -133,15 +134,16 @@ struct EpiStage {
       *reinterpret_cast<uint4*>(b + ((j ^ (r & 7)) << 4)) = w;
     }
   }
-  __device__ void flush(int x, int y) {
+  __device__ void flush(const CUtensorMap* m, int x, int y) {
     fence_async_smem();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) {
-      tma_store_2d(map, buf + toggle * 4096, x, y);
+      tma_store_2d(m, buf + toggle * 4096, x, y);
       bulk_commit();
     }
     toggle ^= 1;
   }
+  __device__ void flush(int x, int y) { flush(map, x, y); }
   __device__ void drain() {
     if (buf && (threadIdx.x & 31) == 0) bulk_wait<0>();
   }
@@ -152,8 +154,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
                    const __grid_constant__ CUtensorMap mapB1,
-                   const __grid_constant__ CUtensorMap mapOut, const GemmGeom geo, const Epi epi,
-                   const DevStatus st) {
+                   const __grid_constant__ CUtensorMap mapOut,
+                   const __grid_constant__ CUtensorMap mapOut2, const GemmGeom geo,
+                   const Epi epi, const DevStatus st) {
   constexpr bool STAGED = Epi::kStaged;
   constexpr int A_BYTES = GEMM_BM * 128;
   constexpr int B_BYTES = BN * 128;
@@ -179,7 +182,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    if (STAGED) tma_prefetch_map(&mapOut);
+    if (STAGED) {
+      tma_prefetch_map(&mapOut);
+      tma_prefetch_map(&mapOut2);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -275,16 +281,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
-    EpiStage stg{STAGED ? staging + (warp - 2) * 8192 : nullptr, &mapOut, 0};
+    EpiStage stg{STAGED ? staging + (warp - 2) * 8192 : nullptr, &mapOut, &mapOut2, 0};
     int j = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       TileCtx c;
       if (!geo.tile(t, c)) continue;
       const int ab = j & 1;
+      // per-row inputs of the epilogue are fetched while the tile is still computing
+      const float pre = epi.pre(c, r);
       if (!mbar_wait(&accf[ab], (j >> 1) & 1, st, abort)) break;
       tc_fence_after();
       epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r,
-                           stg);
+                           stg, pre);
       tc_fence_before();
       mbar_arrive(&acce[ab]);
       ++j;
@@ -312,27 +320,33 @@ template <class OutT>
 struct OutChunk {
   static constexpr int COLS = sizeof(OutT) == 4 ? 32 : 64;
 };
-__device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok, float* out_row, int col,
-                                     int y, const float (&v)[32], const float (&)[32]) {
+__device__ __forceinline__ void emit(EpiStage& stg, const CUtensorMap* m, bool staged, bool ok,
+                                     float* out_row, int col, int y, const float (&v)[32],
+                                     const float (&)[32]) {
   if (staged) {
     stg.acquire();
     stg.write_f32(threadIdx.x & 31, v);
-    stg.flush(col, y);
+    stg.flush(m, col, y);
   } else if (ok) {
     store_f32x32(out_row + col, v);
   }
 }
-__device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok,
+__device__ __forceinline__ void emit(EpiStage& stg, const CUtensorMap* m, bool staged, bool ok,
                                      __nv_bfloat16* out_row, int col, int y,
                                      const float (&lo)[32], const float (&hi)[32]) {
   if (staged) {
     stg.acquire();
     stg.write_bf16(threadIdx.x & 31, lo, hi);
-    stg.flush(col, y);
+    stg.flush(m, col, y);
   } else if (ok) {
     store_bf16x32(out_row + col, lo);
     store_bf16x32(out_row + col + 32, hi);
   }
+}
+template <class OutT>
+__device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok, OutT* out_row, int col,
+                                     int y, const float (&lo)[32], const float (&hi)[32]) {
+  emit(stg, stg.map, staged, ok, out_row, col, y, lo, hi);
 }
 
 // C[row, col] = OutT(acc * row_scale[row]) (row_scale nullable), columns < N.
@@ -344,13 +358,15 @@ struct EpiStore {
   long long ldo;
   int N;
   const float* row_scale;
+  __device__ float pre(const TileCtx& c, int r) const {
+    return (row_scale && r < c.valid_rows) ? __ldg(row_scale + c.row0 + r) : 1.f;
+  }
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float sc) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
     const int wrow = r & ~31;
     const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
-    const float sc = (row_scale && ok) ? __ldg(row_scale + row) : 1.f;
     constexpr int CW = OutChunk<OutT>::COLS;
 #pragma unroll 1
     for (int cc = 0; cc < BN; cc += CW) {
@@ -381,8 +397,9 @@ struct EpiResidual {
   long long ld_res;
   long long resid_rows;
   int N;
+  __device__ float pre(const TileCtx&, int) const { return 1.f; }
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
     const int wrow = r & ~31;
@@ -412,15 +429,106 @@ struct EpiResidual {
   }
 };
 
+// o_proj of both paths with the residual, feeding the MLP RMSNorm:
+//   h = x[row % BT] + acc                (rows [0, BT) teacher, [BT, 2BT) student)
+//   hg[row]       = h * g_mlp            (gate/up operand; stored through mapOut)
+//   h_S[row - BT] = h  for student rows  (fp32 residual of the output; mapOut2)
+//   ssq[tn][row]  = sum over this tile's columns of h^2  (fixed order)
+template <class E, class ResT>
+struct EpiOprojNorm {
+  static constexpr bool kStaged = true;
+  E* hg;
+  float* hS;
+  float* ssq;
+  const ResT* x;
+  const E* g;
+  long long BT;
+  int d;
+  __device__ float pre(const TileCtx&, int) const { return 1.f; }
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+    const long long wrow0 = c.row0 + (r & ~31);  // first row of this warp
+    const bool wvalid = stg.on() && (r & ~31) + 32 <= c.valid_rows;
+    const bool w_student = wrow0 >= BT;            // whole warp in the student half
+    const bool w_teacher = wrow0 + 32 <= BT;       // whole warp in the teacher half
+    const bool is_student = row >= BT;
+    const ResT* xrow = x + (row % BT) * d;
+    float* hs_row = is_student ? hS + (row - BT) * d : hS;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 64) {
+      const int col = c.tn * BN + cc;
+      if (col >= d) break;
+      float lo[32], hi[32], glo[32], ghi[32];
+      tmem_ld32f(taddr + cc, lo);
+      tmem_ld32f(taddr + cc + 32, hi);
+      if (ok) {
+        float t[32];
+        load_x32(xrow + col, t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) lo[i] += t[i];
+        load_x32(xrow + col + 32, t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hi[i] += t[i];
+      }
+      load_x32(g + col, glo);
+      load_x32(g + col + 32, ghi);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss += lo[i] * lo[i] + hi[i] * hi[i];
+      // fp32 student residual
+      if (wvalid && w_student) {
+        emit(stg, stg.map2, true, ok, hs_row, col, static_cast<int>(wrow0 - BT), lo, lo);
+        emit(stg, stg.map2, true, ok, hs_row, col + 32, static_cast<int>(wrow0 - BT), hi, hi);
+      } else if (!(wvalid && w_teacher) && ok && is_student) {
+        store_f32x32(hs_row + col, lo);
+        store_f32x32(hs_row + col + 32, hi);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        glo[i] *= lo[i];
+        ghi[i] *= hi[i];
+      }
+      E* hg_row = hg + row * d;
+      if constexpr (sizeof(E) == 2) {
+        emit(stg, stg.map, wvalid, ok, hg_row, col, static_cast<int>(wrow0), glo, ghi);
+      } else {
+        emit(stg, stg.map, wvalid, ok, hg_row, col, static_cast<int>(wrow0), glo, glo);
+        emit(stg, stg.map, wvalid, ok, hg_row, col + 32, static_cast<int>(wrow0), ghi, ghi);
+      }
+    }
+    if (ok) ssq[static_cast<long long>(c.tn) * (2 * BT) + row] = ss;
+  }
+};
+
 // Gate/up tile: accumulator columns [0, BN/2) are gate, [BN/2, BN) are up for
 // output columns tn*BN/2 + [0, BN/2).  Z = silu(gate) * up, fp32.
+// When `ssq` is set, the A operand was h * g and RMSNorm is applied here as the
+// row scale (sum_i ssq[i][row] / d_model + eps)^(-1/2) on gate and up alike
+// (u W^T = rstd * ((h * g) W^T)); otherwise A already holds u.
 struct EpiSwiGLU {
   static constexpr bool kStaged = true;
   float* out;
   long long ldo;
   int N;  // d_ff
+  const float* ssq;    // [n_part, rows] partial sums of h^2, nullable
+  int n_part;
+  long long ld_part;
+  float inv_d, eps;
+  __device__ float pre(const TileCtx& c, int r) const {
+    if (!ssq || r >= c.valid_rows) return 1.f;
+    float part[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)  // loads issued together; n_part <= 8 (d_model <= 2048)
+      part[i] = i < n_part ? __ldg(ssq + i * ld_part + c.row0 + r) : 0.f;
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sum += part[i];
+    return rsqrtf(sum * inv_d + eps);
+  }
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
     const int wrow = r & ~31;
@@ -433,63 +541,70 @@ struct EpiSwiGLU {
       tmem_ld32f(taddr + cc, g);
       tmem_ld32f(taddr + BN / 2 + cc, u);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
+      for (int i = 0; i < 32; ++i) {
+        const float gg = g[i] * rs;
+        g[i] = gg / (1.0f + __expf(-gg)) * (u[i] * rs);
+      }
       emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, g, u);
     }
   }
 };
 
-// QKV projection with rotary embedding on the query and key heads.
-// Column n of the accumulator is feature n of [q heads | k heads | v heads].
+// QKV projection with rotary embedding on the query and key heads, written to
+// one token-major tensor qkv [rows, (Hq + 2 Hkv) HD]: q heads, then k heads,
+// then v heads (column n of the accumulator is column n of qkv).  Each head's
+// HD columns are rotated in registers (pairs i, i + HD/2) and leave through the
+// staged TMA store in 64-column pieces.
 template <int HD>
 struct EpiQKVRope {
-  static constexpr bool kStaged = false;
-  __nv_bfloat16* q;
-  __nv_bfloat16* k;
-  __nv_bfloat16* v;
-  int Hq, Hkv, T;
-  const float2* rope_cs;  // [T][HD/2] (cos, sin)
+  static constexpr bool kStaged = true;
+  static constexpr int SPAN = HD >= 64 ? HD : 64;  // columns handled together
+  __nv_bfloat16* qkv;
+  int ld;         // (Hq + 2 Hkv) * HD
+  int n_rope;     // (Hq + Hkv) * HD: columns that get the rotation
+  int T;
+  const float2* rope_cs;  // [HD/2][T] (cos, sin), frequency-major
+  __device__ float pre(const TileCtx&, int) const { return 1.f; }
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&) const {
-    static_assert(BN % HD == 0, "column tile must hold whole heads");
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float) const {
+    static_assert(BN % SPAN == 0, "column tile must hold whole spans");
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const int wrow = r & ~31;
+    const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
     const int t = static_cast<int>(row % T);
-    const int n_heads = Hq + 2 * Hkv;
 #pragma unroll 1
-    for (int h0 = 0; h0 < BN; h0 += HD) {
-      const int head = (c.tn * BN + h0) / HD;
-      if (head >= n_heads) break;
-      float x[HD];
+    for (int h0 = 0; h0 < BN; h0 += SPAN) {
+      const int col0 = c.tn * BN + h0;
+      if (col0 >= ld) break;
+      float x[SPAN];
 #pragma unroll
-      for (int cc = 0; cc < HD; cc += 32) {
+      for (int cc = 0; cc < SPAN; cc += 32) {
         float tmp[32];
         tmem_ld32f(taddr + h0 + cc, tmp);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[cc + i] = tmp[i];
       }
-      if (!ok) continue;
-      __nv_bfloat16* dst;
-      if (head < Hq + Hkv) {
-        const float2* cs = rope_cs + static_cast<long long>(t) * (HD / 2);
+      if (col0 < n_rope) {
+        // SPAN covers SPAN/HD whole heads (all q/k: n_rope is a multiple of SPAN
+        // except when HD = 32 and the q/k/v boundary falls inside a span)
 #pragma unroll
-        for (int i = 0; i < HD / 2; ++i) {
-          const float2 e = __ldg(cs + i);
-          const float a = x[i], b = x[i + HD / 2];
-          x[i] = a * e.x - b * e.y;
-          x[i + HD / 2] = b * e.x + a * e.y;
+        for (int hh = 0; hh < SPAN / HD; ++hh) {
+          if (col0 + hh * HD >= n_rope) break;
+#pragma unroll
+          for (int i = 0; i < HD / 2; ++i) {
+            const float2 e = __ldg(rope_cs + static_cast<long long>(i) * T + t);
+            const float a = x[hh * HD + i], b = x[hh * HD + i + HD / 2];
+            x[hh * HD + i] = a * e.x - b * e.y;
+            x[hh * HD + i + HD / 2] = b * e.x + a * e.y;
+          }
         }
-        dst = head < Hq ? q + (row * Hq + head) * HD : k + (row * Hkv + (head - Hq)) * HD;
-      } else {
-        dst = v + (row * Hkv + (head - Hq - Hkv)) * HD;
       }
 #pragma unroll
-      for (int cc = 0; cc < HD; cc += 32) {
-        float tmp[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) tmp[i] = x[cc + i];
-        store_bf16x32(dst + cc, tmp);
-      }
+      for (int cc = 0; cc < SPAN; cc += 64)
+        emit(stg, staged, ok, qkv + row * ld, col0 + cc, c.row0 + wrow,
+             *reinterpret_cast<const float(*)[32]>(&x[cc]),
+             *reinterpret_cast<const float(*)[32]>(&x[cc + 32]));
     }
   }
 };

@@ -130,7 +130,7 @@ bool make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
 template <class E, int BN, int STAGES, bool DUAL, class Epi>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
                         const CUtensorMap& B1, const CUtensorMap* out_map, const GemmGeom& geo,
-                        const Epi& epi) {
+                        const Epi& epi, const CUtensorMap* out_map2 = nullptr) {
   const int total = geo.total();
   if (total <= 0) return TTCD_OK;
   if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
@@ -139,7 +139,8 @@ ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
   const int grid = total < c.sms ? total : c.sms;
-  kern<<<grid, GEMM_THREADS, smem, c.s>>>(A, B0, B1, out_map ? *out_map : A, geo, epi, c.st);
+  kern<<<grid, GEMM_THREADS, smem, c.s>>>(A, B0, B1, out_map ? *out_map : A,
+                                           out_map2 ? *out_map2 : A, geo, epi, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
 }
@@ -173,6 +174,8 @@ ttcd_status check_params(const ttcd_block_params* p) {
     return TTCD_ERR_INVALID_ARG;
   if (p->head_dim != 32 && p->head_dim != 64 && p->head_dim != 128) return TTCD_ERR_UNSUPPORTED;
   if (p->d_model % 64 != 0 || p->d_ff % 64 != 0) return TTCD_ERR_UNSUPPORTED;
+  if ((p->n_q_heads + 2 * p->n_kv_heads) * p->head_dim % 64 != 0) return TTCD_ERR_UNSUPPORTED;
+  if (p->d_model > 2048) return TTCD_ERR_UNSUPPORTED;  // RMSNorm partial sums: <= 8 tiles
   const long long BT = static_cast<long long>(p->B) * p->T;
   if (2 * BT >= (1ll << 31) || static_cast<long long>(p->d_ff) * p->d_model >= (1ll << 31))
     return TTCD_ERR_UNSUPPORTED;
@@ -185,11 +188,11 @@ struct Layout {
   size_t total;
 };
 enum Buf {
-  B_XN, B_Q, B_K, B_V, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ, B_KSCALE, B_R,
-  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_COUNT
+  B_XN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ, B_KSCALE, B_R,
+  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_COUNT
 };
-const char* kBufNames[B_COUNT] = {"xn", "q", "k", "v", "o", "h", "rope", "u", "Z", "Zs16", "D",
-                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt"};
+const char* kBufNames[B_COUNT] = {"xn", "qkv", "o", "h", "rope", "u", "Z", "Zs16", "D",
+                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt", "hssq"};
 
 struct Dims {
   long long BT, P;
@@ -218,11 +221,10 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
   const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
   if (block) {
     sz[B_XN] = m.BT * m.d * e;
-    sz[B_Q] = m.BT * m.Hq * m.hd * 2;
-    sz[B_K] = m.BT * m.Hkv * m.hd * 2;
-    sz[B_V] = m.BT * m.Hkv * m.hd * 2;
+    sz[B_QKV] = m.BT * m.dqkv * 2;
     sz[B_O] = 2 * m.BT * m.Hq * m.hd * e;
-    sz[B_H] = 2 * m.BT * m.d * 4;
+    sz[B_H] = m.BT * m.d * 4;                        // student residual stream, fp32
+    sz[B_HSSQ] = static_cast<size_t>(cdiv(m.d, 256)) * 2 * m.BT * 4;  // RMSNorm partial sums
     sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 8;
   }
   sz[B_U] = 2 * m.BT * m.d * e;
@@ -262,16 +264,18 @@ T* at(void* ws, const Layout& L, Buf b) {
   } while (0)
 
 // ------------------------------------------------------------------ attention
+// q rows have `ld_q` elements between tokens, k and v rows `ld_kv` (equal to
+// Hq*HD / Hkv*HD for separate tensors, or the qkv width for one packed tensor).
 template <int HD, class OutT>
 ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
                         OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv,
-                        int w_S, int w_T, float scale) {
+                        int w_S, int w_T, float scale, long long ld_q, long long ld_kv) {
   CUtensorMap mq, mk, mv;
   const long long BT = static_cast<long long>(B) * T;
   using bf = __nv_bfloat16;
-  if (!make_map<bf>(&mq, q, static_cast<uint64_t>(Hq) * HD, BT, static_cast<uint64_t>(Hq) * HD * 2, 64, 128) ||
-      !make_map<bf>(&mk, k, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128) ||
-      !make_map<bf>(&mv, v, static_cast<uint64_t>(Hkv) * HD, BT, static_cast<uint64_t>(Hkv) * HD * 2, 64, 128))
+  if (!make_map<bf>(&mq, q, static_cast<uint64_t>(Hq) * HD, BT, ld_q * 2, 64, 128) ||
+      !make_map<bf>(&mk, k, static_cast<uint64_t>(Hkv) * HD, BT, ld_kv * 2, 64, 128) ||
+      !make_map<bf>(&mv, v, static_cast<uint64_t>(Hkv) * HD, BT, ld_kv * 2, 64, 128))
     return TTCD_ERR_CUDA;
   AttnArgs<OutT> a;
   a.o_T = o_T;
@@ -301,23 +305,25 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
 template <class OutT>
 ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
                      OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv, int hd,
-                     int w_S, int w_T, float scale) {
+                     int w_S, int w_T, float scale, long long ld_q, long long ld_kv) {
   switch (hd) {
-    case 32: return launch_attn<32>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale);
-    case 64: return launch_attn<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale);
-    case 128: return launch_attn<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale);
+    case 32: return launch_attn<32>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
+    case 64: return launch_attn<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
+    case 128: return launch_attn<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
     default: return TTCD_ERR_UNSUPPORTED;
   }
 }
 
 // ------------------------------------------------------------------ fast-weight MLP body
 // u (operand type E, [2BT, d], teacher rows first) is already in the workspace.
+// With `hssq` set, u holds h * g_mlp and RMSNorm is finished as a row scale in
+// the gate/up epilogue from the partial sums of squares hssq [n_part, 2BT].
 template <class E, class OutT, class ResT>
 ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
                          const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
                          const E* conv_T, const E* conv_S, const float* beta,
                          const float* state_in, float* state_out, const ResT* h_S, OutT* y,
-                         int mark) {
+                         int mark, const float* hssq) {
   const Dims m = dims_of(p);
   E* u = at<E>(ws, L, B_U);
   float* Z = at<float>(ws, L, B_Z);
@@ -340,7 +346,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
       return TTCD_ERR_CUDA;
     CUtensorMap mo;
     if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
-    EpiSwiGLU e{Z, m.f, m.f};
+    EpiSwiGLU e{Z, m.f, m.f, hssq, cdiv(m.d, 256), 2 * m.BT, 1.0f / m.d, p->rms_eps};
     TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
   }
   stage_mark(c.s, mark + 1);
@@ -547,7 +553,8 @@ ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, v
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(hd));
   return run_attn<__nv_bfloat16>(c, q, k, v, static_cast<__nv_bfloat16*>(o_T),
                                  static_cast<__nv_bfloat16*>(o_S), lse_T, lse_S, B, T, Hq, Hkv,
-                                 hd, w_S, w_T, sc);
+                                 hd, w_S, w_T, sc, static_cast<long long>(Hq) * hd,
+                                 static_cast<long long>(Hkv) * hd);
 }
 
 ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,
@@ -579,14 +586,14 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
         c, p, L, workspace, static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up),
         static_cast<const bf*>(w->w_down), static_cast<const bf*>(w->w_proj),
         static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), beta, state_in,
-        state_out, static_cast<const bf*>(h_S), static_cast<bf*>(y), 0);
+        state_out, static_cast<const bf*>(h_S), static_cast<bf*>(y), 0, nullptr);
   }
   return run_mlp_core<float, float, float>(
       c, p, L, workspace, static_cast<const float*>(w->w_gate),
       static_cast<const float*>(w->w_up), static_cast<const float*>(w->w_down),
       static_cast<const float*>(w->w_proj), static_cast<const float*>(w->conv_T),
       static_cast<const float*>(w->conv_S), beta, state_in, state_out,
-      static_cast<const float*>(h_S), static_cast<float*>(y), 0);
+      static_cast<const float*>(h_S), static_cast<float*>(y), 0, nullptr);
 }
 
 }  // extern "C"
@@ -599,13 +606,12 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
                       void* out, void* ws, const Layout& L) {
   const Dims m = dims_of(p);
   E* xn = at<E>(ws, L, B_XN);
-  __nv_bfloat16* q = at<__nv_bfloat16>(ws, L, B_Q);
-  __nv_bfloat16* k = at<__nv_bfloat16>(ws, L, B_K);
-  __nv_bfloat16* v = at<__nv_bfloat16>(ws, L, B_V);
+  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
   E* o = at<E>(ws, L, B_O);
   float* h = at<float>(ws, L, B_H);
   float2* rope = at<float2>(ws, L, B_ROPE);
   E* u = at<E>(ws, L, B_U);
+  float* hssq = at<float>(ws, L, B_HSSQ);
   const E* xin = static_cast<const E*>(x);
 
   // Rotary table, input RMSNorm.
@@ -624,17 +630,22 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
     if (!map_rows<E>(&mA, xn, m.BT, m.d, 128) || !map_rows<E>(&mB, w->w_qkv, m.dqkv, m.d, 256))
       return TTCD_ERR_CUDA;
     const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
+    CUtensorMap mo;
+    if (!make_out_map<__nv_bfloat16>(&mo, qkv, m.BT, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
+    const int n_rope = (m.Hq + m.Hkv) * m.hd;
     switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<32>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<64>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
-      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, nullptr, g, EpiQKVRope<128>{q, k, v, m.Hq, m.Hkv, p->T, rope}))); break;
+      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
+      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
+      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
     }
   }
   stage_mark(c.s, 2);
   // Dual-window attention: o_T rows then o_S rows.
   const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
-  TTCD_TRY(run_attn<E>(c, q, k, v, o, o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq,
-                       m.Hkv, m.hd, p->w_S, p->w_T, sc));
+  TTCD_TRY(run_attn<E>(c, qkv, qkv + static_cast<long long>(m.Hq) * m.hd,
+                       qkv + static_cast<long long>(m.Hq + m.Hkv) * m.hd, o,
+                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq, m.Hkv, m.hd,
+                       p->w_S, p->w_T, sc, m.dqkv, m.dqkv));
   stage_mark(c.s, 3);
   // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
   {
@@ -643,25 +654,24 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
         !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
       return TTCD_ERR_CUDA;
     const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
-    CUtensorMap mo;
-    if (!make_out_map<float>(&mo, h, 2 * m.BT, m.d, m.d)) return TTCD_ERR_CUDA;
-    EpiResidual<float, E> e{h, m.d, xin, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
+    // h_P = x + o_P W_o^T; stores h * g_mlp (gate/up operand), the student
+    // h in fp32, and per-tile sums of h^2 for the MLP RMSNorm.
+    CUtensorMap mo, mo2;
+    if (!make_out_map<E>(&mo, u, 2 * m.BT, m.d, m.d) ||
+        !make_out_map<float>(&mo2, h, m.BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e, &mo2)));
   }
-  stage_mark(c.s, 4);
-  // u_P = RMSNorm(h_P; g_mlp), the gate/up operand.
-  rmsnorm_kernel<float, E, E><<<cdiv(2 * m.BT, 8), 256, 0, c.s>>>(
-      h, static_cast<const E*>(w->g_mlp), u, 2 * m.BT, m.d, p->rms_eps);
-  TTCD_CHECK_LAUNCH();
 
-  const float* h_S = h + m.BT * m.d;
+  const float* h_S = h;
   return run_mlp_core<E, E, float>(c, p, L, ws, static_cast<const E*>(w->w_gate),
                                    static_cast<const E*>(w->w_up),
                                    static_cast<const E*>(w->w_down),
                                    static_cast<const E*>(w->w_proj),
                                    static_cast<const E*>(w->conv_T),
                                    static_cast<const E*>(w->conv_S), beta, nullptr, state_out,
-                                   h_S, static_cast<E*>(out), 5);
+                                   h_S, static_cast<E*>(out), 4, hssq);
 }
 }  // namespace
 

@@ -60,10 +60,10 @@ typedef enum { TTCD_F32 = 0, TTCD_BF16 = 1 } ttcd_dtype;
 typedef struct {
   int B;              /* sequences in the batch                                */
   int T;              /* tokens per sequence                                   */
-  int d_model;        /* d                                                     */
+  int d_model;        /* d, a multiple of 64, at most 2048                     */
   int n_q_heads;      /* Hq                                                    */
   int n_kv_heads;     /* Hkv, Hq % Hkv == 0; query head h reads KV head h/(Hq/Hkv) */
-  int head_dim;       /* hd in {32, 64, 128}                                   */
+  int head_dim;       /* hd in {32, 64, 128}; (Hq + 2 Hkv) hd a multiple of 64 */
   int d_ff;           /* f                                                     */
   int w_S;            /* student window, 1 <= w_S <= w_T                       */
   int w_T;            /* teacher window                                        */
@@ -198,9 +198,12 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  * inspection after a call (same layout for ttcd_fastweight_mlp where named).
  * Names and layouts (row-major):
  *   (E = bf16 for TTCD_BF16, fp32 for TTCD_F32; q, k, v are always bf16)
- *   "xn"   E [B*T, d]             "q" bf16 [B*T, Hq*hd]   "k","v" bf16 [B*T, Hkv*hd]
+ *   "xn"   E [B*T, d]
+ *   "qkv"  bf16 [B*T, (Hq + 2 Hkv) hd]: q heads (rotated), k heads (rotated), v heads
  *   "o"    E [2, B*T, Hq*hd]      (o_T rows, then o_S rows)
- *   "h"    fp32 [2, B*T, d]       "u" E [2, B*T, d]
+ *   "h"    fp32 [B*T, d] (student residual h_S)
+ *   "u"    E [2, B*T, d] (block: h * g_mlp; the MLP RMSNorm's 1/rms is applied as a
+ *          row scale from "hssq" fp32 [ceil(d/256), 2*B*T] partial sums of h^2)
  *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f] (TTCD_BF16 only)
  *   "D"    E [P, f]               "Kp" E [P, f] (unnormalised keys)  "ssq" fp32 [f/64, P]
  *   "R"    E [P, d] (value residual times beta_t / ||Zbar_S[t]||)
@@ -234,9 +237,10 @@ ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream);
  * ttcd_set_stage_events: when n_events > 0, ttcd_block_forward records
  * events[k] (cudaEvent_t handles owned by the caller) on its stream at stage
  * boundary k: 0 start, 1 after the input RMSNorm, 2 after QKV+RoPE, 3 after
- * attention, 4 after o_proj, 5 after the MLP RMSNorm, 6 after gate/up+SwiGLU,
- * 7 after conv/residual/keys, 8 after M = W_down W_proj, 9 after R, 10 after
- * the chunk scan, 11 after the output GEMM.  ttcd_fastweight_mlp records
+ * attention, 4 after o_proj (which also carries the MLP RMSNorm statistics),
+ * 5 after gate/up+SwiGLU, 6 after conv/residual/keys, 7 after
+ * M = W_down W_proj, 8 after R, 9 after the chunk scan, 10 after the output
+ * GEMM.  ttcd_fastweight_mlp records
  * boundaries 0..6 of its own part (start, gate/up, conv, M, R, scan, output).
  * Boundaries at or beyond n_events are skipped; n_events = 0 disables.
  * Process-wide setting, not thread-safe.  At most 16 events.

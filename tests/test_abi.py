@@ -61,7 +61,7 @@ def test_workspace_sizes(lib):
 
 def test_workspace_offsets_are_ordered_and_aligned(lib):
     p = _params()
-    names = ["xn", "q", "k", "v", "o", "h", "u", "Z", "Zs16", "D", "Kp", "ssq", "R", "Wall"]
+    names = ["xn", "qkv", "o", "h", "u", "Z", "Zs16", "D", "Kp", "ssq", "R", "Wall"]
     offs = [ttcd.workspace_offset(p, n) for n in names]
     assert all(o % 1024 == 0 for o in offs)
     assert offs == sorted(offs)

@@ -44,14 +44,15 @@ def _stage_checks(ttcd, p, ws, ref, shape):
     view = lambda n, dt, sh: np64(ttcd.workspace_view(ws, p, n, dt, sh))
     bf, f32 = torch.bfloat16, torch.float32
     op = f32 if shape.dtype == "f32" else bf  # operand type of o, u, D, Kt, Rt, Wall
+    qkv = view("qkv", bf, (BT, (Hq + 2 * Hkv) * hd))
     checks = {
-        "q": (view("q", bf, (BT, Hq * hd)), ref["q"].reshape(BT, -1)),
-        "k": (view("k", bf, (BT, Hkv * hd)), ref["k"].reshape(BT, -1)),
-        "v": (view("v", bf, (BT, Hkv * hd)), ref["v"].reshape(BT, -1)),
+        "q": (qkv[:, :Hq * hd], ref["q"].reshape(BT, -1)),
+        "k": (qkv[:, Hq * hd:(Hq + Hkv) * hd], ref["k"].reshape(BT, -1)),
+        "v": (qkv[:, (Hq + Hkv) * hd:], ref["v"].reshape(BT, -1)),
         "o_T": (view("o", op, (2, BT, Hq * hd))[0], ref["o_T"].reshape(BT, -1)),
         "o_S": (view("o", op, (2, BT, Hq * hd))[1], ref["o_S"].reshape(BT, -1)),
-        "h_T": (view("h", f32, (2, BT, d))[0], ref["h_T"].reshape(BT, -1)),
-        "h_S": (view("h", f32, (2, BT, d))[1], ref["h_S"].reshape(BT, -1)),
+        "h_S": (view("h", f32, (BT, d)), ref["h_S"].reshape(BT, -1)),
+        "hg_T": (view("u", op, (2, BT, d))[0], ref["h_T"].reshape(BT, -1)),  # gains are 1
         "Z_T": (view("Z", f32, (2, BT, f))[0], ref["Z_T"].reshape(BT, -1)),
         "Z_S": (view("Z", f32, (2, BT, f))[1], ref["Z_S"].reshape(BT, -1)),
     }
