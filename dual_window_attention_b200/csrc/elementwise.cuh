@@ -212,6 +212,17 @@ __global__ void key_scale_kernel(const float* __restrict__ ssq_part, int n_part,
   kscale[p] = valid ? beta[static_cast<long long>(b) * T + t] * rsqrtf(ssq + eps) : 0.f;
 }
 
+// rstd[row] = (sum over tiles of ssq[tile][row] / d + eps)^(-1/2): the MLP
+// RMSNorm's row scale from the partial sums the o_proj epilogue wrote.
+__global__ void rms_rstd_kernel(const float* __restrict__ ssq, int n_part, long long rows,
+                                float inv_d, float eps, float* __restrict__ rstd) {
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  float sum = 0.f;
+  for (int i = 0; i < n_part; ++i) sum += ssq[i * rows + r];
+  rstd[r] = rsqrtf(sum * inv_d + eps);
+}
+
 template <class InT>
 __global__ void cast_to_bf16_kernel(const InT* __restrict__ in, __nv_bfloat16* __restrict__ out,
                                     long long n) {

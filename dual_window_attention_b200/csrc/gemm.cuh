@@ -504,28 +504,17 @@ struct EpiOprojNorm {
 
 // Gate/up tile: accumulator columns [0, BN/2) are gate, [BN/2, BN) are up for
 // output columns tn*BN/2 + [0, BN/2).  Z = silu(gate) * up, fp32.
-// When `ssq` is set, the A operand was h * g and RMSNorm is applied here as the
-// row scale (sum_i ssq[i][row] / d_model + eps)^(-1/2) on gate and up alike
-// (u W^T = rstd * ((h * g) W^T)); otherwise A already holds u.
+// When `rstd` is set, the A operand was h * g and RMSNorm is finished here as
+// the row scale rstd[row] on gate and up alike (u W^T = rstd * ((h * g) W^T));
+// otherwise A already holds u.
 struct EpiSwiGLU {
   static constexpr bool kStaged = true;
   float* out;
   long long ldo;
   int N;  // d_ff
-  const float* ssq;    // [n_part, rows] partial sums of h^2, nullable
-  int n_part;
-  long long ld_part;
-  float inv_d, eps;
+  const float* rstd;  // [rows], nullable
   __device__ float pre(const TileCtx& c, int r) const {
-    if (!ssq || r >= c.valid_rows) return 1.f;
-    float part[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)  // loads issued together; n_part <= 8 (d_model <= 2048)
-      part[i] = i < n_part ? __ldg(ssq + i * ld_part + c.row0 + r) : 0.f;
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sum += part[i];
-    return rsqrtf(sum * inv_d + eps);
+    return (rstd && r < c.valid_rows) ? __ldg(rstd + c.row0 + r) : 1.f;
   }
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
@@ -543,7 +532,7 @@ struct EpiSwiGLU {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float gg = g[i] * rs;
-        g[i] = gg / (1.0f + __expf(-gg)) * (u[i] * rs);
+        g[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (u[i] * rs);
       }
       emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, g, u);
     }

@@ -175,7 +175,6 @@ ttcd_status check_params(const ttcd_block_params* p) {
   if (p->head_dim != 32 && p->head_dim != 64 && p->head_dim != 128) return TTCD_ERR_UNSUPPORTED;
   if (p->d_model % 64 != 0 || p->d_ff % 64 != 0) return TTCD_ERR_UNSUPPORTED;
   if ((p->n_q_heads + 2 * p->n_kv_heads) * p->head_dim % 64 != 0) return TTCD_ERR_UNSUPPORTED;
-  if (p->d_model > 2048) return TTCD_ERR_UNSUPPORTED;  // RMSNorm partial sums: <= 8 tiles
   const long long BT = static_cast<long long>(p->B) * p->T;
   if (2 * BT >= (1ll << 31) || static_cast<long long>(p->d_ff) * p->d_model >= (1ll << 31))
     return TTCD_ERR_UNSUPPORTED;
@@ -189,10 +188,11 @@ struct Layout {
 };
 enum Buf {
   B_XN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ, B_KSCALE, B_R,
-  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_COUNT
+  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_RSTD, B_COUNT
 };
 const char* kBufNames[B_COUNT] = {"xn", "qkv", "o", "h", "rope", "u", "Z", "Zs16", "D",
-                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt", "hssq"};
+                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt", "hssq",
+                                  "rstd"};
 
 struct Dims {
   long long BT, P;
@@ -225,6 +225,7 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
     sz[B_O] = 2 * m.BT * m.Hq * m.hd * e;
     sz[B_H] = m.BT * m.d * 4;                        // student residual stream, fp32
     sz[B_HSSQ] = static_cast<size_t>(cdiv(m.d, 256)) * 2 * m.BT * 4;  // RMSNorm partial sums
+    sz[B_RSTD] = 2 * m.BT * 4;                                           // RMSNorm row scales
     sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 8;
   }
   sz[B_U] = 2 * m.BT * m.d * e;
@@ -317,7 +318,8 @@ ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, 
 // ------------------------------------------------------------------ fast-weight MLP body
 // u (operand type E, [2BT, d], teacher rows first) is already in the workspace.
 // With `hssq` set, u holds h * g_mlp and RMSNorm is finished as a row scale in
-// the gate/up epilogue from the partial sums of squares hssq [n_part, 2BT].
+// the gate/up epilogue, from the partial sums of squares hssq [n_part, 2BT]
+// reduced to one 1/rms per row first.
 template <class E, class OutT, class ResT>
 ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
                          const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
@@ -346,7 +348,14 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
       return TTCD_ERR_CUDA;
     CUtensorMap mo;
     if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
-    EpiSwiGLU e{Z, m.f, m.f, hssq, cdiv(m.d, 256), 2 * m.BT, 1.0f / m.d, p->rms_eps};
+    float* rstd = nullptr;
+    if (hssq) {
+      rstd = at<float>(ws, L, B_RSTD);
+      rms_rstd_kernel<<<cdiv(2 * m.BT, 256), 256, 0, c.s>>>(hssq, cdiv(m.d, 256), 2 * m.BT,
+                                                            1.0f / m.d, p->rms_eps, rstd);
+      TTCD_CHECK_LAUNCH();
+    }
+    EpiSwiGLU e{Z, m.f, m.f, rstd};
     TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
   }
   stage_mark(c.s, mark + 1);

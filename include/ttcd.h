@@ -60,7 +60,7 @@ typedef enum { TTCD_F32 = 0, TTCD_BF16 = 1 } ttcd_dtype;
 typedef struct {
   int B;              /* sequences in the batch                                */
   int T;              /* tokens per sequence                                   */
-  int d_model;        /* d, a multiple of 64, at most 2048                     */
+  int d_model;        /* d, a multiple of 64                                   */
   int n_q_heads;      /* Hq                                                    */
   int n_kv_heads;     /* Hkv, Hq % Hkv == 0; query head h reads KV head h/(Hq/Hkv) */
   int head_dim;       /* hd in {32, 64, 128}; (Hq + 2 Hkv) hd a multiple of 64 */
