@@ -5,16 +5,19 @@
 //   causal prefix scan over chunks; README "Model configuration"
 //   (ttt_force_grouped_scan: the fused scan path).
 //
-// One CTA owns a 128 x 128 tile (rows of d, columns of f) of one sequence's
-// d x f state.  It walks the chunks in order.  For chunk i the tensor cores
-// form Delta W_i = R[chunk i]^T . Kp[chunk i] (contraction over the chunk's
-// padded tokens; R [P, d] and Kp [P, f] are token-major, so both operands are
-// MN-major tiles: boxes of BK MN-elements x BK tokens, 128-byte swizzled) in
-// one of two TMEM accumulators, while the epilogue
-// warps fold the previous chunk into the fp32 running state S (a third TMEM
-// region) and emit W_{i+1} = bf16(W_down + S_{i+1}) for the output GEMM.
-// Chunk 0 reads W_0 = bf16(W_down + state_in).  The last state is written to
-// state_out in fp32.
+// One CTA owns a 128 x 192 tile (rows of d, columns of f) of one sequence's
+// d x f state and walks the chunks in order.  For chunk i the tensor cores form
+// Delta W_i = R[chunk i]^T . Kp[chunk i] (contraction over the chunk's padded
+// tokens) in one of two TMEM accumulators (2 x 192 columns), while eight
+// epilogue warps fold the previous chunk into the fp32 running state S, which
+// they keep in registers (each thread: one row, 96 columns), and emit
+// W_{i+1} = W_down + S_{i+1} for the output GEMM.  Chunk 0 reads
+// W_0 = W_down + state_in; the last state goes to state_out in fp32.  N = 192
+// (not 256) gives 128 tiles at the Qwen3 shape, so most SMs get one.
+// MN = true: R [P, d] and Kp [P, f] token-major, read as MN-major operands
+// (bf16, boxes of 64 MN-elements x 64 tokens).  MN = false: their transposes
+// Rt [d, P] and Kt [f, P], read as K-major operands (tf32).
+// Warps: 0 TMA, 1 TMEM + MMA, 2-3 idle, 4-11 epilogue (setmaxnreg 56 / 224).
 #pragma once
 #include "gemm.cuh"
 
@@ -30,22 +33,21 @@ struct ScanArgs {
   int tiles_m, tiles_n;
 };
 
-// MN = true: R [P, d] and Kp [P, f] token-major, read as MN-major operands
-// (bf16).  MN = false: their transposes Rt [d, P] and Kt [f, P], read as
-// K-major operands (used for tf32, whose operands stay K-major).
+constexpr int SCAN_BN = 192;
+constexpr int SCAN_THREADS = 384;
+
 template <class E, int STAGES, bool MN>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(SCAN_THREADS, 1)
     fastweight_scan_kernel(const __grid_constant__ CUtensorMap mapR,
                            const __grid_constant__ CUtensorMap mapK, const ScanArgs<E> a,
                            const DevStatus st) {
-  constexpr int BN = 128;
-  constexpr int BK = ElemTraits<E>::BK;          // tokens per k-block == MN elements per box
+  constexpr int BN = SCAN_BN;
+  constexpr int BK = ElemTraits<E>::BK;  // tokens per k-block == MN elements per box
   constexpr int BOX_BYTES = BK * BK * static_cast<int>(sizeof(E));
-  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;  // 16 KB each either way
+  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int KSTEP_BYTES = (32 / static_cast<int>(sizeof(E))) * 128;  // tokens per MMA x 128 B
   constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, MN, MN);
-  constexpr uint32_t COL_STATE = 256;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -64,12 +66,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int b = blockIdx.x / (a.tiles_n * a.tiles_m);
   const int m0 = tm * GEMM_BM, n0 = tn * BN;
   const int kpc = a.Cp / BK;  // k-blocks per chunk
-  const long long P = static_cast<long long>(gridDim.x / (a.tiles_n * a.tiles_m)) * a.Nc * a.Cp;
-  (void)P;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&accf[s], 1); mbar_init(&acce[s], 128); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&accf[s], 1); mbar_init(&acce[s], 256); }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -85,8 +85,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    if (warp == 0 && lane == 0) {
       int it = 0;
       bool ok = true;
       for (int i = 0; i < a.Nc && ok; ++i) {
@@ -112,9 +113,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       volatile int no_abort = 0;
       for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
         mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       int it = 0;
       bool ok = true;
       for (int i = 0; i < a.Nc && ok; ++i) {
@@ -144,72 +143,71 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_wait(drain, 0, st, &no_abort);
     }
   } else {
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const int row = m0 + r;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    const int q = warp & 3;              // TMEM lane quarter
+    const int half = (warp - 4) >> 2;    // column half of the tile
+    const int row = m0 + q * 32 + lane;
     const bool row_ok = row < a.d;
-    const uint32_t laddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    constexpr int HC = SCAN_BN / 2;     // state columns per thread
+    const int c0 = n0 + half * HC;       // first state column of this thread
+    const uint32_t laddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * HC;
     const long long dfs = static_cast<long long>(a.d) * a.f;
-    // S_0 = state_in (or 0); W_0 = bf16(W_down + S_0).
-#pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
-      const int col = n0 + cc;
-      float s[32];
+    const E* wrow = a.w_down + static_cast<long long>(row) * a.f;
+    float S[HC];
+    // S_0 = state_in (or 0); W_0 = W_down + S_0.
+#pragma unroll
+    for (int cc = 0; cc < HC; cc += 32) {
+      const int col = c0 + cc;
+      float s32[32];
       if (row_ok && col < a.f && a.state_in) {
-        load_x32(a.state_in + b * dfs + static_cast<long long>(row) * a.f + col, s);
+        load_x32(a.state_in + b * dfs + static_cast<long long>(row) * a.f + col, s32);
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[e] = 0.f;
+        for (int e = 0; e < 32; ++e) s32[e] = 0.f;
       }
-      uint32_t u[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(s[e]);
-      tmem_st32(laddr + COL_STATE + cc, u);
+      for (int e = 0; e < 32; ++e) S[cc + e] = s32[e];
       if (row_ok && col < a.f) {
         float w[32];
-        load_x32(a.w_down + static_cast<long long>(row) * a.f + col, w);
+        load_x32(wrow + col, w);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] += s[e];
+        for (int e = 0; e < 32; ++e) w[e] += s32[e];
         store_x32(a.w_all + (static_cast<long long>(b) * a.Nc) * dfs +
                       static_cast<long long>(row) * a.f + col, w);
       }
     }
-    tmem_st_wait();
     for (int i = 0; i < a.Nc; ++i) {
       const int ab = i & 1;
       if (!mbar_wait(&accf[ab], (i >> 1) & 1, st, abort)) break;
       tc_fence_after();
       const bool last = i + 1 == a.Nc;
-#pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
-        const int col = n0 + cc;
-        uint32_t dw[32], sv[32];
-        tmem_ld32(laddr + ab * BN + cc, dw);
-        tmem_ld32(laddr + COL_STATE + cc, sv);
-        tmem_ld_wait();
-        float s[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(sv[e]) + __uint_as_float(dw[e]);
-          sv[e] = __float_as_uint(s[e]);
-        }
-        tmem_st32(laddr + COL_STATE + cc, sv);
-        if (row_ok && col < a.f) {
-          if (!last) {
-            float w[32];
-            load_x32(a.w_down + static_cast<long long>(row) * a.f + col, w);
+      for (int cc = 0; cc < HC; cc += 32) {
+        float dw[32];
+        tmem_ld32f(laddr + ab * BN + cc, dw);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] += s[e];
-            store_x32(a.w_all + (static_cast<long long>(b) * a.Nc + i + 1) * dfs +
-                          static_cast<long long>(row) * a.f + col, w);
-          } else if (a.state_out) {
-            store_f32x32(a.state_out + b * dfs + static_cast<long long>(row) * a.f + col, s);
-          }
-        }
+        for (int e = 0; e < 32; ++e) S[cc + e] += dw[e];
       }
-      tmem_st_wait();
+      // The accumulator is free as soon as it has been read.
       tc_fence_before();
       mbar_arrive(&acce[ab]);
+#pragma unroll
+      for (int cc = 0; cc < HC; cc += 32) {
+        const int col = c0 + cc;
+        if (!row_ok || col >= a.f) continue;
+        float v[32];
+        if (!last) {
+          load_x32(wrow + col, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] += S[cc + e];
+          store_x32(a.w_all + (static_cast<long long>(b) * a.Nc + i + 1) * dfs +
+                        static_cast<long long>(row) * a.f + col, v);
+        } else if (a.state_out) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = S[cc + e];
+          store_f32x32(a.state_out + b * dfs + static_cast<long long>(row) * a.f + col, v);
+        }
+      }
     }
   }
   __syncthreads();

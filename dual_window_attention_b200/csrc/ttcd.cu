@@ -419,7 +419,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
       transpose_kernel<E, E><<<dim3(cdiv(m.f, 32), cdiv(m.P, 32)), tb, 0, c.s>>>(Kp, Kt, static_cast<int>(m.P), m.f);
       TTCD_CHECK_LAUNCH();
       if (!make_map<E>(&mR, Rt, m.P, m.d, m.P * sizeof(E), BK, 128) ||
-          !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), BK, 128))
+          !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), BK, SCAN_BN))
         return TTCD_ERR_CUDA;
     }
     ScanArgs<E> a;
@@ -432,13 +432,13 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     a.state_out = state_out;
     a.w_all = Wall;
     a.tiles_m = cdiv(m.d, 128);
-    a.tiles_n = cdiv(m.f, 128);
-    constexpr int STAGES = 6;
-    constexpr int smem = gemm_smem_bytes<128, STAGES>();
+    a.tiles_n = cdiv(m.f, SCAN_BN);
+    constexpr int STAGES = 4;
+    constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
     auto kern = fastweight_scan_kernel<E, STAGES, MN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
-    kern<<<p->B * a.tiles_m * a.tiles_n, GEMM_THREADS, smem, c.s>>>(mR, mK, a, c.st);
+    kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
     TTCD_CHECK_LAUNCH();
   }
   stage_mark(c.s, mark + 5);
