@@ -291,53 +291,79 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_wait(&k_full[j % ATT_KS], (j / ATT_KS) & 1, st, &no_abort);
       for (int j = max(0, issued_v - ATT_VS); j < issued_v; ++j)
         mbar_wait(&v_full[j % ATT_VS], (j / ATT_VS) & 1, st, &no_abort);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
-      const uint32_t sq[2] = {smem_u32(smem + Cfg::QA_OFF), smem_u32(smem + Cfg::QB_OFF)};
+      // The whole warp walks the loop and one elected lane issues: the MMA
+      // queue holds only a few instructions, so the issuer must not spend its
+      // time rebuilding operand words between groups.  Descriptor low words
+      // (start address, LBO) advance by (offset >> 4); the high words are
+      // constants.
+      constexpr uint32_t HI = sdesc_hi_sw128(1024);
+      const uint32_t q_lo[2] = {sdesc_lo(smem_u32(smem + Cfg::QA_OFF), 16),
+                                sdesc_lo(smem_u32(smem + Cfg::QB_OFF), 16)};
+      const uint32_t k_lo0 = sdesc_lo(smem_u32(smem + Cfg::K_OFF), 16);
+      const uint32_t v_lo0 = sdesc_lo(smem_u32(smem + Cfg::V_OFF), ATT_BM * 128);
       const int nh = hasB ? 2 : 1;
       auto issue_qk = [&](int h, int v) {
-        const uint32_t sk = smem_u32(smem + Cfg::K_OFF + (v % ATT_KS) * Cfg::TILE_BYTES);
+        const uint32_t k_lo = k_lo0 + (((v % ATT_KS) * Cfg::TILE_BYTES) >> 4);
+        const uint32_t qh = h ? q_lo[1] : q_lo[0];
+        const uint32_t d = tmem + h * 128;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (ATT_BM * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + h * 128, sdesc_sw128(sq[h] + off, 16, 1024),
-                      sdesc_sw128(sk + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * (ATT_BM * 128) + (kk & 3) * 32) >> 4;
+            mma_bf16_ss_lh(d, qh + off, HI, k_lo + off, HI, IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_full[h]);
         }
-        mma_commit(&s_full[h]);
+        __syncwarp();
       };
       auto issue_pv = [&](int h, int v) {
-        const uint32_t sv = smem_u32(smem + Cfg::V_OFF + (v % ATT_VS) * Cfg::TILE_BYTES);
+        const uint32_t v_lo = v_lo0 + (((v % ATT_VS) * Cfg::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + 256 + h * 128, pa = tmem + h * 128;
+        const uint32_t acc0 = v > 0 ? 1u : 0u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; ++kk)
-          mma_bf16_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8,
-                      sdesc_sw128(sv + kk * 2048, ATT_BM * 128, 1024), IDESC_PV,
-                      (v > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&o_done[h]);
+          for (int kk = 0; kk < ATT_BN / 16; ++kk)
+            mma_bf16_ts_lh(d, pa + kk * 8, v_lo + ((kk * 2048) >> 4), HI, IDESC_PV,
+                           kk > 0 ? 1u : acc0);
+          mma_commit(&o_done[h]);
+        }
+        __syncwarp();
       };
-      bool ok = mbar_wait(q_full, 0, st, abort) && mbar_wait(&k_full[0], 0, st, abort);
+      // every lane waits; a wait that gave up in any lane ends the loop in all
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
+      };
+      bool ok = wait(q_full, 0) && wait(&k_full[0], 0);
       if (ok) {
         tc_fence_after();
         for (int h = 0; h < nh; ++h) issue_qk(h, 0);
-        mma_commit(&k_empty[0]);
+        if (elect_one()) mma_commit(&k_empty[0]);
+        __syncwarp();
       }
       for (int v = 0; v < vis.nv && ok; ++v) {
         const bool more = v + 1 < vis.nv;
-        if (!mbar_wait(&v_full[v % ATT_VS], (v / ATT_VS) & 1, st, abort)) { ok = false; break; }
-        if (more && !mbar_wait(&k_full[(v + 1) % ATT_KS], ((v + 1) / ATT_KS) & 1, st, abort)) {
+        if (!wait(&v_full[v % ATT_VS], (v / ATT_VS) & 1)) { ok = false; break; }
+        if (more && !wait(&k_full[(v + 1) % ATT_KS], ((v + 1) / ATT_KS) & 1)) {
           ok = false;
           break;
         }
         for (int h = 0; h < nh; ++h) {
-          if (!mbar_wait(&p_full[h], v & 1, st, abort)) { ok = false; break; }
+          if (!wait(&p_full[h], v & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(h, v);
           if (more) issue_qk(h, v + 1);
         }
         if (!ok) break;
-        if (more) mma_commit(&k_empty[(v + 1) % ATT_KS]);
-        mma_commit(&v_empty[v % ATT_VS]);
+        if (elect_one()) {
+          if (more) mma_commit(&k_empty[(v + 1) % ATT_KS]);
+          mma_commit(&v_empty[v % ATT_VS]);
+        }
+        __syncwarp();
       }
-      mma_commit(drain);
+      if (elect_one()) mma_commit(drain);
+      __syncwarp();
       volatile int no_abort = 0;
       mbar_wait(drain, 0, st, &no_abort);
     }
@@ -381,10 +407,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
       }
-      float mx = fmax3(s[0], s[1], s[2]);
+      // row maximum as four independent chains (short dependency latency)
+      float mx4[4];
 #pragma unroll
-      for (int c = 3; c < 127; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
-      mx = fmaxf(mx, s[127]);
+      for (int q = 0; q < 4; ++q) {
+        float m = fmax3(s[32 * q], s[32 * q + 1], s[32 * q + 2]);
+#pragma unroll
+        for (int c = 3; c < 31; c += 2) m = fmax3(m, s[32 * q + c], s[32 * q + c + 1]);
+        mx4[q] = fmaxf(m, s[32 * q + 31]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_tile = mx * sl2;
       if (v == 0) {
         m_ref = m_tile;
@@ -401,21 +433,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // exponentials, row sum, bf16 pack
       const uint64_t sc2 = f2pack(sl2, sl2);
       const uint64_t nm2 = f2pack(-m_ref, -m_ref);
-      uint64_t acc = f2pack(0.f, 0.f);
+      uint64_t acc4[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f),
+                          f2pack(0.f, 0.f)};
       uint32_t P[64];
       if (unmasked) {
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           uint64_t x = fma2(f2pack(s[c], s[c + 1]), sc2, nm2);
           uint64_t e;
-          if ((c & 14) == 14) {  // one pair in eight on the FMA pipe
+          if (((c >> 1) & 3) == 3) {  // one pair in four on the FMA pipe
             e = exp2_poly2(x);
           } else {
             float x0, x1;
             f2unpack(x, x0, x1);
             e = f2pack(ex2_approx(x0), ex2_approx(x1));
           }
-          acc = add2(acc, e);
+          acc4[(c >> 1) & 3] = add2(acc4[(c >> 1) & 3], e);
           float e0, e1;
           f2unpack(e, e0, e1);
           P[c >> 1] = pack_bf16x2(e0, e1);
@@ -427,12 +460,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           float x0, x1;
           f2unpack(x, x0, x1);
           const uint64_t e = f2pack(ex2_approx(x0), ex2_approx(x1));
-          acc = add2(acc, e);
+          acc4[(c >> 1) & 3] = add2(acc4[(c >> 1) & 3], e);
           float e0, e1;
           f2unpack(e, e0, e1);
           P[c >> 1] = pack_bf16x2(e0, e1);
         }
       }
+      const uint64_t acc = add2(add2(acc4[0], acc4[1]), add2(acc4[2], acc4[3]));
       float a0, a1;
       f2unpack(acc, a0, a1);
       l += a0 + a1;

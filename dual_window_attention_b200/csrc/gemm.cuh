@@ -243,40 +243,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      int it = 0, j = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        TileCtx c;
-        if (!geo.tile(t, c)) continue;
-        const int ab = j & 1;
-        if (!mbar_wait(&acce[ab], ((j >> 1) & 1) ^ 1, st, abort)) break;
+    // ------------------------------------------------------------------ MMA issuer
+    // The whole warp walks the loop (operand words stay warp-uniform) and one
+    // elected lane issues; descriptor low words advance by (byte offset >> 4).
+    constexpr uint32_t HI = sdesc_hi_sw128(1024);
+    const uint32_t lo0 = sdesc_lo(smem_u32(smem), 16);
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
+    };
+    int it = 0, j = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      TileCtx c;
+      if (!geo.tile(t, c)) continue;
+      const int ab = j & 1;
+      if (!wait(&acce[ab], ((j >> 1) & 1) ^ 1)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + ab * BN;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!wait(&full[s], (it / STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * BN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, st, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+        const uint32_t a_lo = lo0 + ((s * STAGE_BYTES) >> 4);
+        const uint32_t b_lo = a_lo + (A_BYTES >> 4);
+        if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {  // 4 MMAs of 32 bytes of K per 128-byte row
-            const uint64_t da = sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t db = sdesc_sw128(sb + k * 32, 16, 1024);
-            mma_ss<E>(d_tmem, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < 4; ++k)  // 4 MMAs of 32 bytes of K per 128-byte row
+            mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + 2 * k, HI, IDESC,
+                         (kb | k) != 0 ? 1u : 0u);
           mma_commit(&empty[s]);
         }
-        if (!ok) break;
-        mma_commit(&accf[ab]);
-        ++j;
+        __syncwarp();
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      mma_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, st, &no_abort);
+      if (!ok) break;
+      if (elect_one()) mma_commit(&accf[ab]);
+      __syncwarp();
+      ++j;
     }
+    // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
+    if (elect_one()) mma_commit(drain);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(drain, 0, st, &no_abort);
   } else {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access

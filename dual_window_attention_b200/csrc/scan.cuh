@@ -113,32 +113,42 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       volatile int no_abort = 0;
       for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
         mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
+      // MMA issuer: the whole warp walks the loop, one elected lane issues.
+      constexpr uint32_t HI = sdesc_hi_sw128(1024);
+      const uint32_t lo0 = sdesc_lo(smem_u32(smem), MN ? BOX_BYTES : 16);
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
+      };
       int it = 0;
       bool ok = true;
       for (int i = 0; i < a.Nc && ok; ++i) {
         const int ab = i & 1;
-        if (!mbar_wait(&acce[ab], ((i >> 1) & 1) ^ 1, st, abort)) break;
+        if (!wait(&acce[ab], ((i >> 1) & 1) ^ 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < kpc; ++kb, ++it) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, st, abort)) { ok = false; break; }
+          if (!wait(&full[s], (it / STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+          const uint32_t a_lo = lo0 + ((s * STAGE_BYTES) >> 4);
+          const uint32_t b_lo = a_lo + (A_BYTES >> 4);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t da = MN ? sdesc_sw128(sa + k * KSTEP_BYTES, BOX_BYTES, 1024)
-                                   : sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t db = MN ? sdesc_sw128(sb + k * KSTEP_BYTES, BOX_BYTES, 1024)
-                                   : sdesc_sw128(sb + k * 32, 16, 1024);
-            mma_ss<E>(tmem + ab * BN, da, db, IDESC, (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t off = (MN ? k * KSTEP_BYTES : k * 32) >> 4;
+              mma_ss_lh<E>(tmem + ab * BN, a_lo + off, HI, b_lo + off, HI, IDESC,
+                           (kb | k) != 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
           }
-          mma_commit(&empty[s]);
+          __syncwarp();
         }
         if (!ok) break;
-        mma_commit(&accf[ab]);
+        if (elect_one()) mma_commit(&accf[ab]);
+        __syncwarp();
       }
-      mma_commit(drain);
+      if (elect_one()) mma_commit(drain);
+      __syncwarp();
       volatile int no_abort = 0;
       mbar_wait(drain, 0, st, &no_abort);
     }
