@@ -13,8 +13,10 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -43,6 +45,30 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "dual_window_attn_T16384_ncu.md")
+ATTN_SOURCES = [os.path.join(ROOT, "dual_window_attention_b200", "csrc", n)
+                for n in ("attention.cuh", "ptx.cuh")]
+
+
+def recorded_attention_traffic(T: int):
+    """DRAM bytes (read + write) per attention launch at T tokens, from the
+    committed ncu summary of the 512/8192-window kernel, scaled by T (inputs,
+    outputs and the K/V stream all grow linearly in T).  None once the kernel
+    sources differ from the ones that were profiled."""
+    try:
+        text = open(ATTN_PROFILE).read()
+        digests = "".join(hashlib.sha256(open(f, "rb").read()).hexdigest() for f in ATTN_SOURCES)
+    except OSError:
+        return None
+    m_bytes = re.search(r"traffic_bytes_per_launch_T(\d+): (\d+)", text)
+    m_hash = re.search(r"kernel_sources_sha256_16: ([0-9a-f]+)", text)
+    if not m_bytes or not m_hash:
+        return None
+    if hashlib.sha256(digests.encode()).hexdigest()[:16] != m_hash.group(1):
+        return None
+    return float(m_bytes.group(2)) * T / int(m_bytes.group(1))
 
 
 def attention_flops(shape) -> float:
@@ -308,7 +334,8 @@ def run_ours(args, world, rank, local):
             "roofline": {"kernel": "dual_window_attn_kernel<128>", "bound": "tensor",
                          "achieved": att["achieved"], "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": att["frac"],
-                         "traffic": args.attn_traffic_bytes,
+                         "traffic": (args.attn_traffic_bytes if args.attn_traffic_bytes
+                                     is not None else recorded_attention_traffic(shape.T)),
                          "peak_source": f"{peak_kind} bf16_tflops_sustained",
                          "flops_per_launch": attention_flops(shape)},
             "stages": stages,
@@ -380,7 +407,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=2048)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
     ap.add_argument("--mode", choices=["block", "attn"], default="block",
                     help="block: the whole IP-TTCD block (default); attn: attention alone")
