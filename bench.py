@@ -400,6 +400,60 @@ def run_attention(args, world, rank, local):
                              "flops_per_launch": fl}}), flush=True)
 
 
+def run_stack(args, world, rank, local):
+    """The 28-layer stack of Qwen3-0.6B-shaped blocks, end-to-end prefill tokens/s
+    (B 1 x T 65536 by default, or --B 4 --T 16384): every layer one ttcd_block_forward
+    call on its own weights, one shared workspace."""
+    import dual_window_attention_b200 as ttcd
+    from ttcd_workloads import QWEN3_STACK_B1, QWEN3_STACK_B4
+    ttcd.load_library()
+    base = QWEN3_STACK_B4 if (args.B, args.T) == (4, 16384) else QWEN3_STACK_B1
+    shape = base if (args.B, args.T) == (base.B, base.T) else base.with_(
+        name=f"qwen3_0.6b_stack28_B{args.B}_T{args.T}", B=args.B, T=args.T)
+    dev = torch.device("cuda", local)
+    inp = make_block_inputs(shape, seed=0)
+    x = inp["x"].to(dev)
+    layers = [{k: v.to(dev) for k, v in lw.items()} for lw in inp["layers"]]
+    p = ttcd.BlockParams.from_shape(shape)
+    ws = ttcd.alloc_workspace(ttcd.block_forward_workspace_size(p), dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ttcd.block_stack_forward(x, layers, p, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    barrier(world, local)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = ttcd.kernel_launch_count()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    launches = ttcd.kernel_launch_count() - launches0
+    barrier(world, local)
+    ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    flops = shape.n_layers * sum(a for b, a in stage_costs(shape) if b == "tensor")
+    if rank == 0:
+        print(json.dumps({
+            "metric": "IP-TTCD 28-layer stack prefill tokens/s (Qwen3-0.6B shape)",
+            "value": shape.B * shape.T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": workload_config(shape, {"n_layers": shape.n_layers,
+                                              "parallelism": f"replicas{world}"}),
+            "tflops_per_s": flops / (ms / 1e3) / 1e12,
+            "gpu_launches": launches,
+            "clocks": clk.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -409,12 +463,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
-    ap.add_argument("--mode", choices=["block", "attn"], default="block",
-                    help="block: the whole IP-TTCD block (default); attn: attention alone")
+    ap.add_argument("--mode", choices=["block", "attn", "stack"], default="block",
+                    help="block: the whole IP-TTCD block (default); attn: attention alone; "
+                         "stack: 28 blocks end to end")
     ap.add_argument("--T", type=int, default=65536,
                     help="tokens per sequence (65536 is the benchmark workload; smaller values "
                          "are for profiling)")
-    ap.add_argument("--B", type=int, default=1, help="--mode attn: sequences")
+    ap.add_argument("--B", type=int, default=1, help="--mode attn / stack: sequences")
     ap.add_argument("--windows", default="512/8192",
                     help="--mode attn: comma-separated w_S/w_T pairs")
     ap.add_argument("--attn-traffic-bytes", type=float, default=None,
@@ -426,6 +481,8 @@ def main():
             run_reference(args, world, rank)
         elif args.mode == "attn":
             run_attention(args, world, rank, local)
+        elif args.mode == "stack":
+            run_stack(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

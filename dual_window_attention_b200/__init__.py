@@ -235,6 +235,31 @@ def block_forward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, out
     return out, st_t, workspace
 
 
+def block_stack_forward(x, layers, p: BlockParams, workspace: Optional[torch.Tensor] = None,
+                        stream=None, on_layer=None) -> torch.Tensor:
+    """A stack of IP-TTCD blocks: layer l's output is layer l+1's input.
+
+    ``layers`` is a list of weight dicts (the keys block_forward takes plus each
+    layer's per-token ``beta``).  One workspace serves every layer and two
+    activation buffers alternate, so nothing is allocated per layer.
+    ``on_layer(l, out)``, if given, sees each layer's output before the buffer is
+    reused.  Returns the last layer's output (a fresh tensor, not ``x``)."""
+    need = block_forward_workspace_size(p)
+    if need == 0:
+        raise TTCDError(ERR_INVALID_ARG, "ttcd_block_forward_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    bufs = (torch.empty_like(x), torch.empty_like(x))
+    cur = x
+    for l, w in enumerate(layers):
+        out = bufs[l & 1]
+        block_forward(cur, w["beta"], w, p, out=out, workspace=workspace, stream=stream)
+        if on_layer is not None:
+            on_layer(l, out)
+        cur = out
+    return cur
+
+
 def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams, h_S=None,
                    state_in=None, state_out: bool = False, y=None,
                    workspace: Optional[torch.Tensor] = None, stream=None):

@@ -195,6 +195,20 @@ def windowed_attention_bruteforce(q, k, v, window: int, scale: float):
     return o, lse
 
 
+def windowed_attention_row(q, k, v, window: int, scale: float, b: int, t: int, h: int):
+    """One output row of the windowed attention: query (b, t, h) against keys
+    j in [max(0, t-window+1), t] of KV head h // (Hq/Hkv) (readings R1, R11).
+    For sampled checks of long sequences.  Returns (o[b, t, h], lse[b, h, t])."""
+    G = q.shape[2] // k.shape[2]
+    j0 = max(0, t - window + 1)
+    kk = np.asarray(k[b, j0:t + 1, h // G], np.float64)
+    vv = np.asarray(v[b, j0:t + 1, h // G], np.float64)
+    s = scale * (kk @ np.asarray(q[b, t, h], np.float64))
+    m = s.max()
+    e = np.exp(s - m)
+    return (e[:, None] * vv).sum(0) / e.sum(), m + np.log(e.sum())
+
+
 def dual_window_attention(q, k, v, w_S: int, w_T: int, scale: float):
     """Teacher (w_T) and student (w_S) sliding-window outputs over the same Q/K/V.
 

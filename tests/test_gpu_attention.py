@@ -74,30 +74,59 @@ def test_mask_probe_one_hot_value_bit_exact(ttcd, j):
         np.testing.assert_array_equal(seen, (j <= t) & (j >= t - w + 1))
 
 
-def test_full_size_sampled_rows(ttcd):
-    """T = 65536, 16/8 heads, hd 128, w_S 512, w_T 8192: sampled rows vs the oracle."""
-    B, T, Hq, Hkv, hd, wS, wT = 1, 65536, 16, 8, 128, 512, 8192
-    q, k, v = make_attention_inputs(B, T, Hq, Hkv, hd, seed=0)
-    o_T, o_S, _, _ = ttcd.dual_window_attn(q.cuda(), k.cuda(), v.cuda(), wS, wT)
+@pytest.fixture(scope="module")
+def sweep_inputs():
+    """Q, K, V ~ N(0, 1) at the Qwen3-0.6B head layout, T = 65536 (the attention sweep)."""
+    from ttcd_workloads import ATTN_SWEEP_T
+    q, k, v = make_attention_inputs(1, ATTN_SWEEP_T, 16, 8, 128, seed=0)
+    return (q, k, v), (q.cuda(), k.cuda(), v.cuda()), (np64(q), np64(k), np64(v))
+
+
+def _sampled_rows_error(o_dev, qkv64, w, rows, rng):
+    """max|d| / max|ref| of sampled rows (two random heads per row) against the oracle's
+    row-at-a-time windowed attention."""
+    qn, kn, vn = qkv64
+    got = np64(o_dev)
+    Hq, hd = qn.shape[2], qn.shape[3]
+    err = refmax = 0.0
+    for t in rows:
+        for h in rng.choice(Hq, 2, replace=False):
+            ref, _ = orc.windowed_attention_row(qn, kn, vn, w, hd ** -0.5, 0, int(t), int(h))
+            err = max(err, float(np.max(np.abs(got[0, t, h] - ref))))
+            refmax = max(refmax, float(np.max(np.abs(ref))))
+    return err / refmax
+
+
+def _rows(T, w_S, w_T, rng):
+    edges = [0, 1, 127, 128, w_S - 1, w_S, w_T - 1, w_T, T - 1]
+    return np.unique(np.concatenate([[e for e in edges if 0 <= e < T], rng.integers(0, T, 24)]))
+
+
+def test_full_size_sampled_rows(ttcd, sweep_inputs):
+    """T = 65536, 16/8 heads, hd 128, w_S 512, w_T 8192 (the block's windows): sampled
+    rows of both outputs against the oracle."""
+    _, (q, k, v), qkv64 = sweep_inputs
+    o_T, o_S, _, _ = ttcd.dual_window_attn(q, k, v, 512, 8192)
     torch.cuda.synchronize()
     assert ttcd.get_device_error()[0] == ttcd.OK
     rng = np.random.default_rng(0)
-    rows = np.concatenate([[0, 1, 127, 128, 511, 512, 8191, 8192, 65535],
-                           rng.integers(0, T, 40)])
-    qn, kn, vn = np64(q), np64(k), np64(v)
-    oT, oS = np64(o_T), np64(o_S)
-    scale = hd ** -0.5
-    err = {wT: 0.0, wS: 0.0}
-    refmax = {wT: 0.0, wS: 0.0}
-    for t in rows:
-        for h in rng.choice(Hq, 2, replace=False):
-            g = h // (Hq // Hkv)
-            for w, got in ((wT, oT), (wS, oS)):
-                j0 = max(0, t - w + 1)
-                s = kn[0, j0:t + 1, g] @ qn[0, t, h] * scale
-                p = np.exp(s - s.max())
-                ref = (p[:, None] * vn[0, j0:t + 1, g]).sum(0) / p.sum()
-                err[w] = max(err[w], np.max(np.abs(got[0, t, h] - ref)))
-                refmax[w] = max(refmax[w], np.max(np.abs(ref)))
-    assert err[wT] / refmax[wT] <= TOL_OUT and err[wS] / refmax[wS] <= TOL_OUT
+    rows = _rows(q.shape[1], 512, 8192, rng)
+    assert _sampled_rows_error(o_T, qkv64, 8192, rows, rng) <= TOL_OUT
+    assert _sampled_rows_error(o_S, qkv64, 512, rows, rng) <= TOL_OUT
+    assert torch.isfinite(o_T).all() and torch.isfinite(o_S).all()
+
+
+@pytest.mark.parametrize("w_T", [4096, 8192, 16384])
+@pytest.mark.parametrize("w_S", [256, 512, 1024, 2048])
+def test_window_sweep_full_size_sampled_rows(ttcd, sweep_inputs, w_S, w_T):
+    """The attention sweep at T = 65536 (w_S in {256..2048} x w_T in {4096..16384}):
+    sampled rows, including the rows where either window fills, against the oracle."""
+    _, (q, k, v), qkv64 = sweep_inputs
+    o_T, o_S, _, _ = ttcd.dual_window_attn(q, k, v, w_S, w_T)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    rng = np.random.default_rng(w_S + w_T)
+    rows = _rows(q.shape[1], w_S, w_T, rng)
+    assert _sampled_rows_error(o_T, qkv64, w_T, rows, rng) <= TOL_OUT
+    assert _sampled_rows_error(o_S, qkv64, w_S, rows, rng) <= TOL_OUT
     assert torch.isfinite(o_T).all() and torch.isfinite(o_S).all()

@@ -125,3 +125,19 @@ def test_tiny_workload_dual_windows_bruteforce():
     np.testing.assert_allclose(oS, bS, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(lT, blT, rtol=1e-12)
     np.testing.assert_allclose(lS, blS, rtol=1e-12)
+
+
+def test_single_row_matches_bruteforce():
+    """The row-at-a-time form used for sampled checks of long sequences equals
+    the per-query loop on every row of a small GQA case (2 sequences, ragged
+    windows, rows before and after the window fills)."""
+    g = np.random.default_rng(7)
+    B, T, Hq, Hkv, hd, w = 2, 40, 6, 2, 8, 13
+    q, k, v = (g.standard_normal((B, T, H, hd)) for H in (Hq, Hkv, Hkv))
+    o, lse = orc.windowed_attention_bruteforce(q, k, v, w, 0.3)
+    for b in range(B):
+        for t in (0, 1, 12, 13, 39):
+            for h in range(Hq):
+                orow, l = orc.windowed_attention_row(q, k, v, w, 0.3, b, t, h)
+                np.testing.assert_allclose(orow, o[b, t, h], rtol=1e-12, atol=1e-12)
+                assert abs(l - lse[b, h, t]) < 1e-12
