@@ -79,7 +79,7 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
 // cs[i][t] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
 // Frequency-major, so a warp reading one frequency for 32 consecutive tokens
 // reads 256 contiguous bytes.
-__global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double theta) {
+__global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double theta) {
   const int half = hd / 2;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(T) * half) return;
@@ -88,7 +88,8 @@ __global__ void rope_table_kernel(float2* __restrict__ cs, int T, int hd, double
   const double inv = pow(theta, -2.0 * i / hd);
   double s, c;
   sincos(static_cast<double>(t) * inv, &s, &c);
-  cs[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  // half precision (11-bit significand) is far below the bf16 rounding of q and k
+  cs[idx] = __floats2half2_rn(static_cast<float>(c), static_cast<float>(s));
 }
 
 // Fused short causal convolutions, residual difference and student keys.

@@ -555,53 +555,78 @@ struct EpiSwiGLU {
 template <int HD>
 struct EpiQKVRope {
   static constexpr bool kStaged = true;
-  static constexpr int SPAN = HD >= 64 ? HD : 64;  // columns handled together
+  static constexpr int NF = HD / 2;  // rotation frequencies
   __nv_bfloat16* qkv;
   int ld;         // (Hq + 2 Hkv) * HD
   int n_rope;     // (Hq + Hkv) * HD: columns that get the rotation
   int T;
-  const float2* rope_cs;  // [HD/2][T] (cos, sin), frequency-major
+  const __half2* rope_cs;  // [HD/2][T] (cos, sin), frequency-major
   __device__ float pre(const TileCtx&, int) const { return 1.f; }
+
+  // (x_i, x_{i+NF}) -> (x_i c - x_{i+NF} s, x_{i+NF} c + x_i s) for NF frequencies
+  // starting at f0, in place.
+  template <int N>
+  __device__ static void rotate(float* a, float* b, const uint32_t* tab, int f0, int T) {
+    uint32_t cs[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) cs[i] = __ldg(tab + static_cast<long long>(f0 + i) * T);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      __half2 h;
+      memcpy(&h, &cs[i], 4);
+      const float2 e = __half22float2(h);
+      const float x = a[i], y = b[i];
+      a[i] = x * e.x - y * e.y;
+      b[i] = y * e.x + x * e.y;
+    }
+  }
+
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float) const {
-    static_assert(BN % SPAN == 0, "column tile must hold whole spans");
+    static_assert(BN % 64 == 0 && BN % HD == 0, "column tile must hold whole heads");
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
     const int wrow = r & ~31;
     const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
     const int t = static_cast<int>(row % T);
+    const int tcol = c.tn * BN;
+    const uint32_t* tab = reinterpret_cast<const uint32_t*>(rope_cs) + t;
+    // Rotate the q/k heads of the tile in place in TMEM, 32-column slices at a
+    // time (few live registers), then emit the tile as plain rows.
+    if (tcol < n_rope) {
 #pragma unroll 1
-    for (int h0 = 0; h0 < BN; h0 += SPAN) {
-      const int col0 = c.tn * BN + h0;
-      if (col0 >= ld) break;
-      float x[SPAN];
-#pragma unroll
-      for (int cc = 0; cc < SPAN; cc += 32) {
-        float tmp[32];
-        tmem_ld32f(taddr + h0 + cc, tmp);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[cc + i] = tmp[i];
-      }
-      if (col0 < n_rope) {
-        // SPAN covers SPAN/HD whole heads (all q/k: n_rope is a multiple of SPAN
-        // except when HD = 32 and the q/k/v boundary falls inside a span)
-#pragma unroll
-        for (int hh = 0; hh < SPAN / HD; ++hh) {
-          if (col0 + hh * HD >= n_rope) break;
-#pragma unroll
-          for (int i = 0; i < HD / 2; ++i) {
-            const float2 e = __ldg(rope_cs + static_cast<long long>(i) * T + t);
-            const float a = x[hh * HD + i], b = x[hh * HD + i + HD / 2];
-            x[hh * HD + i] = a * e.x - b * e.y;
-            x[hh * HD + i + HD / 2] = b * e.x + a * e.y;
+      for (int h0 = 0; h0 < BN; h0 += HD) {
+        if (tcol + h0 >= n_rope) break;
+        const uint32_t th = taddr + h0;
+        if constexpr (HD == 32) {
+          uint32_t raw[32];
+          tmem_ld32(th, raw);
+          tmem_ld_wait();
+          float* x = reinterpret_cast<float*>(raw);
+          rotate<16>(x, x + 16, tab, 0, T);
+          tmem_st32(th, raw);
+        } else {
+#pragma unroll 1
+          for (int q = 0; q < NF; q += 32) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(th + q, ra);
+            tmem_ld32(th + NF + q, rb);
+            tmem_ld_wait();
+            rotate<32>(reinterpret_cast<float*>(ra), reinterpret_cast<float*>(rb), tab, q, T);
+            tmem_st32(th + q, ra);
+            tmem_st32(th + NF + q, rb);
           }
         }
       }
-#pragma unroll
-      for (int cc = 0; cc < SPAN; cc += 64)
-        emit(stg, staged, ok, qkv + row * ld, col0 + cc, c.row0 + wrow,
-             *reinterpret_cast<const float(*)[32]>(&x[cc]),
-             *reinterpret_cast<const float(*)[32]>(&x[cc + 32]));
+      tmem_st_wait();
+    }
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 64) {
+      if (tcol + cc >= ld) break;
+      float lo[32], hi[32];
+      tmem_ld32f(taddr + cc, lo);
+      tmem_ld32f(taddr + cc + 32, hi);
+      emit(stg, staged, ok, qkv + row * ld, tcol + cc, c.row0 + wrow, lo, hi);
     }
   }
 };

@@ -226,7 +226,7 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
     sz[B_H] = m.BT * m.d * 4;                        // student residual stream, fp32
     sz[B_HSSQ] = static_cast<size_t>(cdiv(m.d, 256)) * 2 * m.BT * 4;  // RMSNorm partial sums
     sz[B_RSTD] = 2 * m.BT * 4;                                           // RMSNorm row scales
-    sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 8;
+    sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 4;
   }
   sz[B_U] = 2 * m.BT * m.d * e;
   sz[B_Z] = 2 * m.BT * m.f * 4;
@@ -618,7 +618,7 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
   __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
   E* o = at<E>(ws, L, B_O);
   float* h = at<float>(ws, L, B_H);
-  float2* rope = at<float2>(ws, L, B_ROPE);
+  __half2* rope = at<__half2>(ws, L, B_ROPE);
   E* u = at<E>(ws, L, B_U);
   float* hssq = at<float>(ws, L, B_HSSQ);
   const E* xin = static_cast<const E*>(x);
