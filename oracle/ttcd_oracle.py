@@ -222,6 +222,49 @@ def dual_window_attention(q, k, v, w_S: int, w_T: int, scale: float):
     return o_T, o_S, lse_T, lse_S
 
 
+def band_attention(q, k, v, near: int, far: int, scale: float):
+    """Causal band attention with GQA: query t attends to keys j with
+    t - far <= j <= t - near (clipped at 0), softmax over the band only.
+
+    [README] "Fused inference kernels", lse_dual_attn: the teacher window is
+    the student window [t-w_S+1, t] plus a shifted far band [t-w_T+1, t-w_S]
+    (near = w_S, far = w_T - 1), and the two partial attentions merge exactly
+    through their log-sum-exp.  A row whose band holds no key gets o = 0 and
+    lse = -inf (it carries no weight in the merge).  Returns (o, lse).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, T, Hq, hd = q.shape
+    G = Hq // k.shape[2]
+    o = np.zeros_like(q)
+    lse = np.full((B, Hq, T), -np.inf)
+    t = np.arange(T)
+    j = np.arange(T)
+    mask = (j[None, :] <= t[:, None] - near) & (j[None, :] >= t[:, None] - far)
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * (q[b, :, h] @ k[b, :, h // G].T)
+            s = np.where(mask, s, -np.inf)
+            m = s.max(axis=1)
+            rows = np.isfinite(m)
+            e = np.exp(s[rows] - m[rows, None])
+            den = e.sum(axis=1)
+            o[b, rows, h] = (e @ v[b, :, h // G]) / den[:, None]
+            lse[b, h, rows] = m[rows] + np.log(den)
+    return o, lse
+
+
+def lse_merge(o1, lse1, o2, lse2):
+    """Exact merge of two partial softmax attentions over disjoint key sets:
+    o = (o1 e^{lse1} + o2 e^{lse2}) / (e^{lse1} + e^{lse2}), lse = logaddexp.
+    o: [B, T, H, hd]; lse: [B, H, T].  [README] "Fused inference kernels"."""
+    lse = np.logaddexp(lse1, lse2)
+    w1 = np.exp(lse1 - lse).transpose(0, 2, 1)[..., None]
+    w2 = np.exp(lse2 - lse).transpose(0, 2, 1)[..., None]
+    return w1 * np.asarray(o1, np.float64) + w2 * np.asarray(o2, np.float64), lse
+
+
 # ---------------------------------------------------------------------------
 # Fast-weight MLP (in-place TTCD)
 # ---------------------------------------------------------------------------

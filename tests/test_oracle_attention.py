@@ -141,3 +141,42 @@ def test_single_row_matches_bruteforce():
                 orow, l = orc.windowed_attention_row(q, k, v, w, 0.3, b, t, h)
                 np.testing.assert_allclose(orow, o[b, t, h], rtol=1e-12, atol=1e-12)
                 assert abs(l - lse[b, h, t]) < 1e-12
+
+
+def test_band_attention_special_cases():
+    """near = 0, far = w - 1 is the sliding window of w keys; a band that lies
+    before the sequence start is empty (o = 0, lse = -inf)."""
+    q, k, v = _rand_qkv(1, 50, 4, 2, 8, seed=21)
+    for w in (1, 7, 50):
+        o, lse = orc.band_attention(q, k, v, 0, w - 1, 0.4)
+        ow, lsew = orc.windowed_attention(q, k, v, w, 0.4)
+        np.testing.assert_allclose(o, ow, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, lsew, rtol=1e-12, atol=1e-12)
+    o, lse = orc.band_attention(q, k, v, 10, 20, 0.4)
+    assert np.all(o[:, :10] == 0) and np.all(np.isneginf(lse[:, :, :10]))
+    assert np.all(np.isfinite(lse[:, :, 10:]))
+
+
+def test_far_band_matches_per_query_loop_and_merges_to_teacher():
+    """The oracle's far band [t-w_T+1, t-w_S] against an explicit per-query
+    loop, and lse_merge(student window, far band) against the teacher window."""
+    B, T, Hq, Hkv, hd, wS, wT = 2, 70, 4, 2, 8, 9, 33
+    q, k, v = _rand_qkv(B, T, Hq, Hkv, hd, seed=5)
+    scale = hd ** -0.5
+    of, lf = orc.band_attention(q, k, v, wS, wT - 1, scale)
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(T):
+                keys = list(range(max(0, t - wT + 1), t - wS + 1))
+                if not keys:
+                    assert np.isneginf(lf[b, h, t]) and np.all(of[b, t, h] == 0)
+                    continue
+                s = np.array([scale * q[b, t, h] @ k[b, j, h // 2] for j in keys])
+                e = np.exp(s - s.max())
+                np.testing.assert_allclose(of[b, t, h], (e[:, None] * v[b, keys, h // 2]).sum(0) / e.sum(),
+                                           rtol=1e-12, atol=1e-13)
+                np.testing.assert_allclose(lf[b, h, t], s.max() + np.log(e.sum()), rtol=1e-12)
+    oT, oS, lT, lS = orc.dual_window_attention(q, k, v, wS, wT, scale)
+    om, lm = orc.lse_merge(oS, lS, of, lf)
+    np.testing.assert_allclose(om, oT, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lm, lT, rtol=1e-12)
