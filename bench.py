@@ -367,16 +367,24 @@ def run_attention(args, world, rank, local):
     o_T, o_S = torch.empty_like(q), torch.empty_like(q)
     pairs = [(int(a), int(b)) for a, b in (w.split("/") for w in args.windows.split(","))]
     stream = torch.cuda.current_stream()
+    lse_form = args.form == "lse"
+
+    def call(wS, wT):
+        if lse_form:
+            ttcd.dual_window_attn_lse(q, k, v, wS, wT)
+        else:
+            ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
+
     for wS, wT in pairs:
         shape = s0.with_(w_S=wS, w_T=wT)
         for _ in range(args.warmup):
-            ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
+            call(wS, wT)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world, local)
         e0.record(stream)
         for _ in range(args.steps):
-            ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
+            call(wS, wT)
         e1.record(stream)
         torch.cuda.synchronize()
         ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
@@ -385,7 +393,8 @@ def run_attention(args, world, rank, local):
         ach = fl / (ms / 1e3) / 1e12
         if rank == 0:
             print(json.dumps({
-                "metric": "fused dual-window attention tokens/s (Qwen3-0.6B heads)",
+                "metric": ("LSE-combination" if lse_form else "fused") +
+                          " dual-window attention tokens/s (Qwen3-0.6B heads)",
                 "value": shape.B * shape.T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -393,8 +402,8 @@ def run_attention(args, world, rank, local):
                 "config": {"workload": "dual_window_attention", "B": shape.B, "T": shape.T,
                            "n_q_heads": 16, "n_kv_heads": 8, "head_dim": 128, "w_S": wS,
                            "w_T": wT},
-                "roofline": {"kernel": "dual_window_attn_kernel<128>", "bound": "tensor",
-                             "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "roofline": {"kernel": "dual_window_attn_kernel<128>" + (" + lse_merge_kernel" if lse_form else ""),
+                             "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": ach / peaks["bf16_tflops"],
                              "peak_source": f"{peak_kind} bf16_tflops (burst: kernel timed alone)",
                              "flops_per_launch": fl}}), flush=True)
@@ -472,6 +481,8 @@ def main():
     ap.add_argument("--B", type=int, default=1, help="--mode attn / stack: sequences")
     ap.add_argument("--windows", default="512/8192",
                     help="--mode attn: comma-separated w_S/w_T pairs")
+    ap.add_argument("--form", choices=["fused", "lse"], default="fused",
+                    help="--mode attn: fused kernel, or student window + far band merged by LSE")
     ap.add_argument("--attn-traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture")
     args = ap.parse_args()

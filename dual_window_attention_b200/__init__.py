@@ -63,6 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     P, W = ctypes.POINTER(_Params), ctypes.POINTER(_Weights)
     lib.ttcd_dual_window_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
+    lib.ttcd_dual_window_attn_lse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                              i, f, i, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
     lib.ttcd_fastweight_mlp_workspace_size.argtypes = [P]
@@ -180,6 +182,24 @@ def dual_window_attn(q, k, v, w_S: int, w_T: int, scale: float = 0.0, o_T=None, 
                                    _stream(stream))
     _check(st, "ttcd_dual_window_attn")
     return o_T, o_S, lse_T, lse_S
+
+
+def dual_window_attn_lse(q, k, v, w_S: int, w_T: int, scale: float = 0.0, stream=None):
+    """Dual-window attention by LSE combination (student window + far band).
+
+    Returns (o_T, o_S, o_far, lse_T, lse_S, lse_far)."""
+    lib = load_library()
+    B, T, Hq, hd = q.shape
+    Hkv = k.shape[2]
+    o_T, o_S, o_far = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    lse_T = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+    lse_S, lse_far = torch.empty_like(lse_T), torch.empty_like(lse_T)
+    dt = BF16 if q.dtype == torch.bfloat16 else F32
+    st = lib.ttcd_dual_window_attn_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(o_T), _ptr(o_S),
+                                       _ptr(o_far), _ptr(lse_T), _ptr(lse_S), _ptr(lse_far), B, T,
+                                       Hq, Hkv, hd, w_S, w_T, scale, dt, _stream(stream))
+    _check(st, "ttcd_dual_window_attn_lse")
+    return o_T, o_S, o_far, lse_T, lse_S, lse_far
 
 
 def block_forward_workspace_size(p: BlockParams) -> int:

@@ -42,6 +42,8 @@ struct AttnArgs {
   OutT* o_S;
   float* lse_T;  // [B, Hq, T], nullable
   float* lse_S;
+  OutT* o_far;     // split form only: far band [t-w_T+1, t-w_S], [B, T, Hq, HD]
+  float* lse_far;  // split form only: [B, Hq, T]
   int B, T, Hq, Hkv;
   int w_S, w_T;
   float scale_log2;  // softmax scale * log2(e)
@@ -181,7 +183,11 @@ __device__ __forceinline__ void tmem_store_row(uint32_t taddr, float inv_l, OutT
   }
 }
 
-template <int HD, class OutT>
+// SPLIT = false: the fused form (o_T, o_S).  SPLIT = true: the LSE-combination
+// form of the README's lse_dual_attn: the accumulator restarts at the student
+// edge, so phase 2 yields the far band alone (o_far, lse_far) and o_T comes from
+// merging it with the student window through the log-sum-exp (lse_merge_kernel).
+template <int HD, class OutT, bool SPLIT>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     dual_window_attn_kernel(const __grid_constant__ CUtensorMap mapQ,
                             const __grid_constant__ CUtensorMap mapK,
@@ -321,7 +327,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       auto issue_pv = [&](int h, int v) {
         const uint32_t v_lo = v_lo0 + (((v % ATT_VS) * Cfg::TILE_BYTES) >> 4);
         const uint32_t d = tmem + 256 + h * 128, pa = tmem + h * 128;
-        const uint32_t acc0 = v > 0 ? 1u : 0u;
+        // the first visit, and in the split form the first far-band visit, start O afresh
+        const uint32_t acc0 = (v > 0 && !(SPLIT && v == vis.vX)) ? 1u : 0u;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < ATT_BN / 16; ++kk)
@@ -383,7 +390,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const long long orow = (static_cast<long long>(b) * a.T + t) * a.Hq + head;
     const long long li = (static_cast<long long>(b) * a.Hq + head) * a.T + t;
     const float sl2 = a.scale_log2;
-    float m_ref = 0.f, l = 0.f;
+    // m_ref = -inf: nothing visible yet (the first tile, or the far band of the
+    // split form before its first visible key); O is zero for such a row.
+    float m_ref = -INFINITY, l = 0.f;
     bool ok = active;
     for (int v = 0; v < vis.nv && ok; ++v) {
       const int j = vis.tile(v);
@@ -395,6 +404,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // end of the student phase: O / l is o_S (PV of every earlier tile has landed)
         tmem_store_row<HD, OutT>(o_addr, 1.f / l, a.o_S + orow * HD, row_ok);
         if (row_ok && a.lse_S) a.lse_S[li] = (m_ref + __log2f(l)) * 0.6931471805599453f;
+        if (SPLIT) {
+          m_ref = -INFINITY;
+          l = 0.f;
+        }
       }
       float s[128];
       tmem_ld_cols<128>(s_addr, s);
@@ -418,21 +431,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_tile = mx * sl2;
-      if (v == 0) {
-        m_ref = m_tile;
-      } else {
-        const bool grow = m_tile > m_ref + ATT_RESCALE_THRESHOLD;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float m_new = grow ? m_tile : m_ref;
-          const float al = ex2_approx(m_ref - m_new);
-          tmem_scale_row<HD>(o_addr, al);
-          l *= al;
-          m_ref = m_new;
-        }
+      const bool fresh = m_ref == -INFINITY;
+      const bool grow = !fresh && m_tile > m_ref + ATT_RESCALE_THRESHOLD;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_new = grow ? m_tile : m_ref;
+        const float al = grow ? ex2_approx(m_ref - m_new) : 1.f;
+        tmem_scale_row<HD>(o_addr, al);
+        l *= al;
+        m_ref = m_new;
       }
-      // exponentials, row sum, bf16 pack
+      if (fresh) m_ref = m_tile;  // may stay -inf: a row with no visible key in this tile
+      // exponentials, row sum, bf16 pack (a row still at -inf has only masked scores)
+      const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
       const uint64_t sc2 = f2pack(sl2, sl2);
-      const uint64_t nm2 = f2pack(-m_ref, -m_ref);
+      const uint64_t nm2 = f2pack(nm, nm);
       uint64_t acc4[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f),
                           f2pack(0.f, 0.f)};
       uint32_t P[64];
@@ -479,13 +491,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     if (ok && mbar_wait(&o_done[h_local], (vis.nv - 1) & 1, st, abort)) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
-      tmem_store_row<HD, OutT>(o_addr, inv_l, a.o_T + orow * HD, row_ok);
-      if (row_ok && a.lse_T) a.lse_T[li] = lse;
-      if (vis.vX == vis.nv) {  // no teacher-only keys: o_T == o_S
+      // l = 0 only for an empty far band (split form): o = 0, lse = -inf
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse = l > 0.f ? (m_ref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      const bool no_band = vis.vX == vis.nv;  // no teacher-only keys in this tile
+      if (!SPLIT) {
+        tmem_store_row<HD, OutT>(o_addr, inv_l, a.o_T + orow * HD, row_ok);
+        if (row_ok && a.lse_T) a.lse_T[li] = lse;
+      }
+      if (no_band) {  // the accumulator holds the student window: o_T == o_S
         tmem_store_row<HD, OutT>(o_addr, inv_l, a.o_S + orow * HD, row_ok);
         if (row_ok && a.lse_S) a.lse_S[li] = lse;
+      }
+      if (SPLIT) {
+        tmem_store_row<HD, OutT>(o_addr, no_band ? 0.f : inv_l, a.o_far + orow * HD, row_ok);
+        if (row_ok) a.lse_far[li] = no_band ? -INFINITY : lse;
       }
     }
   }
@@ -494,6 +514,61 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// 8 consecutive elements (16-byte aligned) to and from fp32 registers
+__device__ __forceinline__ void ld8f(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = bf16lo_to_f32(w[i]);
+    v[2 * i + 1] = bf16hi_to_f32(w[i]);
+  }
+}
+__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8f(__nv_bfloat16* dst, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ void st8f(float* dst, const float (&v)[8]) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// o_T = (o_S e^{lse_S} + o_far e^{lse_far}) / (e^{lse_S} + e^{lse_far}) and
+// lse_T = logaddexp(lse_S, lse_far): the exact merge of two partial softmax
+// attentions over disjoint key sets (GitHub README "TTCD", "Fused inference
+// kernels", lse_dual_attn).  One thread per 8 output elements of one row
+// (b, t, h); lse [B, Hq, T], o [B, T, Hq, HD].
+template <int HD, class OutT>
+__global__ void lse_merge_kernel(const OutT* __restrict__ o_S, const float* __restrict__ lse_S,
+                                 const OutT* __restrict__ o_far,
+                                 const float* __restrict__ lse_far, OutT* __restrict__ o_T,
+                                 float* __restrict__ lse_T, int T, int Hq, long long rows) {
+  constexpr int PER = 8, TPR = HD / PER;  // elements per thread, threads per row
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = idx / TPR;  // (b * T + t) * Hq + h
+  if (row >= rows) return;
+  const int c = static_cast<int>(idx % TPR) * PER;
+  const int h = static_cast<int>(row % Hq);
+  const long long bt = row / Hq;
+  const int t = static_cast<int>(bt % T);
+  const long long li = (bt / T * Hq + h) * T + t;
+  const float ls = lse_S[li], lf = lse_far[li];
+  const float m = fmaxf(ls, lf);  // lse_S is finite: the diagonal key is in every window
+  const float ws = __expf(ls - m), wf = lf == -INFINITY ? 0.f : __expf(lf - m);
+  const float inv = 1.f / (ws + wf);
+  float x[PER], y[PER];
+  ld8f(o_S + row * HD + c, x);
+  ld8f(o_far + row * HD + c, y);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) x[i] = (x[i] * ws + y[i] * wf) * inv;
+  st8f(o_T + row * HD + c, x);
+  if (c == 0 && lse_T) lse_T[li] = m + __logf(ws + wf);
 }
 
 }  // namespace ttcd

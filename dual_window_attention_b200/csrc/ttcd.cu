@@ -267,10 +267,11 @@ T* at(void* ws, const Layout& L, Buf b) {
 // ------------------------------------------------------------------ attention
 // q rows have `ld_q` elements between tokens, k and v rows `ld_kv` (equal to
 // Hq*HD / Hkv*HD for separate tensors, or the qkv width for one packed tensor).
-template <int HD, class OutT>
+template <int HD, class OutT, bool SPLIT = false>
 ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
                         OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv,
-                        int w_S, int w_T, float scale, long long ld_q, long long ld_kv) {
+                        int w_S, int w_T, float scale, long long ld_q, long long ld_kv,
+                        OutT* o_far = nullptr, float* lse_far = nullptr) {
   CUtensorMap mq, mk, mv;
   const long long BT = static_cast<long long>(B) * T;
   using bf = __nv_bfloat16;
@@ -283,6 +284,8 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   a.o_S = o_S;
   a.lse_T = lse_T;
   a.lse_S = lse_S;
+  a.o_far = o_far;
+  a.lse_far = lse_far;
   a.B = B;
   a.T = T;
   a.Hq = Hq;
@@ -292,7 +295,7 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_qt = (T + ATT_BM - 1) / ATT_BM;
   a.pairs = (Hq / Hkv + 1) / 2;
-  auto kern = dual_window_attn_kernel<HD, OutT>;
+  auto kern = dual_window_attn_kernel<HD, OutT, SPLIT>;
   constexpr int smem = AttnCfg<HD>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -313,6 +316,25 @@ ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, 
     case 128: return launch_attn<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
     default: return TTCD_ERR_UNSUPPORTED;
   }
+}
+
+// The LSE-combination form: the split kernel gives o_S, lse_S and the far band
+// (o_far, lse_far); the merge kernel combines them into o_T (and lse_T).
+template <int HD>
+ttcd_status launch_attn_lse(const Ctx& c, const void* q, const void* k, const void* v,
+                            __nv_bfloat16* o_T, __nv_bfloat16* o_S, __nv_bfloat16* o_far,
+                            float* lse_T, float* lse_S, float* lse_far, int B, int T, int Hq,
+                            int Hkv, int w_S, int w_T, float scale) {
+  TTCD_TRY((launch_attn<HD, __nv_bfloat16, true>(c, q, k, v, nullptr, o_S, nullptr, lse_S, B, T,
+                                                 Hq, Hkv, w_S, w_T, scale,
+                                                 static_cast<long long>(Hq) * HD,
+                                                 static_cast<long long>(Hkv) * HD, o_far, lse_far)));
+  const long long rows = static_cast<long long>(B) * T * Hq;
+  const long long threads = rows * (HD / 8);
+  lse_merge_kernel<HD, __nv_bfloat16><<<static_cast<unsigned>(cdiv(threads, 256)), 256, 0, c.s>>>(
+      o_S, lse_S, o_far, lse_far, o_T, lse_T, T, Hq, rows);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
 }
 
 // ------------------------------------------------------------------ fast-weight MLP body
@@ -564,6 +586,35 @@ ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, v
                                  static_cast<__nv_bfloat16*>(o_S), lse_T, lse_S, B, T, Hq, Hkv,
                                  hd, w_S, w_T, sc, static_cast<long long>(Hq) * hd,
                                  static_cast<long long>(Hkv) * hd);
+}
+
+ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* v, void* o_T,
+                                      void* o_S, void* o_far, float* lse_T, float* lse_S,
+                                      float* lse_far, int B, int T, int Hq, int Hkv, int hd,
+                                      int w_S, int w_T, float scale, ttcd_dtype dtype,
+                                      void* stream) {
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || w_S < 1 || w_T < w_S ||
+      !(scale >= 0.f))
+    return TTCD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_T) || !aligned16(o_S) ||
+      !aligned16(o_far) || !aligned16(lse_S) || !aligned16(lse_far))
+    return TTCD_ERR_INVALID_ARG;
+  if (lse_T && !aligned16(lse_T)) return TTCD_ERR_INVALID_ARG;
+  if (dtype != TTCD_BF16) return dtype == TTCD_F32 ? TTCD_ERR_UNSUPPORTED : TTCD_ERR_INVALID_ARG;
+  if (hd != 32 && hd != 64 && hd != 128) return TTCD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * T * Hq * (hd / 8) >= (1ll << 31) * 256ll)
+    return TTCD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * T >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c));
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(hd));
+  using bf = __nv_bfloat16;
+  bf *oT = static_cast<bf*>(o_T), *oS = static_cast<bf*>(o_S), *oF = static_cast<bf*>(o_far);
+  switch (hd) {
+    case 32: return launch_attn_lse<32>(c, q, k, v, oT, oS, oF, lse_T, lse_S, lse_far, B, T, Hq, Hkv, w_S, w_T, sc);
+    case 64: return launch_attn_lse<64>(c, q, k, v, oT, oS, oF, lse_T, lse_S, lse_far, B, T, Hq, Hkv, w_S, w_T, sc);
+    default: return launch_attn_lse<128>(c, q, k, v, oT, oS, oF, lse_T, lse_S, lse_far, B, T, Hq, Hkv, w_S, w_T, sc);
+  }
 }
 
 ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,

@@ -115,6 +115,30 @@ ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, v
                                   ttcd_dtype dtype, void* stream);
 
 /*
+ * ttcd_dual_window_attn_lse — the same two outputs by LSE combination.
+ *
+ * Defines ([README] "Fused inference kernels", lse_dual_attn): the teacher
+ * window is the student window plus the shifted far band
+ *   far(t) = { j : max(0, t-w_T+1) <= j <= t-w_S },
+ * attended separately and merged exactly through the log-sum-exps:
+ *   o_T = (o_S e^{lse_S} + o_far e^{lse_far}) / (e^{lse_S} + e^{lse_far}),
+ *   lse_T = log(e^{lse_S} + e^{lse_far}).
+ * A row whose far band is empty (t < w_S, or w_S = w_T) gets o_far = 0 and
+ * lse_far = -inf, and then o_T = o_S.  A second implementation of
+ * ttcd_dual_window_attn (one pass over K/V; the accumulator restarts at the
+ * student edge) followed by an elementwise merge.
+ *   q, k, v, o_T, o_S, scale, dtype, errors: as ttcd_dual_window_attn
+ *   o_far      [B, T, Hq, hd]  bf16, device, written (far-band attention)
+ *   lse_S, lse_far [B, Hq, T] fp32, device, written (required: the merge reads them)
+ *   lse_T      [B, Hq, T] fp32, device, nullable
+ */
+ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* v, void* o_T,
+                                      void* o_S, void* o_far, float* lse_T, float* lse_S,
+                                      float* lse_far, int B, int T, int Hq, int Hkv, int hd,
+                                      int w_S, int w_T, float scale, ttcd_dtype dtype,
+                                      void* stream);
+
+/*
  * ttcd_fastweight_mlp — the in-place fast-weight MLP of one block (off-policy).
  *
  * Defines ([REVIEW] 关键设计 2 and 3, flowchart C-F; [PODCAST] cue 29):

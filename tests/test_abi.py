@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_three_entry_points():
     names = declared_functions()
-    for n in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward"):
+    for n in ("ttcd_dual_window_attn", "ttcd_dual_window_attn_lse", "ttcd_fastweight_mlp",
+              "ttcd_block_forward"):
         assert n in names
 
 
@@ -108,3 +109,15 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 128, 2, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ttcd.dual_window_attn(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous(), 16, 64)
+
+
+def test_lse_form_rejects_bad_arguments_on_host(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    f = lib.ttcd_dual_window_attn_lse
+    ok_args = [fake] * 9
+    assert f(*([None] + ok_args[1:]), 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    # lse_S and lse_far are required (the merge reads them)
+    assert f(*(ok_args[:7] + [None, fake]), 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    assert f(*ok_args, 1, 256, 2, 1, 32, 65, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
+    assert f(*ok_args, 1, 256, 2, 1, 48, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_UNSUPPORTED
+    assert f(*ok_args, 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.F32, None) == ttcd.ERR_UNSUPPORTED

@@ -130,3 +130,52 @@ def test_window_sweep_full_size_sampled_rows(ttcd, sweep_inputs, w_S, w_T):
     assert _sampled_rows_error(o_T, qkv64, w_T, rows, rng) <= TOL_OUT
     assert _sampled_rows_error(o_S, qkv64, w_S, rows, rng) <= TOL_OUT
     assert torch.isfinite(o_T).all() and torch.isfinite(o_S).all()
+
+
+# ---------------------------------------------------------------------- LSE combination form
+@pytest.mark.parametrize("B,T,Hq,Hkv,hd,wS,wT", CASES)
+def test_lse_combination_parity(ttcd, B, T, Hq, Hkv, hd, wS, wT):
+    """ttcd_dual_window_attn_lse (student window + far band merged through the
+    log-sum-exp; README "Fused inference kernels", lse_dual_attn) against the
+    oracle: both windows, the far band, and every lse; an empty far band is
+    exactly o = 0, lse = -inf."""
+    q, k, v = make_attention_inputs(B, T, Hq, Hkv, hd, seed=T + hd)
+    o_T, o_S, o_far, lse_T, lse_S, lse_far = ttcd.dual_window_attn_lse(q.cuda(), k.cuda(),
+                                                                       v.cuda(), wS, wT)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    qn, kn, vn = np64(q), np64(k), np64(v)
+    scale = hd ** -0.5
+    rT, rS, rlT, rlS = orc.dual_window_attention(qn, kn, vn, wS, wT, scale)
+    rF, rlF = orc.band_attention(qn, kn, vn, wS, wT - 1, scale)
+    assert rel_max(o_T, rT) <= TOL_OUT
+    assert rel_max(o_S, rS) <= TOL_OUT
+    empty = np.isneginf(rlF)
+    lf = np64(lse_far)
+    assert np.array_equal(np.isneginf(lf), empty)
+    np.testing.assert_allclose(lf[~empty], rlF[~empty], atol=2e-3, rtol=0)
+    of = np64(o_far)
+    assert np.all(of.transpose(0, 2, 1, 3)[empty] == 0)
+    if (~empty).any():
+        assert rel_max(of.transpose(0, 2, 1, 3)[~empty], rF.transpose(0, 2, 1, 3)[~empty]) <= TOL_OUT
+    np.testing.assert_allclose(np64(lse_T), rlT, atol=2e-3, rtol=0)
+    np.testing.assert_allclose(np64(lse_S), rlS, atol=2e-3, rtol=0)
+    # the two implementations agree with each other
+    f_T, f_S, _, _ = ttcd.dual_window_attn(q.cuda(), k.cuda(), v.cuda(), wS, wT)
+    assert rel_max(o_T, f_T) <= TOL_OUT and torch.equal(o_S, f_S)
+
+
+def test_lse_combination_full_size(ttcd, sweep_inputs):
+    """T = 65536, Qwen3 heads, 512/8192: the LSE form against the fused form and,
+    on sampled rows, against the oracle."""
+    _, (q, k, v), qkv64 = sweep_inputs
+    o_T, o_S, o_far, _, _, lse_far = ttcd.dual_window_attn_lse(q, k, v, 512, 8192)
+    f_T, f_S, _, _ = ttcd.dual_window_attn(q, k, v, 512, 8192)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    assert rel_max(o_T, f_T) <= TOL_OUT and torch.equal(o_S, f_S)
+    rng = np.random.default_rng(3)
+    rows = _rows(q.shape[1], 512, 8192, rng)
+    assert _sampled_rows_error(o_T, qkv64, 8192, rows, rng) <= TOL_OUT
+    assert torch.isneginf(lse_far[:, :, :512]).all() and (o_far[:, :512] == 0).all()
+    assert torch.isfinite(lse_far[:, :, 512:]).all()
