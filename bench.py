@@ -146,33 +146,55 @@ class ClockSampler:
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
 
 
-def dist_setup():
+def dist_setup(backend=None, timeout_s: float = 300.0):
+    """One process per GPU from the torchrun environment.  NCCL when CUDA is
+    present (the bench), gloo otherwise (host-side tests of the same code)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=timeout_s),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=timeout_s))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
 
 
+def _nccl() -> bool:
+    import torch.distributed as dist
+    return dist.get_backend() == "nccl"
+
+
 def barrier(world, local):
     if world > 1:
         import torch.distributed as dist
-        dist.barrier(device_ids=[local])
+        if _nccl():
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
 
 
 def max_over_ranks(world, v: float) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if _nccl() else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, units_per_rank: float, ms_local: float):
+    """Replicas: every rank processes its own units.  The job's time per step is
+    the slowest rank's; the job's rate counts the units of all ranks."""
+    ms = max_over_ranks(world, ms_local)
+    return ms, units_per_rank * world / (ms / 1e3)
 
 
 def oracle_throughput(shape, sample_tokens: int, repeats: int = 1):
@@ -278,12 +300,11 @@ def run_ours(args, world, rank, local):
     ttcd.set_stage_events(None)
     launches = ttcd.kernel_launch_count() - launches0
     barrier(world, local)
-    ms = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    ms, value = job_throughput(world, shape.B * shape.T, start.elapsed_time(end) / args.steps)
     st, flags = ttcd.get_device_error()
     if st != ttcd.OK:
         raise RuntimeError(f"device error in timed region: flags={flags}")
     tokens = shape.B * shape.T * world
-    value = tokens / (ms / 1000.0)
 
     # per-stage times (mean over steps) and roofline fractions
     costs = stage_costs(shape)
@@ -323,7 +344,7 @@ def run_ours(args, world, rank, local):
     e2.record(stream)
     torch.cuda.synchronize()
     barrier(world, local)
-    ms_e2e = max_over_ranks(world, s2.elapsed_time(e2)) / args.steps
+    ms_e2e, _ = job_throughput(world, shape.B * shape.T, s2.elapsed_time(e2) / args.steps)
     assert torch.equal(out_h, out.cpu())
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
