@@ -430,6 +430,64 @@ def run_attention(args, world, rank, local):
                              "flops_per_launch": fl}}), flush=True)
 
 
+def run_decode_bench(args, world, rank, local):
+    """Token-by-token decode of the Qwen3-0.6B-shaped block (B sequences in
+    lockstep).  Times --steps consecutive tokens from a position past the teacher
+    window (the cache is full; chunk commits fall inside the timed tokens at their
+    natural rate).  The HBM floor of one token step is the weights it must read:
+    the shared slow weights plus each sequence's W_down + S and K/V window."""
+    import dual_window_attention_b200 as ttcd
+    ttcd.load_library()
+    peaks, peak_kind = load_peaks()
+    shape = QWEN3_0P6B_64K.with_(name="qwen3_0.6b_block_decode", B=args.B, T=1)
+    dev = torch.device("cuda", local)
+    inp = make_block_inputs(shape, seed=0)
+    w = {k: v.to(dev) for k, v in inp["layers"][0].items()}
+    p = ttcd.BlockParams.from_shape(shape)
+    dec = ttcd.Decoder(w, p)
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(args.B, shape.d_model, generator=g).to(torch.bfloat16).to(dev)
+    beta = (0.1 * torch.sigmoid(torch.randn(args.B, generator=g))).to(dev)
+    y = torch.empty_like(x)
+    dec.t = 4 * shape.w_T + 7  # past the window: full K/V reads every step
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        dec.step(x, beta, y)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = ttcd.kernel_launch_count()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            dec.step(x, beta, y)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    launches = ttcd.kernel_launch_count() - launches0
+    ms, value = job_throughput(world, args.B * args.steps, e0.elapsed_time(e1))
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    s_ = shape
+    dqkv = (s_.n_q_heads + 2 * s_.n_kv_heads) * s_.head_dim
+    shared = 2 * (dqkv * s_.d_model + s_.d_model * s_.n_q_heads * s_.head_dim +
+                  2 * s_.d_ff * s_.d_model + s_.d_model * s_.d_ff)
+    per_seq = 2 * s_.d_model * s_.d_ff + 2 * 2 * s_.w_T * s_.n_kv_heads * s_.head_dim
+    bytes_per_step = shared + args.B * per_seq
+    step_ms = ms / args.steps
+    ach = bytes_per_step / (step_ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "IP-TTCD block decode tokens/s (Qwen3-0.6B shape, w_S 512, w_T 8192)",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(shape, {"sequences": args.B, "position": "past w_T",
+                                              "parallelism": f"replicas{world}"}),
+            "roofline": {"kernel": "decode step (all kernels)", "bound": "hbm", "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                         "bytes_per_step": bytes_per_step, "peak_source": f"{peak_kind} hbm_gbs"},
+            "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
+
+
 def run_stack(args, world, rank, local):
     """The 28-layer stack of Qwen3-0.6B-shaped blocks, end-to-end prefill tokens/s
     (B 1 x T 65536 by default, or --B 4 --T 16384): every layer one ttcd_block_forward
@@ -493,13 +551,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
-    ap.add_argument("--mode", choices=["block", "attn", "stack"], default="block",
+    ap.add_argument("--mode", choices=["block", "attn", "stack", "decode"], default="block",
                     help="block: the whole IP-TTCD block (default); attn: attention alone; "
-                         "stack: 28 blocks end to end")
+                         "stack: 28 blocks end to end; decode: one token at a time")
     ap.add_argument("--T", type=int, default=65536,
                     help="tokens per sequence (65536 is the benchmark workload; smaller values "
                          "are for profiling)")
-    ap.add_argument("--B", type=int, default=1, help="--mode attn / stack: sequences")
+    ap.add_argument("--B", type=int, default=1, help="--mode attn / stack / decode: sequences")
     ap.add_argument("--windows", default="512/8192",
                     help="--mode attn: comma-separated w_S/w_T pairs")
     ap.add_argument("--form", choices=["fused", "lse"], default="fused",
@@ -515,6 +573,8 @@ def main():
             run_attention(args, world, rank, local)
         elif args.mode == "stack":
             run_stack(args, world, rank, local)
+        elif args.mode == "decode":
+            run_decode_bench(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

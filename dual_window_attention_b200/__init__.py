@@ -65,6 +65,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_dual_window_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
     lib.ttcd_dual_window_attn_lse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                               i, f, i, vp]
+    lib.ttcd_decode_state_size.argtypes = [P]
+    lib.ttcd_decode_state_size.restype = sz
+    lib.ttcd_decode_workspace_size.argtypes = [P]
+    lib.ttcd_decode_workspace_size.restype = sz
+    lib.ttcd_decode_state_init.argtypes = [W, P, vp, vp, sz, vp, sz, vp]
+    lib.ttcd_block_decode.argtypes = [vp, vp, i, W, P, vp, sz, vp, vp, sz, vp]
+    lib.ttcd_decode_state_read.argtypes = [P, i, vp, sz, vp, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
     lib.ttcd_fastweight_mlp_workspace_size.argtypes = [P]
@@ -278,6 +285,52 @@ def block_stack_forward(x, layers, p: BlockParams, workspace: Optional[torch.Ten
             on_layer(l, out)
         cur = out
     return cur
+
+
+class Decoder:
+    """Token-by-token decode of one block for a batch of B sequences in lockstep.
+
+    Holds the decode state (K/V ring cache, conv history, the current chunk's
+    rows, the fast weight) and a step workspace, both allocated once.
+    ``step(x_t, beta_t)`` takes x_t [B, d] bf16 and beta_t [B] fp32 of the next
+    position and returns y_t [B, d]; ``state()`` is the fast-weight state after
+    the tokens so far (partial chunk included)."""
+
+    def __init__(self, weights: Dict[str, torch.Tensor], p: BlockParams, state_in=None,
+                 device="cuda", stream=None):
+        self.lib = load_library()
+        self.p, self.pc, self.wc = p, p.c(), _weights(weights)
+        self.weights = weights  # keep the tensors alive
+        self.stream = stream
+        n_state = self.lib.ttcd_decode_state_size(ctypes.byref(self.pc))
+        n_ws = self.lib.ttcd_decode_workspace_size(ctypes.byref(self.pc))
+        if n_state == 0 or n_ws == 0:
+            raise TTCDError(ERR_UNSUPPORTED, "ttcd_decode_state_size")
+        self.state = alloc_workspace(n_state, device)
+        self.ws = alloc_workspace(n_ws, device)
+        _check(self.lib.ttcd_decode_state_init(ctypes.byref(self.wc), ctypes.byref(self.pc),
+                                               _ptr(state_in), _ptr(self.state),
+                                               self.state.numel(), _ptr(self.ws), self.ws.numel(),
+                                               _stream(stream)), "ttcd_decode_state_init")
+        self.t = 0
+
+    def step(self, x_t, beta_t, y=None):
+        y = torch.empty_like(x_t) if y is None else y
+        _check(self.lib.ttcd_block_decode(_ptr(x_t), _ptr(beta_t), self.t, ctypes.byref(self.wc),
+                                          ctypes.byref(self.pc), _ptr(self.state),
+                                          self.state.numel(), _ptr(y), _ptr(self.ws),
+                                          self.ws.numel(), _stream(self.stream)),
+               "ttcd_block_decode")
+        self.t += 1
+        return y
+
+    def state_out(self):
+        out = torch.empty(self.p.B, self.p.d_model, self.p.d_ff, device=self.state.device,
+                          dtype=torch.float32)
+        _check(self.lib.ttcd_decode_state_read(ctypes.byref(self.pc), self.t, _ptr(self.state),
+                                               self.state.numel(), _ptr(out),
+                                               _stream(self.stream)), "ttcd_decode_state_read")
+        return out
 
 
 def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams, h_S=None,

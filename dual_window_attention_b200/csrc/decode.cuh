@@ -1,0 +1,311 @@
+// Decode: one token per sequence through the IP-TTCD block, with carried state.
+//
+// The block is causal (papernotes.org review "Learning What to Remember",
+// 方法详解: windowed attention over earlier tokens, causal short convs, an
+// exclusive prefix over chunks), so token t needs only: the K/V of the last
+// w_T tokens, the last conv_k-1 rows of Z_T and Z_S, the r_t and k'_t of the
+// current chunk (its Delta W is formed when the chunk ends), and the fast
+// weight of the current chunk, W_down + S.  These kernels are the
+// memory-bound per-token steps; the dense products run on the tcgen05 GEMM
+// and the chunk commit on the chunk-scan kernel.
+#pragma once
+#include "gemm.cuh"
+
+namespace ttcd {
+
+constexpr int DEC_KC = 256;       // keys per attention split
+constexpr int DEC_THREADS = 128;  // attention split block
+constexpr int DEC_MAXG = 8;       // query heads per KV head handled by one block
+
+// q and k rotated at position t (rotate-half RoPE, angle t * theta^(-2i/hd) in
+// double precision), k and v appended to the ring caches at slot t % W.
+// qkv [B, (Hq + 2 Hkv) hd] fp32 -> q_rot [B, Hq, hd] bf16; kc, vc [B, W, Hkv, hd].
+// grid (B, Hq + 2 Hkv), block hd / 2.
+__global__ void decode_rope_cache_kernel(const float* __restrict__ qkv,
+                                         __nv_bfloat16* __restrict__ q_rot,
+                                         __nv_bfloat16* __restrict__ kc,
+                                         __nv_bfloat16* __restrict__ vc, int Hq, int Hkv, int hd,
+                                         int t, int W, double theta) {
+  const int b = blockIdx.x, head = blockIdx.y, i = threadIdx.x;
+  const int half = hd / 2;
+  const float* src = qkv + static_cast<long long>(b) * (Hq + 2 * Hkv) * hd +
+                     static_cast<long long>(head) * hd;
+  const long long slot = t % W;
+  if (head < Hq + Hkv) {
+    double s, c;
+    sincos(static_cast<double>(t) * pow(theta, -2.0 * i / hd), &s, &c);
+    const float cf = static_cast<float>(c), sf = static_cast<float>(s);
+    const float a = src[i], bb = src[i + half];
+    __nv_bfloat16* dst = head < Hq
+                             ? q_rot + (static_cast<long long>(b) * Hq + head) * hd
+                             : kc + ((b * static_cast<long long>(W) + slot) * Hkv + (head - Hq)) * hd;
+    dst[i] = __float2bfloat16_rn(a * cf - bb * sf);
+    dst[i + half] = __float2bfloat16_rn(bb * cf + a * sf);
+  } else {
+    __nv_bfloat16* dst =
+        vc + ((b * static_cast<long long>(W) + slot) * Hkv + (head - Hq - Hkv)) * hd;
+    dst[i] = __float2bfloat16_rn(src[i]);
+    dst[i + half] = __float2bfloat16_rn(src[i + half]);
+  }
+}
+
+// Both windows of one KV head's query heads over one split of DEC_KC keys of
+// the teacher range [max(0, t-w_T+1), t]; the student window is its last w_S
+// keys.  Partial results (log2-domain max, sum, unnormalised output) per
+// (b, h, window, split): pm, pl [B, Hq, 2, nsplit], po [B, Hq, 2, nsplit, HD].
+// grid (B * Hkv, nsplit), block DEC_THREADS.
+template <int HD>
+__global__ void __launch_bounds__(DEC_THREADS)
+    decode_attn_partial_kernel(const __nv_bfloat16* __restrict__ q_rot,
+                               const __nv_bfloat16* __restrict__ kc,
+                               const __nv_bfloat16* __restrict__ vc, float* __restrict__ pm,
+                               float* __restrict__ pl, float* __restrict__ po, int Hq, int Hkv,
+                               int W, int t, int w_S, int w_T, float scale_log2, int nsplit) {
+  __shared__ float qs[DEC_MAXG][HD];
+  __shared__ float ps[2][DEC_MAXG][DEC_KC];  // scores, then probabilities per window
+  const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv, sp = blockIdx.y;
+  const int G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j_lo = max(0, t - w_T + 1);
+  const int j0 = j_lo + sp * DEC_KC;
+  const int n = max(0, min(t - j0 + 1, DEC_KC));  // keys of this split
+  const int s_lo = max(0, t - w_S + 1) - j0;      // first student key index (may be <0 or >=n)
+  for (int e = tid; e < G * HD; e += DEC_THREADS)
+    qs[e / HD][e % HD] = __bfloat162float(
+        q_rot[(static_cast<long long>(b) * Hq + g * G + e / HD) * HD + e % HD]);
+  __syncthreads();
+  // scores (log2 domain)
+  for (int kk = tid; kk < n; kk += DEC_THREADS) {
+    const long long slot = (j0 + kk) % W;
+    const uint4* krow = reinterpret_cast<const uint4*>(
+        kc + ((b * static_cast<long long>(W) + slot) * Hkv + g) * HD);
+    float acc[DEC_MAXG];
+#pragma unroll
+    for (int hh = 0; hh < DEC_MAXG; ++hh) acc[hh] = 0.f;
+#pragma unroll 4
+    for (int c8 = 0; c8 < HD / 8; ++c8) {
+      const uint4 u = krow[c8];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float k0 = bf16lo_to_f32(w4[q]), k1 = bf16hi_to_f32(w4[q]);
+#pragma unroll
+        for (int hh = 0; hh < DEC_MAXG; ++hh)
+          if (hh < G) acc[hh] += qs[hh][c8 * 8 + 2 * q] * k0 + qs[hh][c8 * 8 + 2 * q + 1] * k1;
+      }
+    }
+    for (int hh = 0; hh < G; ++hh) ps[0][hh][kk] = acc[hh] * scale_log2;
+  }
+  __syncthreads();
+  // per (head, window): maximum, probabilities, sum (one warp per pair)
+  for (int pr = warp; pr < 2 * G; pr += DEC_THREADS / 32) {
+    const int hh = pr >> 1, win = pr & 1;  // win 0: teacher, 1: student
+    const int k_first = win ? max(s_lo, 0) : 0;
+    float m = -INFINITY;
+    for (int kk = k_first + lane; kk < n; kk += 32) m = fmaxf(m, ps[0][hh][kk]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int kk = lane; kk < DEC_KC; kk += 32) {
+      const float p = (kk >= k_first && kk < n) ? exp2f(ps[0][hh][kk] - m) : 0.f;
+      if (win) ps[1][hh][kk] = p;
+      l += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      const long long pi = ((static_cast<long long>(b) * Hq + g * G + hh) * 2 + win) * nsplit + sp;
+      pm[pi] = m;
+      pl[pi] = l;
+    }
+  }
+  __syncthreads();
+  // teacher probabilities in place of the scores (the student ones are in ps[1])
+  for (int pr = warp; pr < G; pr += DEC_THREADS / 32) {
+    const long long pi = ((static_cast<long long>(b) * Hq + g * G + pr) * 2) * nsplit + sp;
+    const float m = pm[pi];
+    for (int kk = lane; kk < DEC_KC; kk += 32)
+      ps[0][pr][kk] = kk < n ? exp2f(ps[0][pr][kk] - m) : 0.f;
+  }
+  __syncthreads();
+  // P.V: one output column per thread, every head and window of the group
+  for (int d = tid; d < HD; d += DEC_THREADS) {
+    float accT[DEC_MAXG], accS[DEC_MAXG];
+#pragma unroll
+    for (int hh = 0; hh < DEC_MAXG; ++hh) accT[hh] = accS[hh] = 0.f;
+    for (int kk = 0; kk < n; ++kk) {
+      const long long slot = (j0 + kk) % W;
+      const float v = __bfloat162float(vc[((b * static_cast<long long>(W) + slot) * Hkv + g) * HD + d]);
+#pragma unroll
+      for (int hh = 0; hh < DEC_MAXG; ++hh)
+        if (hh < G) {
+          accT[hh] += ps[0][hh][kk] * v;
+          accS[hh] += ps[1][hh][kk] * v;
+        }
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      const long long base = ((static_cast<long long>(b) * Hq + g * G + hh) * 2) * nsplit + sp;
+      po[base * HD + d] = accT[hh];
+      po[(base + nsplit) * HD + d] = accS[hh];
+    }
+  }
+}
+
+// Merge the splits: o = sum_s po_s 2^(pm_s - m) / sum_s pl_s 2^(pm_s - m).
+// o [2, B, Hq * HD] bf16 (teacher rows, then student rows).  grid B * Hq * 2, block HD.
+template <int HD>
+__global__ void decode_attn_combine_kernel(const float* __restrict__ pm,
+                                           const float* __restrict__ pl,
+                                           const float* __restrict__ po,
+                                           __nv_bfloat16* __restrict__ o, int B, int Hq,
+                                           int nsplit) {
+  const int r = blockIdx.x;  // ((b * Hq + h) * 2 + win)
+  const int win = r & 1, bh = r >> 1;
+  const int b = bh / Hq, h = bh % Hq;
+  const int d = threadIdx.x;
+  float m = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, pm[static_cast<long long>(r) * nsplit + s]);
+  float l = 0.f, acc = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const long long pi = static_cast<long long>(r) * nsplit + s;
+    const float w = pm[pi] == -INFINITY ? 0.f : exp2f(pm[pi] - m);
+    l += pl[pi] * w;
+    acc += po[pi * HD + d] * w;
+  }
+  o[((static_cast<long long>(win) * B + b) * Hq + h) * HD + d] = __float2bfloat16_rn(acc / l);
+}
+
+// h_P = x + hp_P for both paths (rows 0..B-1 teacher, B..2B-1 student), the
+// student's h kept in fp32, and u_P = RMSNorm(h_P; g) in bf16.  grid 2B, block 256.
+__global__ void decode_residual_norm_kernel(const __nv_bfloat16* __restrict__ x,
+                                            const float* __restrict__ hp,
+                                            const __nv_bfloat16* __restrict__ g,
+                                            __nv_bfloat16* __restrict__ u,
+                                            float* __restrict__ hS, int B, int d, float eps) {
+  __shared__ float red[8];
+  const int r = blockIdx.x, b = r % B;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float h = __bfloat162float(x[static_cast<long long>(b) * d + c]) +
+                    hp[static_cast<long long>(r) * d + c];
+    ss += h * h;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+  const float rstd = rsqrtf(tot / d + eps);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float h = __bfloat162float(x[static_cast<long long>(b) * d + c]) +
+                    hp[static_cast<long long>(r) * d + c];
+    u[static_cast<long long>(r) * d + c] =
+        __float2bfloat16_rn(h * rstd * __bfloat162float(g[c]));
+    if (r >= B) hS[static_cast<long long>(b) * d + c] = h;
+  }
+}
+
+// One token of the short causal convs, the residual difference and the key:
+//   zbar_P = sum_m taps_P[c, m] Z_P[t-m]   (history rows t-1..t-k+1, zero before 0)
+//   D = zbar_T - zbar_S;  k' = zbar_S (unnormalised) into the chunk buffer row t % C;
+//   kscale = beta_t / sqrt(||zbar_S||^2 + eps);  Z_S also as the bf16 output operand.
+// Z [2B, f] fp32 (teacher rows first); hist [2, B, H, f] fp32 ring (slot = position % H).
+// grid B, block 256.
+__global__ void decode_conv_kernel(const float* __restrict__ Z,
+                                   const __nv_bfloat16* __restrict__ tapT,
+                                   const __nv_bfloat16* __restrict__ tapS,
+                                   float* __restrict__ hist, __nv_bfloat16* __restrict__ D,
+                                   __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Zs16,
+                                   const float* __restrict__ beta, float* __restrict__ kscale,
+                                   int B, int f, int k, int t, int C, int Cp, float eps) {
+  __shared__ float red[8];
+  const int b = blockIdx.x;
+  const int H = k > 1 ? k - 1 : 1;
+  float* hT = hist + static_cast<long long>(b) * H * f;
+  float* hSb = hist + (static_cast<long long>(B) + b) * H * f;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < f; c += blockDim.x) {
+    const float zt = Z[static_cast<long long>(b) * f + c];
+    const float zs = Z[(static_cast<long long>(B) + b) * f + c];
+    float bT = __bfloat162float(tapT[static_cast<long long>(c) * k]) * zt;
+    float bS = __bfloat162float(tapS[static_cast<long long>(c) * k]) * zs;
+    for (int m = 1; m < k; ++m) {
+      if (t - m < 0) break;
+      const long long slot = (t - m) % H;
+      bT += __bfloat162float(tapT[static_cast<long long>(c) * k + m]) * hT[slot * f + c];
+      bS += __bfloat162float(tapS[static_cast<long long>(c) * k + m]) * hSb[slot * f + c];
+    }
+    if (k > 1) {  // position t replaces position t-H, which no later token needs
+      hT[static_cast<long long>(t % H) * f + c] = zt;
+      hSb[static_cast<long long>(t % H) * f + c] = zs;
+    }
+    D[static_cast<long long>(b) * f + c] = __float2bfloat16_rn(bT - bS);
+    Kc[(static_cast<long long>(b) * Cp + t % C) * f + c] = __float2bfloat16_rn(bS);
+    Zs16[static_cast<long long>(b) * f + c] = __float2bfloat16_rn(zs);
+    ss += bS * bS;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+    kscale[b] = beta[b] / sqrtf(tot + eps);
+  }
+}
+
+// rows [B, d] -> dst rows b * Cp + row (the current chunk slot of each sequence)
+__global__ void decode_row_copy_kernel(const __nv_bfloat16* __restrict__ src,
+                                       __nv_bfloat16* __restrict__ dst, int B, int d, int Cp,
+                                       int row) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<long long>(B) * d) return;
+  const long long b = i / d, c = i % d;
+  dst[(b * Cp + row) * d + c] = src[i];
+}
+
+// y[b, i] = hS[b, i] + sum_c Weff[b, i, c] Zs[b, c]: the fast-weight read with
+// the current chunk's weight W_down + S.  One warp per output row.
+// grid (cdiv(d, 8), B), block 256.
+__global__ void decode_out_kernel(const __nv_bfloat16* __restrict__ Weff,
+                                  const __nv_bfloat16* __restrict__ Zs,
+                                  const float* __restrict__ hS, __nv_bfloat16* __restrict__ y,
+                                  int d, int f) {
+  const int b = blockIdx.y;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= d) return;
+  const uint4* wr = reinterpret_cast<const uint4*>(Weff + (static_cast<long long>(b) * d + i) * f);
+  const uint4* zr = reinterpret_cast<const uint4*>(Zs + static_cast<long long>(b) * f);
+  float acc = 0.f;
+  for (int c8 = lane; c8 < f / 8; c8 += 32) {
+    const uint4 a = wr[c8], z = zr[c8];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, zw[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      acc += bf16lo_to_f32(aw[q]) * bf16lo_to_f32(zw[q]) + bf16hi_to_f32(aw[q]) * bf16hi_to_f32(zw[q]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0)
+    y[static_cast<long long>(b) * d + i] = __float2bfloat16_rn(hS[static_cast<long long>(b) * d + i] + acc);
+}
+
+// Weff[b] = bf16(W_down + S[b]), 4 elements per thread.
+__global__ void decode_weff_kernel(const __nv_bfloat16* __restrict__ w_down,
+                                   const float* __restrict__ S, __nv_bfloat16* __restrict__ Weff,
+                                   long long df, long long n4) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const long long e = i * 4, w = e % df;
+  const float4 s = *reinterpret_cast<const float4*>(S + e);
+  const uint2 wd = *reinterpret_cast<const uint2*>(w_down + w);
+  uint2 out;
+  out.x = pack_bf16x2(bf16lo_to_f32(wd.x) + s.x, bf16hi_to_f32(wd.x) + s.y);
+  out.y = pack_bf16x2(bf16lo_to_f32(wd.y) + s.z, bf16hi_to_f32(wd.y) + s.w);
+  *reinterpret_cast<uint2*>(Weff + e) = out;
+}
+
+}  // namespace ttcd

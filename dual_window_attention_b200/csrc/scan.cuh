@@ -29,7 +29,7 @@ struct ScanArgs {
   const E* w_down;        // [d, f]
   const float* state_in;  // [B, d, f] nullable
   float* state_out;       // [B, d, f] nullable
-  E* w_all;               // [B*Nc, d, f]
+  E* w_all;               // [B*Nc, d, f], nullable (state only)
   int tiles_m, tiles_n;
 };
 
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       }
 #pragma unroll
       for (int e = 0; e < 32; ++e) S[cc + e] = s32[e];
-      if (row_ok && col < a.f) {
+      if (row_ok && col < a.f && a.w_all) {
         float w[32];
         load_x32(wrow + col, w);
 #pragma unroll
@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         if (!row_ok || col >= a.f) continue;
         float v[32];
         if (!last) {
+          if (!a.w_all) continue;
           load_x32(wrow + col, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] += S[cc + e];

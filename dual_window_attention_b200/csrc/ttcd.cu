@@ -18,6 +18,7 @@
 #include "gemm.cuh"
 #include "ptx.cuh"
 #include "scan.cuh"
+#include "decode.cuh"
 
 using namespace ttcd;
 
@@ -817,6 +818,325 @@ ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream) {
   bounded_wait_test_kernel<<<1, 32, 0, c.s>>>(st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
+}
+
+}  // extern "C"
+
+// ===================================================================== decode
+namespace {
+
+// Decode state (per sequence unless noted), 1 KiB-aligned pieces.
+struct DecState {
+  size_t kc, vc, hist, rc, kx, S, weff, M, wprojT, total;
+};
+DecState dec_state_layout(const ttcd_block_params* p) {
+  const long long B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
+  const long long W = p->w_T, H = p->conv_k > 1 ? p->conv_k - 1 : 1;
+  const long long Cp = (p->chunk + 63) / 64 * 64;
+  size_t sz[9] = {static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // K cache ring
+                  static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // V cache ring
+                  static_cast<size_t>(2 * B * H * f * 4),                // conv history
+                  static_cast<size_t>(B * Cp * d * 2),                   // r rows of the chunk
+                  static_cast<size_t>(B * Cp * f * 2),                   // k' rows of the chunk
+                  static_cast<size_t>(B * d * f * 4),                    // S
+                  static_cast<size_t>(B * d * f * 2),                    // W_down + S
+                  static_cast<size_t>(d * f * 2),                        // M (shared)
+                  static_cast<size_t>(f * f * 2)};                       // W_proj^T (shared)
+  size_t* o[9];
+  DecState L;
+  size_t* fields[9] = {&L.kc, &L.vc, &L.hist, &L.rc, &L.kx, &L.S, &L.weff, &L.M, &L.wprojT};
+  size_t off = 0;
+  for (int i = 0; i < 9; ++i) {
+    *fields[i] = off;
+    off += (sz[i] + 1023) / 1024 * 1024;
+  }
+  (void)o;
+  L.total = off;
+  return L;
+}
+
+// Per-step scratch.
+struct DecWs {
+  size_t xn, qkv, qrot, o, hp, hS, u, Z, Zs, D, ks, r, pm, pl, po, total;
+  int nsplit;
+};
+DecWs dec_ws_layout(const ttcd_block_params* p) {
+  const long long B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
+  const long long Hq = p->n_q_heads, dqkv = (p->n_q_heads + 2 * p->n_kv_heads) * hd;
+  DecWs L;
+  L.nsplit = static_cast<int>(cdiv(p->w_T, DEC_KC));
+  const long long np = B * Hq * 2 * L.nsplit;
+  const size_t sz[15] = {static_cast<size_t>(B * d * 2), static_cast<size_t>(B * dqkv * 4),
+                         static_cast<size_t>(B * Hq * hd * 2), static_cast<size_t>(2 * B * Hq * hd * 2),
+                         static_cast<size_t>(2 * B * d * 4), static_cast<size_t>(B * d * 4),
+                         static_cast<size_t>(2 * B * d * 2), static_cast<size_t>(2 * B * f * 4),
+                         static_cast<size_t>(B * f * 2), static_cast<size_t>(B * f * 2),
+                         static_cast<size_t>(B * 4), static_cast<size_t>(B * d * 2),
+                         static_cast<size_t>(np * 4), static_cast<size_t>(np * 4),
+                         static_cast<size_t>(np * hd * 4)};
+  size_t* fields[15] = {&L.xn, &L.qkv, &L.qrot, &L.o, &L.hp, &L.hS, &L.u, &L.Z, &L.Zs, &L.D,
+                        &L.ks, &L.r, &L.pm, &L.pl, &L.po};
+  size_t off = 0;
+  for (int i = 0; i < 15; ++i) {
+    *fields[i] = off;
+    off += (sz[i] + 1023) / 1024 * 1024;
+  }
+  L.total = off;
+  return L;
+}
+
+ttcd_status check_decode_params(const ttcd_block_params* p) {
+  TTCD_TRY(check_params(p));
+  if (p->dtype != TTCD_BF16) return TTCD_ERR_UNSUPPORTED;
+  if (p->n_q_heads / p->n_kv_heads > DEC_MAXG) return TTCD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->d_model * p->d_ff >= (1ll << 40)) return TTCD_ERR_UNSUPPORTED;
+  return TTCD_OK;
+}
+
+template <class T>
+T* dat(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+// S (in place) += the chunk buffers' R^T K' over their first Cp rows (rows past
+// the chunk's tokens are zero), by the chunk-scan kernel with one chunk.
+ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, const DecState& L,
+                       const __nv_bfloat16* w_down, const float* S_in, float* S_out) {
+  using bf = __nv_bfloat16;
+  const int d = p->d_model, f = p->d_ff, Cp = (p->chunk + 63) / 64 * 64;
+  CUtensorMap mR, mK;
+  constexpr uint32_t BK = ElemTraits<bf>::BK;
+  if (!make_map<bf>(&mR, dat<bf>(state, L.rc), d, static_cast<uint64_t>(p->B) * Cp, d * 2, BK, BK) ||
+      !make_map<bf>(&mK, dat<bf>(state, L.kx), f, static_cast<uint64_t>(p->B) * Cp, f * 2, BK, BK))
+    return TTCD_ERR_CUDA;
+  ScanArgs<bf> a;
+  a.d = d;
+  a.f = f;
+  a.Nc = 1;
+  a.Cp = Cp;
+  a.w_down = w_down;
+  a.state_in = S_in;
+  a.state_out = S_out;
+  a.w_all = nullptr;
+  a.tiles_m = cdiv(d, 128);
+  a.tiles_n = cdiv(f, SCAN_BN);
+  constexpr int STAGES = 4;
+  constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+  auto kern = fastweight_scan_kernel<bf, STAGES, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+ttcd_status dec_weff(const Ctx& c, const ttcd_block_params* p, void* state, const DecState& L,
+                     const __nv_bfloat16* w_down) {
+  const long long df = static_cast<long long>(p->d_model) * p->d_ff;
+  const long long n4 = p->B * df / 4;
+  decode_weff_kernel<<<static_cast<unsigned>(cdiv(n4, 256)), 256, 0, c.s>>>(
+      w_down, dat<float>(state, L.S), dat<__nv_bfloat16>(state, L.weff), df, n4);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+template <int HD>
+ttcd_status dec_attention(const Ctx& c, const ttcd_block_params* p, void* state,
+                          const DecState& S, void* ws, const DecWs& L, int t, float scale) {
+  using bf = __nv_bfloat16;
+  const int B = p->B, Hq = p->n_q_heads, Hkv = p->n_kv_heads;
+  decode_attn_partial_kernel<HD><<<dim3(B * Hkv, L.nsplit), DEC_THREADS, 0, c.s>>>(
+      dat<bf>(ws, L.qrot), dat<bf>(state, S.kc), dat<bf>(state, S.vc), dat<float>(ws, L.pm),
+      dat<float>(ws, L.pl), dat<float>(ws, L.po), Hq, Hkv, p->w_T, t, p->w_S, p->w_T,
+      scale * 1.4426950408889634f, L.nsplit);
+  TTCD_CHECK_LAUNCH();
+  decode_attn_combine_kernel<HD><<<B * Hq * 2, HD, 0, c.s>>>(
+      dat<float>(ws, L.pm), dat<float>(ws, L.pl), dat<float>(ws, L.po), dat<bf>(ws, L.o), B, Hq,
+      L.nsplit);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, int t,
+                       const ttcd_block_weights* w, const ttcd_block_params* p, void* state,
+                       const DecState& S, __nv_bfloat16* y, void* ws, const DecWs& L) {
+  using bf = __nv_bfloat16;
+  const int B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
+  const int Hq = p->n_q_heads, Hkv = p->n_kv_heads, dqkv = (Hq + 2 * Hkv) * hd;
+  const int C = p->chunk, Cp = (C + 63) / 64 * 64;
+  // input RMSNorm and Q/K/V (fp32, rotated once)
+  rmsnorm_kernel<bf, bf, bf><<<cdiv(B, 8), 256, 0, c.s>>>(
+      x, static_cast<const bf*>(w->g_attn), dat<bf>(ws, L.xn), B, d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dat<bf>(ws, L.xn), B, d, 128) ||
+        !map_rows<bf>(&mB, w->w_qkv, dqkv, d, 256) ||
+        !make_out_map<float>(&mo, dat<float>(ws, L.qkv), B, dqkv, dqkv))
+      return TTCD_ERR_CUDA;
+    EpiStore<float> e{dat<float>(ws, L.qkv), dqkv, dqkv, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(B, cdiv(dqkv, 256), d), e)));
+  }
+  decode_rope_cache_kernel<<<dim3(B, Hq + 2 * Hkv), hd / 2, 0, c.s>>>(
+      dat<float>(ws, L.qkv), dat<bf>(ws, L.qrot), dat<bf>(state, S.kc), dat<bf>(state, S.vc), Hq,
+      Hkv, hd, t, p->w_T, static_cast<double>(p->rope_theta));
+  TTCD_CHECK_LAUNCH();
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(hd));
+  switch (hd) {
+    case 32: TTCD_TRY(dec_attention<32>(c, p, state, S, ws, L, t, scale)); break;
+    case 64: TTCD_TRY(dec_attention<64>(c, p, state, S, ws, L, t, scale)); break;
+    default: TTCD_TRY(dec_attention<128>(c, p, state, S, ws, L, t, scale)); break;
+  }
+  // o_proj for both paths, residual, MLP RMSNorm
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dat<bf>(ws, L.o), 2 * B, Hq * hd, 128) ||
+        !map_rows<bf>(&mB, w->w_o, d, Hq * hd, 256) ||
+        !make_out_map<float>(&mo, dat<float>(ws, L.hp), 2 * B, d, d))
+      return TTCD_ERR_CUDA;
+    EpiStore<float> e{dat<float>(ws, L.hp), d, d, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(2 * B, cdiv(d, 256), Hq * hd), e)));
+  }
+  decode_residual_norm_kernel<<<2 * B, 256, 0, c.s>>>(x, dat<float>(ws, L.hp),
+                                                      static_cast<const bf*>(w->g_mlp),
+                                                      dat<bf>(ws, L.u), dat<float>(ws, L.hS), B,
+                                                      d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  // SwiGLU with the slow weights, both paths
+  {
+    CUtensorMap mA, mB0, mB1, mo;
+    if (!map_rows<bf>(&mA, dat<bf>(ws, L.u), 2 * B, d, 128) ||
+        !map_rows<bf>(&mB0, w->w_gate, f, d, 128) || !map_rows<bf>(&mB1, w->w_up, f, d, 128) ||
+        !make_out_map<float>(&mo, dat<float>(ws, L.Z), 2 * B, f, f))
+      return TTCD_ERR_CUDA;
+    EpiSwiGLU e{dat<float>(ws, L.Z), f, f, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * B, cdiv(f, 128), d), e)));
+  }
+  // convs, residual, key (into the chunk buffer), key scale
+  decode_conv_kernel<<<B, 256, 0, c.s>>>(dat<float>(ws, L.Z), static_cast<const bf*>(w->conv_T),
+                                         static_cast<const bf*>(w->conv_S), dat<float>(state, S.hist),
+                                         dat<bf>(ws, L.D), dat<bf>(state, S.kx), dat<bf>(ws, L.Zs),
+                                         beta, dat<float>(ws, L.ks), B, f, p->conv_k, t, C, Cp,
+                                         p->l2_eps);
+  TTCD_CHECK_LAUNCH();
+  // r = (D M^T) beta / ||zbar_S||, into the chunk buffer
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dat<bf>(ws, L.D), B, f, 128) ||
+        !map_rows<bf>(&mB, dat<bf>(state, S.M), d, f, 256) ||
+        !make_out_map<bf>(&mo, dat<bf>(ws, L.r), B, d, d))
+      return TTCD_ERR_CUDA;
+    EpiStore<bf> e{dat<bf>(ws, L.r), d, d, dat<float>(ws, L.ks)};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(B, cdiv(d, 256), f), e)));
+  }
+  decode_row_copy_kernel<<<static_cast<unsigned>(cdiv(static_cast<long long>(B) * d, 256)), 256, 0, c.s>>>(
+      dat<bf>(ws, L.r), dat<bf>(state, S.rc), B, d, Cp, t % C);
+  TTCD_CHECK_LAUNCH();
+  // output with the current chunk's weight W_down + S
+  decode_out_kernel<<<dim3(cdiv(d, 8), B), 256, 0, c.s>>>(dat<bf>(state, S.weff), dat<bf>(ws, L.Zs),
+                                                         dat<float>(ws, L.hS), y, d, f);
+  TTCD_CHECK_LAUNCH();
+  // last token of a chunk: S += this chunk's Delta W, then W_down + S
+  if (t % C == C - 1) {
+    float* Sp = dat<float>(state, S.S);
+    TTCD_TRY(dec_commit(c, p, state, S, static_cast<const bf*>(w->w_down), Sp, Sp));
+    TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down)));
+  }
+  return TTCD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttcd_decode_state_size(const ttcd_block_params* p) {
+  if (check_decode_params(p) != TTCD_OK) return 0;
+  return dec_state_layout(p).total;
+}
+
+size_t ttcd_decode_workspace_size(const ttcd_block_params* p) {
+  if (check_decode_params(p) != TTCD_OK) return 0;
+  return dec_ws_layout(p).total;
+}
+
+ttcd_status ttcd_decode_state_init(const ttcd_block_weights* w, const ttcd_block_params* p,
+                                   const float* state_in, void* state, size_t state_bytes,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_decode_params(p));
+  if (!weights_ok(w, true) || !aligned16(state) || (state_in && !aligned16(state_in)))
+    return TTCD_ERR_INVALID_ARG;
+  const DecState S = dec_state_layout(p);
+  if (state_bytes < S.total) return TTCD_ERR_WORKSPACE;
+  (void)workspace;
+  (void)ws_bytes;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c));
+  using bf = __nv_bfloat16;
+  const int d = p->d_model, f = p->d_ff;
+  if (cudaMemsetAsync(state, 0, S.total, c.s) != cudaSuccess) return TTCD_ERR_CUDA;
+  if (state_in && cudaMemcpyAsync(dat<float>(state, S.S), state_in,
+                                  static_cast<size_t>(p->B) * d * f * 4,
+                                  cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down)));
+  // M = W_down W_proj
+  dim3 tb(32, 8), tg(cdiv(f, 32), cdiv(f, 32));
+  transpose_kernel<bf, bf><<<tg, tb, 0, c.s>>>(static_cast<const bf*>(w->w_proj),
+                                               dat<bf>(state, S.wprojT), f, f);
+  TTCD_CHECK_LAUNCH();
+  CUtensorMap mA, mB, mo;
+  if (!map_rows<bf>(&mA, w->w_down, d, f, 128) ||
+      !map_rows<bf>(&mB, dat<bf>(state, S.wprojT), f, f, 256) ||
+      !make_out_map<bf>(&mo, dat<bf>(state, S.M), d, f, f))
+    return TTCD_ERR_CUDA;
+  EpiStore<bf> e{dat<bf>(state, S.M), f, f, nullptr};
+  return launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(d, cdiv(f, 256), f), e);
+}
+
+ttcd_status ttcd_block_decode(const void* x_t, const float* beta_t, int t,
+                              const ttcd_block_weights* w, const ttcd_block_params* p,
+                              void* state, size_t state_bytes, void* y, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_decode_params(p));
+  if (t < 0 || !aligned16(x_t) || !beta_t || (reinterpret_cast<uintptr_t>(beta_t) & 3u) ||
+      !aligned16(y) || !weights_ok(w, true) || !aligned16(state) || !aligned16(workspace))
+    return TTCD_ERR_INVALID_ARG;
+  const DecState S = dec_state_layout(p);
+  const DecWs L = dec_ws_layout(p);
+  if (state_bytes < S.total || ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c));
+  return run_decode(c, static_cast<const __nv_bfloat16*>(x_t), beta_t, t, w, p, state, S,
+                    static_cast<__nv_bfloat16*>(y), workspace, L);
+}
+
+ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void* state,
+                                   size_t state_bytes, float* state_out, void* stream) {
+  TTCD_TRY(check_decode_params(p));
+  if (t_next < 0 || !aligned16(state) || !aligned16(state_out)) return TTCD_ERR_INVALID_ARG;
+  const DecState S = dec_state_layout(p);
+  if (state_bytes < S.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c));
+  const int d = p->d_model, f = p->d_ff, C = p->chunk, Cp = (C + 63) / 64 * 64;
+  const int n = t_next % C;  // tokens of the current, partial chunk
+  if (n == 0) {
+    return cudaMemcpyAsync(state_out, dat<float>(state, S.S), static_cast<size_t>(p->B) * d * f * 4,
+                           cudaMemcpyDeviceToDevice, c.s) == cudaSuccess
+               ? TTCD_OK
+               : TTCD_ERR_CUDA;
+  }
+  // rows n.. of the chunk buffers still hold the previous chunk: clear them (the
+  // coming tokens of this chunk overwrite them anyway), then S + R^T K'
+  using bf = __nv_bfloat16;
+  for (int b = 0; b < p->B; ++b) {
+    if (cudaMemsetAsync(dat<bf>(state, S.rc) + (static_cast<size_t>(b) * Cp + n) * d, 0,
+                        static_cast<size_t>(Cp - n) * d * 2, c.s) != cudaSuccess ||
+        cudaMemsetAsync(dat<bf>(state, S.kx) + (static_cast<size_t>(b) * Cp + n) * f, 0,
+                        static_cast<size_t>(Cp - n) * f * 2, c.s) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+  }
+  return dec_commit(c, p, state, S, nullptr, dat<float>(state, S.S), state_out);
 }
 
 }  // extern "C"

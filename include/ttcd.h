@@ -213,6 +213,54 @@ ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const 
 /* Bytes of the fixed scratch array used by ttcd_fastweight_mlp_noalloc. */
 size_t ttcd_fastweight_mlp_noalloc_capacity(void);
 
+/*
+ * Decode: the block one token at a time, with carried state.
+ *
+ * Defines the same function as ttcd_block_forward, evaluated incrementally:
+ * the block is causal (windowed attention over earlier tokens, causal convs,
+ * an exclusive prefix over chunks), so the output for token t depends only
+ * on tokens 0..t.  A sequence of ttcd_block_decode calls at t = 0, 1, ..., T-1
+ * therefore returns the rows of ttcd_block_forward's output, and
+ * ttcd_decode_state_read after token T-1 returns its state_out.  ([REVIEW]
+ * 方法详解 and 关键设计 2: the fast weight of chunk i is W_down + the sum of
+ * the earlier chunks' Delta W; [PODCAST] cue 61: decode is not measured on the
+ * pages.)
+ *
+ * The state (caller-owned device memory, ttcd_decode_state_size bytes,
+ * 256-aligned, layout internal to the library) holds, per sequence:
+ *   - the K/V cache of the last w_T tokens (ring buffer, bf16);
+ *   - the last conv_k-1 rows of Z_T and Z_S (conv history, fp32);
+ *   - r_t and k'_t of the current chunk's tokens (bf16);
+ *   - the fast weight S (fp32 [d, f]) and W_down + S (bf16), updated when a
+ *     chunk ends, and M = W_down W_proj.
+ * The batch is B sequences decoded in lockstep (all at position t).
+ *
+ * ttcd_decode_state_init: clears the state and sets S = state_in (nullable:
+ *   zero), W_down + S and M; call before t = 0 and whenever the weights change.
+ * ttcd_block_decode: one token.
+ *   x_t     [B, d] bf16, device;  beta_t [B] fp32, device;  t >= 0, increasing
+ *           by one per call from 0;  y [B, d] bf16, device, written.
+ *   workspace >= ttcd_decode_workspace_size(p) bytes (per-step scratch).
+ *   At the last token of a chunk (t % chunk == chunk-1) the chunk's Delta W is
+ *   added to S before the call returns.
+ * ttcd_decode_state_read: the fast-weight state after tokens 0..t_next-1,
+ *   including the tokens of a partial chunk (as ttcd_block_forward's
+ *   state_out): state_out [B, d, f] fp32, device.
+ * Only TTCD_BF16 is supported (TTCD_F32 -> TTCD_ERR_UNSUPPORTED); p->T is not
+ * used.  Other errors as ttcd_block_forward.
+ */
+size_t ttcd_decode_state_size(const ttcd_block_params* p);
+size_t ttcd_decode_workspace_size(const ttcd_block_params* p);
+ttcd_status ttcd_decode_state_init(const ttcd_block_weights* w, const ttcd_block_params* p,
+                                   const float* state_in, void* state, size_t state_bytes,
+                                   void* workspace, size_t ws_bytes, void* stream);
+ttcd_status ttcd_block_decode(const void* x_t, const float* beta_t, int t,
+                              const ttcd_block_weights* w, const ttcd_block_params* p,
+                              void* state, size_t state_bytes, void* y, void* workspace,
+                              size_t ws_bytes, void* stream);
+ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void* state,
+                                   size_t state_bytes, float* state_out, void* stream);
+
 /* Workspace bytes needed by each entry point; 0 if the parameters are invalid. */
 size_t ttcd_fastweight_mlp_workspace_size(const ttcd_block_params* p);
 size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
