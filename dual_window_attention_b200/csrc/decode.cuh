@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
   __syncthreads();
   // scores (log2 domain)
   for (int kk = tid; kk < n; kk += DEC_THREADS) {
-    const long long slot = (j0 + kk) % W;
+    const long long slot = (j0 + kk) % W;  // two keys per thread: the modulo is not hot
     const uint4* krow = reinterpret_cast<const uint4*>(
         kc + ((b * static_cast<long long>(W) + slot) * Hkv + g) * HD);
     float acc[DEC_MAXG];
@@ -128,25 +128,64 @@ __global__ void __launch_bounds__(DEC_THREADS)
       ps[0][pr][kk] = kk < n ? exp2f(ps[0][pr][kk] - m) : 0.f;
   }
   __syncthreads();
-  // P.V: one output column per thread, every head and window of the group
-  for (int d = tid; d < HD; d += DEC_THREADS) {
-    float accT[DEC_MAXG], accS[DEC_MAXG];
+  // P.V with 16-byte loads: 16 threads cover a 128-column row (8 columns each),
+  // DEC_THREADS / (HD / 8) key groups take every (#groups)-th key, and the
+  // groups are summed through shared memory (reusing the score buffer).
+  {
+    constexpr int TPR = HD / 8;                 // threads per V row
+    constexpr int KG = DEC_THREADS / TPR;       // key groups
+    const int dg = tid % TPR, kg = tid / TPR;
+    float aT[DEC_MAXG][8], aS[DEC_MAXG][8];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh) accT[hh] = accS[hh] = 0.f;
-    for (int kk = 0; kk < n; ++kk) {
-      const long long slot = (j0 + kk) % W;
-      const float v = __bfloat162float(vc[((b * static_cast<long long>(W) + slot) * Hkv + g) * HD + d]);
+    for (int hh = 0; hh < DEC_MAXG; ++hh)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) aT[hh][e] = aS[hh][e] = 0.f;
+    const long long vbase = (b * static_cast<long long>(W)) * Hkv + g;
+    int slot = (j0 + kg) % W;  // ring slot of key kk = kg; advances by KG per step
+#pragma unroll 2
+    for (int kk = kg; kk < n; kk += KG) {
+      const uint4 u = *reinterpret_cast<const uint4*>(vc + ((vbase + static_cast<long long>(slot) * Hkv) * HD + dg * 8));
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      float vv[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        vv[2 * q] = bf16lo_to_f32(w4[q]);
+        vv[2 * q + 1] = bf16hi_to_f32(w4[q]);
+      }
 #pragma unroll
       for (int hh = 0; hh < DEC_MAXG; ++hh)
         if (hh < G) {
-          accT[hh] += ps[0][hh][kk] * v;
-          accS[hh] += ps[1][hh][kk] * v;
+          const float pT = ps[0][hh][kk], pS = ps[1][hh][kk];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            aT[hh][e] += pT * vv[e];
+            aS[hh][e] += pS * vv[e];
+          }
         }
+      slot += KG;
+      if (slot >= W) slot -= W;
     }
-    for (int hh = 0; hh < G; ++hh) {
-      const long long base = ((static_cast<long long>(b) * Hq + g * G + hh) * 2) * nsplit + sp;
-      po[base * HD + d] = accT[hh];
-      po[(base + nsplit) * HD + d] = accS[hh];
+    // Sum the key groups one head at a time through shared memory (the
+    // probabilities are no longer needed: ps is reused, KG * 2 * HD <= 2 * DEC_KC * DEC_MAXG).
+    float* red = &ps[0][0][0];
+#pragma unroll
+    for (int hh = 0; hh < DEC_MAXG; ++hh) {
+      if (hh >= G) break;  // G is the same for the whole block
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        red[(kg * 2 + 0) * HD + dg * 8 + e] = aT[hh][e];
+        red[(kg * 2 + 1) * HD + dg * 8 + e] = aS[hh][e];
+      }
+      __syncthreads();
+      for (int o = tid; o < 2 * HD; o += DEC_THREADS) {
+        const int win = o / HD, d = o % HD;
+        float acc = 0.f;
+        for (int q = 0; q < KG; ++q) acc += red[(q * 2 + win) * HD + d];
+        const long long base =
+            (((static_cast<long long>(b) * Hq + g * G + hh) * 2) + win) * nsplit + sp;
+        po[base * HD + d] = acc;
+      }
     }
   }
 }
@@ -209,23 +248,24 @@ __global__ void decode_residual_norm_kernel(const __nv_bfloat16* __restrict__ x,
 // One token of the short causal convs, the residual difference and the key:
 //   zbar_P = sum_m taps_P[c, m] Z_P[t-m]   (history rows t-1..t-k+1, zero before 0)
 //   D = zbar_T - zbar_S;  k' = zbar_S (unnormalised) into the chunk buffer row t % C;
-//   kscale = beta_t / sqrt(||zbar_S||^2 + eps);  Z_S also as the bf16 output operand.
+//   Z_S also as the bf16 output operand; per-block partial sums of zbar_S^2.
 // Z [2B, f] fp32 (teacher rows first); hist [2, B, H, f] fp32 ring (slot = position % H).
-// grid B, block 256.
+// grid (cdiv(f, 256), B), block 256; ssq_part [B, gridDim.x].
 __global__ void decode_conv_kernel(const float* __restrict__ Z,
                                    const __nv_bfloat16* __restrict__ tapT,
                                    const __nv_bfloat16* __restrict__ tapS,
                                    float* __restrict__ hist, __nv_bfloat16* __restrict__ D,
                                    __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Zs16,
-                                   const float* __restrict__ beta, float* __restrict__ kscale,
-                                   int B, int f, int k, int t, int C, int Cp, float eps) {
+                                   float* __restrict__ ssq_part, int B, int f, int k, int t, int C,
+                                   int Cp) {
   __shared__ float red[8];
-  const int b = blockIdx.x;
+  const int b = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int H = k > 1 ? k - 1 : 1;
-  float* hT = hist + static_cast<long long>(b) * H * f;
-  float* hSb = hist + (static_cast<long long>(B) + b) * H * f;
   float ss = 0.f;
-  for (int c = threadIdx.x; c < f; c += blockDim.x) {
+  if (c < f) {
+    float* hT = hist + static_cast<long long>(b) * H * f;
+    float* hSb = hist + (static_cast<long long>(B) + b) * H * f;
     const float zt = Z[static_cast<long long>(b) * f + c];
     const float zs = Z[(static_cast<long long>(B) + b) * f + c];
     float bT = __bfloat162float(tapT[static_cast<long long>(c) * k]) * zt;
@@ -243,7 +283,7 @@ __global__ void decode_conv_kernel(const float* __restrict__ Z,
     D[static_cast<long long>(b) * f + c] = __float2bfloat16_rn(bT - bS);
     Kc[(static_cast<long long>(b) * Cp + t % C) * f + c] = __float2bfloat16_rn(bS);
     Zs16[static_cast<long long>(b) * f + c] = __float2bfloat16_rn(zs);
-    ss += bS * bS;
+    ss = bS * bS;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -252,7 +292,90 @@ __global__ void decode_conv_kernel(const float* __restrict__ Z,
   if (threadIdx.x == 0) {
     float tot = 0.f;
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
-    kscale[b] = beta[b] / sqrtf(tot + eps);
+    ssq_part[static_cast<long long>(b) * gridDim.x + blockIdx.x] = tot;
+  }
+}
+
+// kscale[b] = beta_t[b] / sqrt(||zbar_S||^2 + eps), the partial sums added in a
+// fixed order.  grid B, block 32.
+__global__ void decode_kscale_kernel(const float* __restrict__ ssq_part, int n_part,
+                                     const float* __restrict__ beta, float* __restrict__ kscale,
+                                     float eps) {
+  const int b = blockIdx.x;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n_part; i += 32) s += ssq_part[static_cast<long long>(b) * n_part + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (threadIdx.x == 0) kscale[b] = beta[b] / sqrtf(s + eps);
+}
+
+// Y[r, n] = epi(W[n, :] . X[r, :]) for R <= DEC_GEMV_ROWS input rows: the
+// dense products of a decode step, whose few rows would leave a 128-row tensor
+// core tile nearly empty.  One warp per weight row n streams W[n] once (16-byte
+// loads) against every input row (from L1).  Epilogues: 0 fp32 store;
+// 1 silu(W[n].x) * (W2[n].x) (SwiGLU, fp32); 2 bf16 store scaled by scale[r].
+// grid cdiv(N, 8), block 256.
+constexpr int DEC_GEMV_ROWS = 16;   // rows one GEMV launch can take
+constexpr int DEC_GEMV_SWITCH = 8;  // up to this many rows the GEMV beats a 128-row GEMM tile (B200, measured)
+template <int EPI>
+__global__ void decode_gemv_kernel(const __nv_bfloat16* __restrict__ Wm,
+                                   const __nv_bfloat16* __restrict__ W2,
+                                   const __nv_bfloat16* __restrict__ X, void* __restrict__ Y,
+                                   const float* __restrict__ scale, int R, int N, int K,
+                                   long long ldy) {
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;
+  constexpr int NW = EPI == 1 ? 2 : 1;
+  float acc[NW][DEC_GEMV_ROWS];
+#pragma unroll
+  for (int q = 0; q < NW; ++q)
+#pragma unroll
+    for (int r = 0; r < DEC_GEMV_ROWS; ++r) acc[q][r] = 0.f;
+  const uint4* w1 = reinterpret_cast<const uint4*>(Wm + static_cast<long long>(n) * K);
+  const uint4* w2 = EPI == 1 ? reinterpret_cast<const uint4*>(W2 + static_cast<long long>(n) * K) : w1;
+  for (int c8 = lane; c8 < K / 8; c8 += 32) {
+    float wv[NW][8];
+#pragma unroll
+    for (int q = 0; q < NW; ++q) {
+      const uint4 u = q ? w2[c8] : w1[c8];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        wv[q][2 * e] = bf16lo_to_f32(w4[e]);
+        wv[q][2 * e + 1] = bf16hi_to_f32(w4[e]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < DEC_GEMV_ROWS; ++r) {
+      if (r >= R) break;
+      const uint4 xu = reinterpret_cast<const uint4*>(X + static_cast<long long>(r) * K)[c8];
+      const uint32_t x4[4] = {xu.x, xu.y, xu.z, xu.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = bf16lo_to_f32(x4[e]), x1 = bf16hi_to_f32(x4[e]);
+#pragma unroll
+        for (int q = 0; q < NW; ++q) acc[q][r] += wv[q][2 * e] * x0 + wv[q][2 * e + 1] * x1;
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < DEC_GEMV_ROWS; ++r) {
+    if (r >= R) break;
+#pragma unroll
+    for (int q = 0; q < NW; ++q)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[q][r] += __shfl_xor_sync(0xffffffffu, acc[q][r], o);
+    if (lane == 0) {
+      if (EPI == 0) {
+        static_cast<float*>(Y)[r * ldy + n] = acc[0][r];
+      } else if (EPI == 1) {
+        const float gg = acc[0][r];
+        static_cast<float*>(Y)[r * ldy + n] = gg / (1.0f + __expf(-gg)) * acc[NW - 1][r];
+      } else {
+        static_cast<__nv_bfloat16*>(Y)[r * ldy + n] = __float2bfloat16_rn(acc[0][r] * scale[r]);
+      }
+    }
   }
 }
 

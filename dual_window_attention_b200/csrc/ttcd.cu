@@ -857,7 +857,7 @@ DecState dec_state_layout(const ttcd_block_params* p) {
 
 // Per-step scratch.
 struct DecWs {
-  size_t xn, qkv, qrot, o, hp, hS, u, Z, Zs, D, ks, r, pm, pl, po, total;
+  size_t xn, qkv, qrot, o, hp, hS, u, Z, Zs, D, ks, r, pm, pl, po, ssq, total;
   int nsplit;
 };
 DecWs dec_ws_layout(const ttcd_block_params* p) {
@@ -866,18 +866,19 @@ DecWs dec_ws_layout(const ttcd_block_params* p) {
   DecWs L;
   L.nsplit = static_cast<int>(cdiv(p->w_T, DEC_KC));
   const long long np = B * Hq * 2 * L.nsplit;
-  const size_t sz[15] = {static_cast<size_t>(B * d * 2), static_cast<size_t>(B * dqkv * 4),
+  const size_t sz[16] = {static_cast<size_t>(B * d * 2), static_cast<size_t>(B * dqkv * 4),
                          static_cast<size_t>(B * Hq * hd * 2), static_cast<size_t>(2 * B * Hq * hd * 2),
                          static_cast<size_t>(2 * B * d * 4), static_cast<size_t>(B * d * 4),
                          static_cast<size_t>(2 * B * d * 2), static_cast<size_t>(2 * B * f * 4),
                          static_cast<size_t>(B * f * 2), static_cast<size_t>(B * f * 2),
                          static_cast<size_t>(B * 4), static_cast<size_t>(B * d * 2),
                          static_cast<size_t>(np * 4), static_cast<size_t>(np * 4),
-                         static_cast<size_t>(np * hd * 4)};
-  size_t* fields[15] = {&L.xn, &L.qkv, &L.qrot, &L.o, &L.hp, &L.hS, &L.u, &L.Z, &L.Zs, &L.D,
-                        &L.ks, &L.r, &L.pm, &L.pl, &L.po};
+                         static_cast<size_t>(np * hd * 4),
+                         static_cast<size_t>(B * cdiv(f, 256) * 4)};
+  size_t* fields[16] = {&L.xn, &L.qkv, &L.qrot, &L.o, &L.hp, &L.hS, &L.u, &L.Z, &L.Zs, &L.D,
+                        &L.ks, &L.r, &L.pm, &L.pl, &L.po, &L.ssq};
   size_t off = 0;
-  for (int i = 0; i < 15; ++i) {
+  for (int i = 0; i < 16; ++i) {
     *fields[i] = off;
     off += (sz[i] + 1023) / 1024 * 1024;
   }
@@ -968,7 +969,14 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   rmsnorm_kernel<bf, bf, bf><<<cdiv(B, 8), 256, 0, c.s>>>(
       x, static_cast<const bf*>(w->g_attn), dat<bf>(ws, L.xn), B, d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
-  {
+  // few rows (2B <= 16): warp-per-row GEMV; otherwise the tcgen05 GEMM
+  const bool gemv = 2 * B <= DEC_GEMV_SWITCH;
+  if (gemv) {
+    decode_gemv_kernel<0><<<cdiv(dqkv, 8), 256, 0, c.s>>>(
+        static_cast<const bf*>(w->w_qkv), nullptr, dat<bf>(ws, L.xn), dat<float>(ws, L.qkv),
+        nullptr, B, dqkv, d, dqkv);
+    TTCD_CHECK_LAUNCH();
+  } else {
     CUtensorMap mA, mB, mo;
     if (!map_rows<bf>(&mA, dat<bf>(ws, L.xn), B, d, 128) ||
         !map_rows<bf>(&mB, w->w_qkv, dqkv, d, 256) ||
@@ -988,7 +996,12 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
     default: TTCD_TRY(dec_attention<128>(c, p, state, S, ws, L, t, scale)); break;
   }
   // o_proj for both paths, residual, MLP RMSNorm
-  {
+  if (gemv) {
+    decode_gemv_kernel<0><<<cdiv(d, 8), 256, 0, c.s>>>(
+        static_cast<const bf*>(w->w_o), nullptr, dat<bf>(ws, L.o), dat<float>(ws, L.hp), nullptr,
+        2 * B, d, Hq * hd, d);
+    TTCD_CHECK_LAUNCH();
+  } else {
     CUtensorMap mA, mB, mo;
     if (!map_rows<bf>(&mA, dat<bf>(ws, L.o), 2 * B, Hq * hd, 128) ||
         !map_rows<bf>(&mB, w->w_o, d, Hq * hd, 256) ||
@@ -1003,7 +1016,12 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
                                                       d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
   // SwiGLU with the slow weights, both paths
-  {
+  if (gemv) {
+    decode_gemv_kernel<1><<<cdiv(f, 8), 256, 0, c.s>>>(
+        static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up), dat<bf>(ws, L.u),
+        dat<float>(ws, L.Z), nullptr, 2 * B, f, d, f);
+    TTCD_CHECK_LAUNCH();
+  } else {
     CUtensorMap mA, mB0, mB1, mo;
     if (!map_rows<bf>(&mA, dat<bf>(ws, L.u), 2 * B, d, 128) ||
         !map_rows<bf>(&mB0, w->w_gate, f, d, 128) || !map_rows<bf>(&mB1, w->w_up, f, d, 128) ||
@@ -1013,14 +1031,22 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
     TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * B, cdiv(f, 128), d), e)));
   }
   // convs, residual, key (into the chunk buffer), key scale
-  decode_conv_kernel<<<B, 256, 0, c.s>>>(dat<float>(ws, L.Z), static_cast<const bf*>(w->conv_T),
-                                         static_cast<const bf*>(w->conv_S), dat<float>(state, S.hist),
-                                         dat<bf>(ws, L.D), dat<bf>(state, S.kx), dat<bf>(ws, L.Zs),
-                                         beta, dat<float>(ws, L.ks), B, f, p->conv_k, t, C, Cp,
-                                         p->l2_eps);
+  const int n_part = cdiv(f, 256);
+  decode_conv_kernel<<<dim3(n_part, B), 256, 0, c.s>>>(
+      dat<float>(ws, L.Z), static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S),
+      dat<float>(state, S.hist), dat<bf>(ws, L.D), dat<bf>(state, S.kx), dat<bf>(ws, L.Zs),
+      dat<float>(ws, L.ssq), B, f, p->conv_k, t, C, Cp);
+  TTCD_CHECK_LAUNCH();
+  decode_kscale_kernel<<<B, 32, 0, c.s>>>(dat<float>(ws, L.ssq), n_part, beta,
+                                          dat<float>(ws, L.ks), p->l2_eps);
   TTCD_CHECK_LAUNCH();
   // r = (D M^T) beta / ||zbar_S||, into the chunk buffer
-  {
+  if (gemv) {
+    decode_gemv_kernel<2><<<cdiv(d, 8), 256, 0, c.s>>>(
+        dat<bf>(state, S.M), nullptr, dat<bf>(ws, L.D), dat<bf>(ws, L.r), dat<float>(ws, L.ks), B,
+        d, f, d);
+    TTCD_CHECK_LAUNCH();
+  } else {
     CUtensorMap mA, mB, mo;
     if (!map_rows<bf>(&mA, dat<bf>(ws, L.D), B, f, 128) ||
         !map_rows<bf>(&mB, dat<bf>(state, S.M), d, f, 256) ||

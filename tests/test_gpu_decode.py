@@ -21,6 +21,8 @@ DEC_A = BlockShape("decode_hd64", "bf16", B=2, T=300, d_model=128, n_q_heads=4, 
                    head_dim=64, d_ff=256, w_S=64, w_T=256, chunk=128, conv_k=4)
 DEC_B = BlockShape("decode_hd128_chunk96", "bf16", B=1, T=230, d_model=256, n_q_heads=4,
                    n_kv_heads=1, head_dim=128, d_ff=512, w_S=40, w_T=150, chunk=96, conv_k=3)
+# nine sequences: 2B = 18 rows take the tensor-core GEMM path instead of the GEMV
+DEC_C = DEC_A.with_(name="decode_batch9_gemm_path", B=9, T=150)
 
 
 @pytest.fixture(scope="module")
@@ -40,7 +42,7 @@ def _decode_all(ttcd, shape, inp, state_in=None):
     return torch.stack(ys, dim=1), dec.state_out(), x, w, p
 
 
-@pytest.mark.parametrize("shape", [DEC_A, DEC_B], ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", [DEC_A, DEC_B, DEC_C], ids=lambda s: s.name)
 def test_decode_matches_block_forward(ttcd, shape):
     inp = make_block_inputs(shape, seed=4)
     y, state, x, w, p = _decode_all(ttcd, shape, inp)
