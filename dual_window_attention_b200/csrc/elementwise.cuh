@@ -79,17 +79,32 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
 // cs[i][t] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
 // Frequency-major, so a warp reading one frequency for 32 consecutive tokens
 // reads 256 contiguous bytes.
+// cos/sin of t * theta^(-2i/hd) for every frequency i < hd/2 and position t < T,
+// frequency-major [hd/2][T].  One thread per frequency and run of ROPE_RUN
+// positions: one double-precision sincos at the run's start, then the angle
+// addition (cos, sin)((t+1)a) = (c cos a - s sin a, s cos a + c sin a) in double
+// precision, whose error over a run stays far below the half-precision output.
+constexpr int ROPE_RUN = 64;
 __global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double theta) {
   const int half = hd / 2;
+  const int runs = (T + ROPE_RUN - 1) / ROPE_RUN;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(T) * half) return;
-  const int i = static_cast<int>(idx / T);
-  const int t = static_cast<int>(idx % T);
-  const double inv = pow(theta, -2.0 * i / hd);
-  double s, c;
-  sincos(static_cast<double>(t) * inv, &s, &c);
-  // half precision (11-bit significand) is far below the bf16 rounding of q and k
-  cs[idx] = __floats2half2_rn(static_cast<float>(c), static_cast<float>(s));
+  if (idx >= static_cast<long long>(half) * runs) return;
+  const int i = static_cast<int>(idx / runs);
+  const int t0 = static_cast<int>(idx % runs) * ROPE_RUN;
+  const double a = pow(theta, -2.0 * i / hd);
+  double s, c, sa, ca;
+  sincos(static_cast<double>(t0) * a, &s, &c);
+  sincos(a, &sa, &ca);
+  __half2* out = cs + static_cast<long long>(i) * T + t0;
+  const int n = min(ROPE_RUN, T - t0);
+  for (int k = 0; k < n; ++k) {
+    // half precision (11-bit significand) is far below the bf16 rounding of q and k
+    out[k] = __floats2half2_rn(static_cast<float>(c), static_cast<float>(s));
+    const double c2 = c * ca - s * sa;
+    s = s * ca + c * sa;
+    c = c2;
+  }
 }
 
 // Fused short causal convolutions, residual difference and student keys.

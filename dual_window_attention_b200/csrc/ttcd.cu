@@ -677,7 +677,7 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
 
   // Rotary table, input RMSNorm.
   stage_mark(c.s, 0);
-  rope_table_kernel<<<cdiv(static_cast<long long>(p->T) * (m.hd / 2), 256), 256, 0, c.s>>>(
+  rope_table_kernel<<<cdiv(static_cast<long long>(cdiv(p->T, ROPE_RUN)) * (m.hd / 2), 256), 256, 0, c.s>>>(
       rope, p->T, m.hd, static_cast<double>(p->rope_theta));
   TTCD_CHECK_LAUNCH();
   rmsnorm_kernel<E, E, E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(
@@ -842,7 +842,6 @@ DecState dec_state_layout(const ttcd_block_params* p) {
                   static_cast<size_t>(B * d * f * 2),                    // W_down + S
                   static_cast<size_t>(d * f * 2),                        // M (shared)
                   static_cast<size_t>(f * f * 2)};                       // W_proj^T (shared)
-  size_t* o[9];
   DecState L;
   size_t* fields[9] = {&L.kc, &L.vc, &L.hist, &L.rc, &L.kx, &L.S, &L.weff, &L.M, &L.wprojT};
   size_t off = 0;
@@ -850,7 +849,6 @@ DecState dec_state_layout(const ttcd_block_params* p) {
     *fields[i] = off;
     off += (sz[i] + 1023) / 1024 * 1024;
   }
-  (void)o;
   L.total = off;
   return L;
 }

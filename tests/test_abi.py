@@ -121,3 +121,25 @@ def test_lse_form_rejects_bad_arguments_on_host(lib):
     assert f(*ok_args, 1, 256, 2, 1, 32, 65, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_INVALID_ARG
     assert f(*ok_args, 1, 256, 2, 1, 48, 16, 64, 0.0, ttcd.BF16, None) == ttcd.ERR_UNSUPPORTED
     assert f(*ok_args, 1, 256, 2, 1, 32, 16, 64, 0.0, ttcd.F32, None) == ttcd.ERR_UNSUPPORTED
+
+
+def test_decode_sizes_and_host_checks(lib):
+    p = _params(dtype=ttcd.BF16).c()
+    n_state = lib.ttcd_decode_state_size(ctypes.byref(p))
+    n_ws = lib.ttcd_decode_workspace_size(ctypes.byref(p))
+    assert n_state > 0 and n_ws > 0
+    # decode is bf16 only; more than 8 query heads per KV head are not supported
+    assert lib.ttcd_decode_state_size(ctypes.byref(_params(dtype=ttcd.F32).c())) == 0
+    assert lib.ttcd_decode_state_size(ctypes.byref(_params(dtype=ttcd.BF16, n_q_heads=16, n_kv_heads=1).c())) == 0
+    fake = 1 << 20
+    w = ttcd._Weights(*([fake] * 10))
+    dec = lib.ttcd_block_decode
+    beta = ctypes.c_void_p(fake)
+    # negative position, null input, short state, short workspace
+    assert dec(fake, beta, -1, ctypes.byref(w), ctypes.byref(p), fake, n_state, fake, fake, n_ws, None) == ttcd.ERR_INVALID_ARG
+    assert dec(None, beta, 0, ctypes.byref(w), ctypes.byref(p), fake, n_state, fake, fake, n_ws, None) == ttcd.ERR_INVALID_ARG
+    assert dec(fake, beta, 0, ctypes.byref(w), ctypes.byref(p), fake, n_state - 1, fake, fake, n_ws, None) == ttcd.ERR_WORKSPACE
+    assert dec(fake, beta, 0, ctypes.byref(w), ctypes.byref(p), fake, n_state, fake, fake, n_ws - 1, None) == ttcd.ERR_WORKSPACE
+    rd = lib.ttcd_decode_state_read
+    assert rd(ctypes.byref(p), -1, fake, n_state, fake, None) == ttcd.ERR_INVALID_ARG
+    assert rd(ctypes.byref(p), 3, fake, n_state - 1, fake, None) == ttcd.ERR_WORKSPACE
