@@ -86,7 +86,7 @@ def stage_costs(s):
     Cp = (s.chunk + 63) // 64 * 64
     P = s.B * s.n_chunks * Cp
     return [
-        ("hbm", BT * d * 2 * 2 + s.T * hd // 2 * 8),
+        ("hbm", BT * d * 2 * 2 + s.T * hd // 2 * 4),  # x in, xn out; half2 cos/sin table
         ("tensor", 2.0 * BT * d * dqkv),
         ("tensor", attention_flops(s)),
         ("tensor", 2.0 * 2 * BT * Hq * hd * d),

@@ -50,6 +50,28 @@ __device__ __forceinline__ float warp_sum(float v) {
 // RMSNorm as the block's pre-norm (papernotes.org review, 方法详解: the shared
 // backbone; the pages leave the skeleton unstated, a pre-norm decoder layer is
 // the plain reading).
+// 8 consecutive elements (16-byte aligned) into fp32 registers, one or two
+// vector loads.
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = bf16lo_to_f32(w[i]);
+    v[2 * i + 1] = bf16hi_to_f32(w[i]);
+  }
+}
+__device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0];
+  const float4 b = reinterpret_cast<const float4*>(src)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// One warp per row; rows up to RMS_CACHE * 256 columns stay in registers
+// between the sum of squares and the scaling (one pass over HBM), longer rows
+// are read again.
+constexpr int RMS_CACHE = 4;
 template <class InT, class GT, class OutT>
 __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict__ g,
                                OutT* __restrict__ out, long long rows, int d, float eps) {
@@ -57,21 +79,43 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const InT* x = in + row * d;
+  float xv[RMS_CACHE][8];
   float ss = 0.f;
-  for (int c = lane * 8; c < d; c += 256) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float v = to_f32(x[c + i]);
-      ss += v * v;
+  for (int q = 0; q < RMS_CACHE; ++q) {
+    const int c = lane * 8 + q * 256;
+    if (c < d) {
+      load8(x + c, xv[q]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss += xv[q][i] * xv[q][i];
     }
+  }
+  for (int c = lane * 8 + RMS_CACHE * 256; c < d; c += 256) {
+    float v[8];
+    load8(x + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
   }
   ss = warp_sum(ss);
   const float rs = rsqrtf(ss / d + eps);
   OutT* y = out + row * d;
-  for (int c = lane * 8; c < d; c += 256) {
-    float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = to_f32(x[c + i]) * rs * to_f32(g[c + i]);
+  for (int q = 0; q < RMS_CACHE; ++q) {
+    const int c = lane * 8 + q * 256;
+    if (c < d) {
+      float gv[8];
+      load8(g + c, gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xv[q][i] *= rs * gv[i];
+      store8(y + c, xv[q]);
+    }
+  }
+  for (int c = lane * 8 + RMS_CACHE * 256; c < d; c += 256) {
+    float v[8], gv[8];
+    load8(x + c, v);
+    load8(g + c, gv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= rs * gv[i];
     store8(y + c, v);
   }
 }
