@@ -70,6 +70,21 @@ def test_equal_windows_reduce_to_plain_swa_block():
     np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-11)
 
 
+def test_distinct_norm_gains_reduce_to_plain_swa_block():
+    """The same reduction with random, different gains for the two RMSNorms:
+    the attention norm takes g_attn, the MLP norm g_mlp (both views share it)."""
+    shape = TINY_F32.with_(w_S=40, w_T=40)
+    inp = make_block_inputs(shape, seed=2)
+    w = {k: _np(v) for k, v in inp["layers"][0].items()}
+    rng = np.random.default_rng(9)
+    w["g_attn"] = 0.5 + rng.random(shape.d_model)
+    w["g_mlp"] = 0.5 + rng.random(shape.d_model)
+    w["conv_T"] = w["conv_S"]
+    res = _block(shape, inp, **{k: w[k] for k in ("g_attn", "g_mlp", "conv_T")})
+    ref = _plain_swa_block(_np(inp["x"]), w, shape, 40)
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-11)
+
+
 def test_student_path_is_block_output_with_static_mlp_when_beta_zero():
     shape = TINY_F32
     inp = make_block_inputs(shape, seed=0)

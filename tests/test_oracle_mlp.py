@@ -159,6 +159,21 @@ def test_identity_convs_and_proj_give_down_projected_difference():
     np.testing.assert_allclose(res["R"], ref, rtol=1e-12, atol=1e-13)
 
 
+def test_value_residual_basis_probe():
+    """r is linear in the difference d_t = zbar_T - zbar_S; a unit difference e_j
+    gives column j of the map, W_down (W_proj e_j) = W_down @ W_proj[:, j] (R12),
+    and the opposite difference gives its negative (R4)."""
+    rng = np.random.default_rng(5)
+    d, f = 3, 7
+    w_down, w_proj = rng.standard_normal((d, f)), rng.standard_normal((f, f))
+    eye = np.eye(f)[None]  # token j carries e_j
+    zero = np.zeros_like(eye)
+    r = orc.value_residual(eye, zero, w_down, w_proj)[0]
+    for j in range(f):
+        np.testing.assert_allclose(r[j], w_down @ w_proj[:, j], rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(orc.value_residual(zero, eye, w_down, w_proj)[0], -r)
+
+
 @pytest.mark.parametrize("chunk", [1, 7, 16, 70, 100])
 def test_parallel_prefix_equals_sequential_recurrence(chunk):
     """Off-policy parallel form == chunk-by-chunk loop with frozen activations."""
