@@ -155,7 +155,7 @@ ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* 
  *   beta       [B, T] fp32, device
  *   state_in   [B, d, f] fp32, device, nullable;  state_out likewise
  *   y          [B, T, d] params.dtype, device, written
- *   workspace  >= ttcd_fastweight_mlp_workspace_size(p) bytes, device, 256-aligned
+ *   workspace  >= ttcd_fastweight_mlp_workspace_size(p) bytes, device, 16-byte aligned
  */
 ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,
                                 const float* beta, const ttcd_block_weights* w,
@@ -175,7 +175,7 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
  *   x, out     [B, T, d] params.dtype, device
  *   beta       [B, T] fp32, device
  *   state_out  [B, d, f] fp32, device, nullable (final fast-weight state)
- *   workspace  >= ttcd_block_forward_workspace_size(p) bytes, device, 256-aligned
+ *   workspace  >= ttcd_block_forward_workspace_size(p) bytes, device, 16-byte aligned
  * The workspace holds every intermediate after the call; their byte offsets
  * are returned by ttcd_block_workspace_offset().
  */
@@ -227,7 +227,7 @@ size_t ttcd_fastweight_mlp_noalloc_capacity(void);
  * pages.)
  *
  * The state (caller-owned device memory, ttcd_decode_state_size bytes,
- * 256-aligned, layout internal to the library) holds, per sequence:
+ * 16-byte aligned, layout internal to the library) holds, per sequence:
  *   - the K/V cache of the last w_T tokens (ring buffer, bf16);
  *   - the last conv_k-1 rows of Z_T and Z_S (conv history, fp32);
  *   - r_t and k'_t of the current chunk's tokens (bf16);
