@@ -52,6 +52,8 @@ MUTANTS = [
     # key normalisation
     ("l2norm_no_sqrt", "return z / np.sqrt(np.sum(z * z, axis=-1, keepdims=True) + eps)",
      "return z / (np.sum(z * z, axis=-1, keepdims=True) + eps)"),
+    ("l2norm_eps_dropped", "return z / np.sqrt(np.sum(z * z, axis=-1, keepdims=True) + eps)",
+     "return z / np.sqrt(np.sum(z * z, axis=-1, keepdims=True))"),
     ("key_from_teacher", "key = l2_normalize_rows(zb_S, l2_eps)", "key = l2_normalize_rows(zb_T, l2_eps)"),
     # attention
     ("window_one_too_wide", "mask = (jj <= tt) & (jj >= tt - window + 1)",
@@ -72,6 +74,10 @@ MUTANTS = [
     ("band_far_edge", "& (j[None, :] >= t[:, None] - far)", "& (j[None, :] > t[:, None] - far)"),
     ("lse_merge_weight", "w2 = np.exp(lse2 - lse)", "w2 = np.exp(lse2 - lse1)"),
     # block wiring
+    ("qkv_k_v_swapped",
+     "k = qkv[..., Hq * hd:(Hq + Hkv) * hd].reshape(B, T, Hkv, hd)\n    v = qkv[..., (Hq + Hkv) * hd:].reshape(B, T, Hkv, hd)",
+     "v = qkv[..., Hq * hd:(Hq + Hkv) * hd].reshape(B, T, Hkv, hd)\n    k = qkv[..., (Hq + Hkv) * hd:].reshape(B, T, Hkv, hd)"),
+    # block wiring
     ("student_residual_dropped", "h_S = x + o_S.reshape(B, T, Hq * hd) @ w_o.T",
      "h_S = o_S.reshape(B, T, Hq * hd) @ w_o.T"),
     ("output_from_teacher_path", "chunk, l2_eps, h_S=h_S, state_in=state_in",
@@ -91,6 +97,8 @@ MUTANTS = [
      "out[b, i] = (r[b, s0:s1] * beta[b, s0:s1, None] ** 2).T @ key[b, s0:s1]"),
     ("inclusive_prefix", "prefixes[:, i] = s\n        s = s + inc[:, i]",
      "s = s + inc[:, i]\n        prefixes[:, i] = s"),
+    ("prefix_starts_at_first_increment", "prefixes[:, i] = s\n        s = s + inc[:, i]",
+     "prefixes[:, i] = s + (inc[:, 0] if i == 0 else 0)\n        s = s + inc[:, i]"),
     ("state_in_ignored",
      "s = np.zeros((B, d, f)) if state_in is None else np.array(state_in, np.float64)",
      "s = np.zeros((B, d, f))"),
