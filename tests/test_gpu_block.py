@@ -84,12 +84,14 @@ def test_block_forward_parity_smollm2_shape(ttcd):
 
 def test_block_forward_qwen3_shape_prefix(ttcd):
     """Qwen3-0.6B-shaped block at T = 65536.  The block is causal, so its first
-    T' outputs equal the oracle run on the first T' tokens (T' = 2 chunks + a
-    ragged tail); the state of the prefix is checked on a separate T' run."""
+    T' outputs equal the oracle run on the first T' tokens.  T' = 10 chunks + a
+    ragged tail of 300: past the 8192-key teacher window, so the last 2349
+    compared rows attend over a full window and read a 10-chunk prefix.  The
+    state of the prefix is checked on a separate T' run."""
     shape = QWEN3_0P6B_64K
     inp = make_block_inputs(shape, seed=0)
     p, out, state, ws = _run(ttcd, shape, inp)
-    Tp = 2 * shape.chunk + 300
+    Tp = 10 * shape.chunk + 300
     ref = oracle_block(shape, inp, T=Tp)
     assert rel_max(out[:, :Tp], ref["out"]) <= TOL_OUT
     assert torch.isfinite(out).all() and torch.isfinite(state).all()
