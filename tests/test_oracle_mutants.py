@@ -2,10 +2,11 @@
 
 Each mutant below plants one plausible mistake in a temporary copy of the
 oracle: a dropped term, a flipped sign, an off-by-one window edge, a transposed
-or swapped operand, an inclusive prefix, a wrong GQA head. For each one the
-oracle's own pin tests (``test_oracle_attention.py``, ``test_oracle_mlp.py``,
-``test_oracle_block.py``) run against the copy, and at least one of them must
-fail. The unmutated copy must pass, which shows that the harness runs the pins
+or swapped operand, an inclusive prefix, a wrong GQA head. The forward mutants
+change ``ttcd_oracle.py``; the backward mutants change ``ttcd_oracle_grad.py``.
+For each one the oracle's own pin tests (``test_oracle_attention.py``,
+``test_oracle_mlp.py``, ``test_oracle_block.py``, ``test_oracle_grad.py``) run
+against the copy, and at least one of them must fail. The unmutated copy must pass, which shows that the harness runs the pins
 at all.
 
 The mistakes stay on the CPU, in the copy; the CUDA path is not involved.
@@ -19,7 +20,8 @@ from concurrent.futures import ThreadPoolExecutor
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PIN_FILES = ["test_oracle_attention.py", "test_oracle_mlp.py", "test_oracle_block.py"]
+PIN_FILES = ["test_oracle_attention.py", "test_oracle_mlp.py", "test_oracle_block.py",
+             "test_oracle_grad.py"]
 
 # (name, exact text in the oracle, replacement). The text must occur exactly once.
 MUTANTS = [
@@ -113,21 +115,54 @@ MUTANTS = [
 ]
 
 
-def _make_tree(dst: str, name: str, old: str, new: str) -> None:
+# Mistakes in the backward oracle: (name, exact text in ttcd_oracle_grad.py, replacement).
+GRAD_MUTANTS = [
+    ("vjp_rmsnorm_no_projection",
+     "dx = r * (dxhat - xhat * np.mean(dxhat * xhat, axis=-1, keepdims=True))", "dx = r * dxhat"),
+    ("vjp_rope_forward_rotation", "d1 * cos + d2 * sin, d2 * cos - d1 * sin",
+     "d1 * cos - d2 * sin, d2 * cos + d1 * sin"),
+    ("vjp_silu_derivative", "return s * (1.0 + a * (1.0 - s))", "return s * (1.0 - s)"),
+    ("vjp_swiglu_gate_up_swapped", "du = da @ wg + db @ wu", "du = da @ wu + db @ wg"),
+    ("vjp_conv_wrong_shift", "dz[:, :T - m, :] += taps[:, m][None, None, :] * dzbar[:, m:, :]",
+     "dz[:, m:, :] += taps[:, m][None, None, :] * dzbar[:, :T - m, :]"),
+    ("vjp_l2norm_no_projection", "return inv * (dk - k * np.sum(k * dk, axis=-1, keepdims=True))",
+     "return inv * dk"),
+    ("vjp_w_proj_transposed", "dD = dE @ wp", "dD = dE @ wp.T"),
+    ("vjp_beta_dropped", "dr[b, s0:s1] = beta[b, s0:s1, None] * rk", "dr[b, s0:s1] = rk"),
+    ("vjp_prefix_inclusive", "d_inc[:, i] = acc\n        acc = acc + d_prefixes[:, i]",
+     "acc = acc + d_prefixes[:, i]\n        d_inc[:, i] = acc"),
+    ("vjp_softmax_no_rowsum",
+     "ds = p * (dp - np.sum(do[b, :, h] * o, axis=1, keepdims=True))", "ds = p * dp"),
+    ("vjp_dk_unscaled", "dk[b, :, kh] += scale * (ds.T @ q[b, :, h])", "dk[b, :, kh] += ds.T @ q[b, :, h]"),
+    ("vjp_residual_sign", "dzb_S = dzb_S - dD", "dzb_S = dzb_S + dD"),
+    ("vjp_read_ignores_fast_weight",
+     'dZ_S[b, s0:s1] = d_out[b, s0:s1] @ (W["w_down"] + fw["S_prefix"][b, i])',
+     'dZ_S[b, s0:s1] = d_out[b, s0:s1] @ W["w_down"]'),
+    ("vjp_teacher_path_dropped_from_x", "dx = dh_T + d_hS", "dx = d_hS"),
+    ("vjp_student_window_as_teacher",
+     'windowed_attention_vjp(fw["q"], fw["k"], fw["v"], w_S, scale, do_S)',
+     'windowed_attention_vjp(fw["q"], fw["k"], fw["v"], w_T, scale, do_S)'),
+]
+ALL_MUTANTS = [(n, "ttcd_oracle.py", o, r) for n, o, r in MUTANTS] + \
+              [(n, "ttcd_oracle_grad.py", o, r) for n, o, r in GRAD_MUTANTS]
+
+
+def _make_tree(dst: str, name: str, target: str, old: str, new: str) -> None:
     """A copy of the oracle, the workload generators and the pin tests, with one mistake."""
     shutil.copytree(os.path.join(ROOT, "ttcd_workloads"), os.path.join(dst, "ttcd_workloads"),
                     ignore=shutil.ignore_patterns("__pycache__"))
-    os.makedirs(os.path.join(dst, "oracle"))
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"),
+                    ignore=shutil.ignore_patterns("__pycache__"))
     os.makedirs(os.path.join(dst, "tests"))
-    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), os.path.join(dst, "oracle"))
     for f in ["conftest.py", "helpers.py", *PIN_FILES]:
         shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests"))
-    src = open(os.path.join(ROOT, "oracle", "ttcd_oracle.py")).read()
-    if name != "unmutated":
-        assert src.count(old) == 1, f"mutant {name}: text found {src.count(old)} times"
-        src = src.replace(old, new)
-    with open(os.path.join(dst, "oracle", "ttcd_oracle.py"), "w") as f:
-        f.write(src)
+    if name == "unmutated":
+        return
+    path = os.path.join(dst, "oracle", target)
+    src = open(path).read()
+    assert src.count(old) == 1, f"mutant {name}: text found {src.count(old)} times"
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
 
 
 def _run_pins(dst: str) -> int:
@@ -140,11 +175,11 @@ def _run_pins(dst: str) -> int:
 
 @pytest.fixture(scope="module")
 def outcomes(tmp_path_factory):
-    cases = [("unmutated", "", "")] + MUTANTS
+    cases = [("unmutated", "", "", "")] + ALL_MUTANTS
     dirs = {}
-    for name, old, new in cases:
+    for name, target, old, new in cases:
         d = str(tmp_path_factory.mktemp(name))
-        _make_tree(d, name, old, new)
+        _make_tree(d, name, target, old, new)
         dirs[name] = d
     with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
         rcs = dict(zip(dirs, ex.map(_run_pins, dirs.values())))
@@ -155,7 +190,7 @@ def test_unmutated_copy_passes_its_pins(outcomes):
     assert outcomes["unmutated"] == 0
 
 
-@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+@pytest.mark.parametrize("name", [m[0] for m in ALL_MUTANTS])
 def test_pins_catch_mutant(outcomes, name):
     # pytest exits 1 when a test failed; 2-5 would mean the copy did not even run
     assert outcomes[name] == 1, f"no pin fails for the planted mistake {name!r} (rc {outcomes[name]})"
