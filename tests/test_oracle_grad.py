@@ -13,7 +13,9 @@ trained by the next-token loss).  It is pinned by:
 - reduction: with equal windows and equal convs the block is a plain
   sliding-window block (D = R = 0), so the gradients of every shared input
   equal torch autograd through a plain block built from library SDPA,
-  rms_norm and silu.
+  rms_norm and silu;
+- single steps against library autograd: the windowed GQA attention (SDPA
+  with a band mask), the causal depthwise conv (conv1d), RMSNorm and SwiGLU.
 """
 import numpy as np
 import pytest
@@ -135,3 +137,71 @@ def test_equal_windows_and_convs_reduce_to_plain_block_autograd():
     (out * torch.from_numpy(g_out)).sum().backward()
     for k in shared:
         np.testing.assert_allclose(g[k], t[k].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=k)
+
+
+# ------------------------------------------------ single steps against library autograd
+
+def _autograd(fn, *arrays, grad_out):
+    ts = [torch.tensor(a, requires_grad=True) for a in arrays]
+    (fn(*ts) * torch.from_numpy(grad_out)).sum().backward()
+    return [t.grad.numpy() for t in ts]
+
+
+@pytest.mark.parametrize("window", [1, 5, 40])
+def test_attention_vjp_matches_sdpa_autograd(window):
+    from oracle.ttcd_oracle_grad import windowed_attention_vjp
+    rng = np.random.default_rng(window)
+    b, n, hq, hkv, hd = 2, 33, 6, 2, 8
+    q, k, v = (rng.standard_normal((b, n, h, hd)) for h in (hq, hkv, hkv))
+    do = rng.standard_normal((b, n, hq, hd))
+    scale = 1.0 / np.sqrt(hd)
+    i = torch.arange(n)
+    mask = (i[None, :] <= i[:, None]) & (i[None, :] > i[:, None] - window)
+
+    def sdpa(qt, kt, vt):
+        g = hq // hkv
+        o = torch.nn.functional.scaled_dot_product_attention(
+            qt.transpose(1, 2), kt.repeat_interleave(g, 2).transpose(1, 2),
+            vt.repeat_interleave(g, 2).transpose(1, 2), attn_mask=mask, scale=scale)
+        return o.transpose(1, 2)
+
+    ref = _autograd(sdpa, q, k, v, grad_out=do)
+    got = windowed_attention_vjp(q, k, v, window, scale, do)
+    for r, g_ in zip(ref, got):
+        np.testing.assert_allclose(g_, r, rtol=1e-10, atol=1e-12)
+
+
+def test_conv_vjp_matches_conv1d_autograd():
+    from oracle.ttcd_oracle_grad import causal_depthwise_conv_vjp
+    rng = np.random.default_rng(4)
+    b, n, f, k = 2, 17, 5, 4
+    z, taps, dzbar = rng.standard_normal((b, n, f)), rng.standard_normal((f, k)), \
+        rng.standard_normal((b, n, f))
+
+    def conv(zt, wt):  # causal depthwise conv: tap m multiplies t - m
+        x = torch.nn.functional.pad(zt.transpose(1, 2), (k - 1, 0))
+        return torch.nn.functional.conv1d(x, wt.flip(-1)[:, None, :], groups=f).transpose(1, 2)
+
+    ref = _autograd(conv, z, taps, grad_out=dzbar)
+    got = causal_depthwise_conv_vjp(z, taps, dzbar)
+    for r, g_ in zip(ref, got):
+        np.testing.assert_allclose(g_, r, rtol=1e-12, atol=1e-13)
+
+
+def test_rmsnorm_and_swiglu_vjps_match_autograd():
+    from oracle.ttcd_oracle_grad import rms_norm_vjp, swiglu_vjp
+    rng = np.random.default_rng(5)
+    x, g, dy = rng.standard_normal((3, 4, 9)), 0.5 + rng.random(9), rng.standard_normal((3, 4, 9))
+    ref = _autograd(lambda xt, gt: torch.nn.functional.rms_norm(xt, (9,), gt, eps=1e-6),
+                    x, g, grad_out=dy)
+    got = rms_norm_vjp(x, g, 1e-6, dy)
+    for r, g_ in zip(ref, got):
+        np.testing.assert_allclose(g_, r, rtol=1e-12, atol=1e-13)
+    u, wg, wu = rng.standard_normal((2, 5, 6)), rng.standard_normal((7, 6)), \
+        rng.standard_normal((7, 6))
+    dz = rng.standard_normal((2, 5, 7))
+    ref = _autograd(lambda ut, a, b: torch.nn.functional.silu(ut @ a.T) * (ut @ b.T),
+                    u, wg, wu, grad_out=dz)
+    got = swiglu_vjp(u, wg, wu, dz)
+    for r, g_ in zip(ref, got):
+        np.testing.assert_allclose(g_, r, rtol=1e-12, atol=1e-13)
