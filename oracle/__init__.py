@@ -1,7 +1,8 @@
 """CPU float64 oracle of the IP-TTCD block (test infrastructure only).
 
 ``ttcd_oracle`` is the forward; ``ttcd_oracle_grad`` is its backward (a
-vector-Jacobian product of the same forward), imported explicitly.
+vector-Jacobian product of the same forward) and ``ttcd_oracle_sharded`` its
+sequence-sharded decomposition; both are imported explicitly.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
 ``--impl reference`` legs may import this package.  The CUDA library does not.

@@ -3,7 +3,9 @@
 Each mutant below plants one plausible mistake in a temporary copy of the
 oracle: a dropped term, a flipped sign, an off-by-one window edge, a transposed
 or swapped operand, an inclusive prefix, a wrong GQA head. The forward mutants
-change ``ttcd_oracle.py``; the backward mutants change ``ttcd_oracle_grad.py``.
+change ``ttcd_oracle.py``, the backward mutants ``ttcd_oracle_grad.py`` and the
+sharding mutants ``ttcd_oracle_sharded.py`` (whose pins,
+``test_oracle_sharded.py``, run for those and for the unmutated copy).
 For each one the oracle's own pin tests (``test_oracle_attention.py``,
 ``test_oracle_mlp.py``, ``test_oracle_block.py``, ``test_oracle_grad.py``) run
 against the copy, and at least one of them must fail. The unmutated copy must pass, which shows that the harness runs the pins
@@ -143,8 +145,20 @@ GRAD_MUTANTS = [
      'windowed_attention_vjp(fw["q"], fw["k"], fw["v"], w_S, scale, do_S)',
      'windowed_attention_vjp(fw["q"], fw["k"], fw["v"], w_T, scale, do_S)'),
 ]
+# Mistakes in the sequence-sharded form (ttcd_oracle_sharded.py).
+SHARD_MUTANTS = [
+    ("shard_kv_halo_one_short", "h0 = max(0, start - (w_T - 1))", "h0 = max(0, start - (w_T - 2))"),
+    ("shard_conv_halo_one_short", "c0 = max(0, start - (conv_k - 1))",
+     "c0 = max(0, start - (conv_k - 2))"),
+    ("shard_state_prefix_inclusive", "for j in range(rank):", "for j in range(rank + 1):"),
+    ("shard_rope_from_zero", "q = _rope_from(q, rope_theta, start)\n    k = _rope_from(k, rope_theta, start)",
+     "q = _rope_from(q, rope_theta, 0)\n    k = _rope_from(k, rope_theta, 0)"),
+]
 ALL_MUTANTS = [(n, "ttcd_oracle.py", o, r) for n, o, r in MUTANTS] + \
-              [(n, "ttcd_oracle_grad.py", o, r) for n, o, r in GRAD_MUTANTS]
+              [(n, "ttcd_oracle_grad.py", o, r) for n, o, r in GRAD_MUTANTS] + \
+              [(n, "ttcd_oracle_sharded.py", o, r) for n, o, r in SHARD_MUTANTS]
+# the sharded pins spawn gloo ranks; they run for the unmutated copy and the sharded mutants
+SHARD_PIN = "test_oracle_sharded.py"
 
 
 def _make_tree(dst: str, name: str, target: str, old: str, new: str) -> None:
@@ -154,7 +168,7 @@ def _make_tree(dst: str, name: str, target: str, old: str, new: str) -> None:
     shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"),
                     ignore=shutil.ignore_patterns("__pycache__"))
     os.makedirs(os.path.join(dst, "tests"))
-    for f in ["conftest.py", "helpers.py", *PIN_FILES]:
+    for f in ["conftest.py", "helpers.py", *PIN_FILES, SHARD_PIN]:
         shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests"))
     if name == "unmutated":
         return
@@ -165,10 +179,11 @@ def _make_tree(dst: str, name: str, target: str, old: str, new: str) -> None:
         f.write(src.replace(old, new))
 
 
-def _run_pins(dst: str) -> int:
+def _run_pins(dst: str, sharded: bool) -> int:
     env = dict(os.environ, OMP_NUM_THREADS="1", MKL_NUM_THREADS="1", PYTHONDONTWRITEBYTECODE="1")
+    files = PIN_FILES + ([SHARD_PIN] if sharded else [])
     cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-           *[os.path.join("tests", f) for f in PIN_FILES]]
+           *[os.path.join("tests", f) for f in files]]
     return subprocess.run(cmd, cwd=dst, env=env, stdout=subprocess.DEVNULL,
                           stderr=subprocess.DEVNULL, timeout=600).returncode
 
@@ -181,8 +196,10 @@ def outcomes(tmp_path_factory):
         d = str(tmp_path_factory.mktemp(name))
         _make_tree(d, name, target, old, new)
         dirs[name] = d
+    sharded = {name: name == "unmutated" or target == "ttcd_oracle_sharded.py"
+               for name, target, _, _ in cases}
     with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
-        rcs = dict(zip(dirs, ex.map(_run_pins, dirs.values())))
+        rcs = dict(zip(dirs, ex.map(lambda n: _run_pins(dirs[n], sharded[n]), dirs)))
     return rcs
 
 
