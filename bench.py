@@ -16,7 +16,6 @@ import datetime
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -28,11 +27,12 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from ttcd_workloads import QWEN3_0P6B_64K, make_block_inputs  # noqa: E402
+from ttcd_workloads import (ATTN_SWEEP_W_S, ATTN_SWEEP_W_T, QWEN3_0P6B_64K,  # noqa: E402
+                            make_block_inputs)
 
 METRIC = "IP-TTCD block prefill tokens/s @64K (Qwen3-0.6B shape); dual-attn % BF16 peak"
 UNIT = "tokens/s"
-STAGES = ["rope+rmsnorm_in", "qkv_gemm_rope", "dual_window_attn", "o_proj_residual_rmsstats",
+STAGES = ["rope+rms_rowscale_in", "qkv_gemm_rope", "dual_window_attn", "o_proj_residual_rmsstats",
           "gate_up_swiglu_rmsnorm", "conv_residual_keys", "M_wdown_wproj", "R_gemm",
           "chunk_scan_dW", "out_gemm"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -47,28 +47,42 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-ATTN_PROFILE = os.path.join(ROOT, "profiles", "dual_window_attn_T16384_ncu.md")
-ATTN_SOURCES = [os.path.join(ROOT, "dual_window_attention_b200", "csrc", n)
-                for n in ("attention.cuh", "ptx.cuh")]
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+CSRC = os.path.join(ROOT, "dual_window_attention_b200", "csrc")
 
 
-def recorded_attention_traffic(T: int):
-    """DRAM bytes (read + write) per attention launch at T tokens, from the
-    committed ncu summary of the 512/8192-window kernel, scaled by T (inputs,
-    outputs and the K/V stream all grow linearly in T).  None once the kernel
+def sources_digest(names) -> str:
+    """sha256 (16 hex digits) over the named kernel sources, in order."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, T: int):
+    """DRAM bytes (read + write) per launch of `kernel` at T tokens, from the ncu
+    capture recorded in profiles/ncu_traffic.json (scaled by T when the capture
+    ran at another length).  None when there is no record, or once the kernel's
     sources differ from the ones that were profiled."""
     try:
-        text = open(ATTN_PROFILE).read()
-        digests = "".join(hashlib.sha256(open(f, "rb").read()).hexdigest() for f in ATTN_SOURCES)
-    except OSError:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f)[kernel]
+        if sources_digest(rec["sources"]) != rec["sources_sha256_16"]:
+            return None
+        return float(rec["bytes_per_launch"]) * T / int(rec["T"])
+    except (OSError, KeyError, ValueError):
         return None
-    m_bytes = re.search(r"traffic_bytes_per_launch_T(\d+): (\d+)", text)
-    m_hash = re.search(r"kernel_sources_sha256_16: ([0-9a-f]+)", text)
-    if not m_bytes or not m_hash:
-        return None
-    if hashlib.sha256(digests.encode()).hexdigest()[:16] != m_hash.group(1):
-        return None
-    return float(m_bytes.group(2)) * T / int(m_bytes.group(1))
+
+
+ATTN_SWEEP_PAIRS = [(wS, wT) for wT in ATTN_SWEEP_W_T for wS in ATTN_SWEEP_W_S]
+
+
+def attention_bytes(shape) -> float:
+    """Compulsory DRAM bytes of one attention launch: q, k, v read once, o_T and
+    o_S written once (bf16)."""
+    BT, hd = shape.B * shape.T, shape.head_dim
+    return 2.0 * BT * hd * ((shape.n_q_heads + 2 * shape.n_kv_heads) + 2 * shape.n_q_heads)
 
 
 def attention_flops(shape) -> float:
@@ -86,7 +100,9 @@ def stage_costs(s):
     Cp = (s.chunk + 63) // 64 * 64
     P = s.B * s.n_chunks * Cp
     return [
-        ("hbm", BT * d * 2 * 2 + s.T * hd // 2 * 4),  # x in, xn out; half2 cos/sin table
+        # x read for the row scales (+ rstd out), W_qkv read and W_qkv diag(g) written,
+        # half2 cos/sin table written
+        ("hbm", BT * d * 2 + BT * 4 + 2 * dqkv * d * 2 + s.T * hd // 2 * 4),
         ("tensor", 2.0 * BT * d * dqkv),
         ("tensor", attention_flops(s)),
         ("tensor", 2.0 * 2 * BT * Hq * hd * d),
@@ -272,17 +288,15 @@ def run_ours(args, world, rank, local):
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
 
-    def step():
-        ttcd.block_forward(x, beta, w, p, out=out, workspace=ws, stream=stream)
+    def step(events=None):
+        ttcd.block_forward(x, beta, w, p, out=out, workspace=ws, stream=stream, events=events)
 
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize()
-    st, flags = ttcd.get_device_error()
-    if st != ttcd.OK:
-        raise RuntimeError(f"device error after warm-up: flags={flags}")
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out during warm-up")
 
-    # ---- device-timed region: K steps, stage events on the launch stream
+    # ---- device-timed region: K steps, each call recording its own stage events
     n_ev = len(STAGES) + 1
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
               for _ in range(args.steps)]
@@ -293,27 +307,25 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
-            ttcd.set_stage_events(events[i])
-            step()
+            step(events[i])
         end.record(stream)
         torch.cuda.synchronize()
-    ttcd.set_stage_events(None)
     launches = ttcd.kernel_launch_count() - launches0
     barrier(world, local)
     ms, value = job_throughput(world, shape.B * shape.T, start.elapsed_time(end) / args.steps)
-    st, flags = ttcd.get_device_error()
-    if st != ttcd.OK:
-        raise RuntimeError(f"device error in timed region: flags={flags}")
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the timed region")
     tokens = shape.B * shape.T * world
 
-    # per-stage times (mean over steps) and roofline fractions
+    # per-stage times (mean over steps) and roofline fractions.  The timed region
+    # is well under a second, so tensor stages are held to the burst GEMM peak.
     costs = stage_costs(shape)
     stage_ms = [statistics.mean(events[i][k].elapsed_time(events[i][k + 1])
                                 for i in range(args.steps)) for k in range(len(STAGES))]
     stages = {}
     for name, (bound, amt), t in zip(STAGES, costs, stage_ms):
         if bound == "tensor":
-            ach, peak, unit = amt / (t / 1e3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+            ach, peak, unit = amt / (t / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
         else:
             ach, peak, unit = amt / (t / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
         stages[name] = {"ms": round(t, 4), "bound": bound, "achieved": round(ach, 2),
@@ -368,19 +380,29 @@ def run_ours(args, world, rank, local):
     barrier(world, local)
     ms_e2e, _ = job_throughput(world, shape.B * shape.T, s2.elapsed_time(e2) / args.steps)
     assert torch.equal(out_h[(args.steps - 1) % 2], out.cpu())
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the end-to-end steps")
 
+    traffic = (args.attn_traffic_bytes if args.attn_traffic_bytes is not None
+               else recorded_traffic("dual_window_attn_kernel<128>", shape.T))
+    att_flops = attention_flops(shape)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(shape, {"parallelism": f"replicas{world}"}),
             "tflops_per_s": total_flops / (ms / 1e3) / 1e12,
             "roofline": {"kernel": "dual_window_attn_kernel<128>", "bound": "tensor",
-                         "achieved": att["achieved"], "peak": peaks["bf16_tflops_sustained"],
+                         "achieved": att["achieved"], "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": att["frac"],
-                         "traffic": (args.attn_traffic_bytes if args.attn_traffic_bytes
-                                     is not None else recorded_attention_traffic(shape.T)),
-                         "peak_source": f"{peak_kind} bf16_tflops_sustained",
-                         "flops_per_launch": attention_flops(shape)},
+                         "frac_of_sustained": round(att["achieved"] /
+                                                    peaks["bf16_tflops_sustained"], 4),
+                         "traffic": traffic,
+                         "algorithmic_bytes": attention_bytes(shape),
+                         "traffic_over_algorithmic": (round(traffic / attention_bytes(shape), 3)
+                                                      if traffic else None),
+                         "peak_source": f"{peak_kind} bf16_tflops (burst: the timed region "
+                                        f"lasts well under a second)",
+                         "flops_per_launch": att_flops},
             "stages": stages,
             "e2e": {"value": tokens / (ms_e2e / 1000.0), "unit": UNIT,
                     "h2d_bytes_per_step": x_h.numel() * x_h.element_size() +
@@ -390,6 +412,21 @@ def run_ours(args, world, rank, local):
                               "step's read-back overlap this step's compute"},
             "gpu_launches": launches,
             "clocks": clk.summary()}
+    del x, w, beta, ws, out, x_d, b_d, o_d, inp
+    torch.cuda.empty_cache()
+    if not args.no_extras:
+        # The other two workloads of the benchmark set, measured in the same run:
+        # the attention sweep (fused form at every window pair, LSE form at
+        # 512/8192) and the 28-layer stack at both batch shapes.
+        line["attention_sweep"] = [
+            measure_attention(args, world, local, wS, wT, "fused", steps=args.extra_steps,
+                              warmup=args.extra_warmup)
+            for wS, wT in ATTN_SWEEP_PAIRS] + [
+            measure_attention(args, world, local, 512, 8192, "lse", steps=args.extra_steps,
+                              warmup=args.extra_warmup)]
+        line["stack"] = [measure_stack(args, world, local, B, T, steps=max(2, args.extra_steps // 2),
+                                       warmup=args.extra_warmup)
+                         for B, T in ((1, 65536), (4, 16384))]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, times = oracle_throughput(shape, args.cpu_sample_tokens)
         line["cpu_baseline"] = {
@@ -400,58 +437,82 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_attention(args, world, rank, local):
-    """Fused dual-window attention alone (Qwen3-0.6B head layout) for each window pair."""
+_ATTN_INPUTS = {}
+
+
+def measure_attention(args, world, local, wS, wT, form, steps, warmup):
+    """Dual-window attention alone at the Qwen3-0.6B head layout (16 / 8 heads,
+    hd 128), B x T from the arguments: device time per call (CUDA events on the
+    launch stream, max over ranks) and the fraction of the burst GEMM peak."""
     import dual_window_attention_b200 as ttcd
-    from ttcd_workloads import QWEN3_0P6B_64K, make_attention_inputs
+    from ttcd_workloads import make_attention_inputs
     ttcd.load_library()
     peaks, peak_kind = load_peaks()
     s0 = QWEN3_0P6B_64K.with_(T=args.T, B=args.B)
-    q, k, v = make_attention_inputs(s0.B, s0.T, s0.n_q_heads, s0.n_kv_heads, s0.head_dim, seed=0)
-    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    key = (s0.B, s0.T, local)
+    if key not in _ATTN_INPUTS:
+        _ATTN_INPUTS.clear()
+        q, k, v = make_attention_inputs(s0.B, s0.T, s0.n_q_heads, s0.n_kv_heads, s0.head_dim,
+                                        seed=0)
+        dev = torch.device("cuda", local)
+        _ATTN_INPUTS[key] = (q.to(dev), k.to(dev), v.to(dev))
+    q, k, v = _ATTN_INPUTS[key]
     o_T, o_S = torch.empty_like(q), torch.empty_like(q)
-    pairs = [(int(a), int(b)) for a, b in (w.split("/") for w in args.windows.split(","))]
     stream = torch.cuda.current_stream()
-    lse_form = args.form == "lse"
 
-    def call(wS, wT):
-        if lse_form:
+    def call():
+        if form == "lse":
             ttcd.dual_window_attn_lse(q, k, v, wS, wT)
         else:
             ttcd.dual_window_attn(q, k, v, wS, wT, o_T=o_T, o_S=o_S)
 
+    shape = s0.with_(w_S=wS, w_T=wT)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
+    if ttcd.get_device_error()[0] != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the attention benchmark")
+    fl = attention_flops(shape)
+    ach = fl / (ms / 1e3) / 1e12
+    return {"form": form, "w_S": wS, "w_T": wT, "B": shape.B, "T": shape.T, "ms": ms,
+            "tokens_per_s": shape.B * shape.T * world / (ms / 1e3), "tflops_per_s": ach,
+            "frac": ach / peaks["bf16_tflops"],
+            "peak_source": f"{peak_kind} bf16_tflops (burst: kernel timed alone)",
+            "steps": steps, "warmup": warmup}
+
+
+def run_attention(args, world, rank, local):
+    """Dual-window attention alone (Qwen3-0.6B head layout) for each window pair."""
+    pairs = [(int(a), int(b)) for a, b in (w.split("/") for w in args.windows.split(","))]
     for wS, wT in pairs:
-        shape = s0.with_(w_S=wS, w_T=wT)
-        for _ in range(args.warmup):
-            call(wS, wT)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world, local)
-        e0.record(stream)
-        for _ in range(args.steps):
-            call(wS, wT)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
-        assert ttcd.get_device_error()[0] == ttcd.OK
-        fl = attention_flops(shape)
-        ach = fl / (ms / 1e3) / 1e12
+        r = measure_attention(args, world, local, wS, wT, args.form, args.steps, args.warmup)
         if rank == 0:
             print(json.dumps({
-                "metric": ("LSE-combination" if lse_form else "fused") +
+                "metric": ("LSE-combination" if args.form == "lse" else "fused") +
                           " dual-window attention tokens/s (Qwen3-0.6B heads)",
-                "value": shape.B * shape.T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "value": r["tokens_per_s"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "dual_window_attention", "B": shape.B, "T": shape.T,
+                "config": {"workload": "dual_window_attention", "B": r["B"], "T": r["T"],
                            "n_q_heads": 16, "n_kv_heads": 8, "head_dim": 128, "w_S": wS,
                            "w_T": wT},
-                "roofline": {"kernel": "dual_window_attn_kernel<128>" + (" + lse_merge_kernel" if lse_form else ""),
-                             "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": ach / peaks["bf16_tflops"],
-                             "peak_source": f"{peak_kind} bf16_tflops (burst: kernel timed alone)",
-                             "flops_per_launch": fl}}), flush=True)
+                "roofline": {"kernel": "dual_window_attn_kernel<128>" +
+                                       (" + lse_merge_kernel" if args.form == "lse" else ""),
+                             "bound": "tensor", "achieved": r["tflops_per_s"],
+                             "peak": load_peaks()[0]["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": r["frac"], "peak_source": r["peak_source"],
+                             "flops_per_launch": attention_flops(
+                                 QWEN3_0P6B_64K.with_(T=r["T"], B=r["B"], w_S=wS, w_T=wT))}}),
+                  flush=True)
 
 
 def run_decode_bench(args, world, rank, local):
@@ -489,7 +550,8 @@ def run_decode_bench(args, world, rank, local):
         torch.cuda.synchronize()
     launches = ttcd.kernel_launch_count() - launches0
     ms, value = job_throughput(world, args.B * args.steps, e0.elapsed_time(e1))
-    assert ttcd.get_device_error()[0] == ttcd.OK
+    if dec.check_status() != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the decode benchmark")
     s_ = shape
     dqkv = (s_.n_q_heads + 2 * s_.n_kv_heads) * s_.head_dim
     shared = 2 * (dqkv * s_.d_model + s_.d_model * s_.n_q_heads * s_.head_dim +
@@ -512,20 +574,20 @@ def run_decode_bench(args, world, rank, local):
             "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
 
 
-def run_stack(args, world, rank, local):
-    """The 28-layer stack of Qwen3-0.6B-shaped blocks, end-to-end prefill tokens/s
-    (B 1 x T 65536 by default, or --B 4 --T 16384): every layer one ttcd_block_forward
-    call on its own weights, one shared workspace."""
+def measure_stack(args, world, local, B, T, steps, warmup):
+    """The 28-layer stack of Qwen3-0.6B-shaped blocks end to end (B x T): every
+    layer one ttcd_block_forward on its own weights, one shared workspace."""
     import dual_window_attention_b200 as ttcd
     from ttcd_workloads import QWEN3_STACK_B1, QWEN3_STACK_B4
     ttcd.load_library()
-    base = QWEN3_STACK_B4 if (args.B, args.T) == (4, 16384) else QWEN3_STACK_B1
-    shape = base if (args.B, args.T) == (base.B, base.T) else base.with_(
-        name=f"qwen3_0.6b_stack28_B{args.B}_T{args.T}", B=args.B, T=args.T)
+    base = QWEN3_STACK_B4 if (B, T) == (4, 16384) else QWEN3_STACK_B1
+    shape = base if (B, T) == (base.B, base.T) else base.with_(
+        name=f"qwen3_0.6b_stack28_B{B}_T{T}", B=B, T=T)
     dev = torch.device("cuda", local)
     inp = make_block_inputs(shape, seed=0)
     x = inp["x"].to(dev)
     layers = [{k: v.to(dev) for k, v in lw.items()} for lw in inp["layers"]]
+    del inp
     p = ttcd.BlockParams.from_shape(shape)
     ws = ttcd.alloc_workspace(ttcd.block_forward_workspace_size(p), dev)
     stream = torch.cuda.current_stream()
@@ -533,37 +595,49 @@ def run_stack(args, world, rank, local):
     def step():
         return ttcd.block_stack_forward(x, layers, p, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
-    torch.cuda.synchronize()
-    assert ttcd.get_device_error()[0] == ttcd.OK
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out during the stack warm-up")
     barrier(world, local)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ttcd.kernel_launch_count()
     with ClockSampler(local) as clk:
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
     launches = ttcd.kernel_launch_count() - launches0
     barrier(world, local)
-    ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
-    assert ttcd.get_device_error()[0] == ttcd.OK
+    ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the stack benchmark")
     flops = shape.n_layers * sum(a for b, a in stage_costs(shape) if b == "tensor")
+    del x, layers, ws
+    torch.cuda.empty_cache()
+    return {"workload": shape.name, "B": shape.B, "T": shape.T, "n_layers": shape.n_layers,
+            "ms_per_pass": ms, "tokens_per_s": shape.B * shape.T * world / (ms / 1e3),
+            "tflops_per_s": flops / (ms / 1e3) / 1e12, "steps": steps, "warmup": warmup,
+            "gpu_launches": launches, "clocks": clk.summary()}
+
+
+def run_stack(args, world, rank, local):
+    """The 28-layer stack of Qwen3-0.6B-shaped blocks, end-to-end prefill tokens/s
+    (B 1 x T 65536 by default, or --B 4 --T 16384)."""
+    r = measure_stack(args, world, local, args.B, args.T, args.steps, args.warmup)
     if rank == 0:
         print(json.dumps({
             "metric": "IP-TTCD 28-layer stack prefill tokens/s (Qwen3-0.6B shape)",
-            "value": shape.B * shape.T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "value": r["tokens_per_s"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_pass"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": workload_config(shape, {"n_layers": shape.n_layers,
-                                              "parallelism": f"replicas{world}"}),
-            "tflops_per_s": flops / (ms / 1e3) / 1e12,
-            "gpu_launches": launches,
-            "clocks": clk.summary()}), flush=True)
+            "config": {"workload": r["workload"], "B": r["B"], "T": r["T"],
+                       "n_layers": r["n_layers"], "parallelism": f"replicas{world}"},
+            "tflops_per_s": r["tflops_per_s"], "gpu_launches": r["gpu_launches"],
+            "clocks": r["clocks"]}), flush=True)
 
 
 def main():
@@ -588,6 +662,11 @@ def main():
                     help="--mode attn: fused kernel, or student window + far band merged by LSE")
     ap.add_argument("--attn-traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="block mode: skip the attention sweep and the 28-layer stack")
+    ap.add_argument("--extra-steps", type=int, default=5,
+                    help="timed calls per attention window pair / stack shape")
+    ap.add_argument("--extra-warmup", type=int, default=3)
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -74,6 +74,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_decode_state_read.argtypes = [P, i, vp, sz, vp, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
+    lib.ttcd_block_forward_profiled.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp,
+                                                ctypes.POINTER(ctypes.c_void_p), i]
+    lib.ttcd_check_device_status.argtypes = [vp, vp]
     lib.ttcd_fastweight_mlp_workspace_size.argtypes = [P]
     lib.ttcd_fastweight_mlp_workspace_size.restype = sz
     lib.ttcd_block_forward_workspace_size.argtypes = [P]
@@ -82,20 +85,22 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
     lib.ttcd_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.ttcd_set_wait_timeout_ns.restype = None
-    lib.ttcd_test_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+    lib.ttcd_test_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
+    lib.ttcd_test_exp2_poly.argtypes = [vp, vp, i, vp]
+    lib.ttcd_test_exp2_poly.restype = i
     lib.ttcd_status_string.argtypes = [i]
     lib.ttcd_status_string.restype = ctypes.c_char_p
     lib.ttcd_version.restype = ctypes.c_char_p
-    lib.ttcd_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
-    lib.ttcd_set_stage_events.restype = i
     lib.ttcd_kernel_launch_count.argtypes = []
     lib.ttcd_kernel_launch_count.restype = ctypes.c_ulonglong
     lib.ttcd_fastweight_mlp_noalloc.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp]
     lib.ttcd_fastweight_mlp_noalloc.restype = i
     lib.ttcd_fastweight_mlp_noalloc_capacity.argtypes = []
     lib.ttcd_fastweight_mlp_noalloc_capacity.restype = sz
-    for fn in ("ttcd_dual_window_attn", "ttcd_fastweight_mlp", "ttcd_block_forward",
-               "ttcd_block_workspace_offset", "ttcd_get_device_error", "ttcd_test_bounded_wait"):
+    for fn in ("ttcd_dual_window_attn", "ttcd_dual_window_attn_lse", "ttcd_fastweight_mlp",
+               "ttcd_block_forward", "ttcd_block_forward_profiled", "ttcd_block_workspace_offset",
+               "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
+               "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read"):
         getattr(lib, fn).restype = i
     _lib = lib
     return lib
@@ -237,14 +242,25 @@ def workspace_view(ws: torch.Tensor, p: BlockParams, name: str, dtype: torch.dty
     return ws[off:off + nbytes].view(dtype).view(*shape)
 
 
+STATUS_BYTES = 256  # TTCD_STATUS_BYTES: the status word's region at the start of a workspace
+
+
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    """A workspace with its status region cleared (the library reads and clears
+    the status word; it never initialises it)."""
+    ws = torch.empty(max(nbytes, STATUS_BYTES), dtype=torch.uint8, device=device)
+    ws[:STATUS_BYTES].zero_()
+    return ws
 
 
 def block_forward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, out=None,
                   state_out: bool = False, workspace: Optional[torch.Tensor] = None,
-                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
-    """One IP-TTCD block forward.  Returns (out, state_out or None, workspace)."""
+                  stream=None, events=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
+    """One IP-TTCD block forward.  Returns (out, state_out or None, workspace).
+
+    ``events``: optional torch.cuda.Event objects recorded at the stage boundaries
+    of this call (ttcd_block_forward_profiled).  Timeouts are recorded in the
+    workspace's status word: read them with ``check_device_status(workspace)``."""
     lib = load_library()
     need = block_forward_workspace_size(p)
     if need == 0:
@@ -255,10 +271,21 @@ def block_forward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, out
     st_t = (torch.empty(p.B, p.d_model, p.d_ff, device=x.device, dtype=torch.float32)
             if state_out else None)
     pc, wc = p.c(), _weights(weights)
-    st = lib.ttcd_block_forward(_ptr(x), _ptr(beta), ctypes.byref(wc), ctypes.byref(pc),
-                                _ptr(st_t), _ptr(out), _ptr(workspace), workspace.numel(),
-                                _stream(stream))
-    _check(st, "ttcd_block_forward")
+    if events:
+        for e in events:  # torch creates the underlying CUDA event on first record
+            if not e.cuda_event:
+                e.record()
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        st = lib.ttcd_block_forward_profiled(_ptr(x), _ptr(beta), ctypes.byref(wc),
+                                             ctypes.byref(pc), _ptr(st_t), _ptr(out),
+                                             _ptr(workspace), workspace.numel(), _stream(stream),
+                                             arr, len(events))
+        _check(st, "ttcd_block_forward_profiled")
+    else:
+        st = lib.ttcd_block_forward(_ptr(x), _ptr(beta), ctypes.byref(wc), ctypes.byref(pc),
+                                    _ptr(st_t), _ptr(out), _ptr(workspace), workspace.numel(),
+                                    _stream(stream))
+        _check(st, "ttcd_block_forward")
     return out, st_t, workspace
 
 
@@ -324,6 +351,10 @@ class Decoder:
         self.t += 1
         return y
 
+    def check_status(self) -> int:
+        """Status of the decode calls so far (reads and clears the state's word)."""
+        return check_device_status(self.state, self.stream)
+
     def state_out(self):
         out = torch.empty(self.p.B, self.p.d_model, self.p.d_ff, device=self.state.device,
                           dtype=torch.float32)
@@ -358,12 +389,20 @@ def fastweight_mlp_noalloc(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: 
                            h_S=None, state_in=None, state_out=None, y=None, stream=None):
     """ttcd_fastweight_mlp without a workspace: for callers that cannot allocate scratch.
 
-    The scratch is the library's fixed 32 MiB device array; larger problems are
-    rejected.  Outputs `y` and `state_out` (fp32 [B, d, f]) are the caller's
-    tensors when given.  Calls that overlap on the GPU race on the shared array.
-    Returns (y, state_out).
+    The library's scratch is its fixed 32 MiB device array; larger problems are
+    rejected.  The outputs are ordinary tensors: ``y`` ([B, T, d], the type of
+    u) and ``state_out`` (fp32 [B, d, f], or True to have one allocated) are
+    the caller's when given, and this wrapper allocates ``y`` when it is None
+    (a caller that may not allocate passes its own).  Calls that overlap on the
+    GPU race on the shared array.  Returns (y, state_out or None).
     """
     lib = load_library()
+    if y is None:
+        y = torch.empty_like(u_S)
+    if state_out is True:
+        state_out = torch.empty(p.B, p.d_model, p.d_ff, device=u_S.device, dtype=torch.float32)
+    elif state_out is False:
+        state_out = None
     pc, wc = p.c(), _weights(weights)
     st = lib.ttcd_fastweight_mlp_noalloc(_ptr(u_T), _ptr(u_S), _ptr(h_S), _ptr(beta),
                                          ctypes.byref(wc), ctypes.byref(pc), _ptr(state_in),
@@ -372,8 +411,16 @@ def fastweight_mlp_noalloc(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: 
     return y, state_out
 
 
+def check_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Status of the calls that used this workspace (or decode state) since the
+    last check: OK or ERR_TIMEOUT.  Reads and clears its status word; synchronises."""
+    return load_library().ttcd_check_device_status(_ptr(workspace), _stream(stream))
+
+
 def get_device_error(stream=None) -> Tuple[int, int]:
-    """(status, raw flags) of the device error word; clears it.  Synchronises."""
+    """(status, raw flags) of the per-device status word of the entry points
+    without a workspace (attention, the MLP without scratch); clears it.
+    Synchronises."""
     flags = ctypes.c_uint32(0)
     st = load_library().ttcd_get_device_error(ctypes.byref(flags), _stream(stream))
     return st, flags.value
@@ -383,21 +430,20 @@ def set_wait_timeout_ns(ns: int) -> None:
     load_library().ttcd_set_wait_timeout_ns(ns)
 
 
-def set_stage_events(events) -> None:
-    """Record torch.cuda.Event objects at the block's stage boundaries (None = off)."""
-    if not events:
-        _check(load_library().ttcd_set_stage_events(None, 0), "set_stage_events")
-        return
-    for e in events:  # torch creates the underlying CUDA event on first record
-        if not e.cuda_event:
-            e.record()
-    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
-    _check(load_library().ttcd_set_stage_events(arr, len(events)), "set_stage_events")
-
-
 def kernel_launch_count() -> int:
     return int(load_library().ttcd_kernel_launch_count())
 
 
-def test_bounded_wait(timeout_ns: int, stream=None) -> int:
-    return load_library().ttcd_test_bounded_wait(timeout_ns, _stream(stream))
+def test_bounded_wait(timeout_ns: int, status: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Self-test of the bounded waits: a wait that nothing ends gives up after
+    ``timeout_ns`` and records a timeout in ``status`` (a workspace or decode
+    state) or, when None, in the per-device word."""
+    return load_library().ttcd_test_bounded_wait(timeout_ns, _ptr(status), _stream(stream))
+
+
+def test_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The attention kernel's FMA-pipe 2^x evaluated at x (fp32 CUDA tensor)."""
+    y = torch.empty_like(x)
+    _check(load_library().ttcd_test_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "ttcd_test_exp2_poly")
+    return y

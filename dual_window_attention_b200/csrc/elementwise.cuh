@@ -120,6 +120,55 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   }
 }
 
+// rstd[r] = (mean(in[r, :]^2) + eps)^(-1/2): the input RMSNorm as a per-row
+// scale, applied in the QKV GEMM epilogue (the block's pre-norm; papernotes.org
+// review, 方法详解, shared backbone; the skeleton is a reading, see the oracle).
+// One warp per row, 16-byte loads, d a multiple of 8.
+template <class InT>
+__global__ void rms_rowscale_kernel(const InT* __restrict__ in, float* __restrict__ rstd,
+                                    long long rows, int d, float eps) {
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const InT* x = in + row * d;
+  float ss = 0.f;
+  for (int c = lane * 8; c < d; c += 256) {
+    float v[8];
+    load8(x + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) rstd[row] = rsqrtf(ss / d + eps);
+}
+
+// out[r, c] = w[r, c] * g[c] for a row-major [rows, cols] weight, 8 elements per
+// thread (cols a multiple of 8): the RMSNorm gain folded into the next GEMM's
+// weight, (x * g) W^T = x (W diag g)^T.  n8 = rows * cols / 8.
+template <class E>
+__global__ void scale_cols_kernel(const E* __restrict__ w, const E* __restrict__ g,
+                                  E* __restrict__ out, long long n8, int cols) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const long long e0 = i * 8;
+  const int c = static_cast<int>(e0 % cols);
+  float v[8], gv[8];
+  load8(w + e0, v);
+  load8(g + c, gv);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] *= gv[k];
+  store8(out + e0, v);
+}
+
+// out[i] = OutT(in[i]), grid-stride (bf16 <-> fp32 conversions of interface tensors).
+template <class InT, class OutT>
+__global__ void cast_kernel(const InT* __restrict__ in, OutT* __restrict__ out, long long n) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += stride)
+    out[i] = from_f32<OutT>(to_f32(in[i]));
+}
+
 // cs[i][t] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
 // Frequency-major, so a warp reading one frequency for 32 consecutive tokens
 // reads 256 contiguous bytes.

@@ -561,7 +561,10 @@ struct EpiQKVRope {
   int n_rope;     // (Hq + Hkv) * HD: columns that get the rotation
   int T;
   const __half2* rope_cs;  // [HD/2][T] (cos, sin), frequency-major
-  __device__ float pre(const TileCtx&, int) const { return 1.f; }
+  const float* rstd;       // [rows] input RMSNorm row scale (the gain is in the weight), nullable
+  __device__ float pre(const TileCtx& c, int r) const {
+    return (rstd && r < c.valid_rows) ? __ldg(rstd + c.row0 + r) : 1.f;
+  }
 
   // (x_i, x_{i+NF}) -> (x_i c - x_{i+NF} s, x_{i+NF} c + x_i s) for NF frequencies
   // starting at f0, in place.
@@ -582,7 +585,7 @@ struct EpiQKVRope {
   }
 
   template <int BN>
-  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float) const {
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     static_assert(BN % 64 == 0 && BN % HD == 0, "column tile must hold whole heads");
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
@@ -626,6 +629,11 @@ struct EpiQKVRope {
       float lo[32], hi[32];
       tmem_ld32f(taddr + cc, lo);
       tmem_ld32f(taddr + cc + 32, hi);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {  // the rotation is linear: the row scale commutes with it
+        lo[i] *= rs;
+        hi[i] *= rs;
+      }
       emit(stg, staged, ok, qkv + row * ld, tcol + cc, c.row0 + wrow, lo, hi);
     }
   }

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -23,9 +24,17 @@
 using namespace ttcd;
 
 // ------------------------------------------------------------------ device state
+// Status word of the entry points that take no workspace (the two attention
+// calls, the MLP without caller scratch, the bounded-wait self-test without a
+// status region): one per device, shared by every caller of those entry points.
+// Entry points with a workspace or a decode state keep their status word in its
+// first bytes instead (kStatusBytes), so concurrent callers never see each
+// other's timeouts.
 __device__ uint32_t g_ttcd_err;
 
 namespace {
+
+constexpr size_t kStatusBytes = TTCD_STATUS_BYTES;
 
 constexpr int kMaxDevices = 64;
 uint64_t g_timeout_ns = 2000000000ull;
@@ -62,21 +71,37 @@ bool init_device(int dev) {
   return true;
 }
 
+constexpr int kMaxStageEvents = 16;
+
+// Everything one call needs to launch: device, stream, where its kernels record
+// a timeout, and (profiled calls only) the caller's stage-boundary events.
 struct Ctx {
   int dev;
   cudaStream_t s;
   DevStatus st;
   int sms;
+  cudaEvent_t const* events;
+  int n_events;
 };
 
-ttcd_status make_ctx(void* stream, Ctx& c) {
+// `status` is the call's status word (the first word of its workspace or decode
+// state), or null for the per-device word of the entry points without one.
+ttcd_status make_ctx(void* stream, Ctx& c, void* status = nullptr) {
   if (cudaGetDevice(&c.dev) != cudaSuccess) return TTCD_ERR_CUDA;
   if (!init_device(c.dev)) return TTCD_ERR_CUDA;
   c.s = static_cast<cudaStream_t>(stream);
-  c.st.err = g_err_ptr[c.dev];
+  c.st.err = status ? static_cast<uint32_t*>(status) : g_err_ptr[c.dev];
   c.st.timeout_ns = g_timeout_ns;
   c.sms = g_num_sms[c.dev];
+  c.events = nullptr;
+  c.n_events = 0;
   return TTCD_OK;
+}
+
+// Records the caller's stage-boundary event `k` on the call's stream (profiled
+// calls only).  A failed record is not a launch error: it is cleared and skipped.
+void stage_mark(const Ctx& c, int k) {
+  if (k < c.n_events && cudaEventRecord(c.events[k], c.s) != cudaSuccess) cudaGetLastError();
 }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -104,16 +129,8 @@ bool map_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
   return make_map<E>(m, ptr, cols, rows, cols * sizeof(E), ElemTraits<E>::BK, box_rows);
 }
 
+// Process-wide diagnostic counter of kernel launches (atomic; not call state).
 std::atomic<unsigned long long> g_launches{0};
-constexpr int kMaxStageEvents = 16;
-cudaEvent_t g_stage_events[kMaxStageEvents];
-int g_n_stage_events = 0;
-
-// Records the stage-boundary event `k` on stream s when profiling hooks are set.
-void stage_mark(cudaStream_t s, int k) {
-  if (k < g_n_stage_events && cudaEventRecord(g_stage_events[k], s) != cudaSuccess)
-    cudaGetLastError();  // a failed profiling record must not be reported as a launch error
-}
 
 #define TTCD_CHECK_LAUNCH()                                      \
   do {                                                           \
@@ -184,16 +201,46 @@ ttcd_status check_params(const ttcd_block_params* p) {
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-  size_t off[24];
+  size_t off[32];
   size_t total;
 };
 enum Buf {
-  B_XN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ, B_KSCALE, B_R,
-  B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_RSTD, B_COUNT
+  B_STATUS, B_WQKVG, B_RSTDIN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ,
+  B_KSCALE, B_R, B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_RSTD, B_X32, B_OUT32, B_HS32,
+  B_W32, B_COUNT
 };
-const char* kBufNames[B_COUNT] = {"xn", "qkv", "o", "h", "rope", "u", "Z", "Zs16", "D",
-                                  "Kp", "ssq", "kscale", "R", "Wall", "M", "WprojT", "Rt", "Kt", "hssq",
-                                  "rstd"};
+static_assert(B_COUNT <= 32, "workspace layout table too small");
+const char* kBufNames[B_COUNT] = {"status", "wqkv_g", "rstd_in", "qkv", "o", "h", "rope", "u",
+                                  "Z", "Zs16", "D", "Kp", "ssq", "kscale", "R", "Wall", "M",
+                                  "WprojT", "Rt", "Kt", "hssq", "rstd", "x32", "out32", "hS32",
+                                  "w32"};
+
+// bf16 problems shorter than one chunk run with fp32 operands (kind::tf32 MMAs):
+// their fast-weight state is the sum of fewer than C rank-1 writes, so the bf16
+// rounding of the MLP input and of D, M, R, K' does not average out over the
+// chunk.  Inputs and weights are widened exactly into the workspace, the output
+// is rounded back to bf16 once.
+bool wide_mode(const ttcd_block_params* p) { return p->dtype == TTCD_BF16 && p->T < p->chunk; }
+
+// fp32 copies of the weights for the wide route, in ttcd_block_weights order.
+struct W32Layout {
+  size_t off[10];
+  size_t total;
+};
+W32Layout w32_layout(const ttcd_block_params* p) {
+  const size_t d = p->d_model, f = p->d_ff, hd = p->head_dim;
+  const size_t dqkv = (p->n_q_heads + 2 * p->n_kv_heads) * hd, dq = p->n_q_heads * hd;
+  const size_t n[10] = {dqkv * d, d * dq, d, d, f * d, f * d, d * f, f * f,
+                        f * p->conv_k, f * p->conv_k};
+  W32Layout L;
+  size_t o = 0;
+  for (int i = 0; i < 10; ++i) {
+    L.off[i] = o;
+    o += (n[i] * 4 + 255) / 256 * 256;
+  }
+  L.total = o;
+  return L;
+}
 
 struct Dims {
   long long BT, P;
@@ -215,13 +262,17 @@ Dims dims_of(const ttcd_block_params* p) {
 }
 
 // Operand buffers hold bf16 for TTCD_BF16 and fp32 (tf32 tensor-core operands)
-// for TTCD_F32; q, k, v stay bf16 (the attention kernel takes bf16).
+// for TTCD_F32 and the wide route; q, k, v stay bf16 (the attention kernel takes
+// bf16).  The status word comes first in every workspace.
 Layout make_layout(const ttcd_block_params* p, bool block) {
   const Dims m = dims_of(p);
   size_t sz[B_COUNT] = {0};
-  const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
+  const bool wide = wide_mode(p);
+  const size_t e = (p->dtype == TTCD_F32 || wide) ? 4 : 2;
+  sz[B_STATUS] = kStatusBytes;
   if (block) {
-    sz[B_XN] = m.BT * m.d * e;
+    sz[B_WQKVG] = static_cast<size_t>(m.dqkv) * m.d * e;  // W_qkv diag(g_attn)
+    sz[B_RSTDIN] = m.BT * 4;                              // input RMSNorm row scales
     sz[B_QKV] = m.BT * m.dqkv * 2;
     sz[B_O] = 2 * m.BT * m.Hq * m.hd * e;
     sz[B_H] = m.BT * m.d * 4;                        // student residual stream, fp32
@@ -243,6 +294,12 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
   if (e == 4) {  // tf32 operands stay K-major: transposed copies for the chunk scan
     sz[B_RT] = m.P * m.d * e;
     sz[B_KT] = m.P * m.f * e;
+  }
+  if (wide) {  // fp32 copies of the bf16 interface tensors
+    if (block) sz[B_X32] = m.BT * m.d * 4;
+    else sz[B_HS32] = m.BT * m.d * 4;
+    sz[B_OUT32] = m.BT * m.d * 4;
+    sz[B_W32] = w32_layout(p).total;
   }
   Layout L;
   size_t o = 0;
@@ -361,7 +418,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   E* Wall = at<E>(ws, L, B_WALL);
   E* M = at<E>(ws, L, B_M);
   E* WprojT = at<E>(ws, L, B_WPROJT);
-  stage_mark(c.s, mark);
+  stage_mark(c, mark);
 
   // Z_P = silu(u_P W_gate^T) * (u_P W_up^T), both paths stacked (slow weights).
   {
@@ -381,7 +438,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiSwiGLU e{Z, m.f, m.f, rstd};
     TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
   }
-  stage_mark(c.s, mark + 1);
+  stage_mark(c, mark + 1);
   // Short convs, residual difference, student keys (unnormalised) and their squares.
   {
     dim3 grid(m.f / CONV_TC, static_cast<unsigned>(m.P / CONV_TP));
@@ -398,7 +455,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
                                                       p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
     TTCD_CHECK_LAUNCH();
   }
-  stage_mark(c.s, mark + 2);
+  stage_mark(c, mark + 2);
   // M = W_down W_proj (associativity of W_down (W_proj d_t)).
   {
     dim3 tb(32, 8), tg(cdiv(m.f, 32), cdiv(m.f, 32));
@@ -412,7 +469,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiStore<E> e{M, m.f, m.f, nullptr};
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
   }
-  stage_mark(c.s, mark + 3);
+  stage_mark(c, mark + 3);
   // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
@@ -423,7 +480,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiStore<E> e{R, m.d, m.d, kscale};
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
   }
-  stage_mark(c.s, mark + 4);
+  stage_mark(c, mark + 4);
   // Delta W per chunk, fp32 exclusive prefix scan, W_i = W_down + S_i.
   {
     CUtensorMap mR, mK;
@@ -464,7 +521,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
     TTCD_CHECK_LAUNCH();
   }
-  stage_mark(c.s, mark + 5);
+  stage_mark(c, mark + 5);
   // y = h_S + (W_down + S_i) Z_S, one GEMM per chunk with its own weight.
   {
     CUtensorMap mA, mB;
@@ -486,7 +543,7 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
   }
-  stage_mark(c.s, mark + 6);
+  stage_mark(c, mark + 6);
   return TTCD_OK;
 }
 
@@ -497,6 +554,230 @@ bool weights_ok(const ttcd_block_weights* w, bool block) {
     if (!aligned16(q)) return false;
   if (block && (!aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(w->g_attn))) return false;
   return true;
+}
+
+// Casts n elements (grid-stride) on the call's stream.
+template <class InT, class OutT>
+ttcd_status launch_cast(const Ctx& c, const void* in, void* out, long long n) {
+  if (n <= 0) return TTCD_OK;
+  const long long blocks = std::min<long long>(cdiv(n, 256), 8ll * c.sms);
+  cast_kernel<InT, OutT><<<static_cast<unsigned>(blocks), 256, 0, c.s>>>(
+      static_cast<const InT*>(in), static_cast<OutT*>(out), n);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+// The wide route: exact fp32 copies of the bf16 weights in the workspace, and a
+// weight table that points at them.  Weights the call does not use may be null.
+ttcd_status widen_weights(const Ctx& c, const ttcd_block_params* p, const ttcd_block_weights* w,
+                          void* ws, const Layout& L, ttcd_block_weights* w32) {
+  const W32Layout WL = w32_layout(p);
+  uint8_t* base = at<uint8_t>(ws, L, B_W32);
+  const size_t d = p->d_model, f = p->d_ff, hd = p->head_dim;
+  const size_t dqkv = (p->n_q_heads + 2 * p->n_kv_heads) * hd, dq = p->n_q_heads * hd;
+  const long long n[10] = {static_cast<long long>(dqkv * d), static_cast<long long>(d * dq),
+                           static_cast<long long>(d), static_cast<long long>(d),
+                           static_cast<long long>(f * d), static_cast<long long>(f * d),
+                           static_cast<long long>(d * f), static_cast<long long>(f * f),
+                           static_cast<long long>(f * p->conv_k),
+                           static_cast<long long>(f * p->conv_k)};
+  const void* src[10] = {w->w_qkv, w->w_o,    w->g_attn, w->g_mlp,  w->w_gate,
+                         w->w_up,  w->w_down, w->w_proj, w->conv_T, w->conv_S};
+  const void** dst[10] = {&w32->w_qkv, &w32->w_o,    &w32->g_attn, &w32->g_mlp,  &w32->w_gate,
+                          &w32->w_up,  &w32->w_down, &w32->w_proj, &w32->conv_T, &w32->conv_S};
+  for (int i = 0; i < 10; ++i) {
+    *dst[i] = nullptr;
+    if (!src[i]) continue;
+    *dst[i] = base + WL.off[i];
+    TTCD_TRY((launch_cast<__nv_bfloat16, float>(c, src[i], base + WL.off[i], n[i])));
+  }
+  return TTCD_OK;
+}
+
+// Reads the status word at `word` after all work queued on s, and clears it.
+ttcd_status read_clear_status(uint32_t* word, cudaStream_t s, uint32_t* flags) {
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  if (v && cudaMemsetAsync(word, 0, sizeof(v), s) != cudaSuccess) return TTCD_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v & DEV_ERR_TIMEOUT) return TTCD_ERR_TIMEOUT;
+  return v ? TTCD_ERR_CUDA : TTCD_OK;
+}
+
+// ttcd_fastweight_mlp with its status word at `status` (null: the per-device word).
+ttcd_status mlp_entry(const void* u_T, const void* u_S, const void* h_S, const float* beta,
+                      const ttcd_block_weights* w, const ttcd_block_params* p,
+                      const float* state_in, float* state_out, void* y, void* workspace,
+                      size_t ws_bytes, void* stream, void* status) {
+  TTCD_TRY(check_params(p));
+  if (!aligned16(u_T) || !aligned16(u_S) || !aligned16(beta) || !aligned16(y) ||
+      !weights_ok(w, false) || !aligned16(workspace))
+    return TTCD_ERR_INVALID_ARG;
+  if ((h_S && !aligned16(h_S)) || (state_in && !aligned16(state_in)) ||
+      (state_out && !aligned16(state_out)))
+    return TTCD_ERR_INVALID_ARG;
+  const Layout L = make_layout(p, false);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, status));
+  const Dims m = dims_of(p);
+  const long long n_u = m.BT * m.d;
+  using bf = __nv_bfloat16;
+  if (wide_mode(p)) {
+    ttcd_block_weights w32;
+    TTCD_TRY(widen_weights(c, p, w, workspace, L, &w32));
+    float* u = at<float>(workspace, L, B_U);
+    TTCD_TRY((launch_cast<bf, float>(c, u_T, u, n_u)));
+    TTCD_TRY((launch_cast<bf, float>(c, u_S, u + n_u, n_u)));
+    float* hs = nullptr;
+    if (h_S) {
+      hs = at<float>(workspace, L, B_HS32);
+      TTCD_TRY((launch_cast<bf, float>(c, h_S, hs, n_u)));
+    }
+    float* y32 = at<float>(workspace, L, B_OUT32);
+    TTCD_TRY((run_mlp_core<float, float, float>(
+        c, p, L, workspace, static_cast<const float*>(w32.w_gate),
+        static_cast<const float*>(w32.w_up), static_cast<const float*>(w32.w_down),
+        static_cast<const float*>(w32.w_proj), static_cast<const float*>(w32.conv_T),
+        static_cast<const float*>(w32.conv_S), beta, state_in, state_out, hs, y32, 0, nullptr)));
+    return launch_cast<float, bf>(c, y32, y, n_u);
+  }
+  const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
+  uint8_t* u = at<uint8_t>(workspace, L, B_U);
+  if (cudaMemcpyAsync(u, u_T, n_u * e, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
+      cudaMemcpyAsync(u + n_u * e, u_S, n_u * e, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  if (p->dtype == TTCD_BF16) {
+    return run_mlp_core<bf, bf, bf>(
+        c, p, L, workspace, static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up),
+        static_cast<const bf*>(w->w_down), static_cast<const bf*>(w->w_proj),
+        static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), beta, state_in,
+        state_out, static_cast<const bf*>(h_S), static_cast<bf*>(y), 0, nullptr);
+  }
+  return run_mlp_core<float, float, float>(
+      c, p, L, workspace, static_cast<const float*>(w->w_gate),
+      static_cast<const float*>(w->w_up), static_cast<const float*>(w->w_down),
+      static_cast<const float*>(w->w_proj), static_cast<const float*>(w->conv_T),
+      static_cast<const float*>(w->conv_S), beta, state_in, state_out,
+      static_cast<const float*>(h_S), static_cast<float*>(y), 0, nullptr);
+}
+
+// The block for operand type E (bf16: kind::f16 tensor cores; fp32: kind::tf32).
+// x, the weights and out are E; the wide route calls it with fp32 copies.
+template <class E>
+ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
+                      const ttcd_block_weights* w, const ttcd_block_params* p,
+                      const float* state_in, float* state_out, void* out, void* ws,
+                      const Layout& L) {
+  const Dims m = dims_of(p);
+  E* wg = at<E>(ws, L, B_WQKVG);
+  float* rstd_in = at<float>(ws, L, B_RSTDIN);
+  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
+  E* o = at<E>(ws, L, B_O);
+  float* h = at<float>(ws, L, B_H);
+  __half2* rope = at<__half2>(ws, L, B_ROPE);
+  E* u = at<E>(ws, L, B_U);
+  float* hssq = at<float>(ws, L, B_HSSQ);
+  const E* xin = static_cast<const E*>(x);
+
+  // Rotary table; the input RMSNorm as a row scale 1/rms(x) applied in the QKV
+  // epilogue, with its gain folded into the weight: xn W^T = rstd (x (W diag g)^T).
+  stage_mark(c, 0);
+  rope_table_kernel<<<cdiv(static_cast<long long>(cdiv(p->T, ROPE_RUN)) * (m.hd / 2), 256), 256, 0, c.s>>>(
+      rope, p->T, m.hd, static_cast<double>(p->rope_theta));
+  TTCD_CHECK_LAUNCH();
+  rms_rowscale_kernel<E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(xin, rstd_in, m.BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  {
+    const long long n8 = static_cast<long long>(m.dqkv) * m.d / 8;
+    scale_cols_kernel<E><<<cdiv(n8, 256), 256, 0, c.s>>>(
+        static_cast<const E*>(w->w_qkv), static_cast<const E*>(w->g_attn), wg, n8, m.d);
+    TTCD_CHECK_LAUNCH();
+  }
+  stage_mark(c, 1);
+
+  // Shared Q/K/V with RoPE.
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<E>(&mA, xin, m.BT, m.d, 128) || !map_rows<E>(&mB, wg, m.dqkv, m.d, 256))
+      return TTCD_ERR_CUDA;
+    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
+    CUtensorMap mo;
+    if (!make_out_map<__nv_bfloat16>(&mo, qkv, m.BT, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
+    const int n_rope = (m.Hq + m.Hkv) * m.hd;
+    switch (m.hd) {
+      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
+      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
+      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
+    }
+  }
+  stage_mark(c, 2);
+  // Dual-window attention: o_T rows then o_S rows.
+  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
+  TTCD_TRY(run_attn<E>(c, qkv, qkv + static_cast<long long>(m.Hq) * m.hd,
+                       qkv + static_cast<long long>(m.Hq + m.Hkv) * m.hd, o,
+                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq, m.Hkv, m.hd,
+                       p->w_S, p->w_T, sc, m.dqkv, m.dqkv));
+  stage_mark(c, 3);
+  // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
+        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
+      return TTCD_ERR_CUDA;
+    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
+    // h_P = x + o_P W_o^T; stores h * g_mlp (gate/up operand), the student
+    // h in fp32, and per-tile sums of h^2 for the MLP RMSNorm.
+    CUtensorMap mo, mo2;
+    if (!make_out_map<E>(&mo, u, 2 * m.BT, m.d, m.d) ||
+        !make_out_map<float>(&mo2, h, m.BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
+    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e, &mo2)));
+  }
+
+  const float* h_S = h;
+  return run_mlp_core<E, E, float>(c, p, L, ws, static_cast<const E*>(w->w_gate),
+                                   static_cast<const E*>(w->w_up),
+                                   static_cast<const E*>(w->w_down),
+                                   static_cast<const E*>(w->w_proj),
+                                   static_cast<const E*>(w->conv_T),
+                                   static_cast<const E*>(w->conv_S), beta, state_in, state_out,
+                                   h_S, static_cast<E*>(out), 4, hssq);
+}
+
+// ttcd_block_forward with optional stage-boundary events (profiled calls).
+ttcd_status block_entry(const void* x, const float* beta, const ttcd_block_weights* w,
+                        const ttcd_block_params* p, const float* state_in, float* state_out,
+                        void* out, void* workspace, size_t ws_bytes, void* stream,
+                        const cudaEvent_t* events, int n_events) {
+  TTCD_TRY(check_params(p));
+  if (!aligned16(x) || !aligned16(beta) || !aligned16(out) || !weights_ok(w, true) ||
+      !aligned16(workspace) || (state_out && !aligned16(state_out)) ||
+      (state_in && !aligned16(state_in)))
+    return TTCD_ERR_INVALID_ARG;
+  const Layout L = make_layout(p, true);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, at<void>(workspace, L, B_STATUS)));
+  c.events = events;
+  c.n_events = n_events;
+  if (p->dtype == TTCD_F32)
+    return run_block<float>(c, x, beta, w, p, state_in, state_out, out, workspace, L);
+  if (wide_mode(p)) {
+    using bf = __nv_bfloat16;
+    const long long n_x = static_cast<long long>(p->B) * p->T * p->d_model;
+    ttcd_block_weights w32;
+    TTCD_TRY(widen_weights(c, p, w, workspace, L, &w32));
+    float* x32 = at<float>(workspace, L, B_X32);
+    float* out32 = at<float>(workspace, L, B_OUT32);
+    TTCD_TRY((launch_cast<bf, float>(c, x, x32, n_x)));
+    TTCD_TRY(run_block<float>(c, x32, beta, &w32, p, state_in, state_out, out32, workspace, L));
+    return launch_cast<float, bf>(c, out32, out, n_x);
+  }
+  return run_block<__nv_bfloat16>(c, x, beta, w, p, state_in, state_out, out, workspace, L);
 }
 
 }  // namespace
@@ -516,17 +797,7 @@ const char* ttcd_status_string(ttcd_status s) {
   return "unknown status";
 }
 
-const char* ttcd_version(void) { return "ttcd 0.1 sm_100a"; }
-
-ttcd_status ttcd_set_stage_events(void* const* events, int n_events) {
-  if (n_events < 0 || n_events > kMaxStageEvents || (n_events > 0 && !events))
-    return TTCD_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i)
-    if (!events[i]) return TTCD_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
-  g_n_stage_events = n_events;
-  return TTCD_OK;
-}
+const char* ttcd_version(void) { return "ttcd 0.2 sm_100a"; }
 
 unsigned long long ttcd_kernel_launch_count(void) { return g_launches.load(); }
 
@@ -555,16 +826,16 @@ ttcd_status ttcd_block_workspace_offset(const ttcd_block_params* p, const char* 
   return TTCD_ERR_INVALID_ARG;
 }
 
+ttcd_status ttcd_check_device_status(void* workspace, void* stream) {
+  if (!aligned16(workspace)) return TTCD_ERR_INVALID_ARG;
+  return read_clear_status(static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream),
+                           nullptr);
+}
+
 ttcd_status ttcd_get_device_error(uint32_t* flags, void* stream) {
   Ctx c;
   TTCD_TRY(make_ctx(stream, c));
-  uint32_t v = 0;
-  if (cudaStreamSynchronize(c.s) != cudaSuccess) return TTCD_ERR_CUDA;
-  if (cudaMemcpy(&v, c.st.err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TTCD_ERR_CUDA;
-  const uint32_t zero = 0;
-  if (cudaMemcpy(c.st.err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return TTCD_ERR_CUDA;
-  if (flags) *flags = v;
-  return (v & DEV_ERR_TIMEOUT) ? TTCD_ERR_TIMEOUT : TTCD_OK;
+  return read_clear_status(c.st.err, c.s, flags);
 }
 
 ttcd_status ttcd_dual_window_attn(const void* q, const void* k, const void* v, void* o_T,
@@ -623,136 +894,31 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
                                 const ttcd_block_params* p, const float* state_in,
                                 float* state_out, void* y, void* workspace, size_t ws_bytes,
                                 void* stream) {
-  TTCD_TRY(check_params(p));
-  if (!aligned16(u_T) || !aligned16(u_S) || !aligned16(beta) || !aligned16(y) ||
-      !weights_ok(w, false) || !aligned16(workspace))
-    return TTCD_ERR_INVALID_ARG;
-  if ((h_S && !aligned16(h_S)) || (state_in && !aligned16(state_in)) ||
-      (state_out && !aligned16(state_out)))
-    return TTCD_ERR_INVALID_ARG;
-  const Layout L = make_layout(p, false);
-  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
-  Ctx c;
-  TTCD_TRY(make_ctx(stream, c));
-  const Dims m = dims_of(p);
-  const size_t e = p->dtype == TTCD_F32 ? 4 : 2;
-  uint8_t* u = at<uint8_t>(workspace, L, B_U);
-  if (cudaMemcpyAsync(u, u_T, m.BT * m.d * e, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
-      cudaMemcpyAsync(u + m.BT * m.d * e, u_S, m.BT * m.d * e, cudaMemcpyDeviceToDevice, c.s) !=
-          cudaSuccess)
-    return TTCD_ERR_CUDA;
-  if (p->dtype == TTCD_BF16) {
-    using bf = __nv_bfloat16;
-    return run_mlp_core<bf, bf, bf>(
-        c, p, L, workspace, static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up),
-        static_cast<const bf*>(w->w_down), static_cast<const bf*>(w->w_proj),
-        static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), beta, state_in,
-        state_out, static_cast<const bf*>(h_S), static_cast<bf*>(y), 0, nullptr);
-  }
-  return run_mlp_core<float, float, float>(
-      c, p, L, workspace, static_cast<const float*>(w->w_gate),
-      static_cast<const float*>(w->w_up), static_cast<const float*>(w->w_down),
-      static_cast<const float*>(w->w_proj), static_cast<const float*>(w->conv_T),
-      static_cast<const float*>(w->conv_S), beta, state_in, state_out,
-      static_cast<const float*>(h_S), static_cast<float*>(y), 0, nullptr);
+  return mlp_entry(u_T, u_S, h_S, beta, w, p, state_in, state_out, y, workspace, ws_bytes,
+                   stream, workspace);
 }
-
-}  // extern "C"
-
-namespace {
-// The block for operand type E (bf16: kind::f16 tensor cores; fp32: kind::tf32).
-template <class E>
-ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
-                      const ttcd_block_weights* w, const ttcd_block_params* p, float* state_out,
-                      void* out, void* ws, const Layout& L) {
-  const Dims m = dims_of(p);
-  E* xn = at<E>(ws, L, B_XN);
-  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
-  E* o = at<E>(ws, L, B_O);
-  float* h = at<float>(ws, L, B_H);
-  __half2* rope = at<__half2>(ws, L, B_ROPE);
-  E* u = at<E>(ws, L, B_U);
-  float* hssq = at<float>(ws, L, B_HSSQ);
-  const E* xin = static_cast<const E*>(x);
-
-  // Rotary table, input RMSNorm.
-  stage_mark(c.s, 0);
-  rope_table_kernel<<<cdiv(static_cast<long long>(cdiv(p->T, ROPE_RUN)) * (m.hd / 2), 256), 256, 0, c.s>>>(
-      rope, p->T, m.hd, static_cast<double>(p->rope_theta));
-  TTCD_CHECK_LAUNCH();
-  rmsnorm_kernel<E, E, E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(
-      xin, static_cast<const E*>(w->g_attn), xn, m.BT, m.d, p->rms_eps);
-  TTCD_CHECK_LAUNCH();
-  stage_mark(c.s, 1);
-
-  // Shared Q/K/V with RoPE.
-  {
-    CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, xn, m.BT, m.d, 128) || !map_rows<E>(&mB, w->w_qkv, m.dqkv, m.d, 256))
-      return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
-    CUtensorMap mo;
-    if (!make_out_map<__nv_bfloat16>(&mo, qkv, m.BT, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
-    const int n_rope = (m.Hq + m.Hkv) * m.hd;
-    switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
-      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
-      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope}))); break;
-    }
-  }
-  stage_mark(c.s, 2);
-  // Dual-window attention: o_T rows then o_S rows.
-  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
-  TTCD_TRY(run_attn<E>(c, qkv, qkv + static_cast<long long>(m.Hq) * m.hd,
-                       qkv + static_cast<long long>(m.Hq + m.Hkv) * m.hd, o,
-                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq, m.Hkv, m.hd,
-                       p->w_S, p->w_T, sc, m.dqkv, m.dqkv));
-  stage_mark(c.s, 3);
-  // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
-  {
-    CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
-        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
-      return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
-    // h_P = x + o_P W_o^T; stores h * g_mlp (gate/up operand), the student
-    // h in fp32, and per-tile sums of h^2 for the MLP RMSNorm.
-    CUtensorMap mo, mo2;
-    if (!make_out_map<E>(&mo, u, 2 * m.BT, m.d, m.d) ||
-        !make_out_map<float>(&mo2, h, m.BT, m.d, m.d))
-      return TTCD_ERR_CUDA;
-    EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e, &mo2)));
-  }
-
-  const float* h_S = h;
-  return run_mlp_core<E, E, float>(c, p, L, ws, static_cast<const E*>(w->w_gate),
-                                   static_cast<const E*>(w->w_up),
-                                   static_cast<const E*>(w->w_down),
-                                   static_cast<const E*>(w->w_proj),
-                                   static_cast<const E*>(w->conv_T),
-                                   static_cast<const E*>(w->conv_S), beta, nullptr, state_out,
-                                   h_S, static_cast<E*>(out), 4, hssq);
-}
-}  // namespace
-
-extern "C" {
 
 ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_block_weights* w,
                                const ttcd_block_params* p, float* state_out, void* out,
                                void* workspace, size_t ws_bytes, void* stream) {
-  TTCD_TRY(check_params(p));
-  if (!aligned16(x) || !aligned16(beta) || !aligned16(out) || !weights_ok(w, true) ||
-      !aligned16(workspace) || (state_out && !aligned16(state_out)))
-    return TTCD_ERR_INVALID_ARG;
-  const Layout L = make_layout(p, true);
-  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
-  Ctx c;
-  TTCD_TRY(make_ctx(stream, c));
-  if (p->dtype == TTCD_F32)
-    return run_block<float>(c, x, beta, w, p, state_out, out, workspace, L);
-  return run_block<__nv_bfloat16>(c, x, beta, w, p, state_out, out, workspace, L);
+  return block_entry(x, beta, w, p, nullptr, state_out, out, workspace, ws_bytes, stream,
+                     nullptr, 0);
 }
+
+ttcd_status ttcd_block_forward_profiled(const void* x, const float* beta,
+                                        const ttcd_block_weights* w, const ttcd_block_params* p,
+                                        float* state_out, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream, void* const* events,
+                                        int n_events) {
+  if (n_events < 0 || n_events > kMaxStageEvents || (n_events > 0 && !events))
+    return TTCD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return TTCD_ERR_INVALID_ARG;
+  return block_entry(x, beta, w, p, nullptr, state_out, out, workspace, ws_bytes, stream,
+                     reinterpret_cast<const cudaEvent_t*>(events), n_events);
+}
+
+}  // extern "C"
 
 // ---------------------------------------------------------------------------
 // Fast-weight MLP without caller-provided scratch.
@@ -766,7 +932,13 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
 // until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_ttcd_noalloc_scratch[kNoAllocScratchBytes];
+namespace {
+// Device address of the array, looked up once per device (host-side state of
+// this file only: not exported).
 void* g_noalloc_scratch_addr[kMaxDevices] = {nullptr};
+}  // namespace
+
+extern "C" {
 
 ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const void* h_S,
                                         const float* beta, const ttcd_block_weights* w,
@@ -789,9 +961,11 @@ ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const 
     }
   }
   // Every byte of scratch that a call reads is written earlier in the same
-  // call, so nothing has to be cleared between calls.
-  return ttcd_fastweight_mlp(u_T, u_S, h_S, beta, w, p, state_in, state_out, y,
-                             g_noalloc_scratch_addr[dev], kNoAllocScratchBytes, stream);
+  // call, so nothing has to be cleared between calls.  Timeouts go to the
+  // per-device status word (ttcd_get_device_error): the caller holds no
+  // workspace to keep one in.
+  return mlp_entry(u_T, u_S, h_S, beta, w, p, state_in, state_out, y,
+                   g_noalloc_scratch_addr[dev], kNoAllocScratchBytes, stream, nullptr);
 }
 
 size_t ttcd_fastweight_mlp_noalloc_capacity(void) { return kNoAllocScratchBytes; }
@@ -809,10 +983,35 @@ __global__ void bounded_wait_test_kernel(DevStatus st) {
   __syncthreads();
 }
 
-ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream) {
-  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return TTCD_ERR_INVALID_ARG;
+// Evaluates the attention kernel's FMA-pipe 2^x (exp2_poly2) at x[0..n-1].
+__global__ void exp2_poly_test_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const long long i = 2ll * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x1 = i + 1 < n ? x[i + 1] : x[i];
+  float y0, y1;
+  f2unpack(exp2_poly2(f2pack(x[i], x1)), y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
+ttcd_status ttcd_test_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y)) || (reinterpret_cast<uintptr_t>(x) & 3u) ||
+      (reinterpret_cast<uintptr_t>(y) & 3u))
+    return TTCD_ERR_INVALID_ARG;
+  if (n == 0) return TTCD_OK;
   Ctx c;
   TTCD_TRY(make_ctx(stream, c));
+  const int threads = (n + 1) / 2;
+  exp2_poly_test_kernel<<<cdiv(threads, 256), 256, 0, c.s>>>(x, y, n);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* status, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return TTCD_ERR_INVALID_ARG;
+  if (status && !aligned16(status)) return TTCD_ERR_INVALID_ARG;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, status));
   DevStatus st = c.st;
   st.timeout_ns = timeout_ns;
   bounded_wait_test_kernel<<<1, 32, 0, c.s>>>(st);
@@ -825,27 +1024,30 @@ ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream) {
 // ===================================================================== decode
 namespace {
 
-// Decode state (per sequence unless noted), 1 KiB-aligned pieces.
+// Decode state (per sequence unless noted), 1 KiB-aligned pieces; the status
+// word of every decode call comes first.
 struct DecState {
-  size_t kc, vc, hist, rc, kx, S, weff, M, wprojT, total;
+  size_t status, kc, vc, hist, rc, kx, S, weff, M, wprojT, total;
 };
 DecState dec_state_layout(const ttcd_block_params* p) {
   const long long B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
   const long long W = p->w_T, H = p->conv_k > 1 ? p->conv_k - 1 : 1;
   const long long Cp = (p->chunk + 63) / 64 * 64;
-  size_t sz[9] = {static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // K cache ring
-                  static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // V cache ring
-                  static_cast<size_t>(2 * B * H * f * 4),                // conv history
-                  static_cast<size_t>(B * Cp * d * 2),                   // r rows of the chunk
-                  static_cast<size_t>(B * Cp * f * 2),                   // k' rows of the chunk
-                  static_cast<size_t>(B * d * f * 4),                    // S
-                  static_cast<size_t>(B * d * f * 2),                    // W_down + S
-                  static_cast<size_t>(d * f * 2),                        // M (shared)
-                  static_cast<size_t>(f * f * 2)};                       // W_proj^T (shared)
+  size_t sz[10] = {kStatusBytes,                                          // status word
+                   static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // K cache ring
+                   static_cast<size_t>(B * W * p->n_kv_heads * hd * 2),   // V cache ring
+                   static_cast<size_t>(2 * B * H * f * 4),                // conv history
+                   static_cast<size_t>(B * Cp * d * 2),                   // r rows of the chunk
+                   static_cast<size_t>(B * Cp * f * 2),                   // k' rows of the chunk
+                   static_cast<size_t>(B * d * f * 4),                    // S
+                   static_cast<size_t>(B * d * f * 2),                    // W_down + S
+                   static_cast<size_t>(d * f * 2),                        // M (shared)
+                   static_cast<size_t>(f * f * 2)};                       // W_proj^T (shared)
   DecState L;
-  size_t* fields[9] = {&L.kc, &L.vc, &L.hist, &L.rc, &L.kx, &L.S, &L.weff, &L.M, &L.wprojT};
+  size_t* fields[10] = {&L.status, &L.kc, &L.vc, &L.hist, &L.rc, &L.kx, &L.S, &L.weff, &L.M,
+                        &L.wprojT};
   size_t off = 0;
-  for (int i = 0; i < 9; ++i) {
+  for (int i = 0; i < 10; ++i) {
     *fields[i] = off;
     off += (sz[i] + 1023) / 1024 * 1024;
   }
@@ -1094,7 +1296,7 @@ ttcd_status ttcd_decode_state_init(const ttcd_block_weights* w, const ttcd_block
   (void)workspace;
   (void)ws_bytes;
   Ctx c;
-  TTCD_TRY(make_ctx(stream, c));
+  TTCD_TRY(make_ctx(stream, c, dat<void>(state, S.status)));
   using bf = __nv_bfloat16;
   const int d = p->d_model, f = p->d_ff;
   if (cudaMemsetAsync(state, 0, S.total, c.s) != cudaSuccess) return TTCD_ERR_CUDA;
@@ -1129,7 +1331,7 @@ ttcd_status ttcd_block_decode(const void* x_t, const float* beta_t, int t,
   const DecWs L = dec_ws_layout(p);
   if (state_bytes < S.total || ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
   Ctx c;
-  TTCD_TRY(make_ctx(stream, c));
+  TTCD_TRY(make_ctx(stream, c, dat<void>(state, S.status)));
   return run_decode(c, static_cast<const __nv_bfloat16*>(x_t), beta_t, t, w, p, state, S,
                     static_cast<__nv_bfloat16*>(y), workspace, L);
 }
@@ -1141,7 +1343,7 @@ ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void*
   const DecState S = dec_state_layout(p);
   if (state_bytes < S.total) return TTCD_ERR_WORKSPACE;
   Ctx c;
-  TTCD_TRY(make_ctx(stream, c));
+  TTCD_TRY(make_ctx(stream, c, dat<void>(state, S.status)));
   const int d = p->d_model, f = p->d_ff, C = p->chunk, Cp = (C + 63) / 64 * 64;
   const int n = t_next % C;  // tokens of the current, partial chunk
   if (n == 0) {

@@ -24,14 +24,23 @@
  *   - Every device pointer must be 16-byte aligned; each tensor's innermost
  *     extent times its element size must be a multiple of 16 bytes.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream) and keep no state between calls except the device error word
- *     read by ttcd_get_device_error() and the profiling hooks below.
+ *     stream) and keep no state between calls: everything a call writes is in
+ *     the caller's buffers.  Calls on different workspaces may run concurrently
+ *     on different streams or host threads.  Process-wide settings are only the
+ *     wait bound (ttcd_set_wait_timeout_ns) and a diagnostic launch counter.
  *   - Arguments are validated on the host before any launch; a bad argument
  *     returns TTCD_ERR_INVALID_ARG or TTCD_ERR_UNSUPPORTED and launches nothing.
- *     A launch failure returns TTCD_ERR_CUDA.  Every device-side wait is
- *     bounded: one that gives up sets the device error word (reported as
- *     TTCD_ERR_TIMEOUT by ttcd_get_device_error) and the kernel returns.  No
- *     entry point aborts, traps or throws.
+ *     A launch failure returns TTCD_ERR_CUDA.
+ *   - Every device-side wait is bounded.  One that gives up records
+ *     TTCD_ERR_TIMEOUT in the call's status word and the kernel returns; no
+ *     entry point aborts, traps or throws.  The status word is the first 4 bytes
+ *     of the call's workspace (block forward, fast-weight MLP) or decode state:
+ *     it accumulates over calls until ttcd_check_device_status() reads and
+ *     clears it, so zero the first TTCD_STATUS_BYTES bytes of a new workspace
+ *     before its first use (ttcd_decode_state_init clears a decode state).
+ *     Entry points without a workspace (the two attention calls and
+ *     ttcd_fastweight_mlp_noalloc) record into one status word per device,
+ *     shared by all their callers and read by ttcd_get_device_error().
  */
 #ifndef TTCD_H_
 #define TTCD_H_
@@ -53,6 +62,10 @@ typedef enum {
 } ttcd_status;
 
 typedef enum { TTCD_F32 = 0, TTCD_BF16 = 1 } ttcd_dtype;
+
+/* Bytes at the start of every workspace and decode state that hold its status
+ * word (the rest of the region is reserved). */
+#define TTCD_STATUS_BYTES 256
 
 /* Shape and hyper-parameters of one block.  Names follow the pages:
  * window_size = teacher window w_T, student window w_S, fast-weight chunk C,
@@ -155,7 +168,13 @@ ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* 
  *   beta       [B, T] fp32, device
  *   state_in   [B, d, f] fp32, device, nullable;  state_out likewise
  *   y          [B, T, d] params.dtype, device, written
- *   workspace  >= ttcd_fastweight_mlp_workspace_size(p) bytes, device, 16-byte aligned
+ *   workspace  >= ttcd_fastweight_mlp_workspace_size(p) bytes, device, 16-byte aligned;
+ *              its first TTCD_STATUS_BYTES bytes hold the call's status word
+ * Precision: TTCD_BF16 contracts bf16 operands with fp32 accumulation, except
+ * when T < chunk: a state written by fewer than `chunk` tokens does not average
+ * out the bf16 rounding of u, D, M, R and k', so such calls widen the inputs and
+ * weights exactly to fp32 in the workspace and contract them as tf32 (fp32
+ * accumulation); y is rounded to bf16 once.  TTCD_F32 always uses tf32.
  */
 ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_S,
                                 const float* beta, const ttcd_block_weights* w,
@@ -175,13 +194,36 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
  *   x, out     [B, T, d] params.dtype, device
  *   beta       [B, T] fp32, device
  *   state_out  [B, d, f] fp32, device, nullable (final fast-weight state)
- *   workspace  >= ttcd_block_forward_workspace_size(p) bytes, device, 16-byte aligned
+ *   workspace  >= ttcd_block_forward_workspace_size(p) bytes, device, 16-byte aligned;
+ *              its first TTCD_STATUS_BYTES bytes hold the call's status word
  * The workspace holds every intermediate after the call; their byte offsets
- * are returned by ttcd_block_workspace_offset().
+ * are returned by ttcd_block_workspace_offset().  The input RMSNorm is applied
+ * as a row scale 1/rms(x) in the QKV epilogue with its gain folded into a copy
+ * of W_qkv (xn W_qkv^T = (x (W_qkv diag g_attn)^T) / rms(x)).  Precision as
+ * ttcd_fastweight_mlp: TTCD_BF16 with T < chunk runs the whole block on fp32
+ * copies (tf32 MMAs; q, k, v stay bf16).
  */
 ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_block_weights* w,
                                const ttcd_block_params* p, float* state_out, void* out,
                                void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * ttcd_block_forward_profiled — ttcd_block_forward that also records the
+ * caller's CUDA events (cudaEvent_t handles, owned by the caller) on `stream`
+ * at its stage boundaries, for per-stage timing.  Not part of the method.
+ *   events[k] is recorded at boundary k: 0 start, 1 after the rotary table, the
+ *   input RMS row scales and the gain-scaled W_qkv, 2 after QKV+RoPE, 3 after
+ *   attention, 4 after o_proj (with the MLP RMSNorm statistics), 5 after
+ *   gate/up+SwiGLU, 6 after conv/residual/keys, 7 after M = W_down W_proj,
+ *   8 after R, 9 after the chunk scan, 10 after the output GEMM.  Boundaries at
+ *   or beyond n_events are skipped; 0 <= n_events <= 16; events[0..n_events-1]
+ *   must be non-null.  The events belong to this call only.
+ */
+ttcd_status ttcd_block_forward_profiled(const void* x, const float* beta,
+                                        const ttcd_block_weights* w, const ttcd_block_params* p,
+                                        float* state_out, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream, void* const* events,
+                                        int n_events);
 
 /*
  * ttcd_fastweight_mlp_noalloc — ttcd_fastweight_mlp for callers that cannot
@@ -204,6 +246,8 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
  *     contents (every byte a call reads is written earlier in the same call, so
  *     nothing needs clearing).  Calls whose kernels overlap on the GPU (other
  *     streams, other host threads) race on it: serialise them.
+ *   - With no workspace to hold a status word, a wait that gives up is recorded
+ *     in the per-device word read by ttcd_get_device_error().
  */
 ttcd_status ttcd_fastweight_mlp_noalloc(const void* u_T, const void* u_S, const void* h_S,
                                         const float* beta, const ttcd_block_weights* w,
@@ -227,7 +271,8 @@ size_t ttcd_fastweight_mlp_noalloc_capacity(void);
  * pages.)
  *
  * The state (caller-owned device memory, ttcd_decode_state_size bytes,
- * 16-byte aligned, layout internal to the library) holds, per sequence:
+ * 16-byte aligned, layout internal to the library) holds the status word of
+ * every decode call in its first TTCD_STATUS_BYTES bytes and, per sequence:
  *   - the K/V cache of the last w_T tokens (ring buffer, bf16);
  *   - the last conv_k-1 rows of Z_T and Z_S (conv history, fp32);
  *   - r_t and k'_t of the current chunk's tokens (bf16);
@@ -269,8 +314,11 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  * Byte offset inside the block_forward workspace of a named intermediate, for
  * inspection after a call (same layout for ttcd_fastweight_mlp where named).
  * Names and layouts (row-major):
- *   (E = bf16 for TTCD_BF16, fp32 for TTCD_F32; q, k, v are always bf16)
- *   "xn"   E [B*T, d]
+ *   (E = bf16 for TTCD_BF16 with T >= chunk, fp32 for TTCD_F32 and for
+ *   TTCD_BF16 with T < chunk; q, k, v are always bf16)
+ *   "status"  uint32 status word (TTCD_STATUS_BYTES reserved)
+ *   "wqkv_g"  E [(Hq + 2 Hkv) hd, d]  W_qkv diag(g_attn)
+ *   "rstd_in" fp32 [B*T]  1/rms of each input row
  *   "qkv"  bf16 [B*T, (Hq + 2 Hkv) hd]: q heads (rotated), k heads (rotated), v heads
  *   "o"    E [2, B*T, Hq*hd]      (o_T rows, then o_S rows)
  *   "h"    fp32 [B*T, d] (student residual h_S)
@@ -287,9 +335,23 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
 ttcd_status ttcd_block_workspace_offset(const ttcd_block_params* p, const char* name,
                                         size_t* offset);
 
-/* Reads and clears the device error word on the current device (synchronises
- * `stream`).  *flags receives the raw bits; returns TTCD_ERR_TIMEOUT if a wait
- * gave up since the last call, TTCD_OK otherwise. */
+/*
+ * ttcd_check_device_status — reads and clears the status word of a workspace
+ * (ttcd_block_forward, ttcd_fastweight_mlp) or of a decode state, after all
+ * work queued on `stream` (synchronises `stream`).  Returns TTCD_ERR_TIMEOUT if
+ * a device wait of a call that used this workspace gave up since the last
+ * check, TTCD_OK otherwise; TTCD_ERR_INVALID_ARG for a null or misaligned
+ * pointer.  Only calls on this workspace are reported: other callers' timeouts
+ * are in their own workspaces.
+ */
+ttcd_status ttcd_check_device_status(void* workspace, void* stream);
+
+/* Reads and clears the per-device status word of the entry points without a
+ * workspace (the attention calls, ttcd_fastweight_mlp_noalloc, and
+ * ttcd_test_bounded_wait with no status region), on the current device
+ * (synchronises `stream`).  *flags receives the raw bits; returns
+ * TTCD_ERR_TIMEOUT if a wait gave up since the last read, TTCD_OK otherwise.
+ * Callers of those entry points share this word. */
 ttcd_status ttcd_get_device_error(uint32_t* flags, void* stream);
 
 /* Bound in nanoseconds on every device-side wait (default 2e9 = 2 s). */
@@ -298,33 +360,31 @@ void ttcd_set_wait_timeout_ns(uint64_t ns);
 /*
  * ttcd_test_bounded_wait — failure-detection self-test.  Launches one CTA that
  * waits on an mbarrier nothing ever arrives at, bounded by `timeout_ns`; the
- * wait gives up, records TTCD_ERR_TIMEOUT in the device error word and the
- * kernel returns normally.  The paper has no counterpart; this exists so a
+ * wait gives up, records TTCD_ERR_TIMEOUT in the status word at `status` (a
+ * workspace or decode state, 16-byte aligned; null: the per-device word) and
+ * the kernel returns normally.  The paper has no counterpart; this exists so a
  * test can check the timeout path without hanging a GPU.
  */
-ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* stream);
+ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* status, void* stream);
 
 /*
- * Profiling hooks (not part of the method; used by the benchmark).
- * ttcd_set_stage_events: when n_events > 0, ttcd_block_forward records
- * events[k] (cudaEvent_t handles owned by the caller) on its stream at stage
- * boundary k: 0 start, 1 after the input RMSNorm, 2 after QKV+RoPE, 3 after
- * attention, 4 after o_proj (which also carries the MLP RMSNorm statistics),
- * 5 after gate/up+SwiGLU, 6 after conv/residual/keys, 7 after
- * M = W_down W_proj, 8 after R, 9 after the chunk scan, 10 after the output
- * GEMM.  ttcd_fastweight_mlp records
- * boundaries 0..6 of its own part (start, gate/up, conv, M, R, scan, output).
- * Boundaries at or beyond n_events are skipped; n_events = 0 disables.
- * Process-wide setting, not thread-safe.  At most 16 events.
+ * ttcd_test_exp2_poly — evaluates, for a test, the 2^x that the attention
+ * kernel computes on the FMA pipe for one exponential pair in four: a cubic in
+ * the fractional part (coefficients fitted to 2^f on [-0.5, 0.5] by
+ * Lawson-reweighted least squares on Chebyshev nodes, relative error 1.01e-4)
+ * scaled by the integer part through the exponent field; inputs below -126 are
+ * clamped.  x, y: n fp32 values, device, 4-byte aligned; y written.  The paper
+ * has no counterpart; it exists so the polynomial can be checked against 2^x.
  */
-ttcd_status ttcd_set_stage_events(void* const* events, int n_events);
+ttcd_status ttcd_test_exp2_poly(const float* x, float* y, int n, void* stream);
 
-/* Number of kernels this library has launched since it was loaded. */
+/* Number of kernels this library has launched since it was loaded (process-wide
+ * diagnostic counter, atomic). */
 unsigned long long ttcd_kernel_launch_count(void);
 
 const char* ttcd_status_string(ttcd_status s);
 
-/* Library version string, e.g. "ttcd 0.1 sm_100a". */
+/* Library version string, e.g. "ttcd 0.2 sm_100a". */
 const char* ttcd_version(void);
 
 #ifdef __cplusplus

@@ -62,12 +62,52 @@ def test_workspace_sizes(lib):
 
 def test_workspace_offsets_are_ordered_and_aligned(lib):
     p = _params()
-    names = ["xn", "qkv", "o", "h", "u", "Z", "Zs16", "D", "Kp", "ssq", "R", "Wall"]
+    names = ["status", "wqkv_g", "rstd_in", "qkv", "o", "h", "u", "Z", "Zs16", "D", "Kp", "ssq",
+             "R", "Wall"]
     offs = [ttcd.workspace_offset(p, n) for n in names]
+    assert offs[0] == 0  # the status word opens every workspace
     assert all(o % 1024 == 0 for o in offs)
     assert offs == sorted(offs)
     with pytest.raises(ttcd.TTCDError):
         ttcd.workspace_offset(p, "nope")
+
+
+def test_short_bf16_problems_take_the_fp32_operand_route(lib):
+    """bf16 with T < chunk runs on fp32 copies: its workspace holds fp32 operands
+    and the widened inputs, weights and output, so it is larger than the bf16
+    workspace of a one-chunk problem, and its intermediates are fp32."""
+    short = _params(dtype=ttcd.BF16, T=31, chunk=32)
+    one_chunk = _params(dtype=ttcd.BF16, T=32, chunk=32)
+    f32_short = _params(dtype=ttcd.F32, T=31, chunk=32)
+    assert ttcd.block_forward_workspace_size(short) > ttcd.block_forward_workspace_size(one_chunk)
+    assert ttcd.block_forward_workspace_size(short) > ttcd.block_forward_workspace_size(f32_short)
+    assert ttcd.fastweight_mlp_workspace_size(short) > ttcd.fastweight_mlp_workspace_size(one_chunk)
+    # "u" holds 2 B T d elements: fp32 on the wide route, bf16 otherwise
+    for p, elem in ((short, 4), (one_chunk, 2)):
+        span = ttcd.workspace_offset(p, "Z") - ttcd.workspace_offset(p, "u")
+        need = 2 * p.B * p.T * p.d_model * elem
+        assert need <= span < need + 1024, (p.T, span, need)
+
+
+def test_check_device_status_validates_on_host(lib):
+    assert lib.ttcd_check_device_status(None, None) == ttcd.ERR_INVALID_ARG
+    assert lib.ttcd_check_device_status(ctypes.c_void_p((1 << 20) + 4), None) == ttcd.ERR_INVALID_ARG
+    assert lib.ttcd_test_bounded_wait(0, None, None) == ttcd.ERR_INVALID_ARG
+    assert lib.ttcd_test_bounded_wait(1000, ctypes.c_void_p((1 << 20) + 8), None) == ttcd.ERR_INVALID_ARG
+
+
+def test_profiled_entry_validates_events_on_host(lib):
+    fake = 1 << 20
+    p = _params().c()
+    w = ttcd._Weights(*([fake] * 10))
+    need = lib.ttcd_block_forward_workspace_size(ctypes.byref(p))
+    f = lib.ttcd_block_forward_profiled
+    ev = (ctypes.c_void_p * 17)(*([fake] * 17))
+    args = (fake, fake, ctypes.byref(w), ctypes.byref(p), None, fake, fake, need, None)
+    assert f(*args, ev, 17) == ttcd.ERR_INVALID_ARG  # at most 16 events
+    assert f(*args, None, 3) == ttcd.ERR_INVALID_ARG
+    assert f(*args, (ctypes.c_void_p * 2)(fake, None), 2) == ttcd.ERR_INVALID_ARG
+    assert f(*args, ev, -1) == ttcd.ERR_INVALID_ARG
 
 
 def test_attention_rejects_bad_arguments_on_host(lib):

@@ -37,8 +37,7 @@ def _decode_all(ttcd, shape, inp, state_in=None):
     p = ttcd.BlockParams.from_shape(shape)
     dec = ttcd.Decoder(w, p, state_in=state_in)
     ys = [dec.step(x[:, t].contiguous(), w["beta"][:, t].contiguous()) for t in range(shape.T)]
-    torch.cuda.synchronize()
-    assert ttcd.get_device_error()[0] == ttcd.OK
+    assert dec.check_status() == ttcd.OK
     return torch.stack(ys, dim=1), dec.state_out(), x, w, p
 
 

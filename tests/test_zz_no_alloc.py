@@ -2,8 +2,12 @@
 the library scratch memory (a host framework owning the whole device pool, or a
 loop that may not call cudaMalloc).  Its scratch is a fixed array inside the
 library, so these checks compare it with ttcd_fastweight_mlp, which takes a
-caller workspace, on two calls in a row: the second call must not be disturbed
-by what the first left in the shared array.
+caller workspace, over several calls in a row.  Each call leaves the shared
+array holding data of another shape: other sequence lengths, a chunk of 96 whose
+padding rows sit where the previous call kept real tokens, an fp32 call and a
+sequence shorter than one chunk (the fp32-operand route).  A buffer that a call
+read without writing first would carry the previous call's values and fail the
+comparison.
 
 This file sorts last so that a run stopping at the first failure has already
 run every other test.
@@ -16,8 +20,16 @@ import torch
 from tests.helpers import TOL_OUT, TOL_STATE, rel_fro, rel_max
 from ttcd_workloads import BlockShape, make_mlp_inputs
 
-SHAPE = BlockShape("noalloc_bf16", "bf16", B=2, T=700, d_model=128, n_q_heads=1, n_kv_heads=1,
-                   head_dim=64, d_ff=256, w_S=1, w_T=1, chunk=128, conv_k=4)
+BASE = BlockShape("noalloc_bf16", "bf16", B=2, T=700, d_model=128, n_q_heads=1, n_kv_heads=1,
+                  head_dim=64, d_ff=256, w_S=1, w_T=1, chunk=128, conv_k=4)
+# Call order: each shape after the first finds the previous one's data in the array.
+SEQUENCE = [
+    (BASE, 11),
+    (BASE.with_(name="noalloc_chunk96", B=1, T=500, chunk=96, conv_k=3), 12),
+    (BASE.with_(name="noalloc_f32", dtype="f32", B=1, T=300, chunk=64), 13),
+    (BASE.with_(name="noalloc_short", B=1, T=50, chunk=128), 14),
+    (BASE, 15),
+]
 
 
 def _lib():
@@ -39,20 +51,39 @@ def _call_noalloc(ttcd, lib, dev, p, h_S=True):
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def test_noalloc_matches_workspace_entry_point_over_calls_of_other_shapes():
     ttcd, lib = _lib()
-    p = ttcd.BlockParams.from_shape(SHAPE)
-    assert ttcd.fastweight_mlp_workspace_size(p) <= lib.ttcd_fastweight_mlp_noalloc_capacity()
-    for seed in (11, 12):  # two calls in a row, different inputs
-        inp = make_mlp_inputs(SHAPE, seed=seed)
+    for shape, seed in SEQUENCE:
+        p = ttcd.BlockParams.from_shape(shape)
+        assert ttcd.fastweight_mlp_workspace_size(p) <= lib.ttcd_fastweight_mlp_noalloc_capacity()
+        inp = make_mlp_inputs(shape, seed=seed)
         dev = {k: v.cuda() for k, v in inp.items()}
-        y_ref, s_ref, _ = ttcd.fastweight_mlp(dev["u_T"], dev["u_S"], dev["beta"], dev, p,
-                                              h_S=dev["h_S"], state_out=True)
+        y_ref, s_ref, ws = ttcd.fastweight_mlp(dev["u_T"], dev["u_S"], dev["beta"], dev, p,
+                                               h_S=dev["h_S"], state_out=True)
+        assert ttcd.check_device_status(ws) == ttcd.OK
         y, s = _call_noalloc(ttcd, lib, dev, p)
         torch.cuda.synchronize()
         assert ttcd.get_device_error()[0] == ttcd.OK
-        assert rel_max(y, y_ref) <= TOL_OUT
-        assert rel_fro(s, s_ref) <= TOL_STATE
+        assert rel_max(y, y_ref) <= TOL_OUT, shape.name
+        assert rel_fro(s, s_ref) <= TOL_STATE, shape.name
+
+
+@pytest.mark.gpu
+def test_noalloc_python_wrapper():
+    """The binding's wrapper: y allocated when not given, state_out=True allocates."""
+    ttcd, _ = _lib()
+    shape = BASE.with_(name="noalloc_wrapper", T=333)
+    p = ttcd.BlockParams.from_shape(shape)
+    dev = {k: v.cuda() for k, v in make_mlp_inputs(shape, seed=16).items()}
+    y_ref, s_ref, _ = ttcd.fastweight_mlp(dev["u_T"], dev["u_S"], dev["beta"], dev, p,
+                                          h_S=dev["h_S"], state_out=True)
+    y, s = ttcd.fastweight_mlp_noalloc(dev["u_T"], dev["u_S"], dev["beta"], dev, p,
+                                       h_S=dev["h_S"], state_out=True)
+    torch.cuda.synchronize()
+    assert ttcd.get_device_error()[0] == ttcd.OK
+    assert y.shape == dev["u_S"].shape and s.shape == (p.B, p.d_model, p.d_ff)
+    assert rel_max(y, y_ref) <= TOL_OUT
+    assert rel_fro(s, s_ref) <= TOL_STATE
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch():
