@@ -33,7 +33,7 @@ from ttcd_workloads import (ATTN_SWEEP_W_S, ATTN_SWEEP_W_T, QWEN3_0P6B_64K,  # n
 METRIC = "IP-TTCD block prefill tokens/s @64K (Qwen3-0.6B shape); dual-attn % BF16 peak"
 UNIT = "tokens/s"
 STAGES = ["rope+rms_rowscale_in", "qkv_gemm_rope", "dual_window_attn", "o_proj_residual_rmsstats",
-          "gate_up_swiglu_rmsnorm", "conv_residual_keys", "M_wdown_wproj", "R_gemm",
+          "gate_up_swiglu_conv_keys", "key_scales", "M_wdown_wproj", "R_gemm",
           "chunk_scan_dW", "out_gemm"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -106,8 +106,10 @@ def stage_costs(s):
         ("tensor", 2.0 * BT * d * dqkv),
         ("tensor", attention_flops(s)),
         ("tensor", 2.0 * 2 * BT * Hq * hd * d),
+        # gate/up for both paths; the epilogue also writes D, K' and Z_S (bf16)
         ("tensor", 2.0 * 2 * BT * d * 2 * f),
-        ("hbm", 2 * BT * f * 4 + 3 * BT * f * 2),
+        # key scales: the per-column-tile partial sums of squares in, one scale out
+        ("hbm", (f // 128 + 2) * P * 4 + BT * 4),
         ("tensor", 2.0 * d * f * f),
         ("tensor", 2.0 * d * f * P),
         ("tensor", 2.0 * d * f * P),

@@ -93,6 +93,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_version.restype = ctypes.c_char_p
     lib.ttcd_kernel_launch_count.argtypes = []
     lib.ttcd_kernel_launch_count.restype = ctypes.c_ulonglong
+    ll = ctypes.c_longlong
+    lib.ttcd_shard_workspace_size.argtypes = [P]
+    lib.ttcd_shard_workspace_size.restype = sz
+    lib.ttcd_shard_qkv.argtypes = [vp, W, P, ll, vp, vp, sz, vp]
+    lib.ttcd_shard_attend.argtypes = [vp, vp, W, P, ll, vp, vp, sz, vp]
+    lib.ttcd_shard_mix.argtypes = [vp, vp, W, P, ll, vp, vp, sz, vp]
+    lib.ttcd_shard_finish.argtypes = [W, P, ll, vp, vp, vp, vp, sz, vp]
     lib.ttcd_fastweight_mlp_noalloc.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp]
     lib.ttcd_fastweight_mlp_noalloc.restype = i
     lib.ttcd_fastweight_mlp_noalloc_capacity.argtypes = []
@@ -100,7 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in ("ttcd_dual_window_attn", "ttcd_dual_window_attn_lse", "ttcd_fastweight_mlp",
                "ttcd_block_forward", "ttcd_block_forward_profiled", "ttcd_block_workspace_offset",
                "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
-               "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read"):
+               "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read",
+               "ttcd_shard_qkv", "ttcd_shard_attend", "ttcd_shard_mix", "ttcd_shard_finish"):
         getattr(lib, fn).restype = i
     _lib = lib
     return lib
@@ -362,6 +370,85 @@ class Decoder:
                                                self.state.numel(), _ptr(out),
                                                _stream(self.stream)), "ttcd_decode_state_read")
         return out
+
+
+class Shard:
+    """One shard of a sequence-sharded block forward: tokens pos0 .. pos0 + p.T - 1
+    of each of the p.B sequences (pos0 a multiple of p.chunk), bf16.
+
+    The four phases run in order on one workspace; between them the caller
+    passes on what the next shard needs (see ``sharding.shard_block_forward``):
+
+        kv_tail = sh.qkv(x)                      # rotated K/V of the last tokens
+        u_tail = sh.attend(x, kv_halo)           # normalised MLP inputs of the last tokens
+        total = sh.mix(beta, u_halo)             # sum of this shard's chunk increments
+        out, state = sh.finish(state_in)         # state_in = earlier shards' totals
+
+    kv rows are [2, Hkv, hd] (K heads then V heads) per token."""
+
+    def __init__(self, weights: Dict[str, torch.Tensor], p: BlockParams, pos0: int,
+                 device="cuda", stream=None):
+        self.lib = load_library()
+        self.p, self.pc, self.wc, self.pos0 = p, p.c(), _weights(weights), int(pos0)
+        self.weights = weights
+        self.stream = stream
+        self.device = torch.device(device)
+        n = self.lib.ttcd_shard_workspace_size(ctypes.byref(self.pc))
+        if n == 0:
+            raise TTCDError(ERR_INVALID_ARG, "ttcd_shard_workspace_size")
+        self.ws = alloc_workspace(n, device)
+        self.n_halo = min(p.w_T - 1, self.pos0)
+        self.kv_width = 2 * p.n_kv_heads * p.head_dim
+
+    def _ws(self):
+        return _ptr(self.ws), self.ws.numel(), _stream(self.stream)
+
+    def qkv(self, x):
+        p = self.p
+        kv_tail = torch.empty(p.B, min(p.T, p.w_T - 1), self.kv_width, device=self.device,
+                              dtype=torch.bfloat16)
+        _check(self.lib.ttcd_shard_qkv(_ptr(x), ctypes.byref(self.wc), ctypes.byref(self.pc),
+                                       self.pos0, _ptr(kv_tail), *self._ws()), "ttcd_shard_qkv")
+        return kv_tail
+
+    def attend(self, x, kv_halo):
+        p = self.p
+        if kv_halo is not None and kv_halo.shape[1] != self.n_halo:
+            raise ValueError(f"K/V halo of {kv_halo.shape[1]} rows, need {self.n_halo}")
+        if self.n_halo == 0:
+            kv_halo = None
+        u_tail = torch.empty(2, p.B, min(p.T, max(p.conv_k - 1, 0)), p.d_model,
+                             device=self.device, dtype=torch.bfloat16)
+        _check(self.lib.ttcd_shard_attend(_ptr(x), _ptr(kv_halo), ctypes.byref(self.wc),
+                                          ctypes.byref(self.pc), self.pos0,
+                                          _ptr(u_tail) if u_tail.numel() else None,
+                                          *self._ws()), "ttcd_shard_attend")
+        return u_tail
+
+    def mix(self, beta, u_halo):
+        p = self.p
+        nh = min(p.conv_k - 1, self.pos0)
+        if nh > 0 and (u_halo is None or u_halo.shape[2] != nh):
+            raise ValueError(f"MLP-input halo of {None if u_halo is None else u_halo.shape[2]} "
+                             f"rows, need {nh}")
+        total = torch.empty(p.B, p.d_model, p.d_ff, device=self.device, dtype=torch.float32)
+        _check(self.lib.ttcd_shard_mix(_ptr(beta), _ptr(u_halo) if nh > 0 else None,
+                                       ctypes.byref(self.wc), ctypes.byref(self.pc), self.pos0,
+                                       _ptr(total), *self._ws()), "ttcd_shard_mix")
+        return total
+
+    def finish(self, state_in=None, state_out: bool = True):
+        p = self.p
+        out = torch.empty(p.B, p.T, p.d_model, device=self.device, dtype=torch.bfloat16)
+        st = (torch.empty(p.B, p.d_model, p.d_ff, device=self.device, dtype=torch.float32)
+              if state_out else None)
+        _check(self.lib.ttcd_shard_finish(ctypes.byref(self.wc), ctypes.byref(self.pc),
+                                          self.pos0, _ptr(state_in), _ptr(st), _ptr(out),
+                                          *self._ws()), "ttcd_shard_finish")
+        return out, st
+
+    def check_status(self) -> int:
+        return check_device_status(self.ws, self.stream)
 
 
 def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams, h_S=None,

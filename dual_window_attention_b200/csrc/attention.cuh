@@ -49,6 +49,12 @@ struct AttnArgs {
   float scale_log2;  // softmax scale * log2(e)
   int n_qt;          // query tiles per sequence
   int pairs;         // head pairs per KV group = ceil(G / 2)
+  // First query row that is computed and stored (0 for a whole sequence).  A
+  // sequence shard puts the keys and values of the tokens before it in rows
+  // [0, q_begin): they are visible to its queries, but no query of theirs is
+  // computed.  The grid covers query tiles q_begin/128 .. n_qt-1, and outputs
+  // and lse rows are indexed by t - q_begin, T - q_begin rows per sequence.
+  int q_begin;
 };
 
 constexpr int ATT_BM = 128;
@@ -386,9 +392,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + h_local * 128;
     const uint32_t o_addr = tmem + lane_off + 256 + h_local * 128;
-    const bool row_ok = t < a.T;
-    const long long orow = (static_cast<long long>(b) * a.T + t) * a.Hq + head;
-    const long long li = (static_cast<long long>(b) * a.Hq + head) * a.T + t;
+    const bool row_ok = t < a.T && t >= a.q_begin;
+    const int T_out = a.T - a.q_begin;
+    const long long orow = (static_cast<long long>(b) * T_out + (t - a.q_begin)) * a.Hq + head;
+    const long long li = (static_cast<long long>(b) * a.Hq + head) * T_out + (t - a.q_begin);
     const float sl2 = a.scale_log2;
     // m_ref = -inf: nothing visible yet (the first tile, or the far band of the
     // split form before its first visible key); O is zero for such a row.

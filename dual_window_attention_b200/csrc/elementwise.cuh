@@ -178,7 +178,9 @@ __global__ void cast_kernel(const InT* __restrict__ in, OutT* __restrict__ out, 
 // addition (cos, sin)((t+1)a) = (c cos a - s sin a, s cos a + c sin a) in double
 // precision, whose error over a run stays far below the half-precision output.
 constexpr int ROPE_RUN = 64;
-__global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double theta) {
+// pos0: absolute position of row 0 (a sequence shard starts past 0).
+__global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double theta,
+                                  long long pos0 = 0) {
   const int half = hd / 2;
   const int runs = (T + ROPE_RUN - 1) / ROPE_RUN;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -187,7 +189,7 @@ __global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, doubl
   const int t0 = static_cast<int>(idx % runs) * ROPE_RUN;
   const double a = pow(theta, -2.0 * i / hd);
   double s, c, sa, ca;
-  sincos(static_cast<double>(t0) * a, &s, &c);
+  sincos(static_cast<double>(pos0 + t0) * a, &s, &c);
   sincos(a, &sa, &ca);
   __half2* out = cs + static_cast<long long>(i) * T + t0;
   const int n = min(ROPE_RUN, T - t0);
@@ -301,6 +303,52 @@ __global__ void __launch_bounds__(256, CONV_MAXK <= 4 ? 3 : 1)
     hT[0] = zt;
     hS[0] = zs;
   }
+}
+
+// Zeroes the padding rows of the chunk-padded [P, f] buffers D and Kp (padded
+// index p = (b*Nc + i)*Cp + j with j at or past chunk i's token count), which
+// the fused gate/up epilogue does not write: the chunk-scan GEMM contracts over
+// whole 64-token blocks, so those rows must hold zeros.  One thread per 8
+// columns of a row (f a multiple of 8).
+template <class E>
+__global__ void pad_rows_zero_kernel(E* __restrict__ D, E* __restrict__ Kp, int f, int T, int C,
+                                     int Cp, int Nc, long long P) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_row = f / 8;
+  const long long p = idx / per_row;
+  if (p >= P) return;
+  const long long rem = p % (static_cast<long long>(Nc) * Cp);
+  const int i = static_cast<int>(rem / Cp), j = static_cast<int>(rem % Cp);
+  if (j < min(C, T - i * C)) return;
+  const int c = static_cast<int>(idx % per_row) * 8;
+  const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  store8(D + p * f + c, z);
+  store8(Kp + p * f + c, z);
+}
+
+// out[path][b][j][:] = u[row][:] * rstd[row], row = path*BT + b*T + T - n + j,
+// for j < n: the MLP inputs u_P = RMSNorm(h_P) of the last n tokens of every
+// sequence (u holds h * g_mlp, rstd the row scales), which a sequence shard
+// hands to the next one as the history of its short convs.  One thread per 8
+// columns; out is [2, B, n, d].
+template <class E>
+__global__ void u_tail_kernel(const E* __restrict__ u, const float* __restrict__ rstd,
+                              E* __restrict__ out, int B, int T, int d, int n, long long BT) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_row = d / 8;
+  const long long r = idx / per_row;
+  if (r >= 2ll * B * n) return;
+  const int c = static_cast<int>(idx % per_row) * 8;
+  const int j = static_cast<int>(r % n);
+  const long long pb = r / n;
+  const int b = static_cast<int>(pb % B), path = static_cast<int>(pb / B);
+  const long long row = path * BT + static_cast<long long>(b) * T + T - n + j;
+  float v[8];
+  load8(u + row * d + c, v);
+  const float s = rstd[row];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] *= s;
+  store8(out + r * d + c, v);
 }
 
 // kscale[p] = beta[b, t] / sqrt(ssq[p] + eps) for real tokens, 0 for padding, where

@@ -23,11 +23,13 @@ struct TileCtx {
   int row0;        // first A row (== output row) of the tile
   int valid_rows;  // rows of this tile inside its group (<= 128)
   int tn;          // column-tile index
-  int group;       // b * Nc + i
+  int group;       // b * Nc + i (paired tiles: the sequence b)
   int b_row0;      // first B row of this group
+  int tok0;        // paired tiles: token of accumulator row 0 (and of row 64)
 };
 
 struct GemmGeom {
+  static constexpr bool kPaired = false;
   int n_seq, T, C, Nc;  // row groups
   int K;                // reduction length (multiple of 64 not required: TMA zero-fills)
   int tiles_m;          // ceil(C / 128)
@@ -50,6 +52,54 @@ struct GemmGeom {
     return c.valid_rows > 0;
   }
 };
+
+// Paired tiles: accumulator rows 0-63 are the teacher rows of tokens
+// [tok0, tok0 + 64) of sequence b and rows 64-127 the student rows of the same
+// tokens (A = [u_T; u_S], the student half `half_rows` rows further down).
+// Consecutive tiles of a sequence overlap by H = conv_k - 1 tokens, so the
+// epilogue holds the H rows before its first output token and the causal conv
+// needs nothing from other tiles: tile tm outputs tokens [tm (64-H), tm (64-H) +
+// 64-H) and starts at tok0 = tm (64-H) - H (rows before token 0 of sequence 0
+// are zero-filled by the TMA load, and zeroed by the epilogue for every b).
+struct PairGeom {
+  static constexpr bool kPaired = true;
+  int n_seq, T, H, K;
+  int tiles_m;  // ceil(T / (64 - H))
+  int tiles_n;
+  long long half_rows;  // B*T: row offset of the student half of A
+  __host__ __device__ int total() const { return n_seq * tiles_m * tiles_n; }
+  __device__ bool tile(int t, TileCtx& c) const {
+    const int tn = t % tiles_n;
+    const int r = t / tiles_n;
+    const int tm = r % tiles_m;
+    const int b = r / tiles_m;
+    c.tn = tn;
+    c.group = b;
+    c.b_row0 = 0;
+    c.tok0 = tm * (64 - H) - H;
+    c.row0 = b * T + c.tok0;
+    c.valid_rows = GEMM_BM;
+    return true;
+  }
+};
+
+// Barrier and AND-vote over the four epilogue warps (named barrier 1, 128
+// threads).  Collective epilogues call them the same number of times in every
+// warp; the vote on each tile's accumulator wait makes an abort uniform, so no
+// warp leaves the tile loop while another waits at a barrier.
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -149,13 +199,13 @@ struct EpiStage {
   }
 };
 
-template <class E, int BN, int STAGES, bool DUAL_B, class Epi>
+template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
                    const __grid_constant__ CUtensorMap mapB1,
                    const __grid_constant__ CUtensorMap mapOut,
-                   const __grid_constant__ CUtensorMap mapOut2, const GemmGeom geo,
+                   const __grid_constant__ CUtensorMap mapOut2, const Geom geo,
                    const Epi epi, const DevStatus st) {
   constexpr bool STAGED = Epi::kStaged;
   constexpr int A_BYTES = GEMM_BM * 128;
@@ -227,7 +277,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(sa, &mapA, &full[s], kb * BK, c.row0);
+          if constexpr (Geom::kPaired) {  // two 64-row boxes: teacher rows, student rows
+            tma_load_2d(sa, &mapA, &full[s], kb * BK, c.row0);
+            tma_load_2d(sa + (GEMM_BM / 2) * 128, &mapA, &full[s], kb * BK,
+                        static_cast<int>(c.row0 + geo.half_rows));
+          } else {
+            tma_load_2d(sa, &mapA, &full[s], kb * BK, c.row0);
+          }
           if (DUAL_B) {
             tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * (BN / 2));
             tma_load_2d(sb + (BN / 2) * 128, &mapB1, &full[s], kb * BK,
@@ -297,7 +353,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int ab = j & 1;
       // per-row inputs of the epilogue are fetched while the tile is still computing
       const float pre = epi.pre(c, r);
-      if (!mbar_wait(&accf[ab], (j >> 1) & 1, st, abort)) break;
+      bool ok = mbar_wait(&accf[ab], (j >> 1) & 1, st, abort);
+      if constexpr (Epi::kCollective) ok = epi_bar_and(ok);
+      if (!ok) break;
       tc_fence_after();
       epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r,
                            stg, pre);
@@ -362,6 +420,7 @@ __device__ __forceinline__ void emit(EpiStage& stg, bool staged, bool ok, OutT* 
 template <class OutT>
 struct EpiStore {
   static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   OutT* out;
   long long ldo;
   int N;
@@ -399,6 +458,7 @@ using EpiStoreBF16 = EpiStore<__nv_bfloat16>;
 template <class OutT, class ResT>
 struct EpiResidual {
   static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   OutT* out;
   long long ldo;
   const ResT* resid;  // nullable
@@ -445,6 +505,7 @@ struct EpiResidual {
 template <class E, class ResT>
 struct EpiOprojNorm {
   static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   E* hg;
   float* hS;
   float* ssq;
@@ -517,6 +578,7 @@ struct EpiOprojNorm {
 // otherwise A already holds u.
 struct EpiSwiGLU {
   static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   float* out;
   long long ldo;
   int N;  // d_ff
@@ -547,6 +609,140 @@ struct EpiSwiGLU {
   }
 };
 
+// Gate/up with SwiGLU, the two short convs, the value-residual difference and
+// the student keys in one epilogue (papernotes.org review "Learning What to
+// Remember", 关键设计 3: Zbar_P = conv_P(Z_P), D = Zbar_T - Zbar_S, K =
+// l2-norm(Zbar_S); the fast weight reads the raw Z_S, 关键设计 2), on paired
+// tiles (PairGeom): accumulator rows 0-63 hold the teacher rows of 64 tokens and
+// rows 64-127 the student rows of the same tokens; columns [0, 128) are gate and
+// [128, 256) up for output columns tn*128 + [0, 128).
+//
+// Per 32-column slice every thread (one accumulator row) forms
+// z = silu(rstd g) (rstd u) in fp32, then the causal depthwise conv along
+// tokens: the k-1 earlier rows of the same path come from lanes below by warp
+// shuffles, and across the warp boundary from the previous quarter's last rows
+// in shared memory.  The tile's first k-1 rows only feed the conv (their outputs
+// belong to the previous tile).  Teacher warps publish Zbar_T in shared memory;
+// the student warp of the same tokens forms D = Zbar_T - Zbar_S and writes D and
+// Kp = Zbar_S (padded chunk layout), the bf16 Z_S (output-GEMM operand) and, per
+// token, the sum of Zbar_S^2 over the tile's 128 columns (the key norm is a row
+// scale applied to R later).  fp32 Z never reaches memory.
+//   z_halo [2, B, k-1, f] fp32: Z rows before token 0 (nullable: zeros)
+//   z_tail [2, B, k-1, f] fp32: written with the last k-1 rows of Z (nullable)
+// Shared memory: the four 8 KB staging regions; region w holds the Zbar_T slice
+// of its warp as [column][lane] (conflict-free) and, at float 1024, the last 8
+// rows of z as [column][row].
+struct EpiSwiGLUConv {
+  static constexpr bool kStaged = true;      // the staging area is the exchange buffer
+  static constexpr bool kCollective = true;  // the four warps exchange rows
+  __nv_bfloat16* D;
+  __nv_bfloat16* Kp;
+  __nv_bfloat16* Zs;
+  float* ssq;          // [ceil(f/128), P]
+  const float* rstd;   // [2BT] MLP RMSNorm row scales, nullable (u already normalised)
+  const __nv_bfloat16* tapT;  // [f, k]
+  const __nv_bfloat16* tapS;
+  const float* z_halo;
+  float* z_tail;
+  int B, T, f, k, C, Cp, Nc;
+  long long BT, P;
+
+  __device__ float pre(const TileCtx& c, int r) const {
+    const int t = c.tok0 + (r & 63);
+    if (!rstd || t < 0 || t >= T) return 1.f;
+    return __ldg(rstd + (r < 64 ? 0 : BT) + static_cast<long long>(c.group) * T + t);
+  }
+
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
+    static_assert(BN == 256, "gate/up tiles are 128 gate + 128 up columns");
+    const int lane = threadIdx.x & 31;
+    const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quarter: rows 32q .. 32q+31
+    const bool student = q >= 2;
+    const int path = student ? 1 : 0;
+    const int rin = r & 63;
+    const int t = c.tok0 + rin;
+    const int b = c.group;
+    const int H = k - 1;
+    const bool real = t >= 0 && t < T;
+    const bool out_row = rin >= H && real;
+    // regions of the quarters: warps 2, 3, 4, 5 serve quarters 2, 3, 0, 1
+    float* base = reinterpret_cast<float*>(stg.buf) - (((threadIdx.x >> 5) - 2) * 2048);
+    auto region = [&](int quarter) { return base + ((quarter + 2) & 3) * 2048; };
+    float* own = region(q);
+    const float* prev_halo = region(q - 1) + 1024;  // odd quarters only
+    const float* partner = region(q - 2);          // student quarters only
+    const __nv_bfloat16* tap = student ? tapS : tapT;
+    long long p = 0;
+    if (t >= 0) p = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
+    float ssq_acc = 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < 128; cc += 32) {
+      const int col0 = c.tn * 128 + cc;
+      if (col0 >= f) break;  // the same for every warp
+      float z[32];
+      {
+        float g[32], u[32];
+        tmem_ld32f(taddr + cc, g);
+        tmem_ld32f(taddr + 128 + cc, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gg = g[i] * rs;
+          z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (u[i] * rs);
+        }
+      }
+      if (!real) {
+        if (t < 0 && z_halo) {
+          load_x32(z_halo + ((static_cast<long long>(path) * B + b) * H + (t + H)) * f + col0, z);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = 0.f;
+        }
+      }
+      if (z_tail && out_row && t >= T - H)
+        store_f32x32(z_tail + ((static_cast<long long>(path) * B + b) * H + (t - (T - H))) * f + col0, z);
+      // the last 8 rows of the even quarters feed the first rows of the odd ones
+      if (!(q & 1) && lane >= 24) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) own[1024 + i * 8 + (lane - 24)] = z[i];
+      }
+      epi_bar_sync();
+      // Zbar[t] = sum_m tap[c][m] z[t - m]  (tap m multiplies position t - m)
+      float zb[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const __nv_bfloat16* tc = tap + static_cast<long long>(col0 + i) * k;
+        float acc = __bfloat162float(tc[0]) * z[i];
+        for (int m = 1; m <= H; ++m) {
+          float nb = __shfl_up_sync(0xffffffffu, z[i], m);
+          if (lane < m) nb = (q & 1) ? prev_halo[i * 8 + 8 - m + lane] : 0.f;
+          acc += __bfloat162float(tc[m]) * nb;
+        }
+        zb[i] = acc;
+      }
+      if (!student) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) own[i * 32 + lane] = zb[i];
+      }
+      epi_bar_sync();
+      if (student) {
+        float d[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          d[i] = partner[i * 32 + lane] - zb[i];
+          ssq_acc += zb[i] * zb[i];
+        }
+        if (out_row) {
+          store_bf16x32(D + p * f + col0, d);
+          store_bf16x32(Kp + p * f + col0, zb);
+          store_bf16x32(Zs + (static_cast<long long>(b) * T + t) * f + col0, z);
+        }
+      }
+    }
+    if (student && out_row) ssq[static_cast<long long>(c.tn) * P + p] = ssq_acc;
+  }
+};
+
 // QKV projection with rotary embedding on the query and key heads, written to
 // one token-major tensor qkv [rows, (Hq + 2 Hkv) HD]: q heads, then k heads,
 // then v heads (column n of the accumulator is column n of qkv).  Each head's
@@ -555,6 +751,7 @@ struct EpiSwiGLU {
 template <int HD>
 struct EpiQKVRope {
   static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   static constexpr int NF = HD / 2;  // rotation frequencies
   __nv_bfloat16* qkv;
   int ld;         // (Hq + 2 Hkv) * HD
@@ -562,6 +759,10 @@ struct EpiQKVRope {
   int T;
   const __half2* rope_cs;  // [HD/2][T] (cos, sin), frequency-major
   const float* rstd;       // [rows] input RMSNorm row scale (the gain is in the weight), nullable
+  // Rows reserved before each sequence's rows in qkv (a sequence shard's K/V
+  // halo): output row = row + (b + 1) * row_shift for sequence b = tile group
+  // (tiles must not straddle sequences when it is nonzero).
+  int row_shift;
   __device__ float pre(const TileCtx& c, int r) const {
     return (rstd && r < c.valid_rows) ? __ldg(rstd + c.row0 + r) : 1.f;
   }
@@ -589,6 +790,7 @@ struct EpiQKVRope {
     static_assert(BN % 64 == 0 && BN % HD == 0, "column tile must hold whole heads");
     const bool ok = r < c.valid_rows;
     const long long row = c.row0 + r;
+    const int shift = (c.group + 1) * row_shift;
     const int wrow = r & ~31;
     const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
     const int t = static_cast<int>(row % T);
@@ -634,7 +836,7 @@ struct EpiQKVRope {
         lo[i] *= rs;
         hi[i] *= rs;
       }
-      emit(stg, staged, ok, qkv + row * ld, tcol + cc, c.row0 + wrow, lo, hi);
+      emit(stg, staged, ok, qkv + (row + shift) * ld, tcol + cc, c.row0 + wrow + shift, lo, hi);
     }
   }
 };

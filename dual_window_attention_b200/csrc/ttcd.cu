@@ -145,14 +145,14 @@ bool make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
   return make_map<OutT>(m, ptr, cols, rows, ld_elems * sizeof(OutT), 128 / sizeof(OutT), 32);
 }
 
-template <class E, int BN, int STAGES, bool DUAL, class Epi>
+template <class E, int BN, int STAGES, bool DUAL, class Epi, class Geom = GemmGeom>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
-                        const CUtensorMap& B1, const CUtensorMap* out_map, const GemmGeom& geo,
+                        const CUtensorMap& B1, const CUtensorMap* out_map, const Geom& geo,
                         const Epi& epi, const CUtensorMap* out_map2 = nullptr) {
   const int total = geo.total();
   if (total <= 0) return TTCD_OK;
   if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
-  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi>;
+  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom>;
   constexpr int smem = gemm_smem_bytes<BN, STAGES, Epi::kStaged>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -207,13 +207,13 @@ struct Layout {
 enum Buf {
   B_STATUS, B_WQKVG, B_RSTDIN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ,
   B_KSCALE, B_R, B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_RSTD, B_X32, B_OUT32, B_HS32,
-  B_W32, B_COUNT
+  B_W32, B_QKVX, B_ZH, B_UH, B_COUNT
 };
 static_assert(B_COUNT <= 32, "workspace layout table too small");
 const char* kBufNames[B_COUNT] = {"status", "wqkv_g", "rstd_in", "qkv", "o", "h", "rope", "u",
                                   "Z", "Zs16", "D", "Kp", "ssq", "kscale", "R", "Wall", "M",
                                   "WprojT", "Rt", "Kt", "hssq", "rstd", "x32", "out32", "hS32",
-                                  "w32"};
+                                  "w32", "qkv_ext", "z_halo", "u_halo"};
 
 // bf16 problems shorter than one chunk run with fp32 operands (kind::tf32 MMAs):
 // their fast-weight state is the sum of fewer than C rank-1 writes, so the bf16
@@ -264,10 +264,10 @@ Dims dims_of(const ttcd_block_params* p) {
 // Operand buffers hold bf16 for TTCD_BF16 and fp32 (tf32 tensor-core operands)
 // for TTCD_F32 and the wide route; q, k, v stay bf16 (the attention kernel takes
 // bf16).  The status word comes first in every workspace.
-Layout make_layout(const ttcd_block_params* p, bool block) {
+Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false) {
   const Dims m = dims_of(p);
   size_t sz[B_COUNT] = {0};
-  const bool wide = wide_mode(p);
+  const bool wide = !shard && wide_mode(p);
   const size_t e = (p->dtype == TTCD_F32 || wide) ? 4 : 2;
   sz[B_STATUS] = kStatusBytes;
   if (block) {
@@ -281,7 +281,7 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
     sz[B_ROPE] = static_cast<size_t>(p->T) * (m.hd / 2) * 4;
   }
   sz[B_U] = 2 * m.BT * m.d * e;
-  sz[B_Z] = 2 * m.BT * m.f * 4;
+  sz[B_Z] = e == 4 ? 2 * m.BT * m.f * 4 : 0;  // bf16: Z stays on chip (fused gate/up + conv)
   sz[B_ZS16] = e == 2 ? m.BT * m.f * 2 : 0;  // fp32 mode reads Z_S directly
   sz[B_D] = m.P * m.f * e;
   sz[B_KP] = m.P * m.f * e;
@@ -294,6 +294,13 @@ Layout make_layout(const ttcd_block_params* p, bool block) {
   if (e == 4) {  // tf32 operands stay K-major: transposed copies for the chunk scan
     sz[B_RT] = m.P * m.d * e;
     sz[B_KT] = m.P * m.f * e;
+  }
+  if (shard) {  // sequence shard: qkv with room for the K/V halo, conv history
+    const size_t H = static_cast<size_t>(p->conv_k - 1);
+    sz[B_QKV] = 0;
+    sz[B_QKVX] = static_cast<size_t>(p->B) * (p->w_T - 1 + p->T) * m.dqkv * 2;
+    sz[B_ZH] = 2 * static_cast<size_t>(p->B) * H * m.f * 4;
+    sz[B_UH] = 2 * static_cast<size_t>(p->B) * H * m.d * e;
   }
   if (wide) {  // fp32 copies of the bf16 interface tensors
     if (block) sz[B_X32] = m.BT * m.d * 4;
@@ -329,7 +336,7 @@ template <int HD, class OutT, bool SPLIT = false>
 ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
                         OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv,
                         int w_S, int w_T, float scale, long long ld_q, long long ld_kv,
-                        OutT* o_far = nullptr, float* lse_far = nullptr) {
+                        OutT* o_far = nullptr, float* lse_far = nullptr, int q_begin = 0) {
   CUtensorMap mq, mk, mv;
   const long long BT = static_cast<long long>(B) * T;
   using bf = __nv_bfloat16;
@@ -353,11 +360,14 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_qt = (T + ATT_BM - 1) / ATT_BM;
   a.pairs = (Hq / Hkv + 1) / 2;
+  a.q_begin = q_begin;
+  if (q_begin < 0 || q_begin >= T) return TTCD_ERR_INVALID_ARG;
   auto kern = dual_window_attn_kernel<HD, OutT, SPLIT>;
   constexpr int smem = AttnCfg<HD>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
-  const long long grid = static_cast<long long>(a.n_qt) * B * Hkv * a.pairs;
+  const long long grid =
+      static_cast<long long>(a.n_qt - q_begin / ATT_BM) * B * Hkv * a.pairs;
   if (grid >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
   kern<<<static_cast<unsigned>(grid), ATT_THREADS, smem, c.s>>>(mq, mk, mv, a, c.st);
   TTCD_CHECK_LAUNCH();
@@ -367,11 +377,12 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
 template <class OutT>
 ttcd_status run_attn(const Ctx& c, const void* q, const void* k, const void* v, OutT* o_T,
                      OutT* o_S, float* lse_T, float* lse_S, int B, int T, int Hq, int Hkv, int hd,
-                     int w_S, int w_T, float scale, long long ld_q, long long ld_kv) {
+                     int w_S, int w_T, float scale, long long ld_q, long long ld_kv,
+                     int q_begin = 0) {
   switch (hd) {
-    case 32: return launch_attn<32>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
-    case 64: return launch_attn<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
-    case 128: return launch_attn<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv);
+    case 32: return launch_attn<32>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv, static_cast<OutT*>(nullptr), nullptr, q_begin);
+    case 64: return launch_attn<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv, static_cast<OutT*>(nullptr), nullptr, q_begin);
+    case 128: return launch_attn<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, B, T, Hq, Hkv, w_S, w_T, scale, ld_q, ld_kv, static_cast<OutT*>(nullptr), nullptr, q_begin);
     default: return TTCD_ERR_UNSUPPORTED;
   }
 }
@@ -400,12 +411,17 @@ ttcd_status launch_attn_lse(const Ctx& c, const void* q, const void* k, const vo
 // With `hssq` set, u holds h * g_mlp and RMSNorm is finished as a row scale in
 // the gate/up epilogue, from the partial sums of squares hssq [n_part, 2BT]
 // reduced to one 1/rms per row first.
-template <class E, class OutT, class ResT>
-ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
-                         const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
-                         const E* conv_T, const E* conv_S, const float* beta,
-                         const float* state_in, float* state_out, const ResT* h_S, OutT* y,
-                         int mark, const float* hssq) {
+// Front half of the fast-weight MLP: from u (operand type E, [2BT, d], teacher
+// rows first, already in the workspace) to D, the keys and R.  When `rstd` is
+// set, u holds h * g_mlp and the MLP RMSNorm is finished as the row scale rstd
+// in the gate/up epilogue.  `z_halo` (bf16 operands only, nullable): Z_T, Z_S of
+// the conv_k - 1 tokens before token 0 ([2, B, conv_k-1, f] fp32; a sequence
+// shard's conv history), zeros when null.
+template <class E>
+ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
+                      const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
+                      const E* conv_T, const E* conv_S, const float* beta, int mark,
+                      const float* rstd, const float* z_halo) {
   const Dims m = dims_of(p);
   E* u = at<E>(ws, L, B_U);
   float* Z = at<float>(ws, L, B_Z);
@@ -415,45 +431,70 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   float* ssq = at<float>(ws, L, B_SSQ);
   float* kscale = at<float>(ws, L, B_KSCALE);
   E* R = at<E>(ws, L, B_R);
-  E* Wall = at<E>(ws, L, B_WALL);
   E* M = at<E>(ws, L, B_M);
   E* WprojT = at<E>(ws, L, B_WPROJT);
   stage_mark(c, mark);
 
-  // Z_P = silu(u_P W_gate^T) * (u_P W_up^T), both paths stacked (slow weights).
-  {
+  if constexpr (sizeof(E) == 2) {
+    // Z_P = silu(u_P W_gate^T) * (u_P W_up^T) for both paths of the same tokens
+    // in one tile, with the convs, D, the unnormalised keys, their sums of
+    // squares and the bf16 Z_S in the epilogue (slow weights, off-policy).
+    const int H = p->conv_k - 1;
     CUtensorMap mA, mB0, mB1;
-    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 128) ||
+    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 64) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 128) ||
         !map_rows<E>(&mB1, w_up, m.f, m.d, 128))
       return TTCD_ERR_CUDA;
-    CUtensorMap mo;
-    if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
-    float* rstd = nullptr;
-    if (hssq) {
-      rstd = at<float>(ws, L, B_RSTD);
-      rms_rstd_kernel<<<cdiv(2 * m.BT, 256), 256, 0, c.s>>>(hssq, cdiv(m.d, 256), 2 * m.BT,
-                                                            1.0f / m.d, p->rms_eps, rstd);
+    PairGeom g;
+    g.n_seq = p->B;
+    g.T = p->T;
+    g.H = H;
+    g.K = m.d;
+    g.tiles_m = cdiv(p->T, 64 - H);
+    g.tiles_n = cdiv(m.f, 128);
+    g.half_rows = m.BT;
+    EpiSwiGLUConv e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
+                    p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
+    TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+    stage_mark(c, mark + 1);
+    if (m.Cp != p->chunk || p->T % p->chunk != 0) {
+      const long long n = m.P * (m.f / 8);
+      pad_rows_zero_kernel<E><<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+          D, Kp, m.f, p->T, p->chunk, m.Cp, m.Nc, m.P);
       TTCD_CHECK_LAUNCH();
     }
-    EpiSwiGLU e{Z, m.f, m.f, rstd};
-    TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
-  }
-  stage_mark(c, mark + 1);
-  // Short convs, residual difference, student keys (unnormalised) and their squares.
-  {
-    dim3 grid(m.f / CONV_TC, static_cast<unsigned>(m.P / CONV_TP));
-    if (p->conv_k <= 4)
-      conv_residual_key_kernel<E, E, 4><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
-                                                               p->T, m.f, p->conv_k, p->chunk,
-                                                               m.Cp, m.Nc, m.BT, m.P);
-    else
-      conv_residual_key_kernel<E, E, 8><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
-                                                               p->T, m.f, p->conv_k, p->chunk,
-                                                               m.Cp, m.Nc, m.BT, m.P);
-    TTCD_CHECK_LAUNCH();
-    key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, m.f / CONV_TC, beta, kscale, p->T,
+    key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, cdiv(m.f, 128), beta, kscale, p->T,
                                                       p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
     TTCD_CHECK_LAUNCH();
+  } else {
+    // fp32 operands (tf32): Z_P = silu(u_P W_gate^T) * (u_P W_up^T) for the stacked
+    // paths into fp32 Z, then the conv/residual/key kernel.
+    {
+      CUtensorMap mA, mB0, mB1;
+      if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) || !map_rows<E>(&mB0, w_gate, m.f, m.d, 128) ||
+          !map_rows<E>(&mB1, w_up, m.f, m.d, 128))
+        return TTCD_ERR_CUDA;
+      CUtensorMap mo;
+      if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
+      EpiSwiGLU e{Z, m.f, m.f, rstd};
+      TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
+    }
+    stage_mark(c, mark + 1);
+    // Short convs, residual difference, student keys (unnormalised) and their squares.
+    {
+      dim3 grid(m.f / CONV_TC, static_cast<unsigned>(m.P / CONV_TP));
+      if (p->conv_k <= 4)
+        conv_residual_key_kernel<E, E, 4><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
+                                                                 p->T, m.f, p->conv_k, p->chunk,
+                                                                 m.Cp, m.Nc, m.BT, m.P);
+      else
+        conv_residual_key_kernel<E, E, 8><<<grid, 256, 0, c.s>>>(Z, conv_T, conv_S, D, Kp, Zs, ssq,
+                                                                 p->T, m.f, p->conv_k, p->chunk,
+                                                                 m.Cp, m.Nc, m.BT, m.P);
+      TTCD_CHECK_LAUNCH();
+      key_scale_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(ssq, m.f / CONV_TC, beta, kscale, p->T,
+                                                        p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
+      TTCD_CHECK_LAUNCH();
+    }
   }
   stage_mark(c, mark + 2);
   // M = W_down W_proj (associativity of W_down (W_proj d_t)).
@@ -481,7 +522,20 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
   }
   stage_mark(c, mark + 4);
-  // Delta W per chunk, fp32 exclusive prefix scan, W_i = W_down + S_i.
+  return TTCD_OK;
+}
+
+// The chunk scan over R and the keys: Delta W_i = R_i^T K'_i, the fp32 exclusive
+// prefix S_i from state_in, and (w_all set) W_i = W_down + S_i per chunk.  With
+// `whole` set, the padded tokens of each sequence form one chunk: state_out is
+// state_in + the sum of all chunk increments (a sequence shard's total).
+template <class E>
+ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
+                        const E* w_down, const float* state_in, float* state_out, E* w_all,
+                        bool whole) {
+  const Dims m = dims_of(p);
+  E* R = at<E>(ws, L, B_R);
+  E* Kp = at<E>(ws, L, B_KP);
   {
     CUtensorMap mR, mK;
     constexpr uint32_t BK = ElemTraits<E>::BK;
@@ -505,12 +559,12 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     ScanArgs<E> a;
     a.d = m.d;
     a.f = m.f;
-    a.Nc = m.Nc;
-    a.Cp = m.Cp;
+    a.Nc = whole ? 1 : m.Nc;
+    a.Cp = whole ? m.Nc * m.Cp : m.Cp;
     a.w_down = w_down;
     a.state_in = state_in;
     a.state_out = state_out;
-    a.w_all = Wall;
+    a.w_all = w_all;
     a.tiles_m = cdiv(m.d, 128);
     a.tiles_n = cdiv(m.f, SCAN_BN);
     constexpr int STAGES = 4;
@@ -521,6 +575,20 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
     kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
     TTCD_CHECK_LAUNCH();
   }
+  return TTCD_OK;
+}
+
+// Back half of the fast-weight MLP: the chunk scan from state_in, then
+// y = h_S + (W_down + S_i) Z_S, one GEMM per chunk with its own weight.
+template <class E, class OutT, class ResT>
+ttcd_status mlp_back(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
+                     const E* w_down, const float* state_in, float* state_out, const ResT* h_S,
+                     OutT* y, int mark) {
+  const Dims m = dims_of(p);
+  float* Z = at<float>(ws, L, B_Z);
+  E* Zs = sizeof(E) == 2 ? at<E>(ws, L, B_ZS16) : nullptr;
+  E* Wall = at<E>(ws, L, B_WALL);
+  TTCD_TRY(launch_scan<E>(c, p, L, ws, w_down, state_in, state_out, Wall, false));
   stage_mark(c, mark + 5);
   // y = h_S + (W_down + S_i) Z_S, one GEMM per chunk with its own weight.
   {
@@ -545,6 +613,17 @@ ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout&
   }
   stage_mark(c, mark + 6);
   return TTCD_OK;
+}
+
+template <class E, class OutT, class ResT>
+ttcd_status run_mlp_core(const Ctx& c, const ttcd_block_params* p, const Layout& L, void* ws,
+                         const E* w_gate, const E* w_up, const E* w_down, const E* w_proj,
+                         const E* conv_T, const E* conv_S, const float* beta,
+                         const float* state_in, float* state_out, const ResT* h_S, OutT* y,
+                         int mark, const float* rstd) {
+  TTCD_TRY(mlp_front<E>(c, p, L, ws, w_gate, w_up, w_down, w_proj, conv_T, conv_S, beta, mark,
+                        rstd, nullptr));
+  return mlp_back<E, OutT, ResT>(c, p, L, ws, w_down, state_in, state_out, h_S, y, mark);
 }
 
 bool weights_ok(const ttcd_block_weights* w, bool block) {
@@ -664,29 +743,22 @@ ttcd_status mlp_entry(const void* u_T, const void* u_S, const void* h_S, const f
       static_cast<const float*>(h_S), static_cast<float*>(y), 0, nullptr);
 }
 
-// The block for operand type E (bf16: kind::f16 tensor cores; fp32: kind::tf32).
-// x, the weights and out are E; the wide route calls it with fp32 copies.
+// S0: rotary table at positions pos0 .., the input RMSNorm as row scales with
+// its gain folded into a copy of W_qkv, and the QKV GEMM with RoPE into qkv.
+// With n_halo > 0 (a sequence shard), each sequence's rows are preceded by
+// n_halo rows reserved for the K/V of the tokens before it, and the GEMM tiles
+// keep to one sequence.
 template <class E>
-ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
-                      const ttcd_block_weights* w, const ttcd_block_params* p,
-                      const float* state_in, float* state_out, void* out, void* ws,
-                      const Layout& L) {
+ttcd_status block_qkv(const Ctx& c, const E* xin, const ttcd_block_weights* w,
+                      const ttcd_block_params* p, void* ws, const Layout& L,
+                      __nv_bfloat16* qkv, int n_halo, long long pos0) {
   const Dims m = dims_of(p);
   E* wg = at<E>(ws, L, B_WQKVG);
   float* rstd_in = at<float>(ws, L, B_RSTDIN);
-  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
-  E* o = at<E>(ws, L, B_O);
-  float* h = at<float>(ws, L, B_H);
   __half2* rope = at<__half2>(ws, L, B_ROPE);
-  E* u = at<E>(ws, L, B_U);
-  float* hssq = at<float>(ws, L, B_HSSQ);
-  const E* xin = static_cast<const E*>(x);
-
-  // Rotary table; the input RMSNorm as a row scale 1/rms(x) applied in the QKV
-  // epilogue, with its gain folded into the weight: xn W^T = rstd (x (W diag g)^T).
   stage_mark(c, 0);
   rope_table_kernel<<<cdiv(static_cast<long long>(cdiv(p->T, ROPE_RUN)) * (m.hd / 2), 256), 256, 0, c.s>>>(
-      rope, p->T, m.hd, static_cast<double>(p->rope_theta));
+      rope, p->T, m.hd, static_cast<double>(p->rope_theta), pos0);
   TTCD_CHECK_LAUNCH();
   rms_rowscale_kernel<E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(xin, rstd_in, m.BT, m.d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
@@ -697,29 +769,47 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
     TTCD_CHECK_LAUNCH();
   }
   stage_mark(c, 1);
-
-  // Shared Q/K/V with RoPE.
-  {
-    CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, xin, m.BT, m.d, 128) || !map_rows<E>(&mB, wg, m.dqkv, m.d, 256))
-      return TTCD_ERR_CUDA;
-    const GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
-    CUtensorMap mo;
-    if (!make_out_map<__nv_bfloat16>(&mo, qkv, m.BT, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
-    const int n_rope = (m.Hq + m.Hkv) * m.hd;
-    switch (m.hd) {
-      case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
-      case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
-      default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in}))); break;
-    }
+  CUtensorMap mA, mB;
+  if (!map_rows<E>(&mA, xin, m.BT, m.d, 128) || !map_rows<E>(&mB, wg, m.dqkv, m.d, 256))
+    return TTCD_ERR_CUDA;
+  GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
+  if (n_halo > 0) {  // one row group per sequence
+    g.n_seq = p->B;
+    g.T = p->T;
+    g.C = p->T;
+    g.tiles_m = cdiv(p->T, GEMM_BM);
+  }
+  CUtensorMap mo;
+  const long long rows_out = m.BT + static_cast<long long>(p->B) * n_halo;
+  if (!make_out_map<__nv_bfloat16>(&mo, qkv, rows_out, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
+  const int n_rope = (m.Hq + m.Hkv) * m.hd;
+  switch (m.hd) {
+    case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
+    case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
+    default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
   }
   stage_mark(c, 2);
+  return TTCD_OK;
+}
+
+// S1-S2b: dual-window attention of each sequence's T rows over keys that start
+// n_halo rows earlier (qkv as block_qkv left it), o_proj of both paths with the
+// residual, and the MLP RMSNorm row scales.
+template <class E>
+ttcd_status block_attend(const Ctx& c, const E* xin, const ttcd_block_weights* w,
+                         const ttcd_block_params* p, void* ws, const Layout& L,
+                         const __nv_bfloat16* qkv, int n_halo) {
+  const Dims m = dims_of(p);
+  E* o = at<E>(ws, L, B_O);
+  float* h = at<float>(ws, L, B_H);
+  E* u = at<E>(ws, L, B_U);
+  float* hssq = at<float>(ws, L, B_HSSQ);
   // Dual-window attention: o_T rows then o_S rows.
   const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
   TTCD_TRY(run_attn<E>(c, qkv, qkv + static_cast<long long>(m.Hq) * m.hd,
                        qkv + static_cast<long long>(m.Hq + m.Hkv) * m.hd, o,
-                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq, m.Hkv, m.hd,
-                       p->w_S, p->w_T, sc, m.dqkv, m.dqkv));
+                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T + n_halo, m.Hq,
+                       m.Hkv, m.hd, p->w_S, p->w_T, sc, m.dqkv, m.dqkv, n_halo));
   stage_mark(c, 3);
   // h_P = x + o_P W_o^T (fp32), both paths in one GEMM.
   {
@@ -737,15 +827,33 @@ ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
     EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
     TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e, &mo2)));
   }
+  // The MLP RMSNorm's 1/rms per row, from the o_proj epilogue's partial sums.
+  rms_rstd_kernel<<<cdiv(2 * m.BT, 256), 256, 0, c.s>>>(hssq, cdiv(m.d, 256), 2 * m.BT,
+                                                        1.0f / m.d, p->rms_eps,
+                                                        at<float>(ws, L, B_RSTD));
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
 
-  const float* h_S = h;
+// The block for operand type E (bf16: kind::f16 tensor cores; fp32: kind::tf32).
+// x, the weights and out are E; the wide route calls it with fp32 copies.
+template <class E>
+ttcd_status run_block(const Ctx& c, const void* x, const float* beta,
+                      const ttcd_block_weights* w, const ttcd_block_params* p,
+                      const float* state_in, float* state_out, void* out, void* ws,
+                      const Layout& L) {
+  const E* xin = static_cast<const E*>(x);
+  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
+  TTCD_TRY(block_qkv<E>(c, xin, w, p, ws, L, qkv, 0, 0));
+  TTCD_TRY(block_attend<E>(c, xin, w, p, ws, L, qkv, 0));
   return run_mlp_core<E, E, float>(c, p, L, ws, static_cast<const E*>(w->w_gate),
                                    static_cast<const E*>(w->w_up),
                                    static_cast<const E*>(w->w_down),
                                    static_cast<const E*>(w->w_proj),
                                    static_cast<const E*>(w->conv_T),
                                    static_cast<const E*>(w->conv_S), beta, state_in, state_out,
-                                   h_S, static_cast<E*>(out), 4, hssq);
+                                   at<float>(ws, L, B_H), static_cast<E*>(out), 4,
+                                   at<float>(ws, L, B_RSTD));
 }
 
 // ttcd_block_forward with optional stage-boundary events (profiled calls).
@@ -916,6 +1024,169 @@ ttcd_status ttcd_block_forward_profiled(const void* x, const float* beta,
     if (!events[i]) return TTCD_ERR_INVALID_ARG;
   return block_entry(x, beta, w, p, nullptr, state_out, out, workspace, ws_bytes, stream,
                      reinterpret_cast<const cudaEvent_t*>(events), n_events);
+}
+
+// ---------------------------------------------------------------- sequence shards
+size_t ttcd_shard_workspace_size(const ttcd_block_params* p) {
+  if (check_params(p) != TTCD_OK || p->dtype != TTCD_BF16) return 0;
+  return make_layout(p, true, true).total;
+}
+
+}  // extern "C"
+
+namespace {
+// Common checks of the shard phases; on success fills the layout and the
+// context (status word in the workspace) and the K/V halo length.
+ttcd_status shard_begin(const ttcd_block_params* p, long long pos0, void* workspace,
+                        size_t ws_bytes, void* stream, Layout& L, Ctx& c, int& n_halo) {
+  TTCD_TRY(check_params(p));
+  if (p->dtype != TTCD_BF16) return TTCD_ERR_UNSUPPORTED;
+  if (pos0 < 0 || pos0 % p->chunk != 0 || !aligned16(workspace)) return TTCD_ERR_INVALID_ARG;
+  if (pos0 + p->T >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
+  L = make_layout(p, true, true);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  TTCD_TRY(make_ctx(stream, c, at<void>(workspace, L, B_STATUS)));
+  n_halo = static_cast<int>(std::min<long long>(p->w_T - 1, pos0));
+  return TTCD_OK;
+}
+
+// Strided copy of `rows` rows of `width` bytes per sequence, as B 2-D copies.
+ttcd_status copy_rows(const Ctx& c, int B, void* dst, size_t dpitch, size_t dseq,
+                      const void* src, size_t spitch, size_t sseq, size_t width, size_t rows) {
+  if (rows == 0) return TTCD_OK;
+  for (int b = 0; b < B; ++b) {
+    if (cudaMemcpy2DAsync(static_cast<uint8_t*>(dst) + b * dseq, dpitch,
+                          static_cast<const uint8_t*>(src) + b * sseq, spitch, width, rows,
+                          cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+  }
+  return TTCD_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ttcd_status ttcd_shard_qkv(const void* x, const ttcd_block_weights* w, const ttcd_block_params* p,
+                           long long pos0, void* kv_tail, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  if (!aligned16(x) || !weights_ok(w, true) || (kv_tail && !aligned16(kv_tail)))
+    return TTCD_ERR_INVALID_ARG;
+  Layout L;
+  Ctx c;
+  int n_halo = 0;
+  TTCD_TRY(shard_begin(p, pos0, workspace, ws_bytes, stream, L, c, n_halo));
+  using bf = __nv_bfloat16;
+  const Dims m = dims_of(p);
+  bf* qkvx = at<bf>(workspace, L, B_QKVX);
+  TTCD_TRY(block_qkv<bf>(c, static_cast<const bf*>(x), w, p, workspace, L, qkvx, n_halo, pos0));
+  if (kv_tail) {  // K, V of this shard's last min(T, w_T - 1) tokens
+    const size_t kvw = 2 * static_cast<size_t>(m.Hkv) * m.hd * 2, rowb = m.dqkv * 2;
+    const size_t nt = std::min(p->T, p->w_T - 1);
+    TTCD_TRY(copy_rows(c, p->B, kv_tail, kvw, nt * kvw,
+                       reinterpret_cast<uint8_t*>(qkvx) + (n_halo + p->T - nt) * rowb +
+                           static_cast<size_t>(m.Hq) * m.hd * 2,
+                       rowb, (n_halo + p->T) * rowb, kvw, nt));
+  }
+  return TTCD_OK;
+}
+
+ttcd_status ttcd_shard_attend(const void* x, const void* kv_halo, const ttcd_block_weights* w,
+                              const ttcd_block_params* p, long long pos0, void* u_tail,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(x) || !weights_ok(w, true) || (u_tail && !aligned16(u_tail)) ||
+      (kv_halo && !aligned16(kv_halo)))
+    return TTCD_ERR_INVALID_ARG;
+  Layout L;
+  Ctx c;
+  int n_halo = 0;
+  TTCD_TRY(shard_begin(p, pos0, workspace, ws_bytes, stream, L, c, n_halo));
+  if (n_halo > 0 && !kv_halo) return TTCD_ERR_INVALID_ARG;
+  using bf = __nv_bfloat16;
+  const Dims m = dims_of(p);
+  bf* qkvx = at<bf>(workspace, L, B_QKVX);
+  const size_t kvw = 2 * static_cast<size_t>(m.Hkv) * m.hd * 2, rowb = m.dqkv * 2;
+  const size_t qw = static_cast<size_t>(m.Hq) * m.hd * 2, seqb = (n_halo + p->T) * rowb;
+  // the halo's K and V in front of each sequence's rows; its query columns zeroed
+  TTCD_TRY(copy_rows(c, p->B, reinterpret_cast<uint8_t*>(qkvx) + qw, rowb, seqb, kv_halo, kvw,
+                     n_halo * kvw, kvw, n_halo));
+  for (int b = 0; n_halo > 0 && b < p->B; ++b)
+    if (cudaMemset2DAsync(reinterpret_cast<uint8_t*>(qkvx) + b * seqb, rowb, 0, qw, n_halo,
+                          c.s) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+  TTCD_TRY(block_attend<bf>(c, static_cast<const bf*>(x), w, p, workspace, L, qkvx, n_halo));
+  if (u_tail && p->conv_k > 1) {  // normalised MLP inputs of the last min(T, k-1) tokens
+    const int n = std::min(p->T, p->conv_k - 1);
+    const long long threads = 2ll * p->B * n * (m.d / 8);
+    u_tail_kernel<bf><<<static_cast<unsigned>(cdiv(threads, 256)), 256, 0, c.s>>>(
+        at<bf>(workspace, L, B_U), at<float>(workspace, L, B_RSTD), static_cast<bf*>(u_tail),
+        p->B, p->T, m.d, n, m.BT);
+    TTCD_CHECK_LAUNCH();
+  }
+  return TTCD_OK;
+}
+
+ttcd_status ttcd_shard_mix(const float* beta, const void* u_halo, const ttcd_block_weights* w,
+                           const ttcd_block_params* p, long long pos0, float* total,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(beta) || !weights_ok(w, false) || !aligned16(total) ||
+      (u_halo && !aligned16(u_halo)))
+    return TTCD_ERR_INVALID_ARG;
+  Layout L;
+  Ctx c;
+  int n_halo = 0;
+  TTCD_TRY(shard_begin(p, pos0, workspace, ws_bytes, stream, L, c, n_halo));
+  using bf = __nv_bfloat16;
+  const Dims m = dims_of(p);
+  const int H = p->conv_k - 1;
+  const int nh = static_cast<int>(std::min<long long>(H, pos0));
+  if (nh > 0 && !u_halo) return TTCD_ERR_INVALID_ARG;
+  float* zh = nullptr;
+  if (H > 0) {
+    // Z_T, Z_S of the H tokens before the shard from the previous shard's u rows
+    // (zero rows, hence zero Z, before the sequence start).
+    bf* uh = at<bf>(workspace, L, B_UH);
+    zh = at<float>(workspace, L, B_ZH);
+    const size_t rowb = static_cast<size_t>(m.d) * 2;
+    if (cudaMemsetAsync(uh, 0, 2 * static_cast<size_t>(p->B) * H * rowb, c.s) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+    for (int pb = 0; nh > 0 && pb < 2 * p->B; ++pb)
+      if (cudaMemcpyAsync(reinterpret_cast<uint8_t*>(uh) + (static_cast<size_t>(pb) * H + (H - nh)) * rowb,
+                          static_cast<const uint8_t*>(u_halo) + static_cast<size_t>(pb) * nh * rowb,
+                          nh * rowb, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+        return TTCD_ERR_CUDA;
+    CUtensorMap mA, mB0, mB1, mo;
+    const long long rows = 2ll * p->B * H;
+    if (!map_rows<bf>(&mA, uh, rows, m.d, 128) || !map_rows<bf>(&mB0, w->w_gate, m.f, m.d, 128) ||
+        !map_rows<bf>(&mB1, w->w_up, m.f, m.d, 128) ||
+        !make_out_map<float>(&mo, zh, rows, m.f, m.f))
+      return TTCD_ERR_CUDA;
+    EpiSwiGLU e{zh, m.f, m.f, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(rows, cdiv(m.f, 128), m.d), e)));
+  }
+  TTCD_TRY(mlp_front<bf>(c, p, L, workspace, static_cast<const bf*>(w->w_gate),
+                         static_cast<const bf*>(w->w_up), static_cast<const bf*>(w->w_down),
+                         static_cast<const bf*>(w->w_proj), static_cast<const bf*>(w->conv_T),
+                         static_cast<const bf*>(w->conv_S), beta, 4,
+                         at<float>(workspace, L, B_RSTD), zh));
+  // this shard's total: all its padded tokens as one chunk, from a zero state
+  return launch_scan<bf>(c, p, L, workspace, static_cast<const bf*>(w->w_down), nullptr, total,
+                         nullptr, true);
+}
+
+ttcd_status ttcd_shard_finish(const ttcd_block_weights* w, const ttcd_block_params* p,
+                              long long pos0, const float* state_in, float* state_out, void* out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!weights_ok(w, false) || !aligned16(out) || (state_in && !aligned16(state_in)) ||
+      (state_out && !aligned16(state_out)))
+    return TTCD_ERR_INVALID_ARG;
+  Layout L;
+  Ctx c;
+  int n_halo = 0;
+  TTCD_TRY(shard_begin(p, pos0, workspace, ws_bytes, stream, L, c, n_halo));
+  using bf = __nv_bfloat16;
+  return mlp_back<bf, bf, float>(c, p, L, workspace, static_cast<const bf*>(w->w_down), state_in,
+                                 state_out, at<float>(workspace, L, B_H), static_cast<bf*>(out),
+                                 4);
 }
 
 }  // extern "C"

@@ -12,8 +12,12 @@ convs, a causal prefix over chunks):
 
 This module moves those with torch.distributed (NCCL between GPUs, gloo on the
 CPU); it does no arithmetic of the method beyond summing the gathered state
-totals in rank order.  The kernels that consume the halos (RoPE at a position
-offset, attention and conv over a leading halo) are not part of the library yet.
+totals in rank order.  ``shard_block_forward`` runs one rank's shard through
+the library's four shard phases (ttcd_shard_qkv, _attend, _mix, _finish) with
+these exchanges between them.  The conv history travels as the earlier
+tokens' MLP inputs u (the library recomputes their Z), so no phase waits on a
+kernel of another rank that has not started.  Halos are copied into this
+rank's own memory (send/recv) before any kernel reads them.
 """
 from __future__ import annotations
 
@@ -89,3 +93,29 @@ def state_prefix(total: torch.Tensor, group: Optional[dist.ProcessGroup] = None,
 
 def _global(group_rank: int, group: Optional[dist.ProcessGroup]) -> int:
     return group_rank if group is None else dist.get_global_rank(group, group_rank)
+
+
+def shard_block_forward(x: torch.Tensor, beta: torch.Tensor, weights, p, pos0: int,
+                        group: Optional[dist.ProcessGroup] = None,
+                        state_in: Optional[torch.Tensor] = None, make_shard=None):
+    """This rank's shard of a sequence-sharded block forward.
+
+    x [B, T, d], beta [B, T]: tokens pos0 .. pos0 + T - 1 of every sequence
+    (``shard_bounds`` gives them), ranks holding consecutive shards in rank
+    order; p describes this shard (p.T = T).  Returns (out [B, T, d], state
+    after this shard [B, d, f]); the last rank's state is the block's state_out.
+
+    ``make_shard(weights, p, pos0)`` builds the object that runs the four
+    phases (default: the CUDA library's ``Shard``); every rank takes the same
+    exchange steps in the same order.
+    """
+    if make_shard is None:
+        from . import Shard as make_shard
+    sh = make_shard(weights, p, pos0)
+    kv_tail = sh.qkv(x)
+    kv_halo = exchange_halo(kv_tail, p.w_T - 1, dim=1, group=group)
+    u_tail = sh.attend(x, kv_halo)
+    u_halo = exchange_halo(u_tail, max(p.conv_k - 1, 0), dim=2, group=group)
+    total = sh.mix(beta, u_halo)
+    s_in = state_prefix(total, group=group, state_in=state_in)
+    return sh.finish(s_in)

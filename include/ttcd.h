@@ -214,7 +214,9 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
  *   events[k] is recorded at boundary k: 0 start, 1 after the rotary table, the
  *   input RMS row scales and the gain-scaled W_qkv, 2 after QKV+RoPE, 3 after
  *   attention, 4 after o_proj (with the MLP RMSNorm statistics), 5 after
- *   gate/up+SwiGLU, 6 after conv/residual/keys, 7 after M = W_down W_proj,
+ *   gate/up+SwiGLU (with bf16 operands, the convs, D and the keys are in the
+ *   same kernel), 6 after the key scales (fp32 operands: the conv/residual/key
+ *   kernel and the key scales), 7 after M = W_down W_proj,
  *   8 after R, 9 after the chunk scan, 10 after the output GEMM.  Boundaries at
  *   or beyond n_events are skipped; 0 <= n_events <= 16; events[0..n_events-1]
  *   must be non-null.  The events belong to this call only.
@@ -224,6 +226,71 @@ ttcd_status ttcd_block_forward_profiled(const void* x, const float* beta,
                                         float* state_out, void* out, void* workspace,
                                         size_t ws_bytes, void* stream, void* const* events,
                                         int n_events);
+
+/*
+ * Sequence-sharded block forward: the four phases of one shard.
+ *
+ * A sequence-parallel run splits every sequence into contiguous shards of whole
+ * chunks, one per rank (GPU), in rank order; only the last shard may end in a
+ * partial chunk.  The block is causal (windowed attention over earlier tokens,
+ * causal short convs, a causal prefix over chunks: [REVIEW] 整体框架 and
+ * 关键设计 2-3; [README] "Model configuration" names flame's context
+ * parallelism for long-context training), so a shard needs three things from
+ * the shards before it, exchanged by the caller between the phases:
+ *   - the rotated K and V of the n_halo = min(w_T - 1, pos0) tokens before it
+ *     (the teacher window's reach);
+ *   - the MLP inputs u_P = RMSNorm(h_P; g_mlp) of the min(conv_k - 1, pos0)
+ *     tokens before it, from which it recomputes their Z_T, Z_S (the short
+ *     convs' history);
+ *   - the sum of the earlier shards' chunk increments (plus the block's
+ *     state_in), its state_in: the exclusive prefix over chunks taken over
+ *     shards first.
+ * Each phase exports what the next shard needs from this one; a halo may span
+ * several earlier shards, so the caller passes on the last rows of (halo it
+ * received, tail this shard exported).  Run on shards in any order subject to
+ * those exchanges, and concatenated, the shards' outputs are the rows of
+ * ttcd_block_forward over the whole sequence and the last shard's state_out is
+ * its state_out.
+ *
+ * Every phase of one shard takes the same p (p->T = this shard's tokens; p->dtype
+ * TTCD_BF16), pos0 (the absolute position of its first token, a multiple of
+ * p->chunk) and workspace (>= ttcd_shard_workspace_size(p) bytes, 16-byte
+ * aligned, status word first), which carries the shard's intermediates from
+ * phase to phase.  kv rows are [2, Hkv, hd] bf16 (K heads, then V heads).
+ *
+ * ttcd_shard_qkv: input RMSNorm, QKV, RoPE at positions pos0 .. pos0 + T - 1.
+ *   x [B, T, d] bf16;  kv_tail [B, min(T, w_T - 1), 2 Hkv hd] bf16, written
+ *   (nullable): the rotated K, V of this shard's last min(T, w_T - 1) tokens.
+ * ttcd_shard_attend: dual-window attention of the shard's queries over
+ *   (K/V halo, own K/V), o_proj for both paths with the residual, MLP RMSNorm.
+ *   kv_halo [B, n_halo, 2 Hkv hd] bf16 (required when n_halo > 0);
+ *   u_tail [2, B, min(T, conv_k - 1), d] bf16, written (nullable): the
+ *   normalised MLP inputs of the shard's last tokens, teacher then student.
+ * ttcd_shard_mix: the fast-weight MLP up to the chunk increments, and their sum.
+ *   beta [B, T] fp32;  u_halo [2, B, min(conv_k - 1, pos0), d] bf16 (required
+ *   when pos0 > 0 and conv_k > 1);  total [B, d, f] fp32, written: the sum of
+ *   this shard's chunk increments Delta W_i.
+ * ttcd_shard_finish: the fp32 prefix from state_in over the shard's chunks and
+ *   the output y = h_S + (W_down + S_i) Z_S.
+ *   state_in [B, d, f] fp32 (nullable: zero);  state_out [B, d, f] fp32
+ *   (nullable): the state after this shard;  out [B, T, d] bf16, written.
+ * Errors as ttcd_block_forward; pos0 < 0 or not a multiple of chunk ->
+ * TTCD_ERR_INVALID_ARG; TTCD_F32 -> TTCD_ERR_UNSUPPORTED.  Precision: bf16
+ * operands at every T (the fp32-operand route of short problems is not taken).
+ */
+size_t ttcd_shard_workspace_size(const ttcd_block_params* p);
+ttcd_status ttcd_shard_qkv(const void* x, const ttcd_block_weights* w, const ttcd_block_params* p,
+                           long long pos0, void* kv_tail, void* workspace, size_t ws_bytes,
+                           void* stream);
+ttcd_status ttcd_shard_attend(const void* x, const void* kv_halo, const ttcd_block_weights* w,
+                              const ttcd_block_params* p, long long pos0, void* u_tail,
+                              void* workspace, size_t ws_bytes, void* stream);
+ttcd_status ttcd_shard_mix(const float* beta, const void* u_halo, const ttcd_block_weights* w,
+                           const ttcd_block_params* p, long long pos0, float* total,
+                           void* workspace, size_t ws_bytes, void* stream);
+ttcd_status ttcd_shard_finish(const ttcd_block_weights* w, const ttcd_block_params* p,
+                              long long pos0, const float* state_in, float* state_out, void* out,
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * ttcd_fastweight_mlp_noalloc — ttcd_fastweight_mlp for callers that cannot
@@ -324,8 +391,11 @@ size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);
  *   "h"    fp32 [B*T, d] (student residual h_S)
  *   "u"    E [2, B*T, d] (block: h * g_mlp; the MLP RMSNorm's 1/rms is applied as a
  *          row scale from "hssq" fp32 [ceil(d/256), 2*B*T] partial sums of h^2)
- *   "Z"    fp32 [2, B*T, f]       "Zs16" bf16 [B*T, f] (TTCD_BF16 only)
- *   "D"    E [P, f]               "Kp" E [P, f] (unnormalised keys)  "ssq" fp32 [f/64, P]
+ *   "Z"    fp32 [2, B*T, f] (E = fp32 only: with bf16 operands Z never leaves the chip)
+ *   "Zs16" bf16 [B*T, f]  Z_S, the output GEMM's operand (E = bf16 only)
+ *   "D"    E [P, f]               "Kp" E [P, f] (unnormalised keys)
+ *   "ssq"  fp32 [n, P]: per-token partial sums of Kp^2 over column blocks of 128
+ *          (E = bf16) or 64 (E = fp32) columns, n = ceil(f / block)
  *   "R"    E [P, d] (value residual times beta_t / ||Zbar_S[t]||)
  *   "Wall" E [B*n_chunks, d, f]   (W_down + S_i per chunk)
  * where P = B * n_chunks * Cp, Cp = chunk rounded up to 64, and token t of

@@ -52,9 +52,18 @@ def _stage_checks(ttcd, p, ws, ref, shape):
         "o_S": (view("o", op, (2, BT, Hq * hd))[1], ref["o_S"].reshape(BT, -1)),
         "h_S": (view("h", f32, (BT, d)), ref["h_S"].reshape(BT, -1)),
         "hg_T": (view("u", op, (2, BT, d))[0], ref["h_T"].reshape(BT, -1)),  # gains are 1
-        "Z_T": (view("Z", f32, (2, BT, f))[0], ref["Z_T"].reshape(BT, -1)),
-        "Z_S": (view("Z", f32, (2, BT, f))[1], ref["Z_S"].reshape(BT, -1)),
     }
+    if op == f32:  # fp32 operands: Z_T, Z_S stored in fp32
+        checks["Z_T"] = (view("Z", f32, (2, BT, f))[0], ref["Z_T"].reshape(BT, -1))
+        checks["Z_S"] = (view("Z", f32, (2, BT, f))[1], ref["Z_S"].reshape(BT, -1))
+    else:  # bf16: Z stays on chip; the fused epilogue writes Z_S, D and the keys
+        Nc, Cp = shape.n_chunks, (shape.chunk + 63) // 64 * 64
+        t = np.arange(shape.T)
+        pidx = ((np.arange(shape.B)[:, None] * Nc + t // shape.chunk) * Cp + t % shape.chunk).ravel()
+        P = shape.B * Nc * Cp
+        checks["Z_S"] = (view("Zs16", bf, (BT, f)), ref["Z_S"].reshape(BT, -1))
+        checks["D"] = (view("D", bf, (P, f))[pidx], ref["D"].reshape(BT, -1))
+        checks["Kp"] = (view("Kp", bf, (P, f))[pidx], ref["zbar_S"].reshape(BT, -1))
     errs = {k: rel_max(g, r) for k, (g, r) in checks.items()}
     bad = {k: e for k, e in errs.items() if e > TOL_OUT}
     assert not bad, bad
