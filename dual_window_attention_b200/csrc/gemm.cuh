@@ -617,23 +617,26 @@ struct EpiSwiGLU {
 // rows 64-127 the student rows of the same tokens; columns [0, 128) are gate and
 // [128, 256) up for output columns tn*128 + [0, 128).
 //
-// Per 32-column slice every thread (one accumulator row) forms
-// z = silu(rstd g) (rstd u) in fp32, then the causal depthwise conv along
-// tokens: the k-1 earlier rows of the same path come from lanes below by warp
-// shuffles, and across the warp boundary from the previous quarter's last rows
-// in shared memory.  The tile's first k-1 rows only feed the conv (their outputs
-// belong to the previous tile).  Teacher warps publish Zbar_T in shared memory;
-// the student warp of the same tokens forms D = Zbar_T - Zbar_S and writes D and
-// Kp = Zbar_S (padded chunk layout), the bf16 Z_S (output-GEMM operand) and, per
-// token, the sum of Zbar_S^2 over the tile's 128 columns (the key norm is a row
-// scale applied to R later).  fp32 Z never reaches memory.
+// Per 32-column slice, in two phases between which the four warps meet once:
+//   A  every thread (one accumulator row) forms z = silu(rstd g) (rstd u) in
+//      fp32 and writes its 32 values to a shared tile [path][row][column]
+//      (16-byte slots swizzled by row, so both the row-wise writes and the
+//      column-wise reads are conflict-free; two tiles alternate by slice);
+//   B  thread (column c, row group g) slides the causal depthwise conv down the
+//      16 rows [16g, 16g + 16) of column c for both paths, with the column's
+//      taps in registers and the k-1 rows before the group read from the tile,
+//      and writes D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and
+//      the bf16 Z_S (output-GEMM operand): a warp writes 64 contiguous bytes of
+//      each row.  Its Kp^2 accumulate per row; one warp reduction per tile
+//      gives the sum over the tile's 128 columns (the key norm becomes a row
+//      scale of R later).
+// The tile's first k-1 rows only feed the conv (their outputs belong to the
+// previous tile); fp32 Z never reaches memory.
 //   z_halo [2, B, k-1, f] fp32: Z rows before token 0 (nullable: zeros)
 //   z_tail [2, B, k-1, f] fp32: written with the last k-1 rows of Z (nullable)
-// Shared memory: the four 8 KB staging regions; region w holds the Zbar_T slice
-// of its warp as [column][lane] (conflict-free) and, at float 1024, the last 8
-// rows of z as [column][row].
+template <int KMAX>  // conv width k <= KMAX
 struct EpiSwiGLUConv {
-  static constexpr bool kStaged = true;      // the staging area is the exchange buffer
+  static constexpr bool kStaged = true;      // the staging area holds the z tiles
   static constexpr bool kCollective = true;  // the four warps exchange rows
   __nv_bfloat16* D;
   __nv_bfloat16* Kp;
@@ -652,94 +655,118 @@ struct EpiSwiGLUConv {
     if (!rstd || t < 0 || t >= T) return 1.f;
     return __ldg(rstd + (r < 64 ? 0 : BT) + static_cast<long long>(c.group) * T + t);
   }
+  // padded index of token t of sequence b in the chunk layout of D, Kp, R
+  __device__ long long pidx(int b, int t) const {
+    return (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
+  }
 
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     static_assert(BN == 256, "gate/up tiles are 128 gate + 128 up columns");
     const int lane = threadIdx.x & 31;
-    const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quarter: rows 32q .. 32q+31
-    const bool student = q >= 2;
-    const int path = student ? 1 : 0;
-    const int rin = r & 63;
-    const int t = c.tok0 + rin;
+    const int rin = r & 63;               // phase A: this thread's row within its path
+    const int path = r >= 64 ? 1 : 0;
+    const int ta = c.tok0 + rin;
     const int b = c.group;
     const int H = k - 1;
-    const bool real = t >= 0 && t < T;
-    const bool out_row = rin >= H && real;
-    // regions of the quarters: warps 2, 3, 4, 5 serve quarters 2, 3, 0, 1
-    float* base = reinterpret_cast<float*>(stg.buf) - (((threadIdx.x >> 5) - 2) * 2048);
-    auto region = [&](int quarter) { return base + ((quarter + 2) & 3) * 2048; };
-    float* own = region(q);
-    const float* prev_halo = region(q - 1) + 1024;  // odd quarters only
-    const float* partner = region(q - 2);          // student quarters only
-    const __nv_bfloat16* tap = student ? tapS : tapT;
-    long long p = 0;
-    if (t >= 0) p = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
-    float ssq_acc = 0.f;
+    // phase B: column `lane` of the slice, rows [16 g, 16 g + 16)
+    const int g = (threadIdx.x >> 5) - 2;
+    uint8_t* tiles = stg.buf - g * 8192;  // the 32 KB staging area: two 16 KB z tiles
+    float ssq_acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ssq_acc[i] = 0.f;
 #pragma unroll 1
-    for (int cc = 0; cc < 128; cc += 32) {
+    for (int s = 0; s < 4; ++s) {
+      const int cc = 32 * s;
       const int col0 = c.tn * 128 + cc;
       if (col0 >= f) break;  // the same for every warp
-      float z[32];
+      uint8_t* tile = tiles + (s & 1) * 16384;
+      // ---- A: z of this row, 32 columns
       {
-        float g[32], u[32];
-        tmem_ld32f(taddr + cc, g);
-        tmem_ld32f(taddr + 128 + cc, u);
+        float z[32];
+        {
+          float gt[32], up[32];
+          tmem_ld32f(taddr + cc, gt);
+          tmem_ld32f(taddr + 128 + cc, up);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float gg = g[i] * rs;
-          z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (u[i] * rs);
+          for (int i = 0; i < 32; ++i) {
+            const float gg = gt[i] * rs;
+            z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (up[i] * rs);
+          }
         }
-      }
-      if (!real) {
-        if (t < 0 && z_halo) {
-          load_x32(z_halo + ((static_cast<long long>(path) * B + b) * H + (t + H)) * f + col0, z);
-        } else {
+        if (ta < 0 || ta >= T) {
+          if (ta < 0 && z_halo) {
+            load_x32(z_halo + ((static_cast<long long>(path) * B + b) * H + (ta + H)) * f + col0, z);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = 0.f;
+            for (int i = 0; i < 32; ++i) z[i] = 0.f;
+          }
         }
-      }
-      if (z_tail && out_row && t >= T - H)
-        store_f32x32(z_tail + ((static_cast<long long>(path) * B + b) * H + (t - (T - H))) * f + col0, z);
-      // the last 8 rows of the even quarters feed the first rows of the odd ones
-      if (!(q & 1) && lane >= 24) {
+        if (z_tail && rin >= H && ta >= T - H && ta < T && ta >= 0)
+          store_f32x32(z_tail + ((static_cast<long long>(path) * B + b) * H + (ta - (T - H))) * f + col0, z);
+        const int R = path * 64 + rin;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) own[1024 + i * 8 + (lane - 24)] = z[i];
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(tile + R * 128 + ((j ^ (R & 7)) << 4)) =
+              make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
       }
       epi_bar_sync();
-      // Zbar[t] = sum_m tap[c][m] z[t - m]  (tap m multiplies position t - m)
-      float zb[32];
+      // ---- B: the conv down column `lane`, rows [16 g, 16 g + 16), both paths
+      {
+        const int col = col0 + lane;
+        float wT[KMAX], wS[KMAX];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const __nv_bfloat16* tc = tap + static_cast<long long>(col0 + i) * k;
-        float acc = __bfloat162float(tc[0]) * z[i];
-        for (int m = 1; m <= H; ++m) {
-          float nb = __shfl_up_sync(0xffffffffu, z[i], m);
-          if (lane < m) nb = (q & 1) ? prev_halo[i * 8 + 8 - m + lane] : 0.f;
-          acc += __bfloat162float(tc[m]) * nb;
+        for (int m = 0; m < KMAX; ++m) {
+          wT[m] = m < k ? __bfloat162float(tapT[static_cast<long long>(col) * k + m]) : 0.f;
+          wS[m] = m < k ? __bfloat162float(tapS[static_cast<long long>(col) * k + m]) : 0.f;
         }
-        zb[i] = acc;
-      }
-      if (!student) {
+        constexpr int W = 16 + KMAX - 1;  // rows 16g - (KMAX-1) .. 16g + 15
+        float zT[W], zS[W];
+        const uint32_t cofs = ((lane >> 2) << 4) | ((lane & 3) << 2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) own[i * 32 + lane] = zb[i];
-      }
-      epi_bar_sync();
-      if (student) {
-        float d[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          d[i] = partner[i * 32 + lane] - zb[i];
-          ssq_acc += zb[i] * zb[i];
+        for (int i = 0; i < W; ++i) {
+          const int row = 16 * g + i - (KMAX - 1);
+          if (row >= 0) {
+            const int RT = row, RS = 64 + row;
+            zT[i] = *reinterpret_cast<const float*>(tile + RT * 128 + (cofs ^ ((RT & 7) << 4)));
+            zS[i] = *reinterpret_cast<const float*>(tile + RS * 128 + (cofs ^ ((RS & 7) << 4)));
+          } else {
+            zT[i] = 0.f;
+            zS[i] = 0.f;
+          }
         }
-        if (out_row) {
-          store_bf16x32(D + p * f + col0, d);
-          store_bf16x32(Kp + p * f + col0, zb);
-          store_bf16x32(Zs + (static_cast<long long>(b) * T + t) * f + col0, z);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int rrow = 16 * g + i;
+          const int t = c.tok0 + rrow;
+          float bT = 0.f, bS = 0.f;
+#pragma unroll
+          for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
+            bT += wT[m] * zT[i + KMAX - 1 - m];
+            bS += wS[m] * zS[i + KMAX - 1 - m];
+          }
+          if (rrow >= H && t >= 0 && t < T) {
+            const long long p = pidx(b, t);
+            D[p * f + col] = __float2bfloat16_rn(bT - bS);
+            Kp[p * f + col] = __float2bfloat16_rn(bS);
+            Zs[(static_cast<long long>(b) * T + t) * f + col] =
+                __float2bfloat16_rn(zS[i + KMAX - 1]);
+            ssq_acc[i] += bS * bS;
+          }
         }
       }
     }
-    if (student && out_row) ssq[static_cast<long long>(c.tn) * P + p] = ssq_acc;
+    // per-token sums of Kp^2 over the tile's columns: one warp reduction per row
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float v = ssq_acc[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      const int rrow = 16 * g + i;
+      const int t = c.tok0 + rrow;
+      if (lane == i && rrow >= H && t >= 0 && t < T)
+        ssq[static_cast<long long>(c.tn) * P + pidx(b, t)] = v;
+    }
   }
 };
 

@@ -129,6 +129,26 @@ bool map_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
   return make_map<E>(m, ptr, cols, rows, cols * sizeof(E), ElemTraits<E>::BK, box_rows);
 }
 
+// Kernels that move registers between warp groups with setmaxnreg: a group's
+// setmaxnreg.inc waits until the registers it asks for are free in the block's
+// launch allocation, so the split must fit in (launch registers x threads) or
+// the block never proceeds.  The split of each such kernel, in registers per
+// block, is checked against the compiled launch count before every launch.
+struct RegSplit {
+  int threads_low, regs_low;    // warps that give registers back (setmaxnreg.dec)
+  int threads_high, regs_high;  // warps that take them (setmaxnreg.inc)
+};
+constexpr RegSplit kAttnRegSplit{128, 56, 256, 224};  // dual_window_attn_kernel
+constexpr RegSplit kScanRegSplit{128, 56, 256, 224};  // fastweight_scan_kernel
+ttcd_status check_reg_split(const void* kern, int threads, const RegSplit& s) {
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return TTCD_ERR_CUDA;
+  const long long pool = static_cast<long long>(attr.numRegs) * threads;
+  const long long need = static_cast<long long>(s.threads_low) * s.regs_low +
+                         static_cast<long long>(s.threads_high) * s.regs_high;
+  return need <= pool ? TTCD_OK : TTCD_ERR_UNSUPPORTED;
+}
+
 // Process-wide diagnostic counter of kernel launches (atomic; not call state).
 std::atomic<unsigned long long> g_launches{0};
 
@@ -369,6 +389,7 @@ ttcd_status launch_attn(const Ctx& c, const void* q, const void* k, const void* 
   const long long grid =
       static_cast<long long>(a.n_qt - q_begin / ATT_BM) * B * Hkv * a.pairs;
   if (grid >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
+  TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), ATT_THREADS, kAttnRegSplit));
   kern<<<static_cast<unsigned>(grid), ATT_THREADS, smem, c.s>>>(mq, mk, mv, a, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
@@ -452,9 +473,15 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
     g.tiles_m = cdiv(p->T, 64 - H);
     g.tiles_n = cdiv(m.f, 128);
     g.half_rows = m.BT;
-    EpiSwiGLUConv e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
-                    p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
-    TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+    if (p->conv_k <= 4) {
+      EpiSwiGLUConv<4> e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
+                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
+      TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<4>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+    } else {
+      EpiSwiGLUConv<8> e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
+                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
+      TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<8>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+    }
     stage_mark(c, mark + 1);
     if (m.Cp != p->chunk || p->T % p->chunk != 0) {
       const long long n = m.P * (m.f / 8);
@@ -572,6 +599,7 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
     auto kern = fastweight_scan_kernel<E, STAGES, MN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
+    TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), SCAN_THREADS, kScanRegSplit));
     kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
     TTCD_CHECK_LAUNCH();
   }
@@ -1397,6 +1425,7 @@ ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, co
   auto kern = fastweight_scan_kernel<bf, STAGES, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
+  TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), SCAN_THREADS, kScanRegSplit));
   kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mR, mK, a, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
