@@ -474,11 +474,12 @@ def measure_attention(args, world, local, wS, wT, form, steps, warmup):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, local)
-    e0.record(stream)
-    for _ in range(steps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(local, period_s=0.002) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
     ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
     if ttcd.get_device_error()[0] != ttcd.OK:
         raise RuntimeError("a device wait timed out in the attention benchmark")
@@ -488,7 +489,7 @@ def measure_attention(args, world, local, wS, wT, form, steps, warmup):
             "tokens_per_s": shape.B * shape.T * world / (ms / 1e3), "tflops_per_s": ach,
             "frac": ach / peaks["bf16_tflops"],
             "peak_source": f"{peak_kind} bf16_tflops (burst: kernel timed alone)",
-            "steps": steps, "warmup": warmup}
+            "steps": steps, "warmup": warmup, "clocks": clk.summary()}
 
 
 def run_attention(args, world, rank, local):
@@ -531,14 +532,18 @@ def run_decode_bench(args, world, rank, local):
     inp = make_block_inputs(shape, seed=0)
     w = {k: v.to(dev) for k, v in inp["layers"][0].items()}
     p = ttcd.BlockParams.from_shape(shape)
-    dec = ttcd.Decoder(w, p)
+    dec = ttcd.Decoder(w, p, graph=args.graph)
     g = torch.Generator().manual_seed(0)
     x = torch.randn(args.B, shape.d_model, generator=g).to(torch.bfloat16).to(dev)
     beta = (0.1 * torch.sigmoid(torch.randn(args.B, generator=g))).to(dev)
     y = torch.empty_like(x)
-    dec.t = 4 * shape.w_T + 7  # past the window: full K/V reads every step
+    if args.graph:  # the decoder's own fixed buffers: no copies around the replays
+        dec.x_buf.copy_(x)
+        dec.b_buf.copy_(beta)
+        x, beta, y = dec.x_buf, dec.b_buf, dec.y_buf
+    dec.seek(4 * shape.w_T + 7)  # past the window: full K/V reads every step
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
+    for _ in range(max(args.warmup, 3 if args.graph else 0)):
         dec.step(x, beta, y)
     torch.cuda.synchronize()
     barrier(world, local)
@@ -551,6 +556,8 @@ def run_decode_bench(args, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
     launches = ttcd.kernel_launch_count() - launches0
+    if args.graph:  # replays launch the captured kernels without the host counter
+        launches += dec.graph_launches * args.steps
     ms, value = job_throughput(world, args.B * args.steps, e0.elapsed_time(e1))
     if dec.check_status() != ttcd.OK:
         raise RuntimeError("a device wait timed out in the decode benchmark")
@@ -569,6 +576,7 @@ def run_decode_bench(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(shape, {"sequences": args.B, "position": "past w_T",
+                                              "launch": "cuda graph" if args.graph else "eager",
                                               "parallelism": f"replicas{world}"}),
             "roofline": {"kernel": "decode step (all kernels)", "bound": "hbm", "achieved": ach,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
@@ -658,6 +666,8 @@ def main():
                     help="tokens per sequence (65536 is the benchmark workload; smaller values "
                          "are for profiling)")
     ap.add_argument("--B", type=int, default=1, help="--mode attn / stack / decode: sequences")
+    ap.add_argument("--graph", action="store_true",
+                    help="--mode decode: replay each token step from one CUDA graph")
     ap.add_argument("--windows", default="512/8192",
                     help="--mode attn: comma-separated w_S/w_T pairs")
     ap.add_argument("--form", choices=["fused", "lse"], default="fused",

@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_decode_workspace_size.restype = sz
     lib.ttcd_decode_state_init.argtypes = [W, P, vp, vp, sz, vp, sz, vp]
     lib.ttcd_block_decode.argtypes = [vp, vp, i, W, P, vp, sz, vp, vp, sz, vp]
+    lib.ttcd_block_decode_next.argtypes = [vp, vp, W, P, vp, sz, vp, vp, sz, vp]
     lib.ttcd_decode_state_read.argtypes = [P, i, vp, sz, vp, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
@@ -108,6 +109,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                "ttcd_block_forward", "ttcd_block_forward_profiled", "ttcd_block_workspace_offset",
                "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
                "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read",
+               "ttcd_block_decode_next",
                "ttcd_shard_qkv", "ttcd_shard_attend", "ttcd_shard_mix", "ttcd_shard_finish"):
         getattr(lib, fn).restype = i
     _lib = lib
@@ -328,11 +330,15 @@ class Decoder:
     Holds the decode state (K/V ring cache, conv history, the current chunk's
     rows, the fast weight) and a step workspace, both allocated once.
     ``step(x_t, beta_t)`` takes x_t [B, d] bf16 and beta_t [B] fp32 of the next
-    position and returns y_t [B, d]; ``state()`` is the fast-weight state after
-    the tokens so far (partial chunk included)."""
+    position and returns y_t [B, d]; ``state_out()`` is the fast-weight state
+    after the tokens so far (partial chunk included).
+
+    ``graph=True``: the steps use ttcd_block_decode_next (the position lives in
+    the state); token 0 runs eagerly, then one step is captured in a CUDA graph
+    with fixed input and output buffers and replayed for every later token."""
 
     def __init__(self, weights: Dict[str, torch.Tensor], p: BlockParams, state_in=None,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, graph: bool = False):
         self.lib = load_library()
         self.p, self.pc, self.wc = p, p.c(), _weights(weights)
         self.weights = weights  # keep the tensors alive
@@ -348,8 +354,50 @@ class Decoder:
                                                self.state.numel(), _ptr(self.ws), self.ws.numel(),
                                                _stream(stream)), "ttcd_decode_state_init")
         self.t = 0
+        self.use_graph, self.graph, self.warm, self.graph_launches = graph, None, False, 0
+        if graph:
+            self.x_buf = torch.empty(p.B, p.d_model, device=device, dtype=torch.bfloat16)
+            self.b_buf = torch.empty(p.B, device=device, dtype=torch.float32)
+            self.y_buf = torch.empty_like(self.x_buf)
+
+    def _next(self):
+        _check(self.lib.ttcd_block_decode_next(_ptr(self.x_buf), _ptr(self.b_buf),
+                                               ctypes.byref(self.wc), ctypes.byref(self.pc),
+                                               _ptr(self.state), self.state.numel(),
+                                               _ptr(self.y_buf), _ptr(self.ws), self.ws.numel(),
+                                               _stream(None)), "ttcd_block_decode_next")
+
+    def seek(self, t: int):
+        """Sets the next position to t (host count and, in graph mode, the
+        state's device position: an int64 at byte 8 of the state)."""
+        self.t = t
+        if self.use_graph:
+            self.state[8:16].copy_(torch.tensor([t], dtype=torch.int64).view(torch.uint8))
 
     def step(self, x_t, beta_t, y=None):
+        """In graph mode x_t, beta_t and y may be x_buf, b_buf and y_buf
+        themselves (no copies)."""
+        if self.use_graph:
+            if x_t.data_ptr() != self.x_buf.data_ptr():
+                self.x_buf.copy_(x_t)
+            if beta_t.data_ptr() != self.b_buf.data_ptr():
+                self.b_buf.copy_(beta_t)
+            if self.graph is None and not self.warm:
+                self._next()  # eager: also loads every kernel before the capture
+                self.warm = True
+            else:
+                if self.graph is None:
+                    torch.cuda.synchronize()
+                    n0 = kernel_launch_count()
+                    self.graph = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(self.graph):
+                        self._next()
+                    self.graph_launches = kernel_launch_count() - n0
+                self.graph.replay()
+            self.t += 1
+            if y is not None and y.data_ptr() == self.y_buf.data_ptr():
+                return y
+            return self.y_buf.clone() if y is None else y.copy_(self.y_buf)
         y = torch.empty_like(x_t) if y is None else y
         _check(self.lib.ttcd_block_decode(_ptr(x_t), _ptr(beta_t), self.t, ctypes.byref(self.wc),
                                           ctypes.byref(self.pc), _ptr(self.state),

@@ -17,6 +17,14 @@ constexpr int DEC_KC = 256;       // keys per attention split
 constexpr int DEC_THREADS = 128;  // attention split block
 constexpr int DEC_MAXG = 8;       // query heads per KV head handled by one block
 
+// Position of the token being decoded: the kernels take it as an argument, or,
+// when `pos` is set, read it from device memory (the decode state's own
+// counter), so that a step's launches have no argument that changes from token
+// to token and the step can be captured once in a CUDA graph and replayed.
+__device__ __forceinline__ int dec_pos(int t, const long long* pos) {
+  return pos ? static_cast<int>(*pos) : t;
+}
+
 // q and k rotated at position t (rotate-half RoPE, angle t * theta^(-2i/hd) in
 // double precision), k and v appended to the ring caches at slot t % W.
 // qkv [B, (Hq + 2 Hkv) hd] fp32 -> q_rot [B, Hq, hd] bf16; kc, vc [B, W, Hkv, hd].
@@ -25,7 +33,9 @@ __global__ void decode_rope_cache_kernel(const float* __restrict__ qkv,
                                          __nv_bfloat16* __restrict__ q_rot,
                                          __nv_bfloat16* __restrict__ kc,
                                          __nv_bfloat16* __restrict__ vc, int Hq, int Hkv, int hd,
-                                         int t, int W, double theta) {
+                                         int t, int W, double theta,
+                                         const long long* pos = nullptr) {
+  t = dec_pos(t, pos);
   const int b = blockIdx.x, head = blockIdx.y, i = threadIdx.x;
   const int half = hd / 2;
   const float* src = qkv + static_cast<long long>(b) * (Hq + 2 * Hkv) * hd +
@@ -60,7 +70,9 @@ __global__ void __launch_bounds__(DEC_THREADS)
                                const __nv_bfloat16* __restrict__ kc,
                                const __nv_bfloat16* __restrict__ vc, float* __restrict__ pm,
                                float* __restrict__ pl, float* __restrict__ po, int Hq, int Hkv,
-                               int W, int t, int w_S, int w_T, float scale_log2, int nsplit) {
+                               int W, int t, int w_S, int w_T, float scale_log2, int nsplit,
+                               const long long* pos = nullptr) {
+  t = dec_pos(t, pos);
   __shared__ float qs[DEC_MAXG][HD];
   __shared__ float ps[2][DEC_MAXG][DEC_KC];  // scores, then probabilities per window
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv, sp = blockIdx.y;
@@ -257,7 +269,8 @@ __global__ void decode_conv_kernel(const float* __restrict__ Z,
                                    float* __restrict__ hist, __nv_bfloat16* __restrict__ D,
                                    __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Zs16,
                                    float* __restrict__ ssq_part, int B, int f, int k, int t, int C,
-                                   int Cp) {
+                                   int Cp, const long long* pos = nullptr) {
+  t = dec_pos(t, pos);
   __shared__ float red[8];
   const int b = blockIdx.y;
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
@@ -380,9 +393,11 @@ __global__ void decode_gemv_kernel(const __nv_bfloat16* __restrict__ Wm,
 }
 
 // rows [B, d] -> dst rows b * Cp + row (the current chunk slot of each sequence)
+// With `pos` set, row = *pos % C.
 __global__ void decode_row_copy_kernel(const __nv_bfloat16* __restrict__ src,
                                        __nv_bfloat16* __restrict__ dst, int B, int d, int Cp,
-                                       int row) {
+                                       int row, const long long* pos = nullptr, int C = 1) {
+  if (pos) row = static_cast<int>(*pos % C);
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= static_cast<long long>(B) * d) return;
   const long long b = i / d, c = i % d;
@@ -416,10 +431,13 @@ __global__ void decode_out_kernel(const __nv_bfloat16* __restrict__ Weff,
     y[static_cast<long long>(b) * d + i] = __float2bfloat16_rn(hS[static_cast<long long>(b) * d + i] + acc);
 }
 
-// Weff[b] = bf16(W_down + S[b]), 4 elements per thread.
+// Weff[b] = bf16(W_down + S[b]), 4 elements per thread.  With `commit_pos`
+// set it acts only at the last token of a chunk (*commit_pos % C == C - 1).
 __global__ void decode_weff_kernel(const __nv_bfloat16* __restrict__ w_down,
                                    const float* __restrict__ S, __nv_bfloat16* __restrict__ Weff,
-                                   long long df, long long n4) {
+                                   long long df, long long n4,
+                                   const long long* commit_pos = nullptr, int C = 1) {
+  if (commit_pos && *commit_pos % C != C - 1) return;
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   const long long e = i * 4, w = e % df;
@@ -430,5 +448,9 @@ __global__ void decode_weff_kernel(const __nv_bfloat16* __restrict__ w_down,
   out.y = pack_bf16x2(bf16lo_to_f32(wd.y) + s.z, bf16hi_to_f32(wd.y) + s.w);
   *reinterpret_cast<uint2*>(Weff + e) = out;
 }
+
+// Advances the decode state's position counter by one token (the last launch
+// of a step that reads the position from device memory).
+__global__ void decode_advance_kernel(long long* __restrict__ pos) { *pos += 1; }
 
 }  // namespace ttcd

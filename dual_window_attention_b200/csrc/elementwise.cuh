@@ -169,37 +169,24 @@ __global__ void cast_kernel(const InT* __restrict__ in, OutT* __restrict__ out, 
     out[i] = from_f32<OutT>(to_f32(in[i]));
 }
 
-// cs[i][t] = (cos, sin)(t * theta^(-2i/hd)), evaluated in double precision.
-// Frequency-major, so a warp reading one frequency for 32 consecutive tokens
-// reads 256 contiguous bytes.
-// cos/sin of t * theta^(-2i/hd) for every frequency i < hd/2 and position t < T,
-// frequency-major [hd/2][T].  One thread per frequency and run of ROPE_RUN
-// positions: one double-precision sincos at the run's start, then the angle
-// addition (cos, sin)((t+1)a) = (c cos a - s sin a, s cos a + c sin a) in double
-// precision, whose error over a run stays far below the half-precision output.
-constexpr int ROPE_RUN = 64;
-// pos0: absolute position of row 0 (a sequence shard starts past 0).
-__global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double theta,
+// cs[i][t] = (cos, sin)((pos0 + t) * theta^(-2i/hd)) for every frequency
+// i < hd/2 and position t < T, frequency-major [hd/2][T]: one thread per entry,
+// the angle and its sincos in double precision, rounded once to half precision
+// (11-bit significands, far below the bf16 rounding of q and k).  A warp
+// writes 32 consecutive positions of one frequency (128 contiguous bytes).
+// pos0: absolute position of row 0 (a sequence shard starts past 0);
+// log2_theta = log2 of the RoPE base, so theta^(-2i/hd) = 2^(-(2i/hd) log2 theta).
+__global__ void rope_table_kernel(__half2* __restrict__ cs, int T, int hd, double log2_theta,
                                   long long pos0 = 0) {
-  const int half = hd / 2;
-  const int runs = (T + ROPE_RUN - 1) / ROPE_RUN;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(half) * runs) return;
-  const int i = static_cast<int>(idx / runs);
-  const int t0 = static_cast<int>(idx % runs) * ROPE_RUN;
-  const double a = pow(theta, -2.0 * i / hd);
-  double s, c, sa, ca;
-  sincos(static_cast<double>(pos0 + t0) * a, &s, &c);
-  sincos(a, &sa, &ca);
-  __half2* out = cs + static_cast<long long>(i) * T + t0;
-  const int n = min(ROPE_RUN, T - t0);
-  for (int k = 0; k < n; ++k) {
-    // half precision (11-bit significand) is far below the bf16 rounding of q and k
-    out[k] = __floats2half2_rn(static_cast<float>(c), static_cast<float>(s));
-    const double c2 = c * ca - s * sa;
-    s = s * ca + c * sa;
-    c = c2;
-  }
+  const int half = hd / 2;
+  if (idx >= static_cast<long long>(half) * T) return;
+  const int i = static_cast<int>(idx / T);
+  const int t = static_cast<int>(idx % T);
+  const double a = exp2(-2.0 * i / hd * log2_theta);
+  double s, c;
+  sincos(static_cast<double>(pos0 + t) * a, &s, &c);
+  cs[idx] = __floats2half2_rn(static_cast<float>(c), static_cast<float>(s));
 }
 
 // Fused short causal convolutions, residual difference and student keys.

@@ -199,7 +199,12 @@ struct EpiStage {
   }
 };
 
-template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom>
+// B_MN = true (bf16 only): B is given as B^T, a row-major [K, N] matrix (N
+// contiguous), and is read as an MN-major tcgen05 operand: TMA boxes of 64
+// N-elements x 64 K-rows, leading-byte offset = one box, 16 K-rows (2048 bytes)
+// per MMA step.
+template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom,
+          bool B_MN = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
@@ -213,7 +218,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
-  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, false);
+  static_assert(!B_MN || (sizeof(E) == 2 && !DUAL_B), "MN-major B: bf16, single B operand");
+  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, B_MN);
+  constexpr int MN_BOX_BYTES = 64 * 64 * 2;  // 64 N-elements x 64 K-rows, bf16
   constexpr int BK = ElemTraits<E>::BK;
 
   extern __shared__ uint8_t smem_raw[];
@@ -288,6 +295,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * (BN / 2));
             tma_load_2d(sb + (BN / 2) * 128, &mapB1, &full[s], kb * BK,
                         c.b_row0 + c.tn * (BN / 2));
+          } else if constexpr (B_MN) {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_2d(sb + q * MN_BOX_BYTES, &mapB0, &full[s], c.tn * BN + 64 * q, kb * BK);
           } else {
             tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * BN);
           }
@@ -304,6 +315,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // elected lane issues; descriptor low words advance by (byte offset >> 4).
     constexpr uint32_t HI = sdesc_hi_sw128(1024);
     const uint32_t lo0 = sdesc_lo(smem_u32(smem), 16);
+    // MN-major B: its leading-byte offset is one box (the low word differs by it)
+    constexpr uint32_t B_LBO_FIX = B_MN ? ((MN_BOX_BYTES >> 4) - 1) << 16 : 0;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
     };
@@ -321,11 +334,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!wait(&full[s], (it / STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_lo = lo0 + ((s * STAGE_BYTES) >> 4);
-        const uint32_t b_lo = a_lo + (A_BYTES >> 4);
+        const uint32_t b_lo = a_lo + (A_BYTES >> 4) + B_LBO_FIX;
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 4 MMAs of 32 bytes of K per 128-byte row
-            mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + 2 * k, HI, IDESC,
+            mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + (B_MN ? k * (2048 >> 4) : 2 * k), HI, IDESC,
                          (kb | k) != 0 ? 1u : 0u);
           mma_commit(&empty[s]);
         }

@@ -31,6 +31,11 @@ struct ScanArgs {
   float* state_out;       // [B, d, f] nullable
   E* w_all;               // [B*Nc, d, f], nullable (state only)
   int tiles_m, tiles_n;
+  // Decode commit from a graph: when set, the kernel acts only at the last
+  // token of a chunk (*commit_pos % commit_C == commit_C - 1) and otherwise
+  // returns at once (every thread of every block alike, before any set-up).
+  const long long* commit_pos;
+  int commit_C;
 };
 
 constexpr int SCAN_BN = 192;
@@ -60,6 +65,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  if (a.commit_pos && *a.commit_pos % a.commit_C != a.commit_C - 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tn = blockIdx.x % a.tiles_n;
   const int tm = (blockIdx.x / a.tiles_n) % a.tiles_m;

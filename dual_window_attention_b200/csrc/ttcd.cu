@@ -594,6 +594,8 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
     a.w_all = w_all;
     a.tiles_m = cdiv(m.d, 128);
     a.tiles_n = cdiv(m.f, SCAN_BN);
+    a.commit_pos = nullptr;
+    a.commit_C = 1;
     constexpr int STAGES = 4;
     constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
     auto kern = fastweight_scan_kernel<E, STAGES, MN>;
@@ -785,8 +787,8 @@ ttcd_status block_qkv(const Ctx& c, const E* xin, const ttcd_block_weights* w,
   float* rstd_in = at<float>(ws, L, B_RSTDIN);
   __half2* rope = at<__half2>(ws, L, B_ROPE);
   stage_mark(c, 0);
-  rope_table_kernel<<<cdiv(static_cast<long long>(cdiv(p->T, ROPE_RUN)) * (m.hd / 2), 256), 256, 0, c.s>>>(
-      rope, p->T, m.hd, static_cast<double>(p->rope_theta), pos0);
+  rope_table_kernel<<<cdiv(static_cast<long long>(p->T) * (m.hd / 2), 256), 256, 0, c.s>>>(
+      rope, p->T, m.hd, std::log2(static_cast<double>(p->rope_theta)), pos0);
   TTCD_CHECK_LAUNCH();
   rms_rowscale_kernel<E><<<cdiv(m.BT, 8), 256, 0, c.s>>>(xin, rstd_in, m.BT, m.d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
@@ -1401,7 +1403,8 @@ T* dat(void* base, size_t off) {
 // S (in place) += the chunk buffers' R^T K' over their first Cp rows (rows past
 // the chunk's tokens are zero), by the chunk-scan kernel with one chunk.
 ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, const DecState& L,
-                       const __nv_bfloat16* w_down, const float* S_in, float* S_out) {
+                       const __nv_bfloat16* w_down, const float* S_in, float* S_out,
+                       const long long* commit_pos = nullptr) {
   using bf = __nv_bfloat16;
   const int d = p->d_model, f = p->d_ff, Cp = (p->chunk + 63) / 64 * 64;
   CUtensorMap mR, mK;
@@ -1420,6 +1423,8 @@ ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, co
   a.w_all = nullptr;
   a.tiles_m = cdiv(d, 128);
   a.tiles_n = cdiv(f, SCAN_BN);
+  a.commit_pos = commit_pos;
+  a.commit_C = p->chunk;
   constexpr int STAGES = 4;
   constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
   auto kern = fastweight_scan_kernel<bf, STAGES, true>;
@@ -1432,24 +1437,26 @@ ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, co
 }
 
 ttcd_status dec_weff(const Ctx& c, const ttcd_block_params* p, void* state, const DecState& L,
-                     const __nv_bfloat16* w_down) {
+                     const __nv_bfloat16* w_down, const long long* commit_pos = nullptr) {
   const long long df = static_cast<long long>(p->d_model) * p->d_ff;
   const long long n4 = p->B * df / 4;
   decode_weff_kernel<<<static_cast<unsigned>(cdiv(n4, 256)), 256, 0, c.s>>>(
-      w_down, dat<float>(state, L.S), dat<__nv_bfloat16>(state, L.weff), df, n4);
+      w_down, dat<float>(state, L.S), dat<__nv_bfloat16>(state, L.weff), df, n4, commit_pos,
+      p->chunk);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
 }
 
 template <int HD>
 ttcd_status dec_attention(const Ctx& c, const ttcd_block_params* p, void* state,
-                          const DecState& S, void* ws, const DecWs& L, int t, float scale) {
+                          const DecState& S, void* ws, const DecWs& L, int t, float scale,
+                          const long long* pos) {
   using bf = __nv_bfloat16;
   const int B = p->B, Hq = p->n_q_heads, Hkv = p->n_kv_heads;
   decode_attn_partial_kernel<HD><<<dim3(B * Hkv, L.nsplit), DEC_THREADS, 0, c.s>>>(
       dat<bf>(ws, L.qrot), dat<bf>(state, S.kc), dat<bf>(state, S.vc), dat<float>(ws, L.pm),
       dat<float>(ws, L.pl), dat<float>(ws, L.po), Hq, Hkv, p->w_T, t, p->w_S, p->w_T,
-      scale * 1.4426950408889634f, L.nsplit);
+      scale * 1.4426950408889634f, L.nsplit, pos);
   TTCD_CHECK_LAUNCH();
   decode_attn_combine_kernel<HD><<<B * Hq * 2, HD, 0, c.s>>>(
       dat<float>(ws, L.pm), dat<float>(ws, L.pl), dat<float>(ws, L.po), dat<bf>(ws, L.o), B, Hq,
@@ -1458,9 +1465,13 @@ ttcd_status dec_attention(const Ctx& c, const ttcd_block_params* p, void* state,
   return TTCD_OK;
 }
 
+// One token.  pos null: the token's position is t (host).  pos set: every
+// kernel reads the position from *pos, the chunk commit runs every step and
+// acts only at a chunk's last token, and the last launch advances *pos.
 ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, int t,
                        const ttcd_block_weights* w, const ttcd_block_params* p, void* state,
-                       const DecState& S, __nv_bfloat16* y, void* ws, const DecWs& L) {
+                       const DecState& S, __nv_bfloat16* y, void* ws, const DecWs& L,
+                       long long* pos = nullptr) {
   using bf = __nv_bfloat16;
   const int B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
   const int Hq = p->n_q_heads, Hkv = p->n_kv_heads, dqkv = (Hq + 2 * Hkv) * hd;
@@ -1487,13 +1498,13 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   }
   decode_rope_cache_kernel<<<dim3(B, Hq + 2 * Hkv), hd / 2, 0, c.s>>>(
       dat<float>(ws, L.qkv), dat<bf>(ws, L.qrot), dat<bf>(state, S.kc), dat<bf>(state, S.vc), Hq,
-      Hkv, hd, t, p->w_T, static_cast<double>(p->rope_theta));
+      Hkv, hd, t, p->w_T, static_cast<double>(p->rope_theta), pos);
   TTCD_CHECK_LAUNCH();
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(hd));
   switch (hd) {
-    case 32: TTCD_TRY(dec_attention<32>(c, p, state, S, ws, L, t, scale)); break;
-    case 64: TTCD_TRY(dec_attention<64>(c, p, state, S, ws, L, t, scale)); break;
-    default: TTCD_TRY(dec_attention<128>(c, p, state, S, ws, L, t, scale)); break;
+    case 32: TTCD_TRY(dec_attention<32>(c, p, state, S, ws, L, t, scale, pos)); break;
+    case 64: TTCD_TRY(dec_attention<64>(c, p, state, S, ws, L, t, scale, pos)); break;
+    default: TTCD_TRY(dec_attention<128>(c, p, state, S, ws, L, t, scale, pos)); break;
   }
   // o_proj for both paths, residual, MLP RMSNorm
   if (gemv) {
@@ -1535,7 +1546,7 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   decode_conv_kernel<<<dim3(n_part, B), 256, 0, c.s>>>(
       dat<float>(ws, L.Z), static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S),
       dat<float>(state, S.hist), dat<bf>(ws, L.D), dat<bf>(state, S.kx), dat<bf>(ws, L.Zs),
-      dat<float>(ws, L.ssq), B, f, p->conv_k, t, C, Cp);
+      dat<float>(ws, L.ssq), B, f, p->conv_k, t, C, Cp, pos);
   TTCD_CHECK_LAUNCH();
   decode_kscale_kernel<<<B, 32, 0, c.s>>>(dat<float>(ws, L.ssq), n_part, beta,
                                           dat<float>(ws, L.ks), p->l2_eps);
@@ -1556,15 +1567,20 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
     TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(B, cdiv(d, 256), f), e)));
   }
   decode_row_copy_kernel<<<static_cast<unsigned>(cdiv(static_cast<long long>(B) * d, 256)), 256, 0, c.s>>>(
-      dat<bf>(ws, L.r), dat<bf>(state, S.rc), B, d, Cp, t % C);
+      dat<bf>(ws, L.r), dat<bf>(state, S.rc), B, d, Cp, t % C, pos, C);
   TTCD_CHECK_LAUNCH();
   // output with the current chunk's weight W_down + S
   decode_out_kernel<<<dim3(cdiv(d, 8), B), 256, 0, c.s>>>(dat<bf>(state, S.weff), dat<bf>(ws, L.Zs),
                                                          dat<float>(ws, L.hS), y, d, f);
   TTCD_CHECK_LAUNCH();
   // last token of a chunk: S += this chunk's Delta W, then W_down + S
-  if (t % C == C - 1) {
-    float* Sp = dat<float>(state, S.S);
+  float* Sp = dat<float>(state, S.S);
+  if (pos) {  // launched every step; the kernels act only at a chunk's last token
+    TTCD_TRY(dec_commit(c, p, state, S, static_cast<const bf*>(w->w_down), Sp, Sp, pos));
+    TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down), pos));
+    decode_advance_kernel<<<1, 1, 0, c.s>>>(pos);
+    TTCD_CHECK_LAUNCH();
+  } else if (t % C == C - 1) {
     TTCD_TRY(dec_commit(c, p, state, S, static_cast<const bf*>(w->w_down), Sp, Sp));
     TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down)));
   }
@@ -1634,6 +1650,25 @@ ttcd_status ttcd_block_decode(const void* x_t, const float* beta_t, int t,
   TTCD_TRY(make_ctx(stream, c, dat<void>(state, S.status)));
   return run_decode(c, static_cast<const __nv_bfloat16*>(x_t), beta_t, t, w, p, state, S,
                     static_cast<__nv_bfloat16*>(y), workspace, L);
+}
+
+ttcd_status ttcd_block_decode_next(const void* x_t, const float* beta_t,
+                                   const ttcd_block_weights* w, const ttcd_block_params* p,
+                                   void* state, size_t state_bytes, void* y, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_decode_params(p));
+  if (!aligned16(x_t) || !beta_t || (reinterpret_cast<uintptr_t>(beta_t) & 3u) ||
+      !aligned16(y) || !weights_ok(w, true) || !aligned16(state) || !aligned16(workspace))
+    return TTCD_ERR_INVALID_ARG;
+  const DecState S = dec_state_layout(p);
+  const DecWs L = dec_ws_layout(p);
+  if (state_bytes < S.total || ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, dat<void>(state, S.status)));
+  // the position counter sits after the status word in the state's status region
+  long long* pos = dat<long long>(state, S.status + 8);
+  return run_decode(c, static_cast<const __nv_bfloat16*>(x_t), beta_t, 0, w, p, state, S,
+                    static_cast<__nv_bfloat16*>(y), workspace, L, pos);
 }
 
 ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void* state,

@@ -373,6 +373,25 @@ ttcd_status ttcd_block_decode(const void* x_t, const float* beta_t, int t,
 ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void* state,
                                    size_t state_bytes, float* state_out, void* stream);
 
+/*
+ * ttcd_block_decode_next — ttcd_block_decode at the state's own position.
+ *
+ * The decode state keeps a position counter, an int64 at byte offset 8 of the
+ * state (0 after ttcd_decode_state_init; a caller may write it on the device
+ * to start elsewhere); this call decodes that position and advances it by one.  Every kernel reads
+ * the position from the state, and the chunk commit is launched at every step
+ * and acts only at the last token of a chunk, so no launch argument depends on
+ * the position: one call can be captured in a CUDA graph and replayed for
+ * every later token (the graph's x_t, beta_t and y buffers stay fixed).  Make
+ * the first call on a device outside a capture.  Arguments and errors as
+ * ttcd_block_decode without t; use either this call or ttcd_block_decode on one
+ * state, not both (ttcd_decode_state_read still takes the next position).
+ */
+ttcd_status ttcd_block_decode_next(const void* x_t, const float* beta_t,
+                                   const ttcd_block_weights* w, const ttcd_block_params* p,
+                                   void* state, size_t state_bytes, void* y, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 /* Workspace bytes needed by each entry point; 0 if the parameters are invalid. */
 size_t ttcd_fastweight_mlp_workspace_size(const ttcd_block_params* p);
 size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);

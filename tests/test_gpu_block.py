@@ -37,7 +37,7 @@ def _run(ttcd, shape, inp, layer=0):
     return p, out, state, ws
 
 
-def _stage_checks(ttcd, p, ws, ref, shape):
+def _stage_checks(ttcd, p, ws, ref, shape, weights=None):
     BT, d, f = shape.B * shape.T, shape.d_model, shape.d_ff
     Hq, Hkv, hd = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
     view = lambda n, dt, sh: np64(ttcd.workspace_view(ws, p, n, dt, sh))
@@ -64,6 +64,8 @@ def _stage_checks(ttcd, p, ws, ref, shape):
         checks["Z_S"] = (view("Zs16", bf, (BT, f)), ref["Z_S"].reshape(BT, -1))
         checks["D"] = (view("D", bf, (P, f))[pidx], ref["D"].reshape(BT, -1))
         checks["Kp"] = (view("Kp", bf, (P, f))[pidx], ref["zbar_S"].reshape(BT, -1))
+        if weights is not None:  # M = W_down W_proj, with W_proj an MN-major GEMM operand
+            checks["M"] = (view("M", bf, (d, f)), np64(weights["w_down"]) @ np64(weights["w_proj"]))
     errs = {k: rel_max(g, r) for k, (g, r) in checks.items()}
     bad = {k: e for k, e in errs.items() if e > TOL_OUT}
     assert not bad, bad
@@ -75,7 +77,7 @@ def test_block_forward_parity_small(ttcd, shape):
     inp = make_block_inputs(shape, seed=0)
     p, out, state, ws = _run(ttcd, shape, inp)
     ref = oracle_block(shape, inp)
-    errs = _stage_checks(ttcd, p, ws, ref, shape)
+    errs = _stage_checks(ttcd, p, ws, ref, shape, inp["layers"][0])
     e_out, e_state = rel_max(out, ref["out"]), rel_fro(state, ref["state_out"])
     print(f"\n{shape.name}: out max-rel {e_out:.2e}, state rel-Frobenius {e_state:.2e}, "
           + ", ".join(f"{k} {v:.1e}" for k, v in errs.items()))

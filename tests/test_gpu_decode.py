@@ -71,3 +71,27 @@ def test_decode_with_state_in(ttcd):
                             w_T=shape.w_T, chunk=shape.chunk, state_in=s0.double().numpy())
     assert rel_max(y, ref["out"]) <= TOL_OUT
     assert rel_fro(state, ref["state_out"]) <= TOL_STATE
+
+
+def test_graph_decode_matches_eager_decode(ttcd):
+    """ttcd_block_decode_next replayed from one CUDA graph (the position read
+    from the state on the device) gives the eager decode's rows bit for bit,
+    across chunk commits, and the oracle's."""
+    shape = DEC_A.with_(name="dec_graph", T=2 * DEC_A.chunk + 37)
+    inp = make_block_inputs(shape, seed=9)
+    x, w = to_device(inp)
+    p = ttcd.BlockParams.from_shape(shape)
+    eager = ttcd.Decoder(w, p)
+    graph = ttcd.Decoder(w, p, graph=True)
+    ye, yg = [], []
+    for t in range(shape.T):
+        xt, bt = x[:, t].contiguous(), w["beta"][:, t].contiguous()
+        ye.append(eager.step(xt, bt))
+        yg.append(graph.step(xt, bt))
+    assert eager.check_status() == ttcd.OK and graph.check_status() == ttcd.OK
+    assert graph.graph is not None
+    ye, yg = torch.stack(ye, dim=1), torch.stack(yg, dim=1)
+    assert torch.equal(ye, yg)
+    assert torch.equal(eager.state_out(), graph.state_out())
+    ref = oracle_block(shape, inp)
+    assert rel_max(yg, ref["out"]) <= TOL_OUT
