@@ -35,7 +35,7 @@ from typing import Dict, Optional
 
 import numpy as np
 
-from .ttcd_oracle import block_forward, rms_norm, silu, window_mask
+from .ttcd_oracle import block_forward, fastweight_mlp, rms_norm, silu, window_mask
 
 # ---------------------------------------------------------------------------
 # One vector-Jacobian product per forward step
@@ -206,6 +206,59 @@ def windowed_attention_vjp(q, k, v, window: int, scale: float, do):
 # ---------------------------------------------------------------------------
 
 
+def fastweight_mlp_backward(u_T, u_S, beta, w_gate, w_up, w_down, w_proj, conv_T, conv_S,
+                            chunk: int, l2_eps: float, d_y, state_in=None,
+                            d_state_out=None) -> Dict[str, np.ndarray]:
+    """Gradients of L through the forward oracle's ``fastweight_mlp`` (same
+    arguments, without h_S), given d_y = dL/dy and d_state_out = dL/d state_out
+    (nullable: zero).  Returns a dict keyed "u_T", "u_S", "beta", "state_in",
+    "w_gate", "w_up", "w_down", "w_proj", "conv_T", "conv_S".
+
+    The steps of the forward in reverse: the chunked read y_t = (W_down +
+    S_i) Z_S[t], the exclusive prefix, the increments, the keys, the value
+    residual, the two convs and the two SwiGLU views (readings G1, G2).
+    """
+    fw = fastweight_mlp(u_T, u_S, beta, w_gate, w_up, w_down, w_proj, conv_T, conv_S, chunk,
+                        l2_eps, state_in=state_in, keep_prefixes=True)
+    w_down = np.asarray(w_down, np.float64)
+    d_y = np.asarray(d_y, np.float64)
+    B, T, d = d_y.shape
+    f = w_down.shape[1]
+    d_state_out = np.zeros((B, d, f)) if d_state_out is None else np.asarray(d_state_out,
+                                                                             np.float64)
+
+    # y_t = (W_down + S_i) Z_S[t] for t in chunk i
+    dZ_S = np.zeros_like(fw["Z_S"])
+    dW_down = np.zeros_like(w_down)
+    d_prefixes = np.zeros_like(fw["S_prefix"])
+    for b in range(B):
+        for i in range(fw["S_prefix"].shape[1]):
+            s0, s1 = i * chunk, min(T, (i + 1) * chunk)
+            dZ_S[b, s0:s1] = d_y[b, s0:s1] @ (w_down + fw["S_prefix"][b, i])
+            g = d_y[b, s0:s1].T @ fw["Z_S"][b, s0:s1]
+            dW_down += g
+            d_prefixes[b, i] = g
+
+    # exclusive prefix, chunk increments, keys, value residual
+    d_inc, d_state_in = exclusive_prefix_vjp(d_prefixes, d_state_out)
+    dR, dK, d_beta = chunk_increments_vjp(fw["R"], fw["K"], beta, chunk, d_inc)
+    dzb_S = l2_normalize_rows_vjp(fw["zbar_S"], l2_eps, dK)
+    dD, dwd, dW_proj = value_residual_vjp(fw["D"], w_down, w_proj, dR)
+    dW_down += dwd
+    dzb_T = dD                      # D = Zbar_T - Zbar_S
+    dzb_S = dzb_S - dD
+
+    # short convs, then SwiGLU of both views with the shared slow weights
+    dZ_T, dconv_T = causal_depthwise_conv_vjp(fw["Z_T"], conv_T, dzb_T)
+    dz, dconv_S = causal_depthwise_conv_vjp(fw["Z_S"], conv_S, dzb_S)
+    dZ_S += dz
+    du_T, dW_gate, dW_up = swiglu_vjp(u_T, w_gate, w_up, dZ_T)
+    du_S, dwg, dwu = swiglu_vjp(u_S, w_gate, w_up, dZ_S)
+    return {"u_T": du_T, "u_S": du_S, "beta": d_beta, "state_in": d_state_in,
+            "w_gate": dW_gate + dwg, "w_up": dW_up + dwu, "w_down": dW_down,
+            "w_proj": dW_proj, "conv_T": dconv_T, "conv_S": dconv_S}
+
+
 def block_backward(x, beta, weights: Dict[str, np.ndarray], d_out, *, n_q_heads: int,
                    n_kv_heads: int, head_dim: int, w_S: int, w_T: int, chunk: int,
                    rms_eps: float = 1e-6, l2_eps: float = 1e-6, rope_theta: float = 1e4,
@@ -233,36 +286,14 @@ def block_backward(x, beta, weights: Dict[str, np.ndarray], d_out, *, n_q_heads:
     d_state_out = np.zeros((B, d, f)) if d_state_out is None else np.asarray(d_state_out,
                                                                              np.float64)
 
-    # out = h_S + y;  y_t = (W_down + S_i) Z_S[t] for t in chunk i
-    d_hS = d_out.copy()
-    dZ_S = np.zeros_like(fw["Z_S"])
-    dW_down = np.zeros_like(W["w_down"])
-    d_prefixes = np.zeros_like(fw["S_prefix"])
-    for b in range(B):
-        for i in range(fw["S_prefix"].shape[1]):
-            s0, s1 = i * chunk, min(T, (i + 1) * chunk)
-            dZ_S[b, s0:s1] = d_out[b, s0:s1] @ (W["w_down"] + fw["S_prefix"][b, i])
-            g = d_out[b, s0:s1].T @ fw["Z_S"][b, s0:s1]
-            dW_down += g
-            d_prefixes[b, i] = g
-
-    # exclusive prefix, chunk increments, keys, value residual
-    d_inc, d_state_in = exclusive_prefix_vjp(d_prefixes, d_state_out)
-    dR, dK, d_beta = chunk_increments_vjp(fw["R"], fw["K"], beta, chunk, d_inc)
-    dzb_S = l2_normalize_rows_vjp(fw["zbar_S"], l2_eps, dK)
-    dD, dwd, dW_proj = value_residual_vjp(fw["D"], W["w_down"], W["w_proj"], dR)
-    dW_down += dwd
-    dzb_T = dD                      # D = Zbar_T - Zbar_S
-    dzb_S = dzb_S - dD
-
-    # short convs, then SwiGLU of both views with the shared slow weights
-    dZ_T, dconv_T = causal_depthwise_conv_vjp(fw["Z_T"], W["conv_T"], dzb_T)
-    dz, dconv_S = causal_depthwise_conv_vjp(fw["Z_S"], W["conv_S"], dzb_S)
-    dZ_S += dz
-    du_T, dW_gate, dW_up = swiglu_vjp(fw["u_T"], W["w_gate"], W["w_up"], dZ_T)
-    du_S, dwg, dwu = swiglu_vjp(fw["u_S"], W["w_gate"], W["w_up"], dZ_S)
-    dW_gate += dwg
-    dW_up += dwu
+    # the fast-weight MLP (everything between the MLP inputs u_P and y)
+    g = fastweight_mlp_backward(fw["u_T"], fw["u_S"], beta, W["w_gate"], W["w_up"],
+                                W["w_down"], W["w_proj"], W["conv_T"], W["conv_S"], chunk,
+                                l2_eps, d_out, state_in=state_in, d_state_out=d_state_out)
+    d_hS = d_out.copy()             # out = h_S + y
+    du_T, du_S, d_beta, d_state_in = g["u_T"], g["u_S"], g["beta"], g["state_in"]
+    dW_gate, dW_up, dW_down, dW_proj = g["w_gate"], g["w_up"], g["w_down"], g["w_proj"]
+    dconv_T, dconv_S = g["conv_T"], g["conv_S"]
 
     # MLP RMSNorm (shared gain) of both views
     dh_T, dg_mlp = rms_norm_vjp(fw["h_T"], W["g_mlp"], rms_eps, du_T)

@@ -205,3 +205,55 @@ def test_rmsnorm_and_swiglu_vjps_match_autograd():
     got = swiglu_vjp(u, wg, wu, dz)
     for r, g_ in zip(ref, got):
         np.testing.assert_allclose(g_, r, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------ the fast-weight MLP on its own
+
+MLP_NAMES = ["u_T", "u_S", "beta", "state_in", "w_gate", "w_up", "w_down", "w_proj", "conv_T",
+             "conv_S"]
+
+
+def _mlp_case(seed=0):
+    x, beta, w, s0, g_out, g_state = _case(seed)
+    rng = np.random.default_rng(seed + 50)
+    args = {"u_T": rng.standard_normal((B, T, D)), "u_S": rng.standard_normal((B, T, D)),
+            "beta": beta, "state_in": s0,
+            **{k: w[k] for k in ("w_gate", "w_up", "w_down", "w_proj", "conv_T", "conv_S")}}
+    return args, g_out, g_state
+
+
+def _mlp_loss(a, g_y, g_state):
+    r = orc.fastweight_mlp(a["u_T"], a["u_S"], a["beta"], a["w_gate"], a["w_up"], a["w_down"],
+                           a["w_proj"], a["conv_T"], a["conv_S"], SHAPE["chunk"], 1e-6,
+                           state_in=a["state_in"])
+    loss = np.sum(g_y * r["y"])
+    if g_state is not None:
+        loss += np.sum(g_state * r["state_out"])
+    return loss
+
+
+@pytest.mark.parametrize("with_state", [True, False], ids=["state", "no_state"])
+@pytest.mark.parametrize("name", MLP_NAMES)
+def test_mlp_backward_matches_central_difference(name, with_state):
+    """fastweight_mlp_backward against central differences of fastweight_mlp
+    (the review's 关键设计 2-3 forward) along a random direction."""
+    from oracle.ttcd_oracle_grad import fastweight_mlp_backward
+    args, g_y, g_state = _mlp_case()
+    if not with_state:
+        g_state = None
+    grads = fastweight_mlp_backward(
+        args["u_T"], args["u_S"], args["beta"], args["w_gate"], args["w_up"], args["w_down"],
+        args["w_proj"], args["conv_T"], args["conv_S"], SHAPE["chunk"], 1e-6, g_y,
+        state_in=args["state_in"], d_state_out=g_state)
+    v = np.random.default_rng(200 + MLP_NAMES.index(name)).standard_normal(args[name].shape)
+    eps = 1e-6
+
+    def at(delta):
+        a = dict(args)
+        a[name] = args[name] + delta * v
+        return _mlp_loss(a, g_y, g_state)
+
+    fd = (at(eps) - at(-eps)) / (2 * eps)
+    an = float(np.sum(grads[name] * v))
+    assert grads[name].shape == args[name].shape
+    assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (fd, an)

@@ -138,8 +138,8 @@ GRAD_MUTANTS = [
     ("vjp_dk_unscaled", "dk[b, :, kh] += scale * (ds.T @ q[b, :, h])", "dk[b, :, kh] += ds.T @ q[b, :, h]"),
     ("vjp_residual_sign", "dzb_S = dzb_S - dD", "dzb_S = dzb_S + dD"),
     ("vjp_read_ignores_fast_weight",
-     'dZ_S[b, s0:s1] = d_out[b, s0:s1] @ (W["w_down"] + fw["S_prefix"][b, i])',
-     'dZ_S[b, s0:s1] = d_out[b, s0:s1] @ W["w_down"]'),
+     'dZ_S[b, s0:s1] = d_y[b, s0:s1] @ (w_down + fw["S_prefix"][b, i])',
+     'dZ_S[b, s0:s1] = d_y[b, s0:s1] @ w_down'),
     ("vjp_teacher_path_dropped_from_x", "dx = dh_T + d_hS", "dx = d_hS"),
     ("vjp_student_window_as_teacher",
      'windowed_attention_vjp(fw["q"], fw["k"], fw["v"], w_S, scale, do_S)',
