@@ -584,6 +584,89 @@ def run_decode_bench(args, world, rank, local):
             "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
 
 
+def window_pairs(T: int, w: int) -> int:
+    """(query, key) pairs of one sequence and head inside a causal window of w keys."""
+    return w * (w + 1) // 2 + (T - w) * w if T >= w else T * (T + 1) // 2
+
+
+def run_backward(args, world, rank, local):
+    """The backward kernels at the Qwen3-0.6B block shape (T = --T, B = --B):
+    ttcd_fastweight_mlp_backward (the forward's front half and chunk scan
+    recomputed inside) and ttcd_dual_window_attn_backward, each timed alone with
+    CUDA events.  FLOPs are the algorithmic contractions of each call."""
+    import dual_window_attention_b200 as ttcd
+    from ttcd_workloads import make_mlp_inputs
+    ttcd.load_library()
+    peaks, peak_kind = load_peaks()
+    shape = QWEN3_0P6B_64K.with_(name=f"qwen3_0.6b_backward_T{args.T}", B=args.B, T=args.T)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    B, T, d, f = shape.B, shape.T, shape.d_model, shape.d_ff
+    Hq, Hkv, hd = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+    BT = B * T
+    Cp = (shape.chunk + 63) // 64 * 64
+    P = B * shape.n_chunks * Cp
+    g = torch.Generator().manual_seed(0)
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    lines = []
+    # fast-weight MLP backward
+    inp = make_mlp_inputs(shape, seed=0)
+    w = {k: v.to(dev) for k, v in inp.items()}
+    d_y = torch.randn(B, T, d, generator=g).to(torch.bfloat16).to(dev)
+    p = ttcd.BlockParams.from_shape(shape)
+    _, ws = ttcd.fastweight_mlp_backward(w["u_T"], w["u_S"], w["beta"], w, p, d_y)
+    ms = timed(lambda: ttcd.fastweight_mlp_backward(w["u_T"], w["u_S"], w["beta"], w, p, d_y,
+                                                    workspace=ws), args.steps, args.warmup)
+    if ttcd.check_device_status(ws) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the MLP backward")
+    recompute = 2 * 2 * BT * 2 * f * d + 2 * d * f * f + 2 * 2 * P * f * d
+    backward = (2 * BT * d * f + 5 * 2 * P * d * f + 2 * 2 * d * f * f + 2 * 2 * 2 * BT * 2 * f * d
+                + 2 * 2 * 2 * BT * f * d)
+    flops = recompute + backward
+    lines.append({"kernel": "ttcd_fastweight_mlp_backward", "ms": ms, "flops": flops,
+                  "tflops_per_s": flops / ms / 1e9})
+    del w, ws, inp
+    # dual-window attention backward
+    q = torch.randn(B, T, Hq, hd, generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn(B, T, Hkv, hd, generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, T, Hkv, hd, generator=g).to(torch.bfloat16).to(dev)
+    o_T, o_S, lse_T, lse_S = ttcd.dual_window_attn(q, k, v, shape.w_S, shape.w_T, lse=True)
+    do_T = torch.randn(B, T, Hq, hd, generator=g).to(torch.bfloat16).to(dev)
+    do_S = torch.randn(B, T, Hq, hd, generator=g).to(torch.bfloat16).to(dev)
+    _, _, _, aws = ttcd.dual_window_attn_backward(q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S,
+                                                  shape.w_S, shape.w_T)
+    ms = timed(lambda: ttcd.dual_window_attn_backward(q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S,
+                                                      shape.w_S, shape.w_T, workspace=aws),
+               args.steps, args.warmup)
+    if ttcd.check_device_status(aws) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the attention backward")
+    # per visible pair and head: S recomputed, dP, dV, dK, dQ (2 hd FLOPs each)
+    pairs = B * Hq * (window_pairs(T, shape.w_T) + window_pairs(T, shape.w_S))
+    flops = 10.0 * hd * pairs
+    lines.append({"kernel": "ttcd_dual_window_attn_backward", "ms": ms, "flops": flops,
+                  "tflops_per_s": flops / ms / 1e9})
+    if rank == 0:
+        for l in lines:
+            l.update({"metric": "backward kernel time (Qwen3-0.6B block shape)",
+                      "config": workload_config(shape), "steps": args.steps,
+                      "warmup": args.warmup, "peak_tflops": peaks["bf16_tflops"],
+                      "frac": l["tflops_per_s"] / peaks["bf16_tflops"],
+                      "peak_source": f"{peak_kind} bf16_tflops"})
+            print(json.dumps(l), flush=True)
+
+
 def measure_stack(args, world, local, B, T, steps, warmup):
     """The 28-layer stack of Qwen3-0.6B-shaped blocks end to end (B x T): every
     layer one ttcd_block_forward on its own weights, one shared workspace."""
@@ -659,7 +742,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
-    ap.add_argument("--mode", choices=["block", "attn", "stack", "decode"], default="block",
+    ap.add_argument("--mode", choices=["block", "attn", "stack", "decode", "backward"],
+                    default="block",
                     help="block: the whole IP-TTCD block (default); attn: attention alone; "
                          "stack: 28 blocks end to end; decode: one token at a time")
     ap.add_argument("--T", type=int, default=65536,
@@ -690,6 +774,8 @@ def main():
             run_stack(args, world, rank, local)
         elif args.mode == "decode":
             run_decode_bench(args, world, rank, local)
+        elif args.mode == "backward":
+            run_backward(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -48,6 +48,11 @@ class _Weights(ctypes.Structure):
 
 WEIGHT_NAMES = tuple(n for n, _ in _Weights._fields_)
 
+
+class _MlpGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_gate", "w_up", "w_down", "w_proj", "conv_T",
+                                               "conv_S")]
+
 _lib = None
 
 
@@ -101,6 +106,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_shard_attend.argtypes = [vp, vp, W, P, ll, vp, vp, sz, vp]
     lib.ttcd_shard_mix.argtypes = [vp, vp, W, P, ll, vp, vp, sz, vp]
     lib.ttcd_shard_finish.argtypes = [W, P, ll, vp, vp, vp, vp, sz, vp]
+    lib.ttcd_dual_window_attn_backward_workspace_size.argtypes = [i, i, i]
+    lib.ttcd_dual_window_attn_backward_workspace_size.restype = sz
+    lib.ttcd_dual_window_attn_backward.argtypes = [vp] * 12 + [i] * 7 + [f, vp, sz, vp]
+    lib.ttcd_fastweight_mlp_backward_workspace_size.argtypes = [P]
+    lib.ttcd_fastweight_mlp_backward_workspace_size.restype = sz
+    lib.ttcd_fastweight_mlp_backward.argtypes = [vp, vp, vp, W, P, vp, vp, vp, vp, vp, vp, vp,
+                                                 ctypes.POINTER(_MlpGrads), vp, sz, vp]
     lib.ttcd_fastweight_mlp_noalloc.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp]
     lib.ttcd_fastweight_mlp_noalloc.restype = i
     lib.ttcd_fastweight_mlp_noalloc_capacity.argtypes = []
@@ -109,7 +121,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                "ttcd_block_forward", "ttcd_block_forward_profiled", "ttcd_block_workspace_offset",
                "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
                "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read",
-               "ttcd_block_decode_next",
+               "ttcd_block_decode_next", "ttcd_fastweight_mlp_backward",
+               "ttcd_dual_window_attn_backward",
                "ttcd_shard_qkv", "ttcd_shard_attend", "ttcd_shard_mix", "ttcd_shard_finish"):
         getattr(lib, fn).restype = i
     _lib = lib
@@ -204,6 +217,29 @@ def dual_window_attn(q, k, v, w_S: int, w_T: int, scale: float = 0.0, o_T=None, 
                                    _stream(stream))
     _check(st, "ttcd_dual_window_attn")
     return o_T, o_S, lse_T, lse_S
+
+
+def dual_window_attn_backward(q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, w_S: int, w_T: int,
+                              scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                              stream=None):
+    """Vector-Jacobian product of ``dual_window_attn`` (bf16, hd 64 or 128):
+    (dq, dk, dv) in fp32 for output gradients do_T, do_S, given the forward's
+    o_T, o_S, lse_T, lse_S.  Returns (dq, dk, dv, workspace)."""
+    lib = load_library()
+    B, T, Hq, hd = q.shape
+    Hkv = k.shape[2]
+    need = int(lib.ttcd_dual_window_attn_backward_workspace_size(B, T, Hq))
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    dq = torch.empty(B, T, Hq, hd, device=q.device, dtype=torch.float32)
+    dk = torch.empty(B, T, Hkv, hd, device=q.device, dtype=torch.float32)
+    dv = torch.empty_like(dk)
+    st = lib.ttcd_dual_window_attn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o_T), _ptr(o_S), _ptr(lse_T), _ptr(lse_S), _ptr(do_T),
+        _ptr(do_S), _ptr(dq), _ptr(dk), _ptr(dv), B, T, Hq, Hkv, hd, w_S, w_T, scale,
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ttcd_dual_window_attn_backward")
+    return dq, dk, dv, workspace
 
 
 def dual_window_attn_lse(q, k, v, w_S: int, w_T: int, scale: float = 0.0, stream=None):
@@ -518,6 +554,39 @@ def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockPar
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "ttcd_fastweight_mlp")
     return y, st_t, workspace
+
+
+def fastweight_mlp_backward(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams,
+                            d_y, state_in=None, d_state_out=None,
+                            workspace: Optional[torch.Tensor] = None, stream=None):
+    """Vector-Jacobian product of ``fastweight_mlp`` (bf16): the gradients of a
+    loss with dL/dy = d_y and dL/dstate_out = d_state_out (or zero) with respect
+    to u_T, u_S, beta, state_in and the MLP weights, all fp32.  Returns
+    (grads dict keyed "u_T", "u_S", "beta", "state_in", "w_gate", "w_up",
+    "w_down", "w_proj", "conv_T", "conv_S"; workspace)."""
+    lib = load_library()
+    need = int(lib.ttcd_fastweight_mlp_backward_workspace_size(ctypes.byref(p.c())))
+    if need == 0:
+        raise TTCDError(ERR_UNSUPPORTED, "ttcd_fastweight_mlp_backward_workspace_size")
+    dev = u_T.device
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    f32 = dict(device=dev, dtype=torch.float32)
+    B, T, d, f, k = p.B, p.T, p.d_model, p.d_ff, p.conv_k
+    g = {"u_T": torch.empty(B, T, d, **f32), "u_S": torch.empty(B, T, d, **f32),
+         "beta": torch.empty(B, T, **f32), "state_in": torch.empty(B, d, f, **f32),
+         "w_gate": torch.empty(f, d, **f32), "w_up": torch.empty(f, d, **f32),
+         "w_down": torch.empty(d, f, **f32), "w_proj": torch.empty(f, f, **f32),
+         "conv_T": torch.empty(f, k, **f32), "conv_S": torch.empty(f, k, **f32)}
+    gc = _MlpGrads(*[_ptr(g[n]) for n, _ in _MlpGrads._fields_])
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_fastweight_mlp_backward(
+        _ptr(u_T), _ptr(u_S), _ptr(beta), ctypes.byref(wc), ctypes.byref(pc), _ptr(state_in),
+        _ptr(d_y), _ptr(d_state_out), _ptr(g["u_T"]), _ptr(g["u_S"]), _ptr(g["beta"]),
+        _ptr(g["state_in"]), ctypes.byref(gc), _ptr(workspace), workspace.numel(),
+        _stream(stream))
+    _check(st, "ttcd_fastweight_mlp_backward")
+    return g, workspace
 
 
 def fastweight_mlp_noalloc(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams,

@@ -523,28 +523,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   }
 }
 
-// 8 consecutive elements (16-byte aligned) to and from fp32 registers
-__device__ __forceinline__ void ld8f(const __nv_bfloat16* src, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(src);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = bf16lo_to_f32(w[i]);
-    v[2 * i + 1] = bf16hi_to_f32(w[i]);
-  }
-}
-__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void st8f(__nv_bfloat16* dst, const float (&v)[8]) {
-  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-}
-__device__ __forceinline__ void st8f(float* dst, const float (&v)[8]) {
-  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
 
 // o_T = (o_S e^{lse_S} + o_far e^{lse_far}) / (e^{lse_S} + e^{lse_far}) and
 // lse_T = logaddexp(lse_S, lse_far): the exact merge of two partial softmax

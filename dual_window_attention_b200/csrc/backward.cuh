@@ -1,0 +1,328 @@
+// Backward of the in-place fast-weight MLP (sm_100a): GEMM epilogues and the
+// memory-bound steps between the GEMMs.
+//
+// papernotes.org review "Learning What to Remember", 关键设计 2-3 and 局限与展望
+// (training runs the whole block, the write path included): the chain rule of
+//   Z_P = silu(u_P W_gate^T) * (u_P W_up^T),  Zbar_P = conv_P(Z_P),
+//   D = Zbar_T - Zbar_S,  r_t = M D_t (M = W_down W_proj),
+//   s_t = beta_t / n_t,  n_t = (|Zbar_S[t]|^2 + eps)^(1/2),
+//   Delta W_i = sum_{t in C_i} s_t r_t Zbar_S[t]^T,  S_{i+1} = S_i + Delta W_i,
+//   y_t = (W_down + S_{i(t)}) Z_S[t],
+// taken in the reverse of that order.  With G_i = dL/dDelta W_i (the reverse
+// prefix of the per-chunk dL/dS_i = sum_{t in C_i} dy_t Z_S[t]^T):
+//   dRt_t = G_i Zbar_S[t]                 (gradient of the scaled row s_t r_t)
+//   E_t   = M^T dRt_t,  dD_t = s_t E_t,  ds_t = D_t . E_t  (= r_t . dRt_t)
+//   dbeta_t = ds_t / n_t,  dZbar_S[t] = G_i^T (s_t r_t) - ds_t beta_t / n_t^3 Zbar_S[t] - dD_t
+//   dM = sum_t s_t dRt_t D_t^T,  dW_down += dM W_proj^T,  dW_proj = W_down^T dM.
+// Rows of the chunk-padded buffers follow the forward's layout: sequence b,
+// chunk i, row j at (b Nc + i) Cp + j, pad rows zero.
+#pragma once
+#include "gemm.cuh"
+
+namespace ttcd {
+
+// out_u[row] = bf16(acc), out_s[row] = bf16(acc * scale[row]); columns < N (a
+// multiple of 64).  Direct stores.
+struct EpiStoreScaledPair {
+  static constexpr bool kStaged = false;
+  static constexpr bool kCollective = false;
+  __nv_bfloat16* out_u;
+  __nv_bfloat16* out_s;
+  long long ldo;
+  int N;
+  const float* scale;
+  __device__ float pre(const TileCtx& c, int r) const {
+    return r < c.valid_rows ? __ldg(scale + c.row0 + r) : 0.f;
+  }
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&, float sc) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      const int col = c.tn * BN + cc;
+      if (col >= N) break;
+      float v[32];
+      tmem_ld32f(taddr + cc, v);
+      if (!ok) continue;
+      store_bf16x32(out_u + row * ldo + col, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= sc;
+      store_bf16x32(out_s + row * ldo + col, v);
+    }
+  }
+};
+
+// acc = E = dRt M (fp32).  dD[row] = scale[row] * E (fp32 [rows, N]) and
+// part[tn][row] = sum over this tile's columns of D[row, col] * E[row, col]
+// (D bf16 [rows, N]); fixed summation order.
+struct EpiBwdE {
+  static constexpr bool kStaged = false;
+  static constexpr bool kCollective = false;
+  float* dD;
+  const __nv_bfloat16* D;
+  float* part;
+  long long rows;
+  int N;
+  const float* scale;
+  __device__ float pre(const TileCtx& c, int r) const {
+    return r < c.valid_rows ? __ldg(scale + c.row0 + r) : 0.f;
+  }
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&, float sc) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+    float dot = 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      const int col = c.tn * BN + cc;
+      if (col >= N) break;
+      float v[32];
+      tmem_ld32f(taddr + cc, v);
+      if (!ok) continue;
+      float dv[32];
+      load_x32(D + row * N + col, dv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        dot = fmaf(dv[i], v[i], dot);
+        v[i] *= sc;
+      }
+      store_f32x32(dD + row * N + col, v);
+    }
+    if (ok) part[static_cast<long long>(c.tn) * rows + row] = dot;
+  }
+};
+
+// out[row] = acc + coef[row] * X[row] - Y[row]  (X bf16, Y and out fp32, all
+// [rows, N]).
+struct EpiBwdZbS {
+  static constexpr bool kStaged = false;
+  static constexpr bool kCollective = false;
+  float* out;
+  const __nv_bfloat16* X;
+  const float* Y;
+  int N;
+  const float* coef;
+  __device__ float pre(const TileCtx& c, int r) const {
+    return r < c.valid_rows ? __ldg(coef + c.row0 + r) : 0.f;
+  }
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&, float cf) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      const int col = c.tn * BN + cc;
+      if (col >= N) break;
+      float v[32];
+      tmem_ld32f(taddr + cc, v);
+      if (!ok) continue;
+      float x[32], y[32];
+      load_x32(X + row * N + col, x);
+      load_x32(Y + row * N + col, y);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += fmaf(cf, x[i], -y[i]);
+      store_f32x32(out + row * N + col, v);
+    }
+  }
+};
+
+// Gate/up recomputed (accumulator columns [0, BN/2) a = u W_gate^T, [BN/2, BN)
+// b = u W_up^T for output columns tn*BN/2 + [0, BN/2)), with dz = dZ[row, col]:
+//   da = dz b silu'(a),  db = dz silu(a),  Z = silu(a) b,
+// silu'(a) = sigma(a) (1 + a (1 - sigma(a))).  dab[row] = [da | db] (bf16, row
+// length 2N), z[row] = Z (bf16, row length N).
+struct EpiSwiGLUBwd {
+  static constexpr bool kStaged = false;
+  static constexpr bool kCollective = false;
+  const float* dZ;
+  __nv_bfloat16* dab;
+  __nv_bfloat16* z;
+  int N;
+  __device__ float pre(const TileCtx&, int) const { return 1.f; }
+  template <int BN>
+  __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage&, float) const {
+    const bool ok = r < c.valid_rows;
+    const long long row = c.row0 + r;
+#pragma unroll 1
+    for (int cc = 0; cc < BN / 2; cc += 32) {
+      const int col = c.tn * (BN / 2) + cc;
+      if (col >= N) break;
+      float a[32], b[32];
+      tmem_ld32f(taddr + cc, a);
+      tmem_ld32f(taddr + BN / 2 + cc, b);
+      if (!ok) continue;
+      float dz[32], zz[32];
+      load_x32(dZ + row * N + col, dz);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float sg = __fdividef(1.0f, 1.0f + __expf(-a[i]));
+        const float si = a[i] * sg;
+        zz[i] = si * b[i];
+        const float da = dz[i] * b[i] * sg * fmaf(a[i], 1.0f - sg, 1.0f);
+        b[i] = dz[i] * si;
+        a[i] = da;
+      }
+      __nv_bfloat16* drow = dab + row * (2ll * N);
+      store_bf16x32(drow + col, a);
+      store_bf16x32(drow + N + col, b);
+      store_bf16x32(z + row * N + col, zz);
+    }
+  }
+};
+
+// dst[(b Nc + i) Cp + j] = src[b T + i C + j] for tokens of the sequence, zero
+// on pad rows; 8 elements (16 bytes) per thread, ncols a multiple of 8.
+template <class E>
+__global__ void chunk_pad_rows_kernel(const E* __restrict__ src, E* __restrict__ dst, int ncols,
+                                      int T, int C, int Cp, int Nc, long long P) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_row = ncols / (16 / static_cast<int>(sizeof(E)));
+  if (idx >= P * per_row) return;
+  const long long p = idx / per_row;
+  const int q = static_cast<int>(idx % per_row);
+  const long long seq = static_cast<long long>(Nc) * Cp;
+  const int b = static_cast<int>(p / seq);
+  const long long rem = p % seq;
+  const int i = static_cast<int>(rem / Cp), j = static_cast<int>(rem % Cp);
+  const int t = i * C + j;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (j < C && t < T)
+    v = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(b) * T + t) * ncols) + q);
+  reinterpret_cast<uint4*>(dst + p * ncols)[q] = v;
+}
+
+// Per padded row: ds = sum of the E epilogue's partial dots, n = (ssq + eps)^(1/2);
+// d_beta[b, t] = ds / n and coef = -ds beta / n^3 (zero on pad rows).
+__global__ void key_backward_kernel(const float* __restrict__ epart, int n_epart,
+                                    const float* __restrict__ ssq_part, int n_ssq,
+                                    const float* __restrict__ beta, float* __restrict__ d_beta,
+                                    float* __restrict__ coef, int T, int C, int Cp, int Nc,
+                                    long long P, float eps) {
+  const long long p = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (p >= P) return;
+  const long long seq = static_cast<long long>(Nc) * Cp;
+  const int b = static_cast<int>(p / seq);
+  const long long rem = p % seq;
+  const int i = static_cast<int>(rem / Cp), j = static_cast<int>(rem % Cp);
+  const int t = i * C + j;
+  if (!(j < C && t < T)) {
+    coef[p] = 0.f;
+    return;
+  }
+  float ds = 0.f, ssq = 0.f;
+  for (int q = 0; q < n_epart; ++q) ds += epart[static_cast<long long>(q) * P + p];
+  for (int q = 0; q < n_ssq; ++q) ssq += ssq_part[static_cast<long long>(q) * P + p];
+  const float inv = rsqrtf(ssq + eps);
+  const long long bt = static_cast<long long>(b) * T + t;
+  d_beta[bt] = ds * inv;
+  coef[p] = -ds * beta[bt] * inv * inv * inv;
+}
+
+// Backward of the causal depthwise convs (tap m multiplies t - m, so the
+// transpose reads t + m) and the sum with the read path's dZ_S:
+//   dZ[path, b, s, c] = sum_{m < k, s + m < T} w_path[c, m] dZbar_path[b, s + m, c]
+//                       (+ dZs_read[b, s, c] for the student path),
+// dZbar_* in the chunk-padded layout, dZ [2, B, T, f] fp32 (teacher first).
+// Four columns per thread.
+__global__ void conv_backward_kernel(const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
+                                     const float* __restrict__ dzs_read,
+                                     const __nv_bfloat16* __restrict__ conv_T,
+                                     const __nv_bfloat16* __restrict__ conv_S,
+                                     float* __restrict__ dZ, int B, int T, int f, int k, int C,
+                                     int Cp, int Nc) {
+  const long long BT = static_cast<long long>(B) * T;
+  const int per_row = f / 4;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= 2 * BT * per_row) return;
+  const long long row = idx / per_row;
+  const int c0 = static_cast<int>(idx % per_row) * 4;
+  const bool student = row >= BT;
+  const long long bt = student ? row - BT : row;
+  const int b = static_cast<int>(bt / T), s = static_cast<int>(bt % T);
+  const float* dzb = student ? dzb_S : dzb_T;
+  const __nv_bfloat16* w = student ? conv_S : conv_T;
+  float4 acc = student ? __ldg(reinterpret_cast<const float4*>(dzs_read + bt * f + c0))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int m = 0; m < k; ++m) {
+    const int t = s + m;
+    if (t >= T) break;
+    const long long pr = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
+    const float4 g = __ldg(reinterpret_cast<const float4*>(dzb + pr * f + c0));
+    acc.x = fmaf(__bfloat162float(w[(c0 + 0) * k + m]), g.x, acc.x);
+    acc.y = fmaf(__bfloat162float(w[(c0 + 1) * k + m]), g.y, acc.y);
+    acc.z = fmaf(__bfloat162float(w[(c0 + 2) * k + m]), g.z, acc.z);
+    acc.w = fmaf(__bfloat162float(w[(c0 + 3) * k + m]), g.w, acc.w);
+  }
+  reinterpret_cast<float4*>(dZ + row * f)[c0 / 4] = acc;
+}
+
+constexpr int TAP_SPLITS = 32;  // token splits of the tap gradient (partials per split)
+constexpr int TAP_LANES = 8;    // row lanes per block
+
+// part[split][path][c][m] = sum over the split's tokens (b, t), t >= m, of
+// dZbar_path[b, t, c] Z_path[b, t - m, c].  Block: 32 columns x 8 row lanes;
+// grid (f / 32, TAP_SPLITS, 2).  Z [2, B, T, f] bf16, dZbar chunk-padded fp32.
+template <int KMAX>
+__global__ void __launch_bounds__(256) conv_tap_grad_kernel(
+    const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
+    const __nv_bfloat16* __restrict__ z, float* __restrict__ part, int B, int T, int f, int k,
+    int C, int Cp, int Nc) {
+  const int lane = threadIdx.x & 31, rl = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
+  const int split = blockIdx.y, path = blockIdx.z;
+  const long long BT = static_cast<long long>(B) * T;
+  const long long per = (BT + TAP_SPLITS - 1) / TAP_SPLITS;
+  const long long r0 = split * per, r1 = min(BT, r0 + per);
+  const float* dzb = path ? dzb_S : dzb_T;
+  const __nv_bfloat16* zp = z + path * BT * f;
+  float acc[KMAX];
+#pragma unroll
+  for (int m = 0; m < KMAX; ++m) acc[m] = 0.f;
+  for (long long bt = r0 + rl; bt < r1; bt += TAP_LANES) {
+    const int b = static_cast<int>(bt / T), t = static_cast<int>(bt % T);
+    const long long pr = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
+    const float g = dzb[pr * f + c];
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m)
+      if (m < k && t >= m) acc[m] = fmaf(g, __bfloat162float(zp[(bt - m) * f + c]), acc[m]);
+  }
+  __shared__ float red[TAP_LANES][KMAX][32];
+#pragma unroll
+  for (int m = 0; m < KMAX; ++m) red[rl][m][lane] = acc[m];
+  __syncthreads();
+  if (rl < KMAX && rl < k) {
+    float s = 0.f;
+    for (int q = 0; q < TAP_LANES; ++q) s += red[q][rl][lane];
+    part[((static_cast<long long>(split) * 2 + path) * f + c) * k + rl] = s;
+  }
+}
+
+// out[path][c][m] = sum over splits of part[split][path][c][m].
+__global__ void conv_tap_reduce_kernel(const float* __restrict__ part, float* __restrict__ out_T,
+                                       float* __restrict__ out_S, int f, int k) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= 2 * f * k) return;
+  const int path = idx / (f * k), e = idx % (f * k);
+  float s = 0.f;
+  for (int q = 0; q < TAP_SPLITS; ++q) s += part[(static_cast<long long>(q) * 2 + path) * f * k + e];
+  (path ? out_S : out_T)[e] = s;
+}
+
+// dW_down = part + sum_b (d_state_in[b] - d_state_out[b])  (d_state_out nullable):
+// the read path's sum_t dy_t Z_S[t]^T is the reverse prefix's total less its start.
+__global__ void dw_down_combine_kernel(const float* __restrict__ part,
+                                       const float* __restrict__ d_state_in,
+                                       const float* __restrict__ d_state_out,
+                                       float* __restrict__ out, int B, long long n) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float s = part[i];
+  for (int b = 0; b < B; ++b) {
+    s += d_state_in[b * n + i];
+    if (d_state_out) s -= d_state_out[b * n + i];
+  }
+  out[i] = s;
+}
+
+}  // namespace ttcd

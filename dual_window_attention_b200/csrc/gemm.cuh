@@ -128,6 +128,28 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
 }
 __device__ __forceinline__ void store_x32(__nv_bfloat16* dst, const float (&v)[32]) { store_bf16x32(dst, v); }
 __device__ __forceinline__ void store_x32(float* dst, const float (&v)[32]) { store_f32x32(dst, v); }
+// 8 consecutive elements (16-byte aligned) to and from fp32 registers
+__device__ __forceinline__ void ld8f(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = bf16lo_to_f32(w[i]);
+    v[2 * i + 1] = bf16hi_to_f32(w[i]);
+  }
+}
+__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8f(__nv_bfloat16* dst, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ void st8f(float* dst, const float (&v)[8]) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
 
 __device__ __forceinline__ void load_x32(const __nv_bfloat16* src, float (&v)[32]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
@@ -202,7 +224,8 @@ struct EpiStage {
 // B_MN = true (bf16 only): B is given as B^T, a row-major [K, N] matrix (N
 // contiguous), and is read as an MN-major tcgen05 operand: TMA boxes of 64
 // N-elements x 64 K-rows, leading-byte offset = one box, 16 K-rows (2048 bytes)
-// per MMA step.
+// per MMA step.  With row groups (b_group_rows > 0) group g's B^T starts at row
+// g * b_group_rows, so K must then be a multiple of 64.
 template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom,
           bool B_MN = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -298,7 +321,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           } else if constexpr (B_MN) {
 #pragma unroll
             for (int q = 0; q < BN / 64; ++q)
-              tma_load_2d(sb + q * MN_BOX_BYTES, &mapB0, &full[s], c.tn * BN + 64 * q, kb * BK);
+              tma_load_2d(sb + q * MN_BOX_BYTES, &mapB0, &full[s], c.tn * BN + 64 * q,
+                          c.b_row0 + kb * BK);
           } else {
             tma_load_2d(sb, &mapB0, &full[s], kb * BK, c.b_row0 + c.tn * BN);
           }
@@ -635,14 +659,14 @@ struct EpiSwiGLU {
 //      fp32 and writes its 32 values to a shared tile [path][row][column]
 //      (16-byte slots swizzled by row, so both the row-wise writes and the
 //      column-wise reads are conflict-free; two tiles alternate by slice);
-//   B  thread (column c, row group g) slides the causal depthwise conv down the
-//      16 rows [16g, 16g + 16) of column c for both paths, with the column's
-//      taps in registers and the k-1 rows before the group read from the tile,
-//      and writes D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and
-//      the bf16 Z_S (output-GEMM operand): a warp writes 64 contiguous bytes of
-//      each row.  Its Kp^2 accumulate per row; one warp reduction per tile
-//      gives the sum over the tile's 128 columns (the key norm becomes a row
-//      scale of R later).
+//   B  thread (row R, column group cg of 8 columns; two rows R and R + 32 per
+//      thread) forms the causal depthwise convs of both paths from the k rows
+//      R - k + 1 .. R of the tile (16-byte shared loads), and writes 8 columns
+//      of D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and of the
+//      bf16 Z_S (output-GEMM operand) with one 16-byte store each.  The row's
+//      padded index is formed once per tile, the taps of the 8 columns once per
+//      slice.  Kp^2 accumulates per row over the slices; four lanes share a
+//      row and reduce once per tile (the key norm becomes a row scale of R).
 // The tile's first k-1 rows only feed the conv (their outputs belong to the
 // previous tile); fp32 Z never reaches memory.
 //   z_halo [2, B, k-1, f] fp32: Z rows before token 0 (nullable: zeros)
@@ -676,18 +700,28 @@ struct EpiSwiGLUConv {
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     static_assert(BN == 256, "gate/up tiles are 128 gate + 128 up columns");
-    const int lane = threadIdx.x & 31;
     const int rin = r & 63;               // phase A: this thread's row within its path
     const int path = r >= 64 ? 1 : 0;
     const int ta = c.tok0 + rin;
     const int b = c.group;
     const int H = k - 1;
-    // phase B: column `lane` of the slice, rows [16 g, 16 g + 16)
-    const int g = (threadIdx.x >> 5) - 2;
-    uint8_t* tiles = stg.buf - g * 8192;  // the 32 KB staging area: two 16 KB z tiles
-    float ssq_acc[16];
+    const int et = static_cast<int>(threadIdx.x) - 64;  // epilogue thread 0..127
+    uint8_t* tiles = stg.buf - ((et >> 5) * 8192);      // the 32 KB staging area: two 16 KB z tiles
+    // phase B: rows et/4 and et/4 + 32, columns 8 cg .. 8 cg + 7 of each slice
+    const int cg = et & 3;
+    int brow[2];
+    bool bval[2];
+    long long bp[2], bz[2];
+    float ssq_acc[2] = {0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 16; ++i) ssq_acc[i] = 0.f;
+    for (int u = 0; u < 2; ++u) {
+      brow[u] = (et >> 2) + 32 * u;
+      const int t = c.tok0 + brow[u];
+      bval[u] = brow[u] >= H && t >= 0 && t < T;
+      const int tt = bval[u] ? t : 0;
+      bp[u] = pidx(b, tt) * f;
+      bz[u] = (static_cast<long long>(b) * T + tt) * f;
+    }
 #pragma unroll 1
     for (int s = 0; s < 4; ++s) {
       const int cc = 32 * s;
@@ -724,61 +758,70 @@ struct EpiSwiGLUConv {
               make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
       }
       epi_bar_sync();
-      // ---- B: the conv down column `lane`, rows [16 g, 16 g + 16), both paths
+      // ---- B: the convs of rows brow[u], columns col0 + 8 cg .. + 7, both paths
       {
-        const int col = col0 + lane;
-        float wT[KMAX], wS[KMAX];
+        const int col = col0 + 8 * cg;
+        float aT[2][8], aS[2][8], z0[2][8];
 #pragma unroll
-        for (int m = 0; m < KMAX; ++m) {
-          wT[m] = m < k ? __bfloat162float(tapT[static_cast<long long>(col) * k + m]) : 0.f;
-          wS[m] = m < k ? __bfloat162float(tapS[static_cast<long long>(col) * k + m]) : 0.f;
-        }
-        constexpr int W = 16 + KMAX - 1;  // rows 16g - (KMAX-1) .. 16g + 15
-        float zT[W], zS[W];
-        const uint32_t cofs = ((lane >> 2) << 4) | ((lane & 3) << 2);
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int i = 0; i < W; ++i) {
-          const int row = 16 * g + i - (KMAX - 1);
-          if (row >= 0) {
-            const int RT = row, RS = 64 + row;
-            zT[i] = *reinterpret_cast<const float*>(tile + RT * 128 + (cofs ^ ((RT & 7) << 4)));
-            zS[i] = *reinterpret_cast<const float*>(tile + RS * 128 + (cofs ^ ((RS & 7) << 4)));
-          } else {
-            zT[i] = 0.f;
-            zS[i] = 0.f;
+          for (int i = 0; i < 8; ++i) { aT[u][i] = 0.f; aS[u][i] = 0.f; z0[u][i] = 0.f; }
+#pragma unroll
+        for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
+          if (m >= k) break;
+          float tT[8], tS[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            tT[i] = __bfloat162float(tapT[static_cast<long long>(col + i) * k + m]);
+            tS[i] = __bfloat162float(tapS[static_cast<long long>(col + i) * k + m]);
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int RT = brow[u] - m, RS = 64 + brow[u] - m;
+            if (RT < 0) continue;
+            float zt[8], zs[8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int j = 2 * cg + h;
+              const float4 x = *reinterpret_cast<const float4*>(tile + RT * 128 + ((j ^ (RT & 7)) << 4));
+              const float4 y = *reinterpret_cast<const float4*>(tile + RS * 128 + ((j ^ (RS & 7)) << 4));
+              zt[4 * h] = x.x; zt[4 * h + 1] = x.y; zt[4 * h + 2] = x.z; zt[4 * h + 3] = x.w;
+              zs[4 * h] = y.x; zs[4 * h + 1] = y.y; zs[4 * h + 2] = y.z; zs[4 * h + 3] = y.w;
+            }
+            if (m == 0) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) z0[u][i] = zs[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              aT[u][i] = fmaf(tT[i], zt[i], aT[u][i]);
+              aS[u][i] = fmaf(tS[i], zs[i], aS[u][i]);
+            }
           }
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int rrow = 16 * g + i;
-          const int t = c.tok0 + rrow;
-          float bT = 0.f, bS = 0.f;
+        for (int u = 0; u < 2; ++u) {
+          if (!bval[u]) continue;
+          float dd[8];
 #pragma unroll
-          for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
-            bT += wT[m] * zT[i + KMAX - 1 - m];
-            bS += wS[m] * zS[i + KMAX - 1 - m];
+          for (int i = 0; i < 8; ++i) {
+            dd[i] = aT[u][i] - aS[u][i];
+            ssq_acc[u] = fmaf(aS[u][i], aS[u][i], ssq_acc[u]);
           }
-          if (rrow >= H && t >= 0 && t < T) {
-            const long long p = pidx(b, t);
-            D[p * f + col] = __float2bfloat16_rn(bT - bS);
-            Kp[p * f + col] = __float2bfloat16_rn(bS);
-            Zs[(static_cast<long long>(b) * T + t) * f + col] =
-                __float2bfloat16_rn(zS[i + KMAX - 1]);
-            ssq_acc[i] += bS * bS;
-          }
+          st8f(D + bp[u] + col, dd);
+          st8f(Kp + bp[u] + col, aS[u]);
+          st8f(Zs + bz[u] + col, z0[u]);
         }
       }
     }
-    // per-token sums of Kp^2 over the tile's columns: one warp reduction per row
+    // per-token sums of Kp^2 over the tile's columns: the four lanes of a row
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float v = ssq_acc[i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      const int rrow = 16 * g + i;
-      const int t = c.tok0 + rrow;
-      if (lane == i && rrow >= H && t >= 0 && t < T)
-        ssq[static_cast<long long>(c.tn) * P + pidx(b, t)] = v;
+    for (int u = 0; u < 2; ++u) {
+      float v = ssq_acc[u];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if (cg == 0 && bval[u])
+        ssq[static_cast<long long>(c.tn) * P + pidx(b, c.tok0 + brow[u])] = v;
     }
   }
 };

@@ -36,6 +36,10 @@ struct ScanArgs {
   // returns at once (every thread of every block alike, before any set-up).
   const long long* commit_pos;
   int commit_C;
+  // Walk the chunks last to first (step j reads chunk Nc-1-j and w_all entries
+  // are written at the chunk they belong to): with w_down null this is the
+  // backward of the exclusive prefix, w_all[i] = state_in + sum_{j>i} Delta_j.
+  bool reverse;
 };
 
 constexpr int SCAN_BN = 192;
@@ -101,7 +105,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, st, abort)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
-          const int y = (b * a.Nc + i) * a.Cp + kb * BK;  // first token of the k-block
+          const int ci = a.reverse ? a.Nc - 1 - i : i;
+          const int y = (b * a.Nc + ci) * a.Cp + kb * BK;  // first token of the k-block
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           if constexpr (MN) {
 #pragma unroll
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
             for (int q = 0; q < BN / BK; ++q)
               tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
             if (i + 1 < a.Nc) {  // the same boxes of the next chunk, into L2
-              const int yn = y + a.Cp;
+              const int yn = a.reverse ? y - a.Cp : y + a.Cp;
 #pragma unroll
               for (int q = 0; q < GEMM_BM / BK; ++q) tma_prefetch_l2_2d(&mapR, m0 + q * BK, yn);
 #pragma unroll
@@ -175,9 +180,12 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     const int c0 = n0 + half * HC;       // first state column of this thread
     const uint32_t laddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * HC;
     const long long dfs = static_cast<long long>(a.d) * a.f;
-    const E* wrow = a.w_down + static_cast<long long>(row) * a.f;
+    const E* wrow = a.w_down ? a.w_down + static_cast<long long>(row) * a.f : nullptr;
+    auto w_index = [&](int j) {  // w_all entry of step j
+      return static_cast<long long>(b) * a.Nc + (a.reverse ? a.Nc - 1 - j : j);
+    };
     float S[HC];
-    // S_0 = state_in (or 0); W_0 = W_down + S_0.
+    // S_0 = state_in (or 0); W_0 = W_down + S_0 (W_down null: 0).
 #pragma unroll
     for (int cc = 0; cc < HC; cc += 32) {
       const int col = c0 + cc;
@@ -192,11 +200,15 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       for (int e = 0; e < 32; ++e) S[cc + e] = s32[e];
       if (row_ok && col < a.f && a.w_all) {
         float w[32];
-        load_x32(wrow + col, w);
+        if (wrow) {
+          load_x32(wrow + col, w);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) w[e] += s32[e];
-        store_x32(a.w_all + (static_cast<long long>(b) * a.Nc) * dfs +
-                      static_cast<long long>(row) * a.f + col, w);
+        store_x32(a.w_all + w_index(0) * dfs + static_cast<long long>(row) * a.f + col, w);
       }
     }
     for (int i = 0; i < a.Nc; ++i) {
@@ -221,11 +233,15 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         float v[32];
         if (!last) {
           if (!a.w_all) continue;
-          load_x32(wrow + col, v);
+          if (wrow) {
+            load_x32(wrow + col, v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0.f;
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] += S[cc + e];
-          store_x32(a.w_all + (static_cast<long long>(b) * a.Nc + i + 1) * dfs +
-                        static_cast<long long>(row) * a.f + col, v);
+          store_x32(a.w_all + w_index(i + 1) * dfs + static_cast<long long>(row) * a.f + col, v);
         } else if (a.state_out) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = S[cc + e];

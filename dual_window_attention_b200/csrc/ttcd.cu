@@ -20,6 +20,8 @@
 #include "ptx.cuh"
 #include "scan.cuh"
 #include "decode.cuh"
+#include "backward.cuh"
+#include "attention_bwd.cuh"
 
 using namespace ttcd;
 
@@ -165,14 +167,15 @@ bool make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
   return make_map<OutT>(m, ptr, cols, rows, ld_elems * sizeof(OutT), 128 / sizeof(OutT), 32);
 }
 
-template <class E, int BN, int STAGES, bool DUAL, class Epi, class Geom = GemmGeom>
+template <class E, int BN, int STAGES, bool DUAL, class Epi, class Geom = GemmGeom,
+          bool B_MN = false>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
                         const CUtensorMap& B1, const CUtensorMap* out_map, const Geom& geo,
                         const Epi& epi, const CUtensorMap* out_map2 = nullptr) {
   const int total = geo.total();
   if (total <= 0) return TTCD_OK;
   if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
-  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom>;
+  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom, B_MN>;
   constexpr int smem = gemm_smem_bytes<BN, STAGES, Epi::kStaged>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -284,10 +287,11 @@ Dims dims_of(const ttcd_block_params* p) {
 // Operand buffers hold bf16 for TTCD_BF16 and fp32 (tf32 tensor-core operands)
 // for TTCD_F32 and the wide route; q, k, v stay bf16 (the attention kernel takes
 // bf16).  The status word comes first in every workspace.
-Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false) {
+Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false,
+                   bool allow_wide = true) {
   const Dims m = dims_of(p);
   size_t sz[B_COUNT] = {0};
-  const bool wide = !shard && wide_mode(p);
+  const bool wide = allow_wide && !shard && wide_mode(p);
   const size_t e = (p->dtype == TTCD_F32 || wide) ? 4 : 2;
   sz[B_STATUS] = kStatusBytes;
   if (block) {
@@ -310,7 +314,7 @@ Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false) {
   sz[B_R] = m.P * m.d * e;
   sz[B_WALL] = static_cast<size_t>(p->B) * m.Nc * m.d * m.f * e;
   sz[B_M] = static_cast<size_t>(m.d) * m.f * e;
-  sz[B_WPROJT] = static_cast<size_t>(m.f) * m.f * e;
+  sz[B_WPROJT] = e == 4 ? static_cast<size_t>(m.f) * m.f * e : 0;  // bf16 reads W_proj MN-major
   if (e == 4) {  // tf32 operands stay K-major: transposed copies for the chunk scan
     sz[B_RT] = m.P * m.d * e;
     sz[B_KT] = m.P * m.f * e;
@@ -524,18 +528,26 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
     }
   }
   stage_mark(c, mark + 2);
-  // M = W_down W_proj (associativity of W_down (W_proj d_t)).
+  // M = W_down W_proj (associativity of W_down (W_proj d_t)).  bf16: W_proj
+  // [K = f, N = f] row-major is read as an MN-major operand; fp32 (tf32
+  // operands stay K-major): through a transposed copy.
   {
-    dim3 tb(32, 8), tg(cdiv(m.f, 32), cdiv(m.f, 32));
-    transpose_kernel<E, E><<<tg, tb, 0, c.s>>>(w_proj, WprojT, m.f, m.f);
-    TTCD_CHECK_LAUNCH();
     CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, w_down, m.d, m.f, 128) || !map_rows<E>(&mB, WprojT, m.f, m.f, 256))
-      return TTCD_ERR_CUDA;
+    if (!map_rows<E>(&mA, w_down, m.d, m.f, 128)) return TTCD_ERR_CUDA;
     CUtensorMap mo;
     if (!make_out_map<E>(&mo, M, m.d, m.f, m.f)) return TTCD_ERR_CUDA;
     EpiStore<E> e{M, m.f, m.f, nullptr};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
+    const GemmGeom g = plain_geom(m.d, cdiv(m.f, 256), m.f);
+    if constexpr (sizeof(E) == 2) {
+      if (!make_map<E>(&mB, w_proj, m.f, m.f, m.f * sizeof(E), 64, 64)) return TTCD_ERR_CUDA;
+      TTCD_TRY((launch_gemm<E, 256, 4, false, EpiStore<E>, GemmGeom, true>(c, mA, mB, mB, &mo, g, e)));
+    } else {
+      dim3 tb(32, 8), tg(cdiv(m.f, 32), cdiv(m.f, 32));
+      transpose_kernel<E, E><<<tg, tb, 0, c.s>>>(w_proj, WprojT, m.f, m.f);
+      TTCD_CHECK_LAUNCH();
+      if (!map_rows<E>(&mB, WprojT, m.f, m.f, 256)) return TTCD_ERR_CUDA;
+      TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
+    }
   }
   stage_mark(c, mark + 3);
   // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
@@ -583,7 +595,7 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
           !make_map<E>(&mK, Kt, m.P, m.f, m.P * sizeof(E), BK, SCAN_BN))
         return TTCD_ERR_CUDA;
     }
-    ScanArgs<E> a;
+    ScanArgs<E> a{};
     a.d = m.d;
     a.f = m.f;
     a.Nc = whole ? 1 : m.Nc;
@@ -1412,7 +1424,7 @@ ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, co
   if (!make_map<bf>(&mR, dat<bf>(state, L.rc), d, static_cast<uint64_t>(p->B) * Cp, d * 2, BK, BK) ||
       !make_map<bf>(&mK, dat<bf>(state, L.kx), f, static_cast<uint64_t>(p->B) * Cp, f * 2, BK, BK))
     return TTCD_ERR_CUDA;
-  ScanArgs<bf> a;
+  ScanArgs<bf> a{};
   a.d = d;
   a.f = f;
   a.Nc = 1;
@@ -1698,6 +1710,473 @@ ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void*
       return TTCD_ERR_CUDA;
   }
   return dec_commit(c, p, state, S, nullptr, dat<float>(state, S.S), state_out);
+}
+
+}  // extern "C"
+
+// ================================================================== MLP backward
+// The chain rule of the fast-weight MLP (backward.cuh has the formulas), bf16
+// operands and fp32 accumulation: the forward's front half and chunk scan are
+// recomputed into the forward workspace, then
+//   dZ_S (read)  = dy (W_down + S_i)                  chunk-grouped GEMM
+//   G_i, dS_in   = reverse prefix of dy_C^T Z_S,C    chunk scan walked backwards
+//   dRt, s dRt   = Zbar_S G_i^T                       chunk-grouped GEMM
+//   E, dD, ds    = dRt M                              GEMM (M read MN-major)
+//   dbeta, coef  = from ds and the key norms
+//   dZbar_S      = (s r) G_i + coef Zbar_S - dD       chunk-grouped GEMM
+//   dM           = sum_t s dRt_t D_t^T;  dW_down, dW_proj from dM
+//   dZ_P         = conv_P^T dZbar_P (+ dZ_S read);  tap gradients
+//   da, db, Z    = gate/up recomputed with dZ          GEMM
+//   du_P         = [da | db] [W_gate; W_up]            GEMM (MN-major)
+//   dW_gate, dW_up = sum_rows da^T u, db^T u           token contractions
+namespace {
+
+struct BwdLayout {
+  Layout F;  // the forward MLP's workspace (bf16 operands), first
+  size_t dyp, zsp, dzsy, drt, dr, dd, epart, coef, dzbs, dm, dm16, dwd, dz, dab, zall, wgu,
+      tpart, dsi, total;
+};
+
+BwdLayout bwd_layout(const ttcd_block_params* p) {
+  const Dims m = dims_of(p);
+  BwdLayout L;
+  L.F = make_layout(p, false, false, false);
+  const size_t n_epart = static_cast<size_t>(cdiv(m.f, 256));
+  const size_t sz[18] = {
+      static_cast<size_t>(m.P) * m.d * 2,                                    // dy, chunk-padded
+      static_cast<size_t>(m.P) * m.f * 2,                                    // Z_S, chunk-padded
+      static_cast<size_t>(m.BT) * m.f * 4,                                   // dZ_S of the read
+      static_cast<size_t>(m.P) * m.d * 2,                                    // dRt
+      static_cast<size_t>(m.P) * m.d * 2,                                    // s dRt
+      static_cast<size_t>(m.P) * m.f * 4,                                    // dD
+      n_epart * m.P * 4,                                                     // ds partials
+      static_cast<size_t>(m.P) * 4,                                          // coef
+      static_cast<size_t>(m.P) * m.f * 4,                                    // dZbar_S
+      static_cast<size_t>(m.d) * m.f * 4,                                    // dM
+      static_cast<size_t>(m.d) * m.f * 2,                                    // dM bf16
+      static_cast<size_t>(m.d) * m.f * 4,                                    // dM W_proj^T
+      2 * static_cast<size_t>(m.BT) * m.f * 4,                               // dZ
+      2 * static_cast<size_t>(m.BT) * 2 * m.f * 2,                           // [da | db]
+      2 * static_cast<size_t>(m.BT) * m.f * 2,                               // Z (recomputed)
+      2 * static_cast<size_t>(m.f) * m.d * 2,                                // [W_gate; W_up]
+      static_cast<size_t>(TAP_SPLITS) * 2 * m.f * p->conv_k * 4,             // tap partials
+      static_cast<size_t>(p->B) * m.d * m.f * 4};                            // dL/dstate_in
+  size_t* f[18] = {&L.dyp, &L.zsp, &L.dzsy, &L.drt, &L.dr, &L.dd, &L.epart, &L.coef, &L.dzbs,
+                   &L.dm, &L.dm16, &L.dwd, &L.dz, &L.dab, &L.zall, &L.wgu, &L.tpart, &L.dsi};
+  size_t off = L.F.total;
+  for (int i = 0; i < 18; ++i) {
+    *f[i] = off;
+    off += (sz[i] + 1023) / 1024 * 1024;
+  }
+  L.total = off;
+  return L;
+}
+
+ttcd_status check_bwd_params(const ttcd_block_params* p) {
+  TTCD_TRY(check_params(p));
+  if (p->dtype != TTCD_BF16) return TTCD_ERR_UNSUPPORTED;
+  const Dims m = dims_of(p);
+  if (2 * m.BT * 2 * m.f >= (1ll << 40) || m.P * static_cast<long long>(m.f) >= (1ll << 40))
+    return TTCD_ERR_UNSUPPORTED;
+  return TTCD_OK;
+}
+
+// Token contraction out[i, j] = sum_r A[r, i] B[r, j] (A [rows, m_dim] and B
+// [rows, n_dim] token-major bf16, row pitches lda / ldb elements), fp32 out
+// [m_dim, n_dim]: the chunk-scan kernel with one chunk of all rows.
+ttcd_status launch_tsum(const Ctx& c, const __nv_bfloat16* A, long long lda, int m_dim,
+                        const __nv_bfloat16* Bm, long long ldb, int n_dim, long long rows,
+                        float* out) {
+  using bf = __nv_bfloat16;
+  CUtensorMap mA, mB;
+  if (!make_map<bf>(&mA, A, m_dim, rows, lda * 2, 64, 64) ||
+      !make_map<bf>(&mB, Bm, n_dim, rows, ldb * 2, 64, 64))
+    return TTCD_ERR_CUDA;
+  ScanArgs<bf> a{};
+  a.d = m_dim;
+  a.f = n_dim;
+  a.Nc = 1;
+  a.Cp = static_cast<int>((rows + 63) / 64 * 64);
+  a.state_out = out;
+  a.tiles_m = cdiv(m_dim, 128);
+  a.tiles_n = cdiv(n_dim, SCAN_BN);
+  a.commit_C = 1;
+  constexpr int STAGES = 4;
+  constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+  auto kern = fastweight_scan_kernel<bf, STAGES, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), SCAN_THREADS, kScanRegSplit));
+  kern<<<a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mA, mB, a, c.st);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+// Chunk-grouped geometry over the chunk-padded rows (every chunk Cp rows).
+GemmGeom padded_chunk_geom(const ttcd_block_params* p, const Dims& m, int K, int tiles_n) {
+  GemmGeom g;
+  g.n_seq = p->B;
+  g.T = m.Nc * m.Cp;
+  g.C = m.Cp;
+  g.Nc = m.Nc;
+  g.K = K;
+  g.tiles_m = cdiv(m.Cp, 128);
+  g.tiles_n = tiles_n;
+  g.b_group_rows = m.d;
+  return g;
+}
+
+ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv_bfloat16* u_S,
+                              const float* beta, const ttcd_block_weights* w,
+                              const ttcd_block_params* p, const float* state_in,
+                              const __nv_bfloat16* d_y, const float* d_state_out, float* du_T,
+                              float* du_S, float* d_beta, float* d_state_in,
+                              const ttcd_mlp_grads* g, void* ws, const BwdLayout& L) {
+  using bf = __nv_bfloat16;
+  const Dims m = dims_of(p);
+  const Layout& F = L.F;
+  const bf* w_gate = static_cast<const bf*>(w->w_gate);
+  const bf* w_up = static_cast<const bf*>(w->w_up);
+  const bf* w_down = static_cast<const bf*>(w->w_down);
+  const bf* w_proj = static_cast<const bf*>(w->w_proj);
+  bf* U = at<bf>(ws, F, B_U);
+  bf* Zs = at<bf>(ws, F, B_ZS16);
+  bf* D = at<bf>(ws, F, B_D);
+  bf* Kp = at<bf>(ws, F, B_KP);
+  float* ssq = at<float>(ws, F, B_SSQ);
+  float* kscale = at<float>(ws, F, B_KSCALE);
+  bf* R = at<bf>(ws, F, B_R);
+  bf* Wall = at<bf>(ws, F, B_WALL);  // W_down + S_i, then G_i
+  bf* M = at<bf>(ws, F, B_M);
+  bf* dyp = dat<bf>(ws, L.dyp);
+  bf* zsp = dat<bf>(ws, L.zsp);
+  float* dzsy = dat<float>(ws, L.dzsy);
+  bf* drt = dat<bf>(ws, L.drt);
+  bf* dr = dat<bf>(ws, L.dr);
+  float* dD = dat<float>(ws, L.dd);
+  float* epart = dat<float>(ws, L.epart);
+  float* coef = dat<float>(ws, L.coef);
+  float* dzbs = dat<float>(ws, L.dzbs);
+  float* dM = dat<float>(ws, L.dm);
+  bf* dM16 = dat<bf>(ws, L.dm16);
+  float* dwd = dat<float>(ws, L.dwd);
+  float* dZ = dat<float>(ws, L.dz);
+  bf* dab = dat<bf>(ws, L.dab);
+  bf* zall = dat<bf>(ws, L.zall);
+  bf* wgu = dat<bf>(ws, L.wgu);
+  float* tpart = dat<float>(ws, L.tpart);
+  float* dsi = d_state_in ? d_state_in : dat<float>(ws, L.dsi);
+  const long long n_u = m.BT * m.d;
+
+  // forward front half and chunk scan, recomputed
+  if (cudaMemcpyAsync(U, u_T, n_u * 2, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
+      cudaMemcpyAsync(U + n_u, u_S, n_u * 2, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  TTCD_TRY(mlp_front<bf>(c, p, F, ws, w_gate, w_up, w_down, w_proj,
+                         static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S),
+                         beta, 0, nullptr, nullptr));
+  TTCD_TRY(launch_scan<bf>(c, p, F, ws, w_down, state_in, nullptr, Wall, false));
+
+  // dZ_S of the read: dy (W_down + S_i), W_i [d, f] read MN-major per chunk
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, d_y, m.BT, m.d, 128) ||
+        !make_map<bf>(&mB, Wall, m.f, static_cast<uint64_t>(p->B) * m.Nc * m.d, m.f * 2, 64, 64) ||
+        !make_out_map<float>(&mo, dzsy, m.BT, m.f, m.f))
+      return TTCD_ERR_CUDA;
+    GemmGeom gg;
+    gg.n_seq = p->B;
+    gg.T = p->T;
+    gg.C = p->chunk;
+    gg.Nc = m.Nc;
+    gg.K = m.d;
+    gg.tiles_m = cdiv(p->chunk, 128);
+    gg.tiles_n = cdiv(m.f, 256);
+    gg.b_group_rows = m.d;
+    EpiStore<float> e{dzsy, m.f, m.f, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(c, mA, mB, mB, &mo, gg, e)));
+  }
+  // G_i and dL/dstate_in: the scan walked backwards over dy_C^T Z_S,C
+  {
+    const long long nd = m.P * (m.d / 8), nf = m.P * (m.f / 8);
+    chunk_pad_rows_kernel<bf><<<static_cast<unsigned>(cdiv(nd, 256)), 256, 0, c.s>>>(
+        d_y, dyp, m.d, p->T, p->chunk, m.Cp, m.Nc, m.P);
+    TTCD_CHECK_LAUNCH();
+    chunk_pad_rows_kernel<bf><<<static_cast<unsigned>(cdiv(nf, 256)), 256, 0, c.s>>>(
+        Zs, zsp, m.f, p->T, p->chunk, m.Cp, m.Nc, m.P);
+    TTCD_CHECK_LAUNCH();
+    CUtensorMap mA, mB;
+    if (!make_map<bf>(&mA, dyp, m.d, m.P, m.d * 2, 64, 64) ||
+        !make_map<bf>(&mB, zsp, m.f, m.P, m.f * 2, 64, 64))
+      return TTCD_ERR_CUDA;
+    ScanArgs<bf> a{};
+    a.d = m.d;
+    a.f = m.f;
+    a.Nc = m.Nc;
+    a.Cp = m.Cp;
+    a.w_down = nullptr;
+    a.state_in = d_state_out;
+    a.state_out = dsi;
+    a.w_all = Wall;
+    a.tiles_m = cdiv(m.d, 128);
+    a.tiles_n = cdiv(m.f, SCAN_BN);
+    a.commit_C = 1;
+    a.reverse = true;
+    constexpr int STAGES = 4;
+    constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+    auto kern = fastweight_scan_kernel<bf, STAGES, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+    TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), SCAN_THREADS, kScanRegSplit));
+    kern<<<p->B * a.tiles_m * a.tiles_n, SCAN_THREADS, smem, c.s>>>(mA, mB, a, c.st);
+    TTCD_CHECK_LAUNCH();
+  }
+  // dRt = Zbar_S G_i^T and s dRt
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<bf>(&mA, Kp, m.P, m.f, 128) ||
+        !map_rows<bf>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 256))
+      return TTCD_ERR_CUDA;
+    EpiStoreScaledPair e{drt, dr, m.d, m.d, kscale};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, nullptr,
+                                             padded_chunk_geom(p, m, m.f, cdiv(m.d, 256)), e)));
+  }
+  // E = dRt M: dD = s E and the partial dots D . E
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<bf>(&mA, drt, m.P, m.d, 128) ||
+        !make_map<bf>(&mB, M, m.f, m.d, m.f * 2, 64, 64))
+      return TTCD_ERR_CUDA;
+    EpiBwdE e{dD, D, epart, m.P, m.f, kscale};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiBwdE, GemmGeom, true>(
+        c, mA, mB, mB, nullptr, plain_geom(m.P, cdiv(m.f, 256), m.d), e)));
+  }
+  key_backward_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(epart, cdiv(m.f, 256), ssq,
+                                                       cdiv(m.f, 128), beta, d_beta, coef, p->T,
+                                                       p->chunk, m.Cp, m.Nc, m.P, p->l2_eps);
+  TTCD_CHECK_LAUNCH();
+  // dZbar_S = (s r) G_i + coef Zbar_S - dD
+  {
+    CUtensorMap mA, mB;
+    if (!map_rows<bf>(&mA, R, m.P, m.d, 128) ||
+        !make_map<bf>(&mB, Wall, m.f, static_cast<uint64_t>(p->B) * m.Nc * m.d, m.f * 2, 64, 64))
+      return TTCD_ERR_CUDA;
+    EpiBwdZbS e{dzbs, Kp, dD, m.f, coef};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiBwdZbS, GemmGeom, true>(
+        c, mA, mB, mB, nullptr, padded_chunk_geom(p, m, m.d, cdiv(m.f, 256)), e)));
+  }
+  // dM = sum_t (s dRt)_t D_t^T;  dW_proj = W_down^T dM;  dW_down = dM W_proj^T + the read's
+  TTCD_TRY(launch_tsum(c, dr, m.d, m.d, D, m.f, m.f, m.P, dM));
+  TTCD_TRY((launch_cast<float, bf>(c, dM, dM16, static_cast<long long>(m.d) * m.f)));
+  TTCD_TRY(launch_tsum(c, w_down, m.f, m.f, dM16, m.f, m.f, m.d, g->w_proj));
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dM16, m.d, m.f, 128) || !map_rows<bf>(&mB, w_proj, m.f, m.f, 256) ||
+        !make_out_map<float>(&mo, dwd, m.d, m.f, m.f))
+      return TTCD_ERR_CUDA;
+    EpiStore<float> e{dwd, m.f, m.f, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.d, cdiv(m.f, 256), m.f), e)));
+  }
+  {
+    const long long n = static_cast<long long>(m.d) * m.f;
+    dw_down_combine_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+        dwd, dsi, d_state_out, g->w_down, p->B, n);
+    TTCD_CHECK_LAUNCH();
+  }
+  // dZ_P through the convs (teacher: dZbar_T = dD), plus the read's dZ_S
+  {
+    const long long n = 2 * m.BT * (m.f / 4);
+    conv_backward_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+        dD, dzbs, dzsy, static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), dZ,
+        p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
+    TTCD_CHECK_LAUNCH();
+  }
+  // gate/up recomputed: [da | db] and Z
+  {
+    CUtensorMap mA, mB0, mB1;
+    if (!map_rows<bf>(&mA, U, 2 * m.BT, m.d, 128) || !map_rows<bf>(&mB0, w_gate, m.f, m.d, 128) ||
+        !map_rows<bf>(&mB1, w_up, m.f, m.d, 128))
+      return TTCD_ERR_CUDA;
+    EpiSwiGLUBwd e{dZ, dab, zall, m.f};
+    TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, nullptr,
+                                            plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
+  }
+  // tap gradients
+  {
+    dim3 grid(m.f / 32, TAP_SPLITS, 2);
+    if (p->conv_k <= 4)
+      conv_tap_grad_kernel<4><<<grid, 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T, m.f,
+                                                     p->conv_k, p->chunk, m.Cp, m.Nc);
+    else
+      conv_tap_grad_kernel<8><<<grid, 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T, m.f,
+                                                     p->conv_k, p->chunk, m.Cp, m.Nc);
+    TTCD_CHECK_LAUNCH();
+    conv_tap_reduce_kernel<<<cdiv(2 * m.f * p->conv_k, 256), 256, 0, c.s>>>(
+        tpart, g->conv_T, g->conv_S, m.f, p->conv_k);
+    TTCD_CHECK_LAUNCH();
+  }
+  // du_P = [da | db] [W_gate; W_up]
+  {
+    const size_t wbytes = static_cast<size_t>(m.f) * m.d * 2;
+    if (cudaMemcpyAsync(wgu, w_gate, wbytes, cudaMemcpyDeviceToDevice, c.s) != cudaSuccess ||
+        cudaMemcpyAsync(wgu + static_cast<size_t>(m.f) * m.d, w_up, wbytes,
+                        cudaMemcpyDeviceToDevice, c.s) != cudaSuccess)
+      return TTCD_ERR_CUDA;
+    CUtensorMap mB;
+    if (!make_map<bf>(&mB, wgu, m.d, 2 * m.f, m.d * 2, 64, 64)) return TTCD_ERR_CUDA;
+    float* du[2] = {du_T, du_S};
+    for (int path = 0; path < 2; ++path) {
+      CUtensorMap mA, mo;
+      if (!map_rows<bf>(&mA, dab + path * m.BT * 2 * m.f, m.BT, 2 * m.f, 128) ||
+          !make_out_map<float>(&mo, du[path], m.BT, m.d, m.d))
+        return TTCD_ERR_CUDA;
+      EpiStore<float> e{du[path], m.d, m.d, nullptr};
+      TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(
+          c, mA, mB, mB, &mo, plain_geom(m.BT, cdiv(m.d, 256), 2 * m.f), e)));
+    }
+  }
+  // dW_gate = sum_rows da^T u, dW_up = sum_rows db^T u (both paths)
+  TTCD_TRY(launch_tsum(c, dab, 2 * m.f, m.f, U, m.d, m.d, 2 * m.BT, g->w_gate));
+  TTCD_TRY(launch_tsum(c, dab + m.f, 2 * m.f, m.f, U, m.d, m.d, 2 * m.BT, g->w_up));
+  return TTCD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttcd_fastweight_mlp_backward_workspace_size(const ttcd_block_params* p) {
+  if (check_bwd_params(p) != TTCD_OK) return 0;
+  return bwd_layout(p).total;
+}
+
+ttcd_status ttcd_fastweight_mlp_backward(const void* u_T, const void* u_S, const float* beta,
+                                         const ttcd_block_weights* w, const ttcd_block_params* p,
+                                         const float* state_in, const void* d_y,
+                                         const float* d_state_out, float* du_T, float* du_S,
+                                         float* d_beta, float* d_state_in,
+                                         const ttcd_mlp_grads* grads, void* workspace,
+                                         size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_bwd_params(p));
+  if (!aligned16(u_T) || !aligned16(u_S) || !aligned16(beta) || !aligned16(d_y) ||
+      !aligned16(du_T) || !aligned16(du_S) || !aligned16(d_beta) || !weights_ok(w, false) ||
+      !aligned16(workspace) || !grads)
+    return TTCD_ERR_INVALID_ARG;
+  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
+      (d_state_in && !aligned16(d_state_in)))
+    return TTCD_ERR_INVALID_ARG;
+  const float* gp[6] = {grads->w_gate, grads->w_up,   grads->w_down,
+                        grads->w_proj, grads->conv_T, grads->conv_S};
+  for (const float* q : gp)
+    if (!aligned16(q)) return TTCD_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(p);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, workspace));
+  using bf = __nv_bfloat16;
+  return mlp_backward_bf16(c, static_cast<const bf*>(u_T), static_cast<const bf*>(u_S), beta, w,
+                           p, state_in, static_cast<const bf*>(d_y), d_state_out, du_T, du_S,
+                           d_beta, d_state_in, grads, workspace, L);
+}
+
+}  // extern "C"
+
+// ================================================================== attention backward
+namespace {
+
+size_t attn_bwd_ws_bytes(int B, int T, int Hq) {
+  const size_t rows = static_cast<size_t>(B) * Hq * T * 4;
+  return kStatusBytes + 2 * ((rows + 1023) / 1024 * 1024);
+}
+
+template <int HD>
+ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const void* v,
+                            const void* o_T, const void* o_S, const float* lse_T,
+                            const float* lse_S, const void* do_T, const void* do_S, float* dq,
+                            float* dk, float* dv, int B, int T, int Hq, int Hkv, int w_S,
+                            int w_T, float scale, void* ws) {
+  using bf = __nv_bfloat16;
+  const long long BT = static_cast<long long>(B) * T;
+  const size_t rows_bytes = (static_cast<size_t>(B) * Hq * T * 4 + 1023) / 1024 * 1024;
+  float* delta_T = dat<float>(ws, kStatusBytes);
+  float* delta_S = dat<float>(ws, kStatusBytes + rows_bytes);
+  // dq is accumulated over the key tiles
+  if (cudaMemsetAsync(dq, 0, static_cast<size_t>(BT) * Hq * HD * 4, c.s) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  const long long rows = BT * Hq;
+  attn_bwd_delta_kernel<HD><<<static_cast<unsigned>(cdiv(2 * rows, 256)), 256, 0, c.s>>>(
+      static_cast<const bf*>(o_T), static_cast<const bf*>(o_S), static_cast<const bf*>(do_T),
+      static_cast<const bf*>(do_S), delta_T, delta_S, T, Hq, rows);
+  TTCD_CHECK_LAUNCH();
+  CUtensorMap mq, mk, mv, mdt, mds;
+  const uint64_t wq = static_cast<uint64_t>(Hq) * HD, wkv = static_cast<uint64_t>(Hkv) * HD;
+  if (!make_map<bf>(&mq, q, wq, BT, wq * 2, 64, 128) || !make_map<bf>(&mk, k, wkv, BT, wkv * 2, 64, 128) ||
+      !make_map<bf>(&mv, v, wkv, BT, wkv * 2, 64, 128) ||
+      !make_map<bf>(&mdt, do_T, wq, BT, wq * 2, 64, 128) ||
+      !make_map<bf>(&mds, do_S, wq, BT, wq * 2, 64, 128))
+    return TTCD_ERR_CUDA;
+  AttnBwdArgs a;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.lse_T = lse_T;
+  a.lse_S = lse_S;
+  a.delta_T = delta_T;
+  a.delta_S = delta_S;
+  a.B = B;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.w_S = w_S;
+  a.w_T = w_T;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_kt = cdiv(T, ATT_BN);
+  auto kern = dual_window_attn_bwd_kernel<HD>;
+  constexpr int smem = AttnBwdCfg<HD>::SMEM;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  const long long grid = static_cast<long long>(a.n_kt) * B * Hkv;
+  if (grid >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
+  TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), ATTB_THREADS, kAttnRegSplit));
+  kern<<<static_cast<unsigned>(grid), ATTB_THREADS, smem, c.s>>>(mq, mk, mv, mdt, mds, a, c.st);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttcd_dual_window_attn_backward_workspace_size(int B, int T, int Hq) {
+  if (B < 1 || T < 1 || Hq < 1) return 0;
+  return attn_bwd_ws_bytes(B, T, Hq);
+}
+
+ttcd_status ttcd_dual_window_attn_backward(const void* q, const void* k, const void* v,
+                                           const void* o_T, const void* o_S, const float* lse_T,
+                                           const float* lse_S, const void* do_T,
+                                           const void* do_S, float* dq, float* dk, float* dv,
+                                           int B, int T, int Hq, int Hkv, int hd, int w_S,
+                                           int w_T, float scale, void* workspace,
+                                           size_t ws_bytes, void* stream) {
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || w_S < 1 || w_T < w_S ||
+      !(scale >= 0.f))
+    return TTCD_ERR_INVALID_ARG;
+  const void* need[] = {q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, dq, dk, dv, workspace};
+  for (const void* x : need)
+    if (!aligned16(x)) return TTCD_ERR_INVALID_ARG;
+  if (hd != 64 && hd != 128) return TTCD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * T * Hq >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
+  if (ws_bytes < attn_bwd_ws_bytes(B, T, Hq)) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, workspace));
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(hd));
+  if (hd == 64)
+    return launch_attn_bwd<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, dq, dk, dv, B, T,
+                               Hq, Hkv, w_S, w_T, sc, workspace);
+  return launch_attn_bwd<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, dq, dk, dv, B, T,
+                              Hq, Hkv, w_S, w_T, sc, workspace);
 }
 
 }  // extern "C"

@@ -151,6 +151,43 @@ ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* 
                                       int w_S, int w_T, float scale, ttcd_dtype dtype,
                                       void* stream);
 
+/* Workspace bytes of ttcd_dual_window_attn_backward (status word and the two
+ * [B, Hq, T] fp32 row dot products); 0 for invalid sizes. */
+size_t ttcd_dual_window_attn_backward_workspace_size(int B, int T, int Hq);
+
+/*
+ * ttcd_dual_window_attn_backward — vector-Jacobian product of ttcd_dual_window_attn.
+ *
+ * For a scalar loss L with dL/do_T = do_T and dL/do_S = do_S, the gradients
+ * with respect to q, k and v, both windows together ([REVIEW] 局限与展望:
+ * training differentiates both attention windows; each window is the softmax
+ * attention of ttcd_dual_window_attn):
+ *   per window P: dV += P^T dO_P,  dS = P (dO_P V^T - rowsum(dO_P o_P)) scale,
+ *                 dK += dS^T Q,  dQ += dS K   (query heads of a group add into
+ *                 their KV head).
+ * P is rebuilt from the forward's log-sum-exp, so the call takes the forward's
+ * o_T, o_S, lse_T and lse_S (from ttcd_dual_window_attn with both lse outputs).
+ *   q, k, v        [B, T, H, hd] bf16, device (as the forward)
+ *   o_T, o_S       [B, T, Hq, hd] bf16, device (the forward's outputs)
+ *   lse_T, lse_S   [B, Hq, T] fp32, device (the forward's log-sum-exps)
+ *   do_T, do_S     [B, T, Hq, hd] bf16, device
+ *   dq             [B, T, Hq, hd] fp32, device, written
+ *   dk, dv         [B, T, Hkv, hd] fp32, device, written
+ *   hd             64 or 128 (32: TTCD_ERR_UNSUPPORTED)
+ *   workspace      >= ttcd_dual_window_attn_backward_workspace_size(B, T, Hq) bytes,
+ *                  device, 16-byte aligned; status word first
+ * Precision: bf16 tensor-core operands (q, k, v, dO and the rebuilt P and dS
+ * rounded to bf16), fp32 accumulation; dq sums the key tiles' contributions
+ * with fp32 atomic adds, so its low bits depend on their order.
+ */
+ttcd_status ttcd_dual_window_attn_backward(const void* q, const void* k, const void* v,
+                                           const void* o_T, const void* o_S, const float* lse_T,
+                                           const float* lse_S, const void* do_T,
+                                           const void* do_S, float* dq, float* dk, float* dv,
+                                           int B, int T, int Hq, int Hkv, int hd, int w_S,
+                                           int w_T, float scale, void* workspace,
+                                           size_t ws_bytes, void* stream);
+
 /*
  * ttcd_fastweight_mlp — the in-place fast-weight MLP of one block (off-policy).
  *
@@ -181,6 +218,51 @@ ttcd_status ttcd_fastweight_mlp(const void* u_T, const void* u_S, const void* h_
                                 const ttcd_block_params* p, const float* state_in,
                                 float* state_out, void* y, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/* fp32 gradients of the fast-weight MLP's weights (device, written, not accumulated). */
+typedef struct {
+  float* w_gate; /* [d_ff, d_model] */
+  float* w_up;   /* [d_ff, d_model] */
+  float* w_down; /* [d_model, d_ff] */
+  float* w_proj; /* [d_ff, d_ff] */
+  float* conv_T; /* [d_ff, conv_k] */
+  float* conv_S; /* [d_ff, conv_k] */
+} ttcd_mlp_grads;
+
+/* Workspace bytes of ttcd_fastweight_mlp_backward; 0 when p is invalid or not TTCD_BF16. */
+size_t ttcd_fastweight_mlp_backward_workspace_size(const ttcd_block_params* p);
+
+/*
+ * ttcd_fastweight_mlp_backward — vector-Jacobian product of ttcd_fastweight_mlp.
+ *
+ * For a scalar loss L with dL/dy = d_y and dL/dstate_out = d_state_out, the
+ * gradients of L with respect to u_T, u_S, beta, state_in and the six MLP
+ * weights, by the chain rule of the steps listed at ttcd_fastweight_mlp taken in
+ * reverse ([REVIEW] 关键设计 2-3; the write path is differentiated too: W_proj,
+ * the two convs and beta reach the loss only through the fast-weight writes;
+ * [REVIEW] 局限与展望 on training cost).  The forward's intermediates are
+ * recomputed in the workspace, so the call takes the forward's inputs.
+ *   u_T, u_S, beta, w, p, state_in: as ttcd_fastweight_mlp (TTCD_BF16 only)
+ *   d_y          [B, T, d] bf16, device
+ *   d_state_out  [B, d, f] fp32, device, nullable (zero)
+ *   du_T, du_S   [B, T, d] fp32, device, written
+ *   d_beta       [B, T] fp32, device, written
+ *   d_state_in   [B, d, f] fp32, device, nullable, written
+ *   grads        the weight gradients (all six pointers required)
+ *   workspace    >= ttcd_fastweight_mlp_backward_workspace_size(p) bytes, device,
+ *                16-byte aligned; status word first, as for the forward
+ * Precision: bf16 GEMM operands (u, dy, Z_S, the per-chunk G_i and W_i, the
+ * row gradients dRt, s dRt and [da | db], dM), fp32 accumulation, fp32
+ * element-wise steps and outputs.
+ * Errors: TTCD_ERR_UNSUPPORTED for TTCD_F32; otherwise as ttcd_fastweight_mlp.
+ */
+ttcd_status ttcd_fastweight_mlp_backward(const void* u_T, const void* u_S, const float* beta,
+                                         const ttcd_block_weights* w, const ttcd_block_params* p,
+                                         const float* state_in, const void* d_y,
+                                         const float* d_state_out, float* du_T, float* du_S,
+                                         float* d_beta, float* d_state_in,
+                                         const ttcd_mlp_grads* grads, void* workspace,
+                                         size_t ws_bytes, void* stream);
 
 /*
  * ttcd_block_forward — forward pass of one IP-TTCD block (student path output).
