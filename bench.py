@@ -75,6 +75,38 @@ def recorded_traffic(kernel: str, T: int):
         return None
 
 
+def record_traffic(csv_path: str, kernel: str, T: int, sources, workload: str, command: str,
+                   algorithmic: float, note: str = "") -> dict:
+    """Writes the DRAM bytes of one ncu capture (a --csv log of
+    gpu__time_duration.sum, dram__bytes_read.sum and dram__bytes_write.sum for
+    one launch) into profiles/ncu_traffic.json under `kernel`, with the digest of
+    the kernel's sources at the time of the capture."""
+    import csv
+    vals = {}
+    with open(csv_path) as f:
+        lines = [l for l in f if l.startswith('"')]
+    for row in csv.DictReader(lines):
+        vals[row["Metric Name"]] = float(row["Metric Value"].replace(",", ""))
+    rec = {"workload": workload, "T": T,
+           "dram_bytes_read": int(vals["dram__bytes_read.sum"]),
+           "dram_bytes_write": int(vals["dram__bytes_write.sum"]),
+           "bytes_per_launch": int(vals["dram__bytes_read.sum"] + vals["dram__bytes_write.sum"]),
+           "algorithmic_bytes": int(algorithmic),
+           "gpu_time_duration_ns_under_ncu": int(vals.get("gpu__time_duration.sum", 0)),
+           "sources": list(sources), "sources_sha256_16": sources_digest(sources),
+           "command": command, "note": note}
+    try:
+        with open(TRAFFIC_JSON) as f:
+            table = json.load(f)
+    except OSError:
+        table = {}
+    table[kernel] = rec
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(table, f, indent=1)
+        f.write("\n")
+    return rec
+
+
 ATTN_SWEEP_PAIRS = [(wS, wT) for wT in ATTN_SWEEP_W_T for wS in ATTN_SWEEP_W_S]
 
 
@@ -763,7 +795,20 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=5,
                     help="timed calls per attention window pair / stack shape")
     ap.add_argument("--extra-warmup", type=int, default=3)
+    ap.add_argument("--record-traffic", metavar="CSV", default=None,
+                    help="write the DRAM bytes of an ncu capture of the attention kernel at "
+                         "--T into profiles/ncu_traffic.json (no GPU work)")
+    ap.add_argument("--record-command", default="", help="with --record-traffic: the capture's command")
     args = ap.parse_args()
+    if args.record_traffic:
+        shape = QWEN3_0P6B_64K.with_(T=args.T)
+        rec = record_traffic(args.record_traffic, "dual_window_attn_kernel<128>", args.T,
+                             ["attention.cuh", "gemm.cuh", "ptx.cuh"],
+                             f"Qwen3-0.6B head layout, B 1, T {args.T}, 16/8 heads, hd 128, "
+                             "w_S 512, w_T 8192", args.record_command, attention_bytes(shape),
+                             "one launch at the full workload (one-pass metrics)")
+        print(json.dumps(rec))
+        return
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

@@ -49,6 +49,10 @@ class _Weights(ctypes.Structure):
 WEIGHT_NAMES = tuple(n for n, _ in _Weights._fields_)
 
 
+class _BlockGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
+
+
 class _MlpGrads(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_gate", "w_up", "w_down", "w_proj", "conv_T",
                                                "conv_S")]
@@ -109,6 +113,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_dual_window_attn_backward_workspace_size.argtypes = [i, i, i]
     lib.ttcd_dual_window_attn_backward_workspace_size.restype = sz
     lib.ttcd_dual_window_attn_backward.argtypes = [vp] * 12 + [i] * 7 + [f, vp, sz, vp]
+    lib.ttcd_block_backward_workspace_size.argtypes = [P]
+    lib.ttcd_block_backward_workspace_size.restype = sz
+    lib.ttcd_block_backward.argtypes = [vp, vp, W, P, vp, vp, vp, vp, vp, vp,
+                                        ctypes.POINTER(_BlockGrads), vp, sz, vp]
     lib.ttcd_fastweight_mlp_backward_workspace_size.argtypes = [P]
     lib.ttcd_fastweight_mlp_backward_workspace_size.restype = sz
     lib.ttcd_fastweight_mlp_backward.argtypes = [vp, vp, vp, W, P, vp, vp, vp, vp, vp, vp, vp,
@@ -122,7 +130,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
                "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read",
                "ttcd_block_decode_next", "ttcd_fastweight_mlp_backward",
-               "ttcd_dual_window_attn_backward",
+               "ttcd_dual_window_attn_backward", "ttcd_block_backward",
                "ttcd_shard_qkv", "ttcd_shard_attend", "ttcd_shard_mix", "ttcd_shard_finish"):
         getattr(lib, fn).restype = i
     _lib = lib
@@ -554,6 +562,36 @@ def fastweight_mlp(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockPar
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "ttcd_fastweight_mlp")
     return y, st_t, workspace
+
+
+def block_backward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, d_out,
+                   state_in=None, d_state_out=None, workspace: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Vector-Jacobian product of ``block_forward`` (bf16, hd 64 or 128): the
+    gradients of a loss with dL/dout = d_out and dL/dstate_out = d_state_out (or
+    zero) with respect to x, beta, state_in and the ten weights, all fp32.
+    Returns (grads dict keyed "x", "beta", "state_in" and the weight names;
+    workspace)."""
+    lib = load_library()
+    need = int(lib.ttcd_block_backward_workspace_size(ctypes.byref(p.c())))
+    if need == 0:
+        raise TTCDError(ERR_UNSUPPORTED, "ttcd_block_backward_workspace_size")
+    dev = x.device
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = {"x": torch.empty(p.B, p.T, p.d_model, **f32), "beta": torch.empty(p.B, p.T, **f32),
+         "state_in": torch.empty(p.B, p.d_model, p.d_ff, **f32)}
+    for n in WEIGHT_NAMES:
+        g[n] = torch.empty(weights[n].shape, **f32)
+    gc = _BlockGrads(*[_ptr(g[n]) for n in WEIGHT_NAMES])
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_block_backward(_ptr(x), _ptr(beta), ctypes.byref(wc), ctypes.byref(pc),
+                                 _ptr(state_in), _ptr(d_out), _ptr(d_state_out), _ptr(g["x"]),
+                                 _ptr(g["beta"]), _ptr(g["state_in"]), ctypes.byref(gc),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ttcd_block_backward")
+    return g, workspace
 
 
 def fastweight_mlp_backward(u_T, u_S, beta, weights: Dict[str, torch.Tensor], p: BlockParams,

@@ -17,6 +17,7 @@
 // Rows of the chunk-padded buffers follow the forward's layout: sequence b,
 // chunk i, row j at (b Nc + i) Cp + j, pad rows zero.
 #pragma once
+#include "elementwise.cuh"
 #include "gemm.cuh"
 
 namespace ttcd {
@@ -323,6 +324,176 @@ __global__ void dw_down_combine_kernel(const float* __restrict__ part,
     if (d_state_out) s -= d_state_out[b * n + i];
   }
   out[i] = s;
+}
+
+// ------------------------------------------------------------ block backward
+// Backward of y = x r g, r = (mean(x^2) + eps)^(-1/2) (the block's RMSNorms):
+//   dx = r (a - xhat mean(a xhat)),  a = dy g,  xhat = x r;  dg = sum_rows dy xhat.
+// One warp per row (grid-stride); dg accumulates per block in shared memory
+// and leaves as one partial row per block, gpart [gridDim.x, d].
+
+// The MLP RMSNorm of both paths (rows t and BT + t of h and du), with the
+// residual of the output (out = h_S + y, so d_out reaches h_S directly):
+//   dh_T = vjp(h_T, du_T),  dh_S = vjp(h_S, du_S) + d_out
+//   dh16 rows t, BT + t = bf16(dh_T), bf16(dh_S);  dx[t] = dh_T + dh_S  (x -> h_P)
+__global__ void __launch_bounds__(256) mlp_norm_backward_kernel(
+    const float* __restrict__ h, const float* __restrict__ du, const __nv_bfloat16* __restrict__ g,
+    const __nv_bfloat16* __restrict__ d_out, __nv_bfloat16* __restrict__ dh16,
+    float* __restrict__ dx, float* __restrict__ gpart, long long BT, int d, float eps) {
+  extern __shared__ float gsum[];  // [d]
+  for (int c = threadIdx.x; c < d; c += blockDim.x) gsum[c] = 0.f;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long t = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+       t < BT; t += nw) {
+    float rr[2], mm[2];
+    // pass 1: r and mean(a xhat) of both rows
+#pragma unroll
+    for (int path = 0; path < 2; ++path) {
+      const long long row = path * BT + t;
+      float ss = 0.f, ax = 0.f;
+      for (int c = lane * 8; c < d; c += 256) {
+        float x[8], dy[8], gv[8];
+        ld8f(h + row * d + c, x);
+        ld8f(du + row * d + c, dy);
+        ld8f(g + c, gv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          ss = fmaf(x[i], x[i], ss);
+          ax = fmaf(dy[i] * gv[i], x[i], ax);
+        }
+      }
+      ss = warp_sum(ss);
+      ax = warp_sum(ax);
+      rr[path] = rsqrtf(ss / d + eps);
+      mm[path] = ax * rr[path] / d;  // mean(a xhat) = r mean(a x)
+    }
+    // pass 2: dh of both rows, dx = dh_T + dh_S, dg
+    for (int c = lane * 8; c < d; c += 256) {
+      float gv[8], dh[2][8];
+      ld8f(g + c, gv);
+#pragma unroll
+      for (int path = 0; path < 2; ++path) {
+        const long long row = path * BT + t;
+        float x[8], dy[8];
+        ld8f(h + row * d + c, x);
+        ld8f(du + row * d + c, dy);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float xh = x[i] * rr[path];
+          dh[path][i] = rr[path] * (dy[i] * gv[i] - xh * mm[path]);
+          atomicAdd(&gsum[c + i], dy[i] * xh);
+        }
+      }
+      float res[8], sum[8];
+      ld8f(d_out + t * d + c, res);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        dh[1][i] += res[i];
+        sum[i] = dh[0][i] + dh[1][i];
+      }
+      st8f(dh16 + t * d + c, dh[0]);
+      st8f(dh16 + (BT + t) * d + c, dh[1]);
+      st8f(dx + t * d + c, sum);
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    gpart[static_cast<long long>(blockIdx.x) * d + c] = gsum[c];
+}
+
+// The input RMSNorm: dx[t] += vjp(x[t], dxn[t]) (x bf16), dg partials.
+__global__ void __launch_bounds__(256) input_norm_backward_kernel(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ dxn,
+    const __nv_bfloat16* __restrict__ g, float* __restrict__ dx, float* __restrict__ gpart,
+    long long BT, int d, float eps) {
+  extern __shared__ float gsum[];  // [d]
+  for (int c = threadIdx.x; c < d; c += blockDim.x) gsum[c] = 0.f;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long t = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+       t < BT; t += nw) {
+    float ss = 0.f, ax = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+      float xv[8], dy[8], gv[8];
+      ld8f(x + t * d + c, xv);
+      ld8f(dxn + t * d + c, dy);
+      ld8f(g + c, gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ss = fmaf(xv[i], xv[i], ss);
+        ax = fmaf(dy[i] * gv[i], xv[i], ax);
+      }
+    }
+    ss = warp_sum(ss);
+    ax = warp_sum(ax);
+    const float r = rsqrtf(ss / d + eps);
+    const float mm = ax * r / d;
+    for (int c = lane * 8; c < d; c += 256) {
+      float xv[8], dy[8], gv[8], o[8];
+      ld8f(x + t * d + c, xv);
+      ld8f(dxn + t * d + c, dy);
+      ld8f(g + c, gv);
+      ld8f(dx + t * d + c, o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float xh = xv[i] * r;
+        o[i] += r * (dy[i] * gv[i] - xh * mm);
+        atomicAdd(&gsum[c + i], dy[i] * xh);
+      }
+      st8f(dx + t * d + c, o);
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    gpart[static_cast<long long>(blockIdx.x) * d + c] = gsum[c];
+}
+
+// out[c] = sum over the rows of part [n, d] (fixed order).
+__global__ void column_sum_kernel(const float* __restrict__ part, float* __restrict__ out, int n,
+                                  int d) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= d) return;
+  float s = 0.f;
+  for (int i = 0; i < n; ++i) s += part[static_cast<long long>(i) * d + c];
+  out[c] = s;
+}
+
+// RoPE backward and packing of the Q/K/V gradients into one bf16 row per token:
+// dqkv[bt] = [R^T dq (Hq heads) | R^T dk (Hkv heads) | dv (Hkv heads)], where
+// R^T turns the pair (d_i, d_{i+hd/2}) at position t by -angle:
+// (d_i c + d_{i+hd/2} s, d_{i+hd/2} c - d_i s); cs [hd/2][T] half2 (cos, sin),
+// the forward's table.  One thread per (token, head, pair); the V heads copy.
+__global__ void rope_backward_pack_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
+                                          const float* __restrict__ dv,
+                                          const __half2* __restrict__ cs,
+                                          __nv_bfloat16* __restrict__ dqkv, long long BT, int T,
+                                          int Hq, int Hkv, int hd) {
+  const int half = hd / 2;
+  const int heads = Hq + 2 * Hkv;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= BT * heads * half) return;
+  const int i = static_cast<int>(idx % half);
+  const int hh = static_cast<int>((idx / half) % heads);
+  const long long bt = idx / (static_cast<long long>(half) * heads);
+  const int t = static_cast<int>(bt % T);
+  const long long ld = static_cast<long long>(heads) * hd;
+  __nv_bfloat16* out = dqkv + bt * ld + static_cast<long long>(hh) * hd;
+  const float* src;
+  if (hh < Hq) src = dq + (bt * Hq + hh) * hd;
+  else if (hh < Hq + Hkv) src = dk + (bt * Hkv + (hh - Hq)) * hd;
+  else src = dv + (bt * Hkv + (hh - Hq - Hkv)) * hd;
+  const float a = src[i], b = src[i + half];
+  if (hh < Hq + Hkv) {
+    const float2 e = __half22float2(cs[static_cast<long long>(i) * T + t]);
+    out[i] = __float2bfloat16_rn(a * e.x + b * e.y);
+    out[i + half] = __float2bfloat16_rn(b * e.x - a * e.y);
+  } else {
+    out[i] = __float2bfloat16_rn(a);
+    out[i + half] = __float2bfloat16_rn(b);
+  }
 }
 
 }  // namespace ttcd

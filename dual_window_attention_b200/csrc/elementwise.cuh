@@ -50,24 +50,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 // RMSNorm as the block's pre-norm (papernotes.org review, 方法详解: the shared
 // backbone; the pages leave the skeleton unstated, a pre-norm decoder layer is
 // the plain reading).
-// 8 consecutive elements (16-byte aligned) into fp32 registers, one or two
-// vector loads.
-__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(src);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = bf16lo_to_f32(w[i]);
-    v[2 * i + 1] = bf16hi_to_f32(w[i]);
-  }
-}
-__device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(src)[0];
-  const float4 b = reinterpret_cast<const float4*>(src)[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
 // One warp per row; rows up to RMS_CACHE * 256 columns stay in registers
 // between the sum of squares and the scaling (one pass over HBM), longer rows
 // are read again.
@@ -85,14 +67,14 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   for (int q = 0; q < RMS_CACHE; ++q) {
     const int c = lane * 8 + q * 256;
     if (c < d) {
-      load8(x + c, xv[q]);
+      ld8f(x + c, xv[q]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) ss += xv[q][i] * xv[q][i];
     }
   }
   for (int c = lane * 8 + RMS_CACHE * 256; c < d; c += 256) {
     float v[8];
-    load8(x + c, v);
+    ld8f(x + c, v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
   }
@@ -104,7 +86,7 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
     const int c = lane * 8 + q * 256;
     if (c < d) {
       float gv[8];
-      load8(g + c, gv);
+      ld8f(g + c, gv);
 #pragma unroll
       for (int i = 0; i < 8; ++i) xv[q][i] *= rs * gv[i];
       store8(y + c, xv[q]);
@@ -112,8 +94,8 @@ __global__ void rmsnorm_kernel(const InT* __restrict__ in, const GT* __restrict_
   }
   for (int c = lane * 8 + RMS_CACHE * 256; c < d; c += 256) {
     float v[8], gv[8];
-    load8(x + c, v);
-    load8(g + c, gv);
+    ld8f(x + c, v);
+    ld8f(g + c, gv);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] *= rs * gv[i];
     store8(y + c, v);
@@ -134,7 +116,7 @@ __global__ void rms_rowscale_kernel(const InT* __restrict__ in, float* __restric
   float ss = 0.f;
   for (int c = lane * 8; c < d; c += 256) {
     float v[8];
-    load8(x + c, v);
+    ld8f(x + c, v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
   }
@@ -153,8 +135,8 @@ __global__ void scale_cols_kernel(const E* __restrict__ w, const E* __restrict__
   const long long e0 = i * 8;
   const int c = static_cast<int>(e0 % cols);
   float v[8], gv[8];
-  load8(w + e0, v);
-  load8(g + c, gv);
+  ld8f(w + e0, v);
+  ld8f(g + c, gv);
 #pragma unroll
   for (int k = 0; k < 8; ++k) v[k] *= gv[k];
   store8(out + e0, v);
@@ -331,7 +313,7 @@ __global__ void u_tail_kernel(const E* __restrict__ u, const float* __restrict__
   const int b = static_cast<int>(pb % B), path = static_cast<int>(pb / B);
   const long long row = path * BT + static_cast<long long>(b) * T + T - n + j;
   float v[8];
-  load8(u + row * d + c, v);
+  ld8f(u + row * d + c, v);
   const float s = rstd[row];
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] *= s;

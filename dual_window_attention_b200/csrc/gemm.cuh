@@ -11,13 +11,14 @@
 // covers rows [b*T + i*C, b*T + min((i+1)*C, T)) and reads B rows starting at
 // (b*Nc + i) * b_group_rows.  A plain GEMM is one sequence with one chunk.
 #pragma once
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace ttcd {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;  // bf16 elements per 128-byte swizzled row
-constexpr int GEMM_THREADS = 192;
 
 struct TileCtx {
   int row0;        // first A row (== output row) of the tile
@@ -83,24 +84,50 @@ struct PairGeom {
   }
 };
 
-// Barrier and AND-vote over the four epilogue warps (named barrier 1, 128
-// threads).  Collective epilogues call them the same number of times in every
-// warp; the vote on each tile's accumulator wait makes an abort uniform, so no
-// warp leaves the tile loop while another waits at a barrier.
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier and AND-vote over the NT epilogue threads (named barrier 1).
+// Collective epilogues call them the same number of times in every warp; the
+// vote on each tile's accumulator wait makes an abort uniform, so no warp
+// leaves the tile loop while another waits at a barrier.
+template <int NT = 128>
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+template <int NT = 128>
 __device__ __forceinline__ bool epi_bar_and(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(static_cast<uint32_t>(v)), "n"(NT)
       : "memory");
   return r != 0;
 }
 
+// Epilogue warps of a GEMM: Epi::kWarps when the epilogue declares it (8: two
+// warps per TMEM lane quarter), else 4.  The kernel runs 2 + kWarps warps.
+template <class Epi, class = void>
+struct EpiWarps {
+  static constexpr int value = 4;
+};
+template <class Epi>
+struct EpiWarps<Epi, std::void_t<decltype(Epi::kWarps)>> {
+  static constexpr int value = Epi::kWarps;
+};
+template <class Epi>
+constexpr int gemm_threads() {
+  return 64 + 32 * EpiWarps<Epi>::value;
+}
+
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  tmem_ld16(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   tmem_ld32(taddr, r);
@@ -128,28 +155,6 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
 }
 __device__ __forceinline__ void store_x32(__nv_bfloat16* dst, const float (&v)[32]) { store_bf16x32(dst, v); }
 __device__ __forceinline__ void store_x32(float* dst, const float (&v)[32]) { store_f32x32(dst, v); }
-// 8 consecutive elements (16-byte aligned) to and from fp32 registers
-__device__ __forceinline__ void ld8f(const __nv_bfloat16* src, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(src);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = bf16lo_to_f32(w[i]);
-    v[2 * i + 1] = bf16hi_to_f32(w[i]);
-  }
-}
-__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void st8f(__nv_bfloat16* dst, const float (&v)[8]) {
-  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-}
-__device__ __forceinline__ void st8f(float* dst, const float (&v)[8]) {
-  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
 
 __device__ __forceinline__ void load_x32(const __nv_bfloat16* src, float (&v)[32]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
@@ -228,7 +233,7 @@ struct EpiStage {
 // g * b_group_rows, so K must then be a multiple of 64.
 template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom,
           bool B_MN = false>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
                    const __grid_constant__ CUtensorMap mapB1,
@@ -272,7 +277,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 128);
+      mbar_init(&acce[b], 32 * EpiWarps<Epi>::value);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -382,7 +387,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
-    EpiStage stg{STAGED ? staging + (warp - 2) * 8192 : nullptr, &mapOut, &mapOut2, 0};
+    // staging slots of 8 KB per lane quarter (8-warp epilogues share them by quarter)
+    EpiStage stg{STAGED ? staging + ((warp - 2) & 3) * 8192 : nullptr, &mapOut, &mapOut2, 0};
     int j = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       TileCtx c;
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       // per-row inputs of the epilogue are fetched while the tile is still computing
       const float pre = epi.pre(c, r);
       bool ok = mbar_wait(&accf[ab], (j >> 1) & 1, st, abort);
-      if constexpr (Epi::kCollective) ok = epi_bar_and(ok);
+      if constexpr (Epi::kCollective) ok = epi_bar_and<32 * EpiWarps<Epi>::value>(ok);
       if (!ok) break;
       tc_fence_after();
       epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r,
@@ -654,19 +660,22 @@ struct EpiSwiGLU {
 // rows 64-127 the student rows of the same tokens; columns [0, 128) are gate and
 // [128, 256) up for output columns tn*128 + [0, 128).
 //
-// Per 32-column slice, in two phases between which the four warps meet once:
-//   A  every thread (one accumulator row) forms z = silu(rstd g) (rstd u) in
-//      fp32 and writes its 32 values to a shared tile [path][row][column]
-//      (16-byte slots swizzled by row, so both the row-wise writes and the
-//      column-wise reads are conflict-free; two tiles alternate by slice);
-//   B  thread (row R, column group cg of 8 columns; two rows R and R + 32 per
-//      thread) forms the causal depthwise convs of both paths from the k rows
-//      R - k + 1 .. R of the tile (16-byte shared loads), and writes 8 columns
-//      of D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and of the
+// Eight epilogue warps, two per TMEM lane quarter (half h = 0, 1).  Per
+// 32-column slice, in two phases between which the eight warps meet once:
+//   A  every thread (one accumulator row, columns 16h .. 16h + 15 of the slice)
+//      forms z = silu(rstd g) (rstd u) in fp32 and writes its 16 values to a
+//      shared tile [path][row][column] (16-byte slots swizzled by row, so both
+//      the row-wise writes and the column reads of phase B are conflict-free;
+//      two tiles alternate by slice);
+//   B  thread (row R, column group cg of 8 columns) forms the causal depthwise
+//      convs of both paths from the k rows R - k + 1 .. R of the tile (16-byte
+//      shared loads; the taps of its 8 columns come as fp32 from a table
+//      [path][f/8][KMAX][8] made once per call), and writes 8 columns of
+//      D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and of the
 //      bf16 Z_S (output-GEMM operand) with one 16-byte store each.  The row's
-//      padded index is formed once per tile, the taps of the 8 columns once per
-//      slice.  Kp^2 accumulates per row over the slices; four lanes share a
-//      row and reduce once per tile (the key norm becomes a row scale of R).
+//      padded index is formed once per tile.  Kp^2 accumulates per row over the
+//      slices; four lanes share a row and reduce once per tile (the key norm
+//      becomes a row scale of R).
 // The tile's first k-1 rows only feed the conv (their outputs belong to the
 // previous tile); fp32 Z never reaches memory.
 //   z_halo [2, B, k-1, f] fp32: Z rows before token 0 (nullable: zeros)
@@ -674,14 +683,14 @@ struct EpiSwiGLU {
 template <int KMAX>  // conv width k <= KMAX
 struct EpiSwiGLUConv {
   static constexpr bool kStaged = true;      // the staging area holds the z tiles
-  static constexpr bool kCollective = true;  // the four warps exchange rows
+  static constexpr bool kCollective = true;  // the warps exchange rows
+  static constexpr int kWarps = 8;
   __nv_bfloat16* D;
   __nv_bfloat16* Kp;
   __nv_bfloat16* Zs;
   float* ssq;          // [ceil(f/128), P]
   const float* rstd;   // [2BT] MLP RMSNorm row scales, nullable (u already normalised)
-  const __nv_bfloat16* tapT;  // [f, k]
-  const __nv_bfloat16* tapS;
+  const float* taps;   // [2][f/8][KMAX][8] fp32: conv_T then conv_S, tap m of column 8c + i
   const float* z_halo;
   float* z_tail;
   int B, T, f, k, C, Cp, Nc;
@@ -700,131 +709,140 @@ struct EpiSwiGLUConv {
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     static_assert(BN == 256, "gate/up tiles are 128 gate + 128 up columns");
-    const int rin = r & 63;               // phase A: this thread's row within its path
+    constexpr int NT = 32 * kWarps;
+    const int et = static_cast<int>(threadIdx.x) - 64;  // epilogue thread 0..255
+    const int half = et >> 7;
+    const int rin = r & 63;  // phase A: this thread's row within its path
     const int path = r >= 64 ? 1 : 0;
     const int ta = c.tok0 + rin;
     const int b = c.group;
     const int H = k - 1;
-    const int et = static_cast<int>(threadIdx.x) - 64;  // epilogue thread 0..127
-    uint8_t* tiles = stg.buf - ((et >> 5) * 8192);      // the 32 KB staging area: two 16 KB z tiles
-    // phase B: rows et/4 and et/4 + 32, columns 8 cg .. 8 cg + 7 of each slice
+    uint8_t* tiles = stg.buf - ((et >> 5) & 3) * 8192;  // the 32 KB staging area: two 16 KB z tiles
+    // phase B: row et / 4, columns 8 cg .. 8 cg + 7 of each slice
     const int cg = et & 3;
-    int brow[2];
-    bool bval[2];
-    long long bp[2], bz[2];
-    float ssq_acc[2] = {0.f, 0.f};
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      brow[u] = (et >> 2) + 32 * u;
-      const int t = c.tok0 + brow[u];
-      bval[u] = brow[u] >= H && t >= 0 && t < T;
-      const int tt = bval[u] ? t : 0;
-      bp[u] = pidx(b, tt) * f;
-      bz[u] = (static_cast<long long>(b) * T + tt) * f;
-    }
+    const int brow = et >> 2;
+    const int bt = c.tok0 + brow;
+    const bool bval = brow >= H && bt >= 0 && bt < T;
+    const long long bp = pidx(b, bval ? bt : 0) * f;
+    const long long bz = (static_cast<long long>(b) * T + (bval ? bt : 0)) * f;
+    float ssq_acc = 0.f;
 #pragma unroll 1
     for (int s = 0; s < 4; ++s) {
       const int cc = 32 * s;
       const int col0 = c.tn * 128 + cc;
       if (col0 >= f) break;  // the same for every warp
       uint8_t* tile = tiles + (s & 1) * 16384;
-      // ---- A: z of this row, 32 columns
+      // ---- A: z of this row, 16 columns
       {
-        float z[32];
+        const int ch = cc + 16 * half;  // first column of this half within the tile
+        float z[16];
         {
-          float gt[32], up[32];
-          tmem_ld32f(taddr + cc, gt);
-          tmem_ld32f(taddr + 128 + cc, up);
+          float gt[16], up[16];
+          tmem_ld16f(taddr + ch, gt);
+          tmem_ld16f(taddr + 128 + ch, up);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 16; ++i) {
             const float gg = gt[i] * rs;
             z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (up[i] * rs);
           }
         }
+        const int zc = col0 + 16 * half;  // global column of z[0]
         if (ta < 0 || ta >= T) {
           if (ta < 0 && z_halo) {
-            load_x32(z_halo + ((static_cast<long long>(path) * B + b) * H + (ta + H)) * f + col0, z);
+            const float* src = z_halo + ((static_cast<long long>(path) * B + b) * H + (ta + H)) * f + zc;
+            float lo[8], hi[8];
+            ld8f(src, lo);
+            ld8f(src + 8, hi);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { z[i] = lo[i]; z[8 + i] = hi[i]; }
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = 0.f;
+            for (int i = 0; i < 16; ++i) z[i] = 0.f;
           }
         }
-        if (z_tail && rin >= H && ta >= T - H && ta < T && ta >= 0)
-          store_f32x32(z_tail + ((static_cast<long long>(path) * B + b) * H + (ta - (T - H))) * f + col0, z);
+        if (z_tail && rin >= H && ta >= T - H && ta < T && ta >= 0) {
+          float* dst = z_tail + ((static_cast<long long>(path) * B + b) * H + (ta - (T - H))) * f + zc;
+          st8f(dst, *reinterpret_cast<const float(*)[8]>(&z[0]));
+          st8f(dst + 8, *reinterpret_cast<const float(*)[8]>(&z[8]));
+        }
         const int R = path * 64 + rin;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4*>(tile + R * 128 + ((j ^ (R & 7)) << 4)) =
+        for (int j = 0; j < 4; ++j) {
+          const int jj = 4 * half + j;
+          *reinterpret_cast<float4*>(tile + R * 128 + ((jj ^ (R & 7)) << 4)) =
               make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
+        }
       }
-      epi_bar_sync();
-      // ---- B: the convs of rows brow[u], columns col0 + 8 cg .. + 7, both paths
+      epi_bar_sync<NT>();
+      // ---- B: the convs of row brow, columns col0 + 8 cg .. + 7, both paths
       {
         const int col = col0 + 8 * cg;
-        float aT[2][8], aS[2][8], z0[2][8];
+        const float* tT = taps + (static_cast<long long>(col >> 3) * KMAX) * 8;
+        const float* tS = tT + static_cast<long long>(f) * KMAX;
+        float aT[8], aS[8], z0[8];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) { aT[u][i] = 0.f; aS[u][i] = 0.f; z0[u][i] = 0.f; }
+        for (int i = 0; i < 8; ++i) { aT[i] = 0.f; aS[i] = 0.f; z0[i] = 0.f; }
 #pragma unroll
         for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
-          if (m >= k) break;
-          float tT[8], tS[8];
+          if (m >= k || brow - m < 0) break;
+          float wT[8], wS[8], zt[8], zs[8];
+          ld8f(tT + m * 8, wT);
+          ld8f(tS + m * 8, wS);
+          const int RT = brow - m, RS = 64 + brow - m;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 2 * cg + h;
+            const float4 x = *reinterpret_cast<const float4*>(tile + RT * 128 + ((j ^ (RT & 7)) << 4));
+            const float4 y = *reinterpret_cast<const float4*>(tile + RS * 128 + ((j ^ (RS & 7)) << 4));
+            zt[4 * h] = x.x; zt[4 * h + 1] = x.y; zt[4 * h + 2] = x.z; zt[4 * h + 3] = x.w;
+            zs[4 * h] = y.x; zs[4 * h + 1] = y.y; zs[4 * h + 2] = y.z; zs[4 * h + 3] = y.w;
+          }
+          if (m == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) z0[i] = zs[i];
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            tT[i] = __bfloat162float(tapT[static_cast<long long>(col + i) * k + m]);
-            tS[i] = __bfloat162float(tapS[static_cast<long long>(col + i) * k + m]);
-          }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int RT = brow[u] - m, RS = 64 + brow[u] - m;
-            if (RT < 0) continue;
-            float zt[8], zs[8];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int j = 2 * cg + h;
-              const float4 x = *reinterpret_cast<const float4*>(tile + RT * 128 + ((j ^ (RT & 7)) << 4));
-              const float4 y = *reinterpret_cast<const float4*>(tile + RS * 128 + ((j ^ (RS & 7)) << 4));
-              zt[4 * h] = x.x; zt[4 * h + 1] = x.y; zt[4 * h + 2] = x.z; zt[4 * h + 3] = x.w;
-              zs[4 * h] = y.x; zs[4 * h + 1] = y.y; zs[4 * h + 2] = y.z; zs[4 * h + 3] = y.w;
-            }
-            if (m == 0) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) z0[u][i] = zs[i];
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              aT[u][i] = fmaf(tT[i], zt[i], aT[u][i]);
-              aS[u][i] = fmaf(tS[i], zs[i], aS[u][i]);
-            }
+            aT[i] = fmaf(wT[i], zt[i], aT[i]);
+            aS[i] = fmaf(wS[i], zs[i], aS[i]);
           }
         }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (!bval[u]) continue;
+        if (bval) {
           float dd[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            dd[i] = aT[u][i] - aS[u][i];
-            ssq_acc[u] = fmaf(aS[u][i], aS[u][i], ssq_acc[u]);
+            dd[i] = aT[i] - aS[i];
+            ssq_acc = fmaf(aS[i], aS[i], ssq_acc);
           }
-          st8f(D + bp[u] + col, dd);
-          st8f(Kp + bp[u] + col, aS[u]);
-          st8f(Zs + bz[u] + col, z0[u]);
+          st8f(D + bp + col, dd);
+          st8f(Kp + bp + col, aS);
+          st8f(Zs + bz + col, z0);
         }
       }
     }
     // per-token sums of Kp^2 over the tile's columns: the four lanes of a row
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float v = ssq_acc[u];
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      if (cg == 0 && bval[u])
-        ssq[static_cast<long long>(c.tn) * P + pidx(b, c.tok0 + brow[u])] = v;
-    }
+    float v = ssq_acc;
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    if (cg == 0 && bval) ssq[static_cast<long long>(c.tn) * P + pidx(b, bt)] = v;
   }
 };
+
+// taps[path][c / 8][m][c % 8] = conv_path[c, m] (fp32, zero for m >= k): the
+// table the gate/up conv epilogue reads, 8 columns of one tap per 32 bytes.
+template <int KMAX>
+__global__ void conv_tap_table_kernel(const __nv_bfloat16* __restrict__ conv_T,
+                                      const __nv_bfloat16* __restrict__ conv_S,
+                                      float* __restrict__ taps, int f, int k) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= 2 * f * KMAX) return;
+  const int path = idx / (f * KMAX);
+  const int e = idx % (f * KMAX);
+  const int c8 = e / (KMAX * 8), m = (e / 8) % KMAX, ci = e % 8;
+  const int col = c8 * 8 + ci;
+  const __nv_bfloat16* w = path ? conv_S : conv_T;
+  taps[idx] = m < k ? __bfloat162float(w[static_cast<long long>(col) * k + m]) : 0.f;
+}
 
 // QKV projection with rotary embedding on the query and key heads, written to
 // one token-major tensor qkv [rows, (Hq + 2 Hkv) HD]: q heads, then k heads,

@@ -115,13 +115,6 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
 #pragma unroll
             for (int q = 0; q < BN / BK; ++q)
               tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
-            if (i + 1 < a.Nc) {  // the same boxes of the next chunk, into L2
-              const int yn = a.reverse ? y - a.Cp : y + a.Cp;
-#pragma unroll
-              for (int q = 0; q < GEMM_BM / BK; ++q) tma_prefetch_l2_2d(&mapR, m0 + q * BK, yn);
-#pragma unroll
-              for (int q = 0; q < BN / BK; ++q) tma_prefetch_l2_2d(&mapK, n0 + q * BK, yn);
-            }
           } else {
             tma_load_2d(sa, &mapR, &full[s], y, m0);
             tma_load_2d(sa + A_BYTES, &mapK, &full[s], y, n0);

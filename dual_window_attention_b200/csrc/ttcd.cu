@@ -180,7 +180,7 @@ ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
   const int grid = total < c.sms ? total : c.sms;
-  kern<<<grid, GEMM_THREADS, smem, c.s>>>(A, B0, B1, out_map ? *out_map : A,
+  kern<<<grid, gemm_threads<Epi>(), smem, c.s>>>(A, B0, B1, out_map ? *out_map : A,
                                            out_map2 ? *out_map2 : A, geo, epi, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
@@ -230,13 +230,13 @@ struct Layout {
 enum Buf {
   B_STATUS, B_WQKVG, B_RSTDIN, B_QKV, B_O, B_H, B_ROPE, B_U, B_Z, B_ZS16, B_D, B_KP, B_SSQ,
   B_KSCALE, B_R, B_WALL, B_M, B_WPROJT, B_RT, B_KT, B_HSSQ, B_RSTD, B_X32, B_OUT32, B_HS32,
-  B_W32, B_QKVX, B_ZH, B_UH, B_COUNT
+  B_W32, B_QKVX, B_ZH, B_UH, B_TAPS, B_COUNT
 };
 static_assert(B_COUNT <= 32, "workspace layout table too small");
 const char* kBufNames[B_COUNT] = {"status", "wqkv_g", "rstd_in", "qkv", "o", "h", "rope", "u",
                                   "Z", "Zs16", "D", "Kp", "ssq", "kscale", "R", "Wall", "M",
                                   "WprojT", "Rt", "Kt", "hssq", "rstd", "x32", "out32", "hS32",
-                                  "w32", "qkv_ext", "z_halo", "u_halo"};
+                                  "w32", "qkv_ext", "z_halo", "u_halo", "taps"};
 
 // bf16 problems shorter than one chunk run with fp32 operands (kind::tf32 MMAs):
 // their fast-weight state is the sum of fewer than C rank-1 writes, so the bf16
@@ -307,6 +307,7 @@ Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false,
   sz[B_U] = 2 * m.BT * m.d * e;
   sz[B_Z] = e == 4 ? 2 * m.BT * m.f * 4 : 0;  // bf16: Z stays on chip (fused gate/up + conv)
   sz[B_ZS16] = e == 2 ? m.BT * m.f * 2 : 0;  // fp32 mode reads Z_S directly
+  sz[B_TAPS] = e == 2 ? 2 * static_cast<size_t>(m.f) * 8 * 4 : 0;  // fp32 conv tap table
   sz[B_D] = m.P * m.f * e;
   sz[B_KP] = m.P * m.f * e;
   sz[B_SSQ] = m.P * 4 * (m.f / 64);
@@ -477,12 +478,19 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
     g.tiles_m = cdiv(p->T, 64 - H);
     g.tiles_n = cdiv(m.f, 128);
     g.half_rows = m.BT;
+    float* taps = at<float>(ws, L, B_TAPS);
     if (p->conv_k <= 4) {
-      EpiSwiGLUConv<4> e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
+      conv_tap_table_kernel<4><<<cdiv(2 * m.f * 4, 256), 256, 0, c.s>>>(conv_T, conv_S, taps, m.f,
+                                                                        p->conv_k);
+      TTCD_CHECK_LAUNCH();
+      EpiSwiGLUConv<4> e{D, Kp, Zs, ssq, rstd, taps, z_halo, nullptr,
                          p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
       TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<4>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
     } else {
-      EpiSwiGLUConv<8> e{D, Kp, Zs, ssq, rstd, conv_T, conv_S, z_halo, nullptr,
+      conv_tap_table_kernel<8><<<cdiv(2 * m.f * 8, 256), 256, 0, c.s>>>(conv_T, conv_S, taps, m.f,
+                                                                        p->conv_k);
+      TTCD_CHECK_LAUNCH();
+      EpiSwiGLUConv<8> e{D, Kp, Zs, ssq, rstd, taps, z_halo, nullptr,
                          p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
       TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<8>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
     }
@@ -2089,12 +2097,14 @@ size_t attn_bwd_ws_bytes(int B, int T, int Hq) {
   return kStatusBytes + 2 * ((rows + 1023) / 1024 * 1024);
 }
 
+// q rows have ld_q elements between tokens, k and v rows ld_kv (as launch_attn);
+// o, dO, dq, dk, dv are dense.
 template <int HD>
 ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const void* v,
                             const void* o_T, const void* o_S, const float* lse_T,
                             const float* lse_S, const void* do_T, const void* do_S, float* dq,
                             float* dk, float* dv, int B, int T, int Hq, int Hkv, int w_S,
-                            int w_T, float scale, void* ws) {
+                            int w_T, float scale, void* ws, long long ld_q, long long ld_kv) {
   using bf = __nv_bfloat16;
   const long long BT = static_cast<long long>(B) * T;
   const size_t rows_bytes = (static_cast<size_t>(B) * Hq * T * 4 + 1023) / 1024 * 1024;
@@ -2110,8 +2120,9 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
   TTCD_CHECK_LAUNCH();
   CUtensorMap mq, mk, mv, mdt, mds;
   const uint64_t wq = static_cast<uint64_t>(Hq) * HD, wkv = static_cast<uint64_t>(Hkv) * HD;
-  if (!make_map<bf>(&mq, q, wq, BT, wq * 2, 64, 128) || !make_map<bf>(&mk, k, wkv, BT, wkv * 2, 64, 128) ||
-      !make_map<bf>(&mv, v, wkv, BT, wkv * 2, 64, 128) ||
+  if (!make_map<bf>(&mq, q, wq, BT, ld_q * 2, 64, 128) ||
+      !make_map<bf>(&mk, k, wkv, BT, ld_kv * 2, 64, 128) ||
+      !make_map<bf>(&mv, v, wkv, BT, ld_kv * 2, 64, 128) ||
       !make_map<bf>(&mdt, do_T, wq, BT, wq * 2, 64, 128) ||
       !make_map<bf>(&mds, do_S, wq, BT, wq * 2, 64, 128))
     return TTCD_ERR_CUDA;
@@ -2172,11 +2183,224 @@ ttcd_status ttcd_dual_window_attn_backward(const void* q, const void* k, const v
   Ctx c;
   TTCD_TRY(make_ctx(stream, c, workspace));
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(hd));
+  const long long lq = static_cast<long long>(Hq) * hd, lkv = static_cast<long long>(Hkv) * hd;
   if (hd == 64)
     return launch_attn_bwd<64>(c, q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, dq, dk, dv, B, T,
-                               Hq, Hkv, w_S, w_T, sc, workspace);
+                               Hq, Hkv, w_S, w_T, sc, workspace, lq, lkv);
   return launch_attn_bwd<128>(c, q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, dq, dk, dv, B, T,
-                              Hq, Hkv, w_S, w_T, sc, workspace);
+                              Hq, Hkv, w_S, w_T, sc, workspace, lq, lkv);
+}
+
+}  // extern "C"
+
+// ================================================================== block backward
+// The chain rule of the block forward (run_block) in reverse, bf16 operands:
+// the forward up to the MLP inputs is recomputed (q, k, v with RoPE, both
+// attention outputs with their log-sum-exps, h_P = x + o_P W_o^T in fp32, u_P),
+// then the MLP backward, the MLP RMSNorm backward with the output residual,
+// o_proj's two GEMMs, the attention backward, RoPE's transpose, the QKV GEMMs
+// and the input RMSNorm backward.
+namespace {
+
+constexpr int NORM_BLOCKS = 296;  // blocks of the RMSNorm backward kernels (2 per SM)
+
+struct BlockBwdLayout {
+  Layout F;    // the forward block workspace: qkv, o, the RoPE table, row scales
+  BwdLayout M; // the MLP backward's workspace, at offset `mlp`
+  size_t mlp, lse_T, lse_S, h, u, du, dh, dO, dq, dk, dv, dqkv, xn, dxn, gpart, attn, total;
+};
+
+BlockBwdLayout block_bwd_layout(const ttcd_block_params* p) {
+  const Dims m = dims_of(p);
+  BlockBwdLayout L;
+  L.F = make_layout(p, true, false, false);
+  L.M = bwd_layout(p);
+  const size_t BT = static_cast<size_t>(m.BT), d = m.d, dq = static_cast<size_t>(m.Hq) * m.hd,
+               dkv = static_cast<size_t>(m.Hkv) * m.hd;
+  const size_t sz[16] = {L.M.total,
+                         static_cast<size_t>(p->B) * m.Hq * p->T * 4,  // lse_T
+                         static_cast<size_t>(p->B) * m.Hq * p->T * 4,  // lse_S
+                         2 * BT * d * 4,                               // h_T, h_S
+                         2 * BT * d * 2,                               // u_T, u_S
+                         2 * BT * d * 4,                               // du_T, du_S
+                         2 * BT * d * 2,                               // dh (bf16)
+                         2 * BT * dq * 2,                              // do_T, do_S
+                         BT * dq * 4,                                  // dq
+                         BT * dkv * 4,                                 // dk
+                         BT * dkv * 4,                                 // dv
+                         BT * static_cast<size_t>(m.dqkv) * 2,         // dqkv (bf16)
+                         BT * d * 2,                                   // xn (bf16)
+                         BT * d * 4,                                   // dxn
+                         2 * static_cast<size_t>(NORM_BLOCKS) * d * 4, // RMSNorm gain partials
+                         attn_bwd_ws_bytes(p->B, p->T, m.Hq)};
+  size_t* f[16] = {&L.mlp, &L.lse_T, &L.lse_S, &L.h, &L.u, &L.du, &L.dh, &L.dO, &L.dq, &L.dk,
+                   &L.dv, &L.dqkv, &L.xn, &L.dxn, &L.gpart, &L.attn};
+  size_t off = L.F.total;
+  for (int i = 0; i < 16; ++i) {
+    *f[i] = off;
+    off += (sz[i] + 1023) / 1024 * 1024;
+  }
+  L.total = off;
+  return L;
+}
+
+ttcd_status block_backward_bf16(const Ctx& c, const __nv_bfloat16* x, const float* beta,
+                                const ttcd_block_weights* w, const ttcd_block_params* p,
+                                const float* state_in, const __nv_bfloat16* d_out,
+                                const float* d_state_out, float* dx, float* d_beta,
+                                float* d_state_in, const ttcd_block_grads* g, void* ws,
+                                const BlockBwdLayout& L) {
+  using bf = __nv_bfloat16;
+  const Dims m = dims_of(p);
+  const Layout& F = L.F;
+  const long long BT = m.BT, dq = static_cast<long long>(m.Hq) * m.hd;
+  bf* qkv = at<bf>(ws, F, B_QKV);
+  bf* o = at<bf>(ws, F, B_O);
+  float* lse_T = dat<float>(ws, L.lse_T);
+  float* lse_S = dat<float>(ws, L.lse_S);
+  float* h = dat<float>(ws, L.h);
+  bf* u = dat<bf>(ws, L.u);
+  float* du = dat<float>(ws, L.du);
+  bf* dh = dat<bf>(ws, L.dh);
+  bf* dO = dat<bf>(ws, L.dO);
+  float* gq = dat<float>(ws, L.dq);
+  float* gk = dat<float>(ws, L.dk);
+  float* gv = dat<float>(ws, L.dv);
+  bf* dqkv = dat<bf>(ws, L.dqkv);
+  bf* xn = dat<bf>(ws, L.xn);
+  float* dxn = dat<float>(ws, L.dxn);
+  float* gpart = dat<float>(ws, L.gpart);
+  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
+
+  // ---- forward up to the MLP inputs
+  TTCD_TRY(block_qkv<bf>(c, x, w, p, ws, F, qkv, 0, 0));
+  TTCD_TRY(run_attn<bf>(c, qkv, qkv + dq, qkv + dq + static_cast<long long>(m.Hkv) * m.hd, o,
+                        o + BT * dq, lse_T, lse_S, p->B, p->T, m.Hq, m.Hkv, m.hd, p->w_S, p->w_T,
+                        sc, m.dqkv, m.dqkv));
+  {  // h_P = x + o_P W_o^T, fp32, both paths
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, o, 2 * BT, dq, 128) || !map_rows<bf>(&mB, w->w_o, m.d, dq, 256) ||
+        !make_out_map<float>(&mo, h, 2 * BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    EpiResidual<float, bf> e{h, m.d, x, m.d, BT, m.d};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(2 * BT, cdiv(m.d, 256), static_cast<int>(dq)), e)));
+  }
+  rmsnorm_kernel<float, bf, bf><<<cdiv(2 * BT, 8), 256, 0, c.s>>>(
+      h, static_cast<const bf*>(w->g_mlp), u, 2 * BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+
+  // ---- the fast-weight MLP
+  const ttcd_mlp_grads mg{g->w_gate, g->w_up, g->w_down, g->w_proj, g->conv_T, g->conv_S};
+  TTCD_TRY(mlp_backward_bf16(c, u, u + BT * m.d, beta, w, p, state_in, d_out, d_state_out, du,
+                             du + BT * m.d, d_beta, d_state_in, &mg, dat<void>(ws, L.mlp), L.M));
+
+  // ---- MLP RMSNorm of both paths and the output residual: dh (bf16), dx = dh_T + dh_S
+  const size_t norm_smem = static_cast<size_t>(m.d) * 4;
+  mlp_norm_backward_kernel<<<NORM_BLOCKS, 256, norm_smem, c.s>>>(
+      h, du, static_cast<const bf*>(w->g_mlp), d_out, dh, dx, gpart, BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  column_sum_kernel<<<cdiv(m.d, 256), 256, 0, c.s>>>(gpart, g->g_mlp, NORM_BLOCKS, m.d);
+  TTCD_CHECK_LAUNCH();
+
+  // ---- o_proj: dO = dh W_o (W_o [d, Hq hd] read MN-major), dW_o = dh^T o
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dh, 2 * BT, m.d, 128) ||
+        !make_map<bf>(&mB, w->w_o, dq, m.d, dq * 2, 64, 64) ||
+        !make_out_map<bf>(&mo, dO, 2 * BT, dq, dq))
+      return TTCD_ERR_CUDA;
+    EpiStore<bf> e{dO, dq, static_cast<int>(dq), nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<bf>, GemmGeom, true>(
+        c, mA, mB, mB, &mo, plain_geom(2 * BT, cdiv(dq, 256), m.d), e)));
+  }
+  TTCD_TRY(launch_tsum(c, dh, m.d, m.d, o, dq, static_cast<int>(dq), 2 * BT, g->w_o));
+
+  // ---- attention (q, k, v are strided views of qkv)
+  {
+    void* aws = dat<void>(ws, L.attn);
+    const bf* qp = qkv;
+    const bf* kp = qkv + dq;
+    const bf* vp = qkv + dq + static_cast<long long>(m.Hkv) * m.hd;
+    if (m.hd == 64)
+      TTCD_TRY(launch_attn_bwd<64>(c, qp, kp, vp, o, o + BT * dq, lse_T, lse_S, dO, dO + BT * dq,
+                                   gq, gk, gv, p->B, p->T, m.Hq, m.Hkv, p->w_S, p->w_T, sc, aws,
+                                   m.dqkv, m.dqkv));
+    else
+      TTCD_TRY(launch_attn_bwd<128>(c, qp, kp, vp, o, o + BT * dq, lse_T, lse_S, dO, dO + BT * dq,
+                                    gq, gk, gv, p->B, p->T, m.Hq, m.Hkv, p->w_S, p->w_T, sc, aws,
+                                    m.dqkv, m.dqkv));
+  }
+  {  // RoPE's transpose, packed with dv into one bf16 row per token
+    const long long n = BT * (m.Hq + 2 * m.Hkv) * (m.hd / 2);
+    rope_backward_pack_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+        gq, gk, gv, at<__half2>(ws, F, B_ROPE), dqkv, BT, p->T, m.Hq, m.Hkv, m.hd);
+    TTCD_CHECK_LAUNCH();
+  }
+
+  // ---- QKV: dxn = dqkv W_qkv (W_qkv [dqkv, d] read MN-major), dW_qkv = dqkv^T xn
+  {
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<bf>(&mA, dqkv, BT, m.dqkv, 128) ||
+        !make_map<bf>(&mB, w->w_qkv, m.d, m.dqkv, static_cast<uint64_t>(m.d) * 2, 64, 64) ||
+        !make_out_map<float>(&mo, dxn, BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    EpiStore<float> e{dxn, m.d, m.d, nullptr};
+    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(
+        c, mA, mB, mB, &mo, plain_geom(BT, cdiv(m.d, 256), m.dqkv), e)));
+  }
+  rmsnorm_kernel<bf, bf, bf><<<cdiv(BT, 8), 256, 0, c.s>>>(
+      x, static_cast<const bf*>(w->g_attn), xn, BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  TTCD_TRY(launch_tsum(c, dqkv, m.dqkv, m.dqkv, xn, m.d, m.d, BT, g->w_qkv));
+
+  // ---- input RMSNorm
+  input_norm_backward_kernel<<<NORM_BLOCKS, 256, norm_smem, c.s>>>(
+      x, dxn, static_cast<const bf*>(w->g_attn), dx, gpart + static_cast<long long>(NORM_BLOCKS) * m.d,
+      BT, m.d, p->rms_eps);
+  TTCD_CHECK_LAUNCH();
+  column_sum_kernel<<<cdiv(m.d, 256), 256, 0, c.s>>>(
+      gpart + static_cast<long long>(NORM_BLOCKS) * m.d, g->g_attn, NORM_BLOCKS, m.d);
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttcd_block_backward_workspace_size(const ttcd_block_params* p) {
+  if (check_bwd_params(p) != TTCD_OK) return 0;
+  if (p->head_dim != 64 && p->head_dim != 128) return 0;
+  return block_bwd_layout(p).total;
+}
+
+ttcd_status ttcd_block_backward(const void* x, const float* beta, const ttcd_block_weights* w,
+                                const ttcd_block_params* p, const float* state_in,
+                                const void* d_out, const float* d_state_out, float* dx,
+                                float* d_beta, float* d_state_in, const ttcd_block_grads* grads,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_bwd_params(p));
+  if (p->head_dim != 64 && p->head_dim != 128) return TTCD_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(beta) || !aligned16(d_out) || !aligned16(dx) ||
+      !aligned16(d_beta) || !weights_ok(w, true) || !aligned16(workspace) || !grads)
+    return TTCD_ERR_INVALID_ARG;
+  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
+      (d_state_in && !aligned16(d_state_in)))
+    return TTCD_ERR_INVALID_ARG;
+  const float* gp[10] = {grads->w_qkv, grads->w_o,    grads->g_attn, grads->g_mlp,
+                         grads->w_gate, grads->w_up,  grads->w_down, grads->w_proj,
+                         grads->conv_T, grads->conv_S};
+  for (const float* q : gp)
+    if (!aligned16(q)) return TTCD_ERR_INVALID_ARG;
+  if (static_cast<size_t>(p->d_model) * 4 > 48 * 1024) return TTCD_ERR_UNSUPPORTED;
+  const BlockBwdLayout L = block_bwd_layout(p);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, workspace));
+  using bf = __nv_bfloat16;
+  return block_backward_bf16(c, static_cast<const bf*>(x), beta, w, p, state_in,
+                             static_cast<const bf*>(d_out), d_state_out, dx, d_beta, d_state_in,
+                             grads, workspace, L);
 }
 
 }  // extern "C"

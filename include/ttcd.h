@@ -289,6 +289,52 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
                                const ttcd_block_params* p, float* state_out, void* out,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* fp32 gradients of the block's weights (device, written, not accumulated);
+ * fields in the order and shapes of ttcd_block_weights. */
+typedef struct {
+  float* w_qkv;  /* [(Hq + 2 Hkv) hd, d] */
+  float* w_o;    /* [d, Hq hd] */
+  float* g_attn; /* [d] */
+  float* g_mlp;  /* [d] */
+  float* w_gate; /* [f, d] */
+  float* w_up;   /* [f, d] */
+  float* w_down; /* [d, f] */
+  float* w_proj; /* [f, f] */
+  float* conv_T; /* [f, conv_k] */
+  float* conv_S; /* [f, conv_k] */
+} ttcd_block_grads;
+
+/* Workspace bytes of ttcd_block_backward; 0 when p is invalid, not TTCD_BF16
+ * or head_dim is not 64 or 128. */
+size_t ttcd_block_backward_workspace_size(const ttcd_block_params* p);
+
+/*
+ * ttcd_block_backward — vector-Jacobian product of ttcd_block_forward.
+ *
+ * For a scalar loss L with dL/dout = d_out and dL/dstate_out = d_state_out,
+ * the gradients of L with respect to x, beta, state_in and every weight: the
+ * chain rule of the steps listed at ttcd_block_forward in reverse ([REVIEW]
+ * 方法详解 flowchart A-F, 关键设计 2-3; training differentiates the whole block,
+ * [REVIEW] 局限与展望).  The forward is recomputed in the workspace.
+ *   x, beta, w, p, state_in: as ttcd_block_forward (TTCD_BF16, hd 64 or 128)
+ *   d_out        [B, T, d] bf16, device
+ *   d_state_out  [B, d, f] fp32, device, nullable (zero)
+ *   dx           [B, T, d] fp32, device, written
+ *   d_beta       [B, T] fp32, device, written
+ *   d_state_in   [B, d, f] fp32, device, nullable, written
+ *   grads        the ten weight gradients (all required)
+ *   workspace    >= ttcd_block_backward_workspace_size(p) bytes, device, 16-byte
+ *                aligned; status word first
+ * Precision: as ttcd_fastweight_mlp_backward and ttcd_dual_window_attn_backward;
+ * the RMSNorm backward steps are fp32.
+ * Errors: TTCD_ERR_UNSUPPORTED for TTCD_F32, head_dim 32 or d_model > 12288.
+ */
+ttcd_status ttcd_block_backward(const void* x, const float* beta, const ttcd_block_weights* w,
+                                const ttcd_block_params* p, const float* state_in,
+                                const void* d_out, const float* d_state_out, float* dx,
+                                float* d_beta, float* d_state_in, const ttcd_block_grads* grads,
+                                void* workspace, size_t ws_bytes, void* stream);
+
 /*
  * ttcd_block_forward_profiled — ttcd_block_forward that also records the
  * caller's CUDA events (cudaEvent_t handles, owned by the caller) on `stream`
