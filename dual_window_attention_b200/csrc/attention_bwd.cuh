@@ -20,16 +20,21 @@
 // visit is added to the fp32 dq in global memory (vector atomics).
 //
 // Pipeline (one CTA, 384 threads):
-//   warp 0      TMA producer: K and V once, then Q and dO per visit
-//   warp 1      TMEM owner and tcgen05.mma issuer (one thread)
-//   warps 4..7  thread = key row: P^T and dS^T rows into shared memory, and at
-//               the end the dK and dV rows
+//   warp 0      TMA producer: K and V once, then Q and dO per visit (two stages)
+//   warp 1      TMEM owner and tcgen05.mma issuer (one thread), per visit v:
+//               dV(v), S(v+1), dK(v) dQ(v), dP(v+1), so that the next visit's
+//               scores form while the key-row threads work on dS(v)
+//   warps 4..7  thread = key row: P^T (into TMEM, over its S^T row) and dS^T
+//               (into shared memory), and at the end the dK and dV rows
 //   warps 8..11 thread = query row: the dQ tile of each visit into dq
-// TMEM (512 columns): S^T [0,128), dP^T [128,256) (reused for the dQ tile once
-// dS^T is formed), dK [256, 256+HD), dV [256+HD, 256+2HD).
+// TMEM (512 columns): S^T [0,128), whose first 64 columns take P^T as packed
+// bf16 pairs (the A operand of dV, as P is for O in the forward); dP^T
+// [128,256), reused for the dQ tile once dS^T is formed; dK [256, 256+HD), dV
+// [256+HD, 256+2HD).  The tensor pipe runs one CTA's MMAs in issue order, so
+// S(v+1) overwrites P^T(v) only after dV(v) has read it.
 // Shared memory operands (128-byte swizzle, 64-column panels of 128 rows):
-// K, V, Q, dO tiles as loaded by TMA; P^T and dS^T written by the key-row
-// threads.  The same tile is read K-major or MN-major by choosing the
+// K, V, and two stages of Q and dO as loaded by TMA; dS^T written by the
+// key-row threads.  The same tile is read K-major or MN-major by choosing the
 // descriptor: Q is the B operand of S^T (K-major) and of dK (MN-major), dS^T is
 // the A operand of dK (K-major) and, read as dS, of dQ (MN-major).
 #pragma once
@@ -59,14 +64,13 @@ struct AttnBwdCfg {
   static_assert(HD == 64 || HD == 128, "head_dim 64 or 128");
   static constexpr int PANELS = HD / 64;
   static constexpr int TILE = PANELS * 128 * 128;  // K, V, Q, dO tiles
-  static constexpr int PT_TILE = 2 * 128 * 128;    // P^T, dS^T: 128 x 128 bf16
+  static constexpr int DS_TILE = 2 * 128 * 128;    // dS^T: 128 x 128 bf16
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
-  static constexpr int Q_OFF = V_OFF + TILE;
-  static constexpr int DO_OFF = Q_OFF + TILE;
-  static constexpr int PT_OFF = DO_OFF + TILE;
-  static constexpr int DS_OFF = PT_OFF + PT_TILE;
-  static constexpr int LSE_OFF = DS_OFF + PT_TILE;  // 128 floats
+  static constexpr int Q_OFF = V_OFF + TILE;       // two stages
+  static constexpr int DO_OFF = Q_OFF + 2 * TILE;  // two stages
+  static constexpr int DS_OFF = DO_OFF + 2 * TILE;
+  static constexpr int LSE_OFF = DS_OFF + DS_TILE;  // 128 floats
   static constexpr int DEL_OFF = LSE_OFF + 512;     // 128 floats
   static constexpr int BAR_OFF = DEL_OFF + 512;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
@@ -137,14 +141,12 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
   float* dlt = reinterpret_cast<float*>(smem + Cfg::DEL_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qdo_full = bars + 1;
-  uint64_t* qdo_empty = bars + 2;
-  uint64_t* s_full = bars + 3;
-  uint64_t* s_free = bars + 4;    // 128 arrivals
-  uint64_t* dp_full = bars + 5;
-  uint64_t* dp_free = bars + 6;   // 128 arrivals
-  uint64_t* p_ready = bars + 7;   // 128 arrivals
-  uint64_t* pt_free = bars + 8;
+  uint64_t* qdo_full = bars + 1;   // 2 stages
+  uint64_t* qdo_empty = bars + 3;  // 2 stages
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* dp_free = bars + 7;   // 128 arrivals
+  uint64_t* p_ready = bars + 8;   // 128 arrivals
   uint64_t* ds_ready = bars + 9;  // 128 arrivals
   uint64_t* dst_free = bars + 10;
   uint64_t* dq_full = bars + 11;
@@ -165,8 +167,7 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 14; ++i) {
-      const bool many = bars + i == s_free || bars + i == dp_free || bars + i == p_ready ||
-                        bars + i == ds_ready;
+      const bool many = bars + i == dp_free || bars + i == p_ready || bars + i == ds_ready;
       mbar_init(bars + i, many ? 128 : 1);
     }
     *abort = 0;
@@ -203,22 +204,24 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         bool stu;
         vis.get(v, hg, qt, stu);
         const int h = hk * G + hg;
-        if (!mbar_wait(qdo_empty, (v & 1) ^ 1, st, abort)) break;
-        mbar_arrive_expect_tx(qdo_full, 2 * LOAD_BYTES);
+        const int sg = v & 1;
+        if (!mbar_wait(&qdo_empty[sg], ((v >> 1) & 1) ^ 1, st, abort)) break;
+        mbar_arrive_expect_tx(&qdo_full[sg], 2 * LOAD_BYTES);
         const CUtensorMap* mdo = stu ? &mapDOS : &mapDOT;
 #pragma unroll
         for (int p = 0; p < Cfg::PANELS; ++p) {
-          tma_load_2d(smem + Cfg::Q_OFF + p * PANEL, &mapQ, qdo_full, h * HD + 64 * p,
-                      row_base + qt * ATT_BM);
-          tma_load_2d(smem + Cfg::DO_OFF + p * PANEL, mdo, qdo_full, h * HD + 64 * p,
-                      row_base + qt * ATT_BM);
+          tma_load_2d(smem + Cfg::Q_OFF + sg * Cfg::TILE + p * PANEL, &mapQ, &qdo_full[sg],
+                      h * HD + 64 * p, row_base + qt * ATT_BM);
+          tma_load_2d(smem + Cfg::DO_OFF + sg * Cfg::TILE + p * PANEL, mdo, &qdo_full[sg],
+                      h * HD + 64 * p, row_base + qt * ATT_BM);
         }
         ++issued;
       }
       // every load issued lands before the CTA can exit
       volatile int no_abort = 0;
       mbar_wait(kv_full, 0, st, &no_abort);
-      if (issued > 0) mbar_wait(qdo_full, (issued - 1) & 1, st, &no_abort);
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait(&qdo_full[j & 1], (j >> 1) & 1, st, &no_abort);
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
@@ -226,13 +229,13 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
       const uint32_t v_lo = sdesc_lo(smem_u32(smem + Cfg::V_OFF), 16);
       const uint32_t q_lo = sdesc_lo(smem_u32(smem + Cfg::Q_OFF), 16);
       const uint32_t do_lo = sdesc_lo(smem_u32(smem + Cfg::DO_OFF), 16);
-      const uint32_t pt_lo = sdesc_lo(smem_u32(smem + Cfg::PT_OFF), 16);
       const uint32_t ds_lo = sdesc_lo(smem_u32(smem + Cfg::DS_OFF), 16);
       // MN-major views: leading byte offset = one 64-column panel
       const uint32_t q_mn = sdesc_lo(smem_u32(smem + Cfg::Q_OFF), PANEL);
       const uint32_t do_mn = sdesc_lo(smem_u32(smem + Cfg::DO_OFF), PANEL);
       const uint32_t k_mn = sdesc_lo(smem_u32(smem + Cfg::K_OFF), PANEL);
       const uint32_t ds_mn = sdesc_lo(smem_u32(smem + Cfg::DS_OFF), PANEL);
+      constexpr uint32_t STAGE = Cfg::TILE >> 4;  // descriptor step of one Q / dO stage
       // K-major step kk of 16 elements: panel kk/4, 32 bytes within the row
       auto koff = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * PANEL + (kk & 3) * 32) >> 4); };
       // MN-major step kk of 16 rows: 16 x 128 bytes
@@ -240,54 +243,72 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
       };
-      bool ok = wait(kv_full, 0);
-      for (int v = 0; v < nv && ok; ++v) {
-        const uint32_t ph = v & 1;
-        if (!wait(qdo_full, ph) || !wait(s_free, ph ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        if (elect_one()) {  // S^T = K Q^T
+      auto issue_s = [&](int v) {  // S^T = K Q^T
+        const uint32_t qs = q_lo + (v & 1) * STAGE;
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
-            mma_bf16_ss_lh(tmem, k_lo + koff(kk), HI, q_lo + koff(kk), HI, ID_SS, kk > 0 ? 1u : 0u);
+            mma_bf16_ss_lh(tmem, k_lo + koff(kk), HI, qs + koff(kk), HI, ID_SS, kk > 0 ? 1u : 0u);
           mma_commit(s_full);
         }
         __syncwarp();
-        if (!wait(dp_free, ph ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        if (elect_one()) {  // dP^T = V dO^T
+      };
+      auto issue_dp = [&](int v) {  // dP^T = V dO^T
+        const uint32_t ds_ = do_lo + (v & 1) * STAGE;
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
-            mma_bf16_ss_lh(tmem + 128, v_lo + koff(kk), HI, do_lo + koff(kk), HI, ID_SS,
+            mma_bf16_ss_lh(tmem + 128, v_lo + koff(kk), HI, ds_ + koff(kk), HI, ID_SS,
                            kk > 0 ? 1u : 0u);
           mma_commit(dp_full);
         }
         __syncwarp();
+      };
+      bool ok = wait(kv_full, 0) && wait(&qdo_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int v = 0; v < nv && ok; ++v) {
+        const uint32_t ph = v & 1;
+        const int sg = v & 1;
+        const bool more = v + 1 < nv;
         if (!wait(p_ready, ph)) { ok = false; break; }
         tc_fence_after();
-        if (elect_one()) {  // dV += P^T dO
+        if (elect_one()) {  // dV += P^T dO, P^T from TMEM
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss_lh(tmem + 256 + HD, pt_lo + koff(kk), HI, do_mn + moff(kk), HI, ID_KB,
-                           (v > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(pt_free);
+            mma_bf16_ts_lh(tmem + 256 + HD, tmem + kk * 8, do_mn + sg * STAGE + moff(kk), HI,
+                           ID_KB, (v > 0 || kk > 0) ? 1u : 0u);
         }
         __syncwarp();
+        if (more) {  // the next visit's scores, behind dV in the tensor pipe
+          if (!wait(&qdo_full[(v + 1) & 1], ((v + 1) >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(v + 1);
+        }
         if (!wait(ds_ready, ph)) { ok = false; break; }
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-            mma_bf16_ss_lh(tmem + 256, ds_lo + koff(kk), HI, q_mn + moff(kk), HI, ID_KB,
-                           (v > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss_lh(tmem + 256, ds_lo + koff(kk), HI, q_mn + sg * STAGE + moff(kk), HI,
+                           ID_KB, (v > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // dQ = dS K, into the dP^T columns
             mma_bf16_ss_lh(tmem + 128, ds_mn + moff(kk), HI, k_mn + moff(kk), HI, ID_MM,
                            kk > 0 ? 1u : 0u);
           mma_commit(dq_full);
           mma_commit(dst_free);
-          mma_commit(qdo_empty);
+          mma_commit(&qdo_empty[sg]);
         }
         __syncwarp();
+        if (more) {  // the next dP^T once dQ(v) has left its columns
+          if (!wait(dp_free, ph)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(v + 1);
+        }
       }
       if (elect_one()) {
         mma_commit(kv_done);
@@ -306,7 +327,6 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_off;
     const uint32_t dp_addr = tmem + lane_off + 128;
-    uint8_t* pt_tile = smem + Cfg::PT_OFF;
     uint8_t* ds_tile = smem + Cfg::DS_OFF;
     const float LOG2E = 1.4426950408889634f;
     bool ok = true;
@@ -349,12 +369,11 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
           P[c >> 1] = pack_bf16x2(p0, p1);
         }
       }
+      // P^T over the first 64 columns of this row's S^T (the A operand of dV)
+      tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&P[0]));
+      tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&P[32]));
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(s_free);
-      if (!mbar_wait(pt_free, ph ^ 1, st, abort)) { ok = false; continue; }
-      st_tile_row(pt_tile, 0, r, &P[0]);
-      st_tile_row(pt_tile, 1, r, &P[32]);
-      fence_async_smem();
       mbar_arrive(p_ready);
       // dS^T = P^T (dP^T - delta) scale
       if (!mbar_wait(dp_full, ph, st, abort)) { ok = false; continue; }

@@ -669,8 +669,9 @@ struct EpiSwiGLU {
 //      two tiles alternate by slice);
 //   B  thread (row R, column group cg of 8 columns) forms the causal depthwise
 //      convs of both paths from the k rows R - k + 1 .. R of the tile (16-byte
-//      shared loads; the taps of its 8 columns come as fp32 from a table
-//      [path][f/8][KMAX][8] made once per call), and writes 8 columns of
+//      shared loads; the taps of its 8 columns come from a bf16 table
+//      [path][f/8][KMAX][8] made once per call, loaded at the start of the
+//      slice so that they arrive during phase A), and writes 8 columns of
 //      D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and of the
 //      bf16 Z_S (output-GEMM operand) with one 16-byte store each.  The row's
 //      padded index is formed once per tile.  Kp^2 accumulates per row over the
@@ -690,7 +691,7 @@ struct EpiSwiGLUConv {
   __nv_bfloat16* Zs;
   float* ssq;          // [ceil(f/128), P]
   const float* rstd;   // [2BT] MLP RMSNorm row scales, nullable (u already normalised)
-  const float* taps;   // [2][f/8][KMAX][8] fp32: conv_T then conv_S, tap m of column 8c + i
+  const __nv_bfloat16* taps;  // [2][f/8][KMAX][8]: conv_T then conv_S, tap m of column 8c + i
   const float* z_halo;
   float* z_tail;
   int B, T, f, k, C, Cp, Nc;
@@ -732,6 +733,18 @@ struct EpiSwiGLUConv {
       const int col0 = c.tn * 128 + cc;
       if (col0 >= f) break;  // the same for every warp
       uint8_t* tile = tiles + (s & 1) * 16384;
+      // phase B's taps (8 columns x k per path, one 16-byte word per tap), loaded
+      // now so that they arrive during phase A
+      uint4 tw[2][KMAX];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(taps) + static_cast<long long>((col0 >> 3) + cg) * KMAX;
+#pragma unroll
+        for (int m = 0; m < KMAX; ++m) {
+          tw[0][m] = m < k ? __ldg(src + m) : make_uint4(0u, 0u, 0u, 0u);
+          tw[1][m] = m < k ? __ldg(src + static_cast<long long>(f / 8) * KMAX + m)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       // ---- A: z of this row, 16 columns
       {
         const int ch = cc + 16 * half;  // first column of this half within the tile
@@ -777,8 +790,6 @@ struct EpiSwiGLUConv {
       // ---- B: the convs of row brow, columns col0 + 8 cg .. + 7, both paths
       {
         const int col = col0 + 8 * cg;
-        const float* tT = taps + (static_cast<long long>(col >> 3) * KMAX) * 8;
-        const float* tS = tT + static_cast<long long>(f) * KMAX;
         float aT[8], aS[8], z0[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) { aT[i] = 0.f; aS[i] = 0.f; z0[i] = 0.f; }
@@ -786,8 +797,17 @@ struct EpiSwiGLUConv {
         for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
           if (m >= k || brow - m < 0) break;
           float wT[8], wS[8], zt[8], zs[8];
-          ld8f(tT + m * 8, wT);
-          ld8f(tS + m * 8, wS);
+          {
+            const uint32_t uT[4] = {tw[0][m].x, tw[0][m].y, tw[0][m].z, tw[0][m].w};
+            const uint32_t uS[4] = {tw[1][m].x, tw[1][m].y, tw[1][m].z, tw[1][m].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              wT[2 * i] = bf16lo_to_f32(uT[i]);
+              wT[2 * i + 1] = bf16hi_to_f32(uT[i]);
+              wS[2 * i] = bf16lo_to_f32(uS[i]);
+              wS[2 * i + 1] = bf16hi_to_f32(uS[i]);
+            }
+          }
           const int RT = brow - m, RS = 64 + brow - m;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -828,12 +848,12 @@ struct EpiSwiGLUConv {
   }
 };
 
-// taps[path][c / 8][m][c % 8] = conv_path[c, m] (fp32, zero for m >= k): the
-// table the gate/up conv epilogue reads, 8 columns of one tap per 32 bytes.
+// taps[path][c / 8][m][c % 8] = conv_path[c, m] (bf16, zero for m >= k): the
+// table the gate/up conv epilogue reads, 8 columns of one tap per 16 bytes.
 template <int KMAX>
 __global__ void conv_tap_table_kernel(const __nv_bfloat16* __restrict__ conv_T,
                                       const __nv_bfloat16* __restrict__ conv_S,
-                                      float* __restrict__ taps, int f, int k) {
+                                      __nv_bfloat16* __restrict__ taps, int f, int k) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= 2 * f * KMAX) return;
   const int path = idx / (f * KMAX);
@@ -841,7 +861,7 @@ __global__ void conv_tap_table_kernel(const __nv_bfloat16* __restrict__ conv_T,
   const int c8 = e / (KMAX * 8), m = (e / 8) % KMAX, ci = e % 8;
   const int col = c8 * 8 + ci;
   const __nv_bfloat16* w = path ? conv_S : conv_T;
-  taps[idx] = m < k ? __bfloat162float(w[static_cast<long long>(col) * k + m]) : 0.f;
+  taps[idx] = m < k ? w[static_cast<long long>(col) * k + m] : __float2bfloat16_rn(0.f);
 }
 
 // QKV projection with rotary embedding on the query and key heads, written to

@@ -307,7 +307,7 @@ Layout make_layout(const ttcd_block_params* p, bool block, bool shard = false,
   sz[B_U] = 2 * m.BT * m.d * e;
   sz[B_Z] = e == 4 ? 2 * m.BT * m.f * 4 : 0;  // bf16: Z stays on chip (fused gate/up + conv)
   sz[B_ZS16] = e == 2 ? m.BT * m.f * 2 : 0;  // fp32 mode reads Z_S directly
-  sz[B_TAPS] = e == 2 ? 2 * static_cast<size_t>(m.f) * 8 * 4 : 0;  // fp32 conv tap table
+  sz[B_TAPS] = e == 2 ? 2 * static_cast<size_t>(m.f) * 8 * 2 : 0;  // bf16 conv tap table
   sz[B_D] = m.P * m.f * e;
   sz[B_KP] = m.P * m.f * e;
   sz[B_SSQ] = m.P * 4 * (m.f / 64);
@@ -478,7 +478,7 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
     g.tiles_m = cdiv(p->T, 64 - H);
     g.tiles_n = cdiv(m.f, 128);
     g.half_rows = m.BT;
-    float* taps = at<float>(ws, L, B_TAPS);
+    __nv_bfloat16* taps = at<__nv_bfloat16>(ws, L, B_TAPS);
     if (p->conv_k <= 4) {
       conv_tap_table_kernel<4><<<cdiv(2 * m.f * 4, 256), 256, 0, c.s>>>(conv_T, conv_S, taps, m.f,
                                                                         p->conv_k);
