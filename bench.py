@@ -461,6 +461,8 @@ def run_ours(args, world, rank, local):
         line["stack"] = [measure_stack(args, world, local, B, T, steps=max(2, args.extra_steps // 2),
                                        warmup=args.extra_warmup)
                          for B, T in ((1, 65536), (4, 16384))]
+        # the backward kernels at the same block shape (B 1, T 65536)
+        line["backward"] = measure_backward(args, local, 1, shape.T, steps=3, warmup=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, times = oracle_throughput(shape, args.cpu_sample_tokens)
         line["cpu_baseline"] = {
@@ -622,7 +624,15 @@ def window_pairs(T: int, w: int) -> int:
 
 
 def run_backward(args, world, rank, local):
-    """The backward kernels at the Qwen3-0.6B block shape (T = --T, B = --B):
+    """`--mode backward`: one JSON line per backward kernel."""
+    lines = measure_backward(args, local, args.B, args.T, args.steps, args.warmup)
+    if rank == 0:
+        for l in lines:
+            print(json.dumps(l), flush=True)
+
+
+def measure_backward(args, local, B_, T_, steps, warmup):
+    """The backward kernels at the Qwen3-0.6B block shape (B_ x T_):
     ttcd_fastweight_mlp_backward (the forward's front half and chunk scan
     recomputed inside) and ttcd_dual_window_attn_backward, each timed alone with
     CUDA events.  FLOPs are the algorithmic contractions of each call."""
@@ -630,7 +640,7 @@ def run_backward(args, world, rank, local):
     from ttcd_workloads import make_mlp_inputs
     ttcd.load_library()
     peaks, peak_kind = load_peaks()
-    shape = QWEN3_0P6B_64K.with_(name=f"qwen3_0.6b_backward_T{args.T}", B=args.B, T=args.T)
+    shape = QWEN3_0P6B_64K.with_(name=f"qwen3_0.6b_backward_T{T_}", B=B_, T=T_)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     B, T, d, f = shape.B, shape.T, shape.d_model, shape.d_ff
@@ -660,7 +670,7 @@ def run_backward(args, world, rank, local):
     p = ttcd.BlockParams.from_shape(shape)
     _, ws = ttcd.fastweight_mlp_backward(w["u_T"], w["u_S"], w["beta"], w, p, d_y)
     ms = timed(lambda: ttcd.fastweight_mlp_backward(w["u_T"], w["u_S"], w["beta"], w, p, d_y,
-                                                    workspace=ws), args.steps, args.warmup)
+                                                    workspace=ws), steps, warmup)
     if ttcd.check_device_status(ws) != ttcd.OK:
         raise RuntimeError("a device wait timed out in the MLP backward")
     recompute = 2 * 2 * BT * 2 * f * d + 2 * d * f * f + 2 * 2 * P * f * d
@@ -681,7 +691,7 @@ def run_backward(args, world, rank, local):
                                                   shape.w_S, shape.w_T)
     ms = timed(lambda: ttcd.dual_window_attn_backward(q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S,
                                                       shape.w_S, shape.w_T, workspace=aws),
-               args.steps, args.warmup)
+               steps, warmup)
     if ttcd.check_device_status(aws) != ttcd.OK:
         raise RuntimeError("a device wait timed out in the attention backward")
     # per visible pair and head: S recomputed, dP, dV, dK, dQ (2 hd FLOPs each)
@@ -689,14 +699,15 @@ def run_backward(args, world, rank, local):
     flops = 10.0 * hd * pairs
     lines.append({"kernel": "ttcd_dual_window_attn_backward", "ms": ms, "flops": flops,
                   "tflops_per_s": flops / ms / 1e9})
-    if rank == 0:
-        for l in lines:
-            l.update({"metric": "backward kernel time (Qwen3-0.6B block shape)",
-                      "config": workload_config(shape), "steps": args.steps,
-                      "warmup": args.warmup, "peak_tflops": peaks["bf16_tflops"],
-                      "frac": l["tflops_per_s"] / peaks["bf16_tflops"],
-                      "peak_source": f"{peak_kind} bf16_tflops"})
-            print(json.dumps(l), flush=True)
+    for l in lines:
+        l.update({"metric": "backward kernel time (Qwen3-0.6B block shape)",
+                  "config": workload_config(shape), "steps": steps, "warmup": warmup,
+                  "peak_tflops": peaks["bf16_tflops"],
+                  "frac": l["tflops_per_s"] / peaks["bf16_tflops"],
+                  "peak_source": f"{peak_kind} bf16_tflops"})
+    del q, k, v, o_T, o_S, lse_T, lse_S, do_T, do_S, aws
+    torch.cuda.empty_cache()
+    return lines
 
 
 def measure_stack(args, world, local, B, T, steps, warmup):
@@ -791,7 +802,7 @@ def main():
     ap.add_argument("--attn-traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture")
     ap.add_argument("--no-extras", action="store_true",
-                    help="block mode: skip the attention sweep and the 28-layer stack")
+                    help="block mode: skip the attention sweep, the 28-layer stack and the backward kernels")
     ap.add_argument("--extra-steps", type=int, default=5,
                     help="timed calls per attention window pair / stack shape")
     ap.add_argument("--extra-warmup", type=int, default=3)

@@ -20,7 +20,9 @@
 // visit is added to the fp32 dq in global memory (vector atomics).
 //
 // Pipeline (one CTA, 384 threads):
-//   warp 0      TMA producer: K and V once, then Q and dO per visit (two stages)
+//   warp 0      TMA producer: K and V once, then per visit Q with the visit's
+//               128 rows of lse (base 2) and delta (two stages; Q is last read
+//               by dK), and dO (one stage; last read by dV, early in the visit)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one thread), per visit v:
 //               dV(v), S(v+1), dK(v) dQ(v), dP(v+1), so that the next visit's
 //               scores form while the key-row threads work on dS(v)
@@ -33,7 +35,7 @@
 // [256+HD, 256+2HD).  The tensor pipe runs one CTA's MMAs in issue order, so
 // S(v+1) overwrites P^T(v) only after dV(v) has read it.
 // Shared memory operands (128-byte swizzle, 64-column panels of 128 rows):
-// K, V, and two stages of Q and dO as loaded by TMA; dS^T written by the
+// K, V, two stages of Q and one of dO as loaded by TMA; dS^T written by the
 // key-row threads.  The same tile is read K-major or MN-major by choosing the
 // descriptor: Q is the B operand of S^T (K-major) and of dK (MN-major), dS^T is
 // the A operand of dK (K-major) and, read as dS, of dQ (MN-major).
@@ -46,9 +48,10 @@ struct AttnBwdArgs {
   float* dq;  // [B, T, Hq, HD], accumulated (zeroed by the caller)
   float* dk;  // [B, T, Hkv, HD]
   float* dv;
-  const float* lse_T;    // [B, Hq, T]
-  const float* lse_S;
-  const float* delta_T;  // [B, Hq, T]
+  // per (b, h) rows of Tp = n_kt * 128 floats, padded past T (lse2 +inf, delta 0):
+  const float* lse2_T;   // log2(e) lse_T
+  const float* lse2_S;
+  const float* delta_T;  // rowsum(dO_T o_T)
   const float* delta_S;
   int B, T, Hq, Hkv;
   int w_S, w_T;
@@ -68,11 +71,11 @@ struct AttnBwdCfg {
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
   static constexpr int Q_OFF = V_OFF + TILE;       // two stages
-  static constexpr int DO_OFF = Q_OFF + 2 * TILE;  // two stages
-  static constexpr int DS_OFF = DO_OFF + 2 * TILE;
-  static constexpr int LSE_OFF = DS_OFF + DS_TILE;  // 128 floats
-  static constexpr int DEL_OFF = LSE_OFF + 512;     // 128 floats
-  static constexpr int BAR_OFF = DEL_OFF + 512;
+  static constexpr int DO_OFF = Q_OFF + 2 * TILE;  // one stage
+  static constexpr int DS_OFF = DO_OFF + TILE;
+  static constexpr int LSE_OFF = DS_OFF + DS_TILE;  // 2 stages of 128 floats
+  static constexpr int DEL_OFF = LSE_OFF + 1024;    // 2 stages of 128 floats
+  static constexpr int BAR_OFF = DEL_OFF + 1024;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
 };
 
@@ -92,22 +95,6 @@ struct BwdVisits {
     qt = kt + (student ? u - nT : u);
   }
 };
-
-// Named barrier 2 over the 128 key-row threads, and-reducing a flag: every
-// thread reaches it each visit (a failed wait only clears its flag), so the
-// threads leave the visit loop together.
-__device__ __forceinline__ bool key_rows_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 2, 128, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(v ? 1u : 0u)
-      : "memory");
-  return r != 0;
-}
 
 // One 128-byte row of a P^T / dS^T tile: 64 bf16 (32 packed words) of row r in
 // panel `panel`, 16-byte chunks placed by the 128-byte swizzle.
@@ -137,22 +124,22 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* lse2 = reinterpret_cast<float*>(smem + Cfg::LSE_OFF);
-  float* dlt = reinterpret_cast<float*>(smem + Cfg::DEL_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qdo_full = bars + 1;   // 2 stages
-  uint64_t* qdo_empty = bars + 3;  // 2 stages
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* dp_free = bars + 7;   // 128 arrivals
-  uint64_t* p_ready = bars + 8;   // 128 arrivals
-  uint64_t* ds_ready = bars + 9;  // 128 arrivals
-  uint64_t* dst_free = bars + 10;
-  uint64_t* dq_full = bars + 11;
-  uint64_t* kv_done = bars + 12;
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* q_full = bars + 1;    // 2 stages (Q, lse2, delta)
+  uint64_t* q_empty = bars + 3;   // 2 stages
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;
+  uint64_t* s_full = bars + 7;
+  uint64_t* dp_full = bars + 8;
+  uint64_t* dp_free = bars + 9;   // 128 arrivals
+  uint64_t* p_ready = bars + 10;  // 128 arrivals
+  uint64_t* ds_ready = bars + 11; // 128 arrivals
+  uint64_t* dst_free = bars + 12;
+  uint64_t* dq_full = bars + 13;
+  uint64_t* kv_done = bars + 14;
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -166,7 +153,7 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
   const int nv = G * vis.per_head();
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 14; ++i) {
+    for (int i = 0; i < 16; ++i) {
       const bool many = bars + i == dp_free || bars + i == p_ready || bars + i == ds_ready;
       mbar_init(bars + i, many ? 128 : 1);
     }
@@ -198,30 +185,40 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         tma_load_2d(smem + Cfg::K_OFF + p * PANEL, &mapK, kv_full, hk * HD + 64 * p, row_base + k0);
         tma_load_2d(smem + Cfg::V_OFF + p * PANEL, &mapV, kv_full, hk * HD + 64 * p, row_base + k0);
       }
-      int issued = 0;
+      int issued = 0, issued_do = 0;
       for (int v = 0; v < nv; ++v) {
         int hg, qt;
         bool stu;
         vis.get(v, hg, qt, stu);
         const int h = hk * G + hg;
         const int sg = v & 1;
-        if (!mbar_wait(&qdo_empty[sg], ((v >> 1) & 1) ^ 1, st, abort)) break;
-        mbar_arrive_expect_tx(&qdo_full[sg], 2 * LOAD_BYTES);
+        if (!mbar_wait(&q_empty[sg], ((v >> 1) & 1) ^ 1, st, abort)) break;
+        mbar_arrive_expect_tx(&q_full[sg], LOAD_BYTES + 2 * 512);
+#pragma unroll
+        for (int p = 0; p < Cfg::PANELS; ++p)
+          tma_load_2d(smem + Cfg::Q_OFF + sg * Cfg::TILE + p * PANEL, &mapQ, &q_full[sg],
+                      h * HD + 64 * p, row_base + qt * ATT_BM);
+        const long long li = (static_cast<long long>(b) * a.Hq + h) * (a.n_kt * ATT_BM) + qt * ATT_BM;
+        bulk_load(smem + Cfg::LSE_OFF + sg * 512, (stu ? a.lse2_S : a.lse2_T) + li, 512,
+                  &q_full[sg]);
+        bulk_load(smem + Cfg::DEL_OFF + sg * 512, (stu ? a.delta_S : a.delta_T) + li, 512,
+                  &q_full[sg]);
+        if (!mbar_wait(do_empty, (v & 1) ^ 1, st, abort)) { ++issued; break; }
+        mbar_arrive_expect_tx(do_full, LOAD_BYTES);
         const CUtensorMap* mdo = stu ? &mapDOS : &mapDOT;
 #pragma unroll
-        for (int p = 0; p < Cfg::PANELS; ++p) {
-          tma_load_2d(smem + Cfg::Q_OFF + sg * Cfg::TILE + p * PANEL, &mapQ, &qdo_full[sg],
-                      h * HD + 64 * p, row_base + qt * ATT_BM);
-          tma_load_2d(smem + Cfg::DO_OFF + sg * Cfg::TILE + p * PANEL, mdo, &qdo_full[sg],
-                      h * HD + 64 * p, row_base + qt * ATT_BM);
-        }
+        for (int p = 0; p < Cfg::PANELS; ++p)
+          tma_load_2d(smem + Cfg::DO_OFF + p * PANEL, mdo, do_full, h * HD + 64 * p,
+                      row_base + qt * ATT_BM);
+        ++issued_do;
         ++issued;
       }
       // every load issued lands before the CTA can exit
       volatile int no_abort = 0;
       mbar_wait(kv_full, 0, st, &no_abort);
       for (int j = max(0, issued - 2); j < issued; ++j)
-        mbar_wait(&qdo_full[j & 1], (j >> 1) & 1, st, &no_abort);
+        mbar_wait(&q_full[j & 1], (j >> 1) & 1, st, &no_abort);
+      if (issued_do > 0) mbar_wait(do_full, (issued_do - 1) & 1, st, &no_abort);
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
@@ -254,7 +251,8 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         __syncwarp();
       };
       auto issue_dp = [&](int v) {  // dP^T = V dO^T
-        const uint32_t ds_ = do_lo + (v & 1) * STAGE;
+        const uint32_t ds_ = do_lo;
+        (void)v;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
@@ -264,11 +262,15 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         }
         __syncwarp();
       };
-      bool ok = wait(kv_full, 0) && wait(&qdo_full[0], 0);
+      bool ok = wait(kv_full, 0) && wait(&q_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        issue_dp(0);
+        ok = wait(do_full, 0);
+        if (ok) {
+          tc_fence_after();
+          issue_dp(0);
+        }
       }
       for (int v = 0; v < nv && ok; ++v) {
         const uint32_t ph = v & 1;
@@ -279,12 +281,13 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         if (elect_one()) {  // dV += P^T dO, P^T from TMEM
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts_lh(tmem + 256 + HD, tmem + kk * 8, do_mn + sg * STAGE + moff(kk), HI,
-                           ID_KB, (v > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts_lh(tmem + 256 + HD, tmem + kk * 8, do_mn + moff(kk), HI, ID_KB,
+                           (v > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(do_empty);  // dO(v) is read for the last time
         }
         __syncwarp();
         if (more) {  // the next visit's scores, behind dV in the tensor pipe
-          if (!wait(&qdo_full[(v + 1) & 1], ((v + 1) >> 1) & 1)) { ok = false; break; }
+          if (!wait(&q_full[(v + 1) & 1], ((v + 1) >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_s(v + 1);
         }
@@ -301,11 +304,11 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
                            kk > 0 ? 1u : 0u);
           mma_commit(dq_full);
           mma_commit(dst_free);
-          mma_commit(&qdo_empty[sg]);
+          mma_commit(&q_empty[sg]);
         }
         __syncwarp();
         if (more) {  // the next dP^T once dQ(v) has left its columns
-          if (!wait(dp_free, ph)) { ok = false; break; }
+          if (!wait(dp_free, ph) || !wait(do_full, (v + 1) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_dp(v + 1);
         }
@@ -328,32 +331,21 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
     const uint32_t s_addr = tmem + lane_off;
     const uint32_t dp_addr = tmem + lane_off + 128;
     uint8_t* ds_tile = smem + Cfg::DS_OFF;
-    const float LOG2E = 1.4426950408889634f;
     bool ok = true;
     for (int v = 0; v < nv; ++v) {
       const uint32_t ph = v & 1;
       int hg, qt;
       bool stu;
       vis.get(v, hg, qt, stu);
-      const int h = hk * G + hg;
       const int q0 = qt * ATT_BM;
       const int w = stu ? a.w_S : a.w_T;
-      // every thread has finished the previous visit (and its reads of lse2 and
-      // dlt); all leave together if a wait anywhere gave up
-      ok = key_rows_and(ok);
-      if (!ok) break;
-      // this visit's log-sum-exp (base 2) and delta per query column
-      {
-        const int t = q0 + r;
-        const long long li = (static_cast<long long>(b) * a.Hq + h) * a.T + t;
-        const bool in = t < a.T;
-        lse2[r] = in ? (stu ? a.lse_S : a.lse_T)[li] * LOG2E : INFINITY;
-        dlt[r] = in ? (stu ? a.delta_S : a.delta_T)[li] : 0.f;
-      }
-      asm volatile("bar.sync 2, 128;" ::: "memory");
+      // this visit's lse (base 2) and delta per query column, copied with Q and dO
+      if (!mbar_wait(&q_full[v & 1], (v >> 1) & 1, st, abort)) { ok = false; break; }
+      const float* lse2 = reinterpret_cast<const float*>(smem + Cfg::LSE_OFF + (v & 1) * 512);
+      const float* dlt = reinterpret_cast<const float*>(smem + Cfg::DEL_OFF + (v & 1) * 512);
       // visible query columns of key j: c - lo in [0, w - 1], lo = j - q0
       const int lo = j - q0;
-      if (!mbar_wait(s_full, ph, st, abort)) { ok = false; continue; }
+      if (!mbar_wait(s_full, ph, st, abort)) { ok = false; break; }
       tc_fence_after();
       uint32_t P[64];
 #pragma unroll
@@ -376,7 +368,7 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
       tc_fence_before();
       mbar_arrive(p_ready);
       // dS^T = P^T (dP^T - delta) scale
-      if (!mbar_wait(dp_full, ph, st, abort)) { ok = false; continue; }
+      if (!mbar_wait(dp_full, ph, st, abort)) { ok = false; break; }
       tc_fence_after();
       uint32_t D[64];
 #pragma unroll
@@ -393,7 +385,7 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
         }
       }
       tc_fence_before();
-      if (!mbar_wait(dst_free, ph ^ 1, st, abort)) { ok = false; continue; }
+      if (!mbar_wait(dst_free, ph ^ 1, st, abort)) { ok = false; break; }
       st_tile_row(ds_tile, 0, r, &D[0]);
       st_tile_row(ds_tile, 1, r, &D[32]);
       fence_async_smem();
@@ -449,19 +441,35 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
   }
 }
 
-// delta[b, h, t] = sum_d dO[b, t, h, d] O[b, t, h, d] (fp32) for both windows:
-// one thread per (window, row), 8 elements per load.
+// Per (b, h) row of Tp floats, both windows: delta[t] = sum_d dO[b, t, h, d]
+// O[b, t, h, d] and lse2[t] = log2(e) lse[b, h, t] for t < T; past T, delta 0 and
+// lse2 +inf (so that the rebuilt P is 0 there).  One thread per (window, b, h, t).
 template <int HD>
-__global__ void attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o_T,
-                                      const __nv_bfloat16* __restrict__ o_S,
-                                      const __nv_bfloat16* __restrict__ do_T,
-                                      const __nv_bfloat16* __restrict__ do_S,
-                                      float* __restrict__ delta_T, float* __restrict__ delta_S,
-                                      int T, int Hq, long long rows) {
+__global__ void attn_bwd_rows_kernel(const __nv_bfloat16* __restrict__ o_T,
+                                     const __nv_bfloat16* __restrict__ o_S,
+                                     const __nv_bfloat16* __restrict__ do_T,
+                                     const __nv_bfloat16* __restrict__ do_S,
+                                     const float* __restrict__ lse_T,
+                                     const float* __restrict__ lse_S, float* __restrict__ delta_T,
+                                     float* __restrict__ delta_S, float* __restrict__ lse2_T,
+                                     float* __restrict__ lse2_S, int T, int Tp, int Hq,
+                                     long long rows) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= 2 * rows) return;
-  const bool stu = idx >= rows;
-  const long long row = stu ? idx - rows : idx;  // (b, t, h) row-major
+  if (idx >= 2 * rows * Tp) return;
+  const bool stu = idx >= rows * Tp;
+  const long long e = stu ? idx - rows * Tp : idx;
+  const int t = static_cast<int>(e % Tp);
+  const long long bh = e / Tp;  // b * Hq + h
+  float* delta = stu ? delta_S : delta_T;
+  float* lse2 = stu ? lse2_S : lse2_T;
+  if (t >= T) {
+    delta[e] = 0.f;
+    lse2[e] = INFINITY;
+    return;
+  }
+  const long long b = bh / Hq;
+  const int h = static_cast<int>(bh % Hq);
+  const long long row = (b * T + t) * Hq + h;  // (b, t, h) row of o and dO
   const __nv_bfloat16* o = (stu ? o_S : o_T) + row * HD;
   const __nv_bfloat16* g = (stu ? do_S : do_T) + row * HD;
   float s = 0.f;
@@ -473,11 +481,8 @@ __global__ void attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o_T,
 #pragma unroll
     for (int i = 0; i < 8; ++i) s = fmaf(x[i], y[i], s);
   }
-  const int h = static_cast<int>(row % Hq);
-  const long long bt = row / Hq;
-  const int t = static_cast<int>(bt % T);
-  const long long b = bt / T;
-  (stu ? delta_S : delta_T)[(b * Hq + h) * T + t] = s;
+  delta[e] = s;
+  lse2[e] = (stu ? lse_S : lse_T)[bh * T + t] * 1.4426950408889634f;
 }
 
 }  // namespace ttcd

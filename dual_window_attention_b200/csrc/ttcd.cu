@@ -2092,9 +2092,14 @@ ttcd_status ttcd_fastweight_mlp_backward(const void* u_T, const void* u_S, const
 // ================================================================== attention backward
 namespace {
 
+// status word, then delta_T, delta_S, lse2_T, lse2_S: [B Hq][Tp] fp32 each,
+// Tp = T rounded up to the 128-query tile.
+size_t attn_bwd_rows_bytes(int B, int T, int Hq) {
+  const size_t Tp = static_cast<size_t>(T + ATT_BM - 1) / ATT_BM * ATT_BM;
+  return (static_cast<size_t>(B) * Hq * Tp * 4 + 1023) / 1024 * 1024;
+}
 size_t attn_bwd_ws_bytes(int B, int T, int Hq) {
-  const size_t rows = static_cast<size_t>(B) * Hq * T * 4;
-  return kStatusBytes + 2 * ((rows + 1023) / 1024 * 1024);
+  return kStatusBytes + 4 * attn_bwd_rows_bytes(B, T, Hq);
 }
 
 // q rows have ld_q elements between tokens, k and v rows ld_kv (as launch_attn);
@@ -2107,16 +2112,21 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
                             int w_T, float scale, void* ws, long long ld_q, long long ld_kv) {
   using bf = __nv_bfloat16;
   const long long BT = static_cast<long long>(B) * T;
-  const size_t rows_bytes = (static_cast<size_t>(B) * Hq * T * 4 + 1023) / 1024 * 1024;
+  const size_t rows_bytes = attn_bwd_rows_bytes(B, T, Hq);
   float* delta_T = dat<float>(ws, kStatusBytes);
   float* delta_S = dat<float>(ws, kStatusBytes + rows_bytes);
+  float* lse2_T = dat<float>(ws, kStatusBytes + 2 * rows_bytes);
+  float* lse2_S = dat<float>(ws, kStatusBytes + 3 * rows_bytes);
   // dq is accumulated over the key tiles
   if (cudaMemsetAsync(dq, 0, static_cast<size_t>(BT) * Hq * HD * 4, c.s) != cudaSuccess)
     return TTCD_ERR_CUDA;
-  const long long rows = BT * Hq;
-  attn_bwd_delta_kernel<HD><<<static_cast<unsigned>(cdiv(2 * rows, 256)), 256, 0, c.s>>>(
+  const int n_kt = cdiv(T, ATT_BN);
+  const int Tp = n_kt * ATT_BN;
+  const long long rows = static_cast<long long>(B) * Hq;
+  attn_bwd_rows_kernel<HD><<<static_cast<unsigned>(cdiv(2 * rows * Tp, 256)), 256, 0, c.s>>>(
       static_cast<const bf*>(o_T), static_cast<const bf*>(o_S), static_cast<const bf*>(do_T),
-      static_cast<const bf*>(do_S), delta_T, delta_S, T, Hq, rows);
+      static_cast<const bf*>(do_S), lse_T, lse_S, delta_T, delta_S, lse2_T, lse2_S, T, Tp, Hq,
+      rows);
   TTCD_CHECK_LAUNCH();
   CUtensorMap mq, mk, mv, mdt, mds;
   const uint64_t wq = static_cast<uint64_t>(Hq) * HD, wkv = static_cast<uint64_t>(Hkv) * HD;
@@ -2130,8 +2140,8 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.lse_T = lse_T;
-  a.lse_S = lse_S;
+  a.lse2_T = lse2_T;
+  a.lse2_S = lse2_S;
   a.delta_T = delta_T;
   a.delta_S = delta_S;
   a.B = B;
@@ -2142,7 +2152,7 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
   a.w_T = w_T;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.n_kt = cdiv(T, ATT_BN);
+  a.n_kt = n_kt;
   auto kern = dual_window_attn_bwd_kernel<HD>;
   constexpr int smem = AttnBwdCfg<HD>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

@@ -151,8 +151,9 @@ ttcd_status ttcd_dual_window_attn_lse(const void* q, const void* k, const void* 
                                       int w_S, int w_T, float scale, ttcd_dtype dtype,
                                       void* stream);
 
-/* Workspace bytes of ttcd_dual_window_attn_backward (status word and the two
- * [B, Hq, T] fp32 row dot products); 0 for invalid sizes. */
+/* Workspace bytes of ttcd_dual_window_attn_backward (status word, and per
+ * window the [B, Hq, T] row dot products and base-2 log-sum-exps, padded to a
+ * multiple of 128 tokens, fp32); 0 for invalid sizes. */
 size_t ttcd_dual_window_attn_backward_workspace_size(int B, int T, int Hq);
 
 /*
