@@ -419,19 +419,19 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
       const int t = qt * ATT_BM + r;
       if (!mbar_wait(dq_full, v & 1, st, abort)) break;
       tc_fence_after();
-      float* dst = a.dq + ((static_cast<long long>(b) * a.T + t) * a.Hq + h) * HD;
+      // the whole row into registers first: the columns are free for the next
+      // dP^T as soon as they have been read, while the adds are still in flight
+      float x[HD];
 #pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        float x[32];
-        tmem_ld32f(dq_addr + c, x);
-        if (t < a.T) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            atomicAdd(reinterpret_cast<float4*>(dst + c + i), make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]));
-        }
-      }
+      for (int c = 0; c < HD; c += 32) tmem_ld32f(dq_addr + c, *reinterpret_cast<float(*)[32]>(&x[c]));
       tc_fence_before();
       mbar_arrive(dp_free);
+      if (t < a.T) {
+        float* dst = a.dq + ((static_cast<long long>(b) * a.T + t) * a.Hq + h) * HD;
+#pragma unroll
+        for (int i = 0; i < HD; i += 4)
+          atomicAdd(reinterpret_cast<float4*>(dst + i), make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]));
+      }
     }
   }
   __syncthreads();
