@@ -107,7 +107,10 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
 }
 
 // Epilogue warps of a GEMM: Epi::kWarps when the epilogue declares it (8: two
-// warps per TMEM lane quarter), else 4.  The kernel runs 2 + kWarps warps.
+// warps per TMEM lane quarter), else 4.  With 4 the kernel runs warps 0-5 (0 TMA,
+// 1 MMA, 2-5 epilogue); with 8 it runs warps 0-11, the epilogue on warps 4-11
+// (two whole warpgroups, 2-3 idle), and setmaxnreg moves registers from the
+// control warpgroup (56) to the epilogue warpgroups (224).
 template <class Epi, class = void>
 struct EpiWarps {
   static constexpr int value = 4;
@@ -117,9 +120,44 @@ struct EpiWarps<Epi, std::void_t<decltype(Epi::kWarps)>> {
   static constexpr int value = Epi::kWarps;
 };
 template <class Epi>
-constexpr int gemm_threads() {
-  return 64 + 32 * EpiWarps<Epi>::value;
+constexpr int gemm_epi_warp0() {
+  return EpiWarps<Epi>::value == 8 ? 4 : 2;
 }
+template <class Epi>
+constexpr int gemm_threads() {
+  return 32 * gemm_epi_warp0<Epi>() + 32 * EpiWarps<Epi>::value;
+}
+// Shared memory the epilogue keeps after the operand stages: Epi::kStagingBytes
+// when declared, else 4 warps x 8 KB of TMA-store staging for staged epilogues.
+template <class Epi, class = void>
+struct EpiStagingBytes {
+  static constexpr int value = Epi::kStaged ? 4 * 8192 : 0;
+};
+template <class Epi>
+struct EpiStagingBytes<Epi, std::void_t<decltype(Epi::kStagingBytes)>> {
+  static constexpr int value = Epi::kStagingBytes;
+};
+// Extra mbarriers for the epilogue's own use (Epi::kExtraBars, each initialised
+// with Epi::kExtraBarCount arrivals), and whether the epilogue releases the
+// TMEM accumulator itself (Epi::kSelfRelease: it arrives on stg.release).
+template <class Epi, class = void>
+struct EpiExtraBars {
+  static constexpr int value = 0;
+  static constexpr int count = 1;
+};
+template <class Epi>
+struct EpiExtraBars<Epi, std::void_t<decltype(Epi::kExtraBars)>> {
+  static constexpr int value = Epi::kExtraBars;
+  static constexpr int count = Epi::kExtraBarCount;
+};
+template <class Epi, class = void>
+struct EpiSelfRelease {
+  static constexpr bool value = false;
+};
+template <class Epi>
+struct EpiSelfRelease<Epi, std::void_t<decltype(Epi::kSelfRelease)>> {
+  static constexpr bool value = Epi::kSelfRelease;
+};
 
 __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -185,6 +223,9 @@ struct EpiStage {
   const CUtensorMap* map;   // first output tensor map (box: 128 bytes x 32 rows)
   const CUtensorMap* map2;  // second output tensor map (same box), when an epilogue has two
   int toggle;
+  uint64_t* xbars = nullptr;    // the epilogue's extra mbarriers
+  uint64_t* release = nullptr;  // the tile's accumulator-empty barrier (self-releasing epilogues)
+  int tiles = 0;                // tiles this thread has run (self-releasing epilogues count them)
   __device__ bool on() const { return buf != nullptr; }
   // Before writing into the current buffer: its previous store has read it.
   __device__ void acquire() {
@@ -254,8 +295,10 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* staging = smem + STAGES * STAGE_BYTES;  // 4 warps x 8 KB when STAGED
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + (STAGED ? 4 * 8192 : 0));
+  constexpr int NX = EpiExtraBars<Epi>::value;
+  uint8_t* staging = smem + STAGES * STAGE_BYTES;  // the epilogue's shared memory
+  uint64_t* xbars = reinterpret_cast<uint64_t*>(staging + EpiStagingBytes<Epi>::value);
+  uint64_t* full = xbars + NX;
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
@@ -271,6 +314,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
       tma_prefetch_map(&mapOut);
       tma_prefetch_map(&mapOut2);
     }
+    for (int i = 0; i < NX; ++i) mbar_init(&xbars[i], EpiExtraBars<Epi>::count);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -296,8 +340,13 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = geo.total();
   const int nk = (geo.K + BK - 1) / BK;
+  constexpr int EPI0 = gemm_epi_warp0<Epi>();
+  // 8 epilogue warps: the launch's 384 x 168 registers are split 128 x 56 (warps
+  // 0-3) + 256 x 224 (warps 4-11), each warp setting its limit in its own branch
+  constexpr bool SPLIT_REGS = EpiWarps<Epi>::value == 8;
 
   if (warp == 0) {
+    if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       int it = 0;
@@ -339,6 +388,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
         mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
     }
   } else if (warp == 1) {
+    if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     // ------------------------------------------------------------------ MMA issuer
     // The whole warp walks the loop (operand words stay warp-uniform) and one
     // elected lane issues; descriptor low words advance by (byte offset >> 4).
@@ -383,12 +433,16 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     __syncwarp();
     volatile int no_abort = 0;
     mbar_wait(drain, 0, st, &no_abort);
+  } else if (warp < EPI0) {
+    if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
   } else {
+    if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
     // staging slots of 8 KB per lane quarter (8-warp epilogues share them by quarter)
-    EpiStage stg{STAGED ? staging + ((warp - 2) & 3) * 8192 : nullptr, &mapOut, &mapOut2, 0};
+    EpiStage stg{STAGED ? staging + ((warp - EPI0) & 3) * 8192 : nullptr, &mapOut, &mapOut2, 0};
+    stg.xbars = xbars;
     int j = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       TileCtx c;
@@ -400,10 +454,13 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
       if constexpr (Epi::kCollective) ok = epi_bar_and<32 * EpiWarps<Epi>::value>(ok);
       if (!ok) break;
       tc_fence_after();
+      stg.release = &acce[ab];
       epi.template run<BN>(c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN, r,
                            stg, pre);
-      tc_fence_before();
-      mbar_arrive(&acce[ab]);
+      if constexpr (!EpiSelfRelease<Epi>::value) {
+        tc_fence_before();
+        mbar_arrive(&acce[ab]);
+      }
       ++j;
     }
     stg.drain();
@@ -418,6 +475,11 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
 template <int BN, int STAGES, bool STAGED = false>
 constexpr int gemm_smem_bytes() {
   return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + (STAGED ? 4 * 8192 : 0) + 256;
+}
+template <class Epi, int BN, int STAGES>
+constexpr int gemm_smem_bytes_for() {
+  return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + EpiStagingBytes<Epi>::value +
+         8 * EpiExtraBars<Epi>::value + 256;
 }
 
 // ------------------------------------------------------------------ epilogues
@@ -660,32 +722,39 @@ struct EpiSwiGLU {
 // rows 64-127 the student rows of the same tokens; columns [0, 128) are gate and
 // [128, 256) up for output columns tn*128 + [0, 128).
 //
-// Eight epilogue warps, two per TMEM lane quarter (half h = 0, 1).  Per
-// 32-column slice, in two phases between which the eight warps meet once:
-//   A  every thread (one accumulator row, columns 16h .. 16h + 15 of the slice)
-//      forms z = silu(rstd g) (rstd u) in fp32 and writes its 16 values to a
-//      shared tile [path][row][column] (16-byte slots swizzled by row, so both
-//      the row-wise writes and the column reads of phase B are conflict-free;
-//      two tiles alternate by slice);
-//   B  thread (row R, column group cg of 8 columns) forms the causal depthwise
-//      convs of both paths from the k rows R - k + 1 .. R of the tile (16-byte
-//      shared loads; the taps of its 8 columns come from a bf16 table
-//      [path][f/8][KMAX][8] made once per call, loaded at the start of the
-//      slice so that they arrive during phase A), and writes 8 columns of
+// Eight epilogue warps in two groups that pass the tile's four 32-column
+// slices through four shared z tiles (16 KB each: [path][row][column] fp32,
+// 16-byte slots swizzled by row, so both the row-wise writes and the column
+// reads are conflict-free), with one full and one free mbarrier per slice:
+//   producers (warps 4-7, thread = accumulator row) form z = silu(rstd g)
+//      (rstd u) for each slice and write it to the slice's tile once the
+//      consumers have freed it; after the last TMEM read they release the
+//      accumulator, so the next-but-one tile's MMAs need not wait for the convs;
+//   consumers (warps 8-11, thread = rows R and R + 32 of column group cg of 8
+//      columns) form the causal depthwise convs of both paths from the k rows
+//      R - k + 1 .. R of the tile (16-byte shared loads; the taps of the 8
+//      columns come from a bf16 table [path][f/8][KMAX][8] made once per call,
+//      loaded before the slice is waited for), and write 8 columns of
 //      D = Zbar_T - Zbar_S and Kp = Zbar_S (padded chunk layout) and of the
-//      bf16 Z_S (output-GEMM operand) with one 16-byte store each.  The row's
-//      padded index is formed once per tile.  Kp^2 accumulates per row over the
-//      slices; four lanes share a row and reduce once per tile (the key norm
-//      becomes a row scale of R).
+//      bf16 Z_S (output-GEMM operand) with one 16-byte store each.  Kp^2
+//      accumulates per row; four lanes share a row and reduce once per tile
+//      (the key norm becomes a row scale of R).
+// The producers run up to one tile ahead of the consumers.  Every wait is a
+// bounded mbarrier wait; no named barrier is used, so the tile loop needs no
+// collective vote.
 // The tile's first k-1 rows only feed the conv (their outputs belong to the
 // previous tile); fp32 Z never reaches memory.
 //   z_halo [2, B, k-1, f] fp32: Z rows before token 0 (nullable: zeros)
 //   z_tail [2, B, k-1, f] fp32: written with the last k-1 rows of Z (nullable)
 template <int KMAX>  // conv width k <= KMAX
 struct EpiSwiGLUConv {
-  static constexpr bool kStaged = true;      // the staging area holds the z tiles
-  static constexpr bool kCollective = true;  // the warps exchange rows
+  static constexpr bool kStaged = true;
+  static constexpr bool kCollective = false;
   static constexpr int kWarps = 8;
+  static constexpr int kStagingBytes = 4 * 16384;  // the four slice tiles
+  static constexpr int kExtraBars = 8;             // slice full [0, 4), slice free [4, 8)
+  static constexpr int kExtraBarCount = 128;
+  static constexpr bool kSelfRelease = true;
   __nv_bfloat16* D;
   __nv_bfloat16* Kp;
   __nv_bfloat16* Zs;
@@ -696,6 +765,7 @@ struct EpiSwiGLUConv {
   float* z_tail;
   int B, T, f, k, C, Cp, Nc;
   long long BT, P;
+  DevStatus st;        // where a wait that gives up is recorded
 
   __device__ float pre(const TileCtx& c, int r) const {
     const int t = c.tok0 + (r & 63);
@@ -710,34 +780,85 @@ struct EpiSwiGLUConv {
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
     static_assert(BN == 256, "gate/up tiles are 128 gate + 128 up columns");
-    constexpr int NT = 32 * kWarps;
-    const int et = static_cast<int>(threadIdx.x) - 64;  // epilogue thread 0..255
-    const int half = et >> 7;
-    const int rin = r & 63;  // phase A: this thread's row within its path
-    const int path = r >= 64 ? 1 : 0;
-    const int ta = c.tok0 + rin;
+    const int et = static_cast<int>(threadIdx.x) - 128;  // epilogue thread 0..255 (warps 4-11)
+    const uint32_t par = stg.tiles & 1;                  // each slice barrier completes once per tile
+    ++stg.tiles;
+    uint64_t* full = stg.xbars;
+    uint64_t* freed = stg.xbars + 4;
+    uint8_t* tiles = stg.buf - ((et >> 5) & 3) * 8192;  // the 64 KB slice-tile area
     const int b = c.group;
     const int H = k - 1;
-    uint8_t* tiles = stg.buf - ((et >> 5) & 3) * 8192;  // the 32 KB staging area: two 16 KB z tiles
-    // phase B: row et / 4, columns 8 cg .. 8 cg + 7 of each slice
-    const int cg = et & 3;
-    const int brow = et >> 2;
-    const int bt = c.tok0 + brow;
-    const bool bval = brow >= H && bt >= 0 && bt < T;
-    const long long bp = pidx(b, bval ? bt : 0) * f;
-    const long long bz = (static_cast<long long>(b) * T + (bval ? bt : 0)) * f;
-    float ssq_acc = 0.f;
+    const int nslice = min(4, (f - c.tn * 128) / 32);  // f is a multiple of 64
+    volatile int no_abort = 0;
+    if (et < 128) {
+      // ------------------------------------------------------------ producers
+      const int rin = r & 63;
+      const int path = r >= 64 ? 1 : 0;
+      const int ta = c.tok0 + rin;
+      const int R = path * 64 + rin;
+#pragma unroll 1
+      for (int s = 0; s < 4; ++s) {
+        float z[32];
+        const int col0 = c.tn * 128 + 32 * s;
+        if (s < nslice) {
+          float gt[32], up[32];
+          tmem_ld32f(taddr + 32 * s, gt);
+          tmem_ld32f(taddr + 128 + 32 * s, up);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gg = gt[i] * rs;
+            z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (up[i] * rs);
+          }
+          if (ta < 0 || ta >= T) {
+            if (ta < 0 && z_halo) {
+              load_x32(z_halo + ((static_cast<long long>(path) * B + b) * H + (ta + H)) * f + col0, z);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) z[i] = 0.f;
+            }
+          }
+          if (z_tail && rin >= H && ta >= T - H && ta < T && ta >= 0)
+            store_f32x32(z_tail + ((static_cast<long long>(path) * B + b) * H + (ta - (T - H))) * f + col0, z);
+        }
+        if (s == nslice - 1) {  // the accumulator has been read: release it
+          tc_fence_before();
+          mbar_arrive(stg.release);
+        }
+        mbar_wait(&freed[s], par ^ 1, st, &no_abort);
+        if (s < nslice) {
+          uint8_t* tile = tiles + s * 16384;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(tile + R * 128 + ((j ^ (R & 7)) << 4)) =
+                make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
+        }
+        mbar_arrive(&full[s]);
+      }
+      return;
+    }
+    // -------------------------------------------------------------- consumers
+    mbar_arrive(stg.release);  // consumers never touch the accumulator
+    const int ec = et - 128;
+    const int cg = ec & 3;
+    int brow[2];
+    bool bval[2];
+    long long bp[2], bz[2];
+    float ssq_acc[2] = {0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      brow[u] = (ec >> 2) + 32 * u;
+      const int t = c.tok0 + brow[u];
+      bval[u] = brow[u] >= H && t >= 0 && t < T;
+      const int tt = bval[u] ? t : 0;
+      bp[u] = pidx(b, tt) * f;
+      bz[u] = (static_cast<long long>(b) * T + tt) * f;
+    }
 #pragma unroll 1
     for (int s = 0; s < 4; ++s) {
-      const int cc = 32 * s;
-      const int col0 = c.tn * 128 + cc;
-      if (col0 >= f) break;  // the same for every warp
-      uint8_t* tile = tiles + (s & 1) * 16384;
-      // phase B's taps (8 columns x k per path, one 16-byte word per tap), loaded
-      // now so that they arrive during phase A
+      const int col = c.tn * 128 + 32 * s + 8 * cg;
       uint4 tw[2][KMAX];
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(taps) + static_cast<long long>((col0 >> 3) + cg) * KMAX;
+      if (s < nslice) {
+        const uint4* src = reinterpret_cast<const uint4*>(taps) + static_cast<long long>(col >> 3) * KMAX;
 #pragma unroll
         for (int m = 0; m < KMAX; ++m) {
           tw[0][m] = m < k ? __ldg(src + m) : make_uint4(0u, 0u, 0u, 0u);
@@ -745,58 +866,18 @@ struct EpiSwiGLUConv {
                            : make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      // ---- A: z of this row, 16 columns
-      {
-        const int ch = cc + 16 * half;  // first column of this half within the tile
-        float z[16];
-        {
-          float gt[16], up[16];
-          tmem_ld16f(taddr + ch, gt);
-          tmem_ld16f(taddr + 128 + ch, up);
+      mbar_wait(&full[s], par, st, &no_abort);
+      if (s < nslice) {
+        const uint8_t* tile = tiles + s * 16384;
+        float aT[2][8], aS[2][8], z0[2][8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float gg = gt[i] * rs;
-            z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (up[i] * rs);
-          }
-        }
-        const int zc = col0 + 16 * half;  // global column of z[0]
-        if (ta < 0 || ta >= T) {
-          if (ta < 0 && z_halo) {
-            const float* src = z_halo + ((static_cast<long long>(path) * B + b) * H + (ta + H)) * f + zc;
-            float lo[8], hi[8];
-            ld8f(src, lo);
-            ld8f(src + 8, hi);
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) { z[i] = lo[i]; z[8 + i] = hi[i]; }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = 0.f;
-          }
-        }
-        if (z_tail && rin >= H && ta >= T - H && ta < T && ta >= 0) {
-          float* dst = z_tail + ((static_cast<long long>(path) * B + b) * H + (ta - (T - H))) * f + zc;
-          st8f(dst, *reinterpret_cast<const float(*)[8]>(&z[0]));
-          st8f(dst + 8, *reinterpret_cast<const float(*)[8]>(&z[8]));
-        }
-        const int R = path * 64 + rin;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int jj = 4 * half + j;
-          *reinterpret_cast<float4*>(tile + R * 128 + ((jj ^ (R & 7)) << 4)) =
-              make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
-        }
-      }
-      epi_bar_sync<NT>();
-      // ---- B: the convs of row brow, columns col0 + 8 cg .. + 7, both paths
-      {
-        const int col = col0 + 8 * cg;
-        float aT[8], aS[8], z0[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { aT[i] = 0.f; aS[i] = 0.f; z0[i] = 0.f; }
+          for (int i = 0; i < 8; ++i) { aT[u][i] = 0.f; aS[u][i] = 0.f; z0[u][i] = 0.f; }
 #pragma unroll
         for (int m = 0; m < KMAX; ++m) {  // tap m multiplies position t - m
-          if (m >= k || brow - m < 0) break;
-          float wT[8], wS[8], zt[8], zs[8];
+          if (m >= k) break;
+          float wT[8], wS[8];
           {
             const uint32_t uT[4] = {tw[0][m].x, tw[0][m].y, tw[0][m].z, tw[0][m].w};
             const uint32_t uS[4] = {tw[1][m].x, tw[1][m].y, tw[1][m].z, tw[1][m].w};
@@ -808,43 +889,57 @@ struct EpiSwiGLUConv {
               wS[2 * i + 1] = bf16hi_to_f32(uS[i]);
             }
           }
-          const int RT = brow - m, RS = 64 + brow - m;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int j = 2 * cg + h;
-            const float4 x = *reinterpret_cast<const float4*>(tile + RT * 128 + ((j ^ (RT & 7)) << 4));
-            const float4 y = *reinterpret_cast<const float4*>(tile + RS * 128 + ((j ^ (RS & 7)) << 4));
-            zt[4 * h] = x.x; zt[4 * h + 1] = x.y; zt[4 * h + 2] = x.z; zt[4 * h + 3] = x.w;
-            zs[4 * h] = y.x; zs[4 * h + 1] = y.y; zs[4 * h + 2] = y.z; zs[4 * h + 3] = y.w;
-          }
-          if (m == 0) {
+          for (int u = 0; u < 2; ++u) {
+            const int RT = brow[u] - m, RS = 64 + brow[u] - m;
+            if (RT < 0) continue;
+            float zt[8], zs[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) z0[i] = zs[i];
-          }
+            for (int h = 0; h < 2; ++h) {
+              const int j = 2 * cg + h;
+              const float4 x = *reinterpret_cast<const float4*>(tile + RT * 128 + ((j ^ (RT & 7)) << 4));
+              const float4 y = *reinterpret_cast<const float4*>(tile + RS * 128 + ((j ^ (RS & 7)) << 4));
+              zt[4 * h] = x.x; zt[4 * h + 1] = x.y; zt[4 * h + 2] = x.z; zt[4 * h + 3] = x.w;
+              zs[4 * h] = y.x; zs[4 * h + 1] = y.y; zs[4 * h + 2] = y.z; zs[4 * h + 3] = y.w;
+            }
+            if (m == 0) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            aT[i] = fmaf(wT[i], zt[i], aT[i]);
-            aS[i] = fmaf(wS[i], zs[i], aS[i]);
+              for (int i = 0; i < 8; ++i) z0[u][i] = zs[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              aT[u][i] = fmaf(wT[i], zt[i], aT[u][i]);
+              aS[u][i] = fmaf(wS[i], zs[i], aS[u][i]);
+            }
           }
         }
-        if (bval) {
+        // the slice's reads are done: the producers may refill it
+        mbar_arrive(&freed[s]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (!bval[u]) continue;
           float dd[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            dd[i] = aT[i] - aS[i];
-            ssq_acc = fmaf(aS[i], aS[i], ssq_acc);
+            dd[i] = aT[u][i] - aS[u][i];
+            ssq_acc[u] = fmaf(aS[u][i], aS[u][i], ssq_acc[u]);
           }
-          st8f(D + bp + col, dd);
-          st8f(Kp + bp + col, aS);
-          st8f(Zs + bz + col, z0);
+          st8f(D + bp[u] + col, dd);
+          st8f(Kp + bp[u] + col, aS[u]);
+          st8f(Zs + bz[u] + col, z0[u]);
         }
+      } else {
+        mbar_arrive(&freed[s]);
       }
     }
     // per-token sums of Kp^2 over the tile's columns: the four lanes of a row
-    float v = ssq_acc;
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    if (cg == 0 && bval) ssq[static_cast<long long>(c.tn) * P + pidx(b, bt)] = v;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float v = ssq_acc[u];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if (cg == 0 && bval[u]) ssq[static_cast<long long>(c.tn) * P + pidx(b, c.tok0 + brow[u])] = v;
+    }
   }
 };
 

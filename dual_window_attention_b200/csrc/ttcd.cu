@@ -142,6 +142,7 @@ struct RegSplit {
 };
 constexpr RegSplit kAttnRegSplit{128, 56, 256, 224};  // dual_window_attn_kernel
 constexpr RegSplit kScanRegSplit{128, 56, 256, 224};  // fastweight_scan_kernel
+constexpr RegSplit kGemm8RegSplit{128, 56, 256, 224};  // gemm_tc_kernel with 8 epilogue warps
 ttcd_status check_reg_split(const void* kern, int threads, const RegSplit& s) {
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return TTCD_ERR_CUDA;
@@ -176,10 +177,15 @@ ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B
   if (total <= 0) return TTCD_OK;
   if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
   auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom, B_MN>;
-  constexpr int smem = gemm_smem_bytes<BN, STAGES, Epi::kStaged>();
+  constexpr int smem = gemm_smem_bytes_for<Epi, BN, STAGES>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
   const int grid = total < c.sms ? total : c.sms;
+  if constexpr (EpiWarps<Epi>::value == 8) {
+    const ttcd_status rs = check_reg_split(reinterpret_cast<const void*>(kern), gemm_threads<Epi>(),
+                                           kGemm8RegSplit);
+    if (rs != TTCD_OK) return rs;
+  }
   kern<<<grid, gemm_threads<Epi>(), smem, c.s>>>(A, B0, B1, out_map ? *out_map : A,
                                            out_map2 ? *out_map2 : A, geo, epi, c.st);
   TTCD_CHECK_LAUNCH();
@@ -484,15 +490,15 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
                                                                         p->conv_k);
       TTCD_CHECK_LAUNCH();
       EpiSwiGLUConv<4> e{D, Kp, Zs, ssq, rstd, taps, z_halo, nullptr,
-                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
-      TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<4>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P, c.st};
+      TTCD_TRY((launch_gemm<E, 256, 3, true, EpiSwiGLUConv<4>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
     } else {
       conv_tap_table_kernel<8><<<cdiv(2 * m.f * 8, 256), 256, 0, c.s>>>(conv_T, conv_S, taps, m.f,
                                                                         p->conv_k);
       TTCD_CHECK_LAUNCH();
       EpiSwiGLUConv<8> e{D, Kp, Zs, ssq, rstd, taps, z_halo, nullptr,
-                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P};
-      TTCD_TRY((launch_gemm<E, 256, 4, true, EpiSwiGLUConv<8>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
+                         p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, m.BT, m.P, c.st};
+      TTCD_TRY((launch_gemm<E, 256, 3, true, EpiSwiGLUConv<8>, PairGeom>(c, mA, mB0, mB1, &mA, g, e)));
     }
     stage_mark(c, mark + 1);
     if (m.Cp != p->chunk || p->T % p->chunk != 0) {
