@@ -183,3 +183,53 @@ def test_decode_sizes_and_host_checks(lib):
     rd = lib.ttcd_decode_state_read
     assert rd(ctypes.byref(p), -1, fake, n_state, fake, None) == ttcd.ERR_INVALID_ARG
     assert rd(ctypes.byref(p), 3, fake, n_state - 1, fake, None) == ttcd.ERR_WORKSPACE
+    # the device-position form takes the same checks, without t
+    nxt = lib.ttcd_block_decode_next
+    assert nxt(None, beta, ctypes.byref(w), ctypes.byref(p), fake, n_state, fake, fake, n_ws, None) == ttcd.ERR_INVALID_ARG
+    assert nxt(fake, beta, ctypes.byref(w), ctypes.byref(p), fake, n_state - 1, fake, fake, n_ws, None) == ttcd.ERR_WORKSPACE
+    assert nxt(fake, beta, ctypes.byref(w), ctypes.byref(p), fake, n_state, fake, fake, n_ws - 1, None) == ttcd.ERR_WORKSPACE
+
+
+def test_backward_sizes_and_host_checks(lib):
+    """The three backward entry points: bf16 only, hd 64 or 128 for the
+    attention and the block, and every pointer and size checked on the host."""
+    p = _params(dtype=ttcd.BF16, head_dim=64, d_model=128, d_ff=256)
+    pc = p.c()
+    n_mlp = lib.ttcd_fastweight_mlp_backward_workspace_size(ctypes.byref(pc))
+    n_blk = lib.ttcd_block_backward_workspace_size(ctypes.byref(pc))
+    assert n_blk > n_mlp > ttcd.fastweight_mlp_workspace_size(p) > 0
+    assert lib.ttcd_fastweight_mlp_backward_workspace_size(ctypes.byref(_params(dtype=ttcd.F32).c())) == 0
+    assert lib.ttcd_block_backward_workspace_size(ctypes.byref(_params(dtype=ttcd.BF16).c())) == 0  # hd 32
+    n_att = lib.ttcd_dual_window_attn_backward_workspace_size(1, 256, 2)
+    assert n_att >= ttcd.STATUS_BYTES + 4 * 2 * 256 * 4
+    assert lib.ttcd_dual_window_attn_backward_workspace_size(0, 256, 2) == 0
+    fake = 1 << 20
+    w = ttcd._Weights(*([fake] * 10))
+    g = ttcd._MlpGrads(*([fake] * 6))
+    mlp = lib.ttcd_fastweight_mlp_backward
+    args = [fake, fake, fake, ctypes.byref(w), ctypes.byref(pc), None, fake, None, fake, fake, fake,
+            None, ctypes.byref(g), fake, n_mlp, None]
+    bad = list(args); bad[6] = None                   # no d_y
+    assert mlp(*bad) == ttcd.ERR_INVALID_ARG
+    bad = list(args); bad[12] = None                  # no gradient table
+    assert mlp(*bad) == ttcd.ERR_INVALID_ARG
+    bad = list(args); bad[14] = n_mlp - 1             # short workspace
+    assert mlp(*bad) == ttcd.ERR_WORKSPACE
+    bg = ttcd._BlockGrads(*([fake] * 10))
+    blk = lib.ttcd_block_backward
+    args = [fake, fake, ctypes.byref(w), ctypes.byref(pc), None, fake, None, fake, fake, None,
+            ctypes.byref(bg), fake, n_blk, None]
+    bad = list(args); bad[5] = None                   # no d_out
+    assert blk(*bad) == ttcd.ERR_INVALID_ARG
+    bad = list(args); bad[12] = n_blk - 1
+    assert blk(*bad) == ttcd.ERR_WORKSPACE
+    att = lib.ttcd_dual_window_attn_backward
+    a = [fake] * 12 + [1, 256, 2, 1, 64, 16, 64, 0.0, fake, n_att, None]
+    bad = list(a); bad[16] = 32                       # hd 32
+    assert att(*bad) == ttcd.ERR_UNSUPPORTED
+    bad = list(a); bad[17], bad[18] = 65, 64          # w_S > w_T
+    assert att(*bad) == ttcd.ERR_INVALID_ARG
+    bad = list(a); bad[9] = None                      # no dq
+    assert att(*bad) == ttcd.ERR_INVALID_ARG
+    bad = list(a); bad[21] = n_att - 1
+    assert att(*bad) == ttcd.ERR_WORKSPACE
