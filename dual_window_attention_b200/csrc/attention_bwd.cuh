@@ -17,7 +17,7 @@
 // formed transposed, S^T = K Q^T, so that keys are TMEM lanes: P^T and dS^T are
 // then the A operands of dV += P^T dO and dK += dS^T Q, which accumulate in TMEM
 // over all visits and are stored once, without atomics.  dQ = dS K of each
-// visit is added to the fp32 dq in global memory (vector atomics).
+// visit is added to the fp32 dq in global memory by TMA reductions.
 //
 // Pipeline (one CTA, 384 threads):
 //   warp 0      TMA producer: K and V once, then per visit Q with the visit's
@@ -28,7 +28,8 @@
 //               scores form while the key-row threads work on dS(v)
 //   warps 4..7  thread = key row: P^T (into TMEM, over its S^T row) and dS^T
 //               (into shared memory), and at the end the dK and dV rows
-//   warps 8..11 thread = query row: the dQ tile of each visit into dq
+//   warps 8..11 thread = query row: the dQ tile of each visit into dq (TMA
+//               reduce-add of 32 x 32 boxes staged in shared memory)
 // TMEM (512 columns): S^T [0,128), whose first 64 columns take P^T as packed
 // bf16 pairs (the A operand of dV, as P is for O in the forward); dP^T
 // [128,256), reused for the dQ tile once dS^T is formed; dK [256, 256+HD), dV
@@ -73,7 +74,8 @@ struct AttnBwdCfg {
   static constexpr int Q_OFF = V_OFF + TILE;       // two stages
   static constexpr int DO_OFF = Q_OFF + 2 * TILE;  // one stage
   static constexpr int DS_OFF = DO_OFF + TILE;
-  static constexpr int LSE_OFF = DS_OFF + DS_TILE;  // 2 stages of 128 floats
+  static constexpr int DQ_OFF = DS_OFF + DS_TILE;   // 4 warps x 32 rows x 128 bytes
+  static constexpr int LSE_OFF = DQ_OFF + 4 * 4096;  // 2 stages of 128 floats
   static constexpr int DEL_OFF = LSE_OFF + 1024;    // 2 stages of 128 floats
   static constexpr int BAR_OFF = DEL_OFF + 1024;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
                                 const __grid_constant__ CUtensorMap mapV,
                                 const __grid_constant__ CUtensorMap mapDOT,
                                 const __grid_constant__ CUtensorMap mapDOS,
+                                const __grid_constant__ CUtensorMap mapDQ,
                                 const AttnBwdArgs a, const DevStatus st) {
   using Cfg = AttnBwdCfg<HD>;
   constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
@@ -408,31 +411,45 @@ __global__ void __launch_bounds__(ATTB_THREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
     // ----------------------------------------------------- query rows: dQ tiles
+    // Each visit's dQ tile is added to dq by TMA reductions (fp32 add in L2),
+    // 32 rows x 32 columns at a time through this warp's 4 KB staging box
+    // (128-byte swizzle).  Rows past a sequence's end carry exact zeros (P = 0
+    // there), so a box reaching into the next sequence adds nothing to it.
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t dq_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 128;
+    uint8_t* box = smem + Cfg::DQ_OFF + quarter * 4096;
     for (int v = 0; v < nv; ++v) {
       int hg, qt;
       bool stu;
       vis.get(v, hg, qt, stu);
       const int h = hk * G + hg;
-      const int t = qt * ATT_BM + r;
       if (!mbar_wait(dq_full, v & 1, st, abort)) break;
       tc_fence_after();
       // the whole row into registers first: the columns are free for the next
-      // dP^T as soon as they have been read, while the adds are still in flight
+      // dP^T as soon as they have been read
       float x[HD];
 #pragma unroll
       for (int c = 0; c < HD; c += 32) tmem_ld32f(dq_addr + c, *reinterpret_cast<float(*)[32]>(&x[c]));
       tc_fence_before();
       mbar_arrive(dp_free);
-      if (t < a.T) {
-        float* dst = a.dq + ((static_cast<long long>(b) * a.T + t) * a.Hq + h) * HD;
+      const int y = b * a.T + qt * ATT_BM + quarter * 32;
 #pragma unroll
-        for (int i = 0; i < HD; i += 4)
-          atomicAdd(reinterpret_cast<float4*>(dst + i), make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]));
+      for (int c = 0; c < HD; c += 32) {
+        if (lane == 0) bulk_wait_read<0>();  // the previous box has been read out
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+              make_float4(x[c + 4 * j], x[c + 4 * j + 1], x[c + 4 * j + 2], x[c + 4 * j + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(&mapDQ, box, h * HD + c, y);
+          bulk_commit();
+        }
       }
     }
+    if (lane == 0) bulk_wait<0>();  // every reduction has completed
   }
   __syncthreads();
   if (warp == 1) {

@@ -2142,6 +2142,8 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
       !make_map<bf>(&mdt, do_T, wq, BT, wq * 2, 64, 128) ||
       !make_map<bf>(&mds, do_S, wq, BT, wq * 2, 64, 128))
     return TTCD_ERR_CUDA;
+  CUtensorMap mdq;  // dq as [BT, Hq * HD] fp32, boxes of 32 columns x 32 rows
+  if (!make_map<float>(&mdq, dq, wq, BT, wq * 4, 32, 32)) return TTCD_ERR_CUDA;
   AttnBwdArgs a;
   a.dq = dq;
   a.dk = dk;
@@ -2166,7 +2168,7 @@ ttcd_status launch_attn_bwd(const Ctx& c, const void* q, const void* k, const vo
   const long long grid = static_cast<long long>(a.n_kt) * B * Hkv;
   if (grid >= (1ll << 31)) return TTCD_ERR_UNSUPPORTED;
   TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), ATTB_THREADS, kAttnRegSplit));
-  kern<<<static_cast<unsigned>(grid), ATTB_THREADS, smem, c.s>>>(mq, mk, mv, mdt, mds, a, c.st);
+  kern<<<static_cast<unsigned>(grid), ATTB_THREADS, smem, c.s>>>(mq, mk, mv, mdt, mds, mdq, a, c.st);
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
 }

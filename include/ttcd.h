@@ -179,7 +179,7 @@ size_t ttcd_dual_window_attn_backward_workspace_size(int B, int T, int Hq);
  *                  device, 16-byte aligned; status word first
  * Precision: bf16 tensor-core operands (q, k, v, dO and the rebuilt P and dS
  * rounded to bf16), fp32 accumulation; dq sums the key tiles' contributions
- * with fp32 atomic adds, so its low bits depend on their order.
+ * with fp32 reductions in L2, so its low bits depend on their order.
  */
 ttcd_status ttcd_dual_window_attn_backward(const void* q, const void* k, const void* v,
                                            const void* o_T, const void* o_S, const float* lse_T,
