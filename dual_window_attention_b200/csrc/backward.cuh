@@ -225,78 +225,151 @@ __global__ void key_backward_kernel(const float* __restrict__ epart, int n_epart
 //   dZ[path, b, s, c] = sum_{m < k, s + m < T} w_path[c, m] dZbar_path[b, s + m, c]
 //                       (+ dZs_read[b, s, c] for the student path),
 // dZbar_* in the chunk-padded layout, dZ [2, B, T, f] fp32 (teacher first).
-// Four columns per thread.
-__global__ void conv_backward_kernel(const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
-                                     const float* __restrict__ dzs_read,
-                                     const __nv_bfloat16* __restrict__ conv_T,
-                                     const __nv_bfloat16* __restrict__ conv_S,
-                                     float* __restrict__ dZ, int B, int T, int f, int k, int C,
-                                     int Cp, int Nc) {
-  const long long BT = static_cast<long long>(B) * T;
-  const int per_row = f / 4;
+// Thread = (path, sequence, 4 columns, CONV_BWD_ROWS consecutive tokens): it
+// slides a window of k dZbar rows down its tokens (one 16-byte load per row)
+// and takes its taps from the forward's bf16 table [path][f/8][KMAX][8]; the
+// padded row index advances without divisions.
+constexpr int CONV_BWD_ROWS = 16;
+
+template <int KMAX>
+__global__ void __launch_bounds__(256) conv_backward_kernel(
+    const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
+    const float* __restrict__ dzs_read, const __nv_bfloat16* __restrict__ taps,
+    float* __restrict__ dZ, int B, int T, int f, int k, int C, int Cp, int Nc) {
+  const int f4 = f / 4;
+  const int nrb = (T + CONV_BWD_ROWS - 1) / CONV_BWD_ROWS;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= 2 * BT * per_row) return;
-  const long long row = idx / per_row;
-  const int c0 = static_cast<int>(idx % per_row) * 4;
-  const bool student = row >= BT;
-  const long long bt = student ? row - BT : row;
-  const int b = static_cast<int>(bt / T), s = static_cast<int>(bt % T);
-  const float* dzb = student ? dzb_S : dzb_T;
-  const __nv_bfloat16* w = student ? conv_S : conv_T;
-  float4 acc = student ? __ldg(reinterpret_cast<const float4*>(dzs_read + bt * f + c0))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int m = 0; m < k; ++m) {
-    const int t = s + m;
-    if (t >= T) break;
-    const long long pr = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
-    const float4 g = __ldg(reinterpret_cast<const float4*>(dzb + pr * f + c0));
-    acc.x = fmaf(__bfloat162float(w[(c0 + 0) * k + m]), g.x, acc.x);
-    acc.y = fmaf(__bfloat162float(w[(c0 + 1) * k + m]), g.y, acc.y);
-    acc.z = fmaf(__bfloat162float(w[(c0 + 2) * k + m]), g.z, acc.z);
-    acc.w = fmaf(__bfloat162float(w[(c0 + 3) * k + m]), g.w, acc.w);
+  if (idx >= 2ll * B * nrb * f4) return;
+  const int c4 = static_cast<int>(idx % f4);
+  const long long rest = idx / f4;
+  const int rb = static_cast<int>(rest % nrb);
+  const int b = static_cast<int>((rest / nrb) % B);
+  const int path = static_cast<int>(rest / (static_cast<long long>(nrb) * B));
+  const int c0 = 4 * c4;
+  const float* dzb = path ? dzb_S : dzb_T;
+  // taps of the 4 columns: 8 bf16 of tap m hold columns 8 (c0 / 8) .. + 7
+  float w[KMAX][4];
+  {
+    const uint4* tp = reinterpret_cast<const uint4*>(taps) +
+                      (static_cast<long long>(path) * (f / 8) + c0 / 8) * KMAX;
+    const int half = (c0 / 4) & 1;
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m) {
+      const uint4 u = __ldg(tp + m);
+      const uint32_t a = half ? u.z : u.x, bb = half ? u.w : u.y;
+      w[m][0] = bf16lo_to_f32(a);
+      w[m][1] = bf16hi_to_f32(a);
+      w[m][2] = bf16lo_to_f32(bb);
+      w[m][3] = bf16hi_to_f32(bb);
+    }
   }
-  reinterpret_cast<float4*>(dZ + row * f)[c0 / 4] = acc;
+  const int s0 = rb * CONV_BWD_ROWS;
+  const int s1 = min(T, s0 + CONV_BWD_ROWS);
+  // window: win[m] = dZbar row s + m (zero past T); rows up to s + KMAX - 1 are
+  // held (their taps are zero when m >= k), so every index is static
+  float4 win[KMAX];
+  int ci = s0 / C, cj = s0 % C;  // chunk and row within it of the next row to load
+  auto next_row = [&]() {
+    const long long pr = (static_cast<long long>(b) * Nc + ci) * Cp + cj;
+    if (++cj == C) { cj = 0; ++ci; }
+    return __ldg(reinterpret_cast<const float4*>(dzb + pr * f + c0));
+  };
+#pragma unroll
+  for (int m = 0; m < KMAX - 1; ++m)
+    win[m + 1] = s0 + m < T ? next_row() : make_float4(0.f, 0.f, 0.f, 0.f);
+  const long long BT = static_cast<long long>(B) * T;
+  for (int s = s0; s < s1; ++s) {
+#pragma unroll
+    for (int m = 0; m < KMAX - 1; ++m) win[m] = win[m + 1];
+    win[KMAX - 1] = s + KMAX - 1 < T ? next_row() : make_float4(0.f, 0.f, 0.f, 0.f);
+    const long long bt = static_cast<long long>(b) * T + s;
+    float4 acc = path ? __ldg(reinterpret_cast<const float4*>(dzs_read + bt * f + c0))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m) {
+      if (m >= k) break;
+      acc.x = fmaf(w[m][0], win[m].x, acc.x);
+      acc.y = fmaf(w[m][1], win[m].y, acc.y);
+      acc.z = fmaf(w[m][2], win[m].z, acc.z);
+      acc.w = fmaf(w[m][3], win[m].w, acc.w);
+    }
+    reinterpret_cast<float4*>(dZ + (path * BT + bt) * f)[c4] = acc;
+  }
 }
 
-constexpr int TAP_SPLITS = 32;  // token splits of the tap gradient (partials per split)
-constexpr int TAP_LANES = 8;    // row lanes per block
+constexpr int TAP_SPLITS = 128;  // token splits of the tap gradient (partials per split)
 
 // part[split][path][c][m] = sum over the split's tokens (b, t), t >= m, of
-// dZbar_path[b, t, c] Z_path[b, t - m, c].  Block: 32 columns x 8 row lanes;
-// grid (f / 32, TAP_SPLITS, 2).  Z [2, B, T, f] bf16, dZbar chunk-padded fp32.
+// dZbar_path[b, t, c] Z_path[b, t - m, c].  Thread = (path, 8 columns, split):
+// it walks its contiguous tokens keeping the last k rows of Z in registers
+// (one 16-byte load of Z and two of dZbar per token).  Z [2, B, T, f] bf16,
+// dZbar chunk-padded fp32.
 template <int KMAX>
 __global__ void __launch_bounds__(256) conv_tap_grad_kernel(
     const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
     const __nv_bfloat16* __restrict__ z, float* __restrict__ part, int B, int T, int f, int k,
     int C, int Cp, int Nc) {
-  const int lane = threadIdx.x & 31, rl = threadIdx.x >> 5;
-  const int c = blockIdx.x * 32 + lane;
-  const int split = blockIdx.y, path = blockIdx.z;
+  const int f8 = f / 8;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= 2 * f8 * TAP_SPLITS) return;
+  const int c8 = idx % f8;
+  const int split = (idx / f8) % TAP_SPLITS;
+  const int path = idx / (f8 * TAP_SPLITS);
   const long long BT = static_cast<long long>(B) * T;
   const long long per = (BT + TAP_SPLITS - 1) / TAP_SPLITS;
   const long long r0 = split * per, r1 = min(BT, r0 + per);
   const float* dzb = path ? dzb_S : dzb_T;
-  const __nv_bfloat16* zp = z + path * BT * f;
-  float acc[KMAX];
+  const __nv_bfloat16* zp = z + path * BT * f + c8 * 8;
+  float acc[KMAX][8];
 #pragma unroll
-  for (int m = 0; m < KMAX; ++m) acc[m] = 0.f;
-  for (long long bt = r0 + rl; bt < r1; bt += TAP_LANES) {
-    const int b = static_cast<int>(bt / T), t = static_cast<int>(bt % T);
-    const long long pr = (static_cast<long long>(b) * Nc + t / C) * Cp + t % C;
-    const float g = dzb[pr * f + c];
+  for (int m = 0; m < KMAX; ++m)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
+  float zw[KMAX][8];  // zw[m] = Z row t - m
+#pragma unroll
+  for (int m = 0; m < KMAX; ++m)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) zw[m][i] = 0.f;
+  if (r0 < r1) {
+    int b = static_cast<int>(r0 / T), t = static_cast<int>(r0 % T);
+    // the k - 1 rows before the split's first token (same sequence only)
+#pragma unroll
+    for (int m = 1; m < KMAX; ++m)
+      if (m < k && t - m >= 0) ld8f(zp + (r0 - m) * f, zw[m]);
+    int ci = t / C, cj = t % C;
+    for (long long bt = r0; bt < r1; ++bt) {
+      if (t == T) {  // next sequence: the window restarts from zeros
+        t = 0;
+        ++b;
+        ci = 0;
+        cj = 0;
+#pragma unroll
+        for (int m = 1; m < KMAX; ++m)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) zw[m][i] = 0.f;
+      }
+      ld8f(zp + bt * f, zw[0]);
+      float g[8];
+      ld8f(dzb + ((static_cast<long long>(b) * Nc + ci) * Cp + cj) * f + c8 * 8, g);
+#pragma unroll
+      for (int m = 0; m < KMAX; ++m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(g[i], zw[m][i], acc[m][i]);
+      // shift the window: row t becomes t - 1 for the next token
+#pragma unroll
+      for (int m = KMAX - 1; m > 0; --m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zw[m][i] = zw[m - 1][i];
+      ++t;
+      if (++cj == C) { cj = 0; ++ci; }
+    }
+  }
+  float* dst = part + ((static_cast<long long>(split) * 2 + path) * f + c8 * 8) * k;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int m = 0; m < KMAX; ++m)
-      if (m < k && t >= m) acc[m] = fmaf(g, __bfloat162float(zp[(bt - m) * f + c]), acc[m]);
-  }
-  __shared__ float red[TAP_LANES][KMAX][32];
-#pragma unroll
-  for (int m = 0; m < KMAX; ++m) red[rl][m][lane] = acc[m];
-  __syncthreads();
-  if (rl < KMAX && rl < k) {
-    float s = 0.f;
-    for (int q = 0; q < TAP_LANES; ++q) s += red[q][rl][lane];
-    part[((static_cast<long long>(split) * 2 + path) * f + c) * k + rl] = s;
-  }
+      if (m < k) dst[i * k + m] = acc[m][i];
 }
 
 // out[path][c][m] = sum over splits of part[split][path][c][m].

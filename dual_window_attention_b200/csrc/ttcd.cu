@@ -1999,10 +1999,14 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
   }
   // dZ_P through the convs (teacher: dZbar_T = dD), plus the read's dZ_S
   {
-    const long long n = 2 * m.BT * (m.f / 4);
-    conv_backward_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
-        dD, dzbs, dzsy, static_cast<const bf*>(w->conv_T), static_cast<const bf*>(w->conv_S), dZ,
-        p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
+    const bf* taps = at<bf>(ws, F, B_TAPS);  // the forward's table, [path][f/8][KMAX][8]
+    const long long n = 2ll * p->B * cdiv(p->T, CONV_BWD_ROWS) * (m.f / 4);
+    if (p->conv_k <= 4)
+      conv_backward_kernel<4><<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+          dD, dzbs, dzsy, taps, dZ, p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
+    else
+      conv_backward_kernel<8><<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, c.s>>>(
+          dD, dzbs, dzsy, taps, dZ, p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
     TTCD_CHECK_LAUNCH();
   }
   // gate/up recomputed: [da | db] and Z
@@ -2017,13 +2021,13 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
   }
   // tap gradients
   {
-    dim3 grid(m.f / 32, TAP_SPLITS, 2);
+    const int nt = 2 * (m.f / 8) * TAP_SPLITS;
     if (p->conv_k <= 4)
-      conv_tap_grad_kernel<4><<<grid, 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T, m.f,
-                                                     p->conv_k, p->chunk, m.Cp, m.Nc);
+      conv_tap_grad_kernel<4><<<cdiv(nt, 256), 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T,
+                                                             m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
     else
-      conv_tap_grad_kernel<8><<<grid, 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T, m.f,
-                                                     p->conv_k, p->chunk, m.Cp, m.Nc);
+      conv_tap_grad_kernel<8><<<cdiv(nt, 256), 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T,
+                                                             m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
     TTCD_CHECK_LAUNCH();
     conv_tap_reduce_kernel<<<cdiv(2 * m.f * p->conv_k, 256), 256, 0, c.s>>>(
         tpart, g->conv_T, g->conv_S, m.f, p->conv_k);
