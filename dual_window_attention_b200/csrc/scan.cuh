@@ -18,6 +18,17 @@
 // (bf16, boxes of 64 MN-elements x 64 tokens).  MN = false: their transposes
 // Rt [d, P] and Kt [f, P], read as K-major operands (tf32).
 // Warps: 0 TMA, 1 TMEM + MMA, 2-3 idle, 4-11 epilogue (setmaxnreg 56 / 224).
+//
+// PAIR = true (bf16, token-major operands): a cluster of two CTAs shares one
+// 256 x 192 tile through M = 256 MMAs (tcgen05 .cta_group::2).  Each CTA loads
+// its own 128 rows of R and half of the tile's key columns (96, as three boxes
+// of 32 columns in the 64-byte swizzle), so each k-block moves 28 KB into each
+// SM instead of 40 KB: the operand bytes per FLOP from L2 drop by 30 %.  Rank 0
+// waits for both CTAs' bytes on its own full barriers, issues the MMAs and
+// commits them to both CTAs' stage and accumulator barriers; each CTA's
+// epilogue folds its own 128 rows and releases the accumulator on rank 0's
+// barrier.  Both CTAs end at a cluster barrier, so neither leaves while the
+// other's MMAs or arrivals can still touch its shared memory.
 #pragma once
 #include "gemm.cuh"
 
@@ -44,19 +55,44 @@ struct ScanArgs {
 
 constexpr int SCAN_BN = 192;
 constexpr int SCAN_THREADS = 384;
+constexpr int SCAN_PAIR_BOX = 32;  // key columns per 64-byte-swizzled box of a pair CTA
 
-template <class E, int STAGES, bool MN>
+// Rows of d per tile (per pair of CTAs when PAIR).
+template <bool PAIR>
+constexpr int scan_tile_rows() {
+  return PAIR ? 2 * GEMM_BM : GEMM_BM;
+}
+template <class E, bool PAIR>
+constexpr int scan_stage_bytes() {
+  return GEMM_BM * 128 + (PAIR ? SCAN_BN / 2 : SCAN_BN) * 128;
+}
+template <class E, int STAGES, bool PAIR>
+constexpr int scan_smem_bytes() {
+  return 1024 + STAGES * scan_stage_bytes<E, PAIR>() + 256;
+}
+
+template <class E, int STAGES, bool MN, bool PAIR = false, bool B64 = PAIR>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
     fastweight_scan_kernel(const __grid_constant__ CUtensorMap mapR,
                            const __grid_constant__ CUtensorMap mapK, const ScanArgs<E> a,
                            const DevStatus st) {
+  static_assert(!PAIR || (MN && sizeof(E) == 2), "CTA pairs take bf16 token-major operands");
+  static_assert(!B64 || (MN && sizeof(E) == 2), "64-byte swizzled keys are bf16 token-major");
+  static_assert(!PAIR || B64, "a pair CTA's 96 key columns take the 64-byte swizzle");
   constexpr int BN = SCAN_BN;
   constexpr int BK = ElemTraits<E>::BK;  // tokens per k-block == MN elements per box
   constexpr int BOX_BYTES = BK * BK * static_cast<int>(sizeof(E));
-  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = BN * 128;
+  constexpr int B_COLS = PAIR ? BN / 2 : BN;  // key columns this CTA loads
+  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = B_COLS * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static_assert(STAGE_BYTES == scan_stage_bytes<E, PAIR>(), "stage size");
   constexpr int KSTEP_BYTES = (32 / static_cast<int>(sizeof(E))) * 128;  // tokens per MMA x 128 B
-  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, MN, MN);
+  // B64 (the pair's keys): 64-byte rows, so a K step of 16 tokens is 1024
+  // bytes and the 32-column panels lie one box (32 x 64 tokens x 2 B) apart.
+  constexpr int PBOX_BYTES = SCAN_PAIR_BOX * BK * 2;
+  constexpr int B_KSTEP_BYTES = B64 ? 16 * 64 : KSTEP_BYTES;
+  constexpr uint32_t IDESC =
+      idesc_f32acc(scan_tile_rows<PAIR>(), BN, ElemTraits<E>::FMT, MN, MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -69,17 +105,20 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  if (a.commit_pos && *a.commit_pos % a.commit_C != a.commit_C - 1) return;
+  if (!PAIR && a.commit_pos && *a.commit_pos % a.commit_C != a.commit_C - 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tn = blockIdx.x % a.tiles_n;
-  const int tm = (blockIdx.x / a.tiles_n) % a.tiles_m;
-  const int b = blockIdx.x / (a.tiles_n * a.tiles_m);
-  const int m0 = tm * GEMM_BM, n0 = tn * BN;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tn = tile % a.tiles_n;
+  const int tm = (tile / a.tiles_n) % a.tiles_m;
+  const int b = tile / (a.tiles_n * a.tiles_m);
+  const int m0 = tm * scan_tile_rows<PAIR>() + static_cast<int>(rank) * GEMM_BM;  // this CTA's rows
+  const int n0 = tn * BN;
   const int kpc = a.Cp / BK;  // k-blocks per chunk
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&accf[s], 1); mbar_init(&acce[s], 256); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&accf[s], 1); mbar_init(&acce[s], PAIR ? 512 : 256); }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -87,11 +126,20 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     tma_prefetch_map(&mapK);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
     tc_fence_before();
   }
-  __syncthreads();
+  // A pair meets here before any arrival or byte count crosses to rank 0.
+  if constexpr (PAIR)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -100,36 +148,68 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     if (warp == 0 && lane == 0) {
       int it = 0;
       bool ok = true;
+      // Pair: both CTAs count their bytes on rank 0's full barriers.
+      const uint32_t full0 = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
       for (int i = 0; i < a.Nc && ok; ++i) {
         for (int kb = 0; kb < kpc; ++kb, ++it) {
           const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, st, abort)) { ok = false; break; }
+          if (!mbar_wait<PAIR>(&empty[s], ((it / STAGES) & 1) ^ 1, st, abort)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
           const int ci = a.reverse ? a.Nc - 1 - i : i;
           const int y = (b * a.Nc + ci) * a.Cp + kb * BK;  // first token of the k-block
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          if constexpr (MN) {
+          if constexpr (PAIR) {
+            const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < GEMM_BM / BK; ++q)
-              tma_load_2d(sa + q * BOX_BYTES, &mapR, &full[s], m0 + q * BK, y);
+              tma_load_2d_pair(sa + q * BOX_BYTES, &mapR, fb, m0 + q * BK, y);
+            const int nb = n0 + static_cast<int>(rank) * B_COLS;
 #pragma unroll
-            for (int q = 0; q < BN / BK; ++q)
-              tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
+            for (int q = 0; q < B_COLS / SCAN_PAIR_BOX; ++q)
+              tma_load_2d_pair(sa + A_BYTES + q * PBOX_BYTES, &mapK, fb,
+                               nb + q * SCAN_PAIR_BOX, y);
           } else {
-            tma_load_2d(sa, &mapR, &full[s], y, m0);
-            tma_load_2d(sa + A_BYTES, &mapK, &full[s], y, n0);
+            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+            if constexpr (MN) {
+#pragma unroll
+              for (int q = 0; q < GEMM_BM / BK; ++q)
+                tma_load_2d(sa + q * BOX_BYTES, &mapR, &full[s], m0 + q * BK, y);
+              if constexpr (B64) {
+#pragma unroll
+                for (int q = 0; q < BN / SCAN_PAIR_BOX; ++q)
+                  tma_load_2d(sa + A_BYTES + q * PBOX_BYTES, &mapK, &full[s],
+                              n0 + q * SCAN_PAIR_BOX, y);
+              } else {
+#pragma unroll
+                for (int q = 0; q < BN / BK; ++q)
+                  tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
+              }
+            } else {
+              tma_load_2d(sa, &mapR, &full[s], y, m0);
+              tma_load_2d(sa + A_BYTES, &mapK, &full[s], y, n0);
+            }
           }
         }
       }
       volatile int no_abort = 0;
-      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-        mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
-    } else if (warp == 1) {
-      // MMA issuer: the whole warp walks the loop, one elected lane issues.
+      if constexpr (PAIR) {
+        // Until rank 0's MMAs have consumed the last stages: then no load of
+        // this CTA and no commit to its stage barriers is still in flight.
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait<true>(&empty[j % STAGES], (j / STAGES) & 1, st, abort);
+      } else {
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
+      }
+    } else if (warp == 1 && rank == 0) {
+      // MMA issuer (rank 0 of a pair): the whole warp walks the loop, one
+      // elected lane issues.
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
+      constexpr uint32_t HI_B = B64 ? sdesc_hi_sw64(512) : HI;
       const uint32_t lo0 = sdesc_lo(smem_u32(smem), MN ? BOX_BYTES : 16);
+      const uint32_t lo0_b = sdesc_lo(smem_u32(smem), B64 ? PBOX_BYTES : (MN ? BOX_BYTES : 16));
       auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
+        return __all_sync(0xffffffffu, mbar_wait<PAIR>(bar, parity, st, abort));
       };
       int it = 0;
       bool ok = true;
@@ -142,26 +222,50 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
           if (!wait(&full[s], (it / STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_lo = lo0 + ((s * STAGE_BYTES) >> 4);
-          const uint32_t b_lo = a_lo + (A_BYTES >> 4);
+          const uint32_t b_lo = lo0_b + ((s * STAGE_BYTES + A_BYTES) >> 4);
           if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t off = (MN ? k * KSTEP_BYTES : k * 32) >> 4;
-              mma_ss_lh<E>(tmem + ab * BN, a_lo + off, HI, b_lo + off, HI, IDESC,
-                           (kb | k) != 0 ? 1u : 0u);
+              const uint32_t off_b = (MN ? k * B_KSTEP_BYTES : k * 32) >> 4;
+              if constexpr (PAIR)
+                mma_bf16_ss_lh_pair(tmem + ab * BN, a_lo + off, HI, b_lo + off_b, HI_B, IDESC,
+                                    (kb | k) != 0 ? 1u : 0u);
+              else
+                mma_ss_lh<E>(tmem + ab * BN, a_lo + off, HI, b_lo + off_b, HI_B, IDESC,
+                             (kb | k) != 0 ? 1u : 0u);
             }
-            mma_commit(&empty[s]);
+            if constexpr (PAIR)
+              mma_commit_pair_mask(&empty[s], 0x3);
+            else
+              mma_commit(&empty[s]);
           }
           __syncwarp();
         }
         if (!ok) break;
-        if (elect_one()) mma_commit(&accf[ab]);
+        if (elect_one()) {
+          if constexpr (PAIR)
+            mma_commit_pair_mask(&accf[ab], 0x3);
+          else
+            mma_commit(&accf[ab]);
+        }
         __syncwarp();
       }
-      if (elect_one()) mma_commit(drain);
+      if (elect_one()) {
+        if constexpr (PAIR)
+          mma_commit_pair_own(drain);
+        else
+          mma_commit(drain);
+      }
       __syncwarp();
       volatile int no_abort = 0;
       mbar_wait(drain, 0, st, &no_abort);
+      if constexpr (PAIR) {
+        // The epilogues' releases of the last two accumulators (some arrive
+        // from the other CTA) land before this CTA may leave.
+        for (int i = a.Nc; i < a.Nc + 2; ++i)
+          if (i >= 2) mbar_wait<true>(&acce[i & 1], ((i >> 1) & 1) ^ 1, st, abort);
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
@@ -178,6 +282,12 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       return static_cast<long long>(b) * a.Nc + (a.reverse ? a.Nc - 1 - j : j);
     };
     float S[HC];
+    // bf16: the thread's HC columns of W_down stay in registers as packed
+    // pairs, so the chunk loop below issues no global loads (they would queue
+    // in L2 behind the operand stream and stall the release of the next
+    // accumulator).
+    constexpr bool WREG = sizeof(E) == 2;
+    uint32_t wd[WREG ? HC / 2 : 1];
     // S_0 = state_in (or 0); W_0 = W_down + S_0 (W_down null: 0).
 #pragma unroll
     for (int cc = 0; cc < HC; cc += 32) {
@@ -191,9 +301,27 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       }
 #pragma unroll
       for (int e = 0; e < 32; ++e) S[cc + e] = s32[e];
+      if constexpr (WREG) {
+        const bool have = wrow && row_ok && col < a.f && a.w_all;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 w4 = have ? reinterpret_cast<const uint4*>(wrow + col)[u]
+                                : make_uint4(0u, 0u, 0u, 0u);
+          wd[cc / 2 + 4 * u + 0] = w4.x;
+          wd[cc / 2 + 4 * u + 1] = w4.y;
+          wd[cc / 2 + 4 * u + 2] = w4.z;
+          wd[cc / 2 + 4 * u + 3] = w4.w;
+        }
+      }
       if (row_ok && col < a.f && a.w_all) {
         float w[32];
-        if (wrow) {
+        if constexpr (WREG) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            w[2 * e] = bf16lo_to_f32(wd[cc / 2 + e]);
+            w[2 * e + 1] = bf16hi_to_f32(wd[cc / 2 + e]);
+          }
+        } else if (wrow) {
           load_x32(wrow + col, w);
         } else {
 #pragma unroll
@@ -204,9 +332,11 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         store_x32(a.w_all + w_index(0) * dfs + static_cast<long long>(row) * a.f + col, w);
       }
     }
+    // Pair: the accumulator is released on rank 0's barrier.
+    const uint32_t acce0 = PAIR ? mapa_shared(smem_u32(acce), 0) : 0u;
     for (int i = 0; i < a.Nc; ++i) {
       const int ab = i & 1;
-      if (!mbar_wait(&accf[ab], (i >> 1) & 1, st, abort)) break;
+      if (!mbar_wait<PAIR>(&accf[ab], (i >> 1) & 1, st, abort)) break;
       tc_fence_after();
       const bool last = i + 1 == a.Nc;
 #pragma unroll
@@ -218,7 +348,10 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       }
       // The accumulator is free as soon as it has been read.
       tc_fence_before();
-      mbar_arrive(&acce[ab]);
+      if constexpr (PAIR)
+        mbar_arrive_cluster(acce0 + 8u * static_cast<uint32_t>(ab));
+      else
+        mbar_arrive(&acce[ab]);
 #pragma unroll
       for (int cc = 0; cc < HC; cc += 32) {
         const int col = c0 + cc;
@@ -226,7 +359,13 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         float v[32];
         if (!last) {
           if (!a.w_all) continue;
-          if (wrow) {
+          if constexpr (WREG) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              v[2 * e] = bf16lo_to_f32(wd[cc / 2 + e]);
+              v[2 * e + 1] = bf16hi_to_f32(wd[cc / 2 + e]);
+            }
+          } else if (wrow) {
             load_x32(wrow + col, v);
           } else {
 #pragma unroll
@@ -243,10 +382,20 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       }
     }
   }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+  if constexpr (PAIR) {
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc_pair(tmem, 512);
+    }
+  } else {
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
   }
 }
 

@@ -110,10 +110,11 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 
 // 2-D tensor map of element type E (bf16 or fp32): `outer` rows of `inner`
 // elements, row pitch in bytes, box of box_inner x box_outer elements,
-// 128-byte swizzle.
+// 128-byte swizzle unless given.
 template <class E>
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -121,7 +122,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
   const CUtensorMapDataType dt =
       sizeof(E) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -578,6 +579,36 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
   return TTCD_OK;
 }
 
+// The bf16 chunk scan on CTA pairs: `tiles` pair tiles, two CTAs each, launched
+// as clusters of two.
+ttcd_status launch_scan_pair(const Ctx& c, const CUtensorMap& mR, const CUtensorMap& mK,
+                             const ScanArgs<__nv_bfloat16>& a, int tiles) {
+  constexpr int STAGES = 6;
+  constexpr int smem = scan_smem_bytes<__nv_bfloat16, STAGES, true>();
+  auto kern = fastweight_scan_kernel<__nv_bfloat16, STAGES, true, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  TTCD_TRY(check_reg_split(reinterpret_cast<const void*>(kern), SCAN_THREADS, kScanRegSplit));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2u * static_cast<unsigned>(tiles));
+  cfg.blockDim = dim3(SCAN_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mR, mK, a, c.st) != cudaSuccess) {
+    cudaGetLastError();
+    return TTCD_ERR_CUDA;
+  }
+  TTCD_CHECK_LAUNCH();
+  return TTCD_OK;
+}
+
 // The chunk scan over R and the keys: Delta W_i = R_i^T K'_i, the fp32 exclusive
 // prefix S_i from state_in, and (w_all set) W_i = W_down + S_i per chunk.  With
 // `whole` set, the padded tokens of each sequence form one chunk: state_out is
@@ -593,9 +624,13 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
     CUtensorMap mR, mK;
     constexpr uint32_t BK = ElemTraits<E>::BK;
     constexpr bool MN = sizeof(E) == 2;
+    // bf16 with more than one 128-row tile of d: CTA pairs on 256 x 192 tiles.
+    const bool pair = MN && m.d > GEMM_BM;
     if (MN) {
       if (!make_map<E>(&mR, R, m.d, m.P, m.d * sizeof(E), BK, BK) ||
-          !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), BK, BK))
+          (pair ? !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), SCAN_PAIR_BOX, BK,
+                               CU_TENSOR_MAP_SWIZZLE_64B)
+                : !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), BK, BK)))
         return TTCD_ERR_CUDA;
     } else {
       E* Rt = at<E>(ws, L, B_RT);
@@ -618,10 +653,13 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
     a.state_in = state_in;
     a.state_out = state_out;
     a.w_all = w_all;
-    a.tiles_m = cdiv(m.d, 128);
+    a.tiles_m = cdiv(m.d, pair ? 2 * GEMM_BM : GEMM_BM);
     a.tiles_n = cdiv(m.f, SCAN_BN);
     a.commit_pos = nullptr;
     a.commit_C = 1;
+    if constexpr (MN) {
+      if (pair) return launch_scan_pair(c, mR, mK, a, p->B * a.tiles_m * a.tiles_n);
+    }
     constexpr int STAGES = 4;
     constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
     auto kern = fastweight_scan_kernel<E, STAGES, MN>;

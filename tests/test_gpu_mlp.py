@@ -19,6 +19,11 @@ MLP_SHAPES = [
                head_dim=64, d_ff=384, w_S=1, w_T=1, chunk=256, conv_k=4),
     BlockShape("mlp_f32_chunk40", "f32", B=1, T=333, d_model=64, n_q_heads=1, n_kv_heads=1,
                head_dim=64, d_ff=128, w_S=1, w_T=1, chunk=40, conv_k=2),
+    # d and f ragged for the chunk scan's 256 x 192 CTA-pair tiles: the last
+    # pair of rows has one CTA with 64 valid rows and one with none, the last
+    # column tile 64 valid key columns in its first CTA and none in its second
+    BlockShape("mlp_bf16_pair_ragged", "bf16", B=2, T=700, d_model=320, n_q_heads=1,
+               n_kv_heads=1, head_dim=64, d_ff=448, w_S=1, w_T=1, chunk=192, conv_k=3),
     # bf16 shorter than one chunk: the fp32-operand route
     BlockShape("mlp_bf16_short", "bf16", B=2, T=70, d_model=128, n_q_heads=1, n_kv_heads=1,
                head_dim=64, d_ff=256, w_S=1, w_T=1, chunk=128, conv_k=4),
