@@ -315,11 +315,6 @@ __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes)
 __host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
   return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
-// The same for the 64-byte swizzle (layout code 4): 64-byte rows, atoms of
-// 8 rows = 512 bytes.
-__host__ __device__ constexpr uint32_t sdesc_hi_sw64(uint32_t sbo_bytes) {
-  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
-}
 // D[tmem] (+)= A[smem] * B[smem]^T from descriptor halves.
 __device__ __forceinline__ void mma_bf16_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
                                                uint32_t b_lo, uint32_t b_hi, uint32_t idesc,

@@ -21,14 +21,14 @@
 //
 // PAIR = true (bf16, token-major operands): a cluster of two CTAs shares one
 // 256 x 192 tile through M = 256 MMAs (tcgen05 .cta_group::2).  Each CTA loads
-// its own 128 rows of R and half of the tile's key columns (96, as three boxes
-// of 32 columns in the 64-byte swizzle), so each k-block moves 28 KB into each
-// SM instead of 40 KB: the operand bytes per FLOP from L2 drop by 30 %.  Rank 0
-// waits for both CTAs' bytes on its own full barriers, issues the MMAs and
-// commits them to both CTAs' stage and accumulator barriers; each CTA's
-// epilogue folds its own 128 rows and releases the accumulator on rank 0's
-// barrier.  Both CTAs end at a cluster barrier, so neither leaves while the
-// other's MMAs or arrivals can still touch its shared memory.
+// its own 128 rows of R and its half of the tile's key columns (96, as two
+// 64-column boxes whose last 32 columns the MMA does not read), so each
+// k-block moves 32 KB into each SM instead of 40 KB.  Rank 0 waits for both
+// CTAs' bytes on its own full barriers, issues the MMAs and commits them to
+// both CTAs' stage and accumulator barriers; each CTA's epilogue folds its own
+// 128 rows and releases the accumulator on rank 0's barrier.  Both CTAs end at
+// a cluster barrier, so neither leaves while the other's MMAs or arrivals can
+// still touch its shared memory.
 #pragma once
 #include "gemm.cuh"
 
@@ -55,42 +55,41 @@ struct ScanArgs {
 
 constexpr int SCAN_BN = 192;
 constexpr int SCAN_THREADS = 384;
-constexpr int SCAN_PAIR_BOX = 32;  // key columns per 64-byte-swizzled box of a pair CTA
 
 // Rows of d per tile (per pair of CTAs when PAIR).
 template <bool PAIR>
 constexpr int scan_tile_rows() {
   return PAIR ? 2 * GEMM_BM : GEMM_BM;
 }
+// Key columns a CTA loads per k-block: all 192, or in a pair two boxes of 64
+// for its 96.
+template <bool PAIR>
+constexpr int scan_b_cols() {
+  return PAIR ? 128 : SCAN_BN;
+}
 template <class E, bool PAIR>
 constexpr int scan_stage_bytes() {
-  return GEMM_BM * 128 + (PAIR ? SCAN_BN / 2 : SCAN_BN) * 128;
+  return GEMM_BM * 128 + scan_b_cols<PAIR>() * 128;
 }
 template <class E, int STAGES, bool PAIR>
 constexpr int scan_smem_bytes() {
   return 1024 + STAGES * scan_stage_bytes<E, PAIR>() + 256;
 }
 
-template <class E, int STAGES, bool MN, bool PAIR = false, bool B64 = PAIR>
+template <class E, int STAGES, bool MN, bool PAIR = false>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
     fastweight_scan_kernel(const __grid_constant__ CUtensorMap mapR,
                            const __grid_constant__ CUtensorMap mapK, const ScanArgs<E> a,
                            const DevStatus st) {
   static_assert(!PAIR || (MN && sizeof(E) == 2), "CTA pairs take bf16 token-major operands");
-  static_assert(!B64 || (MN && sizeof(E) == 2), "64-byte swizzled keys are bf16 token-major");
-  static_assert(!PAIR || B64, "a pair CTA's 96 key columns take the 64-byte swizzle");
   constexpr int BN = SCAN_BN;
   constexpr int BK = ElemTraits<E>::BK;  // tokens per k-block == MN elements per box
   constexpr int BOX_BYTES = BK * BK * static_cast<int>(sizeof(E));
-  constexpr int B_COLS = PAIR ? BN / 2 : BN;  // key columns this CTA loads
-  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = B_COLS * 128;
+  constexpr int B_COLS = PAIR ? BN / 2 : BN;  // key columns of the tile this CTA holds
+  constexpr int A_BYTES = GEMM_BM * 128, B_BYTES = scan_b_cols<PAIR>() * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static_assert(STAGE_BYTES == scan_stage_bytes<E, PAIR>(), "stage size");
   constexpr int KSTEP_BYTES = (32 / static_cast<int>(sizeof(E))) * 128;  // tokens per MMA x 128 B
-  // B64 (the pair's keys): 64-byte rows, so a K step of 16 tokens is 1024
-  // bytes and the 32-column panels lie one box (32 x 64 tokens x 2 B) apart.
-  constexpr int PBOX_BYTES = SCAN_PAIR_BOX * BK * 2;
-  constexpr int B_KSTEP_BYTES = B64 ? 16 * 64 : KSTEP_BYTES;
   constexpr uint32_t IDESC =
       idesc_f32acc(scan_tile_rows<PAIR>(), BN, ElemTraits<E>::FMT, MN, MN);
 
@@ -165,25 +164,17 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
               tma_load_2d_pair(sa + q * BOX_BYTES, &mapR, fb, m0 + q * BK, y);
             const int nb = n0 + static_cast<int>(rank) * B_COLS;
 #pragma unroll
-            for (int q = 0; q < B_COLS / SCAN_PAIR_BOX; ++q)
-              tma_load_2d_pair(sa + A_BYTES + q * PBOX_BYTES, &mapK, fb,
-                               nb + q * SCAN_PAIR_BOX, y);
+            for (int q = 0; q < 2; ++q)
+              tma_load_2d_pair(sa + A_BYTES + q * BOX_BYTES, &mapK, fb, nb + q * BK, y);
           } else {
             mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
             if constexpr (MN) {
 #pragma unroll
               for (int q = 0; q < GEMM_BM / BK; ++q)
                 tma_load_2d(sa + q * BOX_BYTES, &mapR, &full[s], m0 + q * BK, y);
-              if constexpr (B64) {
 #pragma unroll
-                for (int q = 0; q < BN / SCAN_PAIR_BOX; ++q)
-                  tma_load_2d(sa + A_BYTES + q * PBOX_BYTES, &mapK, &full[s],
-                              n0 + q * SCAN_PAIR_BOX, y);
-              } else {
-#pragma unroll
-                for (int q = 0; q < BN / BK; ++q)
-                  tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
-              }
+              for (int q = 0; q < BN / BK; ++q)
+                tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &mapK, &full[s], n0 + q * BK, y);
             } else {
               tma_load_2d(sa, &mapR, &full[s], y, m0);
               tma_load_2d(sa + A_BYTES, &mapK, &full[s], y, n0);
@@ -205,9 +196,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
       // MMA issuer (rank 0 of a pair): the whole warp walks the loop, one
       // elected lane issues.
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
-      constexpr uint32_t HI_B = B64 ? sdesc_hi_sw64(512) : HI;
       const uint32_t lo0 = sdesc_lo(smem_u32(smem), MN ? BOX_BYTES : 16);
-      const uint32_t lo0_b = sdesc_lo(smem_u32(smem), B64 ? PBOX_BYTES : (MN ? BOX_BYTES : 16));
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait<PAIR>(bar, parity, st, abort));
       };
@@ -222,17 +211,16 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
           if (!wait(&full[s], (it / STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_lo = lo0 + ((s * STAGE_BYTES) >> 4);
-          const uint32_t b_lo = lo0_b + ((s * STAGE_BYTES + A_BYTES) >> 4);
+          const uint32_t b_lo = a_lo + (A_BYTES >> 4);
           if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t off = (MN ? k * KSTEP_BYTES : k * 32) >> 4;
-              const uint32_t off_b = (MN ? k * B_KSTEP_BYTES : k * 32) >> 4;
               if constexpr (PAIR)
-                mma_bf16_ss_lh_pair(tmem + ab * BN, a_lo + off, HI, b_lo + off_b, HI_B, IDESC,
+                mma_bf16_ss_lh_pair(tmem + ab * BN, a_lo + off, HI, b_lo + off, HI, IDESC,
                                     (kb | k) != 0 ? 1u : 0u);
               else
-                mma_ss_lh<E>(tmem + ab * BN, a_lo + off, HI, b_lo + off_b, HI_B, IDESC,
+                mma_ss_lh<E>(tmem + ab * BN, a_lo + off, HI, b_lo + off, HI, IDESC,
                              (kb | k) != 0 ? 1u : 0u);
             }
             if constexpr (PAIR)

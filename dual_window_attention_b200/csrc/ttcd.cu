@@ -110,11 +110,10 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 
 // 2-D tensor map of element type E (bf16 or fp32): `outer` rows of `inner`
 // elements, row pitch in bytes, box of box_inner x box_outer elements,
-// 128-byte swizzle unless given.
+// 128-byte swizzle.
 template <class E>
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
-              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -122,7 +121,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
   const CUtensorMapDataType dt =
       sizeof(E) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -628,9 +627,7 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
     const bool pair = MN && m.d > GEMM_BM;
     if (MN) {
       if (!make_map<E>(&mR, R, m.d, m.P, m.d * sizeof(E), BK, BK) ||
-          (pair ? !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), SCAN_PAIR_BOX, BK,
-                               CU_TENSOR_MAP_SWIZZLE_64B)
-                : !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), BK, BK)))
+          !make_map<E>(&mK, Kp, m.f, m.P, m.f * sizeof(E), BK, BK))
         return TTCD_ERR_CUDA;
     } else {
       E* Rt = at<E>(ws, L, B_RT);
