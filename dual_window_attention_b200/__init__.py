@@ -98,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_test_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
     lib.ttcd_test_exp2_poly.argtypes = [vp, vp, i, vp]
     lib.ttcd_test_exp2_poly.restype = i
+    lib.ttcd_attn_timeline_read.argtypes = [ctypes.POINTER(ctypes.c_longlong), sz]
+    lib.ttcd_attn_timeline_read.restype = i
     lib.ttcd_status_string.argtypes = [i]
     lib.ttcd_status_string.restype = ctypes.c_char_p
     lib.ttcd_version.restype = ctypes.c_char_p
@@ -681,6 +683,16 @@ def test_bounded_wait(timeout_ns: int, status: Optional[torch.Tensor] = None, st
     ``timeout_ns`` and records a timeout in ``status`` (a workspace or decode
     state) or, when None, in the per-device word."""
     return load_library().ttcd_test_bounded_wait(timeout_ns, _ptr(status), _stream(stream))
+
+
+def attn_timeline_read():
+    """The instrumented attention kernel's clock64 marks of its last launch as a
+    [2 heads, 128 visits, 8 marks] int64 tensor (libttcd_timeline.so only; the
+    normal library raises TTCDError with status unsupported)."""
+    n = 2 * 128 * 8
+    buf = (ctypes.c_longlong * n)()
+    _check(load_library().ttcd_attn_timeline_read(buf, n), "ttcd_attn_timeline_read")
+    return torch.tensor(list(buf), dtype=torch.int64).view(2, 128, 8)
 
 
 def test_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:

@@ -1,6 +1,11 @@
 """Build libttcd.so in-tree for sm_100a with nvcc (no GPU needed to build).
 
     python -m dual_window_attention_b200.build [--verbose-ptxas]
+    python -m dual_window_attention_b200.build --attn-timeline
+
+The second form builds libttcd_timeline.so, the same library with the attention
+kernel's clock64 timeline compiled in (TTCD_ATTN_TIMELINE=1), for
+`python -m dual_window_attention_b200.timeline`.
 """
 from __future__ import annotations
 
@@ -13,6 +18,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libttcd.so")
+TIMELINE_LIB = os.path.join(PKG, "libttcd_timeline.so")
 SOURCES = [os.path.join(CSRC, "ttcd.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(ROOT, "include", "ttcd.h")]
@@ -32,19 +38,22 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPS)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not needs_build():
+def build(force: bool = False, ptxas_verbose: bool = False, attn_timeline: bool = False) -> str:
+    out = TIMELINE_LIB if attn_timeline else LIB
+    if not force and not attn_timeline and not needs_build():
         return LIB
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2", "-shared",
-           "-I" + os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *SOURCES]
+           "-I" + os.path.join(ROOT, "include"), "-o", out + ".tmp", *SOURCES]
+    if attn_timeline:
+        cmd.insert(1, "-DTTCD_ATTN_TIMELINE=1")
     if ptxas_verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                attn_timeline="--attn-timeline" in sys.argv))

@@ -57,6 +57,35 @@ struct AttnArgs {
   int q_begin;
 };
 
+// Per-visit clock64 timeline of the CTA with blockIdx.x == 0 (the longest
+// query tile of the first head pair), recorded by lane 0 of each head's first
+// softmax warp and by the MMA issuer.  Compiled in only with
+// -DTTCD_ATTN_TIMELINE=1 (`build --attn-timeline` makes a separate library);
+// the library build leaves it out.  Marks per (head, visit):
+//   0 S ready (its mbarrier completed)     4 P stored and published
+//   1 S in registers                       5 MMA issuer: PV of this visit issued
+//   2 row maximum formed                   6 MMA issuer: QK of the next visit issued
+//   3 rescale check done
+#ifndef TTCD_ATTN_TIMELINE
+#define TTCD_ATTN_TIMELINE 0
+#endif
+constexpr int ATT_TL_VISITS = 128;
+constexpr int ATT_TL_MARKS = 8;
+#if TTCD_ATTN_TIMELINE
+__device__ long long g_attn_timeline[2 * ATT_TL_VISITS * ATT_TL_MARKS];
+#endif
+__device__ __forceinline__ void attn_mark(bool on, int h, int v, int k) {
+#if TTCD_ATTN_TIMELINE
+  if (on && v < ATT_TL_VISITS) {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t)::"memory");
+    g_attn_timeline[(h * ATT_TL_VISITS + v) * ATT_TL_MARKS + k] = t;
+  }
+#else
+  (void)on; (void)h; (void)v; (void)k;
+#endif
+}
+
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;
 constexpr int ATT_KS = 2;  // K stages
@@ -362,11 +391,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           ok = false;
           break;
         }
+        const bool tl = TTCD_ATTN_TIMELINE && blockIdx.x == 0 && lane == 0;
         for (int h = 0; h < nh; ++h) {
           if (!wait(&p_full[h], v & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(h, v);
+          attn_mark(tl, h, v, 5);
           if (more) issue_qk(h, v + 1);
+          attn_mark(tl, h, v, 6);
         }
         if (!ok) break;
         if (elect_one()) {
@@ -401,11 +433,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // split form before its first visible key); O is zero for such a row.
     float m_ref = -INFINITY, l = 0.f;
     bool ok = active;
+    const bool tl = TTCD_ATTN_TIMELINE && blockIdx.x == 0 && quarter == 0 && lane == 0;
     for (int v = 0; v < vis.nv && ok; ++v) {
       const int j = vis.tile(v);
       const int k0 = q0 - ATT_BN * j;
       const bool ph2 = v >= vis.vX;
       if (!mbar_wait(&s_full[h_local], v & 1, st, abort)) { ok = false; break; }
+      attn_mark(tl, h_local, v, 0);
       tc_fence_after();
       if (v == vis.vX) {
         // end of the student phase: O / l is o_S (PV of every earlier tile has landed)
@@ -418,6 +452,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       float s[128];
       tmem_ld_cols<128>(s_addr, s);
+      attn_mark(tl, h_local, v, 1);
       // visible key columns [lo, hi] of this row in this tile
       const int lo = ph2 ? t - a.w_T + 1 - k0 : t - a.w_S + 1 - k0;
       const int hi = ph2 ? t - a.w_S - k0 : t - k0;
@@ -437,6 +472,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mx4[q] = fmaxf(m, s[32 * q + 31]);
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      attn_mark(tl, h_local, v, 2);
       const float m_tile = mx * sl2;
       const bool fresh = m_ref == -INFINITY;
       const bool grow = !fresh && m_tile > m_ref + ATT_RESCALE_THRESHOLD;
@@ -448,6 +484,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         m_ref = m_new;
       }
       if (fresh) m_ref = m_tile;  // may stay -inf: a row with no visible key in this tile
+      attn_mark(tl, h_local, v, 3);
       // exponentials, row sum, bf16 pack (a row still at -inf has only masked scores)
       const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
       const uint64_t sc2 = f2pack(sl2, sl2);
@@ -494,6 +531,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[h_local]);
+      attn_mark(tl, h_local, v, 4);
     }
     // ------------------------------------------------------------------ epilogue
     if (ok && mbar_wait(&o_done[h_local], (vis.nv - 1) & 1, st, abort)) {

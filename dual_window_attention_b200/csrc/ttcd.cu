@@ -1345,6 +1345,25 @@ __global__ void bounded_wait_test_kernel(DevStatus st) {
   __syncthreads();
 }
 
+// Copies the attention kernel's clock64 timeline (instrumented build only).
+ttcd_status ttcd_attn_timeline_read(long long* out, size_t n) {
+#if TTCD_ATTN_TIMELINE
+  const size_t total = 2 * ATT_TL_VISITS * ATT_TL_MARKS;
+  if (!out || n < total) return TTCD_ERR_INVALID_ARG;
+  if (cudaMemcpyFromSymbol(out, g_attn_timeline, total * sizeof(long long)) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  void* dev = nullptr;  // cleared for the next launch
+  if (cudaGetSymbolAddress(&dev, g_attn_timeline) != cudaSuccess ||
+      cudaMemset(dev, 0, total * sizeof(long long)) != cudaSuccess)
+    return TTCD_ERR_CUDA;
+  return TTCD_OK;
+#else
+  (void)out;
+  (void)n;
+  return TTCD_ERR_UNSUPPORTED;
+#endif
+}
+
 // Evaluates the attention kernel's FMA-pipe 2^x (exp2_poly2) at x[0..n-1].
 __global__ void exp2_poly_test_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
   const long long i = 2ll * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);

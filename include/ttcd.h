@@ -596,6 +596,20 @@ ttcd_status ttcd_test_bounded_wait(uint64_t timeout_ns, void* status, void* stre
  */
 ttcd_status ttcd_test_exp2_poly(const float* x, float* y, int n, void* stream);
 
+/*
+ * ttcd_attn_timeline_read — diagnostic.  In a library built with
+ * -DTTCD_ATTN_TIMELINE=1 (`python -m dual_window_attention_b200.build
+ * --attn-timeline`, a separate libttcd_timeline.so) the fused attention kernel
+ * records, for the CTA with blockIdx.x == 0, clock64 values at the phase
+ * boundaries of every visit: [head 2][visit 128][mark 8] int64, marks 0 S ready,
+ * 1 S in registers, 2 row maximum, 3 rescale check, 4 P published, 5 PV issued,
+ * 6 next QK issued (7 unused, 0 where not reached).  Copies the 2048 values of
+ * the last launch to host `out` (n >= 2048) and clears them.  Synchronous.
+ * Returns TTCD_ERR_UNSUPPORTED in the normal build.  The paper has no
+ * counterpart; it exists to reproduce the attention kernel's timing diagnosis.
+ */
+ttcd_status ttcd_attn_timeline_read(long long* out, size_t n);
+
 /* Number of kernels this library has launched since it was loaded (process-wide
  * diagnostic counter, atomic). */
 unsigned long long ttcd_kernel_launch_count(void);

@@ -233,3 +233,10 @@ def test_backward_sizes_and_host_checks(lib):
     assert att(*bad) == ttcd.ERR_INVALID_ARG
     bad = list(a); bad[21] = n_att - 1
     assert att(*bad) == ttcd.ERR_WORKSPACE
+
+
+def test_attention_timeline_is_compiled_out_of_the_library(lib):
+    """The clock64 timeline of the attention kernel exists only in the separate
+    instrumented build; the library reports it as unsupported, touching no GPU."""
+    buf = (ctypes.c_longlong * 2048)()
+    assert lib.ttcd_attn_timeline_read(buf, 2048) == ttcd.ERR_UNSUPPORTED
