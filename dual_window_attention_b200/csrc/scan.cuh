@@ -71,9 +71,17 @@ template <class E, bool PAIR>
 constexpr int scan_stage_bytes() {
   return GEMM_BM * 128 + scan_b_cols<PAIR>() * 128;
 }
+// bf16 W entries leave through shared memory: per epilogue warp 32 rows of 96
+// columns (192 bytes) at a 208-byte pitch, so that both the row-per-thread
+// writes and the row-contiguous reads are free of bank conflicts.
+constexpr int SCAN_WROW = 208;
+template <class E>
+constexpr int scan_wstage_bytes() {
+  return sizeof(E) == 2 ? 8 * 32 * SCAN_WROW : 0;
+}
 template <class E, int STAGES, bool PAIR>
 constexpr int scan_smem_bytes() {
-  return 1024 + STAGES * scan_stage_bytes<E, PAIR>() + 256;
+  return 1024 + STAGES * scan_stage_bytes<E, PAIR>() + scan_wstage_bytes<E>() + 256;
 }
 
 template <class E, int STAGES, bool MN, bool PAIR = false>
@@ -96,7 +104,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* wstage = smem + STAGES * STAGE_BYTES;  // bf16: W entry staging rows
+  uint64_t* full = reinterpret_cast<uint64_t*>(wstage + scan_wstage_bytes<E>());
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
@@ -273,9 +282,38 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     // bf16: the thread's HC columns of W_down stay in registers as packed
     // pairs, so the chunk loop below issues no global loads (they would queue
     // in L2 behind the operand stream and stall the release of the next
-    // accumulator).
+    // accumulator), and each W entry is packed into the warp's staging rows
+    // and written row-contiguously: a store instruction then covers about
+    // three rows' 192-byte segments instead of 16 bytes in each of 32 rows.
     constexpr bool WREG = sizeof(E) == 2;
     uint32_t wd[WREG ? HC / 2 : 1];
+    uint8_t* wst = wstage + (warp - 4) * 32 * SCAN_WROW;
+    auto emit_w = [&](int j) {
+      __syncwarp();  // the previous entry's reads of the staging rows are done
+#pragma unroll
+      for (int k = 0; k < HC / 8; ++k) {  // 16-byte chunk k: columns 8k .. 8k+7
+        uint32_t pk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 8 * k + 2 * u;
+          pk[u] = pack_bf16x2(bf16lo_to_f32(wd[e / 2]) + S[e], bf16hi_to_f32(wd[e / 2]) + S[e + 1]);
+        }
+        *reinterpret_cast<uint4*>(wst + lane * SCAN_WROW + 16 * k) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      __syncwarp();
+      E* dst = a.w_all + w_index(j) * dfs;
+      const int r0 = m0 + q * 32;
+#pragma unroll 1
+      for (int it = 0; it < HC / 8; ++it) {  // the warp's 32 x 12 chunks, 32 at a time
+        const int idx = it * 32 + lane;
+        const int rr = idx / (HC / 8), kk = idx - rr * (HC / 8);
+        const int grow = r0 + rr, gcol = c0 + 8 * kk;
+        if (grow < a.d && gcol < a.f)
+          *reinterpret_cast<uint4*>(dst + static_cast<long long>(grow) * a.f + gcol) =
+              *reinterpret_cast<const uint4*>(wst + rr * SCAN_WROW + 16 * kk);
+      }
+    };
     // S_0 = state_in (or 0); W_0 = W_down + S_0 (W_down null: 0).
 #pragma unroll
     for (int cc = 0; cc < HC; cc += 32) {
@@ -300,16 +338,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
           wd[cc / 2 + 4 * u + 2] = w4.z;
           wd[cc / 2 + 4 * u + 3] = w4.w;
         }
-      }
-      if (row_ok && col < a.f && a.w_all) {
+      } else if (row_ok && col < a.f && a.w_all) {
         float w[32];
-        if constexpr (WREG) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            w[2 * e] = bf16lo_to_f32(wd[cc / 2 + e]);
-            w[2 * e + 1] = bf16hi_to_f32(wd[cc / 2 + e]);
-          }
-        } else if (wrow) {
+        if (wrow) {
           load_x32(wrow + col, w);
         } else {
 #pragma unroll
@@ -319,6 +350,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         for (int e = 0; e < 32; ++e) w[e] += s32[e];
         store_x32(a.w_all + w_index(0) * dfs + static_cast<long long>(row) * a.f + col, w);
       }
+    }
+    if constexpr (WREG) {
+      if (a.w_all) emit_w(0);
     }
     // Pair: the accumulator is released on rank 0's barrier.
     const uint32_t acce0 = PAIR ? mapa_shared(smem_u32(acce), 0) : 0u;
@@ -340,20 +374,17 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         mbar_arrive_cluster(acce0 + 8u * static_cast<uint32_t>(ab));
       else
         mbar_arrive(&acce[ab]);
+      if constexpr (WREG) {
+        if (!last && a.w_all) emit_w(i + 1);
+      }
 #pragma unroll
       for (int cc = 0; cc < HC; cc += 32) {
         const int col = c0 + cc;
         if (!row_ok || col >= a.f) continue;
         float v[32];
         if (!last) {
-          if (!a.w_all) continue;
-          if constexpr (WREG) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              v[2 * e] = bf16lo_to_f32(wd[cc / 2 + e]);
-              v[2 * e + 1] = bf16hi_to_f32(wd[cc / 2 + e]);
-            }
-          } else if (wrow) {
+          if (WREG || !a.w_all) continue;
+          if (wrow) {
             load_x32(wrow + col, v);
           } else {
 #pragma unroll

@@ -582,7 +582,7 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
 // as clusters of two.
 ttcd_status launch_scan_pair(const Ctx& c, const CUtensorMap& mR, const CUtensorMap& mK,
                              const ScanArgs<__nv_bfloat16>& a, int tiles) {
-  constexpr int STAGES = 6;
+  constexpr int STAGES = 5;
   constexpr int smem = scan_smem_bytes<__nv_bfloat16, STAGES, true>();
   auto kern = fastweight_scan_kernel<__nv_bfloat16, STAGES, true, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -658,7 +658,7 @@ ttcd_status launch_scan(const Ctx& c, const ttcd_block_params* p, const Layout& 
       if (pair) return launch_scan_pair(c, mR, mK, a, p->B * a.tiles_m * a.tiles_n);
     }
     constexpr int STAGES = 4;
-    constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+    constexpr int smem = scan_smem_bytes<E, STAGES, false>();
     auto kern = fastweight_scan_kernel<E, STAGES, MN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
@@ -1506,7 +1506,7 @@ ttcd_status dec_commit(const Ctx& c, const ttcd_block_params* p, void* state, co
   a.commit_pos = commit_pos;
   a.commit_C = p->chunk;
   constexpr int STAGES = 4;
-  constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+  constexpr int smem = scan_smem_bytes<bf, STAGES, false>();
   auto kern = fastweight_scan_kernel<bf, STAGES, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -1870,7 +1870,7 @@ ttcd_status launch_tsum(const Ctx& c, const __nv_bfloat16* A, long long lda, int
   a.tiles_n = cdiv(n_dim, SCAN_BN);
   a.commit_C = 1;
   constexpr int STAGES = 4;
-  constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+  constexpr int smem = scan_smem_bytes<bf, STAGES, false>();
   auto kern = fastweight_scan_kernel<bf, STAGES, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
@@ -1991,7 +1991,7 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
     a.commit_C = 1;
     a.reverse = true;
     constexpr int STAGES = 4;
-    constexpr int smem = gemm_smem_bytes<SCAN_BN, STAGES>();
+    constexpr int smem = scan_smem_bytes<bf, STAGES, false>();
     auto kern = fastweight_scan_kernel<bf, STAGES, true>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TTCD_ERR_CUDA;
