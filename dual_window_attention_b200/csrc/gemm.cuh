@@ -37,6 +37,26 @@ struct GemmGeom {
   int tiles_n;          // column tiles
   int b_group_rows;     // B row offset per group (0 = shared B)
   __host__ __device__ int total() const { return n_seq * Nc * tiles_m * tiles_n; }
+  // CTA pairs: pair tile t covers row tiles 2p and 2p + 1 of one group; `rank`
+  // picks this CTA's.  True while the pair's first tile has rows; the second
+  // may have none (valid_rows 0), and its CTA still takes part in the MMAs.
+  __host__ __device__ int tiles_m2() const { return (tiles_m + 1) / 2; }
+  __host__ __device__ int total_pairs() const { return n_seq * Nc * tiles_m2() * tiles_n; }
+  __device__ bool tile_pair(int t, int rank, TileCtx& c) const {
+    const int tn = t % tiles_n;
+    const int r = t / tiles_n;
+    const int pm = r % tiles_m2();
+    const int g = r / tiles_m2();
+    const int b = g / Nc, i = g % Nc;
+    const int len = min(C, T - i * C);
+    const int m0 = (2 * pm + rank) * GEMM_BM;
+    c.valid_rows = max(0, min(GEMM_BM, len - m0));
+    c.row0 = b * T + i * C + m0;
+    c.tn = tn;
+    c.group = g;
+    c.b_row0 = g * b_group_rows;
+    return len - 2 * pm * GEMM_BM > 0;
+  }
   __device__ bool tile(int t, TileCtx& c) const {
     const int tn = t % tiles_n;
     const int r = t / tiles_n;
@@ -272,8 +292,16 @@ struct EpiStage {
 // N-elements x 64 K-rows, leading-byte offset = one box, 16 K-rows (2048 bytes)
 // per MMA step.  With row groups (b_group_rows > 0) group g's B^T starts at row
 // g * b_group_rows, so K must then be a multiple of 64.
+//
+// PAIR = true (bf16, one K-major B, plain row tiles): clusters of two CTAs run
+// 256-row tiles as M = 256 MMAs (tcgen05 .cta_group::2).  Each CTA loads its
+// own 128 rows of A and half of the tile's B rows (B is given with BN/2-row
+// boxes), so a k-block moves a third less into each SM.  Rank 0 counts both
+// CTAs' bytes on its full barriers, issues the MMAs and commits them to both
+// CTAs' barriers; each CTA's epilogue handles its own 128 rows and releases
+// the accumulator on rank 0's barrier.
 template <class E, int BN, int STAGES, bool DUAL_B, class Epi, class Geom = GemmGeom,
-          bool B_MN = false>
+          bool B_MN = false, bool PAIR = false>
 __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapB0,
@@ -283,12 +311,16 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
                    const Epi epi, const DevStatus st) {
   constexpr bool STAGED = Epi::kStaged;
   constexpr int A_BYTES = GEMM_BM * 128;
-  constexpr int B_BYTES = BN * 128;
+  constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * 128;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
   static_assert(!B_MN || (sizeof(E) == 2 && !DUAL_B), "MN-major B: bf16, single B operand");
-  constexpr uint32_t IDESC = idesc_f32acc(GEMM_BM, BN, ElemTraits<E>::FMT, false, B_MN);
+  static_assert(!PAIR || (sizeof(E) == 2 && !DUAL_B && !B_MN && !Geom::kPaired &&
+                          !EpiSelfRelease<Epi>::value),
+                "CTA pairs: bf16, one K-major B, plain row tiles, kernel-released accumulator");
+  constexpr uint32_t IDESC =
+      idesc_f32acc(PAIR ? 2 * GEMM_BM : GEMM_BM, BN, ElemTraits<E>::FMT, false, B_MN);
   constexpr int MN_BOX_BYTES = 64 * 64 * 2;  // 64 N-elements x 64 K-rows, bf16
   constexpr int BK = ElemTraits<E>::BK;
 
@@ -321,7 +353,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 32 * EpiWarps<Epi>::value);
+      mbar_init(&acce[b], (PAIR ? 2 : 1) * 32 * EpiWarps<Epi>::value);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -331,14 +363,38 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     if (DUAL_B) tma_prefetch_map(&mapB1);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
     tc_fence_before();
   }
-  __syncthreads();
+  // A pair meets here before any arrival or byte count crosses to rank 0.
+  if constexpr (PAIR)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = geo.total();
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  // Tiles of this CTA: pair tiles (one per cluster) or row tiles.
+  const int total = [&]() {
+    if constexpr (PAIR)
+      return geo.total_pairs();
+    else
+      return geo.total();
+  }();
+  const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  auto get_tile = [&](int t, TileCtx& c) -> bool {
+    if constexpr (PAIR)
+      return geo.tile_pair(t, static_cast<int>(rank), c);
+    else
+      return geo.tile(t, c);
+  };
   const int nk = (geo.K + BK - 1) / BK;
   constexpr int EPI0 = gemm_epi_warp0<Epi>();
   // 8 epilogue warps: the launch's 384 x 168 registers are split 128 x 56 (warps
@@ -351,15 +407,25 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
       // ---------------------------------------------------------------- producer
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const uint32_t full0 = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+      for (int t = t_first; t < total && ok; t += t_step) {
         TileCtx c;
-        if (!geo.tile(t, c)) continue;
+        if (!get_tile(t, c)) continue;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, st, abort)) { ok = false; break; }
+          if (!mbar_wait<PAIR>(&empty[s], ph ^ 1, st, abort)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
+          if constexpr (PAIR) {
+            // both CTAs' bytes land on rank 0's full barrier
+            const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
+            tma_load_2d_pair(sa, &mapA, fb, kb * BK, c.row0);
+            tma_load_2d_pair(sb, &mapB0, fb, kb * BK,
+                             c.b_row0 + c.tn * BN + static_cast<int>(rank) * (BN / 2));
+            continue;
+          }
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           if constexpr (Geom::kPaired) {  // two 64-row boxes: teacher rows, student rows
             tma_load_2d(sa, &mapA, &full[s], kb * BK, c.row0);
@@ -382,10 +448,16 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
           }
         }
       }
-      // Let every load this thread issued land before the CTA can exit.
+      // Let every load this thread issued land before the CTA can exit (a
+      // pair: until rank 0's MMAs have consumed them, so no commit to this
+      // CTA's stage barriers is still in flight either).
       volatile int no_abort = 0;
-      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-        mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
+      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j) {
+        if constexpr (PAIR)
+          mbar_wait<true>(&empty[j % STAGES], (j / STAGES) & 1, st, abort);
+        else
+          mbar_wait(&full[j % STAGES], (j / STAGES) & 1, st, &no_abort);
+      }
     }
   } else if (warp == 1) {
     if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
@@ -397,13 +469,13 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     // MN-major B: its leading-byte offset is one box (the low word differs by it)
     constexpr uint32_t B_LBO_FIX = B_MN ? ((MN_BOX_BYTES >> 4) - 1) << 16 : 0;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, st, abort));
+      return __all_sync(0xffffffffu, mbar_wait<PAIR>(bar, parity, st, abort));
     };
     int it = 0, j = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    bool ok = rank == 0;  // a pair's MMAs are issued by rank 0 alone
+    for (int t = t_first; t < total && ok; t += t_step) {
       TileCtx c;
-      if (!geo.tile(t, c)) continue;
+      if (!get_tile(t, c)) continue;
       const int ab = j & 1;
       if (!wait(&acce[ab], ((j >> 1) & 1) ^ 1)) break;
       tc_fence_after();
@@ -416,23 +488,49 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
         const uint32_t b_lo = a_lo + (A_BYTES >> 4) + B_LBO_FIX;
         if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // 4 MMAs of 32 bytes of K per 128-byte row
-            mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + (B_MN ? k * (2048 >> 4) : 2 * k), HI, IDESC,
-                         (kb | k) != 0 ? 1u : 0u);
-          mma_commit(&empty[s]);
+          for (int k = 0; k < 4; ++k) {  // 4 MMAs of 32 bytes of K per 128-byte row
+            if constexpr (PAIR)
+              mma_bf16_ss_lh_pair(d_tmem, a_lo + 2 * k, HI, b_lo + 2 * k, HI, IDESC,
+                                  (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + (B_MN ? k * (2048 >> 4) : 2 * k), HI,
+                           IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          if constexpr (PAIR)
+            mma_commit_pair_mask(&empty[s], 0x3);
+          else
+            mma_commit(&empty[s]);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (elect_one()) mma_commit(&accf[ab]);
+      if (elect_one()) {
+        if constexpr (PAIR)
+          mma_commit_pair_mask(&accf[ab], 0x3);
+        else
+          mma_commit(&accf[ab]);
+      }
       __syncwarp();
       ++j;
     }
-    // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
-    if (elect_one()) mma_commit(drain);
-    __syncwarp();
-    volatile int no_abort = 0;
-    mbar_wait(drain, 0, st, &no_abort);
+    if (!PAIR || rank == 0) {
+      // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
+      if (elect_one()) {
+        if constexpr (PAIR)
+          mma_commit_pair_own(drain);
+        else
+          mma_commit(drain);
+      }
+      __syncwarp();
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, st, &no_abort);
+      if constexpr (PAIR) {
+        // the epilogues' releases of the last two accumulators (half of them
+        // arrive from the other CTA) land before this CTA may leave
+        for (int jj = j; jj < j + 2; ++jj)
+          if (jj >= 2) mbar_wait<true>(&acce[jj & 1], ((jj >> 1) & 1) ^ 1, st, abort);
+      }
+    }
   } else if (warp < EPI0) {
     if constexpr (SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
   } else {
@@ -444,13 +542,14 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     EpiStage stg{STAGED ? staging + ((warp - EPI0) & 3) * 8192 : nullptr, &mapOut, &mapOut2, 0};
     stg.xbars = xbars;
     int j = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    const uint32_t acce0 = PAIR ? mapa_shared(smem_u32(acce), 0) : 0u;
+    for (int t = t_first; t < total; t += t_step) {
       TileCtx c;
-      if (!geo.tile(t, c)) continue;
+      if (!get_tile(t, c)) continue;
       const int ab = j & 1;
       // per-row inputs of the epilogue are fetched while the tile is still computing
       const float pre = epi.pre(c, r);
-      bool ok = mbar_wait(&accf[ab], (j >> 1) & 1, st, abort);
+      bool ok = mbar_wait<PAIR>(&accf[ab], (j >> 1) & 1, st, abort);
       if constexpr (Epi::kCollective) ok = epi_bar_and<32 * EpiWarps<Epi>::value>(ok);
       if (!ok) break;
       tc_fence_after();
@@ -459,16 +558,29 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
                            stg, pre);
       if constexpr (!EpiSelfRelease<Epi>::value) {
         tc_fence_before();
-        mbar_arrive(&acce[ab]);
+        if constexpr (PAIR)
+          mbar_arrive_cluster(acce0 + 8u * static_cast<uint32_t>(ab));
+        else
+          mbar_arrive(&acce[ab]);
       }
       ++j;
     }
     stg.drain();
   }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+  if constexpr (PAIR) {
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+  } else {
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, TMEM_COLS);
+    }
   }
 }
 
@@ -476,10 +588,10 @@ template <int BN, int STAGES, bool STAGED = false>
 constexpr int gemm_smem_bytes() {
   return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + (STAGED ? 4 * 8192 : 0) + 256;
 }
-template <class Epi, int BN, int STAGES>
+template <class Epi, int BN, int STAGES, bool PAIR = false>
 constexpr int gemm_smem_bytes_for() {
-  return 1024 + STAGES * (GEMM_BM * 128 + BN * 128) + EpiStagingBytes<Epi>::value +
-         8 * EpiExtraBars<Epi>::value + 256;
+  return 1024 + STAGES * (GEMM_BM * 128 + (PAIR ? BN / 2 : BN) * 128) +
+         EpiStagingBytes<Epi>::value + 8 * EpiExtraBars<Epi>::value + 256;
 }
 
 // ------------------------------------------------------------------ epilogues

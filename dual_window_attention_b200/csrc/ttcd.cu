@@ -168,26 +168,53 @@ bool make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
   return make_map<OutT>(m, ptr, cols, rows, ld_elems * sizeof(OutT), 128 / sizeof(OutT), 32);
 }
 
+// PAIR: CTA pairs on 256-row tiles (plain row tiles, one K-major B whose map
+// has BN/2-row boxes), launched as clusters of two.
 template <class E, int BN, int STAGES, bool DUAL, class Epi, class Geom = GemmGeom,
-          bool B_MN = false>
+          bool B_MN = false, bool PAIR = false>
 ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B0,
                         const CUtensorMap& B1, const CUtensorMap* out_map, const Geom& geo,
                         const Epi& epi, const CUtensorMap* out_map2 = nullptr) {
-  const int total = geo.total();
+  int total;
+  if constexpr (PAIR)
+    total = geo.total_pairs();
+  else
+    total = geo.total();
   if (total <= 0) return TTCD_OK;
   if (Epi::kStaged && !out_map) return TTCD_ERR_INVALID_ARG;
-  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom, B_MN>;
-  constexpr int smem = gemm_smem_bytes_for<Epi, BN, STAGES>();
+  auto kern = gemm_tc_kernel<E, BN, STAGES, DUAL, Epi, Geom, B_MN, PAIR>;
+  constexpr int smem = gemm_smem_bytes_for<Epi, BN, STAGES, PAIR>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
-  const int grid = total < c.sms ? total : c.sms;
   if constexpr (EpiWarps<Epi>::value == 8) {
     const ttcd_status rs = check_reg_split(reinterpret_cast<const void*>(kern), gemm_threads<Epi>(),
                                            kGemm8RegSplit);
     if (rs != TTCD_OK) return rs;
   }
-  kern<<<grid, gemm_threads<Epi>(), smem, c.s>>>(A, B0, B1, out_map ? *out_map : A,
-                                           out_map2 ? *out_map2 : A, geo, epi, c.st);
+  const CUtensorMap& o1 = out_map ? *out_map : A;
+  const CUtensorMap& o2 = out_map2 ? *out_map2 : A;
+  if constexpr (PAIR) {
+    const int pairs = total < c.sms / 2 ? total : c.sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * static_cast<unsigned>(pairs));
+    cfg.blockDim = dim3(gemm_threads<Epi>());
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, A, B0, B1, o1, o2, geo, epi, c.st) != cudaSuccess) {
+      cudaGetLastError();
+      return TTCD_ERR_CUDA;
+    }
+  } else {
+    const int grid = total < c.sms ? total : c.sms;
+    kern<<<grid, gemm_threads<Epi>(), smem, c.s>>>(A, B0, B1, o1, o2, geo, epi, c.st);
+  }
   TTCD_CHECK_LAUNCH();
   return TTCD_OK;
 }
@@ -567,12 +594,17 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
   // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
-    if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, 256))
+    constexpr bool kPairR = sizeof(E) == 2;  // bf16: CTA pairs, B in 128-row boxes
+    if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, kPairR ? 128 : 256))
       return TTCD_ERR_CUDA;
     CUtensorMap mo;
     if (!make_out_map<E>(&mo, R, m.P, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiStore<E> e{R, m.d, m.d, kscale};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
+    if constexpr (kPairR)
+      TTCD_TRY((launch_gemm<E, 256, 6, false, EpiStore<E>, GemmGeom, false, true>(
+          c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
+    else
+      TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
   }
   stage_mark(c, mark + 4);
   return TTCD_OK;
