@@ -219,6 +219,25 @@ ttcd_status launch_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B
   return TTCD_OK;
 }
 
+// bf16 GEMMs over plain row tiles with one K-major B run on CTA pairs (256-row
+// tiles, 6 stages); their B operand is then mapped in 128-row boxes.
+template <class E>
+constexpr bool kPairGemm = sizeof(E) == 2;
+template <class E>
+constexpr uint32_t gemm_b_box() {
+  return kPairGemm<E> ? 128u : 256u;
+}
+template <class E, class Epi>
+ttcd_status launch_rows_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B,
+                             const CUtensorMap* out_map, const GemmGeom& geo, const Epi& epi,
+                             const CUtensorMap* out_map2 = nullptr) {
+  if constexpr (kPairGemm<E>)
+    return launch_gemm<E, 256, 6, false, Epi, GemmGeom, false, true>(c, A, B, B, out_map, geo, epi,
+                                                                     out_map2);
+  else
+    return launch_gemm<E, 256, 4, false>(c, A, B, B, out_map, geo, epi, out_map2);
+}
+
 GemmGeom plain_geom(long long rows, int N_tiles, int K) {
   GemmGeom g;
   g.n_seq = 1;
@@ -594,17 +613,12 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
   // R = D M^T (token-major), each row scaled by beta_t / ||Zbar_S[t]||.
   {
     CUtensorMap mA, mB;
-    constexpr bool kPairR = sizeof(E) == 2;  // bf16: CTA pairs, B in 128-row boxes
-    if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, kPairR ? 128 : 256))
+    if (!map_rows<E>(&mA, D, m.P, m.f, 128) || !map_rows<E>(&mB, M, m.d, m.f, gemm_b_box<E>()))
       return TTCD_ERR_CUDA;
     CUtensorMap mo;
     if (!make_out_map<E>(&mo, R, m.P, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiStore<E> e{R, m.d, m.d, kscale};
-    if constexpr (kPairR)
-      TTCD_TRY((launch_gemm<E, 256, 6, false, EpiStore<E>, GemmGeom, false, true>(
-          c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
-    else
-      TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e)));
+    TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, plain_geom(m.P, cdiv(m.d, 256), m.f), e));
   }
   stage_mark(c, mark + 4);
   return TTCD_OK;
@@ -718,7 +732,7 @@ ttcd_status mlp_back(const Ctx& c, const ttcd_block_params* p, const Layout& L, 
     CUtensorMap mA, mB;
     const void* zs = Zs ? static_cast<const void*>(Zs) : static_cast<const void*>(Z + m.BT * m.f);
     if (!map_rows<E>(&mA, zs, m.BT, m.f, 128) ||
-        !map_rows<E>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 256))
+        !map_rows<E>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, gemm_b_box<E>()))
       return TTCD_ERR_CUDA;
     GemmGeom g;
     g.n_seq = p->B;
@@ -732,7 +746,7 @@ ttcd_status mlp_back(const Ctx& c, const ttcd_block_params* p, const Layout& L, 
     CUtensorMap mo;
     if (!make_out_map<OutT>(&mo, y, m.BT, m.d, m.d)) return TTCD_ERR_CUDA;
     EpiResidual<OutT, ResT> e{y, m.d, h_S, m.d, m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e)));
+    TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, e));
   }
   stage_mark(c, mark + 6);
   return TTCD_OK;
@@ -893,7 +907,7 @@ ttcd_status block_qkv(const Ctx& c, const E* xin, const ttcd_block_weights* w,
   }
   stage_mark(c, 1);
   CUtensorMap mA, mB;
-  if (!map_rows<E>(&mA, xin, m.BT, m.d, 128) || !map_rows<E>(&mB, wg, m.dqkv, m.d, 256))
+  if (!map_rows<E>(&mA, xin, m.BT, m.d, 128) || !map_rows<E>(&mB, wg, m.dqkv, m.d, gemm_b_box<E>()))
     return TTCD_ERR_CUDA;
   GemmGeom g = plain_geom(m.BT, cdiv(m.dqkv, 256), m.d);
   if (n_halo > 0) {  // one row group per sequence
@@ -907,9 +921,9 @@ ttcd_status block_qkv(const Ctx& c, const E* xin, const ttcd_block_weights* w,
   if (!make_out_map<__nv_bfloat16>(&mo, qkv, rows_out, m.dqkv, m.dqkv)) return TTCD_ERR_CUDA;
   const int n_rope = (m.Hq + m.Hkv) * m.hd;
   switch (m.hd) {
-    case 32: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
-    case 64: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
-    default: TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo}))); break;
+    case 32: TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, EpiQKVRope<32>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo})); break;
+    case 64: TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, EpiQKVRope<64>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo})); break;
+    default: TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, EpiQKVRope<128>{qkv, m.dqkv, n_rope, p->T, rope, rstd_in, n_halo})); break;
   }
   stage_mark(c, 2);
   return TTCD_OK;
@@ -938,7 +952,7 @@ ttcd_status block_attend(const Ctx& c, const E* xin, const ttcd_block_weights* w
   {
     CUtensorMap mA, mB;
     if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
-        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, 256))
+        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, gemm_b_box<E>()))
       return TTCD_ERR_CUDA;
     const GemmGeom g = plain_geom(2 * m.BT, cdiv(m.d, 256), m.Hq * m.hd);
     // h_P = x + o_P W_o^T; stores h * g_mlp (gate/up operand), the student
@@ -948,7 +962,7 @@ ttcd_status block_attend(const Ctx& c, const E* xin, const ttcd_block_weights* w
         !make_out_map<float>(&mo2, h, m.BT, m.d, m.d))
       return TTCD_ERR_CUDA;
     EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
-    TTCD_TRY((launch_gemm<E, 256, 4, false>(c, mA, mB, mB, &mo, g, e, &mo2)));
+    TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, e, &mo2));
   }
   // The MLP RMSNorm's 1/rms per row, from the o_proj epilogue's partial sums.
   rms_rstd_kernel<<<cdiv(2 * m.BT, 256), 256, 0, c.s>>>(hssq, cdiv(m.d, 256), 2 * m.BT,
