@@ -316,9 +316,9 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
   static_assert(!B_MN || (sizeof(E) == 2 && !DUAL_B), "MN-major B: bf16, single B operand");
-  static_assert(!PAIR || (sizeof(E) == 2 && !DUAL_B && !B_MN && !Geom::kPaired &&
+  static_assert(!PAIR || (sizeof(E) == 2 && !DUAL_B && !Geom::kPaired &&
                           !EpiSelfRelease<Epi>::value),
-                "CTA pairs: bf16, one K-major B, plain row tiles, kernel-released accumulator");
+                "CTA pairs: bf16, one B operand, plain row tiles, kernel-released accumulator");
   constexpr uint32_t IDESC =
       idesc_f32acc(PAIR ? 2 * GEMM_BM : GEMM_BM, BN, ElemTraits<E>::FMT, false, B_MN);
   constexpr int MN_BOX_BYTES = 64 * 64 * 2;  // 64 N-elements x 64 K-rows, bf16
@@ -422,8 +422,16 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
             const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
             tma_load_2d_pair(sa, &mapA, fb, kb * BK, c.row0);
-            tma_load_2d_pair(sb, &mapB0, fb, kb * BK,
-                             c.b_row0 + c.tn * BN + static_cast<int>(rank) * (BN / 2));
+            if constexpr (B_MN) {  // this CTA's BN/2 columns as 64-column boxes
+#pragma unroll
+              for (int q = 0; q < BN / 128; ++q)
+                tma_load_2d_pair(sb + q * MN_BOX_BYTES, &mapB0, fb,
+                                 c.tn * BN + static_cast<int>(rank) * (BN / 2) + 64 * q,
+                                 c.b_row0 + kb * BK);
+            } else {
+              tma_load_2d_pair(sb, &mapB0, fb, kb * BK,
+                               c.b_row0 + c.tn * BN + static_cast<int>(rank) * (BN / 2));
+            }
             continue;
           }
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
@@ -490,8 +498,8 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {  // 4 MMAs of 32 bytes of K per 128-byte row
             if constexpr (PAIR)
-              mma_bf16_ss_lh_pair(d_tmem, a_lo + 2 * k, HI, b_lo + 2 * k, HI, IDESC,
-                                  (kb | k) != 0 ? 1u : 0u);
+              mma_bf16_ss_lh_pair(d_tmem, a_lo + 2 * k, HI, b_lo + (B_MN ? k * (2048 >> 4) : 2 * k),
+                                  HI, IDESC, (kb | k) != 0 ? 1u : 0u);
             else
               mma_ss_lh<E>(d_tmem, a_lo + 2 * k, HI, b_lo + (B_MN ? k * (2048 >> 4) : 2 * k), HI,
                            IDESC, (kb | k) != 0 ? 1u : 0u);

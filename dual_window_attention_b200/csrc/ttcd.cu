@@ -238,6 +238,14 @@ ttcd_status launch_rows_gemm(const Ctx& c, const CUtensorMap& A, const CUtensorM
     return launch_gemm<E, 256, 4, false>(c, A, B, B, out_map, geo, epi, out_map2);
 }
 
+// The same with B given transposed (MN-major, bf16): pairs need no change of map.
+template <class Epi>
+ttcd_status launch_rows_gemm_bmn(const Ctx& c, const CUtensorMap& A, const CUtensorMap& B,
+                                 const CUtensorMap* out_map, const GemmGeom& geo, const Epi& epi) {
+  return launch_gemm<__nv_bfloat16, 256, 6, false, Epi, GemmGeom, true, true>(c, A, B, B, out_map,
+                                                                               geo, epi);
+}
+
 GemmGeom plain_geom(long long rows, int N_tiles, int K) {
   GemmGeom g;
   g.n_seq = 1;
@@ -2008,7 +2016,7 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
     gg.tiles_n = cdiv(m.f, 256);
     gg.b_group_rows = m.d;
     EpiStore<float> e{dzsy, m.f, m.f, nullptr};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(c, mA, mB, mB, &mo, gg, e)));
+    TTCD_TRY((launch_rows_gemm_bmn<EpiStore<float>>(c, mA, mB, &mo, gg, e)));
   }
   // G_i and dL/dstate_in: the scan walked backwards over dy_C^T Z_S,C
   {
@@ -2049,11 +2057,10 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
   {
     CUtensorMap mA, mB;
     if (!map_rows<bf>(&mA, Kp, m.P, m.f, 128) ||
-        !map_rows<bf>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, 256))
+        !map_rows<bf>(&mB, Wall, static_cast<long long>(p->B) * m.Nc * m.d, m.f, gemm_b_box<bf>()))
       return TTCD_ERR_CUDA;
     EpiStoreScaledPair e{drt, dr, m.d, m.d, kscale};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, nullptr,
-                                             padded_chunk_geom(p, m, m.f, cdiv(m.d, 256)), e)));
+    TTCD_TRY(launch_rows_gemm<bf>(c, mA, mB, nullptr, padded_chunk_geom(p, m, m.f, cdiv(m.d, 256)), e));
   }
   // E = dRt M: dD = s E and the partial dots D . E
   {
@@ -2062,8 +2069,7 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
         !make_map<bf>(&mB, M, m.f, m.d, m.f * 2, 64, 64))
       return TTCD_ERR_CUDA;
     EpiBwdE e{dD, D, epart, m.P, m.f, kscale};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiBwdE, GemmGeom, true>(
-        c, mA, mB, mB, nullptr, plain_geom(m.P, cdiv(m.f, 256), m.d), e)));
+    TTCD_TRY((launch_rows_gemm_bmn<EpiBwdE>(c, mA, mB, nullptr, plain_geom(m.P, cdiv(m.f, 256), m.d), e)));
   }
   key_backward_kernel<<<cdiv(m.P, 256), 256, 0, c.s>>>(epart, cdiv(m.f, 256), ssq,
                                                        cdiv(m.f, 128), beta, d_beta, coef, p->T,
@@ -2076,8 +2082,7 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
         !make_map<bf>(&mB, Wall, m.f, static_cast<uint64_t>(p->B) * m.Nc * m.d, m.f * 2, 64, 64))
       return TTCD_ERR_CUDA;
     EpiBwdZbS e{dzbs, Kp, dD, m.f, coef};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiBwdZbS, GemmGeom, true>(
-        c, mA, mB, mB, nullptr, padded_chunk_geom(p, m, m.d, cdiv(m.f, 256)), e)));
+    TTCD_TRY((launch_rows_gemm_bmn<EpiBwdZbS>(c, mA, mB, nullptr, padded_chunk_geom(p, m, m.d, cdiv(m.f, 256)), e)));
   }
   // dM = sum_t (s dRt)_t D_t^T;  dW_proj = W_down^T dM;  dW_down = dM W_proj^T + the read's
   TTCD_TRY(launch_tsum(c, dr, m.d, m.d, D, m.f, m.f, m.P, dM));
@@ -2149,8 +2154,7 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
           !make_out_map<float>(&mo, du[path], m.BT, m.d, m.d))
         return TTCD_ERR_CUDA;
       EpiStore<float> e{du[path], m.d, m.d, nullptr};
-      TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(
-          c, mA, mB, mB, &mo, plain_geom(m.BT, cdiv(m.d, 256), 2 * m.f), e)));
+      TTCD_TRY((launch_rows_gemm_bmn<EpiStore<float>>(c, mA, mB, &mo, plain_geom(m.BT, cdiv(m.d, 256), 2 * m.f), e)));
     }
   }
   // dW_gate = sum_rows da^T u, dW_up = sum_rows db^T u (both paths)
@@ -2401,11 +2405,11 @@ ttcd_status block_backward_bf16(const Ctx& c, const __nv_bfloat16* x, const floa
                         sc, m.dqkv, m.dqkv));
   {  // h_P = x + o_P W_o^T, fp32, both paths
     CUtensorMap mA, mB, mo;
-    if (!map_rows<bf>(&mA, o, 2 * BT, dq, 128) || !map_rows<bf>(&mB, w->w_o, m.d, dq, 256) ||
+    if (!map_rows<bf>(&mA, o, 2 * BT, dq, 128) || !map_rows<bf>(&mB, w->w_o, m.d, dq, gemm_b_box<bf>()) ||
         !make_out_map<float>(&mo, h, 2 * BT, m.d, m.d))
       return TTCD_ERR_CUDA;
     EpiResidual<float, bf> e{h, m.d, x, m.d, BT, m.d};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(2 * BT, cdiv(m.d, 256), static_cast<int>(dq)), e)));
+    TTCD_TRY(launch_rows_gemm<bf>(c, mA, mB, &mo, plain_geom(2 * BT, cdiv(m.d, 256), static_cast<int>(dq)), e));
   }
   rmsnorm_kernel<float, bf, bf><<<cdiv(2 * BT, 8), 256, 0, c.s>>>(
       h, static_cast<const bf*>(w->g_mlp), u, 2 * BT, m.d, p->rms_eps);
@@ -2432,8 +2436,7 @@ ttcd_status block_backward_bf16(const Ctx& c, const __nv_bfloat16* x, const floa
         !make_out_map<bf>(&mo, dO, 2 * BT, dq, dq))
       return TTCD_ERR_CUDA;
     EpiStore<bf> e{dO, dq, static_cast<int>(dq), nullptr};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<bf>, GemmGeom, true>(
-        c, mA, mB, mB, &mo, plain_geom(2 * BT, cdiv(dq, 256), m.d), e)));
+    TTCD_TRY((launch_rows_gemm_bmn<EpiStore<bf>>(c, mA, mB, &mo, plain_geom(2 * BT, cdiv(dq, 256), m.d), e)));
   }
   TTCD_TRY(launch_tsum(c, dh, m.d, m.d, o, dq, static_cast<int>(dq), 2 * BT, g->w_o));
 
@@ -2467,8 +2470,7 @@ ttcd_status block_backward_bf16(const Ctx& c, const __nv_bfloat16* x, const floa
         !make_out_map<float>(&mo, dxn, BT, m.d, m.d))
       return TTCD_ERR_CUDA;
     EpiStore<float> e{dxn, m.d, m.d, nullptr};
-    TTCD_TRY((launch_gemm<bf, 256, 4, false, EpiStore<float>, GemmGeom, true>(
-        c, mA, mB, mB, &mo, plain_geom(BT, cdiv(m.d, 256), m.dqkv), e)));
+    TTCD_TRY((launch_rows_gemm_bmn<EpiStore<float>>(c, mA, mB, &mo, plain_geom(BT, cdiv(m.d, 256), m.dqkv), e)));
   }
   rmsnorm_kernel<bf, bf, bf><<<cdiv(BT, 8), 256, 0, c.s>>>(
       x, static_cast<const bf*>(w->g_attn), xn, BT, m.d, p->rms_eps);
