@@ -84,6 +84,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_decode_state_read.argtypes = [P, i, vp, sz, vp, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
+    lib.ttcd_swa_block_forward.argtypes = [vp, W, P, vp, vp, sz, vp]
+    lib.ttcd_swa_block_forward_workspace_size.argtypes = [P]
+    lib.ttcd_swa_block_forward_workspace_size.restype = sz
     lib.ttcd_block_forward_profiled.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), i]
     lib.ttcd_check_device_status.argtypes = [vp, vp]
@@ -345,16 +348,43 @@ def block_forward(x, beta, weights: Dict[str, torch.Tensor], p: BlockParams, out
     return out, st_t, workspace
 
 
+def swa_block_forward_workspace_size(p: BlockParams) -> int:
+    return int(load_library().ttcd_swa_block_forward_workspace_size(ctypes.byref(p.c())))
+
+
+def swa_block_forward(x, weights: Dict[str, torch.Tensor], p: BlockParams, out=None,
+                      workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One plain sliding-window block (window p.w_T, static MLP): a layer outside
+    the TTT layer set.  Returns (out, workspace)."""
+    lib = load_library()
+    need = swa_block_forward_workspace_size(p)
+    if need == 0:
+        raise TTCDError(ERR_INVALID_ARG, "ttcd_swa_block_forward_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    out = torch.empty_like(x) if out is None else out
+    pc, wc = p.c(), _weights(weights)
+    st = lib.ttcd_swa_block_forward(_ptr(x), ctypes.byref(wc), ctypes.byref(pc), _ptr(out),
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ttcd_swa_block_forward")
+    return out, workspace
+
+
 def block_stack_forward(x, layers, p: BlockParams, workspace: Optional[torch.Tensor] = None,
-                        stream=None, on_layer=None) -> torch.Tensor:
-    """A stack of IP-TTCD blocks: layer l's output is layer l+1's input.
+                        stream=None, on_layer=None, ttt_layers=None) -> torch.Tensor:
+    """A stack of blocks: layer l's output is layer l+1's input.
 
     ``layers`` is a list of weight dicts (the keys block_forward takes plus each
-    layer's per-token ``beta``).  One workspace serves every layer and two
-    activation buffers alternate, so nothing is allocated per layer.
+    layer's per-token ``beta``).  ``ttt_layers`` (an iterable of layer indices,
+    default all) names the IP-TTCD blocks; the other layers are plain
+    sliding-window blocks (swa_block_forward: window p.w_T, static MLP; their
+    beta, w_proj and conv taps are not read).  One workspace serves every layer
+    and two activation buffers alternate, so nothing is allocated per layer.
     ``on_layer(l, out)``, if given, sees each layer's output before the buffer is
     reused.  Returns the last layer's output (a fresh tensor, not ``x``)."""
-    need = block_forward_workspace_size(p)
+    ttt = set(range(len(layers))) if ttt_layers is None else set(ttt_layers)
+    need = max(block_forward_workspace_size(p), swa_block_forward_workspace_size(p))
     if need == 0:
         raise TTCDError(ERR_INVALID_ARG, "ttcd_block_forward_workspace_size")
     if workspace is None:
@@ -363,7 +393,10 @@ def block_stack_forward(x, layers, p: BlockParams, workspace: Optional[torch.Ten
     cur = x
     for l, w in enumerate(layers):
         out = bufs[l & 1]
-        block_forward(cur, w["beta"], w, p, out=out, workspace=workspace, stream=stream)
+        if l in ttt:
+            block_forward(cur, w["beta"], w, p, out=out, workspace=workspace, stream=stream)
+        else:
+            swa_block_forward(cur, w, p, out=out, workspace=workspace, stream=stream)
         if on_layer is not None:
             on_layer(l, out)
         cur = out

@@ -340,9 +340,11 @@ __global__ void key_scale_kernel(const float* __restrict__ ssq_part, int n_part,
 
 // rstd[row] = (sum over tiles of ssq[tile][row] / d + eps)^(-1/2): the MLP
 // RMSNorm's row scale from the partial sums the o_proj epilogue wrote.
+// rows r0 .. rows-1 of the [n_part, rows] partial sums (r0 > 0: a later part only)
 __global__ void rms_rstd_kernel(const float* __restrict__ ssq, int n_part, long long rows,
-                                float inv_d, float eps, float* __restrict__ rstd) {
-  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+                                float inv_d, float eps, float* __restrict__ rstd,
+                                long long r0 = 0) {
+  const long long r = r0 + static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (r >= rows) return;
   float sum = 0.f;
   for (int i = 0; i < n_part; ++i) sum += ssq[i * rows + r];

@@ -36,6 +36,7 @@ struct GemmGeom {
   int tiles_m;          // ceil(C / 128)
   int tiles_n;          // column tiles
   int b_group_rows;     // B row offset per group (0 = shared B)
+  int row_off = 0;      // first A (and output) row of the geometry
   __host__ __device__ int total() const { return n_seq * Nc * tiles_m * tiles_n; }
   // CTA pairs: pair tile t covers row tiles 2p and 2p + 1 of one group; `rank`
   // picks this CTA's.  True while the pair's first tile has rows; the second
@@ -51,7 +52,7 @@ struct GemmGeom {
     const int len = min(C, T - i * C);
     const int m0 = (2 * pm + rank) * GEMM_BM;
     c.valid_rows = max(0, min(GEMM_BM, len - m0));
-    c.row0 = b * T + i * C + m0;
+    c.row0 = row_off + b * T + i * C + m0;
     c.tn = tn;
     c.group = g;
     c.b_row0 = g * b_group_rows;
@@ -66,7 +67,7 @@ struct GemmGeom {
     const int len = min(C, T - i * C);
     const int m0 = tm * GEMM_BM;
     c.valid_rows = min(GEMM_BM, len - m0);
-    c.row0 = b * T + i * C + m0;
+    c.row0 = row_off + b * T + i * C + m0;
     c.tn = tn;
     c.group = g;
     c.b_row0 = g * b_group_rows;
@@ -801,35 +802,48 @@ struct EpiOprojNorm {
 // When `rstd` is set, the A operand was h * g and RMSNorm is finished here as
 // the row scale rstd[row] on gate and up alike (u W^T = rstd * ((h * g) W^T));
 // otherwise A already holds u.
+//
+// OutT = bf16 writes 64 columns per step (N a multiple of 64).  Output row of
+// accumulator row `row` is row - out_row0 (the output may start at a later row
+// than A, e.g. the student half of [u_T; u_S]).
+template <class OutT = float>
 struct EpiSwiGLU {
   static constexpr bool kStaged = true;
   static constexpr bool kCollective = false;
-  float* out;
+  OutT* out;
   long long ldo;
   int N;  // d_ff
   const float* rstd;  // [rows], nullable
+  long long out_row0 = 0;
   __device__ float pre(const TileCtx& c, int r) const {
     return (rstd && r < c.valid_rows) ? __ldg(rstd + c.row0 + r) : 1.f;
   }
+  __device__ static void swiglu32(uint32_t taddr, int cc, int half, float rs, float (&z)[32]) {
+    float u[32];
+    tmem_ld32f(taddr + cc, z);
+    tmem_ld32f(taddr + half + cc, u);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float gg = z[i] * rs;
+      z[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (u[i] * rs);
+    }
+  }
   template <int BN>
   __device__ void run(const TileCtx& c, uint32_t taddr, int r, EpiStage& stg, float rs) const {
+    constexpr int STEP = sizeof(OutT) == 2 ? 64 : 32;
     const bool ok = r < c.valid_rows;
-    const long long row = c.row0 + r;
+    const long long row = c.row0 + r - out_row0;
     const int wrow = r & ~31;
     const bool staged = stg.on() && wrow + 32 <= c.valid_rows;
+    const int y = static_cast<int>(c.row0 - out_row0) + wrow;
 #pragma unroll 1
-    for (int cc = 0; cc < BN / 2; cc += 32) {
+    for (int cc = 0; cc < BN / 2; cc += STEP) {
       const int col = c.tn * (BN / 2) + cc;
       if (col >= N) break;
-      float g[32], u[32];
-      tmem_ld32f(taddr + cc, g);
-      tmem_ld32f(taddr + BN / 2 + cc, u);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float gg = g[i] * rs;
-        g[i] = __fdividef(gg, 1.0f + __expf(-gg)) * (u[i] * rs);
-      }
-      emit(stg, staged, ok, out + row * ldo, col, c.row0 + wrow, g, u);
+      float lo[32], hi[32];
+      swiglu32(taddr, cc, BN / 2, rs, lo);
+      if constexpr (STEP == 64) swiglu32(taddr, cc + 32, BN / 2, rs, hi);
+      emit(stg, staged, ok, out + row * ldo, col, y, lo, hi);
     }
   }
 };

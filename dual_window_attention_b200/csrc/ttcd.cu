@@ -574,7 +574,7 @@ ttcd_status mlp_front(const Ctx& c, const ttcd_block_params* p, const Layout& L,
         return TTCD_ERR_CUDA;
       CUtensorMap mo;
       if (!make_out_map<float>(&mo, Z, 2 * m.BT, m.f, m.f)) return TTCD_ERR_CUDA;
-      EpiSwiGLU e{Z, m.f, m.f, rstd};
+      EpiSwiGLU<float> e{Z, m.f, m.f, rstd};
       TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * m.BT, cdiv(m.f, 128), m.d), e)));
     }
     stage_mark(c, mark + 1);
@@ -1033,10 +1033,104 @@ ttcd_status block_entry(const void* x, const float* beta, const ttcd_block_weigh
   return run_block<__nv_bfloat16>(c, x, beta, w, p, state_in, state_out, out, workspace, L);
 }
 
+// A plain sliding-window block (a layer outside ttt_layers): QKV with RoPE,
+// one attention window w_T (the fused kernel with w_S = w_T writes the same
+// output twice: o_T into the teacher half of o, o_S into the student half),
+// o_proj + residual + RMS statistics over the student half only, SwiGLU with
+// the static weights over the same rows, and out = h + W_down Z.
+template <class E>
+ttcd_status run_swa_block(const Ctx& c, const void* x, const ttcd_block_weights* w,
+                          const ttcd_block_params* p, void* out, void* ws, const Layout& L) {
+  const Dims m = dims_of(p);
+  const E* xin = static_cast<const E*>(x);
+  __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, L, B_QKV);
+  TTCD_TRY(block_qkv<E>(c, xin, w, p, ws, L, qkv, 0, 0));
+  E* o = at<E>(ws, L, B_O);
+  float* h = at<float>(ws, L, B_H);
+  E* u = at<E>(ws, L, B_U);
+  float* hssq = at<float>(ws, L, B_HSSQ);
+  float* rstd = at<float>(ws, L, B_RSTD);
+  const float sc = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(m.hd));
+  TTCD_TRY(run_attn<E>(c, qkv, qkv + static_cast<long long>(m.Hq) * m.hd,
+                       qkv + static_cast<long long>(m.Hq + m.Hkv) * m.hd, o,
+                       o + m.BT * m.Hq * m.hd, nullptr, nullptr, p->B, p->T, m.Hq, m.Hkv, m.hd,
+                       p->w_T, p->w_T, sc, m.dqkv, m.dqkv, 0));
+  stage_mark(c, 3);
+  {  // h = x + o W_o^T over the student rows [BT, 2BT) of o
+    CUtensorMap mA, mB, mo, mo2;
+    if (!map_rows<E>(&mA, o, 2 * m.BT, static_cast<long long>(m.Hq) * m.hd, 128) ||
+        !map_rows<E>(&mB, w->w_o, m.d, static_cast<long long>(m.Hq) * m.hd, gemm_b_box<E>()) ||
+        !make_out_map<E>(&mo, u, 2 * m.BT, m.d, m.d) ||
+        !make_out_map<float>(&mo2, h, m.BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    GemmGeom g = plain_geom(m.BT, cdiv(m.d, 256), m.Hq * m.hd);
+    g.row_off = static_cast<int>(m.BT);
+    EpiOprojNorm<E, E> e{u, h, hssq, xin, static_cast<const E*>(w->g_mlp), m.BT, m.d};
+    TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, g, e, &mo2));
+  }
+  rms_rstd_kernel<<<cdiv(m.BT, 256), 256, 0, c.s>>>(hssq, cdiv(m.d, 256), 2 * m.BT, 1.0f / m.d,
+                                                    p->rms_eps, rstd, m.BT);
+  TTCD_CHECK_LAUNCH();
+  stage_mark(c, 4);
+  // Z = silu(u W_gate^T) * (u W_up^T) over the same rows: bf16 Z_S, or fp32 into
+  // the student half of Z
+  E* zs = sizeof(E) == 2 ? at<E>(ws, L, B_ZS16) : reinterpret_cast<E*>(at<float>(ws, L, B_Z) + m.BT * m.f);
+  {
+    CUtensorMap mA, mB0, mB1, mo;
+    if (!map_rows<E>(&mA, u, 2 * m.BT, m.d, 128) ||
+        !map_rows<E>(&mB0, w->w_gate, m.f, m.d, 128) || !map_rows<E>(&mB1, w->w_up, m.f, m.d, 128) ||
+        !make_out_map<E>(&mo, zs, m.BT, m.f, m.f))
+      return TTCD_ERR_CUDA;
+    GemmGeom g = plain_geom(m.BT, cdiv(m.f, 128), m.d);
+    g.row_off = static_cast<int>(m.BT);
+    EpiSwiGLU<E> e{zs, m.f, m.f, rstd, m.BT};
+    TTCD_TRY((launch_gemm<E, 256, 4, true>(c, mA, mB0, mB1, &mo, g, e)));
+  }
+  stage_mark(c, 5);
+  {  // out = h + W_down Z
+    CUtensorMap mA, mB, mo;
+    if (!map_rows<E>(&mA, zs, m.BT, m.f, 128) ||
+        !map_rows<E>(&mB, w->w_down, m.d, m.f, gemm_b_box<E>()) ||
+        !make_out_map<E>(&mo, out, m.BT, m.d, m.d))
+      return TTCD_ERR_CUDA;
+    EpiResidual<E, float> e{static_cast<E*>(out), m.d, h, m.d, m.BT, m.d};
+    TTCD_TRY(launch_rows_gemm<E>(c, mA, mB, &mo, plain_geom(m.BT, cdiv(m.d, 256), m.f), e));
+  }
+  stage_mark(c, 6);
+  return TTCD_OK;
+}
+
+ttcd_status swa_block_entry(const void* x, const ttcd_block_weights* w,
+                            const ttcd_block_params* p, void* out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  TTCD_TRY(check_params(p));
+  if (!aligned16(x) || !aligned16(out) || !aligned16(workspace) || !w || !aligned16(w->w_qkv) ||
+      !aligned16(w->w_o) || !aligned16(w->g_attn) || !aligned16(w->g_mlp) ||
+      !aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down))
+    return TTCD_ERR_INVALID_ARG;
+  const Layout L = make_layout(p, true, false, false);
+  if (ws_bytes < L.total) return TTCD_ERR_WORKSPACE;
+  Ctx c;
+  TTCD_TRY(make_ctx(stream, c, at<void>(workspace, L, B_STATUS)));
+  if (p->dtype == TTCD_F32) return run_swa_block<float>(c, x, w, p, out, workspace, L);
+  return run_swa_block<__nv_bfloat16>(c, x, w, p, out, workspace, L);
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
 extern "C" {
+
+size_t ttcd_swa_block_forward_workspace_size(const ttcd_block_params* p) {
+  if (check_params(p) != TTCD_OK) return 0;
+  return make_layout(p, true, false, false).total;
+}
+
+ttcd_status ttcd_swa_block_forward(const void* x, const ttcd_block_weights* w,
+                                   const ttcd_block_params* p, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  return swa_block_entry(x, w, p, out, workspace, ws_bytes, stream);
+}
 
 const char* ttcd_status_string(ttcd_status s) {
   switch (s) {
@@ -1305,7 +1399,7 @@ ttcd_status ttcd_shard_mix(const float* beta, const void* u_halo, const ttcd_blo
         !map_rows<bf>(&mB1, w->w_up, m.f, m.d, 128) ||
         !make_out_map<float>(&mo, zh, rows, m.f, m.f))
       return TTCD_ERR_CUDA;
-    EpiSwiGLU e{zh, m.f, m.f, nullptr};
+    EpiSwiGLU<float> e{zh, m.f, m.f, nullptr};
     TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(rows, cdiv(m.f, 128), m.d), e)));
   }
   TTCD_TRY(mlp_front<bf>(c, p, L, workspace, static_cast<const bf*>(w->w_gate),
@@ -1672,7 +1766,7 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
         !map_rows<bf>(&mB0, w->w_gate, f, d, 128) || !map_rows<bf>(&mB1, w->w_up, f, d, 128) ||
         !make_out_map<float>(&mo, dat<float>(ws, L.Z), 2 * B, f, f))
       return TTCD_ERR_CUDA;
-    EpiSwiGLU e{dat<float>(ws, L.Z), f, f, nullptr};
+    EpiSwiGLU<float> e{dat<float>(ws, L.Z), f, f, nullptr};
     TTCD_TRY((launch_gemm<bf, 256, 4, true>(c, mA, mB0, mB1, &mo, plain_geom(2 * B, cdiv(f, 128), d), e)));
   }
   // convs, residual, key (into the chunk buffer), key scale

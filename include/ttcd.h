@@ -290,6 +290,27 @@ ttcd_status ttcd_block_forward(const void* x, const float* beta, const ttcd_bloc
                                const ttcd_block_params* p, float* state_out, void* out,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * ttcd_swa_block_forward — one plain sliding-window transformer block: a layer
+ * of an IP-TTCD model that is not in its TTT layer set (GitHub README "TTCD",
+ * "Model configuration": ttt_layers picks the layers that learn at test time;
+ * window_size is the attention window of every layer, the teacher window).
+ * It has no student path and no fast weights:
+ *   xn = RMSNorm(x; g_attn);  q,k,v = xn W_qkv^T;  q,k = RoPE(q,k)
+ *   h = x + SWA_{w_T}(q, k, v) W_o^T     (keys [t - w_T + 1, t], GQA)
+ *   out = h + W_down (silu(u W_gate^T) * (u W_up^T)),  u = RMSNorm(h; g_mlp)
+ * Arguments and layouts as ttcd_block_forward; params.w_S, chunk, conv_k,
+ * l2_eps and the weights w_proj, conv_T, conv_S are not read (they may be
+ * null).  workspace >= ttcd_swa_block_forward_workspace_size(p) bytes, 16-byte
+ * aligned, status word first.  Precision: bf16 operands (TTCD_BF16, at every
+ * T) or fp32 with tf32 MMAs (TTCD_F32); q, k, v and the attention are bf16;
+ * fp32 accumulation and residual.  Errors as ttcd_block_forward.
+ */
+ttcd_status ttcd_swa_block_forward(const void* x, const ttcd_block_weights* w,
+                                   const ttcd_block_params* p, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream);
+size_t ttcd_swa_block_forward_workspace_size(const ttcd_block_params* p);
+
 /* fp32 gradients of the block's weights (device, written, not accumulated);
  * fields in the order and shapes of ttcd_block_weights. */
 typedef struct {

@@ -11,5 +11,5 @@ from .ttcd_oracle import *  # noqa: F401,F403
 from .ttcd_oracle import (block_forward, causal_depthwise_conv, chunk_increments,
                           distillation_loss, dual_window_attention, exclusive_prefix,
                           fastweight_mlp, l2_normalize_rows, qkv_projection, rms_norm,
-                          rope, silu, swiglu, value_residual, window_mask,
+                          rope, silu, swa_block_forward, swiglu, value_residual, window_mask,
                           windowed_attention, windowed_attention_bruteforce)

@@ -43,6 +43,9 @@ Readings where the pages are silent or garbled (each repeated where used):
   R11 GQA: query head h reads KV head h // (Hq / Hkv).
   R12 W_proj is applied first: r_t = W_down (W_proj d_t), as written.
   R13 a partial last chunk is allowed; its Delta W counts only in the final state.
+  R18 a layer outside the TTT layer set ([README] "Model configuration",
+     ttt_layers) is the same skeleton with one sliding window of w_T keys
+     (window_size) and the static MLP: no student path, no fast weights.
 
 Parity pins (tests/test_oracle_*.py) tie each function to something other than
 itself: brute-force loops, textbook/library special cases, closed forms and
@@ -403,6 +406,32 @@ def block_forward(x, beta, weights: Dict[str, np.ndarray], *, n_q_heads: int,
            "h_T": h_T, "h_S": h_S, "u_T": u_T, "u_S": u_S}
     res.update(mlp)
     return res
+
+
+def swa_block_forward(x, weights: Dict[str, np.ndarray], *, n_q_heads: int, n_kv_heads: int,
+                      head_dim: int, window: int, rms_eps: float = 1e-6,
+                      rope_theta: float = 1e4,
+                      softmax_scale: Optional[float] = None) -> Dict[str, np.ndarray]:
+    """Forward pass of a plain sliding-window block: a layer outside the TTT
+    layer set ([README] "Model configuration": ttt_layers, window_size; reading
+    R18; skeleton R10, R11).
+
+      h = x + SWA_window(RoPE(q), RoPE(k), v) W_o^T,  q,k,v = RMSNorm(x) W_qkv^T
+      out = h + W_down SwiGLU(RMSNorm(h))
+    """
+    x = np.asarray(x, np.float64)
+    Hq, Hkv, hd = n_q_heads, n_kv_heads, head_dim
+    sm_scale = softmax_scale if softmax_scale else 1.0 / np.sqrt(float(hd))
+    xn = rms_norm(x, weights["g_attn"], rms_eps)
+    q, k, v = qkv_projection(xn, weights["w_qkv"], Hq, Hkv, hd)
+    q, k = rope(q, rope_theta), rope(k, rope_theta)
+    o, lse = windowed_attention(q, k, v, window, sm_scale)
+    B, T = x.shape[:2]
+    h = x + o.reshape(B, T, Hq * hd) @ np.asarray(weights["w_o"], np.float64).T
+    u = rms_norm(h, weights["g_mlp"], rms_eps)
+    z = swiglu(u, weights["w_gate"], weights["w_up"])
+    out = h + z @ np.asarray(weights["w_down"], np.float64).T
+    return {"q": q, "k": k, "v": v, "o": o, "lse": lse, "h": h, "u": u, "z": z, "out": out}
 
 
 # ---------------------------------------------------------------------------

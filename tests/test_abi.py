@@ -240,3 +240,21 @@ def test_attention_timeline_is_compiled_out_of_the_library(lib):
     instrumented build; the library reports it as unsupported, touching no GPU."""
     buf = (ctypes.c_longlong * 2048)()
     assert lib.ttcd_attn_timeline_read(buf, 2048) == ttcd.ERR_UNSUPPORTED
+
+
+def test_plain_block_rejects_bad_arguments_on_host(lib):
+    """ttcd_swa_block_forward validates on the host; it needs none of the fast-weight
+    pointers (w_proj, conv_T, conv_S may be null)."""
+    fake = 1 << 20
+    p = _params().c()
+    w_plain = ttcd._Weights(*([fake] * 7 + [0, 0, 0]))  # w_proj, conv_T, conv_S null
+    need = lib.ttcd_swa_block_forward_workspace_size(ctypes.byref(p))
+    assert need > 0
+    sb = lib.ttcd_swa_block_forward
+    assert sb(None, ctypes.byref(w_plain), ctypes.byref(p), fake, fake, need, None) == ttcd.ERR_INVALID_ARG
+    assert sb(fake, ctypes.byref(w_plain), ctypes.byref(p), fake, fake, need - 1, None) == ttcd.ERR_WORKSPACE
+    w_no_down = ttcd._Weights(*([fake] * 6 + [0, 0, 0, 0]))
+    assert sb(fake, ctypes.byref(w_no_down), ctypes.byref(p), fake, fake, need, None) == ttcd.ERR_INVALID_ARG
+    bad = _params(head_dim=48).c()
+    assert lib.ttcd_swa_block_forward_workspace_size(ctypes.byref(bad)) == 0
+    assert sb(fake, ctypes.byref(w_plain), ctypes.byref(bad), fake, fake, need, None) == ttcd.ERR_UNSUPPORTED

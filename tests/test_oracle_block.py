@@ -94,6 +94,39 @@ def test_student_path_is_block_output_with_static_mlp_when_beta_zero():
     np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-11)
 
 
+def _swa(shape, inp, window, layer=0):
+    w = {k: _np(v) for k, v in inp["layers"][layer].items()}
+    return orc.swa_block_forward(_np(inp["x"]), w, n_q_heads=shape.n_q_heads,
+                                 n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim,
+                                 window=window, rms_eps=shape.rms_eps,
+                                 rope_theta=shape.rope_theta)
+
+
+@pytest.mark.parametrize("window", [1, 16, 64, 300])
+def test_plain_swa_block_matches_torch_built_block(window):
+    """The oracle's plain sliding-window block (a layer outside the TTT layer
+    set) against the block written with torch float64 library routines, with
+    distinct norm gains."""
+    shape = TINY_F32
+    inp = make_block_inputs(shape, seed=4)
+    rng = np.random.default_rng(5)
+    inp["layers"][0]["g_attn"] = torch.from_numpy(0.5 + rng.random(shape.d_model))
+    inp["layers"][0]["g_mlp"] = torch.from_numpy(0.5 + rng.random(shape.d_model))
+    w = {k: _np(v) for k, v in inp["layers"][0].items()}
+    res = _swa(shape, inp, window)
+    ref = _plain_swa_block(_np(inp["x"]), w, shape, window)
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-11)
+
+
+def test_plain_swa_block_is_the_ttcd_block_with_one_window_and_no_update():
+    """With w_S = w_T and beta = 0 the IP-TTCD block's student output is the plain
+    block of window w_T, whatever the conv taps and W_proj."""
+    shape = TINY_F32.with_(w_S=64, w_T=64)
+    inp = make_block_inputs(shape, seed=6)
+    res = _block(shape, inp, beta=np.zeros((1, shape.T)))
+    np.testing.assert_allclose(_swa(shape, inp, 64)["out"], res["out"], rtol=1e-10, atol=1e-11)
+
+
 def test_block_attention_matches_bruteforce_on_tiny_workload():
     shape = TINY_F32
     inp = make_block_inputs(shape, seed=0)

@@ -34,6 +34,13 @@ MUTANTS = [
      "ms = np.mean(np.abs(x), axis=-1, keepdims=True)"),
     ("rmsnorm_eps_outside_sqrt", "return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)",
      "return x / (np.sqrt(ms) + eps) * np.asarray(g, dtype=np.float64)"),
+    # plain sliding-window block (a layer outside the TTT layer set)
+    ("swa_block_no_mlp_residual", "out = h + z @ np.asarray(weights[\"w_down\"], np.float64).T",
+     "out = z @ np.asarray(weights[\"w_down\"], np.float64).T"),
+    ("swa_block_rope_on_q_only", "q, k = rope(q, rope_theta), rope(k, rope_theta)",
+     "q = rope(q, rope_theta)"),
+    ("swa_block_mlp_norm_uses_attn_gain", 'u = rms_norm(h, weights["g_mlp"], rms_eps)',
+     'u = rms_norm(h, weights["g_attn"], rms_eps)'),
     ("mlp_norm_uses_attn_gain",
      'u_T = rms_norm(h_T, weights["g_mlp"], rms_eps)\n    u_S = rms_norm(h_S, weights["g_mlp"], rms_eps)',
      'u_T = rms_norm(h_T, weights["g_attn"], rms_eps)\n    u_S = rms_norm(h_S, weights["g_attn"], rms_eps)'),
