@@ -461,6 +461,9 @@ def run_ours(args, world, rank, local):
         line["stack"] = [measure_stack(args, world, local, B, T, steps=max(2, args.extra_steps // 2),
                                        warmup=args.extra_warmup)
                          for B, T in ((1, 65536), (4, 16384))]
+        # the plain sliding-window block of layers outside the TTT layer set
+        line["swa_block"] = measure_swa_block(args, world, local, steps=args.extra_steps,
+                                              warmup=args.extra_warmup)
         # the backward kernels at the same block shape (B 1, T 65536)
         line["backward"] = measure_backward(args, local, 1, shape.T, steps=3, warmup=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -757,6 +760,49 @@ def measure_stack(args, world, local, B, T, steps, warmup):
             "ms_per_pass": ms, "tokens_per_s": shape.B * shape.T * world / (ms / 1e3),
             "tflops_per_s": flops / (ms / 1e3) / 1e12, "steps": steps, "warmup": warmup,
             "gpu_launches": launches, "clocks": clk.summary()}
+
+
+def measure_swa_block(args, world, local, steps, warmup):
+    """The plain sliding-window block of the layers outside the TTT layer set
+    (ttcd_swa_block_forward: one w_T = 8192 window, static MLP) at the Qwen3
+    block shape, B 1, T 65536."""
+    import dual_window_attention_b200 as ttcd
+    ttcd.load_library()
+    shape = QWEN3_0P6B_64K
+    dev = torch.device("cuda", local)
+    inp = make_block_inputs(shape, seed=0)
+    x = inp["x"].to(dev)
+    w = {k: v.to(dev) for k, v in inp["layers"][0].items()
+         if k not in ("beta", "w_proj", "conv_T", "conv_S")}
+    del inp
+    p = ttcd.BlockParams.from_shape(shape)
+    ws = ttcd.alloc_workspace(ttcd.swa_block_forward_workspace_size(p), dev)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        ttcd.swa_block_forward(x, w, p, out=out, workspace=ws, stream=stream)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        ttcd.swa_block_forward(x, w, p, out=out, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
+    if ttcd.check_device_status(ws, stream) != ttcd.OK:
+        raise RuntimeError("a device wait timed out in the plain-block benchmark")
+    BT, d, f = shape.B * shape.T, shape.d_model, shape.d_ff
+    hq, hkv, hd = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+    attn = 4.0 * hd * hq * sum(min(t + 1, shape.w_T) for t in range(shape.T)) * shape.B
+    gemm = 2.0 * BT * d * (hq + 2 * hkv) * hd + 2.0 * BT * hq * hd * d + 2.0 * BT * d * 2 * f \
+        + 2.0 * BT * f * d
+    del x, w, ws, out
+    torch.cuda.empty_cache()
+    return {"workload": "qwen3_0.6b_plain_swa_block_T65536", "window": shape.w_T, "ms": ms,
+            "tokens_per_s": BT * world / (ms / 1e3),
+            "tflops_per_s": (attn + gemm) / (ms / 1e3) / 1e12, "steps": steps, "warmup": warmup}
 
 
 def run_stack(args, world, rank, local):
