@@ -38,9 +38,13 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPS)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, attn_timeline: bool = False) -> str:
-    out = TIMELINE_LIB if attn_timeline else LIB
-    if not force and not attn_timeline and not needs_build():
+def build(force: bool = False, ptxas_verbose: bool = False, attn_timeline: bool = False,
+          out: str = None) -> str:
+    """Builds the library (or, attn_timeline, the instrumented one) at `out`
+    (default: in the package) and returns its path."""
+    if out is None:
+        out = TIMELINE_LIB if attn_timeline else LIB
+    if not force and not attn_timeline and out == LIB and not needs_build():
         return LIB
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2", "-shared",

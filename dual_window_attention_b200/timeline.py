@@ -56,14 +56,16 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--T", type=int, default=16384)
     ap.add_argument("--windows", default="512/8192", help="w_S/w_T")
+    ap.add_argument("--lib", default=None, help="the instrumented library (default: the package's)")
     args = ap.parse_args(argv)
     import dual_window_attention_b200 as m
     from dual_window_attention_b200 import build
 
-    if not os.path.exists(build.TIMELINE_LIB):
-        raise SystemExit("libttcd_timeline.so is missing: run "
+    lib = args.lib or build.TIMELINE_LIB
+    if not os.path.exists(lib):
+        raise SystemExit(f"{lib} is missing: run "
                          "`python -m dual_window_attention_b200.build --attn-timeline`")
-    m.load_library(build.TIMELINE_LIB)
+    m.load_library(lib)
     w_S, w_T = (int(x) for x in args.windows.split("/"))
     g = torch.Generator(device="cuda").manual_seed(0)
     q = torch.randn(1, args.T, 16, 128, device="cuda", generator=g).to(torch.bfloat16)

@@ -17,19 +17,18 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _timeline_lib():
+@pytest.fixture(scope="module")
+def timeline_lib(tmp_path_factory):
+    """A fresh instrumented build of the current sources (never a stale copy)."""
     from dual_window_attention_b200 import build
-    if not os.path.exists(build.TIMELINE_LIB):
-        build.build(attn_timeline=True)
-    return build.TIMELINE_LIB
+    return build.build(attn_timeline=True,
+                       out=str(tmp_path_factory.mktemp("timeline") / "libttcd_timeline.so"))
 
 
-def test_timeline_marks_are_ordered():
-    _timeline_lib()
+def test_timeline_marks_are_ordered(timeline_lib):
     code = r"""
-import torch, dual_window_attention_b200 as m
-from dual_window_attention_b200 import build
-m.load_library(build.TIMELINE_LIB)
+import sys, torch, dual_window_attention_b200 as m
+m.load_library(sys.argv[1])
 T = 4096
 g = torch.Generator(device="cuda").manual_seed(0)
 q = torch.randn(1, T, 16, 128, device="cuda", generator=g).to(torch.bfloat16)
@@ -51,14 +50,14 @@ for h in range(2):
 assert m.attn_timeline_read().abs().sum() == 0  # cleared by the read
 print("ok")
 """
-    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
+    r = subprocess.run([sys.executable, "-c", code, timeline_lib], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
 
 
-def test_timeline_tool_prints_the_phases():
-    _timeline_lib()
-    r = subprocess.run([sys.executable, "-m", "dual_window_attention_b200.timeline", "--T", "8192"],
-                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+def test_timeline_tool_prints_the_phases(timeline_lib):
+    r = subprocess.run([sys.executable, "-m", "dual_window_attention_b200.timeline", "--T", "8192",
+                        "--lib", timeline_lib], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "visit period" in r.stdout and "head 1" in r.stdout, r.stdout
