@@ -297,89 +297,113 @@ __global__ void __launch_bounds__(256) conv_backward_kernel(
   }
 }
 
-constexpr int TAP_SPLITS = 128;  // token splits of the tap gradient (partials per split)
+constexpr int TAP_SPLITS = 128;  // most token splits of the tap gradient (partials per split)
+constexpr int TAP_THREADS = 128;
+
+__device__ __forceinline__ void bf16x4_to_f32(uint2 u, float (&v)[4]) {
+  v[0] = bf16lo_to_f32(u.x);
+  v[1] = bf16hi_to_f32(u.x);
+  v[2] = bf16lo_to_f32(u.y);
+  v[3] = bf16hi_to_f32(u.y);
+}
 
 // part[split][path][c][m] = sum over the split's tokens (b, t), t >= m, of
-// dZbar_path[b, t, c] Z_path[b, t - m, c].  Thread = (path, 8 columns, split):
+// dZbar_path[b, t, c] Z_path[b, t - m, c].  Thread = (path, 4 columns, split):
 // it walks its contiguous tokens keeping the last k rows of Z in registers
-// (one 16-byte load of Z and two of dZbar per token).  Z [2, B, T, f] bf16,
+// (packed bf16) and a ring of the next TAP_AHEAD tokens' Z (8 bytes) and dZbar
+// (16 bytes) in flight while it accumulates the current one.  The host picks
+// nsplit <= TAP_SPLITS so that the grid fits one wave.  Z [2, B, T, f] bf16,
 // dZbar chunk-padded fp32.
+constexpr int TAP_AHEAD = 4;
 template <int KMAX>
-__global__ void __launch_bounds__(256) conv_tap_grad_kernel(
+__global__ void __launch_bounds__(TAP_THREADS, KMAX <= 4 ? 6 : 4) conv_tap_grad_kernel(
     const float* __restrict__ dzb_T, const float* __restrict__ dzb_S,
     const __nv_bfloat16* __restrict__ z, float* __restrict__ part, int B, int T, int f, int k,
-    int C, int Cp, int Nc) {
-  const int f8 = f / 8;
+    int C, int Cp, int Nc, int nsplit) {
+  const int f4 = f / 4;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= 2 * f8 * TAP_SPLITS) return;
-  const int c8 = idx % f8;
-  const int split = (idx / f8) % TAP_SPLITS;
-  const int path = idx / (f8 * TAP_SPLITS);
+  if (idx >= 2 * f4 * nsplit) return;
+  const int c4 = idx % f4;
+  const int split = (idx / f4) % nsplit;
+  const int path = idx / (f4 * nsplit);
   const long long BT = static_cast<long long>(B) * T;
-  const long long per = (BT + TAP_SPLITS - 1) / TAP_SPLITS;
+  const long long per = (BT + nsplit - 1) / nsplit;
   const long long r0 = split * per, r1 = min(BT, r0 + per);
-  const float* dzb = path ? dzb_S : dzb_T;
-  const __nv_bfloat16* zp = z + path * BT * f + c8 * 8;
-  float acc[KMAX][8];
+  const float* dzb = (path ? dzb_S : dzb_T) + c4 * 4;
+  const __nv_bfloat16* zp = z + path * BT * f + c4 * 4;
+  float acc[KMAX][4];
 #pragma unroll
   for (int m = 0; m < KMAX; ++m)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
-  float zw[KMAX][8];  // zw[m] = Z row t - m
+    for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
+  uint2 zw[KMAX];  // zw[m] = Z row t - m, 4 bf16
 #pragma unroll
-  for (int m = 0; m < KMAX; ++m)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) zw[m][i] = 0.f;
+  for (int m = 0; m < KMAX; ++m) zw[m] = make_uint2(0u, 0u);
   if (r0 < r1) {
-    int b = static_cast<int>(r0 / T), t = static_cast<int>(r0 % T);
+    int t = static_cast<int>(r0 % T);  // position of the token being summed
     // the k - 1 rows before the split's first token (same sequence only)
 #pragma unroll
     for (int m = 1; m < KMAX; ++m)
-      if (m < k && t - m >= 0) ld8f(zp + (r0 - m) * f, zw[m]);
-    int ci = t / C, cj = t % C;
-    for (long long bt = r0; bt < r1; ++bt) {
-      if (t == T) {  // next sequence: the window restarts from zeros
-        t = 0;
-        ++b;
-        ci = 0;
-        cj = 0;
+      if (m < k && t - m >= 0) zw[m] = __ldg(reinterpret_cast<const uint2*>(zp + (r0 - m) * f));
+    // load cursor: the next token to fetch, as (sequence, chunk, row in chunk)
+    long long lr = r0;
+    int lb = static_cast<int>(r0 / T), lci = t / C, lcj = t % C, lt = t;
+    uint2 zr[TAP_AHEAD];
+    float4 gr[TAP_AHEAD];
+    auto fetch = [&](uint2& zd, float4& gd) {
+      zd = __ldg(reinterpret_cast<const uint2*>(zp + lr * f));
+      gd = __ldg(reinterpret_cast<const float4*>(
+          dzb + ((static_cast<long long>(lb) * Nc + lci) * Cp + lcj) * f));
+      ++lr;
+      ++lt;
+      if (++lcj == C) { lcj = 0; ++lci; }
+      if (lt == T) { lt = 0; ++lb; lci = 0; lcj = 0; }
+    };
 #pragma unroll
-        for (int m = 1; m < KMAX; ++m)
+    for (int j = 0; j < TAP_AHEAD; ++j)
+      if (lr < r1) fetch(zr[j], gr[j]);
+    for (long long bt = r0; bt < r1; bt += TAP_AHEAD) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) zw[m][i] = 0.f;
+      for (int j = 0; j < TAP_AHEAD; ++j) {
+        if (bt + j < r1) {
+          if (t == 0) {  // a sequence starts: the window restarts from zeros
+#pragma unroll
+            for (int m = 1; m < KMAX; ++m) zw[m] = make_uint2(0u, 0u);
+          }
+          zw[0] = zr[j];
+          const float g[4] = {gr[j].x, gr[j].y, gr[j].z, gr[j].w};
+          if (lr < r1) fetch(zr[j], gr[j]);  // refill the slot TAP_AHEAD tokens ahead
+#pragma unroll
+          for (int m = 0; m < KMAX; ++m) {
+            float zf[4];
+            bf16x4_to_f32(zw[m], zf);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[m][i] = fmaf(g[i], zf[i], acc[m][i]);
+          }
+          // shift the window: row t becomes t - 1 for the next token
+#pragma unroll
+          for (int m = KMAX - 1; m > 0; --m) zw[m] = zw[m - 1];
+          if (++t == T) t = 0;
+        }
       }
-      ld8f(zp + bt * f, zw[0]);
-      float g[8];
-      ld8f(dzb + ((static_cast<long long>(b) * Nc + ci) * Cp + cj) * f + c8 * 8, g);
-#pragma unroll
-      for (int m = 0; m < KMAX; ++m)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(g[i], zw[m][i], acc[m][i]);
-      // shift the window: row t becomes t - 1 for the next token
-#pragma unroll
-      for (int m = KMAX - 1; m > 0; --m)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) zw[m][i] = zw[m - 1][i];
-      ++t;
-      if (++cj == C) { cj = 0; ++ci; }
     }
   }
-  float* dst = part + ((static_cast<long long>(split) * 2 + path) * f + c8 * 8) * k;
+  float* dst = part + ((static_cast<long long>(split) * 2 + path) * f + c4 * 4) * k;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int m = 0; m < KMAX; ++m)
       if (m < k) dst[i * k + m] = acc[m][i];
 }
 
-// out[path][c][m] = sum over splits of part[split][path][c][m].
+// out[path][c][m] = sum over the nsplit splits of part[split][path][c][m].
 __global__ void conv_tap_reduce_kernel(const float* __restrict__ part, float* __restrict__ out_T,
-                                       float* __restrict__ out_S, int f, int k) {
+                                       float* __restrict__ out_S, int f, int k, int nsplit) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= 2 * f * k) return;
   const int path = idx / (f * k), e = idx % (f * k);
   float s = 0.f;
-  for (int q = 0; q < TAP_SPLITS; ++q) s += part[(static_cast<long long>(q) * 2 + path) * f * k + e];
+  for (int q = 0; q < nsplit; ++q) s += part[(static_cast<long long>(q) * 2 + path) * f * k + e];
   (path ? out_S : out_T)[e] = s;
 }
 

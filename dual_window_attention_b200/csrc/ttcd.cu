@@ -2220,16 +2220,21 @@ ttcd_status mlp_backward_bf16(const Ctx& c, const __nv_bfloat16* u_T, const __nv
   }
   // tap gradients
   {
-    const int nt = 2 * (m.f / 8) * TAP_SPLITS;
-    if (p->conv_k <= 4)
-      conv_tap_grad_kernel<4><<<cdiv(nt, 256), 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T,
-                                                             m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
-    else
-      conv_tap_grad_kernel<8><<<cdiv(nt, 256), 256, 0, c.s>>>(dD, dzbs, zall, tpart, p->B, p->T,
-                                                             m.f, p->conv_k, p->chunk, m.Cp, m.Nc);
+    // one wave: as many token splits as resident threads allow, at most TAP_SPLITS
+    auto tap_kernel = p->conv_k <= 4 ? conv_tap_grad_kernel<4> : conv_tap_grad_kernel<8>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tap_kernel, TAP_THREADS, 0) !=
+        cudaSuccess)
+      return TTCD_ERR_CUDA;
+    const long long resident = static_cast<long long>(std::max(per_sm, 1)) * c.sms * TAP_THREADS;
+    const int nsplit = static_cast<int>(
+        std::min<long long>(TAP_SPLITS, std::max<long long>(1, resident / (2 * (m.f / 4)))));
+    const int nt = 2 * (m.f / 4) * nsplit;
+    tap_kernel<<<cdiv(nt, TAP_THREADS), TAP_THREADS, 0, c.s>>>(
+        dD, dzbs, zall, tpart, p->B, p->T, m.f, p->conv_k, p->chunk, m.Cp, m.Nc, nsplit);
     TTCD_CHECK_LAUNCH();
     conv_tap_reduce_kernel<<<cdiv(2 * m.f * p->conv_k, 256), 256, 0, c.s>>>(
-        tpart, g->conv_T, g->conv_S, m.f, p->conv_k);
+        tpart, g->conv_T, g->conv_S, m.f, p->conv_k, nsplit);
     TTCD_CHECK_LAUNCH();
   }
   // du_P = [da | db] [W_gate; W_up]
