@@ -59,11 +59,26 @@ __global__ void decode_rope_cache_kernel(const float* __restrict__ qkv,
   }
 }
 
+// Shared memory of one attention split: the split's K rows, then its V rows,
+// at a pitch of HD * 2 + 16 bytes (a quarter warp reading 16 bytes from each
+// of 8 consecutive rows, or 8 consecutive 16-byte pieces of one row, meets
+// no bank twice), the group's q in fp32 and the two windows' scores.
+template <int HD>
+constexpr int dec_pitch() { return HD * 2 + 16; }
+template <int HD>
+constexpr int dec_attn_smem_bytes(int G) {
+  return DEC_KC * dec_pitch<HD>() + G * HD * 4 + 2 * G * DEC_KC * 4;
+}
+
 // Both windows of one KV head's query heads over one split of DEC_KC keys of
 // the teacher range [max(0, t-w_T+1), t]; the student window is its last w_S
-// keys.  Partial results (log2-domain max, sum, unnormalised output) per
-// (b, h, window, split): pm, pl [B, Hq, 2, nsplit], po [B, Hq, 2, nsplit, HD].
-// grid (B * Hkv, nsplit), block DEC_THREADS.
+// keys.  The block copies the split's K rows into shared memory with all
+// copies in flight at once, forms the scores, starts the same copy of the V
+// rows over the K rows, and runs the softmax while they arrive.  Partial
+// results (log2-domain max, sum, unnormalised output) per (b, h, window,
+// split): pm, pl [B, Hq, 2, nsplit], po [B, Hq, 2, nsplit, HD].
+// grid (B * Hkv, nsplit), block DEC_THREADS, dynamic shared memory
+// dec_attn_smem_bytes<HD>(Hq / Hkv).
 template <int HD>
 __global__ void __launch_bounds__(DEC_THREADS)
     decode_attn_partial_kernel(const __nv_bfloat16* __restrict__ q_rot,
@@ -73,24 +88,42 @@ __global__ void __launch_bounds__(DEC_THREADS)
                                int W, int t, int w_S, int w_T, float scale_log2, int nsplit,
                                const long long* pos = nullptr) {
   t = dec_pos(t, pos);
-  __shared__ float qs[DEC_MAXG][HD];
-  __shared__ float ps[2][DEC_MAXG][DEC_KC];  // scores, then probabilities per window
+  constexpr int PITCH = dec_pitch<HD>();
+  constexpr int TPR = HD / 8;              // 16-byte pieces per row
+  constexpr int RPP = DEC_THREADS / TPR;   // rows per pass of the block
+  static_assert(DEC_THREADS % TPR == 0 && RPP * 2 * HD * 4 <= DEC_KC * PITCH,
+                "the key-group reduction must fit the row tile");
+  extern __shared__ __align__(16) unsigned char dsm[];
+  unsigned char* tile = dsm;
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv, sp = blockIdx.y;
   const int G = Hq / Hkv;
+  float* qs = reinterpret_cast<float*>(dsm + DEC_KC * PITCH);  // [G][HD]
+  float* ps = qs + G * HD;                                      // [2][G][DEC_KC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j_lo = max(0, t - w_T + 1);
   const int j0 = j_lo + sp * DEC_KC;
   const int n = max(0, min(t - j0 + 1, DEC_KC));  // keys of this split
   const int s_lo = max(0, t - w_S + 1) - j0;      // first student key index (may be <0 or >=n)
+  // this thread's 16-byte piece of every RPP-th row: rows r0, r0 + RPP, ...
+  const int piece = tid % TPR, r0 = tid / TPR;
+  const long long row_stride = static_cast<long long>(Hkv) * HD;  // elements between ring slots
+  const long long head_base = (static_cast<long long>(b) * W * Hkv + g) * HD + piece * 8;
+  auto copy_rows = [&](const __nv_bfloat16* cache) {
+    int slot = (j0 + r0) % W;
+    for (int r = r0; r < n; r += RPP) {
+      cp_async16(tile + r * PITCH + piece * 16, cache + head_base + slot * row_stride);
+      slot += RPP;
+      if (slot >= W) slot -= W;
+    }
+  };
+  copy_rows(kc);
   for (int e = tid; e < G * HD; e += DEC_THREADS)
-    qs[e / HD][e % HD] = __bfloat162float(
-        q_rot[(static_cast<long long>(b) * Hq + g * G + e / HD) * HD + e % HD]);
+    qs[e] = __bfloat162float(q_rot[(static_cast<long long>(b) * Hq + g * G) * HD + e]);
+  cp_async_wait_all();
   __syncthreads();
-  // scores (log2 domain)
+  // scores (log2 domain), one key row per thread at a time
   for (int kk = tid; kk < n; kk += DEC_THREADS) {
-    const long long slot = (j0 + kk) % W;  // two keys per thread: the modulo is not hot
-    const uint4* krow = reinterpret_cast<const uint4*>(
-        kc + ((b * static_cast<long long>(W) + slot) * Hkv + g) * HD);
+    const uint4* krow = reinterpret_cast<const uint4*>(tile + kk * PITCH);
     float acc[DEC_MAXG];
 #pragma unroll
     for (int hh = 0; hh < DEC_MAXG; ++hh) acc[hh] = 0.f;
@@ -103,24 +136,28 @@ __global__ void __launch_bounds__(DEC_THREADS)
         const float k0 = bf16lo_to_f32(w4[q]), k1 = bf16hi_to_f32(w4[q]);
 #pragma unroll
         for (int hh = 0; hh < DEC_MAXG; ++hh)
-          if (hh < G) acc[hh] += qs[hh][c8 * 8 + 2 * q] * k0 + qs[hh][c8 * 8 + 2 * q + 1] * k1;
+          if (hh < G)
+            acc[hh] += qs[hh * HD + c8 * 8 + 2 * q] * k0 + qs[hh * HD + c8 * 8 + 2 * q + 1] * k1;
       }
     }
-    for (int hh = 0; hh < G; ++hh) ps[0][hh][kk] = acc[hh] * scale_log2;
+    for (int hh = 0; hh < G; ++hh) ps[hh * DEC_KC + kk] = acc[hh] * scale_log2;
   }
   __syncthreads();
+  copy_rows(vc);  // V over K, in flight during the softmax
   // per (head, window): maximum, probabilities, sum (one warp per pair)
+  float* pT = ps;                 // [G][DEC_KC]: teacher scores, then probabilities
+  float* pS = ps + G * DEC_KC;    // [G][DEC_KC]: student probabilities
   for (int pr = warp; pr < 2 * G; pr += DEC_THREADS / 32) {
     const int hh = pr >> 1, win = pr & 1;  // win 0: teacher, 1: student
     const int k_first = win ? max(s_lo, 0) : 0;
     float m = -INFINITY;
-    for (int kk = k_first + lane; kk < n; kk += 32) m = fmaxf(m, ps[0][hh][kk]);
+    for (int kk = k_first + lane; kk < n; kk += 32) m = fmaxf(m, pT[hh * DEC_KC + kk]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float l = 0.f;
     for (int kk = lane; kk < DEC_KC; kk += 32) {
-      const float p = (kk >= k_first && kk < n) ? exp2f(ps[0][hh][kk] - m) : 0.f;
-      if (win) ps[1][hh][kk] = p;
+      const float p = (kk >= k_first && kk < n) ? exp2f(pT[hh * DEC_KC + kk] - m) : 0.f;
+      if (win) pS[hh * DEC_KC + kk] = p;
       l += p;
     }
 #pragma unroll
@@ -132,31 +169,28 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
   }
   __syncthreads();
-  // teacher probabilities in place of the scores (the student ones are in ps[1])
+  // teacher probabilities in place of the scores
   for (int pr = warp; pr < G; pr += DEC_THREADS / 32) {
     const long long pi = ((static_cast<long long>(b) * Hq + g * G + pr) * 2) * nsplit + sp;
     const float m = pm[pi];
     for (int kk = lane; kk < DEC_KC; kk += 32)
-      ps[0][pr][kk] = kk < n ? exp2f(ps[0][pr][kk] - m) : 0.f;
+      pT[pr * DEC_KC + kk] = kk < n ? exp2f(pT[pr * DEC_KC + kk] - m) : 0.f;
   }
+  cp_async_wait_all();
   __syncthreads();
-  // P.V with 16-byte loads: 16 threads cover a 128-column row (8 columns each),
-  // DEC_THREADS / (HD / 8) key groups take every (#groups)-th key, and the
-  // groups are summed through shared memory (reusing the score buffer).
+  // P.V from shared memory: TPR threads cover a row (8 columns each), RPP key
+  // groups take every RPP-th key, and the groups are summed through shared
+  // memory (reusing the row tile).
   {
-    constexpr int TPR = HD / 8;                 // threads per V row
-    constexpr int KG = DEC_THREADS / TPR;       // key groups
-    const int dg = tid % TPR, kg = tid / TPR;
+    const int dg = piece, kg = r0;
     float aT[DEC_MAXG][8], aS[DEC_MAXG][8];
 #pragma unroll
     for (int hh = 0; hh < DEC_MAXG; ++hh)
 #pragma unroll
       for (int e = 0; e < 8; ++e) aT[hh][e] = aS[hh][e] = 0.f;
-    const long long vbase = (b * static_cast<long long>(W)) * Hkv + g;
-    int slot = (j0 + kg) % W;  // ring slot of key kk = kg; advances by KG per step
 #pragma unroll 2
-    for (int kk = kg; kk < n; kk += KG) {
-      const uint4 u = *reinterpret_cast<const uint4*>(vc + ((vbase + static_cast<long long>(slot) * Hkv) * HD + dg * 8));
+    for (int kk = kg; kk < n; kk += RPP) {
+      const uint4 u = *reinterpret_cast<const uint4*>(tile + kk * PITCH + dg * 16);
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
       float vv[8];
 #pragma unroll
@@ -167,19 +201,16 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
       for (int hh = 0; hh < DEC_MAXG; ++hh)
         if (hh < G) {
-          const float pT = ps[0][hh][kk], pS = ps[1][hh][kk];
+          const float wT = pT[hh * DEC_KC + kk], wS = pS[hh * DEC_KC + kk];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            aT[hh][e] += pT * vv[e];
-            aS[hh][e] += pS * vv[e];
+            aT[hh][e] += wT * vv[e];
+            aS[hh][e] += wS * vv[e];
           }
         }
-      slot += KG;
-      if (slot >= W) slot -= W;
     }
-    // Sum the key groups one head at a time through shared memory (the
-    // probabilities are no longer needed: ps is reused, KG * 2 * HD <= 2 * DEC_KC * DEC_MAXG).
-    float* red = &ps[0][0][0];
+    // Sum the key groups one head at a time (RPP * 2 * HD floats fit the tile).
+    float* red = reinterpret_cast<float*>(tile);
 #pragma unroll
     for (int hh = 0; hh < DEC_MAXG; ++hh) {
       if (hh >= G) break;  // G is the same for the whole block
@@ -193,7 +224,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int o = tid; o < 2 * HD; o += DEC_THREADS) {
         const int win = o / HD, d = o % HD;
         float acc = 0.f;
-        for (int q = 0; q < KG; ++q) acc += red[(q * 2 + win) * HD + d];
+        for (int q = 0; q < RPP; ++q) acc += red[(q * 2 + win) * HD + d];
         const long long base =
             (((static_cast<long long>(b) * Hq + g * G + hh) * 2) + win) * nsplit + sp;
         po[base * HD + d] = acc;
@@ -201,7 +232,6 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
   }
 }
-
 // Merge the splits: o = sum_s po_s 2^(pm_s - m) / sum_s pl_s 2^(pm_s - m).
 // o [2, B, Hq * HD] bf16 (teacher rows, then student rows).  grid B * Hq * 2, block HD.
 template <int HD>
