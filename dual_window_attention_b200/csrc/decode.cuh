@@ -14,7 +14,7 @@
 namespace ttcd {
 
 constexpr int DEC_KC = 256;       // keys per attention split
-constexpr int DEC_THREADS = 128;  // attention split block
+constexpr int DEC_THREADS = 256;  // attention split block
 constexpr int DEC_MAXG = 8;       // query heads per KV head handled by one block
 
 // Position of the token being decoded: the kernels take it as an argument, or,
@@ -77,9 +77,10 @@ constexpr int dec_attn_smem_bytes(int G) {
 // rows over the K rows, and runs the softmax while they arrive.  Partial
 // results (log2-domain max, sum, unnormalised output) per (b, h, window,
 // split): pm, pl [B, Hq, 2, nsplit], po [B, Hq, 2, nsplit, HD].
+// GM >= Hq / Hkv bounds the query heads per KV head (the register arrays).
 // grid (B * Hkv, nsplit), block DEC_THREADS, dynamic shared memory
 // dec_attn_smem_bytes<HD>(Hq / Hkv).
-template <int HD>
+template <int HD, int GM>
 __global__ void __launch_bounds__(DEC_THREADS)
     decode_attn_partial_kernel(const __nv_bfloat16* __restrict__ q_rot,
                                const __nv_bfloat16* __restrict__ kc,
@@ -124,9 +125,9 @@ __global__ void __launch_bounds__(DEC_THREADS)
   // scores (log2 domain), one key row per thread at a time
   for (int kk = tid; kk < n; kk += DEC_THREADS) {
     const uint4* krow = reinterpret_cast<const uint4*>(tile + kk * PITCH);
-    float acc[DEC_MAXG];
+    float acc[GM];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh) acc[hh] = 0.f;
+    for (int hh = 0; hh < GM; ++hh) acc[hh] = 0.f;
 #pragma unroll 4
     for (int c8 = 0; c8 < HD / 8; ++c8) {
       const uint4 u = krow[c8];
@@ -135,12 +136,14 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int q = 0; q < 4; ++q) {
         const float k0 = bf16lo_to_f32(w4[q]), k1 = bf16hi_to_f32(w4[q]);
 #pragma unroll
-        for (int hh = 0; hh < DEC_MAXG; ++hh)
+        for (int hh = 0; hh < GM; ++hh)
           if (hh < G)
             acc[hh] += qs[hh * HD + c8 * 8 + 2 * q] * k0 + qs[hh * HD + c8 * 8 + 2 * q + 1] * k1;
       }
     }
-    for (int hh = 0; hh < G; ++hh) ps[hh * DEC_KC + kk] = acc[hh] * scale_log2;
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh)
+      if (hh < G) ps[hh * DEC_KC + kk] = acc[hh] * scale_log2;
   }
   __syncthreads();
   copy_rows(vc);  // V over K, in flight during the softmax
@@ -183,9 +186,9 @@ __global__ void __launch_bounds__(DEC_THREADS)
   // memory (reusing the row tile).
   {
     const int dg = piece, kg = r0;
-    float aT[DEC_MAXG][8], aS[DEC_MAXG][8];
+    float aT[GM][8], aS[GM][8];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh)
+    for (int hh = 0; hh < GM; ++hh)
 #pragma unroll
       for (int e = 0; e < 8; ++e) aT[hh][e] = aS[hh][e] = 0.f;
 #pragma unroll 2
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
         vv[2 * q + 1] = bf16hi_to_f32(w4[q]);
       }
 #pragma unroll
-      for (int hh = 0; hh < DEC_MAXG; ++hh)
+      for (int hh = 0; hh < GM; ++hh)
         if (hh < G) {
           const float wT = pT[hh * DEC_KC + kk], wS = pS[hh * DEC_KC + kk];
 #pragma unroll
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
     // Sum the key groups one head at a time (RPP * 2 * HD floats fit the tile).
     float* red = reinterpret_cast<float*>(tile);
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh) {
+    for (int hh = 0; hh < GM; ++hh) {
       if (hh >= G) break;  // G is the same for the whole block
       __syncthreads();
 #pragma unroll

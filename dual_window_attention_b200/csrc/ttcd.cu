@@ -1681,11 +1681,13 @@ ttcd_status dec_attention(const Ctx& c, const ttcd_block_params* p, void* state,
                           const long long* pos) {
   using bf = __nv_bfloat16;
   const int B = p->B, Hq = p->n_q_heads, Hkv = p->n_kv_heads;
-  const int smem = dec_attn_smem_bytes<HD>(Hq / Hkv);
-  if (cudaFuncSetAttribute(decode_attn_partial_kernel<HD>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  const int G = Hq / Hkv;
+  const int smem = dec_attn_smem_bytes<HD>(G);
+  auto kern = G <= 2 ? decode_attn_partial_kernel<HD, 2>
+                     : (G <= 4 ? decode_attn_partial_kernel<HD, 4> : decode_attn_partial_kernel<HD, 8>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTCD_ERR_CUDA;
-  decode_attn_partial_kernel<HD><<<dim3(B * Hkv, L.nsplit), DEC_THREADS, smem, c.s>>>(
+  kern<<<dim3(B * Hkv, L.nsplit), DEC_THREADS, smem, c.s>>>(
       dat<bf>(ws, L.qrot), dat<bf>(state, S.kc), dat<bf>(state, S.vc), dat<float>(ws, L.pm),
       dat<float>(ws, L.pl), dat<float>(ws, L.po), Hq, Hkv, p->w_T, t, p->w_S, p->w_T,
       scale * 1.4426950408889634f, L.nsplit, pos);
