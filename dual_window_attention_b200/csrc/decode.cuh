@@ -65,9 +65,17 @@ __global__ void decode_rope_cache_kernel(const float* __restrict__ qkv,
 // no bank twice), the group's q in fp32 and the two windows' scores.
 template <int HD>
 constexpr int dec_pitch() { return HD * 2 + 16; }
+// The row tile, also the scratch of the final key-group sums (fp32, two
+// windows, DEC_THREADS / (HD / 8) groups).
+template <int HD>
+constexpr int dec_tile_bytes() {
+  return DEC_KC * dec_pitch<HD>() > (DEC_THREADS / (HD / 8)) * 2 * HD * 4
+             ? DEC_KC * dec_pitch<HD>()
+             : (DEC_THREADS / (HD / 8)) * 2 * HD * 4;
+}
 template <int HD>
 constexpr int dec_attn_smem_bytes(int G) {
-  return DEC_KC * dec_pitch<HD>() + G * HD * 4 + 2 * G * DEC_KC * 4;
+  return dec_tile_bytes<HD>() + G * HD * 4 + 2 * G * DEC_KC * 4;
 }
 
 // Both windows of one KV head's query heads over one split of DEC_KC keys of
@@ -92,13 +100,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
   constexpr int PITCH = dec_pitch<HD>();
   constexpr int TPR = HD / 8;              // 16-byte pieces per row
   constexpr int RPP = DEC_THREADS / TPR;   // rows per pass of the block
-  static_assert(DEC_THREADS % TPR == 0 && RPP * 2 * HD * 4 <= DEC_KC * PITCH,
+  static_assert(DEC_THREADS % TPR == 0 && RPP * 2 * HD * 4 <= dec_tile_bytes<HD>(),
                 "the key-group reduction must fit the row tile");
   extern __shared__ __align__(16) unsigned char dsm[];
   unsigned char* tile = dsm;
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv, sp = blockIdx.y;
   const int G = Hq / Hkv;
-  float* qs = reinterpret_cast<float*>(dsm + DEC_KC * PITCH);  // [G][HD]
+  float* qs = reinterpret_cast<float*>(dsm + dec_tile_bytes<HD>());  // [G][HD]
   float* ps = qs + G * HD;                                      // [2][G][DEC_KC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j_lo = max(0, t - w_T + 1);
