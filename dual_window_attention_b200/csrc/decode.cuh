@@ -13,6 +13,16 @@
 
 namespace ttcd {
 
+// 16-byte global -> shared copy that bypasses L1 (both addresses 16-byte aligned);
+// completion by cp_async_wait_all in the issuing thread, then a block barrier.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 constexpr int DEC_KC = 256;       // keys per attention split
 constexpr int DEC_THREADS = 256;  // attention split block
 constexpr int DEC_MAXG = 8;       // query heads per KV head handled by one block
@@ -350,24 +360,47 @@ __global__ void decode_conv_kernel(const float* __restrict__ Z,
   }
 }
 
-// kscale[b] = beta_t[b] / sqrt(||zbar_S||^2 + eps), the partial sums added in a
-// fixed order.  grid B, block 32.
+// beta_t[b] / sqrt(||zbar_S||^2 + eps) from the conv kernel's partial sums,
+// added in a fixed order (lane-strided, then a butterfly): every lane of the
+// calling warp returns the same value.
+__device__ __forceinline__ float dec_key_scale(const float* __restrict__ ssq_part, int n_part,
+                                               const float* __restrict__ beta, float eps, int b,
+                                               int lane) {
+  float s = 0.f;
+  for (int i = lane; i < n_part; i += 32) s += ssq_part[static_cast<long long>(b) * n_part + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return beta[b] / sqrtf(s + eps);
+}
+
+// kscale[b] = dec_key_scale(b).  grid B, block 32.
 __global__ void decode_kscale_kernel(const float* __restrict__ ssq_part, int n_part,
                                      const float* __restrict__ beta, float* __restrict__ kscale,
                                      float eps) {
-  const int b = blockIdx.x;
-  float s = 0.f;
-  for (int i = threadIdx.x; i < n_part; i += 32) s += ssq_part[static_cast<long long>(b) * n_part + i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (threadIdx.x == 0) kscale[b] = beta[b] / sqrtf(s + eps);
+  const float k = dec_key_scale(ssq_part, n_part, beta, eps, blockIdx.x, threadIdx.x);
+  if (threadIdx.x == 0) kscale[blockIdx.x] = k;
 }
+
+// Epilogue arguments of the key-row GEMV (EPI 2): the key scale from the conv
+// kernel's partial sums, and the destination row of the current chunk slot
+// (row (pos ? *pos : t) % C of each sequence's Cp-row block).
+struct DecKeyRowEpi {
+  const float* ssq_part;
+  int n_part;
+  const float* beta;
+  float eps;
+  const long long* pos;
+  int t;
+  int C;
+  int Cp;
+};
 
 // Y[r, n] = epi(W[n, :] . X[r, :]) for R <= DEC_GEMV_ROWS input rows: the
 // dense products of a decode step, whose few rows would leave a 128-row tensor
 // core tile nearly empty.  One warp per weight row n streams W[n] once (16-byte
 // loads) against every input row (from L1).  Epilogues: 0 fp32 store;
-// 1 silu(W[n].x) * (W2[n].x) (SwiGLU, fp32); 2 bf16 store scaled by scale[r].
+// 1 silu(W[n].x) * (W2[n].x) (SwiGLU, fp32); 2 bf16 store scaled by the key
+// scale of row r into its chunk-slot row (kr).
 // grid cdiv(N, 8), block 256.
 constexpr int DEC_GEMV_ROWS = 16;   // rows one GEMV launch can take
 constexpr int DEC_GEMV_SWITCH = 8;  // up to this many rows the GEMV beats a 128-row GEMM tile (B200, measured)
@@ -375,12 +408,13 @@ template <int EPI>
 __global__ void decode_gemv_kernel(const __nv_bfloat16* __restrict__ Wm,
                                    const __nv_bfloat16* __restrict__ W2,
                                    const __nv_bfloat16* __restrict__ X, void* __restrict__ Y,
-                                   const float* __restrict__ scale, int R, int N, int K,
-                                   long long ldy) {
+                                   int R, int N, int K, long long ldy,
+                                   DecKeyRowEpi kr = DecKeyRowEpi{}) {
   const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (n >= N) return;
   constexpr int NW = EPI == 1 ? 2 : 1;
+  const int slot_row = EPI == 2 ? static_cast<int>((kr.pos ? *kr.pos : kr.t) % kr.C) : 0;
   float acc[NW][DEC_GEMV_ROWS];
 #pragma unroll
   for (int q = 0; q < NW; ++q)
@@ -426,9 +460,13 @@ __global__ void decode_gemv_kernel(const __nv_bfloat16* __restrict__ Wm,
       } else if (EPI == 1) {
         const float gg = acc[0][r];
         static_cast<float*>(Y)[r * ldy + n] = gg / (1.0f + __expf(-gg)) * acc[NW - 1][r];
-      } else {
-        static_cast<__nv_bfloat16*>(Y)[r * ldy + n] = __float2bfloat16_rn(acc[0][r] * scale[r]);
       }
+    }
+    if (EPI == 2) {  // whole warp: the key scale's butterfly
+      const float ks = dec_key_scale(kr.ssq_part, kr.n_part, kr.beta, kr.eps, r, lane);
+      if (lane == 0)
+        static_cast<__nv_bfloat16*>(Y)[(static_cast<long long>(r) * kr.Cp + slot_row) * ldy + n] =
+            __float2bfloat16_rn(acc[0][r] * ks);
     }
   }
 }

@@ -1718,8 +1718,8 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   const bool gemv = 2 * B <= DEC_GEMV_SWITCH;
   if (gemv) {
     decode_gemv_kernel<0><<<cdiv(dqkv, 8), 256, 0, c.s>>>(
-        static_cast<const bf*>(w->w_qkv), nullptr, dat<bf>(ws, L.xn), dat<float>(ws, L.qkv),
-        nullptr, B, dqkv, d, dqkv);
+        static_cast<const bf*>(w->w_qkv), nullptr, dat<bf>(ws, L.xn), dat<float>(ws, L.qkv), B,
+        dqkv, d, dqkv);
     TTCD_CHECK_LAUNCH();
   } else {
     CUtensorMap mA, mB, mo;
@@ -1743,8 +1743,8 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   // o_proj for both paths, residual, MLP RMSNorm
   if (gemv) {
     decode_gemv_kernel<0><<<cdiv(d, 8), 256, 0, c.s>>>(
-        static_cast<const bf*>(w->w_o), nullptr, dat<bf>(ws, L.o), dat<float>(ws, L.hp), nullptr,
-        2 * B, d, Hq * hd, d);
+        static_cast<const bf*>(w->w_o), nullptr, dat<bf>(ws, L.o), dat<float>(ws, L.hp), 2 * B, d,
+        Hq * hd, d);
     TTCD_CHECK_LAUNCH();
   } else {
     CUtensorMap mA, mB, mo;
@@ -1764,7 +1764,7 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   if (gemv) {
     decode_gemv_kernel<1><<<cdiv(f, 8), 256, 0, c.s>>>(
         static_cast<const bf*>(w->w_gate), static_cast<const bf*>(w->w_up), dat<bf>(ws, L.u),
-        dat<float>(ws, L.Z), nullptr, 2 * B, f, d, f);
+        dat<float>(ws, L.Z), 2 * B, f, d, f);
     TTCD_CHECK_LAUNCH();
   } else {
     CUtensorMap mA, mB0, mB1, mo;
@@ -1782,16 +1782,17 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
       dat<float>(state, S.hist), dat<bf>(ws, L.D), dat<bf>(state, S.kx), dat<bf>(ws, L.Zs),
       dat<float>(ws, L.ssq), B, f, p->conv_k, t, C, Cp, pos);
   TTCD_CHECK_LAUNCH();
-  decode_kscale_kernel<<<B, 32, 0, c.s>>>(dat<float>(ws, L.ssq), n_part, beta,
-                                          dat<float>(ws, L.ks), p->l2_eps);
-  TTCD_CHECK_LAUNCH();
-  // r = (D M^T) beta / ||zbar_S||, into the chunk buffer
+  // r = (D M^T) beta / ||zbar_S||, into the chunk buffer: the GEMV forms the
+  // key scale and writes the chunk slot itself
   if (gemv) {
+    DecKeyRowEpi kr{dat<float>(ws, L.ssq), n_part, beta, p->l2_eps, pos, t, C, Cp};
     decode_gemv_kernel<2><<<cdiv(d, 8), 256, 0, c.s>>>(
-        dat<bf>(state, S.M), nullptr, dat<bf>(ws, L.D), dat<bf>(ws, L.r), dat<float>(ws, L.ks), B,
-        d, f, d);
+        dat<bf>(state, S.M), nullptr, dat<bf>(ws, L.D), dat<bf>(state, S.rc), B, d, f, d, kr);
     TTCD_CHECK_LAUNCH();
   } else {
+    decode_kscale_kernel<<<B, 32, 0, c.s>>>(dat<float>(ws, L.ssq), n_part, beta,
+                                            dat<float>(ws, L.ks), p->l2_eps);
+    TTCD_CHECK_LAUNCH();
     CUtensorMap mA, mB, mo;
     if (!map_rows<bf>(&mA, dat<bf>(ws, L.D), B, f, 128) ||
         !map_rows<bf>(&mB, dat<bf>(state, S.M), d, f, 256) ||
@@ -1799,10 +1800,10 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
       return TTCD_ERR_CUDA;
     EpiStore<bf> e{dat<bf>(ws, L.r), d, d, dat<float>(ws, L.ks)};
     TTCD_TRY((launch_gemm<bf, 256, 4, false>(c, mA, mB, mB, &mo, plain_geom(B, cdiv(d, 256), f), e)));
+    decode_row_copy_kernel<<<static_cast<unsigned>(cdiv(static_cast<long long>(B) * d, 256)), 256, 0, c.s>>>(
+        dat<bf>(ws, L.r), dat<bf>(state, S.rc), B, d, Cp, t % C, pos, C);
+    TTCD_CHECK_LAUNCH();
   }
-  decode_row_copy_kernel<<<static_cast<unsigned>(cdiv(static_cast<long long>(B) * d, 256)), 256, 0, c.s>>>(
-      dat<bf>(ws, L.r), dat<bf>(state, S.rc), B, d, Cp, t % C, pos, C);
-  TTCD_CHECK_LAUNCH();
   // output with the current chunk's weight W_down + S
   decode_out_kernel<<<dim3(cdiv(d, 8), B), 256, 0, c.s>>>(dat<bf>(state, S.weff), dat<bf>(ws, L.Zs),
                                                          dat<float>(ws, L.hS), y, d, f);
