@@ -23,6 +23,9 @@ DEC_B = BlockShape("decode_hd128_chunk96", "bf16", B=1, T=230, d_model=256, n_q_
                    n_kv_heads=1, head_dim=128, d_ff=512, w_S=40, w_T=150, chunk=96, conv_k=3)
 # nine sequences: 2B = 18 rows take the tensor-core GEMM path instead of the GEMV
 DEC_C = DEC_A.with_(name="decode_batch9_gemm_path", B=9, T=150)
+# eight sequences (2B = 16 rows: the tensor-core GEMM path), the largest batch
+# the decode benchmark runs
+DEC_E = DEC_A.with_(name="decode_batch8", B=8, T=140)
 # eight query heads per KV head at hd 32, a teacher window of two 256-key splits
 DEC_D = BlockShape("decode_hd32_gqa8", "bf16", B=2, T=340, d_model=128, n_q_heads=8,
                    n_kv_heads=1, head_dim=32, d_ff=256, w_S=48, w_T=300, chunk=128, conv_k=4)
@@ -44,7 +47,7 @@ def _decode_all(ttcd, shape, inp, state_in=None):
     return torch.stack(ys, dim=1), dec.state_out(), x, w, p
 
 
-@pytest.mark.parametrize("shape", [DEC_A, DEC_B, DEC_C, DEC_D], ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", [DEC_A, DEC_B, DEC_C, DEC_D, DEC_E], ids=lambda s: s.name)
 def test_decode_matches_block_forward(ttcd, shape):
     inp = make_block_inputs(shape, seed=4)
     y, state, x, w, p = _decode_all(ttcd, shape, inp)
