@@ -404,6 +404,10 @@ struct DecKeyRowEpi {
 // grid cdiv(N, 8), block 256.
 constexpr int DEC_GEMV_ROWS = 16;   // rows one GEMV launch can take
 constexpr int DEC_GEMV_SWITCH = 8;  // up to this many rows the GEMV beats a 128-row GEMM tile (B200, measured)
+// The products with B rows (QKV, and r over the long K = d_ff) take the GEMV
+// up to this many rows; their few-CTA GEMM grids lose to it until then (B200,
+// measured per B with the CUDA graph).
+constexpr int DEC_GEMV_SWITCH_B = 6;
 template <int EPI>
 __global__ void decode_gemv_kernel(const __nv_bfloat16* __restrict__ Wm,
                                    const __nv_bfloat16* __restrict__ W2,

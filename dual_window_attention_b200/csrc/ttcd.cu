@@ -1714,9 +1714,10 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   rmsnorm_kernel<bf, bf, bf><<<cdiv(B, 8), 256, 0, c.s>>>(
       x, static_cast<const bf*>(w->g_attn), dat<bf>(ws, L.xn), B, d, p->rms_eps);
   TTCD_CHECK_LAUNCH();
-  // few rows (2B <= 16): warp-per-row GEMV; otherwise the tcgen05 GEMM
-  const bool gemv = 2 * B <= DEC_GEMV_SWITCH;
-  if (gemv) {
+  // few rows: warp-per-row GEMV; otherwise the tcgen05 GEMM
+  const bool gemv_B = B <= DEC_GEMV_SWITCH_B;      // QKV and r: B rows
+  const bool gemv = 2 * B <= DEC_GEMV_SWITCH;       // o_proj and gate/up: both paths, 2B rows
+  if (gemv_B) {
     decode_gemv_kernel<0><<<cdiv(dqkv, 8), 256, 0, c.s>>>(
         static_cast<const bf*>(w->w_qkv), nullptr, dat<bf>(ws, L.xn), dat<float>(ws, L.qkv), B,
         dqkv, d, dqkv);
@@ -1784,7 +1785,7 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   TTCD_CHECK_LAUNCH();
   // r = (D M^T) beta / ||zbar_S||, into the chunk buffer: the GEMV forms the
   // key scale and writes the chunk slot itself
-  if (gemv) {
+  if (gemv_B) {
     DecKeyRowEpi kr{dat<float>(ws, L.ssq), n_part, beta, p->l2_eps, pos, t, C, Cp};
     decode_gemv_kernel<2><<<cdiv(d, 8), 256, 0, c.s>>>(
         dat<bf>(state, S.M), nullptr, dat<bf>(ws, L.D), dat<bf>(state, S.rc), B, d, f, d, kr);

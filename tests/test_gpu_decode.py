@@ -23,9 +23,9 @@ DEC_B = BlockShape("decode_hd128_chunk96", "bf16", B=1, T=230, d_model=256, n_q_
                    n_kv_heads=1, head_dim=128, d_ff=512, w_S=40, w_T=150, chunk=96, conv_k=3)
 # nine sequences: 2B = 18 rows take the tensor-core GEMM path instead of the GEMV
 DEC_C = DEC_A.with_(name="decode_batch9_gemm_path", B=9, T=150)
-# eight sequences (2B = 16 rows: the tensor-core GEMM path), the largest batch
-# the decode benchmark runs
-DEC_E = DEC_A.with_(name="decode_batch8", B=8, T=140)
+# six sequences: the B-row products (QKV, r) on the GEMV, the 2B-row products
+# (o_proj, gate/up) on the tensor-core GEMM
+DEC_E = DEC_A.with_(name="decode_batch6_mixed_path", B=6, T=140)
 # eight query heads per KV head at hd 32, a teacher window of two 256-key splits
 DEC_D = BlockShape("decode_hd32_gqa8", "bf16", B=2, T=340, d_model=128, n_q_heads=8,
                    n_kv_heads=1, head_dim=32, d_ff=256, w_S=48, w_T=300, chunk=128, conv_k=4)
