@@ -143,25 +143,27 @@ __global__ void __launch_bounds__(DEC_THREADS)
   // scores (log2 domain), one key row per thread at a time
   for (int kk = tid; kk < n; kk += DEC_THREADS) {
     const uint4* krow = reinterpret_cast<const uint4*>(tile + kk * PITCH);
-    float acc[GM];
+    // even and odd columns summed apart, two per packed FMA
+    float2 acc[GM];
 #pragma unroll
-    for (int hh = 0; hh < GM; ++hh) acc[hh] = 0.f;
+    for (int hh = 0; hh < GM; ++hh) acc[hh] = make_float2(0.f, 0.f);
 #pragma unroll 4
     for (int c8 = 0; c8 < HD / 8; ++c8) {
       const uint4 u = krow[c8];
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float k0 = bf16lo_to_f32(w4[q]), k1 = bf16hi_to_f32(w4[q]);
+        const float2 k2 = make_float2(bf16lo_to_f32(w4[q]), bf16hi_to_f32(w4[q]));
 #pragma unroll
         for (int hh = 0; hh < GM; ++hh)
           if (hh < G)
-            acc[hh] += qs[hh * HD + c8 * 8 + 2 * q] * k0 + qs[hh * HD + c8 * 8 + 2 * q + 1] * k1;
+            acc[hh] = __ffma2_rn(*reinterpret_cast<const float2*>(&qs[hh * HD + c8 * 8 + 2 * q]),
+                                 k2, acc[hh]);
       }
     }
 #pragma unroll
     for (int hh = 0; hh < GM; ++hh)
-      if (hh < G) ps[hh * DEC_KC + kk] = acc[hh] * scale_log2;
+      if (hh < G) ps[hh * DEC_KC + kk] = (acc[hh].x + acc[hh].y) * scale_log2;
   }
   __syncthreads();
   copy_rows(vc);  // V over K, in flight during the softmax
@@ -204,32 +206,40 @@ __global__ void __launch_bounds__(DEC_THREADS)
   // memory (reusing the row tile).
   {
     const int dg = piece, kg = r0;
-    float aT[GM][8], aS[GM][8];
+    float2 aT2[GM][4], aS2[GM][4];  // column pairs, two per packed FMA
 #pragma unroll
     for (int hh = 0; hh < GM; ++hh)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) aT[hh][e] = aS[hh][e] = 0.f;
+      for (int e = 0; e < 4; ++e) aT2[hh][e] = aS2[hh][e] = make_float2(0.f, 0.f);
 #pragma unroll 2
     for (int kk = kg; kk < n; kk += RPP) {
       const uint4 u = *reinterpret_cast<const uint4*>(tile + kk * PITCH + dg * 16);
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-      float vv[8];
+      float2 vv[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        vv[2 * q] = bf16lo_to_f32(w4[q]);
-        vv[2 * q + 1] = bf16hi_to_f32(w4[q]);
-      }
+      for (int q = 0; q < 4; ++q) vv[q] = make_float2(bf16lo_to_f32(w4[q]), bf16hi_to_f32(w4[q]));
 #pragma unroll
       for (int hh = 0; hh < GM; ++hh)
         if (hh < G) {
           const float wT = pT[hh * DEC_KC + kk], wS = pS[hh * DEC_KC + kk];
+          const float2 wT2 = make_float2(wT, wT), wS2 = make_float2(wS, wS);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            aT[hh][e] += wT * vv[e];
-            aS[hh][e] += wS * vv[e];
+          for (int e = 0; e < 4; ++e) {
+            aT2[hh][e] = __ffma2_rn(wT2, vv[e], aT2[hh][e]);
+            aS2[hh][e] = __ffma2_rn(wS2, vv[e], aS2[hh][e]);
           }
         }
     }
+    float aT[GM][8], aS[GM][8];
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        aT[hh][2 * e] = aT2[hh][e].x;
+        aT[hh][2 * e + 1] = aT2[hh][e].y;
+        aS[hh][2 * e] = aS2[hh][e].x;
+        aS[hh][2 * e + 1] = aS2[hh][e].y;
+      }
     // Sum the key groups one head at a time (RPP * 2 * HD floats fit the tile).
     float* red = reinterpret_cast<float*>(tile);
 #pragma unroll
