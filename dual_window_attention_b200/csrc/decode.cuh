@@ -524,22 +524,25 @@ __global__ void decode_out_kernel(const __nv_bfloat16* __restrict__ Weff,
     y[static_cast<long long>(b) * d + i] = __float2bfloat16_rn(hS[static_cast<long long>(b) * d + i] + acc);
 }
 
-// Weff[b] = bf16(W_down + S[b]), 4 elements per thread.  With `commit_pos`
+// Weff[b] = bf16(W_down + S[b]), 4 elements per thread and step.  With `commit_pos`
 // set it acts only at the last token of a chunk (*commit_pos % C == C - 1).
 __global__ void decode_weff_kernel(const __nv_bfloat16* __restrict__ w_down,
                                    const float* __restrict__ S, __nv_bfloat16* __restrict__ Weff,
                                    long long df, long long n4,
                                    const long long* commit_pos = nullptr, int C = 1) {
   if (commit_pos && *commit_pos % C != C - 1) return;
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n4) return;
-  const long long e = i * 4, w = e % df;
-  const float4 s = *reinterpret_cast<const float4*>(S + e);
-  const uint2 wd = *reinterpret_cast<const uint2*>(w_down + w);
-  uint2 out;
-  out.x = pack_bf16x2(bf16lo_to_f32(wd.x) + s.x, bf16hi_to_f32(wd.x) + s.y);
-  out.y = pack_bf16x2(bf16lo_to_f32(wd.y) + s.z, bf16hi_to_f32(wd.y) + s.w);
-  *reinterpret_cast<uint2*>(Weff + e) = out;
+  // grid-stride over a small fixed grid: in a replayed decode step the launch
+  // usually only checks the position and exits
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long e = i * 4, w = e % df;
+    const float4 s = *reinterpret_cast<const float4*>(S + e);
+    const uint2 wd = *reinterpret_cast<const uint2*>(w_down + w);
+    uint2 out;
+    out.x = pack_bf16x2(bf16lo_to_f32(wd.x) + s.x, bf16hi_to_f32(wd.x) + s.y);
+    out.y = pack_bf16x2(bf16lo_to_f32(wd.y) + s.z, bf16hi_to_f32(wd.y) + s.w);
+    *reinterpret_cast<uint2*>(Weff + e) = out;
+  }
 }
 
 // Advances the decode state's position counter by one token (the last launch

@@ -1668,7 +1668,8 @@ ttcd_status dec_weff(const Ctx& c, const ttcd_block_params* p, void* state, cons
                      const __nv_bfloat16* w_down, const long long* commit_pos = nullptr) {
   const long long df = static_cast<long long>(p->d_model) * p->d_ff;
   const long long n4 = p->B * df / 4;
-  decode_weff_kernel<<<static_cast<unsigned>(cdiv(n4, 256)), 256, 0, c.s>>>(
+  const long long blocks = std::min<long long>(cdiv(n4, 256), 2LL * c.sms);
+  decode_weff_kernel<<<static_cast<unsigned>(blocks), 256, 0, c.s>>>(
       w_down, dat<float>(state, L.S), dat<__nv_bfloat16>(state, L.weff), df, n4, commit_pos,
       p->chunk);
   TTCD_CHECK_LAUNCH();
