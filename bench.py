@@ -338,6 +338,7 @@ def run_ours(args, world, rank, local):
     barrier(world, local)
     torch.cuda.synchronize()
     launches0 = ttcd.kernel_launch_count()
+    replayed0 = dec.replayed_launches
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
@@ -586,6 +587,7 @@ def run_decode_bench(args, world, rank, local):
     barrier(world, local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ttcd.kernel_launch_count()
+    replayed0 = dec.replayed_launches
     with ClockSampler(local) as clk:
         e0.record(stream)
         for _ in range(args.steps):
@@ -594,7 +596,7 @@ def run_decode_bench(args, world, rank, local):
         torch.cuda.synchronize()
     launches = ttcd.kernel_launch_count() - launches0
     if args.graph:  # replays launch the captured kernels without the host counter
-        launches += dec.graph_launches * args.steps
+        launches += dec.replayed_launches - replayed0
     ms, value = job_throughput(world, args.B * args.steps, e0.elapsed_time(e1))
     if dec.check_status() != ttcd.OK:
         raise RuntimeError("a device wait timed out in the decode benchmark")
@@ -742,6 +744,7 @@ def measure_stack(args, world, local, B, T, steps, warmup):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ttcd.kernel_launch_count()
+    replayed0 = dec.replayed_launches
     with ClockSampler(local) as clk:
         e0.record(stream)
         for _ in range(steps):

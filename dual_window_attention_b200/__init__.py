@@ -81,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttcd_decode_state_init.argtypes = [W, P, vp, vp, sz, vp, sz, vp]
     lib.ttcd_block_decode.argtypes = [vp, vp, i, W, P, vp, sz, vp, vp, sz, vp]
     lib.ttcd_block_decode_next.argtypes = [vp, vp, W, P, vp, sz, vp, vp, sz, vp]
+    lib.ttcd_block_decode_next_ex.argtypes = [vp, vp, W, P, vp, sz, vp, vp, sz, i, vp]
     lib.ttcd_decode_state_read.argtypes = [P, i, vp, sz, vp, vp]
     lib.ttcd_fastweight_mlp.argtypes = [vp, vp, vp, vp, W, P, vp, vp, vp, vp, sz, vp]
     lib.ttcd_block_forward.argtypes = [vp, vp, W, P, vp, vp, vp, sz, vp]
@@ -134,7 +135,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                "ttcd_block_forward", "ttcd_block_forward_profiled", "ttcd_block_workspace_offset",
                "ttcd_get_device_error", "ttcd_check_device_status", "ttcd_test_bounded_wait",
                "ttcd_decode_state_init", "ttcd_block_decode", "ttcd_decode_state_read",
-               "ttcd_block_decode_next", "ttcd_fastweight_mlp_backward",
+               "ttcd_block_decode_next", "ttcd_block_decode_next_ex", "ttcd_fastweight_mlp_backward",
                "ttcd_dual_window_attn_backward", "ttcd_block_backward",
                "ttcd_shard_qkv", "ttcd_shard_attend", "ttcd_shard_mix", "ttcd_shard_finish"):
         getattr(lib, fn).restype = i
@@ -412,9 +413,11 @@ class Decoder:
     position and returns y_t [B, d]; ``state_out()`` is the fast-weight state
     after the tokens so far (partial chunk included).
 
-    ``graph=True``: the steps use ttcd_block_decode_next (the position lives in
-    the state); token 0 runs eagerly, then one step is captured in a CUDA graph
-    with fixed input and output buffers and replayed for every later token."""
+    ``graph=True``: the steps use ttcd_block_decode_next_ex (the position lives
+    in the state); token 0 runs eagerly, then two steps are captured in CUDA
+    graphs with fixed input and output buffers: an ordinary step without the
+    chunk commit's launches, replayed for every later token, and a commit step,
+    replayed at the last token of each chunk (the host's position decides)."""
 
     def __init__(self, weights: Dict[str, torch.Tensor], p: BlockParams, state_in=None,
                  device="cuda", stream=None, graph: bool = False):
@@ -433,18 +436,23 @@ class Decoder:
                                                self.state.numel(), _ptr(self.ws), self.ws.numel(),
                                                _stream(stream)), "ttcd_decode_state_init")
         self.t = 0
-        self.use_graph, self.graph, self.warm, self.graph_launches = graph, None, False, 0
+        self.use_graph, self.warm = graph, False
+        # captured steps: key True = with the chunk commit, False = without
+        self.graphs = {True: None, False: None}
+        self.graph_launches = {True: 0, False: 0}  # kernels per replay of each
+        self.replayed_launches = 0  # kernels launched by all replays so far
         if graph:
             self.x_buf = torch.empty(p.B, p.d_model, device=device, dtype=torch.bfloat16)
             self.b_buf = torch.empty(p.B, device=device, dtype=torch.float32)
             self.y_buf = torch.empty_like(self.x_buf)
 
-    def _next(self):
-        _check(self.lib.ttcd_block_decode_next(_ptr(self.x_buf), _ptr(self.b_buf),
-                                               ctypes.byref(self.wc), ctypes.byref(self.pc),
-                                               _ptr(self.state), self.state.numel(),
-                                               _ptr(self.y_buf), _ptr(self.ws), self.ws.numel(),
-                                               _stream(None)), "ttcd_block_decode_next")
+    def _next(self, commit: bool = True):
+        _check(self.lib.ttcd_block_decode_next_ex(_ptr(self.x_buf), _ptr(self.b_buf),
+                                                  ctypes.byref(self.wc), ctypes.byref(self.pc),
+                                                  _ptr(self.state), self.state.numel(),
+                                                  _ptr(self.y_buf), _ptr(self.ws),
+                                                  self.ws.numel(), int(commit), _stream(None)),
+               "ttcd_block_decode_next_ex")
 
     def seek(self, t: int):
         """Sets the next position to t (host count and, in graph mode, the
@@ -461,18 +469,21 @@ class Decoder:
                 self.x_buf.copy_(x_t)
             if beta_t.data_ptr() != self.b_buf.data_ptr():
                 self.b_buf.copy_(beta_t)
-            if self.graph is None and not self.warm:
-                self._next()  # eager: also loads every kernel before the capture
+            if not self.warm:
+                self._next()  # eager: also loads every kernel before the captures
                 self.warm = True
             else:
-                if self.graph is None:
+                commit = self.t % self.p.chunk == self.p.chunk - 1
+                if self.graphs[commit] is None:
                     torch.cuda.synchronize()
                     n0 = kernel_launch_count()
-                    self.graph = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(self.graph):
-                        self._next()
-                    self.graph_launches = kernel_launch_count() - n0
-                self.graph.replay()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        self._next(commit)
+                    self.graphs[commit] = g
+                    self.graph_launches[commit] = kernel_launch_count() - n0
+                self.graphs[commit].replay()
+                self.replayed_launches += self.graph_launches[commit]
             self.t += 1
             if y is not None and y.data_ptr() == self.y_buf.data_ptr():
                 return y

@@ -1706,7 +1706,7 @@ ttcd_status dec_attention(const Ctx& c, const ttcd_block_params* p, void* state,
 ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, int t,
                        const ttcd_block_weights* w, const ttcd_block_params* p, void* state,
                        const DecState& S, __nv_bfloat16* y, void* ws, const DecWs& L,
-                       long long* pos = nullptr) {
+                       long long* pos = nullptr, bool commit = true) {
   using bf = __nv_bfloat16;
   const int B = p->B, d = p->d_model, f = p->d_ff, hd = p->head_dim;
   const int Hq = p->n_q_heads, Hkv = p->n_kv_heads, dqkv = (Hq + 2 * Hkv) * hd;
@@ -1812,9 +1812,11 @@ ttcd_status run_decode(const Ctx& c, const __nv_bfloat16* x, const float* beta, 
   TTCD_CHECK_LAUNCH();
   // last token of a chunk: S += this chunk's Delta W, then W_down + S
   float* Sp = dat<float>(state, S.S);
-  if (pos) {  // launched every step; the kernels act only at a chunk's last token
-    TTCD_TRY(dec_commit(c, p, state, S, static_cast<const bf*>(w->w_down), Sp, Sp, pos));
-    TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down), pos));
+  if (pos) {  // launched unless the caller omits them; they act only at a chunk's last token
+    if (commit) {
+      TTCD_TRY(dec_commit(c, p, state, S, static_cast<const bf*>(w->w_down), Sp, Sp, pos));
+      TTCD_TRY(dec_weff(c, p, state, S, static_cast<const bf*>(w->w_down), pos));
+    }
     decode_advance_kernel<<<1, 1, 0, c.s>>>(pos);
     TTCD_CHECK_LAUNCH();
   } else if (t % C == C - 1) {
@@ -1893,6 +1895,14 @@ ttcd_status ttcd_block_decode_next(const void* x_t, const float* beta_t,
                                    const ttcd_block_weights* w, const ttcd_block_params* p,
                                    void* state, size_t state_bytes, void* y, void* workspace,
                                    size_t ws_bytes, void* stream) {
+  return ttcd_block_decode_next_ex(x_t, beta_t, w, p, state, state_bytes, y, workspace, ws_bytes,
+                                   1, stream);
+}
+
+ttcd_status ttcd_block_decode_next_ex(const void* x_t, const float* beta_t,
+                                      const ttcd_block_weights* w, const ttcd_block_params* p,
+                                      void* state, size_t state_bytes, void* y, void* workspace,
+                                      size_t ws_bytes, int commit, void* stream) {
   TTCD_TRY(check_decode_params(p));
   if (!aligned16(x_t) || !beta_t || (reinterpret_cast<uintptr_t>(beta_t) & 3u) ||
       !aligned16(y) || !weights_ok(w, true) || !aligned16(state) || !aligned16(workspace))
@@ -1905,7 +1915,7 @@ ttcd_status ttcd_block_decode_next(const void* x_t, const float* beta_t,
   // the position counter sits after the status word in the state's status region
   long long* pos = dat<long long>(state, S.status + 8);
   return run_decode(c, static_cast<const __nv_bfloat16*>(x_t), beta_t, 0, w, p, state, S,
-                    static_cast<__nv_bfloat16*>(y), workspace, L, pos);
+                    static_cast<__nv_bfloat16*>(y), workspace, L, pos, commit != 0);
 }
 
 ttcd_status ttcd_decode_state_read(const ttcd_block_params* p, int t_next, void* state,

@@ -542,6 +542,22 @@ ttcd_status ttcd_block_decode_next(const void* x_t, const float* beta_t,
                                    void* state, size_t state_bytes, void* y, void* workspace,
                                    size_t ws_bytes, void* stream);
 
+/*
+ * ttcd_block_decode_next_ex — ttcd_block_decode_next with the chunk commit
+ * optional.  commit != 0: as ttcd_block_decode_next.  commit == 0: the step
+ * omits the chunk commit's launches (the chunk scan that adds the chunk's
+ * Delta W to the state, and the W_down + S refresh), which act only at the
+ * last token of a chunk; the caller must pass commit != 0 at every position
+ * p with p % chunk == chunk - 1, or the chunk's Delta W is lost.  This lets a
+ * caller capture two CUDA graphs, an ordinary step and a commit step, and
+ * replay the ordinary one for chunk - 1 of every chunk tokens.  Arguments
+ * and errors otherwise as ttcd_block_decode_next.
+ */
+ttcd_status ttcd_block_decode_next_ex(const void* x_t, const float* beta_t,
+                                      const ttcd_block_weights* w, const ttcd_block_params* p,
+                                      void* state, size_t state_bytes, void* y, void* workspace,
+                                      size_t ws_bytes, int commit, void* stream);
+
 /* Workspace bytes needed by each entry point; 0 if the parameters are invalid. */
 size_t ttcd_fastweight_mlp_workspace_size(const ttcd_block_params* p);
 size_t ttcd_block_forward_workspace_size(const ttcd_block_params* p);

@@ -80,9 +80,11 @@ def test_decode_with_state_in(ttcd):
 
 
 def test_graph_decode_matches_eager_decode(ttcd):
-    """ttcd_block_decode_next replayed from one CUDA graph (the position read
-    from the state on the device) gives the eager decode's rows bit for bit,
-    across chunk commits, and the oracle's."""
+    """ttcd_block_decode_next_ex replayed from two CUDA graphs, an ordinary
+    step without the chunk commit's launches and a commit step at each chunk's
+    last token (the position read from the state on the device), gives the
+    eager decode's rows and state bit for bit, across chunk commits, and the
+    oracle's."""
     shape = DEC_A.with_(name="dec_graph", T=2 * DEC_A.chunk + 37)
     inp = make_block_inputs(shape, seed=9)
     x, w = to_device(inp)
@@ -95,7 +97,7 @@ def test_graph_decode_matches_eager_decode(ttcd):
         ye.append(eager.step(xt, bt))
         yg.append(graph.step(xt, bt))
     assert eager.check_status() == ttcd.OK and graph.check_status() == ttcd.OK
-    assert graph.graph is not None
+    assert graph.graphs[False] is not None and graph.graphs[True] is not None
     ye, yg = torch.stack(ye, dim=1), torch.stack(yg, dim=1)
     assert torch.equal(ye, yg)
     assert torch.equal(eager.state_out(), graph.state_out())
