@@ -338,7 +338,6 @@ def run_ours(args, world, rank, local):
     barrier(world, local)
     torch.cuda.synchronize()
     launches0 = ttcd.kernel_launch_count()
-    replayed0 = dec.replayed_launches
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
@@ -744,7 +743,6 @@ def measure_stack(args, world, local, B, T, steps, warmup):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ttcd.kernel_launch_count()
-    replayed0 = dec.replayed_launches
     with ClockSampler(local) as clk:
         e0.record(stream)
         for _ in range(steps):
